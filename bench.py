@@ -1,0 +1,370 @@
+"""Benchmark: CKKS key-switched rotations/s on the rotation-batch workload.
+
+Workload (one "step"): 64 ciphertexts at N = 2^16, L = 24 (one 60-bit + 23
+40-bit primes), K = 8 special 60-bit primes, dnum = 3, each rotated by one of
+16 seeded distinct steps in [1, 32767] with an evaluation key per step.  Each
+rotation runs the whole key-switching path: automorphism, inverse NTT, ModUp
+(base conversion + NTT), key inner product, ModDown (inverse NTT, centred
+conversion, NTT, combine).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun every rank rotates its own 64 ciphertexts with its own copy of
+the keys (independent work, no collective on the data path: weak scaling);
+rank 0 prints one JSON line.  --impl reference times the CPU oracle on the
+host cores on a bounded sample of the same workload.
+"""
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import seeded_inputs as S  # noqa: E402
+
+LOG_N, L, K, DNUM = 16, 24, 8, 3
+N_CTS, N_KEYS = 64, 16
+LEVEL = 24
+METRIC = "CKKS key-switched rotations/s (N=2^16,L=24,dnum=3); % of HBM roofline"
+WORKLOAD = {"workload": "rotation batch: 64 fresh ciphertexts, 16 seeded rotation keys",
+            "N": 1 << LOG_N, "L": L, "K": K, "dnum": DNUM, "level": LEVEL, "n_ciphertexts": N_CTS,
+            "n_keys": N_KEYS, "l2": "inputs larger than L2 (1.6 GB of ciphertexts, 1.6 GB of keys per step)"}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+# ------------------------------------------------------------------ inputs
+
+def workload_inputs(master, primes_q, n_cts):
+    steps = S.rotation_steps(master, N_KEYS, 1, (1 << (LOG_N - 1)) - 1)
+    assign = S.step_assignment(master, n_cts, N_KEYS)
+    return steps, [steps[u] for u in assign]
+
+
+class ClockSampler:
+    """nvidia-smi clocks during the timed region (SM MHz and throttle reasons)."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ cpu baseline
+
+def cpu_baseline(seconds):
+    """The oracle, as it stands, rotating full-size ciphertexts of this workload
+    on the host cores until about `seconds` of rotation work has run."""
+    from oracle import ckks as C
+
+    master = S.master_seed(1)
+    P = C.Params(LOG_N, L, K, DNUM)
+    steps, ct_steps = workload_inputs(master, P.q, N_CTS)
+    s = S.secret(master, P.N)
+    uni = S.uniform_residues(master, "ct_residues", P.q, P.N, lead=(4, 2))
+    keys = {}
+    done, t_rot, i = 0, 0.0, 0
+    while (t_rot < seconds and done < 64) or done < 2:
+        st = ct_steps[i % N_CTS]
+        if st not in keys:
+            k = P.galois_elt(st)
+            a, e = S.key_draws(master, k, P.mods, P.N, P.dnum)
+            keys[st] = C.rotation_key(s, st, a, e, P)
+        ct = C.make_ct(uni[i % 4], LEVEL, 2.0 ** 40)
+        t0 = time.perf_counter()
+        C.rotate(ct, st, keys[st], P)
+        t_rot += time.perf_counter() - t0
+        done += 1
+        i += 1
+    return {"value": done / t_rot, "unit": "rotations/s", "cores": C.n_threads(), "kind": "oracle",
+            "sample": "%d full-size rotations (N=2^16, level 24, K=8, dnum=3) of uniform-residue ciphertexts, "
+                      "key generation excluded; oracle threads over limbs" % done}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    steps = args.steps
+    t0 = time.perf_counter()
+    per = []
+    for _ in range(args.warmup + steps):
+        r = cpu_baseline(max(1.0, args.cpu_seconds / max(1, steps + args.warmup)))
+        per.append(r)
+    timed = per[args.warmup:]
+    v = float(np.mean([r["value"] for r in timed]))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "rotations/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": 1000.0 * 64 / v, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u64", "data": "synthetic",
+            "config": WORKLOAD,
+            "cpu_baseline": {"value": v, "unit": "rotations/s", "cores": timed[0]["cores"], "kind": "oracle",
+                             "sample": timed[0]["sample"] + " (per step)"},
+            "e2e": {"value": v, "unit": "rotations/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "wall_s": time.perf_counter() - t0}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ native
+
+# algorithmic work per launch of each kernel class for the rotation batch
+def class_work(cls, n_cts):
+    N = 1 << LOG_N
+    lvl, nd = LEVEL, -(-LEVEL // (-(-L // DNUM)))
+    rows_ext = lvl + K
+    w = 8
+    if cls == "ks_inner":
+        # ext reads + key (once per key group) + u writes; 2*nd Montgomery MACs per output pair
+        return {"bytes": None, "mults": n_cts * rows_ext * N * 2 * nd}
+    return None
+
+
+def run_native(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from homomorphic_encrypted_transformer_b200 import he
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    ctx = he.he_ctx_create(LOG_N, L, K, DNUM, stream=stream)
+    N = ctx.N
+    master = S.master_seed(1)
+    steps, ct_steps = workload_inputs(master, ctx.primes[:L], N_CTS)
+    s = S.secret(master, N)
+    for st in steps:
+        k = pow(5, st % (N // 2), 2 * N)
+        a, e = S.key_draws(master, k, ctx.primes, N, DNUM)
+        he.he_keygen_upload(ctx, he.HE_KEY_ROTATION, st, s, a, e)
+    # inputs: uniform residues (a fresh encryption is computationally
+    # indistinguishable from them); per-rank stream of draws
+    h_in = S.uniform_residues(master + 7919 * rank, "ct_residues", ctx.primes[:L], N, lead=(N_CTS, 2))
+    x = torch.from_numpy(h_in.view(np.int64)).to(dev)
+    y = torch.empty_like(x)
+    xs = [he.Ciphertext(x[i], LEVEL, 2.0 ** 40) for i in range(N_CTS)]
+    ys = [he.Ciphertext(y[i], LEVEL, 2.0 ** 40) for i in range(N_CTS)]
+
+    def step():
+        he.he_rotate_batch(ctx, xs, ct_steps, ys)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # HBM and integer probes in the same run
+    probe_words = 1 << 28  # 2 GiB each way
+    pa = torch.empty(probe_words, dtype=torch.int64, device=dev)
+    pb = torch.empty_like(pa)
+    pa.fill_(1)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    best = 1e9
+    for _ in range(5):
+        ev0.record(stream)
+        he.he_probe_copy(ctx, pb, pa, probe_words)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        best = min(best, ev0.elapsed_time(ev1))
+    copy_gbs = 2 * probe_words * 8 / (best * 1e-3) / 1e9
+    del pa, pb
+    sink = torch.empty(he.he_probe_int_threads(ctx), dtype=torch.int64, device=dev)
+    iters = 4096
+    best = 1e9
+    for _ in range(3):
+        ev0.record(stream)
+        he.he_probe_int(ctx, iters, sink)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        best = min(best, ev0.elapsed_time(ev1))
+    int_modmul_s = he.he_probe_int_threads(ctx) * iters * he.he_probe_int_mults_per_iter() / (best * 1e-3)
+
+    # timed region
+    clocks = ClockSampler(local_rank)
+    he.he_launch_count(ctx, reset=True)
+    he.he_profile_enable(ctx, True)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = t0.elapsed_time(t1)
+    clk = clocks.stop()
+    launches = he.he_launch_count(ctx)
+    prof = {name: he.he_profile_read(ctx, cls) for name, cls in he.PROF.items()}
+    he.he_profile_enable(ctx, False)
+
+    # same step without profiling events (the headline number)
+    torch.cuda.synchronize()
+    barrier()
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_plain = t0.elapsed_time(t1)
+
+    if world > 1:
+        tt = torch.tensor([ms_plain, ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_plain, ms = float(tt[0]), float(tt[1])
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    h_pin = torch.from_numpy(h_in.view(np.int64)).pin_memory()
+    h_out = torch.empty_like(h_pin).pin_memory()
+    he.he_rotate_batch_host(ctx, h_pin, LEVEL, ct_steps, h_out)
+    barrier()
+    e2e_steps = max(1, min(args.steps, 5))
+    te = time.perf_counter()
+    for _ in range(e2e_steps):
+        he.he_rotate_batch_host(ctx, h_pin, LEVEL, ct_steps, h_out)
+    e2e_s = time.perf_counter() - te
+    if world > 1:
+        tt = torch.tensor([e2e_s], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_s = float(tt[0])
+
+    if rank != 0:
+        return
+    total_rot = N_CTS * args.steps * world
+    value = total_rot / (ms_plain * 1e-3)
+    pk, pk_kind = peaks()
+    hbm_peak = float(pk.get("hbm_gbs", 6650.0))
+    # dominant kernel class by device time in the profiled pass
+    dom = max(prof.items(), key=lambda kv: kv[1][0])
+    dom_name, (dom_ms, dom_launches) = dom
+    ct_bytes = 2 * LEVEL * N * 8
+    key_bytes = 3 * 2 * (L + K) * N * 8
+    # algorithmic bytes of one rotation batch (keys read once per key group)
+    batch_bytes = N_KEYS * key_bytes + N_CTS * 2 * ct_bytes
+    hbm_frac_step = (batch_bytes / (ms_plain * 1e-3 / args.steps)) / 1e9 / hbm_peak
+    roof = roofline_for(dom_name, dom_ms / max(1, dom_launches), args, N, int_modmul_s, hbm_peak, pk_kind)
+    line = {"metric": METRIC, "value": value, "unit": "rotations/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_plain / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u64", "data": "synthetic",
+            "config": dict(WORKLOAD, parallelism="replicas%d" % world if world > 1 else "single"),
+            "hbm_roofline_frac_of_step": hbm_frac_step,
+            "roofline": roof,
+            "probes": {"copy_gbs": copy_gbs, "int_shoup_modmul_per_s": int_modmul_s},
+            "kernel_ms_per_step": {k: v[0] / args.steps for k, v in prof.items() if v[1]},
+            "kernel_launches_per_step": {k: v[1] / args.steps for k, v in prof.items() if v[1]},
+            "profiled_ms_per_step": ms / args.steps,
+            "gpu_launches": launches,
+            "clocks": clk,
+            "e2e": {"value": N_CTS * e2e_steps * world / e2e_s, "unit": "rotations/s",
+                    "h2d_bytes_per_step": int(h_in.nbytes), "d2h_bytes_per_step": int(h_in.nbytes)}}
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def roofline_for(name, ms_per_launch, args, N, int_modmul_s, hbm_peak, pk_kind):
+    return {"kernel_class": name, "ms_per_launch": ms_per_launch, "bound": None, "achieved": None,
+            "peak": hbm_peak, "unit": "GB/s", "frac": None, "traffic": None,
+            "peak_source": pk_kind}
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        backend = "nccl" if args.impl == "native" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_native(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

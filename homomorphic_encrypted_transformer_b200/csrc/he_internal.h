@@ -1,0 +1,131 @@
+// Internal state of the RNS-CKKS engine.  Not part of the ABI.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <map>
+#include <string>
+#include <vector>
+
+#include "../../include/he.h"
+#include "kernels.cuh"
+#include "modarith.cuh"
+
+namespace he {
+
+constexpr int kMaxPrimes = 64;
+
+// ModUp fast base conversion of one digit at one level, on device:
+//   y_i = [x_i * qhat_inv_i]_{q_i} for the digit's source primes,
+//   out_t = sum_i y_i * (qhat_i mod t) for every row t of Q_level and P
+//   (rows of the digit itself reproduce x: the sum collapses to x_t there).
+struct ConvTable {
+    int n_src;
+    int src_row;            // first row of the digit (its primes are rows src_row..src_row+n_src-1)
+    ulonglong2* d_src;      // [n_src] {qhat_inv_i mod q_i, shoup}
+    ulonglong2* d_mat;      // [n_src][level + K] {qhat_i mod t, shoup}
+};
+
+struct Key {
+    uint64_t* d = nullptr;  // [digits][2][L+K][N] in Montgomery form (value * 2^64 mod p)
+};
+
+struct ProfSlot {
+    double ms = 0;
+    long long launches = 0;
+};
+
+struct ProfPending {
+    int cls;
+    cudaEvent_t a, b;
+};
+
+}  // namespace he
+
+struct he_ctx {
+    int log_n = 0, N = 0, L = 0, K = 0, dnum = 0, alpha = 0;
+    std::vector<uint64_t> primes;  // L + K, prime index space
+    std::vector<uint64_t> psi;
+    cudaStream_t stream = nullptr;
+    std::string err;
+    int device = 0;
+
+    std::vector<he::DevPrime> hprime;
+    he::DevPrime* d_prime = nullptr;   // [L+K]
+    ulonglong2* d_tw_fwd = nullptr;    // [L+K][N] {psi^brev(i), shoup}
+    ulonglong2* d_tw_inv = nullptr;    // [L+K][N] {psi^-brev(i), shoup}; entry 1 times N^-1
+    ulonglong2* d_inv_last = nullptr;  // [L+K] {N^-1, shoup}
+
+    std::vector<std::vector<he::ConvTable>> modup;  // [level][digit], level 1..L
+    ulonglong2* d_md_pcoef = nullptr;  // [K] {(P/p_k)^-1 mod p_k, shoup}
+    ulonglong2* d_md_mat = nullptr;    // [K][L] {(P/p_k) mod q_i, shoup}
+    uint64_t* d_md_negP = nullptr;     // [L] -P mod q_i (correction of a negative centred term)
+    ulonglong2* d_md_pinv = nullptr;   // [L] {P^-1 mod q_i, shoup}
+    std::vector<uint64_t> h_Pmod;      // [L+K] P mod prime (0 on the p's)
+    ulonglong2* d_rs_inv = nullptr;    // [L][L] {q_l^-1 mod q_i, shoup}
+    uint64_t* d_rs_qmod = nullptr;     // [L][L] q_l mod q_i
+
+    std::map<uint64_t, he::Key> rot_keys;  // by Galois element
+    he::Key relin;
+
+    uint64_t* scratch[4] = {nullptr, nullptr, nullptr, nullptr};
+    size_t scratch_words[4] = {0, 0, 0, 0};
+    uint64_t* io_buf = nullptr;  // device staging of the host-buffer entry point
+    size_t io_words = 0;
+
+    bool prof_on = false;
+    he::ProfSlot prof[HE_PROF_N];
+    std::vector<he::ProfPending> prof_pending;
+    std::vector<cudaEvent_t> ev_pool;
+    long long launches = 0;
+};
+
+namespace he {
+
+int set_err(he_ctx* c, int code, const char* fmt, ...);
+int check_cuda(he_ctx* c, cudaError_t e, const char* what);
+
+void prof_begin(he_ctx* c, int cls);
+int prof_end(he_ctx* c, int cls);
+
+uint64_t galois_elt(const he_ctx* c, int32_t step);
+
+RowSet rowset(uint64_t* base, long long group_stride, int per_group, const int* prime_idx);
+RowSet rowset_contig(uint64_t* base, int per_group, int N, const std::vector<int>& prime_idx);
+std::vector<int> prime_range(int first, int count);
+// Rows of Q_level then all of P: 0..level-1, L..L+K-1
+std::vector<int> ext_primes(const he_ctx* c, int level);
+
+int ntt_setup(he_ctx* c);
+int ntt_fwd_set(he_ctx* c, const RowSet& rs, int n_rows);
+int ntt_inv_set(he_ctx* c, const RowSet& rs, int n_rows);
+
+// Key switching of polynomials d[i] (evaluation domain, [level][N] each) with
+// one key.  Writes out[i] = [2][level][N]:
+//   out0 = KS(d)_0 + add0[i],  out1 = KS(d)_1 + add1[i]   (null adds are skipped).
+// With galois != 0 the switched polynomial is sigma_galois(d[i]), and add0 is
+// also read through sigma_galois when sig_add0 is set (rotation).
+struct KsIoList {
+    uint64_t galois = 0;
+    bool sig_add0 = false;
+    std::vector<const uint64_t*> d;
+    std::vector<uint64_t*> out;
+    std::vector<const uint64_t*> add0;
+    std::vector<const uint64_t*> add1;
+};
+int key_switch(he_ctx* c, int level, const Key& key, const KsIoList& io);
+size_t key_switch_scratch_words(const he_ctx* c, int n, int level);
+int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, int n);
+
+// Scratch slots: 0 = key switching internals, 1 = rescale temporaries,
+// 2 = HMult temporaries and key generation, 3 = driver buffers (polynomial
+// evaluation, BSGS).  A call only uses slots below the ones its callers hold.
+constexpr int kScratchSlots = 4;
+int scratch_slot(he_ctx* c, int slot, size_t words, uint64_t** out);
+
+// out[i] = rescale(in[i]) for n ciphertexts at `level` (out may equal in).
+int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int level);
+
+int elementwise_setup(he_ctx* c);
+
+}  // namespace he

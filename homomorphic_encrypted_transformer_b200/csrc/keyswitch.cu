@@ -1,0 +1,370 @@
+// Hybrid key switching (Han-Ki, CT-RSA 2020, section 3) and rotation.
+//
+//   KS_evk(d) = ModDown( sum_j ModUp_j(d) (.) evk_j ),
+//   ModUp_j: coefficients of digit j's primes -> fast base conversion onto
+//            every prime of Q_level and P, back to the evaluation domain;
+//   ModDown: (x - Conv_{P->q}([x]_P)) * P^-1 with the conversion terms taken
+//            in the centred range, so the result is round(x/P) - v, |v| <= K/2.
+//   rot_r(ct) = (sigma_k(c0), 0) + KS_{evk_r}(sigma_k(c1)),  k = 5^r mod 2N.
+#include <algorithm>
+
+#include "he_internal.h"
+#include "ntt.cuh"
+
+namespace he {
+
+constexpr int kMaxBatch = 32;
+constexpr int kMaxDigits = 15;
+
+struct PtrList {
+    const uint64_t* p[kMaxBatch];
+};
+struct MutPtrList {
+    uint64_t* p[kMaxBatch];
+};
+
+// Evaluation-domain index whose value sigma_k moves to index j:
+// storage j is the point psi^(2 brev(j)+1); sigma_k(a) there is a(psi^((2 brev(j)+1) k)).
+__device__ __forceinline__ int automorph_src(int j, int logn, uint64_t k) {
+    unsigned m = __brev((unsigned)j) >> (32 - logn);
+    uint64_t e = ((2ull * m + 1) * k) & ((2ull << logn) - 1);
+    unsigned m2 = (unsigned)((e - 1) >> 1);
+    return (int)(__brev(m2) >> (32 - logn));
+}
+
+// coef[i][r][c] = d_i[r][src(c)] (or a plain copy when galois == 0).
+__global__ void k_gather(PtrList in, uint64_t* __restrict__ out, int level, int logn, uint64_t galois) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x;
+    int r = blockIdx.y, i = blockIdx.z;
+    if (c >= N) return;
+    int src = galois ? automorph_src(c, logn, galois) : c;
+    out[((size_t)i * level + r) * N + c] = in.p[i][(size_t)r * N + src];
+}
+
+struct ModupArgs {
+    int n_digits;
+    int n_src[kMaxDigits];
+    int src_row[kMaxDigits];
+    const ulonglong2* src[kMaxDigits];
+    const ulonglong2* mat[kMaxDigits];
+    uint8_t tprime[64];  // prime index of each of the level+K rows
+};
+
+// ext[i][j][t][c] = sum_s [x_s qhat_inv_s]_{q_s} (qhat_s mod t_prime)  (coefficient domain)
+__global__ void k_modup_conv(const uint64_t* __restrict__ coef, uint64_t* __restrict__ ext, ModupArgs a,
+                             const DevPrime* __restrict__ pr, int level, int n_rows, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x;
+    int j = blockIdx.y, i = blockIdx.z;
+    if (c >= N) return;
+    const int ns = a.n_src[j], s0 = a.src_row[j];
+    uint64_t y[16];
+    for (int s = 0; s < ns; s++) {
+        uint64_t q = pr[s0 + s].q;
+        uint64_t x = coef[((size_t)i * level + s0 + s) * N + c];
+        ulonglong2 w = a.src[j][s];
+        y[s] = mul_shoup(x, w.x, w.y, q);
+    }
+    uint64_t* o = ext + (((size_t)i * a.n_digits + j) * n_rows) * N + c;
+    const ulonglong2* m = a.mat[j];
+    for (int t = 0; t < n_rows; t++) {
+        uint64_t q = pr[a.tprime[t]].q;
+        uint64_t acc = 0;
+        for (int s = 0; s < ns; s++) {
+            ulonglong2 w = m[(size_t)s * n_rows + t];
+            acc = csub(acc + mul_shoup_lazy(y[s], w.x, w.y, q), 2 * q);
+        }
+        o[(size_t)t * N] = csub(acc, q);
+    }
+}
+
+// u[i][0/1][t][c] = sum_j ext[i][j][t][c] * key_j[b/a][row(t)][c]   (key in Montgomery form)
+__global__ void k_ks_inner(const uint64_t* __restrict__ ext, const uint64_t* __restrict__ key, uint64_t* __restrict__ u,
+                           int n_digits, int n_rows, int level, int L, int LK, const DevPrime* __restrict__ pr,
+                           ModupArgs a, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x;
+    int t = blockIdx.y, i = blockIdx.z;
+    if (c >= N) return;
+    int krow = t < level ? t : L + (t - level);
+    DevPrime p = pr[a.tprime[t]];
+    U128 acc0 = {0, 0}, acc1 = {0, 0};
+    for (int j = 0; j < n_digits; j++) {
+        uint64_t x = ext[(((size_t)i * n_digits + j) * n_rows + t) * N + c];
+        const uint64_t* kb = key + (((size_t)j * 2 + 0) * LK + krow) * N;
+        const uint64_t* ka = key + (((size_t)j * 2 + 1) * LK + krow) * N;
+        mac128(acc0, x, kb[c]);
+        mac128(acc1, x, ka[c]);
+    }
+    uint64_t* o = u + ((size_t)i * 2 * n_rows) * N + c;
+    o[(size_t)t * N] = csub(redc_lazy(acc0.hi, acc0.lo, p.q, p.qinv_neg), p.q);
+    o[(size_t)(n_rows + t) * N] = csub(redc_lazy(acc1.hi, acc1.lo, p.q, p.qinv_neg), p.q);
+}
+
+// tmp[i][k][r][c] = sum_p y_p (P/p mod q_r) with y_p = [x_p (P/p)^-1]_p taken centred.
+__global__ void k_moddown_conv(const uint64_t* __restrict__ u, uint64_t* __restrict__ tmp, int level, int K, int L,
+                               const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ pcoef,
+                               const ulonglong2* __restrict__ mat, const uint64_t* __restrict__ negP, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x;
+    int poly = blockIdx.y, i = blockIdx.z;  // poly in {0, 1}
+    if (c >= N) return;
+    const int n_rows = level + K;
+    const uint64_t* x = u + (((size_t)i * 2 + poly) * n_rows + level) * N + c;
+    uint64_t y[16];
+    unsigned neg = 0;
+    for (int k = 0; k < K; k++) {
+        uint64_t p = pr[L + k].q;
+        ulonglong2 w = pcoef[k];
+        y[k] = mul_shoup(x[(size_t)k * N], w.x, w.y, p);
+        if (y[k] > (p >> 1)) neg |= 1u << k;
+    }
+    uint64_t* o = tmp + (((size_t)i * 2 + poly) * level) * N + c;
+    for (int r = 0; r < level; r++) {
+        uint64_t q = pr[r].q;
+        uint64_t acc = 0;
+        for (int k = 0; k < K; k++) {
+            ulonglong2 w = mat[(size_t)k * L + r];
+            uint64_t term = csub(mul_shoup_lazy(y[k], w.x, w.y, q), q);
+            if (neg >> k & 1u) term += negP[r];  // (y - p) (P/p) = y (P/p) - P
+            acc = csub(acc + term, 2 * q);
+        }
+        o[(size_t)r * N] = csub(acc, q);
+    }
+}
+
+// out_i[poly][r][c] = (u[poly][r] - tmp[poly][r]) P^-1 + add_poly
+__global__ void k_moddown_combine(const uint64_t* __restrict__ u, const uint64_t* __restrict__ tmp, MutPtrList out,
+                                  PtrList add0, PtrList add1, int sig_add0, uint64_t galois, int level, int K,
+                                  const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ pinv, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x;
+    int r = blockIdx.y % level, poly = blockIdx.y / level, i = blockIdx.z;
+    if (c >= N) return;
+    const int n_rows = level + K;
+    uint64_t q = pr[r].q;
+    uint64_t uv = u[(((size_t)i * 2 + poly) * n_rows + r) * N + c];
+    uint64_t tv = tmp[(((size_t)i * 2 + poly) * level + r) * N + c];
+    ulonglong2 w = pinv[r];
+    uint64_t v = mul_shoup(uv + q - tv, w.x, w.y, q);
+    const uint64_t* ad = poly == 0 ? add0.p[i] : add1.p[i];
+    if (ad) {
+        int src = (poly == 0 && sig_add0 && galois) ? automorph_src(c, logn, galois) : c;
+        v = add_mod(v, ad[(size_t)r * N + src], q);
+    }
+    out.p[i][((size_t)poly * level + r) * N + c] = v;
+}
+
+static ModupArgs modup_args(he_ctx* c, int level) {
+    ModupArgs a;
+    auto& tabs = c->modup[level];
+    a.n_digits = (int)tabs.size();
+    for (int j = 0; j < a.n_digits; j++) {
+        a.n_src[j] = tabs[j].n_src;
+        a.src_row[j] = tabs[j].src_row;
+        a.src[j] = tabs[j].d_src;
+        a.mat[j] = tabs[j].d_mat;
+    }
+    std::vector<int> ep = ext_primes(c, level);
+    for (size_t t = 0; t < ep.size(); t++) a.tprime[t] = (uint8_t)ep[t];
+    return a;
+}
+
+static int lc(he_ctx* c, const char* what) {
+    c->launches++;
+    return check_cuda(c, cudaGetLastError(), what);
+}
+
+size_t key_switch_scratch_words(const he_ctx* c, int n, int level) {
+    size_t nd = (level + c->alpha - 1) / c->alpha, nr = level + c->K;
+    return (size_t)c->N * n * (level + nd * nr + 2 * nr + 2 * level);
+}
+
+int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList& io) {
+    const int N = c->N, K = c->K, L = c->L, LK = L + K;
+    const int n_rows = level + K;
+    ModupArgs ma = modup_args(c, level);
+    const int nd = ma.n_digits;
+    uint64_t* base;
+    int rc = scratch_slot(c, 0, key_switch_scratch_words(c, n, level), &base);
+    if (rc) return rc;
+    uint64_t* coef = base;
+    uint64_t* ext = coef + (size_t)n * level * N;
+    uint64_t* u = ext + (size_t)n * nd * n_rows * N;
+    uint64_t* tmp = u + (size_t)n * 2 * n_rows * N;
+
+    PtrList din;
+    MutPtrList dout;
+    PtrList a0, a1;
+    for (int i = 0; i < kMaxBatch; i++) {
+        din.p[i] = i < n ? io.d[i] : nullptr;
+        dout.p[i] = i < n ? io.out[i] : nullptr;
+        a0.p[i] = i < n ? io.add0[i] : nullptr;
+        a1.p[i] = i < n ? io.add1[i] : nullptr;
+    }
+    const int TB = 256;
+    dim3 blk(TB);
+    int gx = (N + TB - 1) / TB;
+
+    prof_begin(c, HE_PROF_AUTOMORPH);
+    k_gather<<<dim3(gx, level, n), blk, 0, c->stream>>>(din, coef, level, c->log_n, io.galois);
+    if ((rc = lc(c, "gather"))) return rc;
+    prof_end(c, HE_PROF_AUTOMORPH);
+
+    std::vector<int> qp = prime_range(0, level);
+    if ((rc = ntt_inv_set(c, rowset_contig(coef, level, N, qp), n * level))) return rc;
+
+    prof_begin(c, HE_PROF_MODUP);
+    k_modup_conv<<<dim3(gx, nd, n), blk, 0, c->stream>>>(coef, ext, ma, c->d_prime, level, n_rows, c->log_n);
+    if ((rc = lc(c, "modup_conv"))) return rc;
+    prof_end(c, HE_PROF_MODUP);
+
+    std::vector<int> ep = ext_primes(c, level);
+    if ((rc = ntt_fwd_set(c, rowset_contig(ext, n_rows, N, ep), n * nd * n_rows))) return rc;
+
+    prof_begin(c, HE_PROF_KS_INNER);
+    k_ks_inner<<<dim3(gx, n_rows, n), blk, 0, c->stream>>>(ext, key.d, u, nd, n_rows, level, L, LK, c->d_prime, ma,
+                                                           c->log_n);
+    if ((rc = lc(c, "ks_inner"))) return rc;
+    prof_end(c, HE_PROF_KS_INNER);
+
+    std::vector<int> pp = prime_range(L, K);
+    RowSet prs = rowset(u + (size_t)level * N, (long long)n_rows * N, K, pp.data());
+    if ((rc = ntt_inv_set(c, prs, n * 2 * K))) return rc;
+
+    prof_begin(c, HE_PROF_MODDOWN);
+    k_moddown_conv<<<dim3(gx, 2, n), blk, 0, c->stream>>>(u, tmp, level, K, L, c->d_prime, c->d_md_pcoef,
+                                                          c->d_md_mat, c->d_md_negP, c->log_n);
+    if ((rc = lc(c, "moddown_conv"))) return rc;
+    prof_end(c, HE_PROF_MODDOWN);
+
+    if ((rc = ntt_fwd_set(c, rowset_contig(tmp, level, N, qp), n * 2 * level))) return rc;
+
+    prof_begin(c, HE_PROF_MODDOWN);
+    k_moddown_combine<<<dim3(gx, 2 * level, n), blk, 0, c->stream>>>(u, tmp, dout, a0, a1, io.sig_add0 ? 1 : 0,
+                                                                     io.galois, level, K, c->d_prime, c->d_md_pinv,
+                                                                     c->log_n);
+    if ((rc = lc(c, "moddown_combine"))) return rc;
+    prof_end(c, HE_PROF_MODDOWN);
+    return HE_OK;
+}
+
+int key_switch(he_ctx* c, int level, const Key& key, const KsIoList& io) {
+    int n = (int)io.d.size();
+    for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
+        int m = std::min(kMaxBatch, n - i0);
+        KsIoList sub;
+        sub.galois = io.galois;
+        sub.sig_add0 = io.sig_add0;
+        sub.d.assign(io.d.begin() + i0, io.d.begin() + i0 + m);
+        sub.out.assign(io.out.begin() + i0, io.out.begin() + i0 + m);
+        sub.add0.assign(io.add0.begin() + i0, io.add0.begin() + i0 + m);
+        sub.add1.assign(io.add1.begin() + i0, io.add1.begin() + i0 + m);
+        int rc = key_switch_chunk(c, m, level, key, sub);
+        if (rc) return rc;
+    }
+    return HE_OK;
+}
+
+static int ct_ok(he_ctx* c, const he_ct* x, const char* what) {
+    if (!x || !x->data) return set_err(c, HE_EINVAL, "%s: null ciphertext", what);
+    if (x->level < 1 || x->level > c->L) return set_err(c, HE_ELEVEL, "%s: level %d out of range", what, x->level);
+    if (!x->is_ntt) return set_err(c, HE_EDOMAIN, "%s: ciphertext not in the evaluation domain", what);
+    return HE_OK;
+}
+
+int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, int n) {
+    if (n < 0) return set_err(c, HE_EINVAL, "rotate: negative count");
+    if (n == 0) return HE_OK;
+    if (!in || !out || !steps) return set_err(c, HE_EINVAL, "rotate: null argument");
+    int level = in[0].level;
+    for (int i = 0; i < n; i++) {
+        int rc = ct_ok(c, &in[i], "rotate");
+        if (rc) return rc;
+        if (in[i].level != level) return set_err(c, HE_ELEVEL, "rotate: mixed levels in a batch");
+        if (!out[i].data) return set_err(c, HE_EINVAL, "rotate: null output");
+        if (out[i].data == in[i].data) return set_err(c, HE_EINVAL, "rotate: output aliases input");
+    }
+    // group by Galois element so that each key is streamed once per group
+    std::map<uint64_t, std::vector<int>> groups;
+    for (int i = 0; i < n; i++) {
+        uint64_t g = galois_elt(c, steps[i]);
+        if (g != 1 && !c->rot_keys.count(g))
+            return set_err(c, HE_ENOKEY, "rotate: no key for step %d (galois %llu)", steps[i], (unsigned long long)g);
+        groups[g].push_back(i);
+    }
+    const size_t ct_words = (size_t)2 * level * c->N;
+    for (auto& kv : groups) {
+        if (kv.first == 1) {  // rotation by a multiple of N/2: identity
+            for (int i : kv.second) {
+                int rc = check_cuda(c, cudaMemcpyAsync(out[i].data, in[i].data, ct_words * 8,
+                                                       cudaMemcpyDeviceToDevice, c->stream), "rotate copy");
+                if (rc) return rc;
+            }
+            continue;
+        }
+        KsIoList io;
+        io.galois = kv.first;
+        io.sig_add0 = true;
+        for (int i : kv.second) {
+            io.d.push_back(in[i].data + (size_t)level * c->N);
+            io.out.push_back(out[i].data);
+            io.add0.push_back(in[i].data);
+            io.add1.push_back(nullptr);
+        }
+        int rc = key_switch(c, level, c->rot_keys[kv.first], io);
+        if (rc) return rc;
+    }
+    for (int i = 0; i < n; i++) {
+        out[i].level = level;
+        out[i].scale = in[i].scale;
+        out[i].is_ntt = 1;
+    }
+    return HE_OK;
+}
+
+}  // namespace he
+
+using namespace he;
+
+extern "C" int he_rotate(he_ctx* c, const he_ct* in, int32_t step, he_ct* out) {
+    if (!c) return HE_EINVAL;
+    return rotate_many(c, in, &step, out, 1);
+}
+
+extern "C" int he_rotate_batch(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, int n) {
+    if (!c) return HE_EINVAL;
+    return rotate_many(c, in, steps, out, n);
+}
+
+extern "C" int he_rotate_batch_host(he_ctx* c, const uint64_t* h_in, int level, const int32_t* steps,
+                                    uint64_t* h_out, int n) {
+    if (!c) return HE_EINVAL;
+    if (!h_in || !h_out || !steps || n < 0 || level < 1 || level > c->L)
+        return set_err(c, HE_EINVAL, "he_rotate_batch_host: bad arguments");
+    const size_t ct_words = (size_t)2 * level * c->N, total = ct_words * n;
+    if (2 * total > c->io_words) {
+        cudaStreamSynchronize(c->stream);
+        cudaFree(c->io_buf);
+        c->io_buf = nullptr;
+        c->io_words = 0;
+        int rc = check_cuda(c, cudaMalloc(&c->io_buf, 2 * total * 8), "io buffer");
+        if (rc) return rc;
+        c->io_words = 2 * total;
+    }
+    uint64_t* din = c->io_buf;
+    uint64_t* dout = c->io_buf + total;
+    int rc = check_cuda(c, cudaMemcpyAsync(din, h_in, total * 8, cudaMemcpyHostToDevice, c->stream), "H2D");
+    if (rc) return rc;
+    std::vector<he_ct> in(n), out(n);
+    for (int i = 0; i < n; i++) {
+        in[i] = he_ct{din + i * ct_words, level, 1.0, 1};
+        out[i] = he_ct{dout + i * ct_words, level, 1.0, 1};
+    }
+    rc = rotate_many(c, in.data(), steps, out.data(), n);
+    if (rc) return rc;
+    rc = check_cuda(c, cudaMemcpyAsync(h_out, dout, total * 8, cudaMemcpyDeviceToHost, c->stream), "D2H");
+    if (rc) return rc;
+    return he_sync(c);
+}

@@ -1,0 +1,247 @@
+/*
+ * he.h -- C ABI of the B200 RNS-CKKS polynomial engine (libhe.so).
+ *
+ * The engine is the data-parallel hot path under encrypted Transformer
+ * inference as AEGIS describes it (AEGIS: Scaling Long-Sequence Homomorphic
+ * Encrypted Transformer Inference, gist.science summary): CKKS ciphertexts
+ * are RNS polynomials split into modulus limbs along a modulus chain, and
+ * the operations that dominate are key switching and rotation (section 1
+ * "Problem", items 2-3), the local plaintext-weight x ciphertext product of
+ * the FFN (section 2.2) and the polynomial approximation of Softmax (section
+ * 2.3).  The pages define no API; the calls below follow that statement of
+ * the problem.  Below the CKKS level the arithmetic is the textbook one:
+ * Cheon-Han-Kim-Kim-Song, "A Full RNS Variant of Approximate Homomorphic
+ * Encryption" (SAC 2018) and the hybrid key switching of Han-Ki (CT-RSA 2020).
+ *
+ * Conventions for every call
+ *  - Return value: HE_OK (0) or a negative HE_E* code; he_last_error(ctx)
+ *    then holds a one-line message.  Argument errors are reported before
+ *    anything is enqueued.  CUDA errors of enqueued work are reported by the
+ *    next call that checks the stream, or by he_sync().
+ *  - Work is enqueued on the context's CUDA stream and is asynchronous
+ *    unless stated otherwise.  Host buffers passed to a call may be reused
+ *    as soon as it returns.
+ *  - Residues are uint64 in canonical form [0, q).  N = 2^log_n.
+ *  - Prime index space: 0..n_q-1 are q_0..q_{L-1} (the ciphertext modulus
+ *    chain), n_q..n_q+n_p-1 are the special primes p_0..p_{K-1}.
+ *  - A polynomial "limb" is N contiguous residues for one prime.  A
+ *    ciphertext at level l (l limbs q_0..q_{l-1}) is [2][l][N] uint64,
+ *    limb-major, c0 then c1, in the evaluation (NTT) domain: storage index j
+ *    holds the value at psi^(2*brev(j)+1), psi the smallest primitive 2N-th
+ *    root of unity mod the limb's prime.
+ *  - Ciphertext and plaintext buffers are device memory owned by the caller.
+ *    The context owns its tables, keys and scratch, and frees them in
+ *    he_ctx_destroy().
+ *  - A context is not thread-safe: one host thread at a time.
+ */
+#ifndef HE_B200_H
+#define HE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HE_OK 0
+#define HE_EINVAL (-1)   /* bad argument (null pointer, size, alignment, unsupported value) */
+#define HE_ELEVEL (-2)   /* level or scale mismatch between operands */
+#define HE_ENOKEY (-3)   /* no rotation / relinearisation key uploaded for the request */
+#define HE_EDOMAIN (-4)  /* operand not in the evaluation (NTT) domain */
+#define HE_ENOMEM (-5)   /* device allocation failed */
+#define HE_ECUDA (-6)    /* CUDA runtime error (message in he_last_error) */
+#define HE_ETIMEOUT (-7) /* reserved: a bounded device wait gave up */
+
+#define HE_KEY_ROTATION 0
+#define HE_KEY_RELIN 1
+
+typedef struct he_ctx he_ctx;
+
+/*
+ * Parameter set.  The pages fix none; the primes follow this rule unless
+ * given explicitly: every prime = 1 (mod 2N); a downward scan per bit size
+ * yields, in order, q_0 (q0_bits), p_0..p_{K-1} (p_bits), q_1..q_{L-1}
+ * (q_bits).  alpha = ceil(n_q / dnum) primes per key-switching digit.
+ * Requires 10 <= log_n <= 16, 1 <= n_q, 1 <= n_p, n_q + n_p <= 64,
+ * 1 <= dnum <= n_q, and n_p >= alpha (the special modulus must cover a digit).
+ * Zero bit sizes select 60 / 40 / 60.
+ */
+typedef struct {
+    int log_n;
+    int n_q;
+    int n_p;
+    int dnum;
+    int q0_bits;
+    int q_bits;
+    int p_bits;
+    const uint64_t* q; /* optional host array of n_q primes, or NULL */
+    const uint64_t* p; /* optional host array of n_p primes, or NULL */
+} he_params;
+
+/* A ciphertext: data is a device pointer to [2][level][N] uint64. */
+typedef struct {
+    uint64_t* data;
+    int level;
+    double scale;
+    int is_ntt;
+} he_ct;
+
+/* Context ------------------------------------------------------------------ */
+
+/* Host only (no device work): validates params and writes the n_q + n_p
+ * primes (prime index order) and their psi.  Either output may be NULL. */
+int he_derive_primes(const he_params* params, uint64_t* primes_out, uint64_t* psi_out);
+
+/* Builds the RNS tables on the host (primes, roots, twiddles, conversion
+ * constants) and uploads them.  cuda_stream: a cudaStream_t or NULL for the
+ * legacy default stream.  Synchronous.  *out receives the context. */
+int he_ctx_create(const he_params* params, void* cuda_stream, he_ctx** out);
+int he_ctx_destroy(he_ctx* ctx);
+int he_set_stream(he_ctx* ctx, void* cuda_stream);
+/* Blocks until the context's stream is idle; returns HE_ECUDA on a pending error. */
+int he_sync(he_ctx* ctx);
+const char* he_last_error(const he_ctx* ctx);
+/* Host copies of the n_q + n_p primes / of their psi (smallest primitive 2N-th roots). */
+int he_get_primes(const he_ctx* ctx, uint64_t* out);
+int he_get_psi(const he_ctx* ctx, uint64_t* out);
+
+/* Keys --------------------------------------------------------------------- */
+
+/*
+ * Computes one switching key on the device from caller-supplied random
+ * parts and keeps it in the context (hybrid key switching, Han-Ki section 3):
+ *   for digit j < ceil(L/alpha), on every prime of Q and P,
+ *     b_j = -a_j s + e_j + g_j s',  g_j = P on the primes of digit j, 0 elsewhere;
+ *   s' = sigma_k(s), k = 5^(step mod N/2) mod 2N   (kind HE_KEY_ROTATION)
+ *   s' = s^2                                        (kind HE_KEY_RELIN, step ignored)
+ * s: host int8[N] ternary secret coefficients.
+ * a: host uint64 [dnum][n_q+n_p][N], uniform residues, used as evaluation-domain values.
+ * e: host int32 [dnum][N], small error coefficients.
+ * Only the first ceil(L/alpha) digits of a and e are read.  Uploading a key
+ * that exists replaces it.  Synchronous.
+ */
+int he_keygen_upload(he_ctx* ctx, int kind, int32_t step, const int8_t* s, const uint64_t* a,
+                     const int32_t* e);
+/* Copies a key back in canonical residues: host uint64 [digits][2][n_q+n_p][N] (b then a). */
+int he_key_download(he_ctx* ctx, int kind, int32_t step, uint64_t* host_out);
+/* Number of key-switching digits at the top level, ceil(L / alpha). */
+int he_key_digits(const he_ctx* ctx);
+
+/* Transforms --------------------------------------------------------------- */
+
+/*
+ * In-place batched negacyclic NTT (coefficients -> evaluation values, storage
+ * index j = value at psi^(2 brev(j)+1)) / its inverse (including N^-1).
+ * d: device [n_polys][n_limbs][N]; limb i of every poly uses prime index
+ * first_prime + i.  Inputs must be canonical; outputs are canonical.
+ */
+int he_ntt_fwd(he_ctx* ctx, uint64_t* d, int n_polys, int n_limbs, int first_prime);
+int he_ntt_inv(he_ctx* ctx, uint64_t* d, int n_polys, int n_limbs, int first_prime);
+
+/* Operations --------------------------------------------------------------- */
+
+/*
+ * Slot rotation (AEGIS section 1 item 2: rotation needs key switching):
+ *   rot_r(ct) = (sigma_k(c0), 0) + KS_{evk_r}(sigma_k(c1)),  k = 5^(r mod N/2) mod 2N,
+ * slot j of the result = slot j + r of the input.  KS = ModUp (fast base
+ * conversion of each digit onto the other primes), inner product with the
+ * key, ModDown with centred conversion from P.  out gets in's level and
+ * scale; out->data must not overlap in->data.
+ */
+int he_rotate(he_ctx* ctx, const he_ct* in, int32_t step, he_ct* out);
+/* n independent rotations (in[i] by steps[i] into out[i]); all at one level.
+ * Ciphertexts that share a step share one read of its key. */
+int he_rotate_batch(he_ctx* ctx, const he_ct* in, const int32_t* steps, he_ct* out, int n);
+/* Host-buffer form of he_rotate_batch: h_in / h_out are host [n][2][level][N];
+ * the call copies in, rotates, copies out and waits.  Pinned host memory
+ * gives full copy bandwidth.  Synchronous. */
+int he_rotate_batch_host(he_ctx* ctx, const uint64_t* h_in, int level, const int32_t* steps,
+                         uint64_t* h_out, int n);
+
+/* Tensor, relinearise (key switch of d2 with the s^2 key), rescale.
+ * a and b at the same level l >= 2; out at level l-1, scale (sa*sb)/q_{l-1}.
+ * out->data must not overlap the inputs. */
+int he_hmult_relin_rescale(he_ctx* ctx, const he_ct* a, const he_ct* b, he_ct* out);
+/* Divide by q_{l-1} with rounding: c'_i = (c_i - [c_{l-1}]) q_{l-1}^-1 mod q_i with
+ * [c_{l-1}] the centred coefficient representative.  In place: level-1, scale/q_{l-1}. */
+int he_rescale(he_ctx* ctx, he_ct* inout);
+
+/* Helpers: ct + ct (same level; scale of a kept), ct * K (integer, any sign),
+ * ct + K (K added to the constant coefficient: every slot gains K/scale),
+ * keep limbs q_0..q_{level-1}.  out may equal the input. */
+int he_add(he_ctx* ctx, const he_ct* a, const he_ct* b, he_ct* out);
+int he_mul_const(he_ctx* ctx, const he_ct* in, int64_t K, he_ct* out);
+int he_add_const(he_ctx* ctx, he_ct* inout, int64_t K);
+int he_drop_level(he_ctx* ctx, const he_ct* in, int level, he_ct* out);
+
+/*
+ * Plaintext-weight x ciphertext block product by the diagonal method with
+ * baby-step/giant-step (AEGIS section 2.2: the FFN is a local polynomial
+ * multiplication per output group).  For each token group t < n_groups and
+ * output block i < n_out:
+ *   Y[t][i] = rescale( sum_g rot_{stride*bs*g}( sum_{j,b} pt[i][j][g][b] (.) rot_{stride*b}(X[t][j]) ) )
+ * x: n_groups*n_in ciphertexts (group-major) at one level l >= 2.
+ * d_pt: device [n_out][n_in][gs][bs][l][N] evaluation-domain plaintexts,
+ *       encoded at pt_scale.
+ * y: n_groups*n_out ciphertexts (group-major) with room for level l; they
+ *    come back at level l-1, scale x.scale*pt_scale/q_{l-1}.
+ * Needs rotation keys for stride*b (0<b<bs) and stride*bs*g (0<g<gs).
+ */
+int he_pmult_accum_bsgs(he_ctx* ctx, const he_ct* x, int n_in, const uint64_t* d_pt, double pt_scale,
+                        int n_out, int bs, int gs, int slot_stride, int n_groups, he_ct* y);
+
+/*
+ * Degree-15 polynomial sum_k c_k x^k by Paterson-Stockmeyer with 4 baby
+ * powers (AEGIS section 2.3: Softmax by polynomial approximation):
+ *   x2 = HMRR(x,x); x3 = HMRR(x2, drop(x)); x4 = HMRR(x2,x2);
+ *   q_i = sum_{j<4} c_{4i+j} x^j built at (level, T): each x^j is dropped to
+ *         level+1, multiplied by K = round_half_away(c*T*q_level/S_j) (fp64,
+ *         left to right) and rescaled; the constant adds round_half_away(c*T);
+ *   acc = q_3 at (l0-3, top_scale); acc = HMRR(acc, drop(x4)) + q_i, i = 2, 1, 0,
+ *         each q_i at the accumulator's exact level and scale.
+ * HMRR = he_hmult_relin_rescale.  x: n ciphertexts at level l0 >= 7;
+ * out: n ciphertexts with room for level l0; they come back at level l0-6.
+ */
+int he_poly_eval_ps15(he_ctx* ctx, const he_ct* x, int n, const double* coeffs, double top_scale,
+                      he_ct* out);
+
+/* Measurement -------------------------------------------------------------- */
+
+/* Kernel classes timed by the profiler. */
+#define HE_PROF_NTT_FWD 0
+#define HE_PROF_NTT_INV 1
+#define HE_PROF_MODUP 2
+#define HE_PROF_KS_INNER 3
+#define HE_PROF_MODDOWN 4
+#define HE_PROF_AUTOMORPH 5
+#define HE_PROF_ELEMENTWISE 6
+#define HE_PROF_RESCALE 7
+#define HE_PROF_PMULT 8
+#define HE_PROF_N 9
+
+/* enable != 0: every kernel launch is bracketed by CUDA events on the
+ * context's stream and its time is added to its class.  Resets the totals. */
+int he_profile_enable(he_ctx* ctx, int enable);
+/* Waits for the stream, then returns total milliseconds and launches of one class. */
+int he_profile_read(he_ctx* ctx, int cls, double* total_ms, long long* launches);
+/* Kernels this context has launched since creation or the last reset. */
+long long he_launch_count(he_ctx* ctx, int reset);
+
+/* HBM copy probe: dst[i] = src[i] for n_words uint64 (device pointers),
+ * grid-stride, 16-byte accesses.  Asynchronous. */
+int he_probe_copy(he_ctx* ctx, uint64_t* dst, const uint64_t* src, size_t n_words);
+/* Integer probe: every thread of a full-GPU grid runs `iters` rounds of
+ * independent 64-bit Shoup modular multiplications in registers and writes
+ * one word to sink[thread].  sink: device, >= he_probe_int_threads() words.
+ * Asynchronous. */
+int he_probe_int(he_ctx* ctx, int iters, uint64_t* sink);
+long long he_probe_int_threads(he_ctx* ctx);
+/* 64-bit modular multiplications one he_probe_int thread performs per iteration. */
+int he_probe_int_mults_per_iter(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HE_B200_H */

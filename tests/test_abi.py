@@ -1,0 +1,71 @@
+"""The C ABI (include/he.h): library loads, exports every declared symbol,
+derives the same parameters as the oracle, and rejects bad arguments on the
+host.  No device work."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from oracle import ckks as C
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def he():
+    import __graft_entry__
+
+    __graft_entry__.build()
+    from homomorphic_encrypted_transformer_b200 import he as mod
+
+    return mod
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "he.h")).read()
+    return re.findall(r"^\s*(?:int|const char\*|long long)\s+(he_\w+)\(", src, re.M)
+
+
+def test_header_declares_the_hot_path_calls():
+    names = set(declared_functions())
+    for n in ["he_keygen_upload", "he_ntt_fwd", "he_ntt_inv", "he_rotate", "he_hmult_relin_rescale",
+              "he_pmult_accum_bsgs", "he_rescale"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(he):
+    lib = ctypes.CDLL(he.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert hasattr(he, name), "binding lacks " + name
+
+
+@pytest.mark.parametrize("log_n,L,K,dnum", [(12, 3, 1, 3), (16, 24, 8, 3), (11, 3, 1, 3), (12, 8, 3, 3),
+                                            (10, 7, 3, 3)])
+def test_library_derives_oracle_primes_and_roots(he, log_n, L, K, dnum):
+    P = C.Params(log_n, L, K, dnum)
+    primes, psi = he.he_derive_primes(log_n, L, K, dnum)
+    assert primes == P.mods
+    assert psi == P.psi
+
+
+@pytest.mark.parametrize("args", [(9, 3, 1, 3), (17, 3, 1, 3), (12, 0, 1, 1), (12, 3, 0, 3), (12, 3, 1, 4),
+                                  (12, 24, 4, 3), (12, 40, 30, 3)])
+def test_invalid_parameters_rejected_on_host(he, args):
+    with pytest.raises(he.HEError) as ei:
+        he.he_derive_primes(*args)
+    assert ei.value.code == he.HE_EINVAL
+    with pytest.raises(he.HEError) as ei:
+        he.he_ctx_create(*args)
+    assert ei.value.code == he.HE_EINVAL
+
+
+def test_explicit_primes_checked(he):
+    P = C.Params(12, 3, 1, 3)
+    primes, _ = he.he_derive_primes(12, 3, 1, 3, q=P.q, p=P.p)
+    assert primes == P.mods
+    with pytest.raises(he.HEError):  # not = 1 mod 2N
+        he.he_derive_primes(12, 3, 1, 3, q=[P.q[0], P.q[1], 1000003], p=P.p)
+    with pytest.raises(he.HEError):  # repeated prime
+        he.he_derive_primes(12, 3, 1, 3, q=[P.q[0], P.q[1], P.q[1]], p=P.p)

@@ -1,0 +1,152 @@
+"""GPU parity: switching keys and key-switched rotation vs the oracle, bit-exact
+on every residue, plus decrypted slots within 1e-5 of the rolled plaintext."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import ckks as C
+import seeded_inputs as S
+from tests.helpers import Setup, host, lib
+
+pytestmark = pytest.mark.gpu
+
+
+def test_keygen_matches_oracle_tiny():
+    he = lib()
+    st = Setup(12, 3, 1, 3, seed=S.master_seed(0))
+    for step in (1, 2, -1):
+        st.upload_rot(step)
+        got = he.he_key_download(st.ctx, he.HE_KEY_ROTATION, step)
+        b, a = st.oracle_rot_key(step)
+        assert np.array_equal(got[:, 0], b) and np.array_equal(got[:, 1], a)
+    st.upload_relin()
+    got = he.he_key_download(st.ctx, he.HE_KEY_RELIN, 0)
+    b, a = st.oracle_relin_key()
+    assert np.array_equal(got[:, 0], b) and np.array_equal(got[:, 1], a)
+
+
+def test_keygen_matches_oracle_full_size():
+    he = lib()
+    st = Setup(16, 24, 8, 3, seed=S.master_seed(1))
+    st.upload_rot(12345)
+    got = he.he_key_download(st.ctx, he.HE_KEY_ROTATION, 12345)
+    b, a = st.oracle_rot_key(12345)
+    assert np.array_equal(got[:, 0], b) and np.array_equal(got[:, 1], a)
+
+
+def test_rotation_tiny_config():
+    """N=2^12, 3+1 primes, steps {1, 2, -1}."""
+    he = lib()
+    st = Setup(12, 3, 1, 3, seed=S.master_seed(0))
+    P = st.P
+    z = S.complex_slots(st.seed, P.n_slots, -1, 1)
+    ct = st.encrypt(z, 3)
+    x = st.to_gpu(ct)
+    for step in (1, 2, -1):
+        st.upload_rot(step)
+        y = st.empty_gpu(3)
+        he.he_rotate(st.ctx, x, step, y)
+        he.he_sync(st.ctx)
+        want = C.rotate(ct, step, st.oracle_rot_key(step), P)
+        assert y.level == 3 and y.scale == ct["scale"]
+        assert np.array_equal(st.from_gpu(y), want["c"])
+        assert np.max(np.abs(C.decrypt_decode(want, st.s, P) - np.roll(z, -step))) < 1e-5
+
+
+@pytest.mark.parametrize("level", [7, 5, 4, 1])
+def test_rotation_mid_levels(level):
+    """Several primes per digit (alpha = 3), partial last digits, level 1."""
+    he = lib()
+    st = Setup(11, 7, 3, 3, seed=44)
+    P = st.P
+    z = S.complex_slots(st.seed, P.n_slots, -1, 1)
+    ct = st.encrypt(z, level)
+    step = 5
+    st.upload_rot(step)
+    x = st.to_gpu(ct)
+    y = st.empty_gpu(level)
+    he.he_rotate(st.ctx, x, step, y)
+    he.he_sync(st.ctx)
+    want = C.rotate(ct, step, st.oracle_rot_key(step), P)
+    assert np.array_equal(st.from_gpu(y), want["c"])
+
+
+def test_rotation_errors():
+    he = lib()
+    st = Setup(12, 3, 1, 3, seed=3)
+    z = S.complex_slots(st.seed, st.P.n_slots, -1, 1)
+    x = st.to_gpu(st.encrypt(z, 3))
+    y = st.empty_gpu(3)
+    with pytest.raises(he.HEError) as ei:
+        he.he_rotate(st.ctx, x, 7, y)
+    assert ei.value.code == he.HE_ENOKEY
+    with pytest.raises(he.HEError) as ei:
+        he.he_rotate(st.ctx, x, 7, x)
+    assert ei.value.code == he.HE_EINVAL
+    x.is_ntt = False
+    st.upload_rot(7)
+    with pytest.raises(he.HEError) as ei:
+        he.he_rotate(st.ctx, x, 7, y)
+    assert ei.value.code == he.HE_EDOMAIN
+
+
+def _rotation_batch_inputs(st, n_cts, n_keys):
+    P = st.P
+    steps = S.rotation_steps(st.seed, n_keys, 1, P.n_slots - 1)
+    assign = S.step_assignment(st.seed, n_cts, n_keys)
+    return steps, [steps[u] for u in assign]
+
+
+def test_rotation_batch_full_size_sampled():
+    """The rotation-batch workload (N=2^16, L=24, K=8, dnum=3, 64 ciphertexts,
+    16 seeded keys) in the launch configuration the benchmark times; three
+    ciphertexts chosen by seed are recomputed by the oracle."""
+    he = lib()
+    st = Setup(16, 24, 8, 3, seed=S.master_seed(1))
+    P = st.P
+    n_cts, n_keys = 64, 16
+    steps, ct_steps = _rotation_batch_inputs(st, n_cts, n_keys)
+    for s_ in steps:
+        st.upload_rot(s_)
+    sample = S.choose_groups(st.seed, n_cts, 3)
+    # real encryptions at the sampled positions, uniform residues elsewhere
+    # (a fresh encryption is computationally indistinguishable from uniform)
+    xs, cts = [], {}
+    uni = S.uniform_residues(st.seed, "ct_residues", P.q, P.N, lead=(n_cts, 2))
+    for i in range(n_cts):
+        if i in sample:
+            z = S.complex_slots(st.seed, P.n_slots, -1, 1, i)
+            cts[i] = (st.encrypt(z, 24, ct_id=i), z)
+            xs.append(st.to_gpu(cts[i][0]))
+        else:
+            xs.append(st.to_gpu(C.make_ct(uni[i], 24, 2.0 ** 40)))
+    ys = [st.empty_gpu(24) for _ in range(n_cts)]
+    he.he_rotate_batch(st.ctx, xs, ct_steps, ys)
+    he.he_sync(st.ctx)
+    for i in sample:
+        ct, z = cts[i]
+        want = C.rotate(ct, ct_steps[i], st.oracle_rot_key(ct_steps[i]), P)
+        assert np.array_equal(st.from_gpu(ys[i]), want["c"]), i
+        assert np.max(np.abs(C.decrypt_decode(want, st.s, P) - np.roll(z, -ct_steps[i]))) < 1e-5
+    # the uniform-residue ciphertexts: outputs canonical
+    for i in range(n_cts):
+        out = st.from_gpu(ys[i])
+        assert np.all(out < np.array(P.q, dtype=np.uint64)[None, :, None])
+
+
+def test_rotation_batch_host_buffers():
+    """The host-buffer entry point gives the same residues as the device one."""
+    he = lib()
+    st = Setup(12, 3, 1, 3, seed=5)
+    P = st.P
+    n = 5
+    steps = [1, 2, 1, 3, 2]
+    for s_ in set(steps):
+        st.upload_rot(s_)
+    cts = [st.encrypt(S.complex_slots(st.seed, P.n_slots, -1, 1, i), 3, ct_id=i) for i in range(n)]
+    h_in = np.stack([c["c"] for c in cts])
+    h_out = np.zeros_like(h_in)
+    he.he_rotate_batch_host(st.ctx, h_in, 3, steps, h_out)
+    for i in range(n):
+        want = C.rotate(cts[i], steps[i], st.oracle_rot_key(steps[i]), P)
+        assert np.array_equal(h_out[i], want["c"])
