@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--case", default="rotation", choices=["rotation", "ntt"],
+                    help="ntt: NTT-only kernel case for profiler captures (no JSON metric line)")
     return ap.parse_args()
 
 
@@ -173,16 +175,24 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------------------ native
 
-# algorithmic work per launch of each kernel class for the rotation batch
-def class_work(cls, n_cts):
-    N = 1 << LOG_N
-    lvl, nd = LEVEL, -(-LEVEL // (-(-L // DNUM)))
-    rows_ext = lvl + K
-    w = 8
-    if cls == "ks_inner":
-        # ext reads + key (once per key group) + u writes; 2*nd Montgomery MACs per output pair
-        return {"bytes": None, "mults": n_cts * rows_ext * N * 2 * nd}
-    return None
+def run_ntt_case(args, local_rank):
+    """Kernel case for profiler captures: forward and inverse NTT of 512
+    limbs of 2^16 words (256 MiB, larger than L2), all 32 primes cycled."""
+    import torch
+
+    from homomorphic_encrypted_transformer_b200 import he
+
+    torch.cuda.set_device(local_rank)
+    ctx = he.he_ctx_create(LOG_N, L, K, DNUM, stream=torch.cuda.current_stream())
+    n_polys, n_limbs = 16, L + K
+    h = S.uniform_residues(S.master_seed(1), "ntt_residues", ctx.primes, ctx.N, lead=(n_polys,))
+    d = torch.from_numpy(h.view(np.int64)).cuda()
+    for _ in range(args.warmup + args.steps):
+        he.he_ntt_fwd(ctx, d, n_polys, n_limbs, 0)
+        he.he_ntt_inv(ctx, d, n_polys, n_limbs, 0)
+    torch.cuda.synchronize()
+    ok = np.array_equal(d.cpu().numpy().view(np.uint64), h)
+    print(json.dumps({"case": "ntt", "rows": n_polys * n_limbs, "roundtrip_ok": bool(ok)}))
 
 
 def run_native(args, rank, world, local_rank):
@@ -306,14 +316,13 @@ def run_native(args, rank, world, local_rank):
     pk, pk_kind = peaks()
     hbm_peak = float(pk.get("hbm_gbs", 6650.0))
     # dominant kernel class by device time in the profiled pass
-    dom = max(prof.items(), key=lambda kv: kv[1][0])
-    dom_name, (dom_ms, dom_launches) = dom
+    dom_name = max(prof, key=lambda k: prof[k][0])
     ct_bytes = 2 * LEVEL * N * 8
     key_bytes = 3 * 2 * (L + K) * N * 8
     # algorithmic bytes of one rotation batch (keys read once per key group)
     batch_bytes = N_KEYS * key_bytes + N_CTS * 2 * ct_bytes
     hbm_frac_step = (batch_bytes / (ms_plain * 1e-3 / args.steps)) / 1e9 / hbm_peak
-    roof = roofline_for(dom_name, dom_ms / max(1, dom_launches), args, N, int_modmul_s, hbm_peak, pk_kind)
+    roof = roofline_for(dom_name, prof[dom_name], int_modmul_s, hbm_peak, pk_kind)
     line = {"metric": METRIC, "value": value, "unit": "rotations/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_plain / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u64", "data": "synthetic",
@@ -321,7 +330,7 @@ def run_native(args, rank, world, local_rank):
             "hbm_roofline_frac_of_step": hbm_frac_step,
             "roofline": roof,
             "probes": {"copy_gbs": copy_gbs, "int_shoup_modmul_per_s": int_modmul_s},
-            "kernel_ms_per_step": {k: v[0] / args.steps for k, v in prof.items() if v[1]},
+            "kernel_ms_per_step": {k: round(v[0] / args.steps, 4) for k, v in prof.items() if v[1]},
             "kernel_launches_per_step": {k: v[1] / args.steps for k, v in prof.items() if v[1]},
             "profiled_ms_per_step": ms / args.steps,
             "gpu_launches": launches,
@@ -333,10 +342,36 @@ def run_native(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
-def roofline_for(name, ms_per_launch, args, N, int_modmul_s, hbm_peak, pk_kind):
-    return {"kernel_class": name, "ms_per_launch": ms_per_launch, "bound": None, "achieved": None,
-            "peak": hbm_peak, "unit": "GB/s", "frac": None, "traffic": None,
-            "peak_source": pk_kind}
+# ncu dram bytes (read + write) over algorithmic bytes, per kernel, from the
+# committed captures in profiles/ (a 512-limb launch; the benchmark's launches
+# process 288 limbs on average, so the traffic is scaled by limbs processed).
+# Remove an entry when its kernel changes.
+NCU_TRAFFIC_RATIO = {"ntt_fwd_cols": 540.3 / 536.9, "ntt_fwd_rows": 859.7 / 536.9}
+
+
+def roofline_for(name, prof_entry, int_modmul_s, hbm_peak, pk_kind):
+    """Roofline of the dominant kernel class: its algorithmic bytes and
+    modular multiplications per launch (counted by the library as it
+    launches) against its CUDA-event duration.  The binding resource is the
+    one whose peak gives the longer ideal time."""
+    ms, launches, nbytes, mults = prof_entry
+    launches = max(1, launches)
+    t = ms * 1e-3 / launches
+    b, m = nbytes / launches, mults / launches
+    t_hbm = b / (hbm_peak * 1e9)
+    t_alu = m / int_modmul_s if int_modmul_s > 0 else 0.0
+    traffic = NCU_TRAFFIC_RATIO[name] * b if name in NCU_TRAFFIC_RATIO else None
+    if t_hbm >= t_alu:
+        ach = b / t / 1e9
+        return {"kernel": name, "bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
+                "frac": ach / hbm_peak, "traffic": traffic, "algorithmic_bytes_per_launch": b,
+                "ms_per_launch": t * 1e3, "peak_source": pk_kind + " (MEASURED_PEAKS.json hbm_gbs)"}
+    ach = m / t / 1e9
+    peak = int_modmul_s / 1e9
+    return {"kernel": name, "bound": "alu", "achieved": ach, "peak": peak, "unit": "Gmodmul/s",
+            "frac": ach / peak, "traffic": traffic, "algorithmic_modmuls_per_launch": m,
+            "algorithmic_bytes_per_launch": b, "ms_per_launch": t * 1e3,
+            "peak_source": "in-run probe: register-only 64-bit Shoup modular products, full grid"}
 
 
 def main():
@@ -357,6 +392,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.case == "ntt":
+            run_ntt_case(args, local_rank)
         else:
             run_native(args, rank, world, local_rank)
     finally:

@@ -187,14 +187,17 @@ void prof_begin(he_ctx* c, int cls) {
     p.cls = cls;
     p.a = ev_get(c);
     p.b = nullptr;
+    p.bytes = p.mults = 0;
     cudaEventRecord(p.a, c->stream);
     c->prof_pending.push_back(p);
 }
 
-int prof_end(he_ctx* c, int cls) {
+int prof_end(he_ctx* c, int cls, double bytes, double mults) {
     if (!c->prof_on || c->prof_pending.empty()) return HE_OK;
     ProfPending& p = c->prof_pending.back();
     if (p.cls != cls || p.b) return HE_OK;
+    p.bytes = bytes;
+    p.mults = mults;
     p.b = ev_get(c);
     cudaEventRecord(p.b, c->stream);
     return HE_OK;
@@ -209,6 +212,8 @@ static int prof_collect(he_ctx* c) {
             cudaEventElapsedTime(&ms, p.a, p.b);
             c->prof[p.cls].ms += ms;
             c->prof[p.cls].launches += 1;
+            c->prof[p.cls].bytes += p.bytes;
+            c->prof[p.cls].mults += p.mults;
             c->ev_pool.push_back(p.b);
         }
         c->ev_pool.push_back(p.a);
@@ -520,12 +525,15 @@ extern "C" int he_profile_enable(he_ctx* c, int enable) {
     return HE_OK;
 }
 
-extern "C" int he_profile_read(he_ctx* c, int cls, double* ms, long long* launches) {
+extern "C" int he_profile_read(he_ctx* c, int cls, double* ms, long long* launches, double* bytes,
+                               double* mults) {
     if (!c || cls < 0 || cls >= HE_PROF_N) return HE_EINVAL;
     int rc = prof_collect(c);
     if (rc) return rc;
     if (ms) *ms = c->prof[cls].ms;
     if (launches) *launches = c->prof[cls].launches;
+    if (bytes) *bytes = c->prof[cls].bytes;
+    if (mults) *mults = c->prof[cls].mults;
     return HE_OK;
 }
 

@@ -33,11 +33,13 @@ struct Key {
 struct ProfSlot {
     double ms = 0;
     long long launches = 0;
+    double bytes = 0, mults = 0;
 };
 
 struct ProfPending {
     int cls;
     cudaEvent_t a, b;
+    double bytes, mults;
 };
 
 }  // namespace he
@@ -85,8 +87,10 @@ namespace he {
 int set_err(he_ctx* c, int code, const char* fmt, ...);
 int check_cuda(he_ctx* c, cudaError_t e, const char* what);
 
+// Brackets launches of one class with events; prof_end records the
+// algorithmic work (HBM bytes, modular multiplications) of what it closes.
 void prof_begin(he_ctx* c, int cls);
-int prof_end(he_ctx* c, int cls);
+int prof_end(he_ctx* c, int cls, double bytes = 0, double mults = 0);
 
 uint64_t galois_elt(const he_ctx* c, int32_t step);
 

@@ -207,10 +207,14 @@ int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList
     dim3 blk(TB);
     int gx = (N + TB - 1) / TB;
 
+    const double limbB = 8.0 * N;
+    int sum_src = 0;
+    for (int j = 0; j < nd; j++) sum_src += ma.n_src[j];
+
     prof_begin(c, HE_PROF_AUTOMORPH);
     k_gather<<<dim3(gx, level, n), blk, 0, c->stream>>>(din, coef, level, c->log_n, io.galois);
     if ((rc = lc(c, "gather"))) return rc;
-    prof_end(c, HE_PROF_AUTOMORPH);
+    prof_end(c, HE_PROF_AUTOMORPH, 2.0 * n * level * limbB, 0);
 
     std::vector<int> qp = prime_range(0, level);
     if ((rc = ntt_inv_set(c, rowset_contig(coef, level, N, qp), n * level))) return rc;
@@ -218,7 +222,8 @@ int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList
     prof_begin(c, HE_PROF_MODUP);
     k_modup_conv<<<dim3(gx, nd, n), blk, 0, c->stream>>>(coef, ext, ma, c->d_prime, level, n_rows, c->log_n);
     if ((rc = lc(c, "modup_conv"))) return rc;
-    prof_end(c, HE_PROF_MODUP);
+    prof_end(c, HE_PROF_MODUP, (double)n * (sum_src + nd * n_rows) * limbB,
+             (double)n * N * (sum_src + (double)sum_src * n_rows));
 
     std::vector<int> ep = ext_primes(c, level);
     if ((rc = ntt_fwd_set(c, rowset_contig(ext, n_rows, N, ep), n * nd * n_rows))) return rc;
@@ -227,26 +232,31 @@ int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList
     k_ks_inner<<<dim3(gx, n_rows, n), blk, 0, c->stream>>>(ext, key.d, u, nd, n_rows, level, L, LK, c->d_prime, ma,
                                                            c->log_n);
     if ((rc = lc(c, "ks_inner"))) return rc;
-    prof_end(c, HE_PROF_KS_INNER);
+    prof_end(c, HE_PROF_KS_INNER, ((double)n * nd * n_rows + 2.0 * nd * n_rows + 2.0 * n * n_rows) * limbB,
+             (double)n * n_rows * N * (2.0 * nd + 2));
 
     std::vector<int> pp = prime_range(L, K);
     RowSet prs = rowset(u + (size_t)level * N, (long long)n_rows * N, K, pp.data());
     if ((rc = ntt_inv_set(c, prs, n * 2 * K))) return rc;
 
-    prof_begin(c, HE_PROF_MODDOWN);
+    prof_begin(c, HE_PROF_MODDOWN_CONV);
     k_moddown_conv<<<dim3(gx, 2, n), blk, 0, c->stream>>>(u, tmp, level, K, L, c->d_prime, c->d_md_pcoef,
                                                           c->d_md_mat, c->d_md_negP, c->log_n);
     if ((rc = lc(c, "moddown_conv"))) return rc;
-    prof_end(c, HE_PROF_MODDOWN);
+    prof_end(c, HE_PROF_MODDOWN_CONV, 2.0 * n * (K + level) * limbB, 2.0 * n * N * (K + (double)K * level));
 
     if ((rc = ntt_fwd_set(c, rowset_contig(tmp, level, N, qp), n * 2 * level))) return rc;
 
-    prof_begin(c, HE_PROF_MODDOWN);
+    prof_begin(c, HE_PROF_MODDOWN_COMBINE);
     k_moddown_combine<<<dim3(gx, 2 * level, n), blk, 0, c->stream>>>(u, tmp, dout, a0, a1, io.sig_add0 ? 1 : 0,
                                                                      io.galois, level, K, c->d_prime, c->d_md_pinv,
                                                                      c->log_n);
     if ((rc = lc(c, "moddown_combine"))) return rc;
-    prof_end(c, HE_PROF_MODDOWN);
+    {
+        int n_add = 0;
+        for (int i = 0; i < n; i++) n_add += (io.add0[i] != nullptr) + (io.add1[i] != nullptr);
+        prof_end(c, HE_PROF_MODDOWN_COMBINE, (6.0 * n + n_add) * level * limbB, 2.0 * n * level * N);
+    }
     return HE_OK;
 }
 

@@ -106,31 +106,37 @@ int ntt_fwd_set(he_ctx* c, const RowSet& rs, int n_rows) {
     if (n_rows <= 0) return HE_OK;
     NttShape sh = ntt_shape(c->log_n);
     dim3 g1(sh.col_tiles, n_rows), g2(sh.row_tiles, n_rows);
-    prof_begin(c, HE_PROF_NTT_FWD);
+    const double bytes = 16.0 * c->N * n_rows, half = 0.5 * c->N * n_rows;
+    prof_begin(c, HE_PROF_NTT_FWD_COLS);
     k_ntt_fwd_cols<<<g1, 256, sh.smem_cols, c->stream>>>(rs, c->d_prime, c->d_tw_fwd, c->log_n, sh.s1, sh.tc);
     int rc = launch_check(c, "ntt_fwd_cols");
     if (rc) return rc;
+    prof_end(c, HE_PROF_NTT_FWD_COLS, bytes, half * sh.s1);
+    prof_begin(c, HE_PROF_NTT_FWD_ROWS);
     k_ntt_fwd_rows<<<g2, 256, sh.smem_rows, c->stream>>>(rs, c->d_prime, c->d_tw_fwd, c->log_n, sh.s1, sh.tr);
     rc = launch_check(c, "ntt_fwd_rows");
     if (rc) return rc;
     c->launches += 2;
-    return prof_end(c, HE_PROF_NTT_FWD);
+    return prof_end(c, HE_PROF_NTT_FWD_ROWS, bytes, half * sh.s2);
 }
 
 int ntt_inv_set(he_ctx* c, const RowSet& rs, int n_rows) {
     if (n_rows <= 0) return HE_OK;
     NttShape sh = ntt_shape(c->log_n);
     dim3 g1(sh.col_tiles, n_rows), g2(sh.row_tiles, n_rows);
-    prof_begin(c, HE_PROF_NTT_INV);
+    const double bytes = 16.0 * c->N * n_rows, half = 0.5 * c->N * n_rows;
+    prof_begin(c, HE_PROF_NTT_INV_ROWS);
     k_ntt_inv_rows<<<g2, 256, sh.smem_rows, c->stream>>>(rs, c->d_prime, c->d_tw_inv, c->log_n, sh.s1, sh.tr);
     int rc = launch_check(c, "ntt_inv_rows");
     if (rc) return rc;
+    prof_end(c, HE_PROF_NTT_INV_ROWS, bytes, half * sh.s2);
+    prof_begin(c, HE_PROF_NTT_INV_COLS);
     k_ntt_inv_cols<<<g1, 256, sh.smem_cols, c->stream>>>(rs, c->d_prime, c->d_tw_inv, c->d_inv_last, c->log_n, sh.s1,
                                                           sh.tc);
     rc = launch_check(c, "ntt_inv_cols");
     if (rc) return rc;
     c->launches += 2;
-    return prof_end(c, HE_PROF_NTT_INV);
+    return prof_end(c, HE_PROF_NTT_INV_COLS, bytes, half * sh.s1);
 }
 
 int ntt_setup(he_ctx* c) {

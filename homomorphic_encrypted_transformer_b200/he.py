@@ -30,8 +30,8 @@ HE_ETIMEOUT = -7
 HE_KEY_ROTATION = 0
 HE_KEY_RELIN = 1
 
-PROF = {"ntt_fwd": 0, "ntt_inv": 1, "modup": 2, "ks_inner": 3, "moddown": 4, "automorph": 5,
-        "elementwise": 6, "rescale": 7, "pmult": 8}
+PROF = {"ntt_fwd_cols": 0, "ntt_fwd_rows": 1, "ntt_inv_rows": 2, "ntt_inv_cols": 3, "modup": 4, "ks_inner": 5,
+        "moddown_conv": 6, "moddown_combine": 7, "automorph": 8, "elementwise": 9, "rescale": 10, "pmult": 11}
 
 _CODES = {HE_EINVAL: "HE_EINVAL", HE_ELEVEL: "HE_ELEVEL", HE_ENOKEY: "HE_ENOKEY", HE_EDOMAIN: "HE_EDOMAIN",
           HE_ENOMEM: "HE_ENOMEM", HE_ECUDA: "HE_ECUDA", HE_ETIMEOUT: "HE_ETIMEOUT"}
@@ -92,7 +92,8 @@ _sig("he_pmult_accum_bsgs", _i, _vp, ctypes.POINTER(he_ct), _i, _vp, ctypes.c_do
      ctypes.POINTER(he_ct))
 _sig("he_poly_eval_ps15", _i, _vp, ctypes.POINTER(he_ct), _i, _vp, ctypes.c_double, ctypes.POINTER(he_ct))
 _sig("he_profile_enable", _i, _vp, _i)
-_sig("he_profile_read", _i, _vp, _i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong))
+_sig("he_profile_read", _i, _vp, _i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong),
+     ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double))
 _sig("he_launch_count", ctypes.c_longlong, _vp, _i)
 _sig("he_probe_copy", _i, _vp, _vp, _vp, ctypes.c_size_t)
 _sig("he_probe_int", _i, _vp, _i, _vp)
@@ -330,10 +331,14 @@ def he_profile_enable(ctx, enable):
 
 
 def he_profile_read(ctx, cls):
+    """(total ms, launches, algorithmic HBM bytes, modular multiplications) of one class."""
     ms = ctypes.c_double()
     n = ctypes.c_longlong()
-    _check(ctx, _lib.he_profile_read(ctx.ptr, cls, ctypes.byref(ms), ctypes.byref(n)))
-    return ms.value, n.value
+    b = ctypes.c_double()
+    m = ctypes.c_double()
+    _check(ctx, _lib.he_profile_read(ctx.ptr, cls, ctypes.byref(ms), ctypes.byref(n), ctypes.byref(b),
+                                     ctypes.byref(m)))
+    return ms.value, n.value, b.value, m.value
 
 
 def he_launch_count(ctx, reset=False):

@@ -209,22 +209,30 @@ int he_poly_eval_ps15(he_ctx* ctx, const he_ct* x, int n, const double* coeffs, 
 /* Measurement -------------------------------------------------------------- */
 
 /* Kernel classes timed by the profiler. */
-#define HE_PROF_NTT_FWD 0
-#define HE_PROF_NTT_INV 1
-#define HE_PROF_MODUP 2
-#define HE_PROF_KS_INNER 3
-#define HE_PROF_MODDOWN 4
-#define HE_PROF_AUTOMORPH 5
-#define HE_PROF_ELEMENTWISE 6
-#define HE_PROF_RESCALE 7
-#define HE_PROF_PMULT 8
-#define HE_PROF_N 9
+#define HE_PROF_NTT_FWD_COLS 0
+#define HE_PROF_NTT_FWD_ROWS 1
+#define HE_PROF_NTT_INV_ROWS 2
+#define HE_PROF_NTT_INV_COLS 3
+#define HE_PROF_MODUP 4
+#define HE_PROF_KS_INNER 5
+#define HE_PROF_MODDOWN_CONV 6
+#define HE_PROF_MODDOWN_COMBINE 7
+#define HE_PROF_AUTOMORPH 8
+#define HE_PROF_ELEMENTWISE 9
+#define HE_PROF_RESCALE 10
+#define HE_PROF_PMULT 11
+#define HE_PROF_N 12
 
 /* enable != 0: every kernel launch is bracketed by CUDA events on the
  * context's stream and its time is added to its class.  Resets the totals. */
 int he_profile_enable(he_ctx* ctx, int enable);
-/* Waits for the stream, then returns total milliseconds and launches of one class. */
-int he_profile_read(he_ctx* ctx, int cls, double* total_ms, long long* launches);
+/* Waits for the stream, then returns total milliseconds and launches of one
+ * class, and the algorithmic work of those launches: bytes that must cross
+ * HBM (each input read once, each output written once) and 64-bit modular
+ * multiplications (NTT butterflies, conversion and inner-product products).
+ * Any output pointer may be NULL. */
+int he_profile_read(he_ctx* ctx, int cls, double* total_ms, long long* launches, double* bytes,
+                    double* modmuls);
 /* Kernels this context has launched since creation or the last reset. */
 long long he_launch_count(he_ctx* ctx, int reset);
 

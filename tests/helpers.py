@@ -89,7 +89,7 @@ class Setup:
 
     def from_gpu(self, gct):
         lev = gct.level
-        return host(gct.data)[: 2 * lev * self.P.N].reshape(2, lev, self.P.N)
+        return host(gct.data).reshape(-1)[: 2 * lev * self.P.N].reshape(2, lev, self.P.N)
 
 
 def random_rows(seed, mods, n_polys, N):
