@@ -14,6 +14,7 @@
 namespace he {
 
 constexpr int kMaxPrimes = 64;
+constexpr int kMaxDevices = 64;
 
 // ModUp fast base conversion of one digit at one level, on device:
 //   y_i = [x_i * qhat_inv_i]_{q_i} for the digit's source primes,

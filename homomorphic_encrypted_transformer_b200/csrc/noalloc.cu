@@ -1,0 +1,114 @@
+// he_rescale_noalloc: the rescale of he_rescale with its scratch memory in a
+// fixed device array of this library instead of memory the context allocates.
+//
+// Who needs it: callers that must not allocate device memory while they run.
+// Examples are serving runtimes that reserve all of a GPU's memory up front
+// and hand it out themselves, processes whose remaining device memory belongs
+// to another allocator, and latency-sensitive callers that cannot afford the
+// device-wide synchronisation a cudaMalloc/cudaFree may cause.  This entry
+// point calls neither, nor any routine that allocates.
+//
+// The scratch array below (HE_NOALLOC_SCRATCH_WORDS uint64 = 4.5 MiB) is held
+// by every GPU that loads the library until the process exits.  All calls
+// share it and it keeps the last call's contents; two calls that overlap on
+// the GPU (different streams or contexts without ordering) race on it.  Every
+// word a call reads was written earlier in the same call, so nothing needs
+// clearing between calls.
+//
+// Host code cannot use the array's name as a device address (in host code
+// the symbol is a stand-in, not device memory), so the first call on each
+// device looks its address up with cudaGetSymbolAddress while that device is
+// current and caches it.  That first call should come before any stream
+// capture begins.
+#include <mutex>
+
+#include "he_internal.h"
+
+namespace he {
+
+__global__ void k_rescale_lift(const uint64_t* __restrict__ last, uint64_t* __restrict__ out, int lm1, uint64_t ql,
+                               const uint64_t* __restrict__ qmod, const DevPrime* __restrict__ pr, int logn);
+__global__ void k_rescale_combine(const uint64_t* __restrict__ in, const uint64_t* __restrict__ lift,
+                                  uint64_t* __restrict__ out, int level, const ulonglong2* __restrict__ qinv,
+                                  const DevPrime* __restrict__ pr, int logn);
+
+static __device__ __align__(256) uint64_t g_noalloc_scratch[HE_NOALLOC_SCRATCH_WORDS];
+
+static std::mutex g_noalloc_mu;
+static uint64_t* g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of the scratch array on c's device (looked up once per device).
+static int noalloc_scratch(he_ctx* c, uint64_t** out) {
+    if (c->device < 0 || c->device >= kMaxDevices)
+        return set_err(c, HE_EINVAL, "he_rescale_noalloc: device %d out of range", c->device);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[c->device]) {
+        int prev = -1;
+        int rc = check_cuda(c, cudaGetDevice(&prev), "he_rescale_noalloc: cudaGetDevice");
+        if (rc) return rc;
+        if (prev != c->device && (rc = check_cuda(c, cudaSetDevice(c->device), "he_rescale_noalloc: cudaSetDevice")))
+            return rc;
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (prev != c->device) cudaSetDevice(prev);
+        if ((rc = check_cuda(c, e, "he_rescale_noalloc: cudaGetSymbolAddress"))) return rc;
+        g_noalloc_ptr[c->device] = (uint64_t*)p;
+    }
+    *out = g_noalloc_ptr[c->device];
+    return HE_OK;
+}
+
+}  // namespace he
+
+using namespace he;
+
+extern "C" int he_rescale_noalloc(he_ctx* c, const he_ct* in, he_ct* out) {
+    if (!c) return HE_EINVAL;
+    if (!in || !in->data || !out || !out->data) return set_err(c, HE_EINVAL, "he_rescale_noalloc: null argument");
+    if (!in->is_ntt) return set_err(c, HE_EDOMAIN, "he_rescale_noalloc: input not in the evaluation domain");
+    const int level = in->level, N = c->N, lm1 = level - 1;
+    if (level < 2 || level > c->L)
+        return set_err(c, HE_ELEVEL, "he_rescale_noalloc: level %d cannot be rescaled", level);
+    const size_t in_words = (size_t)2 * level * N, out_words = (size_t)2 * lm1 * N;
+    const uint64_t *ib = in->data, *ie = in->data + in_words;
+    const uint64_t *ob = out->data, *oe = out->data + out_words;
+    if (ib < oe && ob < ie) return set_err(c, HE_EINVAL, "he_rescale_noalloc: output overlaps the input");
+    // scratch: the last limb [N] and a chunk of lifted limbs [chunk][N]
+    if ((size_t)2 * N > HE_NOALLOC_SCRATCH_WORDS)
+        return set_err(c, HE_EINVAL, "he_rescale_noalloc: N = %d needs %zu scratch words, the maximum is %u", N,
+                       (size_t)2 * N, (unsigned)HE_NOALLOC_SCRATCH_WORDS);
+    if (c->prof_on) return set_err(c, HE_EINVAL, "he_rescale_noalloc: not available while profiling is enabled");
+    uint64_t* scratch;
+    int rc = noalloc_scratch(c, &scratch);
+    if (rc) return rc;
+    const int chunk = (int)(HE_NOALLOC_SCRATCH_WORDS / N) - 1;
+    uint64_t* last = scratch;
+    uint64_t* lift = scratch + N;
+    const uint64_t ql = c->primes[lm1];
+    const int gx = (N + 255) / 256;
+    for (int poly = 0; poly < 2; poly++) {
+        rc = check_cuda(c, cudaMemcpyAsync(last, in->data + ((size_t)poly * level + lm1) * N, (size_t)N * 8,
+                                           cudaMemcpyDeviceToDevice, c->stream), "he_rescale_noalloc: copy");
+        if (rc) return rc;
+        std::vector<int> pl(1, lm1);
+        if ((rc = ntt_inv_set(c, rowset_contig(last, 1, N, pl), 1))) return rc;
+        for (int i0 = 0; i0 < lm1; i0 += chunk) {
+            const int m = lm1 - i0 < chunk ? lm1 - i0 : chunk;
+            k_rescale_lift<<<dim3(gx, m, 1), 256, 0, c->stream>>>(last, lift, lm1, ql,
+                                                                 c->d_rs_qmod + (size_t)lm1 * c->L + i0,
+                                                                 c->d_prime + i0, c->log_n);
+            c->launches++;
+            if ((rc = check_cuda(c, cudaGetLastError(), "he_rescale_noalloc: lift"))) return rc;
+            if ((rc = ntt_fwd_set(c, rowset_contig(lift, m, N, prime_range(i0, m)), m))) return rc;
+            k_rescale_combine<<<dim3(gx, m, 1), 256, 0, c->stream>>>(
+                in->data + ((size_t)poly * level + i0) * N, lift, out->data + ((size_t)poly * lm1 + i0) * N, level,
+                c->d_rs_inv + (size_t)lm1 * c->L + i0, c->d_prime + i0, c->log_n);
+            c->launches++;
+            if ((rc = check_cuda(c, cudaGetLastError(), "he_rescale_noalloc: combine"))) return rc;
+        }
+    }
+    out->level = lm1;
+    out->scale = in->scale / (double)ql;
+    out->is_ntt = 1;
+    return HE_OK;
+}

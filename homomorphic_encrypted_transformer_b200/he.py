@@ -84,6 +84,7 @@ _sig("he_rotate_batch", _i, _vp, ctypes.POINTER(he_ct), _vp, ctypes.POINTER(he_c
 _sig("he_rotate_batch_host", _i, _vp, _vp, _i, _vp, _vp, _i)
 _sig("he_hmult_relin_rescale", _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct), ctypes.POINTER(he_ct))
 _sig("he_rescale", _i, _vp, ctypes.POINTER(he_ct))
+_sig("he_rescale_noalloc", _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct))
 _sig("he_add", _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct), ctypes.POINTER(he_ct))
 _sig("he_mul_const", _i, _vp, ctypes.POINTER(he_ct), ctypes.c_int64, ctypes.POINTER(he_ct))
 _sig("he_add_const", _i, _vp, ctypes.POINTER(he_ct), ctypes.c_int64)
@@ -280,6 +281,13 @@ def he_rescale(ctx, ct):
     c = ct._c()
     _check(ctx, _lib.he_rescale(ctx.ptr, ctypes.byref(c)))
     ct._update(c)
+
+
+def he_rescale_noalloc(ctx, ct_in, ct_out):
+    """Out-of-place rescale that allocates no device memory (see include/he.h)."""
+    ci, co = ct_in._c(), ct_out._c()
+    _check(ctx, _lib.he_rescale_noalloc(ctx.ptr, ctypes.byref(ci), ctypes.byref(co)))
+    ct_out._update(co)
 
 
 def he_add(ctx, a, b, out):

@@ -167,6 +167,24 @@ int he_hmult_relin_rescale(he_ctx* ctx, const he_ct* a, const he_ct* b, he_ct* o
  * [c_{l-1}] the centred coefficient representative.  In place: level-1, scale/q_{l-1}. */
 int he_rescale(he_ctx* ctx, he_ct* inout);
 
+/*
+ * The same rescale as he_rescale, out of place, for callers that must not
+ * allocate device memory while they run (runtimes that reserve and hand out
+ * all device memory themselves, or that cannot afford the device-wide
+ * synchronisation a cudaMalloc/cudaFree may cause).  The pages have no
+ * counterpart: this is a deployment variant, not part of the method.
+ * It calls no cudaMalloc/cudaFree and no allocating routine.  Its scratch is
+ * a fixed device array of HE_NOALLOC_SCRATCH_WORDS uint64 (4.5 MiB) inside
+ * libhe.so, held by every GPU that loads the library until the process exits.
+ * The first call on a device looks that array's address up (do it before any
+ * stream capture starts).  All calls share the array, so calls that overlap
+ * on the GPU race.  N must satisfy 2N <= HE_NOALLOC_SCRATCH_WORDS (always
+ * true for log_n <= 16).  out must not overlap in; it receives level-1 and
+ * scale/q_{level-1}.  Returns HE_EINVAL while profiling is enabled.
+ */
+#define HE_NOALLOC_SCRATCH_WORDS 589824u
+int he_rescale_noalloc(he_ctx* ctx, const he_ct* in, he_ct* out);
+
 /* Helpers: ct + ct (same level; scale of a kept), ct * K (integer, any sign),
  * ct + K (K added to the constant coefficient: every slot gains K/scale),
  * keep limbs q_0..q_{level-1}.  out may equal the input. */
