@@ -32,33 +32,47 @@ __device__ __forceinline__ int automorph_src(int j, int logn, uint64_t k) {
     return (int)(__brev(m2) >> (32 - logn));
 }
 
-// coef[i][r][c] = d_i[r][src(c)] (or a plain copy when galois == 0).
-__global__ void k_gather(PtrList in, uint64_t* __restrict__ out, int level, int logn, uint64_t galois) {
+// sig[i][r][c] = coef[i][r][c] = d_i[r][src(c)] (a plain copy when galois == 0).
+// sig keeps the evaluation-domain values (the digit's own rows of ModUp);
+// coef is transformed back to coefficients in place afterwards.
+__global__ void k_gather(PtrList in, uint64_t* __restrict__ sig, uint64_t* __restrict__ coef, int level, int logn,
+                         uint64_t galois) {
     const int N = 1 << logn;
     int c = blockIdx.x * blockDim.x + threadIdx.x;
     int r = blockIdx.y, i = blockIdx.z;
     if (c >= N) return;
     int src = galois ? automorph_src(c, logn, galois) : c;
-    out[((size_t)i * level + r) * N + c] = in.p[i][(size_t)r * N + src];
+    uint64_t v = in.p[i][(size_t)r * N + src];
+    size_t o = ((size_t)i * level + r) * N + c;
+    sig[o] = v;
+    coef[o] = v;
 }
 
+// ModUp of digit j at one level.  Rows of Q_level and P are numbered
+// t = 0..n_rows-1 (q_0..q_{level-1}, then p_0..p_{K-1}); the digit owns rows
+// src_row..src_row+n_src-1 and its targets are all the other rows, stored
+// compactly: target row t sits at position t (t < src_row) or t - n_src.
+// ext layout: [digit][ciphertext][n_rows - n_src][N].
 struct ModupArgs {
     int n_digits;
     int n_src[kMaxDigits];
     int src_row[kMaxDigits];
+    long long ext_off[kMaxDigits];  // first limb of digit j's block, per ciphertext count 1
     const ulonglong2* src[kMaxDigits];
     const ulonglong2* mat[kMaxDigits];
     uint8_t tprime[64];  // prime index of each of the level+K rows
 };
 
-// ext[i][j][t][c] = sum_s [x_s qhat_inv_s]_{q_s} (qhat_s mod t_prime)  (coefficient domain)
+// ext_j[i][pos(t)][c] = sum_s [x_s qhat_inv_s]_{q_s} (qhat_s mod t_prime)   (coefficient domain)
+// 128-bit accumulation of the alpha products, one reduction per target.
 __global__ void k_modup_conv(const uint64_t* __restrict__ coef, uint64_t* __restrict__ ext, ModupArgs a,
-                             const DevPrime* __restrict__ pr, int level, int n_rows, int logn) {
+                             const DevPrime* __restrict__ pr, int level, int n_rows, int n_cts, int logn) {
     const int N = 1 << logn;
     int c = blockIdx.x * blockDim.x + threadIdx.x;
     int j = blockIdx.y, i = blockIdx.z;
     if (c >= N) return;
     const int ns = a.n_src[j], s0 = a.src_row[j];
+    const int n_tgt = n_rows - ns;
     uint64_t y[16];
     for (int s = 0; s < ns; s++) {
         uint64_t q = pr[s0 + s].q;
@@ -66,23 +80,27 @@ __global__ void k_modup_conv(const uint64_t* __restrict__ coef, uint64_t* __rest
         ulonglong2 w = a.src[j][s];
         y[s] = mul_shoup(x, w.x, w.y, q);
     }
-    uint64_t* o = ext + (((size_t)i * a.n_digits + j) * n_rows) * N + c;
+    uint64_t* o = ext + ((size_t)a.ext_off[j] * n_cts + (size_t)i * n_tgt) * N + c;
     const ulonglong2* m = a.mat[j];
-    for (int t = 0; t < n_rows; t++) {
-        uint64_t q = pr[a.tprime[t]].q;
-        uint64_t acc = 0;
-        for (int s = 0; s < ns; s++) {
-            ulonglong2 w = m[(size_t)s * n_rows + t];
-            acc = csub(acc + mul_shoup_lazy(y[s], w.x, w.y, q), 2 * q);
+    for (int t = 0, pos = 0; t < n_rows; t++) {
+        if (t == s0) {
+            t += ns - 1;
+            continue;
         }
-        o[(size_t)t * N] = csub(acc, q);
+        DevPrime p = pr[a.tprime[t]];
+        U128 acc = {0, 0};
+        for (int s = 0; s < ns; s++) mac128(acc, y[s], m[(size_t)s * n_rows + t].x);
+        o[(size_t)pos * N] = reduce128(acc, p);
+        pos++;
     }
 }
 
-// u[i][0/1][t][c] = sum_j ext[i][j][t][c] * key_j[b/a][row(t)][c]   (key in Montgomery form)
-__global__ void k_ks_inner(const uint64_t* __restrict__ ext, const uint64_t* __restrict__ key, uint64_t* __restrict__ u,
-                           int n_digits, int n_rows, int level, int L, int LK, const DevPrime* __restrict__ pr,
-                           ModupArgs a, int logn) {
+// u[i][0/1][t][c] = sum_j x_j[t][c] * key_j[b/a][row(t)][c]   (key in Montgomery form),
+// x_j = the evaluation-domain input on digit j's own rows, ext_j elsewhere.
+__global__ void k_ks_inner(const uint64_t* __restrict__ ext, const uint64_t* __restrict__ sig,
+                           const uint64_t* __restrict__ key, uint64_t* __restrict__ u, int n_digits, int n_rows,
+                           int level, int L, int LK, int n_cts, const DevPrime* __restrict__ pr, ModupArgs a,
+                           int logn) {
     const int N = 1 << logn;
     int c = blockIdx.x * blockDim.x + threadIdx.x;
     int t = blockIdx.y, i = blockIdx.z;
@@ -91,7 +109,14 @@ __global__ void k_ks_inner(const uint64_t* __restrict__ ext, const uint64_t* __r
     DevPrime p = pr[a.tprime[t]];
     U128 acc0 = {0, 0}, acc1 = {0, 0};
     for (int j = 0; j < n_digits; j++) {
-        uint64_t x = ext[(((size_t)i * n_digits + j) * n_rows + t) * N + c];
+        const int s0 = a.src_row[j], ns = a.n_src[j];
+        uint64_t x;
+        if (t >= s0 && t < s0 + ns) {
+            x = sig[((size_t)i * level + t) * N + c];
+        } else {
+            int pos = t < s0 ? t : t - ns;
+            x = ext[((size_t)a.ext_off[j] * n_cts + (size_t)i * (n_rows - ns) + pos) * N + c];
+        }
         const uint64_t* kb = key + (((size_t)j * 2 + 0) * LK + krow) * N;
         const uint64_t* ka = key + (((size_t)j * 2 + 1) * LK + krow) * N;
         mac128(acc0, x, kb[c]);
@@ -160,11 +185,14 @@ static ModupArgs modup_args(he_ctx* c, int level) {
     ModupArgs a;
     auto& tabs = c->modup[level];
     a.n_digits = (int)tabs.size();
+    long long off = 0;
     for (int j = 0; j < a.n_digits; j++) {
         a.n_src[j] = tabs[j].n_src;
         a.src_row[j] = tabs[j].src_row;
         a.src[j] = tabs[j].d_src;
         a.mat[j] = tabs[j].d_mat;
+        a.ext_off[j] = off;
+        off += level + c->K - tabs[j].n_src;
     }
     std::vector<int> ep = ext_primes(c, level);
     for (size_t t = 0; t < ep.size(); t++) a.tprime[t] = (uint8_t)ep[t];
@@ -176,9 +204,11 @@ static int lc(he_ctx* c, const char* what) {
     return check_cuda(c, cudaGetLastError(), what);
 }
 
+// coef + sig [n][level], ext [n][sum_j (level+K-|D_j|)], u [n][2][level+K], tmp [n][2][level]
 size_t key_switch_scratch_words(const he_ctx* c, int n, int level) {
     size_t nd = (level + c->alpha - 1) / c->alpha, nr = level + c->K;
-    return (size_t)c->N * n * (level + nd * nr + 2 * nr + 2 * level);
+    size_t ext_rows = nd * nr - level;
+    return (size_t)c->N * n * (2 * level + ext_rows + 2 * nr + 2 * level);
 }
 
 int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList& io) {
@@ -189,9 +219,11 @@ int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList
     uint64_t* base;
     int rc = scratch_slot(c, 0, key_switch_scratch_words(c, n, level), &base);
     if (rc) return rc;
+    const int ext_rows = nd * n_rows - level;  // sum over digits of the target rows
     uint64_t* coef = base;
-    uint64_t* ext = coef + (size_t)n * level * N;
-    uint64_t* u = ext + (size_t)n * nd * n_rows * N;
+    uint64_t* sig = coef + (size_t)n * level * N;
+    uint64_t* ext = sig + (size_t)n * level * N;
+    uint64_t* u = ext + (size_t)n * ext_rows * N;
     uint64_t* tmp = u + (size_t)n * 2 * n_rows * N;
 
     PtrList din;
@@ -212,25 +244,35 @@ int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList
     for (int j = 0; j < nd; j++) sum_src += ma.n_src[j];
 
     prof_begin(c, HE_PROF_AUTOMORPH);
-    k_gather<<<dim3(gx, level, n), blk, 0, c->stream>>>(din, coef, level, c->log_n, io.galois);
+    k_gather<<<dim3(gx, level, n), blk, 0, c->stream>>>(din, sig, coef, level, c->log_n, io.galois);
     if ((rc = lc(c, "gather"))) return rc;
-    prof_end(c, HE_PROF_AUTOMORPH, 2.0 * n * level * limbB, 0);
+    prof_end(c, HE_PROF_AUTOMORPH, 3.0 * n * level * limbB, 0);
 
     std::vector<int> qp = prime_range(0, level);
     if ((rc = ntt_inv_set(c, rowset_contig(coef, level, N, qp), n * level))) return rc;
 
     prof_begin(c, HE_PROF_MODUP);
-    k_modup_conv<<<dim3(gx, nd, n), blk, 0, c->stream>>>(coef, ext, ma, c->d_prime, level, n_rows, c->log_n);
+    k_modup_conv<<<dim3(gx, nd, n), blk, 0, c->stream>>>(coef, ext, ma, c->d_prime, level, n_rows, n, c->log_n);
     if ((rc = lc(c, "modup_conv"))) return rc;
-    prof_end(c, HE_PROF_MODUP, (double)n * (sum_src + nd * n_rows) * limbB,
-             (double)n * N * (sum_src + (double)sum_src * n_rows));
+    {
+        double prods = 0;
+        for (int j = 0; j < nd; j++) prods += (double)ma.n_src[j] * (1 + n_rows - ma.n_src[j]);
+        prof_end(c, HE_PROF_MODUP, (double)n * (sum_src + ext_rows) * limbB, (double)n * N * prods);
+    }
 
     std::vector<int> ep = ext_primes(c, level);
-    if ((rc = ntt_fwd_set(c, rowset_contig(ext, n_rows, N, ep), n * nd * n_rows))) return rc;
+    for (int j = 0; j < nd; j++) {
+        std::vector<int> tp;
+        for (int t = 0; t < n_rows; t++)
+            if (t < ma.src_row[j] || t >= ma.src_row[j] + ma.n_src[j]) tp.push_back(ep[t]);
+        const int nt = (int)tp.size();
+        RowSet rs = rowset_contig(ext + (size_t)ma.ext_off[j] * n * N, nt, N, tp);
+        if ((rc = ntt_fwd_set(c, rs, n * nt))) return rc;
+    }
 
     prof_begin(c, HE_PROF_KS_INNER);
-    k_ks_inner<<<dim3(gx, n_rows, n), blk, 0, c->stream>>>(ext, key.d, u, nd, n_rows, level, L, LK, c->d_prime, ma,
-                                                           c->log_n);
+    k_ks_inner<<<dim3(gx, n_rows, n), blk, 0, c->stream>>>(ext, sig, key.d, u, nd, n_rows, level, L, LK, n,
+                                                           c->d_prime, ma, c->log_n);
     if ((rc = lc(c, "ks_inner"))) return rc;
     prof_end(c, HE_PROF_KS_INNER, ((double)n * nd * n_rows + 2.0 * nd * n_rows + 2.0 * n * n_rows) * limbB,
              (double)n * n_rows * N * (2.0 * nd + 2));

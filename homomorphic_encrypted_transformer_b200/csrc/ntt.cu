@@ -1,89 +1,128 @@
-// Batched negacyclic NTT / inverse NTT over RNS limbs (two passes per
-// transform: column pass and row pass, see ntt.cuh).
+// Batched negacyclic NTT / inverse NTT over RNS limbs: a column pass and a
+// row pass per transform, 16 elements per thread (see ntt.cuh).
 #include "he_internal.h"
 #include "kernels.cuh"
 #include "ntt.cuh"
 
 namespace he {
 
-__global__ void k_ntt_fwd_cols(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all,
-                               int logn, int s1, int tc) {
-    extern __shared__ uint64_t smem[];
-    const int N = 1 << logn, R = 1 << s1, C = N >> s1;
-    uint64_t* sm = smem;
-    ulonglong2* tws = reinterpret_cast<ulonglong2*>(smem + R * tc);
+// shared-memory index of element i of a padded row (one pad word per 16)
+__device__ __forceinline__ int padded(int i) { return i + (i >> 4); }
+
+template <int LOGN>
+__global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS)
+    k_ntt_fwd_cols(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all) {
+    using Cf = NttCfg<LOGN>;
+    __shared__ uint64_t sm[Cf::R * Cf::TC];
     const int row = blockIdx.y;
     const int pidx = rs.prime(row);
     const uint64_t q = pr[pidx].q;
-    const ulonglong2* tw = tw_all + (size_t)pidx * N;
-    uint64_t* a = rs.ptr(row, N);
-    const int col0 = blockIdx.x * tc;
-    for (int e = threadIdx.x; e < R; e += blockDim.x) tws[e] = tw[e];
-    for (int e = threadIdx.x; e < R * tc; e += blockDim.x) {
-        int r = e / tc, cc = e - r * tc;
-        sm[e] = a[(size_t)r * C + col0 + cc];
-    }
+    const ulonglong2* tw = tw_all + (size_t)pidx * Cf::N;
+    uint64_t* a = rs.ptr(row, Cf::N) + blockIdx.x * Cf::TC;
+    const int cc = threadIdx.x % Cf::TC, g = threadIdx.x / Cf::TC;
+    constexpr int RS = Cf::R / 16;
+    uint64_t x[16];
+#pragma unroll
+    for (int k = 0; k < 16; k++) x[k] = a[(size_t)(g + RS * k) * Cf::C + cc];
+    fwd_stages<4>(x, tw, 0, 0, 0, q);
+#pragma unroll
+    for (int k = 0; k < 16; k++) sm[(g + RS * k) * Cf::TC + cc] = x[k];
     __syncthreads();
-    tile_fwd_cols(sm, s1, tc, tws, q);
-    for (int e = threadIdx.x; e < R * tc; e += blockDim.x) {
-        int r = e / tc, cc = e - r * tc;
-        a[(size_t)r * C + col0 + cc] = sm[e];
-    }
+#pragma unroll
+    for (int k = 0; k < 16; k++) x[k] = sm[(16 * g + k) * Cf::TC + cc];
+    fwd_stages<Cf::S1 - 4>(x, tw, 4, 0, 16 * g, q);
+#pragma unroll
+    for (int k = 0; k < 16; k++) a[(size_t)(16 * g + k) * Cf::C + cc] = x[k];
 }
 
-__global__ void k_ntt_fwd_rows(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all,
-                               int logn, int s1, int tr) {
-    extern __shared__ uint64_t smem[];
-    const int N = 1 << logn, s2 = logn - s1, C = 1 << s2;
+template <int LOGN>
+__global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS)
+    k_ntt_fwd_rows(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all) {
+    using Cf = NttCfg<LOGN>;
+    __shared__ uint64_t sm[Cf::TR * Cf::ROW_PITCH];
     const int row = blockIdx.y;
     const int pidx = rs.prime(row);
     const uint64_t q = pr[pidx].q;
-    const ulonglong2* tw = tw_all + (size_t)pidx * N;
-    uint64_t* a = rs.ptr(row, N) + (size_t)blockIdx.x * tr * C;
-    for (int e = threadIdx.x; e < tr * C; e += blockDim.x) smem[e] = a[e];
+    const ulonglong2* tw = tw_all + (size_t)pidx * Cf::N;
+    constexpr int CS = Cf::C / 16;
+    const int p = threadIdx.x % CS, rr = threadIdx.x / CS;
+    const int r = blockIdx.x * Cf::TR + rr;
+    uint64_t* a = rs.ptr(row, Cf::N) + (size_t)r * Cf::C;
+    uint64_t* s = sm + rr * Cf::ROW_PITCH;
+    uint64_t x[16];
+#pragma unroll
+    for (int k = 0; k < 16; k++) x[k] = a[p + CS * k];
+    fwd_stages<4>(x, tw, Cf::S1, r, 0, q);
+#pragma unroll
+    for (int k = 0; k < 16; k++) s[padded(p + CS * k)] = x[k];
     __syncthreads();
-    tile_fwd_rows(smem, s1, s2, tr, blockIdx.x * tr, tw, q);
-    for (int e = threadIdx.x; e < tr * C; e += blockDim.x) a[e] = reduce4q(smem[e], q);
+#pragma unroll
+    for (int k = 0; k < 16; k++) x[k] = s[padded(16 * p + k)];
+    fwd_stages<Cf::S2 - 4>(x, tw, Cf::S1 + 4, r << 4, 16 * p, q);
+    ulonglong2* o = reinterpret_cast<ulonglong2*>(a + 16 * p);
+#pragma unroll
+    for (int k = 0; k < 8; k++) o[k] = make_ulonglong2(reduce4q(x[2 * k], q), reduce4q(x[2 * k + 1], q));
 }
 
-__global__ void k_ntt_inv_rows(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all,
-                               int logn, int s1, int tr) {
-    extern __shared__ uint64_t smem[];
-    const int N = 1 << logn, s2 = logn - s1, C = 1 << s2;
+template <int LOGN>
+__global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS)
+    k_ntt_inv_rows(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all) {
+    using Cf = NttCfg<LOGN>;
+    __shared__ uint64_t sm[Cf::TR * Cf::ROW_PITCH];
     const int row = blockIdx.y;
     const int pidx = rs.prime(row);
     const uint64_t q = pr[pidx].q;
-    const ulonglong2* tw = tw_all + (size_t)pidx * N;
-    uint64_t* a = rs.ptr(row, N) + (size_t)blockIdx.x * tr * C;
-    for (int e = threadIdx.x; e < tr * C; e += blockDim.x) smem[e] = a[e];
+    const ulonglong2* tw = tw_all + (size_t)pidx * Cf::N;
+    constexpr int CS = Cf::C / 16;
+    const int p = threadIdx.x % CS, rr = threadIdx.x / CS;
+    const int r = blockIdx.x * Cf::TR + rr;
+    uint64_t* a = rs.ptr(row, Cf::N) + (size_t)r * Cf::C;
+    uint64_t* s = sm + rr * Cf::ROW_PITCH;
+    uint64_t x[16];
+    const ulonglong2* in = reinterpret_cast<const ulonglong2*>(a + 16 * p);
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+        ulonglong2 v = in[k];
+        x[2 * k] = v.x;
+        x[2 * k + 1] = v.y;
+    }
+    inv_stages<Cf::S2 - 4>(x, tw, Cf::S1 + 4, r << 4, 16 * p, q);
+#pragma unroll
+    for (int k = 0; k < 16; k++) s[padded(16 * p + k)] = x[k];
     __syncthreads();
-    tile_inv_rows(smem, logn, s2, tr, blockIdx.x * tr, tw, q);
-    for (int e = threadIdx.x; e < tr * C; e += blockDim.x) a[e] = smem[e];
+#pragma unroll
+    for (int k = 0; k < 16; k++) x[k] = s[padded(p + CS * k)];
+    inv_stages<4>(x, tw, Cf::S1, r, 0, q);
+#pragma unroll
+    for (int k = 0; k < 16; k++) a[p + CS * k] = x[k];
 }
 
-__global__ void k_ntt_inv_cols(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all,
-                               const ulonglong2* __restrict__ ninv_all, int logn, int s1, int tc) {
-    extern __shared__ uint64_t smem[];
-    const int N = 1 << logn, R = 1 << s1, s2 = logn - s1, C = N >> s1;
-    uint64_t* sm = smem;
-    ulonglong2* tws = reinterpret_cast<ulonglong2*>(smem + R * tc);
+template <int LOGN>
+__global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS)
+    k_ntt_inv_cols(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all,
+                   const ulonglong2* __restrict__ ninv_all) {
+    using Cf = NttCfg<LOGN>;
+    __shared__ uint64_t sm[Cf::R * Cf::TC];
     const int row = blockIdx.y;
     const int pidx = rs.prime(row);
     const uint64_t q = pr[pidx].q;
-    const ulonglong2* tw = tw_all + (size_t)pidx * N;
-    uint64_t* a = rs.ptr(row, N);
-    const int col0 = blockIdx.x * tc;
-    for (int e = threadIdx.x; e < R; e += blockDim.x) tws[e] = tw[e];
-    for (int e = threadIdx.x; e < R * tc; e += blockDim.x) {
-        int r = e / tc, cc = e - r * tc;
-        sm[e] = a[(size_t)r * C + col0 + cc];
-    }
+    const ulonglong2* tw = tw_all + (size_t)pidx * Cf::N;
+    uint64_t* a = rs.ptr(row, Cf::N) + blockIdx.x * Cf::TC;
+    const int cc = threadIdx.x % Cf::TC, g = threadIdx.x / Cf::TC;
+    constexpr int RS = Cf::R / 16;
+    uint64_t x[16];
+#pragma unroll
+    for (int k = 0; k < 16; k++) x[k] = a[(size_t)(16 * g + k) * Cf::C + cc];
+    inv_stages<Cf::S1 - 4>(x, tw, 4, 0, 16 * g, q);
+#pragma unroll
+    for (int k = 0; k < 16; k++) sm[(16 * g + k) * Cf::TC + cc] = x[k];
     __syncthreads();
-    tile_inv_cols(sm, logn, s1, s2, tc, tws, ninv_all[pidx], q);
-    for (int e = threadIdx.x; e < R * tc; e += blockDim.x) {
-        int r = e / tc, cc = e - r * tc;
-        a[(size_t)r * C + col0 + cc] = sm[e];
-    }
+#pragma unroll
+    for (int k = 0; k < 16; k++) x[k] = sm[(g + RS * k) * Cf::TC + cc];
+    inv_stages<4, 1>(x, tw, 0, 0, 0, q);
+    inv_stage0_scaled(x, ldtw(tw + 1), ninv_all[pidx], q);
+#pragma unroll
+    for (int k = 0; k < 16; k++) a[(size_t)(g + RS * k) * Cf::C + cc] = x[k];
 }
 
 NttShape ntt_shape(int logn) {
@@ -92,28 +131,71 @@ NttShape ntt_shape(int logn) {
     s.s2 = logn - s.s1;
     int R = 1 << s.s1, C = 1 << s.s2;
     s.tc = C < 16 ? C : 16;
-    s.tr = R * s.tc / C;
+    s.tr = (4096 / C) < R ? (4096 / C) : R;
     s.col_tiles = C / s.tc;
     s.row_tiles = R / s.tr;
-    s.smem_cols = (size_t)R * s.tc * 8 + (size_t)R * 16;
-    s.smem_rows = (size_t)s.tr * C * 8;
+    s.smem_cols = (size_t)R * s.tc * 8;
+    s.smem_rows = (size_t)s.tr * (C + C / 16) * 8;
     return s;
 }
 
 static int launch_check(he_ctx* c, const char* what) { return check_cuda(c, cudaGetLastError(), what); }
 
+template <int LOGN>
+static void launch_fwd(he_ctx* c, const RowSet& rs, int n_rows, int which) {
+    using Cf = NttCfg<LOGN>;
+    if (which == 0)
+        k_ntt_fwd_cols<LOGN><<<dim3(Cf::COL_TILES, n_rows), Cf::COL_THREADS, 0, c->stream>>>(rs, c->d_prime,
+                                                                                            c->d_tw_fwd);
+    else
+        k_ntt_fwd_rows<LOGN><<<dim3(Cf::ROW_TILES, n_rows), Cf::ROW_THREADS, 0, c->stream>>>(rs, c->d_prime,
+                                                                                            c->d_tw_fwd);
+}
+
+template <int LOGN>
+static void launch_inv(he_ctx* c, const RowSet& rs, int n_rows, int which) {
+    using Cf = NttCfg<LOGN>;
+    if (which == 0)
+        k_ntt_inv_rows<LOGN><<<dim3(Cf::ROW_TILES, n_rows), Cf::ROW_THREADS, 0, c->stream>>>(rs, c->d_prime,
+                                                                                            c->d_tw_inv);
+    else
+        k_ntt_inv_cols<LOGN><<<dim3(Cf::COL_TILES, n_rows), Cf::COL_THREADS, 0, c->stream>>>(
+            rs, c->d_prime, c->d_tw_inv, c->d_inv_last);
+}
+
+static void dispatch(he_ctx* c, const RowSet& rs, int n_rows, bool fwd, int which) {
+    switch (c->log_n) {
+#define HE_NTT_CASE(LN)                                \
+    case LN:                                           \
+        if (fwd)                                       \
+            launch_fwd<LN>(c, rs, n_rows, which);      \
+        else                                           \
+            launch_inv<LN>(c, rs, n_rows, which);      \
+        break;
+        HE_NTT_CASE(10)
+        HE_NTT_CASE(11)
+        HE_NTT_CASE(12)
+        HE_NTT_CASE(13)
+        HE_NTT_CASE(14)
+        HE_NTT_CASE(15)
+        HE_NTT_CASE(16)
+#undef HE_NTT_CASE
+        default:
+            break;
+    }
+}
+
 int ntt_fwd_set(he_ctx* c, const RowSet& rs, int n_rows) {
     if (n_rows <= 0) return HE_OK;
     NttShape sh = ntt_shape(c->log_n);
-    dim3 g1(sh.col_tiles, n_rows), g2(sh.row_tiles, n_rows);
     const double bytes = 16.0 * c->N * n_rows, half = 0.5 * c->N * n_rows;
     prof_begin(c, HE_PROF_NTT_FWD_COLS);
-    k_ntt_fwd_cols<<<g1, 256, sh.smem_cols, c->stream>>>(rs, c->d_prime, c->d_tw_fwd, c->log_n, sh.s1, sh.tc);
+    dispatch(c, rs, n_rows, true, 0);
     int rc = launch_check(c, "ntt_fwd_cols");
     if (rc) return rc;
     prof_end(c, HE_PROF_NTT_FWD_COLS, bytes, half * sh.s1);
     prof_begin(c, HE_PROF_NTT_FWD_ROWS);
-    k_ntt_fwd_rows<<<g2, 256, sh.smem_rows, c->stream>>>(rs, c->d_prime, c->d_tw_fwd, c->log_n, sh.s1, sh.tr);
+    dispatch(c, rs, n_rows, true, 1);
     rc = launch_check(c, "ntt_fwd_rows");
     if (rc) return rc;
     c->launches += 2;
@@ -123,16 +205,14 @@ int ntt_fwd_set(he_ctx* c, const RowSet& rs, int n_rows) {
 int ntt_inv_set(he_ctx* c, const RowSet& rs, int n_rows) {
     if (n_rows <= 0) return HE_OK;
     NttShape sh = ntt_shape(c->log_n);
-    dim3 g1(sh.col_tiles, n_rows), g2(sh.row_tiles, n_rows);
     const double bytes = 16.0 * c->N * n_rows, half = 0.5 * c->N * n_rows;
     prof_begin(c, HE_PROF_NTT_INV_ROWS);
-    k_ntt_inv_rows<<<g2, 256, sh.smem_rows, c->stream>>>(rs, c->d_prime, c->d_tw_inv, c->log_n, sh.s1, sh.tr);
+    dispatch(c, rs, n_rows, false, 0);
     int rc = launch_check(c, "ntt_inv_rows");
     if (rc) return rc;
     prof_end(c, HE_PROF_NTT_INV_ROWS, bytes, half * sh.s2);
     prof_begin(c, HE_PROF_NTT_INV_COLS);
-    k_ntt_inv_cols<<<g1, 256, sh.smem_cols, c->stream>>>(rs, c->d_prime, c->d_tw_inv, c->d_inv_last, c->log_n, sh.s1,
-                                                          sh.tc);
+    dispatch(c, rs, n_rows, false, 1);
     rc = launch_check(c, "ntt_inv_cols");
     if (rc) return rc;
     c->launches += 2;
@@ -140,17 +220,7 @@ int ntt_inv_set(he_ctx* c, const RowSet& rs, int n_rows) {
 }
 
 int ntt_setup(he_ctx* c) {
-    NttShape sh = ntt_shape(c->log_n);
-    size_t m = sh.smem_cols > sh.smem_rows ? sh.smem_cols : sh.smem_rows;
-    if (m > 48 * 1024) {
-        const void* fns[] = {(const void*)k_ntt_fwd_cols, (const void*)k_ntt_fwd_rows, (const void*)k_ntt_inv_rows,
-                             (const void*)k_ntt_inv_cols};
-        for (const void* f : fns) {
-            int rc = check_cuda(c, cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)m),
-                                "ntt smem attribute");
-            if (rc) return rc;
-        }
-    }
+    (void)c;
     return HE_OK;
 }
 
@@ -160,7 +230,8 @@ using namespace he;
 
 extern "C" int he_ntt_fwd(he_ctx* c, uint64_t* d, int n_polys, int n_limbs, int first_prime) {
     if (!c) return HE_EINVAL;
-    if (!d || n_polys < 0 || n_limbs < 0 || first_prime < 0 || first_prime + n_limbs > c->L + c->K)
+    if (!d || n_polys < 0 || n_limbs < 0 || first_prime < 0 || first_prime + n_limbs > c->L + c->K ||
+        ((uintptr_t)d & 15))
         return set_err(c, HE_EINVAL, "he_ntt_fwd: bad arguments");
     RowSet rs = rowset_contig(d, n_limbs, c->N, prime_range(first_prime, n_limbs));
     return ntt_fwd_set(c, rs, n_polys * n_limbs);
@@ -168,7 +239,8 @@ extern "C" int he_ntt_fwd(he_ctx* c, uint64_t* d, int n_polys, int n_limbs, int 
 
 extern "C" int he_ntt_inv(he_ctx* c, uint64_t* d, int n_polys, int n_limbs, int first_prime) {
     if (!c) return HE_EINVAL;
-    if (!d || n_polys < 0 || n_limbs < 0 || first_prime < 0 || first_prime + n_limbs > c->L + c->K)
+    if (!d || n_polys < 0 || n_limbs < 0 || first_prime < 0 || first_prime + n_limbs > c->L + c->K ||
+        ((uintptr_t)d & 15))
         return set_err(c, HE_EINVAL, "he_ntt_inv: bad arguments");
     RowSet rs = rowset_contig(d, n_limbs, c->N, prime_range(first_prime, n_limbs));
     return ntt_inv_set(c, rs, n_polys * n_limbs);

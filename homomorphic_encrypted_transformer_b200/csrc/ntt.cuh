@@ -1,121 +1,124 @@
-// Negacyclic NTT building blocks on shared-memory tiles.
+// Negacyclic NTT building blocks: 16 elements per thread in registers.
 //
 // Transform (textbook negacyclic NTT, bit-reversed output): storage index j
 // of the output holds a(psi^(2 brev(j) + 1)).  Computed by the Cooley-Tukey
 // decimation-in-time network with twiddles psi^brev(m+i) (Longa-Naehrig,
 // "Speeding up the Number Theoretic Transform for Faster Ideal Lattice-Based
-// Cryptography", CANS 2016, algorithms 1 and 2), with Harvey's lazy
-// butterflies.  The inverse is the Gentleman-Sande network with psi^-brev(m+i)
+// Cryptography", CANS 2016, algorithms 1 and 2) with Harvey's lazy
+// butterflies; the inverse is the Gentleman-Sande network with psi^-brev(m+i)
 // and N^-1 folded into its last stage.
 //
-// N = R * C with R = 2^s1 rows and C = 2^s2 columns (index j = r C + c).
-// Forward: stages 0..s1-1 pair rows (one column at a time: "column pass"),
-// stages s1..logN-1 pair elements inside a row ("row pass").  Inverse: the
-// row stages run first, then the column stages.
+// N = R C, R = 2^S1 rows, C = 2^S2 columns, element j = r C + c.  Forward
+// stages 0..S1-1 pair rows ("column pass"), stages S1..LOGN-1 pair elements
+// of one row ("row pass"); the inverse runs the row stages first.  Each pass
+// is two register sub-passes of up to four stages separated by one exchange
+// through shared memory:
+//   column pass, sub-pass A: thread (g, col) holds rows g + (R/16) k, k < 16;
+//                sub-pass B: rows 16 g + k;
+//   row pass,    sub-pass A: thread (row, p) holds columns p + (C/16) k;
+//                sub-pass B: columns 16 p + k.
+// In every sub-pass the stage with pair distance D (in those index units)
+// pairs registers k and k + D, and the twiddle index is 2^s plus the pair's
+// block number, which the formulas below derive from k and the thread's
+// (g, row, p) without division.
 #pragma once
 #include "modarith.cuh"
 
 namespace he {
 
+template <int LOGN>
+struct NttCfg {
+    static constexpr int S1 = (LOGN + 1) / 2;
+    static constexpr int S2 = LOGN - S1;
+    static constexpr int R = 1 << S1;
+    static constexpr int C = 1 << S2;
+    static constexpr int N = 1 << LOGN;
+    // column pass: TC columns x R rows per block, 16 elements per thread
+    static constexpr int TC = C < 16 ? C : 16;
+    static constexpr int COL_THREADS = R * TC / 16;
+    static constexpr int COL_TILES = C / TC;
+    // row pass: TR rows x C columns per block
+    static constexpr int TR = (4096 / C) < R ? (4096 / C) : R;
+    static constexpr int ROW_THREADS = TR * C / 16;
+    static constexpr int ROW_TILES = R / TR;
+    static constexpr int ROW_PITCH = C + C / 16;  // one pad word per 16 (bank spread)
+    static constexpr size_t COL_SMEM = (size_t)R * TC * 8;
+    static constexpr size_t ROW_SMEM = (size_t)TR * ROW_PITCH * 8;
+    static_assert(S1 >= 4 && S1 <= 8 && S2 >= 4 && S2 <= 8, "two sub-passes of at most 4 stages");
+};
+
 // Harvey CT butterfly: x, y in [0, 4q) -> [0, 4q).
-__device__ __forceinline__ void bfly_ct(uint64_t& x, uint64_t& y, const ulonglong2 w, uint64_t q) {
-    uint64_t two_q = 2 * q;
+__device__ __forceinline__ void bfly_ct(uint64_t& x, uint64_t& y, const ulonglong2 w, uint64_t q, uint64_t two_q) {
     uint64_t a = csub(x, two_q);
     uint64_t t = mul_shoup_lazy(y, w.x, w.y, q);
     x = a + t;
-    y = a - t + two_q;
+    y = a + two_q - t;
 }
 
 // Harvey GS butterfly: x, y in [0, 2q) -> [0, 2q).
-__device__ __forceinline__ void bfly_gs(uint64_t& x, uint64_t& y, const ulonglong2 w, uint64_t q) {
-    uint64_t two_q = 2 * q;
+__device__ __forceinline__ void bfly_gs(uint64_t& x, uint64_t& y, const ulonglong2 w, uint64_t q, uint64_t two_q) {
     uint64_t a = x, b = y;
     x = csub(a + b, two_q);
-    y = mul_shoup_lazy(a - b + two_q, w.x, w.y, q);
+    y = mul_shoup_lazy(a + two_q - b, w.x, w.y, q);
 }
 
-// [0, 4q) -> [0, q)
 __device__ __forceinline__ uint64_t reduce4q(uint64_t x, uint64_t q) { return csub(csub(x, 2 * q), q); }
 
-// Column pass of the forward transform on a tile sm[R][tc] (row-major, tc
-// columns of the limb).  Values enter canonical or in [0, 4q) and leave in
-// [0, 4q).  tw_s: the R-1 twiddles psi^brev(1..R-1) staged in shared memory.
-__device__ __forceinline__ void tile_fwd_cols(uint64_t* sm, int s1, int tc, const ulonglong2* tw_s, uint64_t q) {
-    const int R = 1 << s1;
-    for (int s = 0; s < s1; s++) {
-        const int t = R >> (s + 1);
-        for (int b = threadIdx.x; b < (R >> 1) * tc; b += blockDim.x) {
-            int cc = b % tc, p = b / tc;
-            int i = p / t, jr = 2 * i * t + (p - i * t);
-            bfly_ct(sm[jr * tc + cc], sm[(jr + t) * tc + cc], tw_s[(1 << s) + i], q);
+__device__ __forceinline__ ulonglong2 ldtw(const ulonglong2* p) { return __ldg(p); }
+
+// Forward stages on 16 registers.  H stages (H <= 4) with register pair
+// distance 2^(H-1-u) at stage u; the twiddle of the pair starting at k is
+// tw[base(u) + (key(k) >> (H - u))] where key(k) = kofs + k, with
+//   base(u) = (2^(s0+u)) + row_term << u.
+// s0: global index of the first stage; kofs/row_term select the block.
+template <int H>
+__device__ __forceinline__ void fwd_stages(uint64_t (&x)[16], const ulonglong2* __restrict__ tw, int s0, int row_term,
+                                           int kofs, uint64_t q) {
+    const uint64_t two_q = 2 * q;
+#pragma unroll
+    for (int u = 0; u < H; u++) {
+        const int D = 1 << (H - 1 - u);
+        const int base = (1 << (s0 + u)) + (row_term << u);
+#pragma unroll
+        for (int k = 0; k < 16; k++) {
+            if (k & D) continue;
+            ulonglong2 w = ldtw(tw + base + ((kofs + k) >> (H - u)));
+            bfly_ct(x[k], x[k + D], w, q, two_q);
         }
-        __syncthreads();
     }
 }
 
-// Row pass of the forward transform on a tile sm[tr][C] holding rows
-// r0..r0+tr-1.  Leaves values in [0, 4q).  tw: the prime's full twiddle table.
-__device__ __forceinline__ void tile_fwd_rows(uint64_t* sm, int s1, int s2, int tr, int r0, const ulonglong2* tw,
-                                              uint64_t q) {
-    const int C = 1 << s2;
-    for (int s = 0; s < s2; s++) {
-        const int t = C >> (s + 1);
-        const int gs = s1 + s;
-        for (int b = threadIdx.x; b < tr * (C >> 1); b += blockDim.x) {
-            int rr = b >> (s2 - 1), p = b & ((C >> 1) - 1);
-            int i = p / t, jc = 2 * i * t + (p - i * t);
-            ulonglong2 w = tw[(1 << gs) + ((r0 + rr) << s) + i];
-            bfly_ct(sm[rr * C + jc], sm[rr * C + jc + t], w, q);
+// Inverse stages on 16 registers: the forward stages of fwd_stages<H> in
+// reverse order with GS butterflies (same twiddle index formula, inverse
+// table).  Stages u = H-1 down to ULO.
+template <int H, int ULO = 0>
+__device__ __forceinline__ void inv_stages(uint64_t (&x)[16], const ulonglong2* __restrict__ tw, int s0, int row_term,
+                                           int kofs, uint64_t q) {
+    const uint64_t two_q = 2 * q;
+#pragma unroll
+    for (int u = H - 1; u >= ULO; u--) {
+        const int D = 1 << (H - 1 - u);
+        const int base = (1 << (s0 + u)) + (row_term << u);
+#pragma unroll
+        for (int k = 0; k < 16; k++) {
+            if (k & D) continue;
+            ulonglong2 w = ldtw(tw + base + ((kofs + k) >> (H - u)));
+            bfly_gs(x[k], x[k + D], w, q, two_q);
         }
-        __syncthreads();
     }
 }
 
-// Row pass of the inverse transform (stages with t = 1 .. C/2) on sm[tr][C].
-// Values enter in [0, 2q) and leave in [0, 2q).
-__device__ __forceinline__ void tile_inv_rows(uint64_t* sm, int logn, int s2, int tr, int r0, const ulonglong2* tw,
-                                              uint64_t q) {
-    const int C = 1 << s2;
-    for (int u = 0; u < s2; u++) {
-        const int t = 1 << u;
-        const int h = 1 << (logn - 1 - u);  // N / (2t)
-        for (int b = threadIdx.x; b < tr * (C >> 1); b += blockDim.x) {
-            int rr = b >> (s2 - 1), p = b & ((C >> 1) - 1);
-            int i = p >> u, jc = 2 * i * t + (p & (t - 1));
-            int gi = ((r0 + rr) << (s2 - 1 - u)) + i;
-            bfly_gs(sm[rr * C + jc], sm[rr * C + jc + t], tw[h + gi], q);
-        }
-        __syncthreads();
-    }
-}
-
-// Column pass of the inverse transform (stages t = C .. N/2) on sm[R][tc],
-// including N^-1: the last stage multiplies the sum by N^-1 (ninv) and the
-// difference by psi^-brev(1) N^-1 (stored in the table at index 1).
-// Values enter in [0, 2q) and leave canonical.
-__device__ __forceinline__ void tile_inv_cols(uint64_t* sm, int logn, int s1, int s2, int tc, const ulonglong2* tw,
-                                              ulonglong2 ninv, uint64_t q) {
-    const int R = 1 << s1;
-    for (int u = 0; u < s1; u++) {
-        const int tr = 1 << u;                  // distance in rows
-        const int h = 1 << (logn - 1 - s2 - u);  // N / (2t), t = tr C
-        const bool last = (u == s1 - 1);
-        for (int b = threadIdx.x; b < (R >> 1) * tc; b += blockDim.x) {
-            int cc = b % tc, p = b / tc;
-            int i = p >> u, jr = 2 * i * tr + (p & (tr - 1));
-            uint64_t& x = sm[jr * tc + cc];
-            uint64_t& y = sm[(jr + tr) * tc + cc];
-            if (!last) {
-                bfly_gs(x, y, tw[h + i], q);
-            } else {
-                uint64_t two_q = 2 * q;
-                uint64_t a = x, bb = y;
-                ulonglong2 w = tw[1];
-                x = mul_shoup(a + bb, ninv.x, ninv.y, q);
-                y = mul_shoup(a - bb + two_q, w.x, w.y, q);
-            }
-        }
-        __syncthreads();
+// Last inverse stage (global stage 0, pair distance N/2, block 0): the sum is
+// multiplied by N^-1 and the difference by psi^-brev(1) N^-1 (table entry 1).
+// Registers k and k + 8 hold rows g and g + R/2.  Outputs canonical.
+__device__ __forceinline__ void inv_stage0_scaled(uint64_t (&x)[16], const ulonglong2 w1, const ulonglong2 ninv,
+                                                  uint64_t q) {
+    const uint64_t two_q = 2 * q;
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+        uint64_t a = x[k], b = x[k + 8];
+        x[k] = mul_shoup(a + b, ninv.x, ninv.y, q);
+        x[k + 8] = mul_shoup(a + two_q - b, w1.x, w1.y, q);
     }
 }
 

@@ -351,7 +351,7 @@ extern "C" int he_keygen_upload(he_ctx* c, int kind, int32_t step, const int8_t*
     if (rc) return rc;
     int32_t* s32 = (int32_t*)w;
     int32_t* e32 = s32 + N;
-    uint64_t* s_ntt = w + (size_t)N / 2 + (size_t)nd * N / 2 + 1;
+    uint64_t* s_ntt = w + (size_t)N / 2 + (size_t)nd * N / 2;  // 16-byte aligned (N >= 1024)
     uint64_t* sp = s_ntt + (size_t)LK * N;
     uint64_t* e_ntt = sp + (size_t)LK * N;
     uint64_t* a_d = e_ntt + (size_t)LK * N;
