@@ -46,8 +46,9 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--case", default="rotation", choices=["rotation", "ntt"],
-                    help="ntt: NTT-only kernel case for profiler captures (no JSON metric line)")
+    ap.add_argument("--case", default="rotation", choices=["rotation", "ntt", "rot_small"],
+                    help="ntt / rot_small: kernel cases for profiler captures (no JSON metric line): "
+                         "NTT of 512 limbs, or 8 rotations with 2 keys")
     return ap.parse_args()
 
 
@@ -187,12 +188,49 @@ def run_ntt_case(args, local_rank):
     n_polys, n_limbs = 16, L + K
     h = S.uniform_residues(S.master_seed(1), "ntt_residues", ctx.primes, ctx.N, lead=(n_polys,))
     d = torch.from_numpy(h.view(np.int64)).cuda()
-    for _ in range(args.warmup + args.steps):
+    for i in range(args.warmup + args.steps):
+        if i == args.warmup:
+            he.he_profile_enable(ctx, True)
         he.he_ntt_fwd(ctx, d, n_polys, n_limbs, 0)
         he.he_ntt_inv(ctx, d, n_polys, n_limbs, 0)
     torch.cuda.synchronize()
     ok = np.array_equal(d.cpu().numpy().view(np.uint64), h)
-    print(json.dumps({"case": "ntt", "rows": n_polys * n_limbs, "roundtrip_ok": bool(ok)}))
+    res = {"case": "ntt", "rows": n_polys * n_limbs, "roundtrip_ok": bool(ok)}
+    for name in ("ntt_fwd_cols", "ntt_fwd_rows", "ntt_inv_rows", "ntt_inv_cols"):
+        ms, n, _, mults = he.he_profile_read(ctx, he.PROF[name])
+        if n:
+            res[name + "_us"] = round(1e3 * ms / n, 2)
+            res[name + "_Gbfly_s"] = round(mults / (ms * 1e-3) / 1e9, 1)
+    print(json.dumps(res))
+
+
+def run_rot_small_case(args, local_rank):
+    """Kernel case for profiler captures: 8 ciphertexts at level 24 rotated
+    with 2 keys (the launch shapes of one key group of the benchmark, ~1 GB)."""
+    import torch
+
+    from homomorphic_encrypted_transformer_b200 import he
+
+    torch.cuda.set_device(local_rank)
+    ctx = he.he_ctx_create(LOG_N, L, K, DNUM, stream=torch.cuda.current_stream())
+    N = ctx.N
+    master = S.master_seed(1)
+    steps, _ = workload_inputs(master, ctx.primes[:L], N_CTS)
+    steps = steps[:2]
+    s = S.secret(master, N)
+    for st in steps:
+        a, e = S.key_draws(master, pow(5, st % (N // 2), 2 * N), ctx.primes, N, DNUM)
+        he.he_keygen_upload(ctx, he.HE_KEY_ROTATION, st, s, a, e)
+    h = S.uniform_residues(master, "ct_residues", ctx.primes[:L], N, lead=(8, 2))
+    x = torch.from_numpy(h.view(np.int64)).cuda()
+    y = torch.empty_like(x)
+    xs = [he.Ciphertext(x[i], LEVEL, 2.0 ** 40) for i in range(8)]
+    ys = [he.Ciphertext(y[i], LEVEL, 2.0 ** 40) for i in range(8)]
+    cs = [steps[i % 2] for i in range(8)]
+    for _ in range(args.warmup + args.steps):
+        he.he_rotate_batch(ctx, xs, cs, ys)
+    torch.cuda.synchronize()
+    print(json.dumps({"case": "rot_small", "rotations": 8 * (args.warmup + args.steps)}))
 
 
 def run_native(args, rank, world, local_rank):
@@ -346,7 +384,8 @@ def run_native(args, rank, world, local_rank):
 # committed captures in profiles/ (a 512-limb launch; the benchmark's launches
 # process 288 limbs on average, so the traffic is scaled by limbs processed).
 # Remove an entry when its kernel changes.
-NCU_TRAFFIC_RATIO = {"ntt_fwd_cols": 540.3 / 536.9, "ntt_fwd_rows": 859.7 / 536.9}
+NCU_TRAFFIC_RATIO = {"ntt_fwd_cols": 489.0 / 536.9, "ntt_fwd_rows": 595.8 / 536.9, "ntt_inv_rows": 625.4 / 536.9,
+                     "ntt_inv_cols": 488.6 / 536.9}
 
 
 def roofline_for(name, prof_entry, int_modmul_s, hbm_peak, pk_kind):
@@ -394,6 +433,8 @@ def main():
             run_reference(args, rank, world)
         elif args.case == "ntt":
             run_ntt_case(args, local_rank)
+        elif args.case == "rot_small":
+            run_rot_small_case(args, local_rank)
         else:
             run_native(args, rank, world, local_rank)
     finally:

@@ -233,8 +233,23 @@ RowSet rowset(uint64_t* base, long long group_stride, int per_group, const int* 
     r.base = base;
     r.group_stride = group_stride;
     r.per_group = per_group;
-    memset(r.prime_idx, 0, sizeof r.prime_idx);
-    for (int i = 0; i < per_group && i < 64; i++) r.prime_idx[i] = (uint8_t)prime_idx[i];
+    // split the list into runs of consecutive primes (at most three are used)
+    int first[3] = {0, 0, 0}, len[3] = {0, 0, 0}, runs = 0;
+    for (int i = 0; i < per_group; i++) {
+        if (runs > 0 && prime_idx[i] == first[runs - 1] + len[runs - 1]) {
+            len[runs - 1]++;
+        } else {
+            if (runs == 3) abort();  // every caller passes at most three runs
+            first[runs] = prime_idx[i];
+            len[runs] = 1;
+            runs++;
+        }
+    }
+    r.first0 = first[0];
+    r.len0 = len[0];
+    r.first1 = first[1];
+    r.len1 = len[1];
+    r.first2 = first[2];
     return r;
 }
 
@@ -312,7 +327,10 @@ static int build_tables(he_ctx* c) {
                     uint64_t t_ = c->primes[r], prod = 1;
                     for (int i2 = s0; i2 < s1; i2++)
                         if (i2 != i) prod = h_mulmod(prod, c->primes[i2] % t_, t_);
-                    blob.push_back(make_ulonglong2(prod, h_shoup(prod, t_)));
+                    // Montgomery form (x 2^64 mod t): the conversion reduces its
+                    // 128-bit sum with one REDC, which divides by 2^64 again
+                    uint64_t mont = h_mulmod(prod, (uint64_t)(((u128)1 << 64) % t_), t_);
+                    blob.push_back(make_ulonglong2(mont, prod));
                 }
             }
             offs.push_back({so, mo});
@@ -343,7 +361,8 @@ static int build_tables(he_ctx* c) {
             uint64_t qi = c->primes[i], pr = 1;
             for (int k2 = 0; k2 < K; k2++)
                 if (k2 != kk) pr = h_mulmod(pr, c->primes[L + k2] % qi, qi);
-            mat[(size_t)kk * L + i] = make_ulonglong2(pr, h_shoup(pr, qi));
+            uint64_t mont = h_mulmod(pr, (uint64_t)(((u128)1 << 64) % qi), qi);  // Montgomery form
+            mat[(size_t)kk * L + i] = make_ulonglong2(mont, pr);
         }
     }
     for (int i = 0; i < L; i++) {

@@ -24,7 +24,7 @@ struct ConvTable {
     int n_src;
     int src_row;            // first row of the digit (its primes are rows src_row..src_row+n_src-1)
     ulonglong2* d_src;      // [n_src] {qhat_inv_i mod q_i, shoup}
-    ulonglong2* d_mat;      // [n_src][level + K] {qhat_i mod t, shoup}
+    ulonglong2* d_mat;      // [n_src][level + K] {(qhat_i mod t) 2^64 mod t, qhat_i mod t}
 };
 
 struct Key {
@@ -61,7 +61,7 @@ struct he_ctx {
 
     std::vector<std::vector<he::ConvTable>> modup;  // [level][digit], level 1..L
     ulonglong2* d_md_pcoef = nullptr;  // [K] {(P/p_k)^-1 mod p_k, shoup}
-    ulonglong2* d_md_mat = nullptr;    // [K][L] {(P/p_k) mod q_i, shoup}
+    ulonglong2* d_md_mat = nullptr;    // [K][L] {(P/p_k) 2^64 mod q_i, (P/p_k) mod q_i}
     uint64_t* d_md_negP = nullptr;     // [L] -P mod q_i (correction of a negative centred term)
     ulonglong2* d_md_pinv = nullptr;   // [L] {P^-1 mod q_i, shoup}
     std::vector<uint64_t> h_Pmod;      // [L+K] P mod prime (0 on the p's)

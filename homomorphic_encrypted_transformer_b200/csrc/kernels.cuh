@@ -7,14 +7,25 @@
 namespace he {
 
 // A batch of limbs: row r lives at base + (r / per_group) * group_stride
-// + (r % per_group) * N and uses prime index prime_idx[r % per_group].
+// + (r % per_group) * N.  Its prime index is that of position rr = r %
+// per_group in a list made of at most three runs of consecutive primes:
+// rr < len0 -> first0 + rr; rr < len0 + len1 -> first1 + rr - len0;
+// otherwise first2 + rr - len0 - len1.  (Q_level then P, or Q_level minus a
+// digit then P, are such lists.)  Plain scalars keep the struct out of local
+// memory when kernels index it.
 struct RowSet {
     uint64_t* base;
     long long group_stride;  // in uint64 words
     int per_group;
-    uint8_t prime_idx[64];
+    int first0, len0, first1, len1, first2;
 
-    __device__ __forceinline__ int prime(int r) const { return prime_idx[r % per_group]; }
+    __device__ __forceinline__ int prime(int r) const {
+        int rr = r % per_group;
+        if (rr < len0) return first0 + rr;
+        rr -= len0;
+        if (rr < len1) return first1 + rr;
+        return first2 + rr - len1;
+    }
     __device__ __forceinline__ uint64_t* ptr(int r, int N) const {
         int g = r / per_group, rr = r - g * per_group;
         return base + (long long)g * group_stride + (long long)rr * N;

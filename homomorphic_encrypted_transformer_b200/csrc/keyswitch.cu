@@ -63,35 +63,61 @@ struct ModupArgs {
     uint8_t tprime[64];  // prime index of each of the level+K rows
 };
 
-// ext_j[i][pos(t)][c] = sum_s [x_s qhat_inv_s]_{q_s} (qhat_s mod t_prime)   (coefficient domain)
-// 128-bit accumulation of the alpha products, one reduction per target.
-__global__ void k_modup_conv(const uint64_t* __restrict__ coef, uint64_t* __restrict__ ext, ModupArgs a,
-                             const DevPrime* __restrict__ pr, int level, int n_rows, int n_cts, int logn) {
+// Target-side constants of one conversion, staged in shared memory.
+struct ConvTarget {
+    uint64_t q, qinv_neg, one_shoup, pad;
+};
+
+// The conversion matrices are stored in Montgomery form (m 2^64 mod t), so a
+// sum of at most 16 products y m' with y < 2^60 stays below t 2^64 and one
+// REDC returns sum(y m) mod t.
+__device__ __forceinline__ uint64_t redc_t(const U128& x, const ConvTarget& p) {
+    return csub(redc_lazy(x.hi, x.lo, p.q, p.qinv_neg), p.q);
+}
+
+constexpr int kConvMaxTargets = 64;
+
+// ModUp of digit j (NS source primes at rows s0..s0+NS-1), one launch per digit:
+//   ext_j[i][pos(t)][c] = sum_s [x_s qhat_inv_s]_{q_s} (qhat_s mod t)   (coefficient domain)
+// for every target row t (all rows of Q_level and P outside the digit).
+// 128-bit accumulation of the NS products, one reduction per target.
+template <int NS>
+__global__ void __launch_bounds__(256)
+    k_modup_conv(const uint64_t* __restrict__ coef, uint64_t* __restrict__ ext_j, const ulonglong2* __restrict__ src,
+                 const ulonglong2* __restrict__ mat, ModupArgs a, const DevPrime* __restrict__ pr, int level,
+                 int n_rows, int s0, int logn) {
+    __shared__ uint64_t sm_m[NS * kConvMaxTargets];
+    __shared__ ConvTarget sm_t[kConvMaxTargets];
     const int N = 1 << logn;
+    const int n_tgt = n_rows - NS;
+    for (int idx = threadIdx.x; idx < NS * n_tgt; idx += blockDim.x) {
+        int s = idx / n_tgt, tt = idx - s * n_tgt;
+        int t = tt < s0 ? tt : tt + NS;
+        sm_m[s * kConvMaxTargets + tt] = mat[(size_t)s * n_rows + t].x;
+    }
+    for (int tt = threadIdx.x; tt < n_tgt; tt += blockDim.x) {
+        int t = tt < s0 ? tt : tt + NS;
+        DevPrime p = pr[a.tprime[t]];
+        sm_t[tt] = ConvTarget{p.q, p.qinv_neg, p.one_shoup, 0};
+    }
+    __syncthreads();
     int c = blockIdx.x * blockDim.x + threadIdx.x;
-    int j = blockIdx.y, i = blockIdx.z;
+    int i = blockIdx.y;
     if (c >= N) return;
-    const int ns = a.n_src[j], s0 = a.src_row[j];
-    const int n_tgt = n_rows - ns;
-    uint64_t y[16];
-    for (int s = 0; s < ns; s++) {
+    uint64_t y[NS];
+#pragma unroll
+    for (int s = 0; s < NS; s++) {
         uint64_t q = pr[s0 + s].q;
         uint64_t x = coef[((size_t)i * level + s0 + s) * N + c];
-        ulonglong2 w = a.src[j][s];
+        ulonglong2 w = src[s];
         y[s] = mul_shoup(x, w.x, w.y, q);
     }
-    uint64_t* o = ext + ((size_t)a.ext_off[j] * n_cts + (size_t)i * n_tgt) * N + c;
-    const ulonglong2* m = a.mat[j];
-    for (int t = 0, pos = 0; t < n_rows; t++) {
-        if (t == s0) {
-            t += ns - 1;
-            continue;
-        }
-        DevPrime p = pr[a.tprime[t]];
+    uint64_t* o = ext_j + (size_t)i * n_tgt * N + c;
+    for (int tt = 0; tt < n_tgt; tt++) {
         U128 acc = {0, 0};
-        for (int s = 0; s < ns; s++) mac128(acc, y[s], m[(size_t)s * n_rows + t].x);
-        o[(size_t)pos * N] = reduce128(acc, p);
-        pos++;
+#pragma unroll
+        for (int s = 0; s < NS; s++) mac128(acc, y[s], sm_m[s * kConvMaxTargets + tt]);
+        o[(size_t)tt * N] = redc_t(acc, sm_t[tt]);
     }
 }
 
@@ -127,35 +153,53 @@ __global__ void k_ks_inner(const uint64_t* __restrict__ ext, const uint64_t* __r
     o[(size_t)(n_rows + t) * N] = csub(redc_lazy(acc1.hi, acc1.lo, p.q, p.qinv_neg), p.q);
 }
 
-// tmp[i][k][r][c] = sum_p y_p (P/p mod q_r) with y_p = [x_p (P/p)^-1]_p taken centred.
-__global__ void k_moddown_conv(const uint64_t* __restrict__ u, uint64_t* __restrict__ tmp, int level, int K, int L,
-                               const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ pcoef,
-                               const ulonglong2* __restrict__ mat, const uint64_t* __restrict__ negP, int logn) {
+// tmp[i][poly][r][c] = sum_k y'_k (P/p_k mod q_r), y_k = [x_k (P/p_k)^-1]_{p_k},
+// y'_k = y_k or y_k - p_k (centred).  Since p_k (P/p_k) = P for every k, the
+// centring subtracts (number of negative terms) * P; the sum of the y_k
+// products is accumulated in 128 bits and reduced once per target.
+template <int KP>
+__global__ void __launch_bounds__(256)
+    k_moddown_conv(const uint64_t* __restrict__ u, uint64_t* __restrict__ tmp, int level, int L,
+                   const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ pcoef,
+                   const ulonglong2* __restrict__ mat, const uint64_t* __restrict__ negP, int logn) {
+    __shared__ uint64_t sm_m[KP * kConvMaxTargets];
+    __shared__ ConvTarget sm_t[kConvMaxTargets];
+    __shared__ uint64_t sm_neg[kConvMaxTargets];
     const int N = 1 << logn;
+    for (int idx = threadIdx.x; idx < KP * level; idx += blockDim.x) {
+        int k = idx / level, r = idx - k * level;
+        sm_m[k * kConvMaxTargets + r] = mat[(size_t)k * L + r].x;
+    }
+    for (int r = threadIdx.x; r < level; r += blockDim.x) {
+        DevPrime p = pr[r];
+        sm_t[r] = ConvTarget{p.q, p.qinv_neg, p.one_shoup, 0};
+        sm_neg[r] = negP[r];
+    }
+    __syncthreads();
     int c = blockIdx.x * blockDim.x + threadIdx.x;
     int poly = blockIdx.y, i = blockIdx.z;  // poly in {0, 1}
     if (c >= N) return;
-    const int n_rows = level + K;
+    const int n_rows = level + KP;
     const uint64_t* x = u + (((size_t)i * 2 + poly) * n_rows + level) * N + c;
-    uint64_t y[16];
-    unsigned neg = 0;
-    for (int k = 0; k < K; k++) {
+    uint64_t y[KP];
+    uint64_t n_neg = 0;
+#pragma unroll
+    for (int k = 0; k < KP; k++) {
         uint64_t p = pr[L + k].q;
         ulonglong2 w = pcoef[k];
         y[k] = mul_shoup(x[(size_t)k * N], w.x, w.y, p);
-        if (y[k] > (p >> 1)) neg |= 1u << k;
+        n_neg += y[k] > (p >> 1) ? 1u : 0u;
     }
     uint64_t* o = tmp + (((size_t)i * 2 + poly) * level) * N + c;
     for (int r = 0; r < level; r++) {
-        uint64_t q = pr[r].q;
-        uint64_t acc = 0;
-        for (int k = 0; k < K; k++) {
-            ulonglong2 w = mat[(size_t)k * L + r];
-            uint64_t term = csub(mul_shoup_lazy(y[k], w.x, w.y, q), q);
-            if (neg >> k & 1u) term += negP[r];  // (y - p) (P/p) = y (P/p) - P
-            acc = csub(acc + term, 2 * q);
-        }
-        o[(size_t)r * N] = csub(acc, q);
+        U128 acc = {0, 0};
+#pragma unroll
+        for (int k = 0; k < KP; k++) mac128(acc, y[k], sm_m[k * kConvMaxTargets + r]);
+        const ConvTarget t = sm_t[r];
+        uint64_t w = n_neg * sm_neg[r];                   // < 16 q <= 2^64
+        uint64_t wr = w - __umul64hi(w, t.one_shoup) * t.q;  // [0, 2q)
+        uint64_t v = redc_t(acc, t) + wr;                    // [0, 3q)
+        o[(size_t)r * N] = csub(csub(v, 2 * t.q), t.q);
     }
 }
 
@@ -252,8 +296,24 @@ int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList
     if ((rc = ntt_inv_set(c, rowset_contig(coef, level, N, qp), n * level))) return rc;
 
     prof_begin(c, HE_PROF_MODUP);
-    k_modup_conv<<<dim3(gx, nd, n), blk, 0, c->stream>>>(coef, ext, ma, c->d_prime, level, n_rows, n, c->log_n);
-    if ((rc = lc(c, "modup_conv"))) return rc;
+    for (int j = 0; j < nd; j++) {
+        uint64_t* ext_j = ext + (size_t)ma.ext_off[j] * n * N;
+        const int s0 = ma.src_row[j];
+        switch (ma.n_src[j]) {
+#define HE_MU_CASE(S)                                                                                       \
+    case S:                                                                                                 \
+        k_modup_conv<S><<<dim3(gx, n), blk, 0, c->stream>>>(coef, ext_j, ma.src[j], ma.mat[j], ma, c->d_prime, \
+                                                            level, n_rows, s0, c->log_n);                   \
+        break;
+            HE_MU_CASE(1) HE_MU_CASE(2) HE_MU_CASE(3) HE_MU_CASE(4) HE_MU_CASE(5) HE_MU_CASE(6) HE_MU_CASE(7)
+            HE_MU_CASE(8) HE_MU_CASE(9) HE_MU_CASE(10) HE_MU_CASE(11) HE_MU_CASE(12) HE_MU_CASE(13)
+            HE_MU_CASE(14) HE_MU_CASE(15) HE_MU_CASE(16)
+#undef HE_MU_CASE
+            default:
+                return set_err(c, HE_EINVAL, "key switch: digit of %d primes unsupported", ma.n_src[j]);
+        }
+        if ((rc = lc(c, "modup_conv"))) return rc;
+    }
     {
         double prods = 0;
         for (int j = 0; j < nd; j++) prods += (double)ma.n_src[j] * (1 + n_rows - ma.n_src[j]);
@@ -282,8 +342,19 @@ int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList
     if ((rc = ntt_inv_set(c, prs, n * 2 * K))) return rc;
 
     prof_begin(c, HE_PROF_MODDOWN_CONV);
-    k_moddown_conv<<<dim3(gx, 2, n), blk, 0, c->stream>>>(u, tmp, level, K, L, c->d_prime, c->d_md_pcoef,
-                                                          c->d_md_mat, c->d_md_negP, c->log_n);
+    switch (K) {
+#define HE_MD_CASE(KK)                                                                                          \
+    case KK:                                                                                                    \
+        k_moddown_conv<KK><<<dim3(gx, 2, n), blk, 0, c->stream>>>(u, tmp, level, L, c->d_prime, c->d_md_pcoef, \
+                                                                  c->d_md_mat, c->d_md_negP, c->log_n);         \
+        break;
+        HE_MD_CASE(1) HE_MD_CASE(2) HE_MD_CASE(3) HE_MD_CASE(4) HE_MD_CASE(5) HE_MD_CASE(6) HE_MD_CASE(7)
+        HE_MD_CASE(8) HE_MD_CASE(9) HE_MD_CASE(10) HE_MD_CASE(11) HE_MD_CASE(12) HE_MD_CASE(13) HE_MD_CASE(14)
+        HE_MD_CASE(15) HE_MD_CASE(16)
+#undef HE_MD_CASE
+        default:
+            return set_err(c, HE_EINVAL, "key switch: K = %d unsupported", K);
+    }
     if ((rc = lc(c, "moddown_conv"))) return rc;
     prof_end(c, HE_PROF_MODDOWN_CONV, 2.0 * n * (K + level) * limbB, 2.0 * n * N * (K + (double)K * level));
 

@@ -4,13 +4,15 @@
 #include "kernels.cuh"
 #include "ntt.cuh"
 
+
+#define NTT_MIN_BLOCKS 3
 namespace he {
 
 // shared-memory index of element i of a padded row (one pad word per 16)
 __device__ __forceinline__ int padded(int i) { return i + (i >> 4); }
 
 template <int LOGN>
-__global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS)
+__global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS, NTT_MIN_BLOCKS)
     k_ntt_fwd_cols(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all) {
     using Cf = NttCfg<LOGN>;
     __shared__ uint64_t sm[Cf::R * Cf::TC];
@@ -36,7 +38,7 @@ __global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS)
 }
 
 template <int LOGN>
-__global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS)
+__global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
     k_ntt_fwd_rows(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all) {
     using Cf = NttCfg<LOGN>;
     __shared__ uint64_t sm[Cf::TR * Cf::ROW_PITCH];
@@ -65,7 +67,7 @@ __global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS)
 }
 
 template <int LOGN>
-__global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS)
+__global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
     k_ntt_inv_rows(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all) {
     using Cf = NttCfg<LOGN>;
     __shared__ uint64_t sm[Cf::TR * Cf::ROW_PITCH];
@@ -98,7 +100,7 @@ __global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS)
 }
 
 template <int LOGN>
-__global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS)
+__global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS, NTT_MIN_BLOCKS)
     k_ntt_inv_cols(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all,
                    const ulonglong2* __restrict__ ninv_all) {
     using Cf = NttCfg<LOGN>;
