@@ -7,6 +7,7 @@
 #include <cstring>
 
 #include "he_internal.h"
+#include "ntt.cuh"
 
 namespace he {
 
@@ -277,6 +278,8 @@ static int build_tables(he_ctx* c) {
     const int N = c->N, LK = c->L + c->K, L = c->L, K = c->K;
     c->hprime.resize(LK);
     std::vector<ulonglong2> tf((size_t)LK * N), ti((size_t)LK * N), il(LK);
+    std::vector<double> tfd((size_t)LK * N), tid((size_t)LK * N);
+    std::vector<FpMod> fpm(LK);
     std::vector<uint64_t> pw(N), pwi(N);
     for (int r = 0; r < LK; r++) {
         uint64_t q = c->primes[r], psi = c->psi[r], psi_i = h_inv(psi, q);
@@ -292,14 +295,20 @@ static int build_tables(he_ctx* c) {
             if (k == 1) wi = h_mulmod(wi, c->hprime[r].n_inv, q);
             tf[(size_t)r * N + k] = make_ulonglong2(w, h_shoup(w, q));
             ti[(size_t)r * N + k] = make_ulonglong2(wi, h_shoup(wi, q));
+            tfd[(size_t)r * N + k] = (double)w;  // exact for the primes the FP64 path serves
+            tid[(size_t)r * N + k] = (double)wi;
         }
         il[r] = make_ulonglong2(c->hprime[r].n_inv, c->hprime[r].n_inv_shoup);
+        fpm[r] = FpMod{(double)q, 2.0 * (double)q, 1.0 / (double)q, (double)c->hprime[r].n_inv};
     }
     int rc;
     if ((rc = upload(c, &c->d_prime, c->hprime, "prime table"))) return rc;
     if ((rc = upload(c, &c->d_tw_fwd, tf, "forward twiddles"))) return rc;
     if ((rc = upload(c, &c->d_tw_inv, ti, "inverse twiddles"))) return rc;
     if ((rc = upload(c, &c->d_inv_last, il, "N^-1 table"))) return rc;
+    if ((rc = upload(c, &c->d_twd_fwd, tfd, "forward twiddles (fp64)"))) return rc;
+    if ((rc = upload(c, &c->d_twd_inv, tid, "inverse twiddles (fp64)"))) return rc;
+    if ((rc = upload(c, &c->d_fpmod, fpm, "fp64 prime constants"))) return rc;
 
     // ModUp conversion tables for every level and digit.
     c->modup.assign(L + 1, {});
@@ -490,6 +499,9 @@ extern "C" int he_ctx_destroy(he_ctx* c) {
     cudaFree(c->d_tw_fwd);
     cudaFree(c->d_tw_inv);
     cudaFree(c->d_inv_last);
+    cudaFree(c->d_twd_fwd);
+    cudaFree(c->d_twd_inv);
+    cudaFree(c->d_fpmod);
     if (c->L >= 1 && (int)c->modup.size() > 1 && !c->modup[1].empty()) cudaFree(c->modup[1][0].d_src);
     cudaFree(c->d_md_pcoef);
     cudaFree(c->d_md_mat);

@@ -27,6 +27,8 @@ struct ConvTable {
     ulonglong2* d_mat;      // [n_src][level + K] {(qhat_i mod t) 2^64 mod t, qhat_i mod t}
 };
 
+struct FpMod;  // FP64 constants of a prime below 2^44 (ntt.cuh)
+
 struct Key {
     uint64_t* d = nullptr;  // [digits][2][L+K][N] in Montgomery form (value * 2^64 mod p)
 };
@@ -52,12 +54,16 @@ struct he_ctx {
     cudaStream_t stream = nullptr;
     std::string err;
     int device = 0;
+    int sm_count = 148;
 
     std::vector<he::DevPrime> hprime;
     he::DevPrime* d_prime = nullptr;   // [L+K]
     ulonglong2* d_tw_fwd = nullptr;    // [L+K][N] {psi^brev(i), shoup}
     ulonglong2* d_tw_inv = nullptr;    // [L+K][N] {psi^-brev(i), shoup}; entry 1 times N^-1
     ulonglong2* d_inv_last = nullptr;  // [L+K] {N^-1, shoup}
+    double* d_twd_fwd = nullptr;       // [L+K][N] forward twiddles as doubles (exact below 2^53)
+    double* d_twd_inv = nullptr;       // [L+K][N] inverse twiddles as doubles; entry 1 times N^-1
+    he::FpMod* d_fpmod = nullptr;      // [L+K] {q, 2q, 1/q, N^-1} as doubles
 
     std::vector<std::vector<he::ConvTable>> modup;  // [level][digit], level 1..L
     ulonglong2* d_md_pcoef = nullptr;  // [K] {(P/p_k)^-1 mod p_k, shoup}

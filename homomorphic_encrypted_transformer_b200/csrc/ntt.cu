@@ -1,5 +1,7 @@
 // Batched negacyclic NTT / inverse NTT over RNS limbs: a column pass and a
-// row pass per transform, 16 elements per thread (see ntt.cuh).
+// row pass per transform, 16 elements per thread (see ntt.cuh).  Limbs of
+// primes below 2^44 run the butterflies on the FP64 pipe, the others on the
+// integer pipe (the branch is uniform per block: one limb per block).
 #include "he_internal.h"
 #include "kernels.cuh"
 #include "ntt.cuh"
@@ -11,120 +13,174 @@ namespace he {
 // shared-memory index of element i of a padded row (one pad word per 16)
 __device__ __forceinline__ int padded(int i) { return i + (i >> 4); }
 
-template <int LOGN>
-__global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS, NTT_MIN_BLOCKS)
-    k_ntt_fwd_cols(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all) {
+// Element handling of the two arithmetic paths: 64-bit integers with Shoup
+// twiddles (any prime), or exact doubles on the FP64 pipe (primes < 2^44).
+__device__ __forceinline__ uint64_t to_elem(uint64_t v, uint64_t) { return v; }
+__device__ __forceinline__ double to_elem(uint64_t v, double) { return u2d(v); }
+__device__ __forceinline__ uint64_t from_elem(uint64_t v) { return v; }
+__device__ __forceinline__ uint64_t from_elem(double v) { return d2u(v); }
+
+template <int LOGN, typename T, typename TW, typename M>
+__device__ __forceinline__ void fwd_cols_body(T* sm, uint64_t* a, const TW* tw, const M& m) {
     using Cf = NttCfg<LOGN>;
-    __shared__ uint64_t sm[Cf::R * Cf::TC];
-    const int row = blockIdx.y;
-    const int pidx = rs.prime(row);
-    const uint64_t q = pr[pidx].q;
-    const ulonglong2* tw = tw_all + (size_t)pidx * Cf::N;
-    uint64_t* a = rs.ptr(row, Cf::N) + blockIdx.x * Cf::TC;
     const int cc = threadIdx.x % Cf::TC, g = threadIdx.x / Cf::TC;
     constexpr int RS = Cf::R / 16;
-    uint64_t x[16];
+    T x[16];
 #pragma unroll
-    for (int k = 0; k < 16; k++) x[k] = a[(size_t)(g + RS * k) * Cf::C + cc];
-    fwd_stages<4>(x, tw, 0, 0, 0, q);
+    for (int k = 0; k < 16; k++) x[k] = to_elem(a[(size_t)(g + RS * k) * Cf::C + cc], T());
+    fwd_stages<4>(x, tw, 0, 0, 0, m);
 #pragma unroll
     for (int k = 0; k < 16; k++) sm[(g + RS * k) * Cf::TC + cc] = x[k];
     __syncthreads();
 #pragma unroll
     for (int k = 0; k < 16; k++) x[k] = sm[(16 * g + k) * Cf::TC + cc];
-    fwd_stages<Cf::S1 - 4>(x, tw, 4, 0, 16 * g, q);
+    fwd_stages<Cf::S1 - 4>(x, tw, 4, 0, 16 * g, m);
 #pragma unroll
-    for (int k = 0; k < 16; k++) a[(size_t)(16 * g + k) * Cf::C + cc] = x[k];
+    for (int k = 0; k < 16; k++) a[(size_t)(16 * g + k) * Cf::C + cc] = from_elem(x[k]);
 }
 
-template <int LOGN>
-__global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
-    k_ntt_fwd_rows(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all) {
+template <int LOGN, typename T, typename TW, typename M>
+__device__ __forceinline__ void fwd_rows_body(T* sm, uint64_t* a, int r, const TW* tw, const M& m) {
     using Cf = NttCfg<LOGN>;
-    __shared__ uint64_t sm[Cf::TR * Cf::ROW_PITCH];
-    const int row = blockIdx.y;
-    const int pidx = rs.prime(row);
-    const uint64_t q = pr[pidx].q;
-    const ulonglong2* tw = tw_all + (size_t)pidx * Cf::N;
     constexpr int CS = Cf::C / 16;
     const int p = threadIdx.x % CS, rr = threadIdx.x / CS;
-    const int r = blockIdx.x * Cf::TR + rr;
-    uint64_t* a = rs.ptr(row, Cf::N) + (size_t)r * Cf::C;
-    uint64_t* s = sm + rr * Cf::ROW_PITCH;
-    uint64_t x[16];
+    T* s = sm + rr * Cf::ROW_PITCH;
+    T x[16];
 #pragma unroll
-    for (int k = 0; k < 16; k++) x[k] = a[p + CS * k];
-    fwd_stages<4>(x, tw, Cf::S1, r, 0, q);
+    for (int k = 0; k < 16; k++) x[k] = to_elem(a[p + CS * k], T());
+    fwd_stages<4>(x, tw, Cf::S1, r, 0, m);
 #pragma unroll
     for (int k = 0; k < 16; k++) s[padded(p + CS * k)] = x[k];
     __syncthreads();
 #pragma unroll
     for (int k = 0; k < 16; k++) x[k] = s[padded(16 * p + k)];
-    fwd_stages<Cf::S2 - 4>(x, tw, Cf::S1 + 4, r << 4, 16 * p, q);
+    fwd_stages<Cf::S2 - 4>(x, tw, Cf::S1 + 4, r << 4, 16 * p, m);
     ulonglong2* o = reinterpret_cast<ulonglong2*>(a + 16 * p);
 #pragma unroll
-    for (int k = 0; k < 8; k++) o[k] = make_ulonglong2(reduce4q(x[2 * k], q), reduce4q(x[2 * k + 1], q));
+    for (int k = 0; k < 8; k++)
+        o[k] = make_ulonglong2(from_elem(reduce4q(x[2 * k], m)), from_elem(reduce4q(x[2 * k + 1], m)));
 }
 
-template <int LOGN>
-__global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
-    k_ntt_inv_rows(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all) {
+template <int LOGN, typename T, typename TW, typename M>
+__device__ __forceinline__ void inv_rows_body(T* sm, uint64_t* a, int r, const TW* tw, const M& m) {
     using Cf = NttCfg<LOGN>;
-    __shared__ uint64_t sm[Cf::TR * Cf::ROW_PITCH];
-    const int row = blockIdx.y;
-    const int pidx = rs.prime(row);
-    const uint64_t q = pr[pidx].q;
-    const ulonglong2* tw = tw_all + (size_t)pidx * Cf::N;
     constexpr int CS = Cf::C / 16;
     const int p = threadIdx.x % CS, rr = threadIdx.x / CS;
-    const int r = blockIdx.x * Cf::TR + rr;
-    uint64_t* a = rs.ptr(row, Cf::N) + (size_t)r * Cf::C;
-    uint64_t* s = sm + rr * Cf::ROW_PITCH;
-    uint64_t x[16];
+    T* s = sm + rr * Cf::ROW_PITCH;
+    T x[16];
     const ulonglong2* in = reinterpret_cast<const ulonglong2*>(a + 16 * p);
 #pragma unroll
     for (int k = 0; k < 8; k++) {
         ulonglong2 v = in[k];
-        x[2 * k] = v.x;
-        x[2 * k + 1] = v.y;
+        x[2 * k] = to_elem(v.x, T());
+        x[2 * k + 1] = to_elem(v.y, T());
     }
-    inv_stages<Cf::S2 - 4>(x, tw, Cf::S1 + 4, r << 4, 16 * p, q);
+    inv_stages<Cf::S2 - 4>(x, tw, Cf::S1 + 4, r << 4, 16 * p, m);
 #pragma unroll
     for (int k = 0; k < 16; k++) s[padded(16 * p + k)] = x[k];
     __syncthreads();
 #pragma unroll
     for (int k = 0; k < 16; k++) x[k] = s[padded(p + CS * k)];
-    inv_stages<4>(x, tw, Cf::S1, r, 0, q);
+    inv_stages<4>(x, tw, Cf::S1, r, 0, m);
 #pragma unroll
-    for (int k = 0; k < 16; k++) a[p + CS * k] = x[k];
+    for (int k = 0; k < 16; k++) a[p + CS * k] = from_elem(x[k]);
 }
 
 template <int LOGN>
 __global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS, NTT_MIN_BLOCKS)
-    k_ntt_inv_cols(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all,
-                   const ulonglong2* __restrict__ ninv_all) {
+    k_ntt_fwd_cols(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all,
+                   const double* __restrict__ twd_all, const FpMod* __restrict__ fpm) {
     using Cf = NttCfg<LOGN>;
     __shared__ uint64_t sm[Cf::R * Cf::TC];
     const int row = blockIdx.y;
     const int pidx = rs.prime(row);
     const uint64_t q = pr[pidx].q;
-    const ulonglong2* tw = tw_all + (size_t)pidx * Cf::N;
     uint64_t* a = rs.ptr(row, Cf::N) + blockIdx.x * Cf::TC;
+    if (q < kFpPrimeLimit)
+        fwd_cols_body<LOGN>(reinterpret_cast<double*>(sm), a, twd_all + (size_t)pidx * Cf::N, fpm[pidx]);
+    else
+        fwd_cols_body<LOGN>(sm, a, tw_all + (size_t)pidx * Cf::N, q);
+}
+
+template <int LOGN>
+__global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
+    k_ntt_fwd_rows(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all,
+                   const double* __restrict__ twd_all, const FpMod* __restrict__ fpm) {
+    using Cf = NttCfg<LOGN>;
+    __shared__ uint64_t sm[Cf::TR * Cf::ROW_PITCH];
+    const int row = blockIdx.y;
+    const int pidx = rs.prime(row);
+    const uint64_t q = pr[pidx].q;
+    const int r = blockIdx.x * Cf::TR + threadIdx.x / (Cf::C / 16);
+    uint64_t* a = rs.ptr(row, Cf::N) + (size_t)r * Cf::C;
+    if (q < kFpPrimeLimit)
+        fwd_rows_body<LOGN>(reinterpret_cast<double*>(sm), a, r, twd_all + (size_t)pidx * Cf::N, fpm[pidx]);
+    else
+        fwd_rows_body<LOGN>(sm, a, r, tw_all + (size_t)pidx * Cf::N, q);
+}
+
+template <int LOGN>
+__global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
+    k_ntt_inv_rows(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all,
+                   const double* __restrict__ twd_all, const FpMod* __restrict__ fpm) {
+    using Cf = NttCfg<LOGN>;
+    __shared__ uint64_t sm[Cf::TR * Cf::ROW_PITCH];
+    const int row = blockIdx.y;
+    const int pidx = rs.prime(row);
+    const uint64_t q = pr[pidx].q;
+    const int r = blockIdx.x * Cf::TR + threadIdx.x / (Cf::C / 16);
+    uint64_t* a = rs.ptr(row, Cf::N) + (size_t)r * Cf::C;
+    if (q < kFpPrimeLimit)
+        inv_rows_body<LOGN>(reinterpret_cast<double*>(sm), a, r, twd_all + (size_t)pidx * Cf::N, fpm[pidx]);
+    else
+        inv_rows_body<LOGN>(sm, a, r, tw_all + (size_t)pidx * Cf::N, q);
+}
+
+__device__ __forceinline__ void inv_stage0(uint64_t (&x)[16], ulonglong2 w1, ulonglong2 ninv, uint64_t q) {
+    inv_stage0_scaled(x, w1, ninv, q);
+}
+__device__ __forceinline__ void inv_stage0(double (&x)[16], double w1, int, const FpMod& m) {
+    inv_stage0_scaled(x, w1, m);
+}
+
+template <int LOGN, typename T, typename TW, typename M, typename W1, typename NI>
+__device__ __forceinline__ void inv_cols_body(T* sm, uint64_t* a, const TW* tw, const M& m, W1 w1, NI ninv) {
+    using Cf = NttCfg<LOGN>;
     const int cc = threadIdx.x % Cf::TC, g = threadIdx.x / Cf::TC;
     constexpr int RS = Cf::R / 16;
-    uint64_t x[16];
+    T x[16];
 #pragma unroll
-    for (int k = 0; k < 16; k++) x[k] = a[(size_t)(16 * g + k) * Cf::C + cc];
-    inv_stages<Cf::S1 - 4>(x, tw, 4, 0, 16 * g, q);
+    for (int k = 0; k < 16; k++) x[k] = to_elem(a[(size_t)(16 * g + k) * Cf::C + cc], T());
+    inv_stages<Cf::S1 - 4>(x, tw, 4, 0, 16 * g, m);
 #pragma unroll
     for (int k = 0; k < 16; k++) sm[(16 * g + k) * Cf::TC + cc] = x[k];
     __syncthreads();
 #pragma unroll
     for (int k = 0; k < 16; k++) x[k] = sm[(g + RS * k) * Cf::TC + cc];
-    inv_stages<4, 1>(x, tw, 0, 0, 0, q);
-    inv_stage0_scaled(x, ldtw(tw + 1), ninv_all[pidx], q);
+    inv_stages<4, 1>(x, tw, 0, 0, 0, m);
+    inv_stage0(x, w1, ninv, m);
 #pragma unroll
-    for (int k = 0; k < 16; k++) a[(size_t)(g + RS * k) * Cf::C + cc] = x[k];
+    for (int k = 0; k < 16; k++) a[(size_t)(g + RS * k) * Cf::C + cc] = from_elem(x[k]);
+}
+
+template <int LOGN>
+__global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS, NTT_MIN_BLOCKS)
+    k_ntt_inv_cols(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all,
+                   const ulonglong2* __restrict__ ninv_all, const double* __restrict__ twd_all,
+                   const FpMod* __restrict__ fpm) {
+    using Cf = NttCfg<LOGN>;
+    __shared__ uint64_t sm[Cf::R * Cf::TC];
+    const int row = blockIdx.y;
+    const int pidx = rs.prime(row);
+    const uint64_t q = pr[pidx].q;
+    uint64_t* a = rs.ptr(row, Cf::N) + blockIdx.x * Cf::TC;
+    if (q < kFpPrimeLimit) {
+        const double* twd = twd_all + (size_t)pidx * Cf::N;
+        inv_cols_body<LOGN>(reinterpret_cast<double*>(sm), a, twd, fpm[pidx], __ldg(twd + 1), 0);
+    } else {
+        const ulonglong2* tw = tw_all + (size_t)pidx * Cf::N;
+        inv_cols_body<LOGN>(sm, a, tw, q, ldtw(tw + 1), ninv_all[pidx]);
+    }
 }
 
 NttShape ntt_shape(int logn) {
@@ -147,22 +203,22 @@ template <int LOGN>
 static void launch_fwd(he_ctx* c, const RowSet& rs, int n_rows, int which) {
     using Cf = NttCfg<LOGN>;
     if (which == 0)
-        k_ntt_fwd_cols<LOGN><<<dim3(Cf::COL_TILES, n_rows), Cf::COL_THREADS, 0, c->stream>>>(rs, c->d_prime,
-                                                                                            c->d_tw_fwd);
+        k_ntt_fwd_cols<LOGN><<<dim3(Cf::COL_TILES, n_rows), Cf::COL_THREADS, 0, c->stream>>>(
+            rs, c->d_prime, c->d_tw_fwd, c->d_twd_fwd, c->d_fpmod);
     else
-        k_ntt_fwd_rows<LOGN><<<dim3(Cf::ROW_TILES, n_rows), Cf::ROW_THREADS, 0, c->stream>>>(rs, c->d_prime,
-                                                                                            c->d_tw_fwd);
+        k_ntt_fwd_rows<LOGN><<<dim3(Cf::ROW_TILES, n_rows), Cf::ROW_THREADS, 0, c->stream>>>(
+            rs, c->d_prime, c->d_tw_fwd, c->d_twd_fwd, c->d_fpmod);
 }
 
 template <int LOGN>
 static void launch_inv(he_ctx* c, const RowSet& rs, int n_rows, int which) {
     using Cf = NttCfg<LOGN>;
     if (which == 0)
-        k_ntt_inv_rows<LOGN><<<dim3(Cf::ROW_TILES, n_rows), Cf::ROW_THREADS, 0, c->stream>>>(rs, c->d_prime,
-                                                                                            c->d_tw_inv);
+        k_ntt_inv_rows<LOGN><<<dim3(Cf::ROW_TILES, n_rows), Cf::ROW_THREADS, 0, c->stream>>>(
+            rs, c->d_prime, c->d_tw_inv, c->d_twd_inv, c->d_fpmod);
     else
         k_ntt_inv_cols<LOGN><<<dim3(Cf::COL_TILES, n_rows), Cf::COL_THREADS, 0, c->stream>>>(
-            rs, c->d_prime, c->d_tw_inv, c->d_inv_last);
+            rs, c->d_prime, c->d_tw_inv, c->d_inv_last, c->d_twd_inv, c->d_fpmod);
 }
 
 static void dispatch(he_ctx* c, const RowSet& rs, int n_rows, bool fwd, int which) {

@@ -108,6 +108,100 @@ __device__ __forceinline__ void inv_stages(uint64_t (&x)[16], const ulonglong2* 
     }
 }
 
+// ---------------------------------------------------------------------------
+// FP64 arithmetic for primes below 2^44 (the 40-bit primes of the modulus
+// chain).  Residues are held as doubles (exact integers below 2^53) and the
+// modular product runs on the FP64 pipe:
+//   p_hi = fl(y w), p_lo = fma(y, w, -p_hi)          (y w = p_hi + p_lo exactly)
+//   qh = round-to-nearest(p_hi / q) via the 1.5 2^52 magic constant
+//   r = fma(-qh, q, p_hi) + p_lo                     (exact: |r| < q/2 + 2^30)
+//   r < 0 ? r + q : r                                (result in [0, q))
+// The remainder is exact because its true value is an integer far below
+// 2^53, which one rounding of the FMA reproduces.  Checked against integer
+// arithmetic on random and boundary inputs (y < 4q, w < q).
+struct FpMod {
+    double q, two_q, qinv, ninv;
+};
+
+constexpr uint64_t kFpPrimeLimit = 1ull << 44;
+
+__device__ __forceinline__ double fp_modmul(double y, double w, const FpMod& m) {
+    const double MAGIC = 6755399441055744.0;  // 1.5 * 2^52
+    double ph = __dmul_rn(y, w);
+    double pl = __fma_rn(y, w, -ph);
+    double qh = __dsub_rn(__fma_rn(ph, m.qinv, MAGIC), MAGIC);
+    double r = __dadd_rn(__fma_rn(-qh, m.q, ph), pl);
+    return r < 0.0 ? __dadd_rn(r, m.q) : r;
+}
+
+__device__ __forceinline__ double fp_csub(double x, double c) { return x >= c ? __dsub_rn(x, c) : x; }
+
+// exact conversions for integers below 2^52
+__device__ __forceinline__ double u2d(uint64_t x) {
+    return __dsub_rn(__longlong_as_double((long long)(x | 0x4330000000000000ull)), 4503599627370496.0);
+}
+__device__ __forceinline__ uint64_t d2u(double d) {
+    return (uint64_t)__double_as_longlong(__dadd_rn(d, 4503599627370496.0)) & 0x000FFFFFFFFFFFFFull;
+}
+
+// CT butterfly, values in [0, 4q) -> [0, 4q)
+__device__ __forceinline__ void bfly_ct(double& x, double& y, double w, const FpMod& m) {
+    double a = fp_csub(x, m.two_q);
+    double t = fp_modmul(y, w, m);
+    x = __dadd_rn(a, t);
+    y = __dadd_rn(a, __dsub_rn(m.two_q, t));
+}
+
+// GS butterfly, values in [0, 2q) -> [0, 2q)
+__device__ __forceinline__ void bfly_gs(double& x, double& y, double w, const FpMod& m) {
+    double a = x, b = y;
+    x = fp_csub(__dadd_rn(a, b), m.two_q);
+    y = fp_modmul(__dsub_rn(__dadd_rn(a, m.two_q), b), w, m);
+}
+
+__device__ __forceinline__ double reduce4q(double x, const FpMod& m) { return fp_csub(fp_csub(x, m.two_q), m.q); }
+
+template <int H>
+__device__ __forceinline__ void fwd_stages(double (&x)[16], const double* __restrict__ tw, int s0, int row_term,
+                                           int kofs, const FpMod& m) {
+#pragma unroll
+    for (int u = 0; u < H; u++) {
+        const int D = 1 << (H - 1 - u);
+        const int base = (1 << (s0 + u)) + (row_term << u);
+#pragma unroll
+        for (int k = 0; k < 16; k++) {
+            if (k & D) continue;
+            double w = __ldg(tw + base + ((kofs + k) >> (H - u)));
+            bfly_ct(x[k], x[k + D], w, m);
+        }
+    }
+}
+
+template <int H, int ULO = 0>
+__device__ __forceinline__ void inv_stages(double (&x)[16], const double* __restrict__ tw, int s0, int row_term,
+                                           int kofs, const FpMod& m) {
+#pragma unroll
+    for (int u = H - 1; u >= ULO; u--) {
+        const int D = 1 << (H - 1 - u);
+        const int base = (1 << (s0 + u)) + (row_term << u);
+#pragma unroll
+        for (int k = 0; k < 16; k++) {
+            if (k & D) continue;
+            double w = __ldg(tw + base + ((kofs + k) >> (H - u)));
+            bfly_gs(x[k], x[k + D], w, m);
+        }
+    }
+}
+
+__device__ __forceinline__ void inv_stage0_scaled(double (&x)[16], double w1, const FpMod& m) {
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+        double a = x[k], b = x[k + 8];
+        x[k] = fp_modmul(__dadd_rn(a, b), m.ninv, m);
+        x[k + 8] = fp_modmul(__dsub_rn(__dadd_rn(a, m.two_q), b), w1, m);
+    }
+}
+
 // Last inverse stage (global stage 0, pair distance N/2, block 0): the sum is
 // multiplied by N^-1 and the difference by psi^-brev(1) N^-1 (table entry 1).
 // Registers k and k + 8 hold rows g and g + R/2.  Outputs canonical.
