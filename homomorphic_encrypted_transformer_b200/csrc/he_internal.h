@@ -116,15 +116,19 @@ int ntt_inv_set(he_ctx* c, const RowSet& rs, int n_rows);
 //   out0 = KS(d)_0 + add0[i],  out1 = KS(d)_1 + add1[i]   (null adds are skipped).
 // With galois != 0 the switched polynomial is sigma_galois(d[i]), and add0 is
 // also read through sigma_galois when sig_add0 is set (rotation).
+// Entry i switches d[i] with key[i]; entries that share a key should be
+// adjacent (the inner product then reads each key tile once from DRAM for
+// all of them).
 struct KsIoList {
-    uint64_t galois = 0;
     bool sig_add0 = false;
+    std::vector<uint64_t> galois;  // 0: no automorphism
+    std::vector<const uint64_t*> key;
     std::vector<const uint64_t*> d;
     std::vector<uint64_t*> out;
     std::vector<const uint64_t*> add0;
     std::vector<const uint64_t*> add1;
 };
-int key_switch(he_ctx* c, int level, const Key& key, const KsIoList& io);
+int key_switch(he_ctx* c, int level, const KsIoList& io);
 size_t key_switch_scratch_words(const he_ctx* c, int n, int level);
 int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, int n);
 

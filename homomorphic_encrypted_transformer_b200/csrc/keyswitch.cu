@@ -13,7 +13,7 @@
 
 namespace he {
 
-constexpr int kMaxBatch = 32;
+constexpr int kMaxBatch = 64;
 constexpr int kMaxDigits = 15;
 
 struct PtrList {
@@ -21,6 +21,9 @@ struct PtrList {
 };
 struct MutPtrList {
     uint64_t* p[kMaxBatch];
+};
+struct GalList {
+    uint64_t g[kMaxBatch];
 };
 
 // Evaluation-domain index whose value sigma_k moves to index j:
@@ -36,11 +39,12 @@ __device__ __forceinline__ int automorph_src(int j, int logn, uint64_t k) {
 // sig keeps the evaluation-domain values (the digit's own rows of ModUp);
 // coef is transformed back to coefficients in place afterwards.
 __global__ void k_gather(PtrList in, uint64_t* __restrict__ sig, uint64_t* __restrict__ coef, int level, int logn,
-                         uint64_t galois) {
+                         GalList gal) {
     const int N = 1 << logn;
     int c = blockIdx.x * blockDim.x + threadIdx.x;
     int r = blockIdx.y, i = blockIdx.z;
     if (c >= N) return;
+    const uint64_t galois = gal.g[i];
     int src = galois ? automorph_src(c, logn, galois) : c;
     uint64_t v = in.p[i][(size_t)r * N + src];
     size_t o = ((size_t)i * level + r) * N + c;
@@ -84,53 +88,77 @@ constexpr int kConvMaxTargets = 64;
 template <int NS>
 __global__ void __launch_bounds__(256)
     k_modup_conv(const uint64_t* __restrict__ coef, uint64_t* __restrict__ ext_j, const ulonglong2* __restrict__ src,
-                 const ulonglong2* __restrict__ mat, ModupArgs a, const DevPrime* __restrict__ pr, int level,
-                 int n_rows, int s0, int logn) {
+                 const ulonglong2* __restrict__ mat, ModupArgs a, const DevPrime* __restrict__ pr,
+                 const FpMod* __restrict__ fpm, int level, int n_rows, int s0, int logn) {
     __shared__ uint64_t sm_m[NS * kConvMaxTargets];
+    __shared__ double sm_md[NS * kConvMaxTargets];
     __shared__ ConvTarget sm_t[kConvMaxTargets];
+    __shared__ FpMod sm_f[kConvMaxTargets];
     const int N = 1 << logn;
     const int n_tgt = n_rows - NS;
     for (int idx = threadIdx.x; idx < NS * n_tgt; idx += blockDim.x) {
         int s = idx / n_tgt, tt = idx - s * n_tgt;
         int t = tt < s0 ? tt : tt + NS;
-        sm_m[s * kConvMaxTargets + tt] = mat[(size_t)s * n_rows + t].x;
+        ulonglong2 m = mat[(size_t)s * n_rows + t];
+        sm_m[s * kConvMaxTargets + tt] = m.x;
+        sm_md[s * kConvMaxTargets + tt] = (double)m.y;  // exact: below 2^44 where it is used
     }
     for (int tt = threadIdx.x; tt < n_tgt; tt += blockDim.x) {
         int t = tt < s0 ? tt : tt + NS;
         DevPrime p = pr[a.tprime[t]];
         sm_t[tt] = ConvTarget{p.q, p.qinv_neg, p.one_shoup, 0};
+        sm_f[tt] = fpm[a.tprime[t]];
     }
     __syncthreads();
     int c = blockIdx.x * blockDim.x + threadIdx.x;
     int i = blockIdx.y;
     if (c >= N) return;
     uint64_t y[NS];
+    bool narrow[NS];  // source prime below 2^44: y usable unreduced by the FP64 product
 #pragma unroll
     for (int s = 0; s < NS; s++) {
         uint64_t q = pr[s0 + s].q;
         uint64_t x = coef[((size_t)i * level + s0 + s) * N + c];
         ulonglong2 w = src[s];
         y[s] = mul_shoup(x, w.x, w.y, q);
+        narrow[s] = q < kFpPrimeLimit;
     }
     uint64_t* o = ext_j + (size_t)i * n_tgt * N + c;
     for (int tt = 0; tt < n_tgt; tt++) {
-        U128 acc = {0, 0};
+        const ConvTarget t = sm_t[tt];
+        if (t.q < kFpPrimeLimit) {
+            // FP64 path: sum_s y_s m_st mod t, each product exact on the FP64 pipe
+            const FpMod f = sm_f[tt];
+            double acc = 0.0;
 #pragma unroll
-        for (int s = 0; s < NS; s++) mac128(acc, y[s], sm_m[s * kConvMaxTargets + tt]);
-        o[(size_t)tt * N] = redc_t(acc, sm_t[tt]);
+            for (int s = 0; s < NS; s++) {
+                uint64_t ys = y[s];
+                if (!narrow[s]) ys = csub(ys - __umul64hi(ys, t.one_shoup) * t.q, t.q);
+                double term = fp_modmul(u2d(ys), sm_md[s * kConvMaxTargets + tt], f);
+                acc = fp_csub(__dadd_rn(acc, term), f.q);
+            }
+            o[(size_t)tt * N] = d2u(acc);
+        } else {
+            U128 acc = {0, 0};
+#pragma unroll
+            for (int s = 0; s < NS; s++) mac128(acc, y[s], sm_m[s * kConvMaxTargets + tt]);
+            o[(size_t)tt * N] = redc_t(acc, t);
+        }
     }
 }
 
-// u[i][0/1][t][c] = sum_j x_j[t][c] * key_j[b/a][row(t)][c]   (key in Montgomery form),
+// u[i][0/1][t][c] = sum_j x_j[t][c] * key_i,j[b/a][row(t)][c]   (keys in Montgomery form),
 // x_j = the evaluation-domain input on digit j's own rows, ext_j elsewhere.
-__global__ void k_ks_inner(const uint64_t* __restrict__ ext, const uint64_t* __restrict__ sig,
-                           const uint64_t* __restrict__ key, uint64_t* __restrict__ u, int n_digits, int n_rows,
-                           int level, int L, int LK, int n_cts, const DevPrime* __restrict__ pr, ModupArgs a,
-                           int logn) {
+// The ciphertext index is the fastest grid dimension: neighbouring blocks
+// that share a key read the same key tile, which DRAM then serves once.
+__global__ void k_ks_inner(const uint64_t* __restrict__ ext, const uint64_t* __restrict__ sig, PtrList keys,
+                           uint64_t* __restrict__ u, int n_digits, int n_rows, int level, int L, int LK, int n_cts,
+                           const DevPrime* __restrict__ pr, ModupArgs a, int logn) {
     const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x;
-    int t = blockIdx.y, i = blockIdx.z;
+    int i = blockIdx.x, t = blockIdx.z;
+    int c = blockIdx.y * blockDim.x + threadIdx.x;
     if (c >= N) return;
+    const uint64_t* key = keys.p[i];
     int krow = t < level ? t : L + (t - level);
     DevPrime p = pr[a.tprime[t]];
     U128 acc0 = {0, 0}, acc1 = {0, 0};
@@ -205,12 +233,13 @@ __global__ void __launch_bounds__(256)
 
 // out_i[poly][r][c] = (u[poly][r] - tmp[poly][r]) P^-1 + add_poly
 __global__ void k_moddown_combine(const uint64_t* __restrict__ u, const uint64_t* __restrict__ tmp, MutPtrList out,
-                                  PtrList add0, PtrList add1, int sig_add0, uint64_t galois, int level, int K,
+                                  PtrList add0, PtrList add1, int sig_add0, GalList gal, int level, int K,
                                   const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ pinv, int logn) {
     const int N = 1 << logn;
     int c = blockIdx.x * blockDim.x + threadIdx.x;
     int r = blockIdx.y % level, poly = blockIdx.y / level, i = blockIdx.z;
     if (c >= N) return;
+    const uint64_t galois = gal.g[i];
     const int n_rows = level + K;
     uint64_t q = pr[r].q;
     uint64_t uv = u[(((size_t)i * 2 + poly) * n_rows + r) * N + c];
@@ -255,7 +284,7 @@ size_t key_switch_scratch_words(const he_ctx* c, int n, int level) {
     return (size_t)c->N * n * (2 * level + ext_rows + 2 * nr + 2 * level);
 }
 
-int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList& io) {
+int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     const int N = c->N, K = c->K, L = c->L, LK = L + K;
     const int n_rows = level + K;
     ModupArgs ma = modup_args(c, level);
@@ -272,8 +301,11 @@ int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList
 
     PtrList din;
     MutPtrList dout;
-    PtrList a0, a1;
+    PtrList a0, a1, keys;
+    GalList gal;
     for (int i = 0; i < kMaxBatch; i++) {
+        gal.g[i] = i < n ? io.galois[i] : 0;
+        keys.p[i] = i < n ? io.key[i] : nullptr;
         din.p[i] = i < n ? io.d[i] : nullptr;
         dout.p[i] = i < n ? io.out[i] : nullptr;
         a0.p[i] = i < n ? io.add0[i] : nullptr;
@@ -288,7 +320,7 @@ int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList
     for (int j = 0; j < nd; j++) sum_src += ma.n_src[j];
 
     prof_begin(c, HE_PROF_AUTOMORPH);
-    k_gather<<<dim3(gx, level, n), blk, 0, c->stream>>>(din, sig, coef, level, c->log_n, io.galois);
+    k_gather<<<dim3(gx, level, n), blk, 0, c->stream>>>(din, sig, coef, level, c->log_n, gal);
     if ((rc = lc(c, "gather"))) return rc;
     prof_end(c, HE_PROF_AUTOMORPH, 3.0 * n * level * limbB, 0);
 
@@ -303,7 +335,7 @@ int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList
 #define HE_MU_CASE(S)                                                                                       \
     case S:                                                                                                 \
         k_modup_conv<S><<<dim3(gx, n), blk, 0, c->stream>>>(coef, ext_j, ma.src[j], ma.mat[j], ma, c->d_prime, \
-                                                            level, n_rows, s0, c->log_n);                   \
+                                                            c->d_fpmod, level, n_rows, s0, c->log_n);       \
         break;
             HE_MU_CASE(1) HE_MU_CASE(2) HE_MU_CASE(3) HE_MU_CASE(4) HE_MU_CASE(5) HE_MU_CASE(6) HE_MU_CASE(7)
             HE_MU_CASE(8) HE_MU_CASE(9) HE_MU_CASE(10) HE_MU_CASE(11) HE_MU_CASE(12) HE_MU_CASE(13)
@@ -331,8 +363,8 @@ int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList
     }
 
     prof_begin(c, HE_PROF_KS_INNER);
-    k_ks_inner<<<dim3(gx, n_rows, n), blk, 0, c->stream>>>(ext, sig, key.d, u, nd, n_rows, level, L, LK, n,
-                                                           c->d_prime, ma, c->log_n);
+    k_ks_inner<<<dim3(n, gx, n_rows), blk, 0, c->stream>>>(ext, sig, keys, u, nd, n_rows, level, L, LK, n, c->d_prime,
+                                                           ma, c->log_n);
     if ((rc = lc(c, "ks_inner"))) return rc;
     prof_end(c, HE_PROF_KS_INNER, ((double)n * nd * n_rows + 2.0 * nd * n_rows + 2.0 * n * n_rows) * limbB,
              (double)n * n_rows * N * (2.0 * nd + 2));
@@ -362,7 +394,7 @@ int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList
 
     prof_begin(c, HE_PROF_MODDOWN_COMBINE);
     k_moddown_combine<<<dim3(gx, 2 * level, n), blk, 0, c->stream>>>(u, tmp, dout, a0, a1, io.sig_add0 ? 1 : 0,
-                                                                     io.galois, level, K, c->d_prime, c->d_md_pinv,
+                                                                     gal, level, K, c->d_prime, c->d_md_pinv,
                                                                      c->log_n);
     if ((rc = lc(c, "moddown_combine"))) return rc;
     {
@@ -373,18 +405,19 @@ int key_switch_chunk(he_ctx* c, int n, int level, const Key& key, const KsIoList
     return HE_OK;
 }
 
-int key_switch(he_ctx* c, int level, const Key& key, const KsIoList& io) {
+int key_switch(he_ctx* c, int level, const KsIoList& io) {
     int n = (int)io.d.size();
     for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
         int m = std::min(kMaxBatch, n - i0);
         KsIoList sub;
-        sub.galois = io.galois;
         sub.sig_add0 = io.sig_add0;
+        sub.galois.assign(io.galois.begin() + i0, io.galois.begin() + i0 + m);
+        sub.key.assign(io.key.begin() + i0, io.key.begin() + i0 + m);
         sub.d.assign(io.d.begin() + i0, io.d.begin() + i0 + m);
         sub.out.assign(io.out.begin() + i0, io.out.begin() + i0 + m);
         sub.add0.assign(io.add0.begin() + i0, io.add0.begin() + i0 + m);
         sub.add1.assign(io.add1.begin() + i0, io.add1.begin() + i0 + m);
-        int rc = key_switch_chunk(c, m, level, key, sub);
+        int rc = key_switch_chunk(c, m, level, sub);
         if (rc) return rc;
     }
     return HE_OK;
@@ -417,7 +450,10 @@ int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, in
             return set_err(c, HE_ENOKEY, "rotate: no key for step %d (galois %llu)", steps[i], (unsigned long long)g);
         groups[g].push_back(i);
     }
+    // one key-switching pass over every ciphertext, ordered by key
     const size_t ct_words = (size_t)2 * level * c->N;
+    KsIoList io;
+    io.sig_add0 = true;
     for (auto& kv : groups) {
         if (kv.first == 1) {  // rotation by a multiple of N/2: identity
             for (int i : kv.second) {
@@ -427,16 +463,18 @@ int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, in
             }
             continue;
         }
-        KsIoList io;
-        io.galois = kv.first;
-        io.sig_add0 = true;
+        const uint64_t* key = c->rot_keys[kv.first].d;
         for (int i : kv.second) {
+            io.galois.push_back(kv.first);
+            io.key.push_back(key);
             io.d.push_back(in[i].data + (size_t)level * c->N);
             io.out.push_back(out[i].data);
             io.add0.push_back(in[i].data);
             io.add1.push_back(nullptr);
         }
-        int rc = key_switch(c, level, c->rot_keys[kv.first], io);
+    }
+    if (!io.d.empty()) {
+        int rc = key_switch(c, level, io);
         if (rc) return rc;
     }
     for (int i = 0; i < n; i++) {

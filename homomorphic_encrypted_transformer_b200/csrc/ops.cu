@@ -239,7 +239,7 @@ int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vecto
     if (level < 2) return set_err(c, HE_ELEVEL, "hmult: level %d cannot be rescaled", level);
     const int gx = (N + TB - 1) / TB;
     const size_t per = (size_t)5 * level * N;  // d0 d1 d2 | relinearised [2][level]
-    const int chunk = 32;
+    const int chunk = 64;
     for (int i0 = 0; i0 < n; i0 += chunk) {
         int m = std::min(chunk, n - i0);
         uint64_t* base;
@@ -252,12 +252,14 @@ int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vecto
             k_tensor<<<dim3(gx, level), TB, 0, c->stream>>>(a[i0 + i], b[i0 + i], d, level, c->d_prime, c->log_n);
             if ((rc = lc(c, "tensor"))) return rc;
             prof_end(c, HE_PROF_ELEMENTWISE);
+            io.galois.push_back(0);
+            io.key.push_back(c->relin.d);
             io.d.push_back(d + (size_t)2 * level * N);
             io.out.push_back(d + (size_t)3 * level * N);
             io.add0.push_back(d);
             io.add1.push_back(d + (size_t)level * N);
         }
-        if ((rc = key_switch(c, level, c->relin, io))) return rc;
+        if ((rc = key_switch(c, level, io))) return rc;
         std::vector<const uint64_t*> rin(io.out.begin(), io.out.end());
         std::vector<uint64_t*> rout(out.begin() + i0, out.begin() + i0 + m);
         if ((rc = rescale_many(c, rin, rout, level))) return rc;
