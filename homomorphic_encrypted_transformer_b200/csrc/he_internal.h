@@ -110,6 +110,11 @@ std::vector<int> ext_primes(const he_ctx* c, int level);
 int ntt_setup(he_ctx* c);
 int ntt_fwd_set(he_ctx* c, const RowSet& rs, int n_rows);
 int ntt_inv_set(he_ctx* c, const RowSet& rs, int n_rows);
+// Single passes, for callers that fuse the other pass with their own work:
+// the forward column pass (stages 0..S1-1) and the inverse column pass
+// (stages S1-1..0, scaled by N^-1).
+int ntt_fwd_cols_set(he_ctx* c, const RowSet& rs, int n_rows);
+int ntt_inv_cols_set(he_ctx* c, const RowSet& rs, int n_rows);
 
 // Key switching of polynomials d[i] (evaluation domain, [level][N] each) with
 // one key.  Writes out[i] = [2][level][N]:

@@ -32,6 +32,29 @@ struct RowSet {
     }
 };
 
+// Per-ciphertext parameters of batched launches (at most 64 ciphertexts).
+constexpr int kMaxBatch = 64;
+struct PtrList {
+    const uint64_t* p[kMaxBatch];
+};
+struct MutPtrList {
+    uint64_t* p[kMaxBatch];
+};
+struct GalList {
+    uint64_t g[kMaxBatch];
+};
+
+// Evaluation-domain index whose value sigma_k moves to index j (k = 0: j):
+// storage j is the point psi^(2 brev(j)+1); sigma_k(a) there is a(psi^((2 brev(j)+1) k)).
+// An aligned block of 2^m indices maps onto an aligned block of 2^m indices.
+__device__ __forceinline__ int automorph_src(int j, int logn, uint64_t k) {
+    if (!k) return j;
+    unsigned m = __brev((unsigned)j) >> (32 - logn);
+    uint64_t e = ((2ull * m + 1) * k) & ((2ull << logn) - 1);
+    unsigned m2 = (unsigned)((e - 1) >> 1);
+    return (int)(__brev(m2) >> (32 - logn));
+}
+
 struct NttShape {
     int s1, s2;          // log2 of rows (R) and columns (C), N = R C
     int tc, tr;          // columns per column-pass tile, rows per row-pass tile

@@ -13,43 +13,50 @@
 
 namespace he {
 
-constexpr int kMaxBatch = 64;
 constexpr int kMaxDigits = 15;
 
-struct PtrList {
-    const uint64_t* p[kMaxBatch];
-};
-struct MutPtrList {
-    uint64_t* p[kMaxBatch];
-};
-struct GalList {
-    uint64_t g[kMaxBatch];
-};
-
-// Evaluation-domain index whose value sigma_k moves to index j:
-// storage j is the point psi^(2 brev(j)+1); sigma_k(a) there is a(psi^((2 brev(j)+1) k)).
-__device__ __forceinline__ int automorph_src(int j, int logn, uint64_t k) {
-    unsigned m = __brev((unsigned)j) >> (32 - logn);
-    uint64_t e = ((2ull * m + 1) * k) & ((2ull << logn) - 1);
-    unsigned m2 = (unsigned)((e - 1) >> 1);
-    return (int)(__brev(m2) >> (32 - logn));
+// x[k] = d[automorph_src(j0 + k)], k < 16, j0 even.  sigma_k maps the
+// aligned pair {2m, 2m+1} onto an aligned pair (src(j ^ 1) = src(j) ^ 1), so
+// each pair is one 16-byte load, swapped when src(j0 + 2k) is odd.  With
+// k = 0 this is a plain load.
+template <int LOGN, typename T>
+__device__ __forceinline__ void gather_load16(T (&x)[16], const uint64_t* __restrict__ d, int j0, uint64_t galois) {
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+        const int s = automorph_src(j0 + 2 * k, LOGN, galois);
+        const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2*>(d + (s & ~1)));
+        const bool sw = s & 1;
+        x[2 * k] = to_elem(sw ? v.y : v.x, T());
+        x[2 * k + 1] = to_elem(sw ? v.x : v.y, T());
+    }
 }
 
-// sig[i][r][c] = coef[i][r][c] = d_i[r][src(c)] (a plain copy when galois == 0).
-// sig keeps the evaluation-domain values (the digit's own rows of ModUp);
-// coef is transformed back to coefficients in place afterwards.
-__global__ void k_gather(PtrList in, uint64_t* __restrict__ sig, uint64_t* __restrict__ coef, int level, int logn,
-                         GalList gal) {
-    const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x;
-    int r = blockIdx.y, i = blockIdx.z;
-    if (c >= N) return;
-    const uint64_t galois = gal.g[i];
-    int src = galois ? automorph_src(c, logn, galois) : c;
-    uint64_t v = in.p[i][(size_t)r * N + src];
-    size_t o = ((size_t)i * level + r) * N + c;
-    sig[o] = v;
-    coef[o] = v;
+// First pass of the inverse NTT of sigma_{g_i}(d_i), the automorphism folded
+// into its loads: coef[i][t] = inverse row pass of (d_i[t][automorph_src(.)]).
+// Rows t of Q_level have prime index t.  Grid (ROW_TILES, n level).
+template <int LOGN>
+__global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
+    k_inv_rows_gather(PtrList din, GalList gal, uint64_t* __restrict__ coef, int level,
+                      const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all,
+                      const double* __restrict__ twd_all, const FpMod* __restrict__ fpm) {
+    using Cf = NttCfg<LOGN>;
+    __shared__ uint64_t sm[Cf::TR * Cf::ROW_PITCH];
+    const int y = blockIdx.y, i = y / level, t = y - i * level;
+    const uint64_t q = pr[t].q;
+    const int r = blockIdx.x * Cf::TR + threadIdx.x / (Cf::C / 16);
+    const int j0 = r * Cf::C + 16 * row_lane<LOGN>();
+    const uint64_t* d = din.p[i] + (size_t)t * Cf::N;
+    uint64_t* out = coef + (size_t)y * Cf::N + (size_t)r * Cf::C;
+    const uint64_t g = gal.g[i];
+    if (q < kFpPrimeLimit) {
+        double x[16];
+        gather_load16<LOGN>(x, d, j0, g);
+        inv_rows_core<LOGN>(x, reinterpret_cast<double*>(sm), out, r, twd_all + (size_t)t * Cf::N, fpm[t]);
+    } else {
+        uint64_t x[16];
+        gather_load16<LOGN>(x, d, j0, g);
+        inv_rows_core<LOGN>(x, sm, out, r, tw_all + (size_t)t * Cf::N, q);
+    }
 }
 
 // ModUp of digit j at one level.  Rows of Q_level and P are numbered
@@ -148,10 +155,12 @@ __global__ void __launch_bounds__(256)
 }
 
 // u[i][0/1][t][c] = sum_j x_j[t][c] * key_i,j[b/a][row(t)][c]   (keys in Montgomery form),
-// x_j = the evaluation-domain input on digit j's own rows, ext_j elsewhere.
+// x_j = sigma_{g_i}(d_i) on digit j's own rows (read through the
+// automorphism: an aligned group of 32 indices maps onto one, so a warp's
+// loads stay within the same 256 bytes), ext_j elsewhere.
 // The ciphertext index is the fastest grid dimension: neighbouring blocks
 // that share a key read the same key tile, which DRAM then serves once.
-__global__ void k_ks_inner(const uint64_t* __restrict__ ext, const uint64_t* __restrict__ sig, PtrList keys,
+__global__ void k_ks_inner(const uint64_t* __restrict__ ext, PtrList din, GalList gal, PtrList keys,
                            uint64_t* __restrict__ u, int n_digits, int n_rows, int level, int L, int LK, int n_cts,
                            const DevPrime* __restrict__ pr, ModupArgs a, int logn) {
     const int N = 1 << logn;
@@ -159,6 +168,7 @@ __global__ void k_ks_inner(const uint64_t* __restrict__ ext, const uint64_t* __r
     int c = blockIdx.y * blockDim.x + threadIdx.x;
     if (c >= N) return;
     const uint64_t* key = keys.p[i];
+    const int own = automorph_src(c, logn, gal.g[i]);
     int krow = t < level ? t : L + (t - level);
     DevPrime p = pr[a.tprime[t]];
     U128 acc0 = {0, 0}, acc1 = {0, 0};
@@ -166,7 +176,7 @@ __global__ void k_ks_inner(const uint64_t* __restrict__ ext, const uint64_t* __r
         const int s0 = a.src_row[j], ns = a.n_src[j];
         uint64_t x;
         if (t >= s0 && t < s0 + ns) {
-            x = sig[((size_t)i * level + t) * N + c];
+            x = __ldg(din.p[i] + (size_t)t * N + own);
         } else {
             int pos = t < s0 ? t : t - ns;
             x = ext[((size_t)a.ext_off[j] * n_cts + (size_t)i * (n_rows - ns) + pos) * N + c];
@@ -231,27 +241,68 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// out_i[poly][r][c] = (u[poly][r] - tmp[poly][r]) P^-1 + add_poly
-__global__ void k_moddown_combine(const uint64_t* __restrict__ u, const uint64_t* __restrict__ tmp, MutPtrList out,
-                                  PtrList add0, PtrList add1, int sig_add0, GalList gal, int level, int K,
-                                  const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ pinv, int logn) {
-    const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x;
-    int r = blockIdx.y % level, poly = blockIdx.y / level, i = blockIdx.z;
-    if (c >= N) return;
-    const uint64_t galois = gal.g[i];
-    const int n_rows = level + K;
-    uint64_t q = pr[r].q;
-    uint64_t uv = u[(((size_t)i * 2 + poly) * n_rows + r) * N + c];
-    uint64_t tv = tmp[(((size_t)i * 2 + poly) * level + r) * N + c];
-    ulonglong2 w = pinv[r];
-    uint64_t v = mul_shoup(uv + q - tv, w.x, w.y, q);
-    const uint64_t* ad = poly == 0 ? add0.p[i] : add1.p[i];
-    if (ad) {
-        int src = (poly == 0 && sig_add0 && galois) ? automorph_src(c, logn, galois) : c;
-        v = add_mod(v, ad[(size_t)r * N + src], q);
+// Outputs of ModDown: out_i = [2][level][N]; add0/add1 (or null) are added
+// to the two polynomials, add0 read through sigma_{g_i} when sig_add0 is set.
+struct MdOut {
+    MutPtrList out;
+    PtrList add0, add1;
+    GalList gal;
+    int sig_add0;
+};
+
+// Second pass of the forward NTT of tmp fused with the end of ModDown:
+//   out_i[poly][t][c] = (u[poly][t][c] - NTT(tmp)[poly][t][c]) P^-1 + add_poly[t][c].
+// tmp rows are [i][poly][t] (prime index t).  Grid (ROW_TILES, n 2 level).
+template <int LOGN>
+__global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
+    k_fwd_rows_moddown(const uint64_t* __restrict__ tmp, const uint64_t* __restrict__ u, MdOut mo, int level, int K,
+                       const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ pinv,
+                       const ulonglong2* __restrict__ tw_all, const double* __restrict__ twd_all,
+                       const FpMod* __restrict__ fpm) {
+    using Cf = NttCfg<LOGN>;
+    __shared__ uint64_t sm[Cf::TR * Cf::ROW_PITCH];
+    const int y = blockIdx.y, i = y / (2 * level), rem = y - i * 2 * level;
+    const int poly = rem / level, t = rem - poly * level;
+    const uint64_t q = pr[t].q;
+    const int r = blockIdx.x * Cf::TR + threadIdx.x / (Cf::C / 16);
+    const int j0 = r * Cf::C + 16 * row_lane<LOGN>();
+    const uint64_t* a = tmp + (size_t)y * Cf::N + (size_t)r * Cf::C;
+    uint64_t v[16];
+    if (q < kFpPrimeLimit) {
+        const FpMod m = fpm[t];
+        double x[16];
+        row_load_strided<LOGN>(x, a);
+        fwd_rows_core<LOGN>(x, reinterpret_cast<double*>(sm), r, twd_all + (size_t)t * Cf::N, m);
+#pragma unroll
+        for (int k = 0; k < 16; k++) v[k] = d2u(reduce4q(x[k], m));
+    } else {
+        uint64_t x[16];
+        row_load_strided<LOGN>(x, a);
+        fwd_rows_core<LOGN>(x, sm, r, tw_all + (size_t)t * Cf::N, q);
+#pragma unroll
+        for (int k = 0; k < 16; k++) v[k] = reduce4q(x[k], q);
     }
-    out.p[i][((size_t)poly * level + r) * N + c] = v;
+    const size_t off = (size_t)t * Cf::N + j0;  // within a [level][N] polynomial
+    const ulonglong2* up = reinterpret_cast<const ulonglong2*>(u + (size_t)(i * 2 + poly) * (level + K) * Cf::N + off);
+    ulonglong2* op = reinterpret_cast<ulonglong2*>(mo.out.p[i] + (size_t)poly * level * Cf::N + off);
+    const uint64_t* ad = poly == 0 ? mo.add0.p[i] : mo.add1.p[i];
+    const uint64_t g = (poly == 0 && mo.sig_add0) ? mo.gal.g[i] : 0;
+    const ulonglong2 w = pinv[t];
+    const uint64_t* adt = ad ? ad + (size_t)t * Cf::N : nullptr;
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+        const ulonglong2 uv = up[k];
+        uint64_t z0 = mul_shoup(uv.x + q - v[2 * k], w.x, w.y, q);
+        uint64_t z1 = mul_shoup(uv.y + q - v[2 * k + 1], w.x, w.y, q);
+        if (adt) {
+            const int s = automorph_src(j0 + 2 * k, LOGN, g);
+            const ulonglong2 av = __ldg(reinterpret_cast<const ulonglong2*>(adt + (s & ~1)));
+            const bool sw = s & 1;
+            z0 = add_mod(z0, sw ? av.y : av.x, q);
+            z1 = add_mod(z1, sw ? av.x : av.y, q);
+        }
+        op[k] = make_ulonglong2(z0, z1);
+    }
 }
 
 static ModupArgs modup_args(he_ctx* c, int level) {
@@ -277,12 +328,41 @@ static int lc(he_ctx* c, const char* what) {
     return check_cuda(c, cudaGetLastError(), what);
 }
 
-// coef + sig [n][level], ext [n][sum_j (level+K-|D_j|)], u [n][2][level+K], tmp [n][2][level]
+// coef [n][level], ext [n][sum_j (level+K-|D_j|)], u [n][2][level+K], tmp [n][2][level]
 size_t key_switch_scratch_words(const he_ctx* c, int n, int level) {
     size_t nd = (level + c->alpha - 1) / c->alpha, nr = level + c->K;
     size_t ext_rows = nd * nr - level;
-    return (size_t)c->N * n * (2 * level + ext_rows + 2 * nr + 2 * level);
+    return (size_t)c->N * n * (level + ext_rows + 2 * nr + 2 * level);
 }
+
+// Launches of the transform-fused kernels for the context's ring degree.
+template <int LOGN>
+static void launch_inv_rows_gather(he_ctx* c, const PtrList& din, const GalList& gal, uint64_t* coef, int n,
+                                   int level) {
+    using Cf = NttCfg<LOGN>;
+    k_inv_rows_gather<LOGN><<<dim3(Cf::ROW_TILES, n * level), Cf::ROW_THREADS, 0, c->stream>>>(
+        din, gal, coef, level, c->d_prime, c->d_tw_inv, c->d_twd_inv, c->d_fpmod);
+}
+
+template <int LOGN>
+static void launch_fwd_rows_moddown(he_ctx* c, const uint64_t* tmp, const uint64_t* u, const MdOut& mo, int n,
+                                    int level) {
+    using Cf = NttCfg<LOGN>;
+    k_fwd_rows_moddown<LOGN><<<dim3(Cf::ROW_TILES, n * 2 * level), Cf::ROW_THREADS, 0, c->stream>>>(
+        tmp, u, mo, level, c->K, c->d_prime, c->d_md_pinv, c->d_tw_fwd, c->d_twd_fwd, c->d_fpmod);
+}
+
+#define HE_LOGN_SWITCH(c, CALL)                  \
+    switch ((c)->log_n) {                        \
+        case 10: CALL(10); break;                \
+        case 11: CALL(11); break;                \
+        case 12: CALL(12); break;                \
+        case 13: CALL(13); break;                \
+        case 14: CALL(14); break;                \
+        case 15: CALL(15); break;                \
+        case 16: CALL(16); break;                \
+        default: break;                          \
+    }
 
 int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     const int N = c->N, K = c->K, L = c->L, LK = L + K;
@@ -294,38 +374,41 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     if (rc) return rc;
     const int ext_rows = nd * n_rows - level;  // sum over digits of the target rows
     uint64_t* coef = base;
-    uint64_t* sig = coef + (size_t)n * level * N;
-    uint64_t* ext = sig + (size_t)n * level * N;
+    uint64_t* ext = coef + (size_t)n * level * N;
     uint64_t* u = ext + (size_t)n * ext_rows * N;
     uint64_t* tmp = u + (size_t)n * 2 * n_rows * N;
 
-    PtrList din;
-    MutPtrList dout;
-    PtrList a0, a1, keys;
+    PtrList din, keys;
     GalList gal;
+    MdOut mo;
+    mo.sig_add0 = io.sig_add0 ? 1 : 0;
     for (int i = 0; i < kMaxBatch; i++) {
         gal.g[i] = i < n ? io.galois[i] : 0;
         keys.p[i] = i < n ? io.key[i] : nullptr;
         din.p[i] = i < n ? io.d[i] : nullptr;
-        dout.p[i] = i < n ? io.out[i] : nullptr;
-        a0.p[i] = i < n ? io.add0[i] : nullptr;
-        a1.p[i] = i < n ? io.add1[i] : nullptr;
+        mo.out.p[i] = i < n ? io.out[i] : nullptr;
+        mo.add0.p[i] = i < n ? io.add0[i] : nullptr;
+        mo.add1.p[i] = i < n ? io.add1[i] : nullptr;
     }
+    mo.gal = gal;
     const int TB = 256;
     dim3 blk(TB);
     int gx = (N + TB - 1) / TB;
 
     const double limbB = 8.0 * N;
+    const NttShape sh = ntt_shape(c->log_n);
     int sum_src = 0;
     for (int j = 0; j < nd; j++) sum_src += ma.n_src[j];
 
-    prof_begin(c, HE_PROF_AUTOMORPH);
-    k_gather<<<dim3(gx, level, n), blk, 0, c->stream>>>(din, sig, coef, level, c->log_n, gal);
-    if ((rc = lc(c, "gather"))) return rc;
-    prof_end(c, HE_PROF_AUTOMORPH, 3.0 * n * level * limbB, 0);
-
+    // sigma(d) back to coefficients: gathered row pass, then the column pass
+    prof_begin(c, HE_PROF_NTT_INV_ROWS);
+#define HE_IRG(LN) launch_inv_rows_gather<LN>(c, din, gal, coef, n, level)
+    HE_LOGN_SWITCH(c, HE_IRG)
+#undef HE_IRG
+    if ((rc = lc(c, "inv_rows_gather"))) return rc;
+    prof_end(c, HE_PROF_NTT_INV_ROWS, 2.0 * n * level * limbB, 0.5 * N * n * level * sh.s2);
     std::vector<int> qp = prime_range(0, level);
-    if ((rc = ntt_inv_set(c, rowset_contig(coef, level, N, qp), n * level))) return rc;
+    if ((rc = ntt_inv_cols_set(c, rowset_contig(coef, level, N, qp), n * level))) return rc;
 
     prof_begin(c, HE_PROF_MODUP);
     for (int j = 0; j < nd; j++) {
@@ -363,8 +446,8 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     }
 
     prof_begin(c, HE_PROF_KS_INNER);
-    k_ks_inner<<<dim3(n, gx, n_rows), blk, 0, c->stream>>>(ext, sig, keys, u, nd, n_rows, level, L, LK, n, c->d_prime,
-                                                           ma, c->log_n);
+    k_ks_inner<<<dim3(n, gx, n_rows), blk, 0, c->stream>>>(ext, din, gal, keys, u, nd, n_rows, level, L, LK, n,
+                                                           c->d_prime, ma, c->log_n);
     if ((rc = lc(c, "ks_inner"))) return rc;
     prof_end(c, HE_PROF_KS_INNER, ((double)n * nd * n_rows + 2.0 * nd * n_rows + 2.0 * n * n_rows) * limbB,
              (double)n * n_rows * N * (2.0 * nd + 2));
@@ -390,17 +473,19 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     if ((rc = lc(c, "moddown_conv"))) return rc;
     prof_end(c, HE_PROF_MODDOWN_CONV, 2.0 * n * (K + level) * limbB, 2.0 * n * N * (K + (double)K * level));
 
-    if ((rc = ntt_fwd_set(c, rowset_contig(tmp, level, N, qp), n * 2 * level))) return rc;
-
+    // back to the evaluation domain: column pass, then the row pass fused
+    // with (u - tmp) P^-1 + add
+    if ((rc = ntt_fwd_cols_set(c, rowset_contig(tmp, level, N, qp), n * 2 * level))) return rc;
     prof_begin(c, HE_PROF_MODDOWN_COMBINE);
-    k_moddown_combine<<<dim3(gx, 2 * level, n), blk, 0, c->stream>>>(u, tmp, dout, a0, a1, io.sig_add0 ? 1 : 0,
-                                                                     gal, level, K, c->d_prime, c->d_md_pinv,
-                                                                     c->log_n);
-    if ((rc = lc(c, "moddown_combine"))) return rc;
+#define HE_FRM(LN) launch_fwd_rows_moddown<LN>(c, tmp, u, mo, n, level)
+    HE_LOGN_SWITCH(c, HE_FRM)
+#undef HE_FRM
+    if ((rc = lc(c, "fwd_rows_moddown"))) return rc;
     {
         int n_add = 0;
         for (int i = 0; i < n; i++) n_add += (io.add0[i] != nullptr) + (io.add1[i] != nullptr);
-        prof_end(c, HE_PROF_MODDOWN_COMBINE, (6.0 * n + n_add) * level * limbB, 2.0 * n * level * N);
+        prof_end(c, HE_PROF_MODDOWN_COMBINE, (6.0 * n + n_add) * level * limbB,
+                 2.0 * n * level * N * (1.0 + 0.5 * sh.s2));
     }
     return HE_OK;
 }
@@ -425,6 +510,7 @@ int key_switch(he_ctx* c, int level, const KsIoList& io) {
 
 static int ct_ok(he_ctx* c, const he_ct* x, const char* what) {
     if (!x || !x->data) return set_err(c, HE_EINVAL, "%s: null ciphertext", what);
+    if ((uintptr_t)x->data & 15) return set_err(c, HE_EINVAL, "%s: ciphertext not 16-byte aligned", what);
     if (x->level < 1 || x->level > c->L) return set_err(c, HE_ELEVEL, "%s: level %d out of range", what, x->level);
     if (!x->is_ntt) return set_err(c, HE_EDOMAIN, "%s: ciphertext not in the evaluation domain", what);
     return HE_OK;
@@ -439,7 +525,7 @@ int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, in
         int rc = ct_ok(c, &in[i], "rotate");
         if (rc) return rc;
         if (in[i].level != level) return set_err(c, HE_ELEVEL, "rotate: mixed levels in a batch");
-        if (!out[i].data) return set_err(c, HE_EINVAL, "rotate: null output");
+        if (!out[i].data || ((uintptr_t)out[i].data & 15)) return set_err(c, HE_EINVAL, "rotate: null or unaligned output");
         if (out[i].data == in[i].data) return set_err(c, HE_EINVAL, "rotate: output aliases input");
     }
     // group by Galois element so that each key is streamed once per group

@@ -6,19 +6,7 @@
 #include "kernels.cuh"
 #include "ntt.cuh"
 
-
-#define NTT_MIN_BLOCKS 3
 namespace he {
-
-// shared-memory index of element i of a padded row (one pad word per 16)
-__device__ __forceinline__ int padded(int i) { return i + (i >> 4); }
-
-// Element handling of the two arithmetic paths: 64-bit integers with Shoup
-// twiddles (any prime), or exact doubles on the FP64 pipe (primes < 2^44).
-__device__ __forceinline__ uint64_t to_elem(uint64_t v, uint64_t) { return v; }
-__device__ __forceinline__ double to_elem(uint64_t v, double) { return u2d(v); }
-__device__ __forceinline__ uint64_t from_elem(uint64_t v) { return v; }
-__device__ __forceinline__ uint64_t from_elem(double v) { return d2u(v); }
 
 template <int LOGN, typename T, typename TW, typename M>
 __device__ __forceinline__ void fwd_cols_body(T* sm, uint64_t* a, const TW* tw, const M& m) {
@@ -41,49 +29,17 @@ __device__ __forceinline__ void fwd_cols_body(T* sm, uint64_t* a, const TW* tw, 
 
 template <int LOGN, typename T, typename TW, typename M>
 __device__ __forceinline__ void fwd_rows_body(T* sm, uint64_t* a, int r, const TW* tw, const M& m) {
-    using Cf = NttCfg<LOGN>;
-    constexpr int CS = Cf::C / 16;
-    const int p = threadIdx.x % CS, rr = threadIdx.x / CS;
-    T* s = sm + rr * Cf::ROW_PITCH;
     T x[16];
-#pragma unroll
-    for (int k = 0; k < 16; k++) x[k] = to_elem(a[p + CS * k], T());
-    fwd_stages<4>(x, tw, Cf::S1, r, 0, m);
-#pragma unroll
-    for (int k = 0; k < 16; k++) s[padded(p + CS * k)] = x[k];
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < 16; k++) x[k] = s[padded(16 * p + k)];
-    fwd_stages<Cf::S2 - 4>(x, tw, Cf::S1 + 4, r << 4, 16 * p, m);
-    ulonglong2* o = reinterpret_cast<ulonglong2*>(a + 16 * p);
-#pragma unroll
-    for (int k = 0; k < 8; k++)
-        o[k] = make_ulonglong2(from_elem(reduce4q(x[2 * k], m)), from_elem(reduce4q(x[2 * k + 1], m)));
+    row_load_strided<LOGN>(x, a);
+    fwd_rows_core<LOGN>(x, sm, r, tw, m);
+    row_store16(a + 16 * row_lane<LOGN>(), x, m);
 }
 
 template <int LOGN, typename T, typename TW, typename M>
 __device__ __forceinline__ void inv_rows_body(T* sm, uint64_t* a, int r, const TW* tw, const M& m) {
-    using Cf = NttCfg<LOGN>;
-    constexpr int CS = Cf::C / 16;
-    const int p = threadIdx.x % CS, rr = threadIdx.x / CS;
-    T* s = sm + rr * Cf::ROW_PITCH;
     T x[16];
-    const ulonglong2* in = reinterpret_cast<const ulonglong2*>(a + 16 * p);
-#pragma unroll
-    for (int k = 0; k < 8; k++) {
-        ulonglong2 v = in[k];
-        x[2 * k] = to_elem(v.x, T());
-        x[2 * k + 1] = to_elem(v.y, T());
-    }
-    inv_stages<Cf::S2 - 4>(x, tw, Cf::S1 + 4, r << 4, 16 * p, m);
-#pragma unroll
-    for (int k = 0; k < 16; k++) s[padded(16 * p + k)] = x[k];
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < 16; k++) x[k] = s[padded(p + CS * k)];
-    inv_stages<4>(x, tw, Cf::S1, r, 0, m);
-#pragma unroll
-    for (int k = 0; k < 16; k++) a[p + CS * k] = from_elem(x[k]);
+    row_load16(x, a + 16 * row_lane<LOGN>());
+    inv_rows_core<LOGN>(x, sm, a, r, tw, m);
 }
 
 template <int LOGN>
@@ -243,39 +199,37 @@ static void dispatch(he_ctx* c, const RowSet& rs, int n_rows, bool fwd, int whic
     }
 }
 
-int ntt_fwd_set(he_ctx* c, const RowSet& rs, int n_rows) {
+// One pass of a transform, bracketed for the profile: the column pass does
+// stages 0..S1-1, the row pass stages S1..LOGN-1 (each reads and writes
+// every limb once).
+static int ntt_pass(he_ctx* c, const RowSet& rs, int n_rows, bool fwd, int which) {
     if (n_rows <= 0) return HE_OK;
     NttShape sh = ntt_shape(c->log_n);
     const double bytes = 16.0 * c->N * n_rows, half = 0.5 * c->N * n_rows;
-    prof_begin(c, HE_PROF_NTT_FWD_COLS);
-    dispatch(c, rs, n_rows, true, 0);
-    int rc = launch_check(c, "ntt_fwd_cols");
+    const int cls = fwd ? (which == 0 ? HE_PROF_NTT_FWD_COLS : HE_PROF_NTT_FWD_ROWS)
+                        : (which == 0 ? HE_PROF_NTT_INV_ROWS : HE_PROF_NTT_INV_COLS);
+    const bool col_pass = fwd == (which == 0);
+    prof_begin(c, cls);
+    dispatch(c, rs, n_rows, fwd, which);
+    int rc = launch_check(c, fwd ? "ntt_fwd" : "ntt_inv");
     if (rc) return rc;
-    prof_end(c, HE_PROF_NTT_FWD_COLS, bytes, half * sh.s1);
-    prof_begin(c, HE_PROF_NTT_FWD_ROWS);
-    dispatch(c, rs, n_rows, true, 1);
-    rc = launch_check(c, "ntt_fwd_rows");
-    if (rc) return rc;
-    c->launches += 2;
-    return prof_end(c, HE_PROF_NTT_FWD_ROWS, bytes, half * sh.s2);
+    c->launches += 1;
+    return prof_end(c, cls, bytes, half * (col_pass ? sh.s1 : sh.s2));
+}
+
+int ntt_fwd_set(he_ctx* c, const RowSet& rs, int n_rows) {
+    int rc = ntt_pass(c, rs, n_rows, true, 0);
+    return rc ? rc : ntt_pass(c, rs, n_rows, true, 1);
 }
 
 int ntt_inv_set(he_ctx* c, const RowSet& rs, int n_rows) {
-    if (n_rows <= 0) return HE_OK;
-    NttShape sh = ntt_shape(c->log_n);
-    const double bytes = 16.0 * c->N * n_rows, half = 0.5 * c->N * n_rows;
-    prof_begin(c, HE_PROF_NTT_INV_ROWS);
-    dispatch(c, rs, n_rows, false, 0);
-    int rc = launch_check(c, "ntt_inv_rows");
-    if (rc) return rc;
-    prof_end(c, HE_PROF_NTT_INV_ROWS, bytes, half * sh.s2);
-    prof_begin(c, HE_PROF_NTT_INV_COLS);
-    dispatch(c, rs, n_rows, false, 1);
-    rc = launch_check(c, "ntt_inv_cols");
-    if (rc) return rc;
-    c->launches += 2;
-    return prof_end(c, HE_PROF_NTT_INV_COLS, bytes, half * sh.s1);
+    int rc = ntt_pass(c, rs, n_rows, false, 0);
+    return rc ? rc : ntt_pass(c, rs, n_rows, false, 1);
 }
+
+int ntt_fwd_cols_set(he_ctx* c, const RowSet& rs, int n_rows) { return ntt_pass(c, rs, n_rows, true, 0); }
+
+int ntt_inv_cols_set(he_ctx* c, const RowSet& rs, int n_rows) { return ntt_pass(c, rs, n_rows, false, 1); }
 
 int ntt_setup(he_ctx* c) {
     (void)c;

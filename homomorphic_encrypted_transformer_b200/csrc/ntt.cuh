@@ -216,4 +216,90 @@ __device__ __forceinline__ void inv_stage0_scaled(uint64_t (&x)[16], const ulong
     }
 }
 
+// ---------------------------------------------------------------------------
+// Row pass pieces shared by the plain transforms and the fused key-switching
+// kernels.  Thread (rr, p) of a row-pass block owns columns 16 p + k of row
+// r = tile * TR + rr; after the pass the 16 registers hold those columns.
+
+// Blocks per SM the transforms are compiled for (register budget 85).
+constexpr int NTT_MIN_BLOCKS = 3;
+
+// shared-memory index of element i of a padded row (one pad word per 16)
+__device__ __forceinline__ int padded(int i) { return i + (i >> 4); }
+
+__device__ __forceinline__ uint64_t to_elem(uint64_t v, uint64_t) { return v; }
+__device__ __forceinline__ double to_elem(uint64_t v, double) { return u2d(v); }
+__device__ __forceinline__ uint64_t from_elem(uint64_t v) { return v; }
+__device__ __forceinline__ uint64_t from_elem(double v) { return d2u(v); }
+
+template <int LOGN>
+__device__ __forceinline__ int row_lane() { return threadIdx.x % (NttCfg<LOGN>::C / 16); }
+
+// x[k] = a[k], k < 16 (a 16-byte aligned)
+template <typename T>
+__device__ __forceinline__ void row_load16(T (&x)[16], const uint64_t* a) {
+    const ulonglong2* in = reinterpret_cast<const ulonglong2*>(a);
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+        ulonglong2 v = in[k];
+        x[2 * k] = to_elem(v.x, T());
+        x[2 * k + 1] = to_elem(v.y, T());
+    }
+}
+
+// a[k] = x[k] reduced from [0, 4q) to [0, q)
+template <typename T, typename M>
+__device__ __forceinline__ void row_store16(uint64_t* a, T (&x)[16], const M& m) {
+    ulonglong2* o = reinterpret_cast<ulonglong2*>(a);
+#pragma unroll
+    for (int k = 0; k < 8; k++)
+        o[k] = make_ulonglong2(from_elem(reduce4q(x[2 * k], m)), from_elem(reduce4q(x[2 * k + 1], m)));
+}
+
+// x[k] = row[p + CS k], k < 16 (the forward row pass's input layout)
+template <int LOGN, typename T>
+__device__ __forceinline__ void row_load_strided(T (&x)[16], const uint64_t* row) {
+    constexpr int CS = NttCfg<LOGN>::C / 16;
+    const int p = threadIdx.x % CS;
+#pragma unroll
+    for (int k = 0; k < 16; k++) x[k] = to_elem(row[p + CS * k], T());
+}
+
+// Forward row pass (stages S1..LOGN-1) on registers loaded from columns
+// p + CS k of row r; returns columns 16 p + k in [0, 4q).
+template <int LOGN, typename T, typename TW, typename M>
+__device__ __forceinline__ void fwd_rows_core(T (&x)[16], T* sm, int r, const TW* tw, const M& m) {
+    using Cf = NttCfg<LOGN>;
+    constexpr int CS = Cf::C / 16;
+    const int p = threadIdx.x % CS, rr = threadIdx.x / CS;
+    T* s = sm + rr * Cf::ROW_PITCH;
+    fwd_stages<4>(x, tw, Cf::S1, r, 0, m);
+#pragma unroll
+    for (int k = 0; k < 16; k++) s[padded(p + CS * k)] = x[k];
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 16; k++) x[k] = s[padded(16 * p + k)];
+    fwd_stages<Cf::S2 - 4>(x, tw, Cf::S1 + 4, r << 4, 16 * p, m);
+}
+
+// Inverse row pass (stages LOGN-1..S1) on registers loaded from columns
+// 16 p + k of row r; stores columns p + CS k of the result to out_row.
+template <int LOGN, typename T, typename TW, typename M>
+__device__ __forceinline__ void inv_rows_core(T (&x)[16], T* sm, uint64_t* out_row, int r, const TW* tw,
+                                              const M& m) {
+    using Cf = NttCfg<LOGN>;
+    constexpr int CS = Cf::C / 16;
+    const int p = threadIdx.x % CS, rr = threadIdx.x / CS;
+    T* s = sm + rr * Cf::ROW_PITCH;
+    inv_stages<Cf::S2 - 4>(x, tw, Cf::S1 + 4, r << 4, 16 * p, m);
+#pragma unroll
+    for (int k = 0; k < 16; k++) s[padded(16 * p + k)] = x[k];
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 16; k++) x[k] = s[padded(p + CS * k)];
+    inv_stages<4>(x, tw, Cf::S1, r, 0, m);
+#pragma unroll
+    for (int k = 0; k < 16; k++) out_row[p + CS * k] = from_elem(x[k]);
+}
+
 }  // namespace he

@@ -34,19 +34,12 @@ __global__ void k_signed_to_res(const int32_t* __restrict__ src, uint64_t* __res
 }
 
 // out[r][c] = in[r][automorph_src(c)]
-__device__ __forceinline__ int automorph_src2(int j, int logn, uint64_t k) {
-    unsigned m = __brev((unsigned)j) >> (32 - logn);
-    uint64_t e = ((2ull * m + 1) * k) & ((2ull << logn) - 1);
-    unsigned m2 = (unsigned)((e - 1) >> 1);
-    return (int)(__brev(m2) >> (32 - logn));
-}
-
 __global__ void k_automorph_rows(const uint64_t* __restrict__ in, uint64_t* __restrict__ out, uint64_t galois,
                                  int logn) {
     const int N = 1 << logn;
     int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y;
     if (c >= N) return;
-    out[(size_t)r * N + c] = in[(size_t)r * N + automorph_src2(c, logn, galois)];
+    out[(size_t)r * N + c] = in[(size_t)r * N + automorph_src(c, logn, galois)];
 }
 
 __global__ void k_mul_rows(const uint64_t* __restrict__ a, const uint64_t* __restrict__ b, uint64_t* __restrict__ o,
@@ -183,6 +176,7 @@ int elementwise_setup(he_ctx* c) {
 
 static int ct_ok(he_ctx* c, const he_ct* x, const char* what) {
     if (!x || !x->data) return set_err(c, HE_EINVAL, "%s: null ciphertext", what);
+    if ((uintptr_t)x->data & 15) return set_err(c, HE_EINVAL, "%s: ciphertext not 16-byte aligned", what);
     if (x->level < 1 || x->level > c->L) return set_err(c, HE_ELEVEL, "%s: level %d out of range", what, x->level);
     if (!x->is_ntt) return set_err(c, HE_EDOMAIN, "%s: ciphertext not in the evaluation domain", what);
     return HE_OK;
@@ -453,7 +447,7 @@ extern "C" int he_hmult_relin_rescale(he_ctx* c, const he_ct* a, const he_ct* b,
     if (!c) return HE_EINVAL;
     int rc;
     if ((rc = ct_ok(c, a, "hmult")) || (rc = ct_ok(c, b, "hmult"))) return rc;
-    if (!out || !out->data) return set_err(c, HE_EINVAL, "hmult: null output");
+    if (!out || !out->data || ((uintptr_t)out->data & 15)) return set_err(c, HE_EINVAL, "hmult: null or unaligned output");
     if (a->level != b->level) return set_err(c, HE_ELEVEL, "hmult: levels %d and %d differ", a->level, b->level);
     if (out->data == a->data || out->data == b->data) return set_err(c, HE_EINVAL, "hmult: output aliases an input");
     const int level = a->level;

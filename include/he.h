@@ -79,7 +79,9 @@ typedef struct {
     const uint64_t* p; /* optional host array of n_p primes, or NULL */
 } he_params;
 
-/* A ciphertext: data is a device pointer to [2][level][N] uint64. */
+/* A ciphertext: data is a device pointer to [2][level][N] uint64, 16-byte
+ * aligned (kernels move residues in pairs); calls reject other pointers
+ * with HE_EINVAL. */
 typedef struct {
     uint64_t* data;
     int level;
