@@ -27,7 +27,7 @@ struct ConvTable {
     ulonglong2* d_mat;      // [n_src][level + K] {(qhat_i mod t) 2^64 mod t, qhat_i mod t}
 };
 
-struct FpMod;  // FP64 constants of a prime below 2^44 (ntt.cuh)
+struct FpMod;  // FP64 constants of a prime below 2^41 (ntt.cuh)
 
 struct Key {
     uint64_t* d = nullptr;  // [digits][2][L+K][N] in Montgomery form (value * 2^64 mod p)

@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(256)
         int t = tt < s0 ? tt : tt + NS;
         ulonglong2 m = mat[(size_t)s * n_rows + t];
         sm_m[s * kConvMaxTargets + tt] = m.x;
-        sm_md[s * kConvMaxTargets + tt] = (double)m.y;  // exact: below 2^44 where it is used
+        sm_md[s * kConvMaxTargets + tt] = (double)m.y;  // exact: below 2^41 where it is used
     }
     for (int tt = threadIdx.x; tt < n_tgt; tt += blockDim.x) {
         int t = tt < s0 ? tt : tt + NS;
@@ -121,7 +121,8 @@ __global__ void __launch_bounds__(256)
     int i = blockIdx.y;
     if (c >= N) return;
     uint64_t y[NS];
-    bool narrow[NS];  // source prime below 2^44: y usable unreduced by the FP64 product
+    double yd[NS];    // y as a double where the source prime is below 2^41
+    bool narrow[NS];
 #pragma unroll
     for (int s = 0; s < NS; s++) {
         uint64_t q = pr[s0 + s].q;
@@ -129,22 +130,22 @@ __global__ void __launch_bounds__(256)
         ulonglong2 w = src[s];
         y[s] = mul_shoup(x, w.x, w.y, q);
         narrow[s] = q < kFpPrimeLimit;
+        yd[s] = u2d(narrow[s] ? y[s] : 0);
     }
     uint64_t* o = ext_j + (size_t)i * n_tgt * N + c;
     for (int tt = 0; tt < n_tgt; tt++) {
         const ConvTarget t = sm_t[tt];
         if (t.q < kFpPrimeLimit) {
-            // FP64 path: sum_s y_s m_st mod t, each product exact on the FP64 pipe
+            // FP64 path: signed partial products |.| < 5t/8, one reduction at the end
             const FpMod f = sm_f[tt];
             double acc = 0.0;
 #pragma unroll
             for (int s = 0; s < NS; s++) {
-                uint64_t ys = y[s];
-                if (!narrow[s]) ys = csub(ys - __umul64hi(ys, t.one_shoup) * t.q, t.q);
-                double term = fp_modmul(u2d(ys), sm_md[s * kConvMaxTargets + tt], f);
-                acc = fp_csub(__dadd_rn(acc, term), f.q);
+                // a wide source residue first drops to [0, 2t)
+                double ys = narrow[s] ? yd[s] : u2d(y[s] - __umul64hi(y[s], t.one_shoup) * t.q);
+                acc = __dadd_rn(acc, fp_mulmod_s(ys, sm_md[s * kConvMaxTargets + tt], f));
             }
-            o[(size_t)tt * N] = d2u(acc);
+            o[(size_t)tt * N] = d2u(fp_canon(acc, f));
         } else {
             U128 acc = {0, 0};
 #pragma unroll
@@ -274,13 +275,13 @@ __global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
         row_load_strided<LOGN>(x, a);
         fwd_rows_core<LOGN>(x, reinterpret_cast<double*>(sm), r, twd_all + (size_t)t * Cf::N, m);
 #pragma unroll
-        for (int k = 0; k < 16; k++) v[k] = d2u(reduce4q(x[k], m));
+        for (int k = 0; k < 16; k++) v[k] = fwd_canon(x[k], m);
     } else {
         uint64_t x[16];
         row_load_strided<LOGN>(x, a);
         fwd_rows_core<LOGN>(x, sm, r, tw_all + (size_t)t * Cf::N, q);
 #pragma unroll
-        for (int k = 0; k < 16; k++) v[k] = reduce4q(x[k], q);
+        for (int k = 0; k < 16; k++) v[k] = fwd_canon(x[k], q);
     }
     const size_t off = (size_t)t * Cf::N + j0;  // within a [level][N] polynomial
     const ulonglong2* up = reinterpret_cast<const ulonglong2*>(u + (size_t)(i * 2 + poly) * (level + K) * Cf::N + off);

@@ -1,6 +1,6 @@
 // Batched negacyclic NTT / inverse NTT over RNS limbs: a column pass and a
 // row pass per transform, 16 elements per thread (see ntt.cuh).  Limbs of
-// primes below 2^44 run the butterflies on the FP64 pipe, the others on the
+// primes below 2^41 run the butterflies on the FP64 pipe, the others on the
 // integer pipe (the branch is uniform per block: one limb per block).
 #include "he_internal.h"
 #include "kernels.cuh"
@@ -24,7 +24,7 @@ __device__ __forceinline__ void fwd_cols_body(T* sm, uint64_t* a, const TW* tw, 
     for (int k = 0; k < 16; k++) x[k] = sm[(16 * g + k) * Cf::TC + cc];
     fwd_stages<Cf::S1 - 4>(x, tw, 4, 0, 16 * g, m);
 #pragma unroll
-    for (int k = 0; k < 16; k++) a[(size_t)(16 * g + k) * Cf::C + cc] = from_elem(x[k]);
+    for (int k = 0; k < 16; k++) a[(size_t)(16 * g + k) * Cf::C + cc] = raw_out(x[k]);
 }
 
 template <int LOGN, typename T, typename TW, typename M>
@@ -106,7 +106,8 @@ __device__ __forceinline__ void inv_cols_body(T* sm, uint64_t* a, const TW* tw, 
     constexpr int RS = Cf::R / 16;
     T x[16];
 #pragma unroll
-    for (int k = 0; k < 16; k++) x[k] = to_elem(a[(size_t)(16 * g + k) * Cf::C + cc], T());
+    for (int k = 0; k < 16; k++) x[k] = raw_in(a[(size_t)(16 * g + k) * Cf::C + cc], T());
+    inv_cols_prereduce(x, m);
     inv_stages<Cf::S1 - 4>(x, tw, 4, 0, 16 * g, m);
 #pragma unroll
     for (int k = 0; k < 16; k++) sm[(16 * g + k) * Cf::TC + cc] = x[k];
@@ -116,7 +117,7 @@ __device__ __forceinline__ void inv_cols_body(T* sm, uint64_t* a, const TW* tw, 
     inv_stages<4, 1>(x, tw, 0, 0, 0, m);
     inv_stage0(x, w1, ninv, m);
 #pragma unroll
-    for (int k = 0; k < 16; k++) a[(size_t)(g + RS * k) * Cf::C + cc] = from_elem(x[k]);
+    for (int k = 0; k < 16; k++) a[(size_t)(g + RS * k) * Cf::C + cc] = inv_canon(x[k], m);
 }
 
 template <int LOGN>

@@ -62,8 +62,6 @@ __device__ __forceinline__ void bfly_gs(uint64_t& x, uint64_t& y, const ulonglon
     y = mul_shoup_lazy(a + two_q - b, w.x, w.y, q);
 }
 
-__device__ __forceinline__ uint64_t reduce4q(uint64_t x, uint64_t q) { return csub(csub(x, 2 * q), q); }
-
 __device__ __forceinline__ ulonglong2 ldtw(const ulonglong2* p) { return __ldg(p); }
 
 // Forward stages on 16 registers.  H stages (H <= 4) with register pair
@@ -109,34 +107,55 @@ __device__ __forceinline__ void inv_stages(uint64_t (&x)[16], const ulonglong2* 
 }
 
 // ---------------------------------------------------------------------------
-// FP64 arithmetic for primes below 2^44 (the 40-bit primes of the modulus
-// chain).  Residues are held as doubles (exact integers below 2^53) and the
-// modular product runs on the FP64 pipe:
+// FP64 arithmetic for primes below 2^41 (the 40-bit primes of the modulus
+// chain).  Residues are integers held in doubles (exact below 2^53), signed
+// and unreduced inside a transform; the modular product runs on the FP64
+// pipe with a rounded quotient:
 //   p_hi = fl(y w), p_lo = fma(y, w, -p_hi)          (y w = p_hi + p_lo exactly)
-//   qh = round-to-nearest(p_hi / q) via the 1.5 2^52 magic constant
-//   r = fma(-qh, q, p_hi) + p_lo                     (exact: |r| < q/2 + 2^30)
-//   r < 0 ? r + q : r                                (result in [0, q))
-// The remainder is exact because its true value is an integer far below
-// 2^53, which one rounding of the FMA reproduces.  Checked against integer
-// arithmetic on random and boundary inputs (y < 4q, w < q).
+//   qh = nearest integer to p_hi (1/q)  (1.5 2^52 magic constant)
+//   r = fma(-qh, q, p_hi) + p_lo                     (both steps exact)
+// r = y w - qh q exactly, and for |y| <= Y, 0 <= w < q:
+//   |r| <= q (1/2 + 2^-52 Y)  <=  5q/8  for Y <= 2^49
+// (quotient off by at most 1/2 + 2^-53 Y/1, p_lo at most 2^-53 Y q).
+// No branch and no range correction: sums and differences of such values
+// stay exact integers, and the transforms below keep |y| <= 2^49 by
+// construction (bounds at each use).
 struct FpMod {
     double q, two_q, qinv, ninv;
 };
 
-constexpr uint64_t kFpPrimeLimit = 1ull << 44;
+constexpr uint64_t kFpPrimeLimit = 1ull << 41;
 
-__device__ __forceinline__ double fp_modmul(double y, double w, const FpMod& m) {
-    const double MAGIC = 6755399441055744.0;  // 1.5 * 2^52
+constexpr double kFpMagic = 6755399441055744.0;  // 1.5 * 2^52
+
+// r = y w (mod q) with |r| < 5q/8, for |y| <= 2^49 and 0 <= w < q
+__device__ __forceinline__ double fp_mulmod_s(double y, double w, const FpMod& m) {
     double ph = __dmul_rn(y, w);
     double pl = __fma_rn(y, w, -ph);
-    double qh = __dsub_rn(__fma_rn(ph, m.qinv, MAGIC), MAGIC);
-    double r = __dadd_rn(__fma_rn(-qh, m.q, ph), pl);
-    return r < 0.0 ? __dadd_rn(r, m.q) : r;
+    double qh = __dsub_rn(__fma_rn(ph, m.qinv, kFpMagic), kFpMagic);
+    return __dadd_rn(__fma_rn(-qh, m.q, ph), pl);
+}
+
+// r = x (mod q) with |r| <= q/2 (1 + 2^-51 |x|/q), for |x| <= 2^51
+__device__ __forceinline__ double fp_reduce_s(double x, const FpMod& m) {
+    double qh = __dsub_rn(__fma_rn(x, m.qinv, kFpMagic), kFpMagic);
+    return __fma_rn(-qh, m.q, x);
+}
+
+// canonical [0, q) from |r| < q
+__device__ __forceinline__ double fp_from_signed(double r, const FpMod& m) { return r < 0.0 ? __dadd_rn(r, m.q) : r; }
+
+// canonical [0, q) from |x| <= 2^51
+__device__ __forceinline__ double fp_canon(double x, const FpMod& m) { return fp_from_signed(fp_reduce_s(x, m), m); }
+
+// canonical product y w mod q, |y| <= 2^49
+__device__ __forceinline__ double fp_modmul(double y, double w, const FpMod& m) {
+    return fp_from_signed(fp_mulmod_s(y, w, m), m);
 }
 
 __device__ __forceinline__ double fp_csub(double x, double c) { return x >= c ? __dsub_rn(x, c) : x; }
 
-// exact conversions for integers below 2^52
+// exact conversions for integers in [0, 2^52)
 __device__ __forceinline__ double u2d(uint64_t x) {
     return __dsub_rn(__longlong_as_double((long long)(x | 0x4330000000000000ull)), 4503599627370496.0);
 }
@@ -144,22 +163,20 @@ __device__ __forceinline__ uint64_t d2u(double d) {
     return (uint64_t)__double_as_longlong(__dadd_rn(d, 4503599627370496.0)) & 0x000FFFFFFFFFFFFFull;
 }
 
-// CT butterfly, values in [0, 4q) -> [0, 4q)
+// CT butterfly on signed values: |x'|, |y'| <= max(|x|) + 5q/8
 __device__ __forceinline__ void bfly_ct(double& x, double& y, double w, const FpMod& m) {
-    double a = fp_csub(x, m.two_q);
-    double t = fp_modmul(y, w, m);
+    double t = fp_mulmod_s(y, w, m);
+    double a = x;
     x = __dadd_rn(a, t);
-    y = __dadd_rn(a, __dsub_rn(m.two_q, t));
+    y = __dsub_rn(a, t);
 }
 
-// GS butterfly, values in [0, 2q) -> [0, 2q)
+// GS butterfly on signed values: |x'| <= |x| + |y|, |y'| < 5q/8
 __device__ __forceinline__ void bfly_gs(double& x, double& y, double w, const FpMod& m) {
     double a = x, b = y;
-    x = fp_csub(__dadd_rn(a, b), m.two_q);
-    y = fp_modmul(__dsub_rn(__dadd_rn(a, m.two_q), b), w, m);
+    x = __dadd_rn(a, b);
+    y = fp_mulmod_s(__dsub_rn(a, b), w, m);
 }
-
-__device__ __forceinline__ double reduce4q(double x, const FpMod& m) { return fp_csub(fp_csub(x, m.two_q), m.q); }
 
 template <int H>
 __device__ __forceinline__ void fwd_stages(double (&x)[16], const double* __restrict__ tw, int s0, int row_term,
@@ -193,13 +210,40 @@ __device__ __forceinline__ void inv_stages(double (&x)[16], const double* __rest
     }
 }
 
+// Last inverse stage, FP64: outputs |r| < 5q/8 (callers canonicalise).
 __device__ __forceinline__ void inv_stage0_scaled(double (&x)[16], double w1, const FpMod& m) {
 #pragma unroll
     for (int k = 0; k < 8; k++) {
         double a = x[k], b = x[k + 8];
-        x[k] = fp_modmul(__dadd_rn(a, b), m.ninv, m);
-        x[k + 8] = fp_modmul(__dsub_rn(__dadd_rn(a, m.two_q), b), w1, m);
+        x[k] = fp_mulmod_s(__dadd_rn(a, b), m.ninv, m);
+        x[k + 8] = fp_mulmod_s(__dsub_rn(a, b), w1, m);
     }
+}
+
+// Element formats.  Transform inputs and outputs are canonical uint64
+// residues; between the two passes of a transform a limb holds the pass's
+// raw state: unreduced uint64 (integer path: [0, 4q) forward, [0, 2q)
+// inverse) or the bit pattern of a signed double (FP64 path).
+__device__ __forceinline__ uint64_t to_elem(uint64_t v, uint64_t) { return v; }
+__device__ __forceinline__ double to_elem(uint64_t v, double) { return u2d(v); }
+__device__ __forceinline__ uint64_t raw_in(uint64_t v, uint64_t) { return v; }
+__device__ __forceinline__ double raw_in(uint64_t v, double) { return __longlong_as_double((long long)v); }
+__device__ __forceinline__ uint64_t raw_out(uint64_t v) { return v; }
+__device__ __forceinline__ uint64_t raw_out(double v) { return (uint64_t)__double_as_longlong(v); }
+
+// Forward outputs: integer path [0, 4q), FP64 path |x| <= 2^49.
+__device__ __forceinline__ uint64_t reduce4q(uint64_t x, uint64_t q) { return csub(csub(x, 2 * q), q); }
+__device__ __forceinline__ uint64_t fwd_canon(uint64_t x, uint64_t q) { return reduce4q(x, q); }
+__device__ __forceinline__ uint64_t fwd_canon(double x, const FpMod& m) { return d2u(fp_canon(x, m)); }
+// Inverse outputs: integer path canonical already, FP64 path |x| < q.
+__device__ __forceinline__ uint64_t inv_canon(uint64_t x, uint64_t) { return x; }
+__device__ __forceinline__ uint64_t inv_canon(double x, const FpMod& m) { return d2u(fp_from_signed(x, m)); }
+// Inverse column pass input: the FP64 row pass leaves |x| <= 2^8 q; bring it
+// to |x| < q/2 + 1 so that seven more doubling stages stay below 2^49.
+__device__ __forceinline__ void inv_cols_prereduce(uint64_t (&)[16], uint64_t) {}
+__device__ __forceinline__ void inv_cols_prereduce(double (&x)[16], const FpMod& m) {
+#pragma unroll
+    for (int k = 0; k < 16; k++) x[k] = fp_reduce_s(x[k], m);
 }
 
 // Last inverse stage (global stage 0, pair distance N/2, block 0): the sum is
@@ -227,11 +271,6 @@ constexpr int NTT_MIN_BLOCKS = 3;
 // shared-memory index of element i of a padded row (one pad word per 16)
 __device__ __forceinline__ int padded(int i) { return i + (i >> 4); }
 
-__device__ __forceinline__ uint64_t to_elem(uint64_t v, uint64_t) { return v; }
-__device__ __forceinline__ double to_elem(uint64_t v, double) { return u2d(v); }
-__device__ __forceinline__ uint64_t from_elem(uint64_t v) { return v; }
-__device__ __forceinline__ uint64_t from_elem(double v) { return d2u(v); }
-
 template <int LOGN>
 __device__ __forceinline__ int row_lane() { return threadIdx.x % (NttCfg<LOGN>::C / 16); }
 
@@ -247,22 +286,22 @@ __device__ __forceinline__ void row_load16(T (&x)[16], const uint64_t* a) {
     }
 }
 
-// a[k] = x[k] reduced from [0, 4q) to [0, q)
+// a[k] = canonical x[k] (forward transform output)
 template <typename T, typename M>
 __device__ __forceinline__ void row_store16(uint64_t* a, T (&x)[16], const M& m) {
     ulonglong2* o = reinterpret_cast<ulonglong2*>(a);
 #pragma unroll
-    for (int k = 0; k < 8; k++)
-        o[k] = make_ulonglong2(from_elem(reduce4q(x[2 * k], m)), from_elem(reduce4q(x[2 * k + 1], m)));
+    for (int k = 0; k < 8; k++) o[k] = make_ulonglong2(fwd_canon(x[2 * k], m), fwd_canon(x[2 * k + 1], m));
 }
 
-// x[k] = row[p + CS k], k < 16 (the forward row pass's input layout)
+// x[k] = row[p + CS k], k < 16: the forward row pass's input, the column
+// pass's raw state
 template <int LOGN, typename T>
 __device__ __forceinline__ void row_load_strided(T (&x)[16], const uint64_t* row) {
     constexpr int CS = NttCfg<LOGN>::C / 16;
     const int p = threadIdx.x % CS;
 #pragma unroll
-    for (int k = 0; k < 16; k++) x[k] = to_elem(row[p + CS * k], T());
+    for (int k = 0; k < 16; k++) x[k] = raw_in(row[p + CS * k], T());
 }
 
 // Forward row pass (stages S1..LOGN-1) on registers loaded from columns
@@ -283,7 +322,7 @@ __device__ __forceinline__ void fwd_rows_core(T (&x)[16], T* sm, int r, const TW
 }
 
 // Inverse row pass (stages LOGN-1..S1) on registers loaded from columns
-// 16 p + k of row r; stores columns p + CS k of the result to out_row.
+// 16 p + k of row r; stores columns p + CS k of the raw result to out_row.
 template <int LOGN, typename T, typename TW, typename M>
 __device__ __forceinline__ void inv_rows_core(T (&x)[16], T* sm, uint64_t* out_row, int r, const TW* tw,
                                               const M& m) {
@@ -299,7 +338,7 @@ __device__ __forceinline__ void inv_rows_core(T (&x)[16], T* sm, uint64_t* out_r
     for (int k = 0; k < 16; k++) x[k] = s[padded(p + CS * k)];
     inv_stages<4>(x, tw, Cf::S1, r, 0, m);
 #pragma unroll
-    for (int k = 0; k < 16; k++) out_row[p + CS * k] = from_elem(x[k]);
+    for (int k = 0; k < 16; k++) out_row[p + CS * k] = raw_out(x[k]);
 }
 
 }  // namespace he
