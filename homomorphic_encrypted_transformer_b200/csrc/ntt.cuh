@@ -178,36 +178,67 @@ __device__ __forceinline__ void bfly_gs(double& x, double& y, double w, const Fp
     y = fp_mulmod_s(__dsub_rn(a, b), w, m);
 }
 
+// The twiddles of stage u used by one thread are contiguous:
+// tw[base(u) + (kofs >> (H - u)) + i], i < 16 >> (H - u) (kofs is a multiple
+// of 16), and the start is a multiple of their count, so they load as
+// 16-byte pairs.  LC = log2 of the count.
+template <int LC>
+__device__ __forceinline__ void load_stage_tw(double (&w)[8], const double* __restrict__ p) {
+    if constexpr (LC == 0) {
+        w[0] = __ldg(p);
+    } else {
+        const double2* p2 = reinterpret_cast<const double2*>(p);
+#pragma unroll
+        for (int v = 0; v < (1 << LC) / 2; v++) {
+            double2 d = __ldg(p2 + v);
+            w[2 * v] = d.x;
+            w[2 * v + 1] = d.y;
+        }
+    }
+}
+
+template <int H, int U>
+__device__ __forceinline__ void fwd_stage_fp(double (&x)[16], const double* __restrict__ tw, int s0, int row_term,
+                                             int kofs, const FpMod& m) {
+    constexpr int D = 1 << (H - 1 - U);
+    double w[8];
+    load_stage_tw<4 - H + U>(w, tw + (1 << (s0 + U)) + (row_term << U) + (kofs >> (H - U)));
+#pragma unroll
+    for (int k = 0; k < 16; k++) {
+        if (k & D) continue;
+        bfly_ct(x[k], x[k + D], w[k >> (H - U)], m);
+    }
+}
+
+template <int H, int U>
+__device__ __forceinline__ void inv_stage_fp(double (&x)[16], const double* __restrict__ tw, int s0, int row_term,
+                                             int kofs, const FpMod& m) {
+    constexpr int D = 1 << (H - 1 - U);
+    double w[8];
+    load_stage_tw<4 - H + U>(w, tw + (1 << (s0 + U)) + (row_term << U) + (kofs >> (H - U)));
+#pragma unroll
+    for (int k = 0; k < 16; k++) {
+        if (k & D) continue;
+        bfly_gs(x[k], x[k + D], w[k >> (H - U)], m);
+    }
+}
+
 template <int H>
 __device__ __forceinline__ void fwd_stages(double (&x)[16], const double* __restrict__ tw, int s0, int row_term,
                                            int kofs, const FpMod& m) {
-#pragma unroll
-    for (int u = 0; u < H; u++) {
-        const int D = 1 << (H - 1 - u);
-        const int base = (1 << (s0 + u)) + (row_term << u);
-#pragma unroll
-        for (int k = 0; k < 16; k++) {
-            if (k & D) continue;
-            double w = __ldg(tw + base + ((kofs + k) >> (H - u)));
-            bfly_ct(x[k], x[k + D], w, m);
-        }
-    }
+    if constexpr (H > 0) fwd_stage_fp<H, 0>(x, tw, s0, row_term, kofs, m);
+    if constexpr (H > 1) fwd_stage_fp<H, 1>(x, tw, s0, row_term, kofs, m);
+    if constexpr (H > 2) fwd_stage_fp<H, 2>(x, tw, s0, row_term, kofs, m);
+    if constexpr (H > 3) fwd_stage_fp<H, 3>(x, tw, s0, row_term, kofs, m);
 }
 
 template <int H, int ULO = 0>
 __device__ __forceinline__ void inv_stages(double (&x)[16], const double* __restrict__ tw, int s0, int row_term,
                                            int kofs, const FpMod& m) {
-#pragma unroll
-    for (int u = H - 1; u >= ULO; u--) {
-        const int D = 1 << (H - 1 - u);
-        const int base = (1 << (s0 + u)) + (row_term << u);
-#pragma unroll
-        for (int k = 0; k < 16; k++) {
-            if (k & D) continue;
-            double w = __ldg(tw + base + ((kofs + k) >> (H - u)));
-            bfly_gs(x[k], x[k + D], w, m);
-        }
-    }
+    if constexpr (H > 3 && ULO <= 3) inv_stage_fp<H, 3>(x, tw, s0, row_term, kofs, m);
+    if constexpr (H > 2 && ULO <= 2) inv_stage_fp<H, 2>(x, tw, s0, row_term, kofs, m);
+    if constexpr (H > 1 && ULO <= 1) inv_stage_fp<H, 1>(x, tw, s0, row_term, kofs, m);
+    if constexpr (H > 0 && ULO <= 0) inv_stage_fp<H, 0>(x, tw, s0, row_term, kofs, m);
 }
 
 // Last inverse stage, FP64: outputs |r| < 5q/8 (callers canonicalise).

@@ -72,3 +72,33 @@ def test_ntt_bad_arguments_rejected():
     with pytest.raises(he.HEError) as ei:
         he.he_ntt_fwd(st.ctx, d, 1, 5, 0)
     assert ei.value.code == he.HE_EINVAL
+
+
+@pytest.mark.parametrize("q_bits", [41, 42, 30])
+def test_ntt_prime_size_edges(q_bits):
+    """The FP64 butterflies serve primes below 2^41: the largest such primes
+    (the bound analysis at its limit), 42-bit primes (integer path) and small
+    primes, forward and inverse, bit-exact."""
+    he = lib()
+    log_n, L, K = 16, 3, 1
+    P = C.Params(log_n, L, K, 3, q_bits=q_bits)
+    ctx = he.he_ctx_create(log_n, L, K, 3, q_bits=q_bits)
+    assert ctx.primes == P.mods
+    mods = P.mods
+    a = random_rows(31 + q_bits, mods, 2, P.N)
+    for r, q in enumerate(mods):  # extremes in the first polynomial
+        a[0, r, :16] = q - 1
+        a[0, r, 16:32] = 0
+    d = dev(a)
+    he.he_ntt_fwd(ctx, d, 2, len(mods), 0)
+    he.he_sync(ctx)
+    got = host(d, a.shape)
+    for i in range(2):
+        assert np.array_equal(got[i], C.ntt_rows(a[i], mods, P))
+    d2 = dev(a)
+    he.he_ntt_inv(ctx, d2, 2, len(mods), 0)
+    he.he_sync(ctx)
+    got = host(d2, a.shape)
+    for i in range(2):
+        assert np.array_equal(got[i], C.intt_rows(a[i], mods, P))
+    he.he_ctx_destroy(ctx)
