@@ -41,7 +41,7 @@ WORKLOAD = {"workload": "rotation batch: 64 fresh ciphertexts, 16 seeded rotatio
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -295,6 +295,14 @@ def run_native(args, rank, world, local_rank):
         torch.cuda.synchronize()
         best = min(best, ev0.elapsed_time(ev1))
     int_modmul_s = he.he_probe_int_threads(ctx) * iters * he.he_probe_int_mults_per_iter() / (best * 1e-3)
+    best = 1e9
+    for _ in range(3):
+        ev0.record(stream)
+        he.he_probe_fp(ctx, iters, sink)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        best = min(best, ev0.elapsed_time(ev1))
+    fp_modmul_s = he.he_probe_int_threads(ctx) * iters * he.he_probe_int_mults_per_iter() / (best * 1e-3)
 
     # timed region
     clocks = ClockSampler(local_rank)
@@ -311,9 +319,8 @@ def run_native(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     ms = t0.elapsed_time(t1)
-    clk = clocks.stop()
     launches = he.he_launch_count(ctx)
-    prof = {name: he.he_profile_read(ctx, cls) for name, cls in he.PROF.items()}
+    prof = {name: he.he_profile_read(ctx, cls) + (he.he_profile_read_fp(ctx, cls),) for name, cls in he.PROF.items()}
     he.he_profile_enable(ctx, False)
 
     # same step without profiling events (the headline number)
@@ -326,6 +333,7 @@ def run_native(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     ms_plain = t0.elapsed_time(t1)
+    clk = clocks.stop()
 
     if world > 1:
         tt = torch.tensor([ms_plain, ms], device=dev)
@@ -360,16 +368,20 @@ def run_native(args, rank, world, local_rank):
     # algorithmic bytes of one rotation batch (keys read once per key group)
     batch_bytes = N_KEYS * key_bytes + N_CTS * 2 * ct_bytes
     hbm_frac_step = (batch_bytes / (ms_plain * 1e-3 / args.steps)) / 1e9 / hbm_peak
-    roof = roofline_for(dom_name, prof[dom_name], int_modmul_s, hbm_peak, pk_kind)
+    roof = roofline_for(dom_name, prof[dom_name], int_modmul_s, fp_modmul_s, hbm_peak, pk_kind)
     line = {"metric": METRIC, "value": value, "unit": "rotations/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_plain / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u64", "data": "synthetic",
             "config": dict(WORKLOAD, parallelism="replicas%d" % world if world > 1 else "single"),
             "hbm_roofline_frac_of_step": hbm_frac_step,
             "roofline": roof,
-            "probes": {"copy_gbs": copy_gbs, "int_shoup_modmul_per_s": int_modmul_s},
+            "probes": {"copy_gbs": copy_gbs, "int_shoup_modmul_per_s": int_modmul_s,
+                       "fp64_modmul_per_s": fp_modmul_s},
             "kernel_ms_per_step": {k: round(v[0] / args.steps, 4) for k, v in prof.items() if v[1]},
             "kernel_launches_per_step": {k: v[1] / args.steps for k, v in prof.items() if v[1]},
+            "kernel_roofline_frac": {k: round(roofline_for(k, v, int_modmul_s, fp_modmul_s, hbm_peak,
+                                                           pk_kind)["frac"], 3)
+                                     for k, v in prof.items() if v[1]},
             "profiled_ms_per_step": ms / args.steps,
             "gpu_launches": launches,
             "clocks": clk,
@@ -380,25 +392,27 @@ def run_native(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
-# ncu dram bytes (read + write) over algorithmic bytes, per kernel, from the
-# committed captures in profiles/ (a 512-limb launch; the benchmark's launches
-# process 288 limbs on average, so the traffic is scaled by limbs processed).
-# Remove an entry when its kernel changes.
-NCU_TRAFFIC_RATIO = {"ntt_fwd_cols": 489.0 / 536.9, "ntt_fwd_rows": 595.8 / 536.9, "ntt_inv_rows": 625.4 / 536.9,
-                     "ntt_inv_cols": 488.6 / 536.9}
+# ncu dram bytes (read + write) over algorithmic bytes, per kernel class, from
+# the committed capture in profiles/ (rotation of 8 ciphertexts at level 24;
+# the ratio carries over to the benchmark's launches, which move the same
+# rows per ciphertext).  Remove an entry when its kernel changes.
+NCU_TRAFFIC_RATIO = {}
 
 
-def roofline_for(name, prof_entry, int_modmul_s, hbm_peak, pk_kind):
+def roofline_for(name, prof_entry, int_modmul_s, fp_modmul_s, hbm_peak, pk_kind):
     """Roofline of the dominant kernel class: its algorithmic bytes and
     modular multiplications per launch (counted by the library as it
-    launches) against its CUDA-event duration.  The binding resource is the
-    one whose peak gives the longer ideal time."""
-    ms, launches, nbytes, mults = prof_entry
+    launches, split between the integer and the FP64 pipe) against its
+    CUDA-event duration.  The ALU ceiling of the class is the time its
+    products take at the two probes' rates (integer products at the integer
+    probe's rate, FP64 products at the FP64 probe's); the binding resource is
+    the one whose ideal time is longer."""
+    ms, launches, nbytes, mults, mults_fp = prof_entry
     launches = max(1, launches)
     t = ms * 1e-3 / launches
-    b, m = nbytes / launches, mults / launches
+    b, m, m_fp = nbytes / launches, mults / launches, mults_fp / launches
     t_hbm = b / (hbm_peak * 1e9)
-    t_alu = m / int_modmul_s if int_modmul_s > 0 else 0.0
+    t_alu = (m - m_fp) / int_modmul_s + (m_fp / fp_modmul_s if fp_modmul_s > 0 else 0.0)
     traffic = NCU_TRAFFIC_RATIO[name] * b if name in NCU_TRAFFIC_RATIO else None
     if t_hbm >= t_alu:
         ach = b / t / 1e9
@@ -406,11 +420,15 @@ def roofline_for(name, prof_entry, int_modmul_s, hbm_peak, pk_kind):
                 "frac": ach / hbm_peak, "traffic": traffic, "algorithmic_bytes_per_launch": b,
                 "ms_per_launch": t * 1e3, "peak_source": pk_kind + " (MEASURED_PEAKS.json hbm_gbs)"}
     ach = m / t / 1e9
-    peak = int_modmul_s / 1e9
+    peak = m / t_alu / 1e9
     return {"kernel": name, "bound": "alu", "achieved": ach, "peak": peak, "unit": "Gmodmul/s",
             "frac": ach / peak, "traffic": traffic, "algorithmic_modmuls_per_launch": m,
+            "fp64_share": m_fp / m if m else 0.0,
             "algorithmic_bytes_per_launch": b, "ms_per_launch": t * 1e3,
-            "peak_source": "in-run probe: register-only 64-bit Shoup modular products, full grid"}
+            "hbm_frac": (b / t / 1e9) / hbm_peak,
+            "peak_source": "in-run probes (register-only modular products over a full grid): integer Shoup "
+                           "%.0f G/s, FP64 rounded-quotient %.0f G/s, weighted by this class's mix"
+                           % (int_modmul_s / 1e9, fp_modmul_s / 1e9)}
 
 
 def main():

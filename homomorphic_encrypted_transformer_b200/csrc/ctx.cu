@@ -188,17 +188,18 @@ void prof_begin(he_ctx* c, int cls) {
     p.cls = cls;
     p.a = ev_get(c);
     p.b = nullptr;
-    p.bytes = p.mults = 0;
+    p.bytes = p.mults = p.mults_fp = 0;
     cudaEventRecord(p.a, c->stream);
     c->prof_pending.push_back(p);
 }
 
-int prof_end(he_ctx* c, int cls, double bytes, double mults) {
+int prof_end(he_ctx* c, int cls, double bytes, double mults, double mults_fp) {
     if (!c->prof_on || c->prof_pending.empty()) return HE_OK;
     ProfPending& p = c->prof_pending.back();
     if (p.cls != cls || p.b) return HE_OK;
     p.bytes = bytes;
     p.mults = mults;
+    p.mults_fp = mults_fp;
     p.b = ev_get(c);
     cudaEventRecord(p.b, c->stream);
     return HE_OK;
@@ -215,12 +216,26 @@ static int prof_collect(he_ctx* c) {
             c->prof[p.cls].launches += 1;
             c->prof[p.cls].bytes += p.bytes;
             c->prof[p.cls].mults += p.mults;
+            c->prof[p.cls].mults_fp += p.mults_fp;
             c->ev_pool.push_back(p.b);
         }
         c->ev_pool.push_back(p.a);
     }
     c->prof_pending.clear();
     return HE_OK;
+}
+
+bool fp_prime(const he_ctx* c, int prime_idx) { return c->primes[prime_idx] < kFpPrimeLimit; }
+
+long long fp_rows(const he_ctx* c, const RowSet& rs, int n_rows) {
+    long long per = 0, tail = 0;
+    const int rem = n_rows % rs.per_group;
+    for (int r = 0; r < rs.per_group; r++) {
+        int f = fp_prime(c, rs.prime(r));
+        per += f;
+        if (r < rem) tail += f;
+    }
+    return (long long)(n_rows / rs.per_group) * per + tail;
 }
 
 uint64_t galois_elt(const he_ctx* c, int32_t step) {
@@ -565,6 +580,14 @@ extern "C" int he_profile_read(he_ctx* c, int cls, double* ms, long long* launch
     if (launches) *launches = c->prof[cls].launches;
     if (bytes) *bytes = c->prof[cls].bytes;
     if (mults) *mults = c->prof[cls].mults;
+    return HE_OK;
+}
+
+extern "C" int he_profile_read_fp(he_ctx* c, int cls, double* fp_mults) {
+    if (!c || cls < 0 || cls >= HE_PROF_N) return HE_EINVAL;
+    int rc = prof_collect(c);
+    if (rc) return rc;
+    if (fp_mults) *fp_mults = c->prof[cls].mults_fp;
     return HE_OK;
 }
 

@@ -30,19 +30,21 @@ struct ConvTable {
 struct FpMod;  // FP64 constants of a prime below 2^41 (ntt.cuh)
 
 struct Key {
-    uint64_t* d = nullptr;  // [digits][2][L+K][N] in Montgomery form (value * 2^64 mod p)
+    // [digits][2][L+K][N]: rows of primes below 2^41 as doubles, the others in
+    // Montgomery form (value * 2^64 mod p)
+    uint64_t* d = nullptr;
 };
 
 struct ProfSlot {
     double ms = 0;
     long long launches = 0;
-    double bytes = 0, mults = 0;
+    double bytes = 0, mults = 0, mults_fp = 0;
 };
 
 struct ProfPending {
     int cls;
     cudaEvent_t a, b;
-    double bytes, mults;
+    double bytes, mults, mults_fp;
 };
 
 }  // namespace he
@@ -95,9 +97,14 @@ int set_err(he_ctx* c, int code, const char* fmt, ...);
 int check_cuda(he_ctx* c, cudaError_t e, const char* what);
 
 // Brackets launches of one class with events; prof_end records the
-// algorithmic work (HBM bytes, modular multiplications) of what it closes.
+// algorithmic work of what it closes: HBM bytes, modular multiplications,
+// and how many of those run on the FP64 pipe (primes below 2^41).
 void prof_begin(he_ctx* c, int cls);
-int prof_end(he_ctx* c, int cls, double bytes = 0, double mults = 0);
+int prof_end(he_ctx* c, int cls, double bytes = 0, double mults = 0, double mults_fp = 0);
+
+// Rows 0..n_rows-1 of a RowSet whose prime takes the FP64 path.
+long long fp_rows(const he_ctx* c, const RowSet& rs, int n_rows);
+bool fp_prime(const he_ctx* c, int prime_idx);
 
 uint64_t galois_elt(const he_ctx* c, int32_t step);
 

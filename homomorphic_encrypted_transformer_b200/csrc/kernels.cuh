@@ -19,7 +19,7 @@ struct RowSet {
     int per_group;
     int first0, len0, first1, len1, first2;
 
-    __device__ __forceinline__ int prime(int r) const {
+    __host__ __device__ __forceinline__ int prime(int r) const {
         int rr = r % per_group;
         if (rr < len0) return first0 + rr;
         rr -= len0;

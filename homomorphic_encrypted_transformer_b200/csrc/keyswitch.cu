@@ -155,41 +155,69 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// u[i][0/1][t][c] = sum_j x_j[t][c] * key_i,j[b/a][row(t)][c]   (keys in Montgomery form),
+// u[i][0/1][t][c] = sum_j x_j[t][c] * key_i,j[b/a][row(t)][c],
 // x_j = sigma_{g_i}(d_i) on digit j's own rows (read through the
 // automorphism: an aligned group of 32 indices maps onto one, so a warp's
-// loads stay within the same 256 bytes), ext_j elsewhere.
+// loads stay within the same 256 bytes), ext_j elsewhere.  Rows of primes
+// below 2^41 (key stored as doubles) sum signed FP64 products, the others
+// accumulate 128-bit products of the Montgomery-form key and reduce once.
 // The ciphertext index is the fastest grid dimension: neighbouring blocks
 // that share a key read the same key tile, which DRAM then serves once.
-__global__ void k_ks_inner(const uint64_t* __restrict__ ext, PtrList din, GalList gal, PtrList keys,
-                           uint64_t* __restrict__ u, int n_digits, int n_rows, int level, int L, int LK, int n_cts,
-                           const DevPrime* __restrict__ pr, ModupArgs a, int logn) {
+// ND = number of digits (compile time, so that every load of a thread is in
+// flight at once).
+template <int ND>
+__global__ void __launch_bounds__(256)
+    k_ks_inner(const uint64_t* __restrict__ ext, PtrList din, GalList gal, PtrList keys, uint64_t* __restrict__ u,
+               int n_rows, int level, int L, int LK, int n_cts, const DevPrime* __restrict__ pr,
+               const FpMod* __restrict__ fpm, ModupArgs a, int logn) {
     const int N = 1 << logn;
     int i = blockIdx.x, t = blockIdx.z;
     int c = blockIdx.y * blockDim.x + threadIdx.x;
     if (c >= N) return;
     const uint64_t* key = keys.p[i];
     const int own = automorph_src(c, logn, gal.g[i]);
-    int krow = t < level ? t : L + (t - level);
-    DevPrime p = pr[a.tprime[t]];
-    U128 acc0 = {0, 0}, acc1 = {0, 0};
-    for (int j = 0; j < n_digits; j++) {
+    const int krow = t < level ? t : L + (t - level);
+    const int pidx = a.tprime[t];
+    const DevPrime p = pr[pidx];
+    const bool fp = p.q < kFpPrimeLimit;
+    uint64_t xs[ND], kbs[ND], kas[ND];
+#pragma unroll
+    for (int j = 0; j < ND; j++) {
         const int s0 = a.src_row[j], ns = a.n_src[j];
-        uint64_t x;
         if (t >= s0 && t < s0 + ns) {
-            x = __ldg(din.p[i] + (size_t)t * N + own);
+            xs[j] = __ldg(din.p[i] + (size_t)t * N + own);
         } else {
             int pos = t < s0 ? t : t - ns;
-            x = ext[((size_t)a.ext_off[j] * n_cts + (size_t)i * (n_rows - ns) + pos) * N + c];
+            xs[j] = ext[((size_t)a.ext_off[j] * n_cts + (size_t)i * (n_rows - ns) + pos) * N + c];
         }
-        const uint64_t* kb = key + (((size_t)j * 2 + 0) * LK + krow) * N;
-        const uint64_t* ka = key + (((size_t)j * 2 + 1) * LK + krow) * N;
-        mac128(acc0, x, kb[c]);
-        mac128(acc1, x, ka[c]);
+        kbs[j] = key[(((size_t)j * 2 + 0) * LK + krow) * N + c];
+        kas[j] = key[(((size_t)j * 2 + 1) * LK + krow) * N + c];
+    }
+    U128 acc0 = {0, 0}, acc1 = {0, 0};
+    double f0 = 0.0, f1 = 0.0;
+    const FpMod m = fpm[pidx];
+    if (fp) {
+#pragma unroll
+        for (int j = 0; j < ND; j++) {
+            const double xd = u2d(xs[j]);
+            f0 = __dadd_rn(f0, fp_mulmod_s(xd, __longlong_as_double((long long)kbs[j]), m));
+            f1 = __dadd_rn(f1, fp_mulmod_s(xd, __longlong_as_double((long long)kas[j]), m));
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < ND; j++) {
+            mac128(acc0, xs[j], kbs[j]);
+            mac128(acc1, xs[j], kas[j]);
+        }
     }
     uint64_t* o = u + ((size_t)i * 2 * n_rows) * N + c;
-    o[(size_t)t * N] = csub(redc_lazy(acc0.hi, acc0.lo, p.q, p.qinv_neg), p.q);
-    o[(size_t)(n_rows + t) * N] = csub(redc_lazy(acc1.hi, acc1.lo, p.q, p.qinv_neg), p.q);
+    if (fp) {
+        o[(size_t)t * N] = d2u(fp_canon(f0, m));
+        o[(size_t)(n_rows + t) * N] = d2u(fp_canon(f1, m));
+    } else {
+        o[(size_t)t * N] = csub(redc_lazy(acc0.hi, acc0.lo, p.q, p.qinv_neg), p.q);
+        o[(size_t)(n_rows + t) * N] = csub(redc_lazy(acc1.hi, acc1.lo, p.q, p.qinv_neg), p.q);
+    }
 }
 
 // tmp[i][poly][r][c] = sum_k y'_k (P/p_k mod q_r), y_k = [x_k (P/p_k)^-1]_{p_k},
@@ -400,6 +428,9 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     const NttShape sh = ntt_shape(c->log_n);
     int sum_src = 0;
     for (int j = 0; j < nd; j++) sum_src += ma.n_src[j];
+    std::vector<int> ep = ext_primes(c, level);
+    int fp_q = 0;  // primes of Q_level on the FP64 path
+    for (int t = 0; t < level; t++) fp_q += fp_prime(c, t);
 
     // sigma(d) back to coefficients: gathered row pass, then the column pass
     prof_begin(c, HE_PROF_NTT_INV_ROWS);
@@ -407,7 +438,8 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     HE_LOGN_SWITCH(c, HE_IRG)
 #undef HE_IRG
     if ((rc = lc(c, "inv_rows_gather"))) return rc;
-    prof_end(c, HE_PROF_NTT_INV_ROWS, 2.0 * n * level * limbB, 0.5 * N * n * level * sh.s2);
+    prof_end(c, HE_PROF_NTT_INV_ROWS, 2.0 * n * level * limbB, 0.5 * N * n * level * sh.s2,
+             0.5 * N * n * fp_q * sh.s2);
     std::vector<int> qp = prime_range(0, level);
     if ((rc = ntt_inv_cols_set(c, rowset_contig(coef, level, N, qp), n * level))) return rc;
 
@@ -431,12 +463,16 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
         if ((rc = lc(c, "modup_conv"))) return rc;
     }
     {
-        double prods = 0;
-        for (int j = 0; j < nd; j++) prods += (double)ma.n_src[j] * (1 + n_rows - ma.n_src[j]);
-        prof_end(c, HE_PROF_MODUP, (double)n * (sum_src + ext_rows) * limbB, (double)n * N * prods);
+        double prods = 0, prods_fp = 0;
+        for (int j = 0; j < nd; j++) {
+            prods += (double)ma.n_src[j] * (1 + n_rows - ma.n_src[j]);
+            for (int t = 0; t < n_rows; t++)
+                if ((t < ma.src_row[j] || t >= ma.src_row[j] + ma.n_src[j]) && fp_prime(c, ep[t]))
+                    prods_fp += ma.n_src[j];
+        }
+        prof_end(c, HE_PROF_MODUP, (double)n * (sum_src + ext_rows) * limbB, (double)n * N * prods,
+                 (double)n * N * prods_fp);
     }
-
-    std::vector<int> ep = ext_primes(c, level);
     for (int j = 0; j < nd; j++) {
         std::vector<int> tp;
         for (int t = 0; t < n_rows; t++)
@@ -447,11 +483,26 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     }
 
     prof_begin(c, HE_PROF_KS_INNER);
-    k_ks_inner<<<dim3(n, gx, n_rows), blk, 0, c->stream>>>(ext, din, gal, keys, u, nd, n_rows, level, L, LK, n,
-                                                           c->d_prime, ma, c->log_n);
+    switch (nd) {
+#define HE_KS_CASE(D)                                                                                             \
+    case D:                                                                                                       \
+        k_ks_inner<D><<<dim3(n, gx, n_rows), blk, 0, c->stream>>>(ext, din, gal, keys, u, n_rows, level, L, LK, n, \
+                                                                  c->d_prime, c->d_fpmod, ma, c->log_n);         \
+        break;
+        HE_KS_CASE(1) HE_KS_CASE(2) HE_KS_CASE(3) HE_KS_CASE(4) HE_KS_CASE(5) HE_KS_CASE(6) HE_KS_CASE(7)
+        HE_KS_CASE(8) HE_KS_CASE(9) HE_KS_CASE(10) HE_KS_CASE(11) HE_KS_CASE(12) HE_KS_CASE(13) HE_KS_CASE(14)
+        HE_KS_CASE(15)
+#undef HE_KS_CASE
+        default:
+            return set_err(c, HE_EINVAL, "key switch: %d digits unsupported", nd);
+    }
     if ((rc = lc(c, "ks_inner"))) return rc;
-    prof_end(c, HE_PROF_KS_INNER, ((double)n * nd * n_rows + 2.0 * nd * n_rows + 2.0 * n * n_rows) * limbB,
-             (double)n * n_rows * N * (2.0 * nd + 2));
+    {
+        int fp_rows_ks = 0;
+        for (int t = 0; t < n_rows; t++) fp_rows_ks += fp_prime(c, ep[t]);
+        prof_end(c, HE_PROF_KS_INNER, ((double)n * nd * n_rows + 2.0 * nd * n_rows + 2.0 * n * n_rows) * limbB,
+                 (double)n * n_rows * N * 2.0 * nd, (double)n * fp_rows_ks * N * 2.0 * nd);
+    }
 
     std::vector<int> pp = prime_range(L, K);
     RowSet prs = rowset(u + (size_t)level * N, (long long)n_rows * N, K, pp.data());
@@ -486,7 +537,7 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
         int n_add = 0;
         for (int i = 0; i < n; i++) n_add += (io.add0[i] != nullptr) + (io.add1[i] != nullptr);
         prof_end(c, HE_PROF_MODDOWN_COMBINE, (6.0 * n + n_add) * level * limbB,
-                 2.0 * n * level * N * (1.0 + 0.5 * sh.s2));
+                 2.0 * n * level * N * (1.0 + 0.5 * sh.s2), 2.0 * n * fp_q * N * 0.5 * sh.s2);
     }
     return HE_OK;
 }

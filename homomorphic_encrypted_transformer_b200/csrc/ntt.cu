@@ -215,7 +215,8 @@ static int ntt_pass(he_ctx* c, const RowSet& rs, int n_rows, bool fwd, int which
     int rc = launch_check(c, fwd ? "ntt_fwd" : "ntt_inv");
     if (rc) return rc;
     c->launches += 1;
-    return prof_end(c, cls, bytes, half * (col_pass ? sh.s1 : sh.s2));
+    const int stages = col_pass ? sh.s1 : sh.s2;
+    return prof_end(c, cls, bytes, half * stages, 0.5 * c->N * fp_rows(c, rs, n_rows) * stages);
 }
 
 int ntt_fwd_set(he_ctx* c, const RowSet& rs, int n_rows) {

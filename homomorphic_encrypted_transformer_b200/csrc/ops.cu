@@ -5,6 +5,7 @@
 #include <algorithm>
 
 #include "he_internal.h"
+#include "ntt.cuh"
 
 namespace he {
 
@@ -54,7 +55,12 @@ __global__ void k_mul_rows(const uint64_t* __restrict__ a, const uint64_t* __res
 
 // One digit of a switching key, rows = all L+K primes:
 //   b = -a s + e + gmod(r) s'  (gmod = P mod q_r on the digit's rows, else 0)
-// stored in Montgomery form (x 2^64 mod prime).
+// stored in the form the inner product consumes: rows of primes below 2^41
+// as doubles (FP64 products), the others in Montgomery form (x 2^64 mod prime).
+__device__ __forceinline__ uint64_t key_store_form(uint64_t v, const DevPrime& p) {
+    return p.q < kFpPrimeLimit ? (uint64_t)__double_as_longlong((double)v) : mont_mul(v, p.r2, p);
+}
+
 __global__ void k_keygen_digit(const uint64_t* __restrict__ a, const uint64_t* __restrict__ s,
                                const uint64_t* __restrict__ e, const uint64_t* __restrict__ sp, RowConst g,
                                uint64_t* __restrict__ kb, uint64_t* __restrict__ ka, const DevPrime* __restrict__ pr,
@@ -68,18 +74,19 @@ __global__ void k_keygen_digit(const uint64_t* __restrict__ a, const uint64_t* _
     uint64_t as = mul_mod(av, s[k], p);
     uint64_t b = sub_mod(e[k], as, p.q);
     if (g.v[r].x) b = add_mod(b, mul_shoup(sp[k], g.v[r].x, g.v[r].y, p.q), p.q);
-    kb[k] = mont_mul(b, p.r2, p);
-    ka[k] = mont_mul(av, p.r2, p);
+    kb[k] = key_store_form(b, p);
+    ka[k] = key_store_form(av, p);
 }
 
-__global__ void k_from_mont(const uint64_t* __restrict__ in, uint64_t* __restrict__ out, int rows_per_poly,
-                            const DevPrime* __restrict__ pr, int logn) {
+// canonical residues of a stored key
+__global__ void k_key_canonical(const uint64_t* __restrict__ in, uint64_t* __restrict__ out, int rows_per_poly,
+                                const DevPrime* __restrict__ pr, int logn) {
     const int N = 1 << logn;
     int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y;
     if (c >= N) return;
     DevPrime p = pr[r % rows_per_poly];
     size_t k = (size_t)r * N + c;
-    out[k] = mont_mul(in[k], 1, p);
+    out[k] = p.q < kFpPrimeLimit ? (uint64_t)__longlong_as_double((long long)in[k]) : mont_mul(in[k], 1, p);
 }
 
 // d[i] = (a0 b0, a0 b1 + a1 b0, a1 b1), each [level][N]
@@ -420,7 +427,8 @@ extern "C" int he_key_download(he_ctx* c, int kind, int32_t step, uint64_t* host
     uint64_t* tmp;
     int rc = scratch_slot(c, 2, words, &tmp);
     if (rc) return rc;
-    k_from_mont<<<dim3((N + TB - 1) / TB, nd * 2 * LK), TB, 0, c->stream>>>(k->d, tmp, LK, c->d_prime, c->log_n);
+    k_key_canonical<<<dim3((N + TB - 1) / TB, nd * 2 * LK), TB, 0, c->stream>>>(k->d, tmp, LK, c->d_prime,
+                                                                            c->log_n);
     if ((rc = lc(c, "key download"))) return rc;
     rc = check_cuda(c, cudaMemcpyAsync(host_out, tmp, words * 8, cudaMemcpyDeviceToHost, c->stream), "key D2H");
     if (rc) return rc;

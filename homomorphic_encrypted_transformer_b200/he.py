@@ -95,9 +95,11 @@ _sig("he_poly_eval_ps15", _i, _vp, ctypes.POINTER(he_ct), _i, _vp, ctypes.c_doub
 _sig("he_profile_enable", _i, _vp, _i)
 _sig("he_profile_read", _i, _vp, _i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong),
      ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double))
+_sig("he_profile_read_fp", _i, _vp, _i, ctypes.POINTER(ctypes.c_double))
 _sig("he_launch_count", ctypes.c_longlong, _vp, _i)
 _sig("he_probe_copy", _i, _vp, _vp, _vp, ctypes.c_size_t)
 _sig("he_probe_int", _i, _vp, _i, _vp)
+_sig("he_probe_fp", _i, _vp, _i, _vp)
 _sig("he_probe_int_threads", ctypes.c_longlong, _vp)
 _sig("he_probe_int_mults_per_iter", _i)
 
@@ -349,6 +351,13 @@ def he_profile_read(ctx, cls):
     return ms.value, n.value, b.value, m.value
 
 
+def he_profile_read_fp(ctx, cls):
+    """Modular multiplications of one class that ran on the FP64 pipe."""
+    m = ctypes.c_double()
+    _check(ctx, _lib.he_profile_read_fp(ctx.ptr, cls, ctypes.byref(m)))
+    return m.value
+
+
 def he_launch_count(ctx, reset=False):
     return int(_lib.he_launch_count(ctx.ptr, 1 if reset else 0))
 
@@ -359,6 +368,10 @@ def he_probe_copy(ctx, dst, src, n_words):
 
 def he_probe_int(ctx, iters, sink):
     _check(ctx, _lib.he_probe_int(ctx.ptr, iters, _ptr(sink)))
+
+
+def he_probe_fp(ctx, iters, sink):
+    _check(ctx, _lib.he_probe_fp(ctx.ptr, iters, _ptr(sink)))
 
 
 def he_probe_int_threads(ctx):

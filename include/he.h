@@ -253,6 +253,10 @@ int he_profile_enable(he_ctx* ctx, int enable);
  * Any output pointer may be NULL. */
 int he_profile_read(he_ctx* ctx, int cls, double* total_ms, long long* launches, double* bytes,
                     double* modmuls);
+/* Of the modular multiplications he_profile_read reports for a class, those
+ * that ran on the FP64 pipe (residues of primes below 2^41); the rest ran on
+ * the integer pipe. */
+int he_profile_read_fp(he_ctx* ctx, int cls, double* fp_modmuls);
 /* Kernels this context has launched since creation or the last reset. */
 long long he_launch_count(he_ctx* ctx, int reset);
 
@@ -267,6 +271,11 @@ int he_probe_int(he_ctx* ctx, int iters, uint64_t* sink);
 long long he_probe_int_threads(he_ctx* ctx);
 /* 64-bit modular multiplications one he_probe_int thread performs per iteration. */
 int he_probe_int_mults_per_iter(void);
+/* FP64 probe: as he_probe_int, with the FP64 rounded-quotient modular product
+ * (the NTT's and the conversions' arithmetic for primes below 2^41) modulo
+ * the context's largest such prime; same grid, same products per iteration.
+ * HE_EINVAL when the context has no prime below 2^41.  Asynchronous. */
+int he_probe_fp(he_ctx* ctx, int iters, uint64_t* sink);
 
 #ifdef __cplusplus
 }
