@@ -221,26 +221,46 @@ __global__ void __launch_bounds__(256)
 }
 
 // tmp[i][poly][r][c] = sum_k y'_k (P/p_k mod q_r), y_k = [x_k (P/p_k)^-1]_{p_k},
-// y'_k = y_k or y_k - p_k (centred).  Since p_k (P/p_k) = P for every k, the
-// centring subtracts (number of negative terms) * P; the sum of the y_k
-// products is accumulated in 128 bits and reduced once per target.
+// y'_k = y_k or y_k - p_k (centred, |y'_k| < 2^59).  Two arithmetic paths:
+//  - FP64 (targets below 2^41): with y'_k = a_k 2^40 + b_k 2^20 + c_k
+//    (|a_k| < 2^19; b_k, c_k < 2^20) and m_kr = P/p_k mod q_r = h 2^21 + l
+//    (h < 2^20, l < 2^21), every partial product is below 2^41 in magnitude,
+//    so the six sums over k (KP <= 16 terms) are exact doubles below 2^45:
+//      S = T_cl + 2^20 (T_bl + 2 T_ch) + 2^40 (T_al + 2 T_bh) + 2^61 T_ah,
+//    and three rounded-quotient products by 2^20, 2^40, 2^61 mod q_r and one
+//    reduction give S mod q_r.
+//  - integer (the 60-bit q_0): since p_k (P/p_k) = P for every k, the centring
+//    subtracts (number of negative terms) * P; the sum of the y_k products is
+//    accumulated in 128 bits and reduced once.
 template <int KP>
 __global__ void __launch_bounds__(256)
     k_moddown_conv(const uint64_t* __restrict__ u, uint64_t* __restrict__ tmp, int level, int L,
-                   const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ pcoef,
+                   const DevPrime* __restrict__ pr, const FpMod* __restrict__ fpm, const ulonglong2* __restrict__ pcoef,
                    const ulonglong2* __restrict__ mat, const uint64_t* __restrict__ negP, int logn) {
     __shared__ uint64_t sm_m[KP * kConvMaxTargets];
+    __shared__ double2 sm_hl[KP * kConvMaxTargets];  // {h, l} of m_kr
     __shared__ ConvTarget sm_t[kConvMaxTargets];
+    __shared__ FpMod sm_f[kConvMaxTargets];
+    __shared__ double4 sm_pow[kConvMaxTargets];  // {2^20, 2^40, 2^61} mod q_r
     __shared__ uint64_t sm_neg[kConvMaxTargets];
     const int N = 1 << logn;
     for (int idx = threadIdx.x; idx < KP * level; idx += blockDim.x) {
         int k = idx / level, r = idx - k * level;
-        sm_m[k * kConvMaxTargets + r] = mat[(size_t)k * L + r].x;
+        ulonglong2 m = mat[(size_t)k * L + r];
+        sm_m[k * kConvMaxTargets + r] = m.x;
+        sm_hl[k * kConvMaxTargets + r] = make_double2((double)(m.y >> 21), (double)(m.y & ((1ull << 21) - 1)));
     }
     for (int r = threadIdx.x; r < level; r += blockDim.x) {
         DevPrime p = pr[r];
         sm_t[r] = ConvTarget{p.q, p.qinv_neg, p.one_shoup, 0};
+        const FpMod f = fpm[r];
+        sm_f[r] = f;
         sm_neg[r] = negP[r];
+        if (p.q < kFpPrimeLimit) {
+            const double p20 = fp_canon(1048576.0, f), p21 = fp_canon(2097152.0, f);
+            const double p40 = fp_modmul(p20, p20, f);
+            sm_pow[r] = make_double4(p20, p40, fp_modmul(p40, p21, f), 0.0);
+        }
     }
     __syncthreads();
     int c = blockIdx.x * blockDim.x + threadIdx.x;
@@ -258,15 +278,47 @@ __global__ void __launch_bounds__(256)
         n_neg += y[k] > (p >> 1) ? 1u : 0u;
     }
     uint64_t* o = tmp + (((size_t)i * 2 + poly) * level) * N + c;
+    // integer targets first, so that y is dead before the split below
     for (int r = 0; r < level; r++) {
+        const ConvTarget t = sm_t[r];
+        if (t.q < kFpPrimeLimit) continue;
         U128 acc = {0, 0};
 #pragma unroll
         for (int k = 0; k < KP; k++) mac128(acc, y[k], sm_m[k * kConvMaxTargets + r]);
-        const ConvTarget t = sm_t[r];
-        uint64_t w = n_neg * sm_neg[r];                   // < 16 q <= 2^64
+        uint64_t w = n_neg * sm_neg[r];                      // < 16 q <= 2^64
         uint64_t wr = w - __umul64hi(w, t.one_shoup) * t.q;  // [0, 2q)
         uint64_t v = redc_t(acc, t) + wr;                    // [0, 3q)
         o[(size_t)r * N] = csub(csub(v, 2 * t.q), t.q);
+    }
+    double ya[KP], yb[KP], yc[KP];
+#pragma unroll
+    for (int k = 0; k < KP; k++) {
+        const uint64_t p = pr[L + k].q;
+        const long long v = y[k] > (p >> 1) ? (long long)(y[k] - p) : (long long)y[k];
+        ya[k] = (double)(v >> 40);                        // exact: |.| < 2^19
+        yb[k] = (double)((v >> 20) & ((1ll << 20) - 1));  // exact: < 2^20
+        yc[k] = (double)(v & ((1ll << 20) - 1));          // exact: < 2^20
+    }
+    for (int r = 0; r < level; r++) {
+        if (sm_t[r].q >= kFpPrimeLimit) continue;
+        double t_ah = 0, t_al = 0, t_bh = 0, t_bl = 0, t_ch = 0, t_cl = 0;  // exact partial sums
+#pragma unroll
+        for (int k = 0; k < KP; k++) {
+            const double2 m = sm_hl[k * kConvMaxTargets + r];
+            t_ah = __fma_rn(ya[k], m.x, t_ah);
+            t_al = __fma_rn(ya[k], m.y, t_al);
+            t_bh = __fma_rn(yb[k], m.x, t_bh);
+            t_bl = __fma_rn(yb[k], m.y, t_bl);
+            t_ch = __fma_rn(yc[k], m.x, t_ch);
+            t_cl = __fma_rn(yc[k], m.y, t_cl);
+        }
+        const FpMod f = sm_f[r];
+        const double4 pw = sm_pow[r];
+        double acc = fp_reduce_s(t_cl, f);
+        acc = __dadd_rn(acc, fp_mulmod_s(__fma_rn(2.0, t_ch, t_bl), pw.x, f));
+        acc = __dadd_rn(acc, fp_mulmod_s(__fma_rn(2.0, t_bh, t_al), pw.y, f));
+        acc = __dadd_rn(acc, fp_mulmod_s(t_ah, pw.z, f));
+        o[(size_t)r * N] = d2u(fp_canon(acc, f));
     }
 }
 
@@ -512,8 +564,9 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     switch (K) {
 #define HE_MD_CASE(KK)                                                                                          \
     case KK:                                                                                                    \
-        k_moddown_conv<KK><<<dim3(gx, 2, n), blk, 0, c->stream>>>(u, tmp, level, L, c->d_prime, c->d_md_pcoef, \
-                                                                  c->d_md_mat, c->d_md_negP, c->log_n);         \
+        k_moddown_conv<KK><<<dim3(gx, 2, n), blk, 0, c->stream>>>(u, tmp, level, L, c->d_prime, c->d_fpmod,    \
+                                                                  c->d_md_pcoef, c->d_md_mat, c->d_md_negP,    \
+                                                                  c->log_n);                                   \
         break;
         HE_MD_CASE(1) HE_MD_CASE(2) HE_MD_CASE(3) HE_MD_CASE(4) HE_MD_CASE(5) HE_MD_CASE(6) HE_MD_CASE(7)
         HE_MD_CASE(8) HE_MD_CASE(9) HE_MD_CASE(10) HE_MD_CASE(11) HE_MD_CASE(12) HE_MD_CASE(13) HE_MD_CASE(14)
@@ -523,7 +576,12 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
             return set_err(c, HE_EINVAL, "key switch: K = %d unsupported", K);
     }
     if ((rc = lc(c, "moddown_conv"))) return rc;
-    prof_end(c, HE_PROF_MODDOWN_CONV, 2.0 * n * (K + level) * limbB, 2.0 * n * N * (K + (double)K * level));
+    {
+        int fp_t = 0;
+        for (int r = 0; r < level; r++) fp_t += fp_prime(c, r);
+        prof_end(c, HE_PROF_MODDOWN_CONV, 2.0 * n * (K + level) * limbB,
+                 2.0 * n * N * (K + (double)K * (level - fp_t) + 2.0 * K * fp_t), 2.0 * n * N * 2.0 * K * fp_t);
+    }
 
     // back to the evaluation domain: column pass, then the row pass fused
     // with (u - tmp) P^-1 + add

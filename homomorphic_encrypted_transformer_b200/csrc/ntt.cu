@@ -43,7 +43,7 @@ __device__ __forceinline__ void inv_rows_body(T* sm, uint64_t* a, int r, const T
 }
 
 template <int LOGN>
-__global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS, NTT_MIN_BLOCKS)
+__global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS, NTT_COL_MIN_BLOCKS)
     k_ntt_fwd_cols(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all,
                    const double* __restrict__ twd_all, const FpMod* __restrict__ fpm) {
     using Cf = NttCfg<LOGN>;
@@ -121,7 +121,7 @@ __device__ __forceinline__ void inv_cols_body(T* sm, uint64_t* a, const TW* tw, 
 }
 
 template <int LOGN>
-__global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS, NTT_MIN_BLOCKS)
+__global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS, NTT_COL_MIN_BLOCKS)
     k_ntt_inv_cols(RowSet rs, const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all,
                    const ulonglong2* __restrict__ ninv_all, const double* __restrict__ twd_all,
                    const FpMod* __restrict__ fpm) {

@@ -296,7 +296,10 @@ __device__ __forceinline__ void inv_stage0_scaled(uint64_t (&x)[16], const ulong
 // kernels.  Thread (rr, p) of a row-pass block owns columns 16 p + k of row
 // r = tile * TR + rr; after the pass the 16 registers hold those columns.
 
-// Blocks per SM the transforms are compiled for (register budget 85).
+// Blocks per SM the passes are compiled for: column passes 4 (64 registers),
+// row passes 3 (80 registers; at 64 their spills cost more than the added
+// occupancy gains).
+constexpr int NTT_COL_MIN_BLOCKS = 4;
 constexpr int NTT_MIN_BLOCKS = 3;
 
 // shared-memory index of element i of a padded row (one pad word per 16)
