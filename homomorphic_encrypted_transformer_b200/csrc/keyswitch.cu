@@ -364,25 +364,29 @@ __global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
         for (int k = 0; k < 16; k++) v[k] = fwd_canon(x[k], q);
     }
     const size_t off = (size_t)t * Cf::N + j0;  // within a [level][N] polynomial
-    const ulonglong2* up = reinterpret_cast<const ulonglong2*>(u + (size_t)(i * 2 + poly) * (level + K) * Cf::N + off);
-    ulonglong2* op = reinterpret_cast<ulonglong2*>(mo.out.p[i] + (size_t)poly * level * Cf::N + off);
+    const uint64_t* up = u + (size_t)(i * 2 + poly) * (level + K) * Cf::N + off;
+    uint64_t* op = mo.out.p[i] + (size_t)poly * level * Cf::N + off;
     const uint64_t* ad = poly == 0 ? mo.add0.p[i] : mo.add1.p[i];
     const uint64_t g = (poly == 0 && mo.sig_add0) ? mo.gal.g[i] : 0;
     const ulonglong2 w = pinv[t];
     const uint64_t* adt = ad ? ad + (size_t)t * Cf::N : nullptr;
 #pragma unroll
-    for (int k = 0; k < 8; k++) {
-        const ulonglong2 uv = up[k];
-        uint64_t z0 = mul_shoup(uv.x + q - v[2 * k], w.x, w.y, q);
-        uint64_t z1 = mul_shoup(uv.y + q - v[2 * k + 1], w.x, w.y, q);
+    for (int k = 0; k < 4; k++) {
+        uint64_t z[4];
+        ldg256_ro(up + 4 * k, z[0], z[1], z[2], z[3]);
+#pragma unroll
+        for (int e = 0; e < 4; e++) z[e] = mul_shoup(z[e] + q - v[4 * k + e], w.x, w.y, q);
         if (adt) {
-            const int s = automorph_src(j0 + 2 * k, LOGN, g);
-            const ulonglong2 av = __ldg(reinterpret_cast<const ulonglong2*>(adt + (s & ~1)));
-            const bool sw = s & 1;
-            z0 = add_mod(z0, sw ? av.y : av.x, q);
-            z1 = add_mod(z1, sw ? av.x : av.y, q);
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const int s = automorph_src(j0 + 4 * k + 2 * h, LOGN, g);
+                const ulonglong2 av = __ldg(reinterpret_cast<const ulonglong2*>(adt + (s & ~1)));
+                const bool sw = s & 1;
+                z[2 * h] = add_mod(z[2 * h], sw ? av.y : av.x, q);
+                z[2 * h + 1] = add_mod(z[2 * h + 1], sw ? av.x : av.y, q);
+            }
         }
-        op[k] = make_ulonglong2(z0, z1);
+        stg256(op + 4 * k, z[0], z[1], z[2], z[3]);
     }
 }
 

@@ -106,6 +106,22 @@ __device__ __forceinline__ void inv_stages(uint64_t (&x)[16], const ulonglong2* 
     }
 }
 
+// 256-bit global accesses (sm_100 vector width); the address must be 32-byte
+// aligned.  ldg256_ro goes through the read-only path: only for data that no
+// thread writes during the kernel (tables, inputs of out-of-place kernels).
+__device__ __forceinline__ void ldg256_ro(const double* p, double& a, double& b, double& c, double& d) {
+    asm("ld.global.nc.v4.f64 {%0, %1, %2, %3}, [%4];" : "=d"(a), "=d"(b), "=d"(c), "=d"(d) : "l"(p));
+}
+__device__ __forceinline__ void ldg256_ro(const uint64_t* p, uint64_t& a, uint64_t& b, uint64_t& c, uint64_t& d) {
+    asm("ld.global.nc.v4.u64 {%0, %1, %2, %3}, [%4];" : "=l"(a), "=l"(b), "=l"(c), "=l"(d) : "l"(p));
+}
+__device__ __forceinline__ void ldg256(const uint64_t* p, uint64_t& a, uint64_t& b, uint64_t& c, uint64_t& d) {
+    asm volatile("ld.global.v4.u64 {%0, %1, %2, %3}, [%4];" : "=l"(a), "=l"(b), "=l"(c), "=l"(d) : "l"(p) : "memory");
+}
+__device__ __forceinline__ void stg256(uint64_t* p, uint64_t a, uint64_t b, uint64_t c, uint64_t d) {
+    asm volatile("st.global.v4.u64 [%0], {%1, %2, %3, %4};" ::"l"(p), "l"(a), "l"(b), "l"(c), "l"(d) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // FP64 arithmetic for primes below 2^41 (the 40-bit primes of the modulus
 // chain).  Residues are integers held in doubles (exact below 2^53), signed
@@ -186,14 +202,13 @@ template <int LC>
 __device__ __forceinline__ void load_stage_tw(double (&w)[8], const double* __restrict__ p) {
     if constexpr (LC == 0) {
         w[0] = __ldg(p);
+    } else if constexpr (LC == 1) {
+        double2 d = __ldg(reinterpret_cast<const double2*>(p));
+        w[0] = d.x;
+        w[1] = d.y;
     } else {
-        const double2* p2 = reinterpret_cast<const double2*>(p);
 #pragma unroll
-        for (int v = 0; v < (1 << LC) / 2; v++) {
-            double2 d = __ldg(p2 + v);
-            w[2 * v] = d.x;
-            w[2 * v + 1] = d.y;
-        }
+        for (int v = 0; v < (1 << LC) / 4; v++) ldg256_ro(p + 4 * v, w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
     }
 }
 
@@ -308,24 +323,27 @@ __device__ __forceinline__ int padded(int i) { return i + (i >> 4); }
 template <int LOGN>
 __device__ __forceinline__ int row_lane() { return threadIdx.x % (NttCfg<LOGN>::C / 16); }
 
-// x[k] = a[k], k < 16 (a 16-byte aligned)
+// x[k] = a[k], k < 16 (a 128-byte aligned; a may be rewritten by this kernel)
 template <typename T>
 __device__ __forceinline__ void row_load16(T (&x)[16], const uint64_t* a) {
-    const ulonglong2* in = reinterpret_cast<const ulonglong2*>(a);
 #pragma unroll
-    for (int k = 0; k < 8; k++) {
-        ulonglong2 v = in[k];
-        x[2 * k] = to_elem(v.x, T());
-        x[2 * k + 1] = to_elem(v.y, T());
+    for (int v = 0; v < 4; v++) {
+        uint64_t e0, e1, e2, e3;
+        ldg256(a + 4 * v, e0, e1, e2, e3);
+        x[4 * v] = to_elem(e0, T());
+        x[4 * v + 1] = to_elem(e1, T());
+        x[4 * v + 2] = to_elem(e2, T());
+        x[4 * v + 3] = to_elem(e3, T());
     }
 }
 
-// a[k] = canonical x[k] (forward transform output)
+// a[k] = canonical x[k] (forward transform output), a 128-byte aligned
 template <typename T, typename M>
 __device__ __forceinline__ void row_store16(uint64_t* a, T (&x)[16], const M& m) {
-    ulonglong2* o = reinterpret_cast<ulonglong2*>(a);
 #pragma unroll
-    for (int k = 0; k < 8; k++) o[k] = make_ulonglong2(fwd_canon(x[2 * k], m), fwd_canon(x[2 * k + 1], m));
+    for (int v = 0; v < 4; v++)
+        stg256(a + 4 * v, fwd_canon(x[4 * v], m), fwd_canon(x[4 * v + 1], m), fwd_canon(x[4 * v + 2], m),
+               fwd_canon(x[4 * v + 3], m));
 }
 
 // x[k] = row[p + CS k], k < 16: the forward row pass's input, the column
