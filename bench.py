@@ -304,10 +304,9 @@ def run_native(args, rank, world, local_rank):
         best = min(best, ev0.elapsed_time(ev1))
     fp_modmul_s = he.he_probe_int_threads(ctx) * iters * he.he_probe_int_mults_per_iter() / (best * 1e-3)
 
-    # timed region
+    # timed region (the headline number): K steps, no profiling events
     clocks = ClockSampler(local_rank)
     he.he_launch_count(ctx, reset=True)
-    he.he_profile_enable(ctx, True)
     clocks.start()
     barrier()
     torch.cuda.synchronize()
@@ -318,12 +317,13 @@ def run_native(args, rank, world, local_rank):
     t1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms = t0.elapsed_time(t1)
+    ms_plain = t0.elapsed_time(t1)
+    clk = clocks.stop()
     launches = he.he_launch_count(ctx)
-    prof = {name: he.he_profile_read(ctx, cls) + (he.he_profile_read_fp(ctx, cls),) for name, cls in he.PROF.items()}
-    he.he_profile_enable(ctx, False)
 
-    # same step without profiling events (the headline number)
+    # the same steps again with every launch class bracketed by events on the
+    # launching stream: per-kernel device time and algorithmic work
+    he.he_profile_enable(ctx, True)
     torch.cuda.synchronize()
     barrier()
     t0.record(stream)
@@ -332,8 +332,9 @@ def run_native(args, rank, world, local_rank):
     t1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms_plain = t0.elapsed_time(t1)
-    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    prof = {name: he.he_profile_read(ctx, cls) + (he.he_profile_read_fp(ctx, cls),) for name, cls in he.PROF.items()}
+    he.he_profile_enable(ctx, False)
 
     if world > 1:
         tt = torch.tensor([ms_plain, ms], device=dev)

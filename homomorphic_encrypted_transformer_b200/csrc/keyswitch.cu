@@ -91,14 +91,25 @@ constexpr int kConvMaxTargets = 64;
 // ModUp of digit j (NS source primes at rows s0..s0+NS-1), one launch per digit:
 //   ext_j[i][pos(t)][c] = sum_s [x_s qhat_inv_s]_{q_s} (qhat_s mod t)   (coefficient domain)
 // for every target row t (all rows of Q_level and P outside the digit).
-// 128-bit accumulation of the NS products, one reduction per target.
+//  - targets below 2^41: signed FP64 rounded-quotient products, one
+//    reduction at the end;
+//  - 60-bit targets, digit of 40-bit sources (narrow): with y = y1 2^21 + y0
+//    (y0 < 2^21, y1 < 2^20) and the Montgomery-form entry m' = m2 2^42 +
+//    m1 2^21 + m0 (m0, m1 < 2^21, m2 < 2^18) the four sums
+//      V0 = S y0 m0, V1 = S y0 m1 + y1 m0, V2 = S y0 m2 + y1 m1, V3 = S y1 m2
+//    are exact doubles below 2^47 (NS <= 16); the 128-bit value
+//    V0 + V1 2^21 + V2 2^42 + V3 2^63 = S y m' is assembled on the integer
+//    pipe and one REDC gives S y m mod t;
+//  - 60-bit targets, digit with a 60-bit source: 128-bit accumulation of the
+//    NS products, one REDC.
 template <int NS>
 __global__ void __launch_bounds__(256)
     k_modup_conv(const uint64_t* __restrict__ coef, uint64_t* __restrict__ ext_j, const ulonglong2* __restrict__ src,
                  const ulonglong2* __restrict__ mat, ModupArgs a, const DevPrime* __restrict__ pr,
-                 const FpMod* __restrict__ fpm, int level, int n_rows, int s0, int logn) {
+                 const FpMod* __restrict__ fpm, int level, int n_rows, int s0, int all_narrow, int logn) {
     __shared__ uint64_t sm_m[NS * kConvMaxTargets];
     __shared__ double sm_md[NS * kConvMaxTargets];
+    __shared__ double sm_m0[NS * kConvMaxTargets], sm_m1[NS * kConvMaxTargets], sm_m2[NS * kConvMaxTargets];
     __shared__ ConvTarget sm_t[kConvMaxTargets];
     __shared__ FpMod sm_f[kConvMaxTargets];
     const int N = 1 << logn;
@@ -107,8 +118,12 @@ __global__ void __launch_bounds__(256)
         int s = idx / n_tgt, tt = idx - s * n_tgt;
         int t = tt < s0 ? tt : tt + NS;
         ulonglong2 m = mat[(size_t)s * n_rows + t];
-        sm_m[s * kConvMaxTargets + tt] = m.x;
-        sm_md[s * kConvMaxTargets + tt] = (double)m.y;  // exact: below 2^41 where it is used
+        const int o = s * kConvMaxTargets + tt;
+        sm_m[o] = m.x;
+        sm_md[o] = (double)m.y;  // exact: below 2^41 where it is used
+        sm_m0[o] = (double)(m.x & ((1ull << 21) - 1));
+        sm_m1[o] = (double)((m.x >> 21) & ((1ull << 21) - 1));
+        sm_m2[o] = (double)(m.x >> 42);
     }
     for (int tt = threadIdx.x; tt < n_tgt; tt += blockDim.x) {
         int t = tt < s0 ? tt : tt + NS;
@@ -121,7 +136,8 @@ __global__ void __launch_bounds__(256)
     int i = blockIdx.y;
     if (c >= N) return;
     uint64_t y[NS];
-    double yd[NS];    // y as a double where the source prime is below 2^41
+    double yd[NS];      // y as a double where the source prime is below 2^41
+    double y0[NS], y1[NS];
     bool narrow[NS];
 #pragma unroll
     for (int s = 0; s < NS; s++) {
@@ -131,12 +147,13 @@ __global__ void __launch_bounds__(256)
         y[s] = mul_shoup(x, w.x, w.y, q);
         narrow[s] = q < kFpPrimeLimit;
         yd[s] = u2d(narrow[s] ? y[s] : 0);
+        y0[s] = (double)(y[s] & ((1ull << 21) - 1));
+        y1[s] = (double)((y[s] >> 21) & ((1ull << 20) - 1));  // all of it when the digit is narrow
     }
     uint64_t* o = ext_j + (size_t)i * n_tgt * N + c;
     for (int tt = 0; tt < n_tgt; tt++) {
         const ConvTarget t = sm_t[tt];
         if (t.q < kFpPrimeLimit) {
-            // FP64 path: signed partial products |.| < 5t/8, one reduction at the end
             const FpMod f = sm_f[tt];
             double acc = 0.0;
 #pragma unroll
@@ -146,6 +163,23 @@ __global__ void __launch_bounds__(256)
                 acc = __dadd_rn(acc, fp_mulmod_s(ys, sm_md[s * kConvMaxTargets + tt], f));
             }
             o[(size_t)tt * N] = d2u(fp_canon(acc, f));
+        } else if (all_narrow) {
+            double v0 = 0, v1 = 0, v2 = 0, v3 = 0;
+#pragma unroll
+            for (int s = 0; s < NS; s++) {
+                const int k = s * kConvMaxTargets + tt;
+                const double m0 = sm_m0[k], m1 = sm_m1[k], m2 = sm_m2[k];
+                v0 = __fma_rn(y0[s], m0, v0);
+                v1 = __fma_rn(y0[s], m1, __fma_rn(y1[s], m0, v1));
+                v2 = __fma_rn(y0[s], m2, __fma_rn(y1[s], m1, v2));
+                v3 = __fma_rn(y1[s], m2, v3);
+            }
+            const uint64_t w0 = d2u(v0), w1 = d2u(v1), w2 = d2u(v2), w3 = d2u(v3);
+            U128 acc = {w0, 0};
+            add128(acc, w1 << 21, w1 >> 43);
+            add128(acc, w2 << 42, w2 >> 22);
+            add128(acc, w3 << 63, w3 >> 1);
+            o[(size_t)tt * N] = redc_t(acc, t);
         } else {
             U128 acc = {0, 0};
 #pragma unroll
@@ -503,11 +537,13 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     for (int j = 0; j < nd; j++) {
         uint64_t* ext_j = ext + (size_t)ma.ext_off[j] * n * N;
         const int s0 = ma.src_row[j];
+        int narrow_j = 1;  // every source prime of the digit below 2^41
+        for (int s = 0; s < ma.n_src[j]; s++) narrow_j &= fp_prime(c, s0 + s);
         switch (ma.n_src[j]) {
 #define HE_MU_CASE(S)                                                                                       \
     case S:                                                                                                 \
         k_modup_conv<S><<<dim3(gx, n), blk, 0, c->stream>>>(coef, ext_j, ma.src[j], ma.mat[j], ma, c->d_prime, \
-                                                            c->d_fpmod, level, n_rows, s0, c->log_n);       \
+                                                            c->d_fpmod, level, n_rows, s0, narrow_j, c->log_n); \
         break;
             HE_MU_CASE(1) HE_MU_CASE(2) HE_MU_CASE(3) HE_MU_CASE(4) HE_MU_CASE(5) HE_MU_CASE(6) HE_MU_CASE(7)
             HE_MU_CASE(8) HE_MU_CASE(9) HE_MU_CASE(10) HE_MU_CASE(11) HE_MU_CASE(12) HE_MU_CASE(13)

@@ -76,6 +76,12 @@ __device__ __forceinline__ void mac128(U128& acc, uint64_t a, uint64_t b) {
     acc.hi += hi + (acc.lo < lo ? 1ull : 0ull);
 }
 
+// acc += hi 2^64 + lo
+__device__ __forceinline__ void add128(U128& acc, uint64_t lo, uint64_t hi) {
+    acc.lo += lo;
+    acc.hi += hi + (acc.lo < lo ? 1ull : 0ull);
+}
+
 // Any 128-bit value mod q: (hi mod q) 2^64 + lo = (hi mod q)(2^64 mod q) + lo.
 __device__ __forceinline__ uint64_t reduce128(const U128& x, const DevPrime& p) {
     uint64_t h = reduce64(x.hi, p);

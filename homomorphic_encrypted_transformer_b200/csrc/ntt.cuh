@@ -64,48 +64,6 @@ __device__ __forceinline__ void bfly_gs(uint64_t& x, uint64_t& y, const ulonglon
 
 __device__ __forceinline__ ulonglong2 ldtw(const ulonglong2* p) { return __ldg(p); }
 
-// Forward stages on 16 registers.  H stages (H <= 4) with register pair
-// distance 2^(H-1-u) at stage u; the twiddle of the pair starting at k is
-// tw[base(u) + (key(k) >> (H - u))] where key(k) = kofs + k, with
-//   base(u) = (2^(s0+u)) + row_term << u.
-// s0: global index of the first stage; kofs/row_term select the block.
-template <int H>
-__device__ __forceinline__ void fwd_stages(uint64_t (&x)[16], const ulonglong2* __restrict__ tw, int s0, int row_term,
-                                           int kofs, uint64_t q) {
-    const uint64_t two_q = 2 * q;
-#pragma unroll
-    for (int u = 0; u < H; u++) {
-        const int D = 1 << (H - 1 - u);
-        const int base = (1 << (s0 + u)) + (row_term << u);
-#pragma unroll
-        for (int k = 0; k < 16; k++) {
-            if (k & D) continue;
-            ulonglong2 w = ldtw(tw + base + ((kofs + k) >> (H - u)));
-            bfly_ct(x[k], x[k + D], w, q, two_q);
-        }
-    }
-}
-
-// Inverse stages on 16 registers: the forward stages of fwd_stages<H> in
-// reverse order with GS butterflies (same twiddle index formula, inverse
-// table).  Stages u = H-1 down to ULO.
-template <int H, int ULO = 0>
-__device__ __forceinline__ void inv_stages(uint64_t (&x)[16], const ulonglong2* __restrict__ tw, int s0, int row_term,
-                                           int kofs, uint64_t q) {
-    const uint64_t two_q = 2 * q;
-#pragma unroll
-    for (int u = H - 1; u >= ULO; u--) {
-        const int D = 1 << (H - 1 - u);
-        const int base = (1 << (s0 + u)) + (row_term << u);
-#pragma unroll
-        for (int k = 0; k < 16; k++) {
-            if (k & D) continue;
-            ulonglong2 w = ldtw(tw + base + ((kofs + k) >> (H - u)));
-            bfly_gs(x[k], x[k + D], w, q, two_q);
-        }
-    }
-}
-
 // 256-bit global accesses (sm_100 vector width); the address must be 32-byte
 // aligned.  ldg256_ro goes through the read-only path: only for data that no
 // thread writes during the kernel (tables, inputs of out-of-place kernels).
@@ -120,6 +78,77 @@ __device__ __forceinline__ void ldg256(const uint64_t* p, uint64_t& a, uint64_t&
 }
 __device__ __forceinline__ void stg256(uint64_t* p, uint64_t a, uint64_t b, uint64_t c, uint64_t d) {
     asm volatile("st.global.v4.u64 [%0], {%1, %2, %3, %4};" ::"l"(p), "l"(a), "l"(b), "l"(c), "l"(d) : "memory");
+}
+
+// Forward stages on 16 registers.  H stages (H <= 4) with register pair
+// distance 2^(H-1-u) at stage u; the twiddle of the pair starting at k is
+// tw[base(u) + (key(k) >> (H - u))] where key(k) = kofs + k, with
+//   base(u) = (2^(s0+u)) + row_term << u.
+// s0: global index of the first stage; kofs/row_term select the block.
+// kofs is a multiple of 16, so the 16 >> (H - u) twiddles one thread uses at
+// stage u are contiguous and start at a multiple of their count: pairs of
+// them load as one 256-bit access.
+template <int H, int U>
+__device__ __forceinline__ void load_stage_tw_int(ulonglong2 (&w)[8], const ulonglong2* __restrict__ p) {
+    constexpr int LC = 4 - H + U;
+    if constexpr (LC == 0) {
+        w[0] = ldtw(p);
+    } else {
+#pragma unroll
+        for (int v = 0; v < (1 << LC) / 2; v++) {
+            uint64_t a, b, c, d;
+            ldg256_ro(reinterpret_cast<const uint64_t*>(p + 2 * v), a, b, c, d);
+            w[2 * v] = make_ulonglong2(a, b);
+            w[2 * v + 1] = make_ulonglong2(c, d);
+        }
+    }
+}
+
+template <int H, int U>
+__device__ __forceinline__ void fwd_stage_int(uint64_t (&x)[16], const ulonglong2* __restrict__ tw, int s0,
+                                              int row_term, int kofs, uint64_t q) {
+    constexpr int D = 1 << (H - 1 - U);
+    ulonglong2 w[8];
+    load_stage_tw_int<H, U>(w, tw + (1 << (s0 + U)) + (row_term << U) + (kofs >> (H - U)));
+#pragma unroll
+    for (int k = 0; k < 16; k++) {
+        if (k & D) continue;
+        bfly_ct(x[k], x[k + D], w[k >> (H - U)], q, 2 * q);
+    }
+}
+
+template <int H, int U>
+__device__ __forceinline__ void inv_stage_int(uint64_t (&x)[16], const ulonglong2* __restrict__ tw, int s0,
+                                              int row_term, int kofs, uint64_t q) {
+    constexpr int D = 1 << (H - 1 - U);
+    ulonglong2 w[8];
+    load_stage_tw_int<H, U>(w, tw + (1 << (s0 + U)) + (row_term << U) + (kofs >> (H - U)));
+#pragma unroll
+    for (int k = 0; k < 16; k++) {
+        if (k & D) continue;
+        bfly_gs(x[k], x[k + D], w[k >> (H - U)], q, 2 * q);
+    }
+}
+
+template <int H>
+__device__ __forceinline__ void fwd_stages(uint64_t (&x)[16], const ulonglong2* __restrict__ tw, int s0, int row_term,
+                                           int kofs, uint64_t q) {
+    if constexpr (H > 0) fwd_stage_int<H, 0>(x, tw, s0, row_term, kofs, q);
+    if constexpr (H > 1) fwd_stage_int<H, 1>(x, tw, s0, row_term, kofs, q);
+    if constexpr (H > 2) fwd_stage_int<H, 2>(x, tw, s0, row_term, kofs, q);
+    if constexpr (H > 3) fwd_stage_int<H, 3>(x, tw, s0, row_term, kofs, q);
+}
+
+// Inverse stages on 16 registers: the forward stages of fwd_stages<H> in
+// reverse order with GS butterflies (same twiddle index formula, inverse
+// table).  Stages u = H-1 down to ULO.
+template <int H, int ULO = 0>
+__device__ __forceinline__ void inv_stages(uint64_t (&x)[16], const ulonglong2* __restrict__ tw, int s0, int row_term,
+                                           int kofs, uint64_t q) {
+    if constexpr (H > 3 && ULO <= 3) inv_stage_int<H, 3>(x, tw, s0, row_term, kofs, q);
+    if constexpr (H > 2 && ULO <= 2) inv_stage_int<H, 2>(x, tw, s0, row_term, kofs, q);
+    if constexpr (H > 1 && ULO <= 1) inv_stage_int<H, 1>(x, tw, s0, row_term, kofs, q);
+    if constexpr (H > 0 && ULO <= 0) inv_stage_int<H, 0>(x, tw, s0, row_term, kofs, q);
 }
 
 // ---------------------------------------------------------------------------
