@@ -370,11 +370,16 @@ def run_native(args, rank, world, local_rank):
     batch_bytes = N_KEYS * key_bytes + N_CTS * 2 * ct_bytes
     hbm_frac_step = (batch_bytes / (ms_plain * 1e-3 / args.steps)) / 1e9 / hbm_peak
     roof = roofline_for(dom_name, prof[dom_name], int_modmul_s, fp_modmul_s, hbm_peak, pk_kind)
+    # ideal time of a whole step: each class's modular products at the probes'
+    # rates (integer and FP64 pipes taken one after the other)
+    alu_ideal_ms = sum(((v[3] - v[4]) / int_modmul_s + v[4] / fp_modmul_s) * 1e3 for v in prof.values()) / args.steps
     line = {"metric": METRIC, "value": value, "unit": "rotations/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_plain / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u64", "data": "synthetic",
             "config": dict(WORKLOAD, parallelism="replicas%d" % world if world > 1 else "single"),
             "hbm_roofline_frac_of_step": hbm_frac_step,
+            "alu_ideal_ms_per_step": alu_ideal_ms,
+            "alu_roofline_frac_of_step": alu_ideal_ms / (ms_plain / args.steps),
             "roofline": roof,
             "probes": {"copy_gbs": copy_gbs, "int_shoup_modmul_per_s": int_modmul_s,
                        "fp64_modmul_per_s": fp_modmul_s},

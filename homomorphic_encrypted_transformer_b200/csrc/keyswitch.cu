@@ -558,8 +558,12 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
         double prods = 0, prods_fp = 0;
         for (int j = 0; j < nd; j++) {
             prods += (double)ma.n_src[j] * (1 + n_rows - ma.n_src[j]);
+            // FP64 pipe: 40-bit targets, and every target of a digit of 40-bit
+            // sources (exact FP64 partial sums, six FMAs per product)
+            int narrow_j = 1;
+            for (int s = 0; s < ma.n_src[j]; s++) narrow_j &= fp_prime(c, ma.src_row[j] + s);
             for (int t = 0; t < n_rows; t++)
-                if ((t < ma.src_row[j] || t >= ma.src_row[j] + ma.n_src[j]) && fp_prime(c, ep[t]))
+                if ((t < ma.src_row[j] || t >= ma.src_row[j] + ma.n_src[j]) && (narrow_j || fp_prime(c, ep[t])))
                     prods_fp += ma.n_src[j];
         }
         prof_end(c, HE_PROF_MODUP, (double)n * (sum_src + ext_rows) * limbB, (double)n * N * prods,
