@@ -528,6 +528,10 @@ extern "C" int he_ctx_destroy(he_ctx* c) {
     cudaFree(c->relin.d);
     for (int i = 0; i < kScratchSlots; i++) cudaFree(c->scratch[i]);
     cudaFree(c->io_buf);
+    if (c->io_h2d) cudaStreamSynchronize(c->io_h2d), cudaStreamDestroy(c->io_h2d);
+    if (c->io_d2h) cudaStreamSynchronize(c->io_d2h), cudaStreamDestroy(c->io_d2h);
+    for (cudaEvent_t e : c->io_ev)
+        if (e) cudaEventDestroy(e);
     for (auto& p : c->prof_pending) {
         if (p.a) cudaEventDestroy(p.a);
         if (p.b) cudaEventDestroy(p.b);

@@ -83,6 +83,8 @@ struct he_ctx {
     size_t scratch_words[4] = {0, 0, 0, 0};
     uint64_t* io_buf = nullptr;  // device staging of the host-buffer entry point
     size_t io_words = 0;
+    cudaStream_t io_h2d = nullptr, io_d2h = nullptr;  // its copy streams (one per direction)
+    cudaEvent_t io_ev[6] = {};                         // per staging buffer: uploaded, rotated, downloaded
 
     bool prof_on = false;
     he::ProfSlot prof[HE_PROF_N];

@@ -739,33 +739,97 @@ extern "C" int he_rotate_batch(he_ctx* c, const he_ct* in, const int32_t* steps,
     return rotate_many(c, in, steps, out, n);
 }
 
+// Host-buffer rotation, pipelined: the ciphertexts, ordered by Galois element
+// (so that a chunk holds few distinct keys), go through the GPU in chunks of
+// kIoChunk.  Two staging buffers per direction let chunk k+1's upload and
+// chunk k-1's download (one copy engine each) overlap chunk k's rotation.
+constexpr int kIoChunk = 8;
+
+static int io_setup(he_ctx* c, size_t words) {
+    int rc;
+    if (words > c->io_words) {
+        cudaStreamSynchronize(c->stream);
+        cudaFree(c->io_buf);
+        c->io_buf = nullptr;
+        c->io_words = 0;
+        if ((rc = check_cuda(c, cudaMalloc(&c->io_buf, words * 8), "io buffer"))) return rc;
+        c->io_words = words;
+    }
+    if (!c->io_h2d && (rc = check_cuda(c, cudaStreamCreateWithFlags(&c->io_h2d, cudaStreamNonBlocking), "io stream")))
+        return rc;
+    if (!c->io_d2h && (rc = check_cuda(c, cudaStreamCreateWithFlags(&c->io_d2h, cudaStreamNonBlocking), "io stream")))
+        return rc;
+    for (cudaEvent_t& e : c->io_ev)
+        if (!e && (rc = check_cuda(c, cudaEventCreateWithFlags(&e, cudaEventDisableTiming), "io event"))) return rc;
+    return HE_OK;
+}
+
+static int io_drain(he_ctx* c, int rc) {
+    cudaStreamSynchronize(c->io_h2d);
+    cudaStreamSynchronize(c->stream);
+    cudaStreamSynchronize(c->io_d2h);
+    return rc;
+}
+
 extern "C" int he_rotate_batch_host(he_ctx* c, const uint64_t* h_in, int level, const int32_t* steps,
                                     uint64_t* h_out, int n) {
     if (!c) return HE_EINVAL;
     if (!h_in || !h_out || !steps || n < 0 || level < 1 || level > c->L)
         return set_err(c, HE_EINVAL, "he_rotate_batch_host: bad arguments");
-    const size_t ct_words = (size_t)2 * level * c->N, total = ct_words * n;
-    if (2 * total > c->io_words) {
-        cudaStreamSynchronize(c->stream);
-        cudaFree(c->io_buf);
-        c->io_buf = nullptr;
-        c->io_words = 0;
-        int rc = check_cuda(c, cudaMalloc(&c->io_buf, 2 * total * 8), "io buffer");
-        if (rc) return rc;
-        c->io_words = 2 * total;
-    }
-    uint64_t* din = c->io_buf;
-    uint64_t* dout = c->io_buf + total;
-    int rc = check_cuda(c, cudaMemcpyAsync(din, h_in, total * 8, cudaMemcpyHostToDevice, c->stream), "H2D");
-    if (rc) return rc;
-    std::vector<he_ct> in(n), out(n);
+    if (n == 0) return HE_OK;
+    std::vector<uint64_t> gal(n);
     for (int i = 0; i < n; i++) {
-        in[i] = he_ct{din + i * ct_words, level, 1.0, 1};
-        out[i] = he_ct{dout + i * ct_words, level, 1.0, 1};
+        gal[i] = galois_elt(c, steps[i]);
+        if (gal[i] != 1 && !c->rot_keys.count(gal[i]))
+            return set_err(c, HE_ENOKEY, "he_rotate_batch_host: no key for step %d", steps[i]);
     }
-    rc = rotate_many(c, in.data(), steps, out.data(), n);
+    std::vector<int> order(n);
+    for (int i = 0; i < n; i++) order[i] = i;
+    std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return gal[x] < gal[y]; });
+
+    const size_t ct_words = (size_t)2 * level * c->N, ct_bytes = ct_words * 8;
+    const int chunk = std::min(kIoChunk, n);
+    int rc = io_setup(c, 4 * (size_t)chunk * ct_words);
     if (rc) return rc;
-    rc = check_cuda(c, cudaMemcpyAsync(h_out, dout, total * 8, cudaMemcpyDeviceToHost, c->stream), "D2H");
-    if (rc) return rc;
+    cudaEvent_t* up = c->io_ev;        // [2] upload of buffer b done
+    cudaEvent_t* done = c->io_ev + 2;  // [2] rotation of buffer b done
+    cudaEvent_t* down = c->io_ev + 4;  // [2] download of buffer b done
+    const int n_chunks = (n + chunk - 1) / chunk;
+    for (int k = 0; k < n_chunks; k++) {
+        const int b = k & 1, i0 = k * chunk, m = std::min(chunk, n - i0);
+        uint64_t* din = c->io_buf + (size_t)b * chunk * ct_words;
+        uint64_t* dout = c->io_buf + (size_t)(2 + b) * chunk * ct_words;
+        // upload, once chunk k-2 no longer reads this buffer
+        if (k >= 2) cudaStreamWaitEvent(c->io_h2d, done[b], 0);
+        for (int j = 0; j < m; j++) {
+            rc = check_cuda(c, cudaMemcpyAsync(din + j * ct_words, h_in + (size_t)order[i0 + j] * ct_words, ct_bytes,
+                                               cudaMemcpyHostToDevice, c->io_h2d), "H2D");
+            if (rc) return io_drain(c, rc);
+        }
+        cudaEventRecord(up[b], c->io_h2d);
+        // rotate, once uploaded and once chunk k-2's download left the output buffer
+        cudaStreamWaitEvent(c->stream, up[b], 0);
+        if (k >= 2) cudaStreamWaitEvent(c->stream, down[b], 0);
+        std::vector<he_ct> in(m), out(m);
+        std::vector<int32_t> st(m);
+        for (int j = 0; j < m; j++) {
+            in[j] = he_ct{din + j * ct_words, level, 1.0, 1};
+            out[j] = he_ct{dout + j * ct_words, level, 1.0, 1};
+            st[j] = steps[order[i0 + j]];
+        }
+        rc = rotate_many(c, in.data(), st.data(), out.data(), m);
+        if (rc) return io_drain(c, rc);
+        cudaEventRecord(done[b], c->stream);
+        // download
+        cudaStreamWaitEvent(c->io_d2h, done[b], 0);
+        for (int j = 0; j < m; j++) {
+            rc = check_cuda(c, cudaMemcpyAsync(h_out + (size_t)order[i0 + j] * ct_words, dout + j * ct_words, ct_bytes,
+                                               cudaMemcpyDeviceToHost, c->io_d2h), "D2H");
+            if (rc) return io_drain(c, rc);
+        }
+        cudaEventRecord(down[b], c->io_d2h);
+    }
+    rc = check_cuda(c, cudaStreamSynchronize(c->io_d2h), "D2H sync");
+    if (rc) return io_drain(c, rc);
     return he_sync(c);
 }

@@ -156,8 +156,11 @@ int he_rotate(he_ctx* ctx, const he_ct* in, int32_t step, he_ct* out);
  * Ciphertexts that share a step share one read of its key. */
 int he_rotate_batch(he_ctx* ctx, const he_ct* in, const int32_t* steps, he_ct* out, int n);
 /* Host-buffer form of he_rotate_batch: h_in / h_out are host [n][2][level][N];
- * the call copies in, rotates, copies out and waits.  Pinned host memory
- * gives full copy bandwidth.  Synchronous. */
+ * the call copies in, rotates, copies out and waits.  The ciphertexts pass
+ * through the GPU in chunks of 8, ordered by step, with uploads, rotations and
+ * downloads of consecutive chunks overlapped (device staging: 4 chunks, held
+ * by the context).  Pinned host memory gives full copy bandwidth.  h_out may
+ * not overlap h_in.  Synchronous. */
 int he_rotate_batch_host(he_ctx* ctx, const uint64_t* h_in, int level, const int32_t* steps,
                          uint64_t* h_out, int n);
 

@@ -150,3 +150,31 @@ def test_rotation_batch_host_buffers():
     for i in range(n):
         want = C.rotate(cts[i], steps[i], st.oracle_rot_key(steps[i]), P)
         assert np.array_equal(h_out[i], want["c"])
+
+
+def test_rotation_batch_host_buffers_pipelined():
+    """21 ciphertexts pass the host-buffer entry in three chunks (both staging
+    buffers reused); steps unsorted, repeated, and one identity rotation
+    (step N/2, Galois element 1)."""
+    he = lib()
+    st = Setup(12, 3, 1, 3, seed=6)
+    P = st.P
+    n = 21
+    steps = [3, 1, 2, 1, 7, 3, 2, P.n_slots, 1, 7, 2, 3, 1, 1, 2, 7, 3, 2, 1, 7, 3]
+    for s_ in set(steps):
+        if s_ != P.n_slots:
+            st.upload_rot(s_)
+    cts = [st.encrypt(S.complex_slots(st.seed, P.n_slots, -1, 1, i), 3, ct_id=i) for i in range(n)]
+    h_in = np.stack([c["c"] for c in cts])
+    h_out = np.zeros_like(h_in)
+    he.he_rotate_batch_host(st.ctx, h_in, 3, steps, h_out)
+    for i in range(n):
+        if steps[i] == P.n_slots:
+            assert np.array_equal(h_out[i], h_in[i])
+            continue
+        want = C.rotate(cts[i], steps[i], st.oracle_rot_key(steps[i]), P)
+        assert np.array_equal(h_out[i], want["c"]), i
+    # a second call reuses the staging buffers and the copy streams
+    h_out2 = np.zeros_like(h_in)
+    he.he_rotate_batch_host(st.ctx, h_in, 3, steps, h_out2)
+    assert np.array_equal(h_out2, h_out)
