@@ -88,90 +88,110 @@ __device__ __forceinline__ uint64_t redc_t(const U128& x, const ConvTarget& p) {
 
 constexpr int kConvMaxTargets = 64;
 
+// Targets of one ModUp conversion split by arithmetic path; entries are
+// positions tt (0..n_rows-|D_j|-1) in the digit's output block.
+constexpr int kConvMaxInt = 32;
+struct ConvLists {
+    int n_fp, n_int;
+    uint8_t fp_tt[kConvMaxTargets];
+    uint8_t int_tt[kConvMaxInt];
+};
+
 // ModUp of digit j (NS source primes at rows s0..s0+NS-1), one launch per digit:
-//   ext_j[i][pos(t)][c] = sum_s [x_s qhat_inv_s]_{q_s} (qhat_s mod t)   (coefficient domain)
+//   ext_j[i][tt][c] = sum_s [x_s qhat_inv_s]_{q_s} (qhat_s mod t)   (coefficient domain)
 // for every target row t (all rows of Q_level and P outside the digit).
-//  - targets below 2^41: signed FP64 rounded-quotient products, one
-//    reduction at the end;
-//  - 60-bit targets, digit of 40-bit sources (narrow): with y = y1 2^21 + y0
+//  - targets below 2^41 (two per iteration): signed FP64 rounded-quotient
+//    products, one reduction at the end;
+//  - 60-bit targets, digit of 40-bit sources (NARROW): with y = y1 2^21 + y0
 //    (y0 < 2^21, y1 < 2^20) and the Montgomery-form entry m' = m2 2^42 +
 //    m1 2^21 + m0 (m0, m1 < 2^21, m2 < 2^18) the four sums
 //      V0 = S y0 m0, V1 = S y0 m1 + y1 m0, V2 = S y0 m2 + y1 m1, V3 = S y1 m2
 //    are exact doubles below 2^47 (NS <= 16); the 128-bit value
 //    V0 + V1 2^21 + V2 2^42 + V3 2^63 = S y m' is assembled on the integer
 //    pipe and one REDC gives S y m mod t;
-//  - 60-bit targets, digit with a 60-bit source: 128-bit accumulation of the
-//    NS products, one REDC.
-template <int NS>
+//  - 60-bit targets of a digit with a 60-bit source: 128-bit accumulation of
+//    the NS products, one REDC.
+template <int NS, bool NARROW>
 __global__ void __launch_bounds__(256)
     k_modup_conv(const uint64_t* __restrict__ coef, uint64_t* __restrict__ ext_j, const ulonglong2* __restrict__ src,
-                 const ulonglong2* __restrict__ mat, ModupArgs a, const DevPrime* __restrict__ pr,
-                 const FpMod* __restrict__ fpm, int level, int n_rows, int s0, int all_narrow, int logn) {
-    __shared__ uint64_t sm_m[NS * kConvMaxTargets];
-    __shared__ double sm_md[NS * kConvMaxTargets];
-    __shared__ double sm_m0[NS * kConvMaxTargets], sm_m1[NS * kConvMaxTargets], sm_m2[NS * kConvMaxTargets];
-    __shared__ ConvTarget sm_t[kConvMaxTargets];
-    __shared__ FpMod sm_f[kConvMaxTargets];
+                 const ulonglong2* __restrict__ mat, ModupArgs a, const __grid_constant__ ConvLists cl,
+                 const DevPrime* __restrict__ pr,
+                 const FpMod* __restrict__ fpm, int level, int n_rows, int s0, int logn) {
+    __shared__ double sm_fm[NS * kConvMaxTargets];  // [s][f]: FP64 targets in list order
+    __shared__ FpMod sm_ff[kConvMaxTargets];
+    __shared__ ConvTarget sm_ft[kConvMaxTargets];  // (wide sources: reduction into [0, 2t))
+    __shared__ double2 sm_i01[NARROW ? NS * kConvMaxInt : 1];
+    __shared__ double sm_i2[NARROW ? NS * kConvMaxInt : 1];
+    __shared__ uint64_t sm_im[NARROW ? 1 : NS * kConvMaxInt];
+    __shared__ ConvTarget sm_it[kConvMaxInt];
+    __shared__ int sm_ftt[kConvMaxTargets], sm_itt[kConvMaxInt];  // output rows, list order
     const int N = 1 << logn;
     const int n_tgt = n_rows - NS;
-    for (int idx = threadIdx.x; idx < NS * n_tgt; idx += blockDim.x) {
-        int s = idx / n_tgt, tt = idx - s * n_tgt;
-        int t = tt < s0 ? tt : tt + NS;
-        ulonglong2 m = mat[(size_t)s * n_rows + t];
-        const int o = s * kConvMaxTargets + tt;
-        sm_m[o] = m.x;
-        sm_md[o] = (double)m.y;  // exact: below 2^41 where it is used
-        sm_m0[o] = (double)(m.x & ((1ull << 21) - 1));
-        sm_m1[o] = (double)((m.x >> 21) & ((1ull << 21) - 1));
-        sm_m2[o] = (double)(m.x >> 42);
+    const int n_fp = cl.n_fp, n_int = cl.n_int;
+    for (int f = threadIdx.x; f < n_fp; f += blockDim.x) sm_ftt[f] = cl.fp_tt[f];
+    for (int g = threadIdx.x; g < n_int; g += blockDim.x) sm_itt[g] = cl.int_tt[g];
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < NS * n_fp; idx += blockDim.x) {
+        int s = idx / n_fp, f = idx - s * n_fp;
+        int tt = sm_ftt[f], t = tt < s0 ? tt : tt + NS;
+        sm_fm[s * kConvMaxTargets + f] = (double)mat[(size_t)s * n_rows + t].y;  // exact: below 2^41
     }
-    for (int tt = threadIdx.x; tt < n_tgt; tt += blockDim.x) {
-        int t = tt < s0 ? tt : tt + NS;
+    for (int idx = threadIdx.x; idx < NS * n_int; idx += blockDim.x) {
+        int s = idx / n_int, g = idx - s * n_int;
+        int tt = sm_itt[g], t = tt < s0 ? tt : tt + NS;
+        uint64_t m = mat[(size_t)s * n_rows + t].x;
+        if constexpr (NARROW) {
+            sm_i01[s * kConvMaxInt + g] =
+                make_double2((double)(m & ((1ull << 21) - 1)), (double)((m >> 21) & ((1ull << 21) - 1)));
+            sm_i2[s * kConvMaxInt + g] = (double)(m >> 42);
+        } else {
+            sm_im[s * kConvMaxInt + g] = m;
+        }
+    }
+    for (int f = threadIdx.x; f < n_fp; f += blockDim.x) {
+        int tt = sm_ftt[f], t = tt < s0 ? tt : tt + NS;
         DevPrime p = pr[a.tprime[t]];
-        sm_t[tt] = ConvTarget{p.q, p.qinv_neg, p.one_shoup, 0};
-        sm_f[tt] = fpm[a.tprime[t]];
+        sm_ff[f] = fpm[a.tprime[t]];
+        sm_ft[f] = ConvTarget{p.q, p.qinv_neg, p.one_shoup, 0};
+    }
+    for (int g = threadIdx.x; g < n_int; g += blockDim.x) {
+        int tt = sm_itt[g], t = tt < s0 ? tt : tt + NS;
+        DevPrime p = pr[a.tprime[t]];
+        sm_it[g] = ConvTarget{p.q, p.qinv_neg, p.one_shoup, 0};
     }
     __syncthreads();
     int c = blockIdx.x * blockDim.x + threadIdx.x;
     int i = blockIdx.y;
     if (c >= N) return;
     uint64_t y[NS];
-    double yd[NS];      // y as a double where the source prime is below 2^41
-    double y0[NS], y1[NS];
-    bool narrow[NS];
+    double yd[NS];  // y as a double (sources below 2^41)
 #pragma unroll
     for (int s = 0; s < NS; s++) {
         uint64_t q = pr[s0 + s].q;
         uint64_t x = coef[((size_t)i * level + s0 + s) * N + c];
         ulonglong2 w = src[s];
         y[s] = mul_shoup(x, w.x, w.y, q);
-        narrow[s] = q < kFpPrimeLimit;
-        yd[s] = u2d(narrow[s] ? y[s] : 0);
-        y0[s] = (double)(y[s] & ((1ull << 21) - 1));
-        y1[s] = (double)((y[s] >> 21) & ((1ull << 20) - 1));  // all of it when the digit is narrow
+        yd[s] = u2d(q < kFpPrimeLimit ? y[s] : 0);
     }
     uint64_t* o = ext_j + (size_t)i * n_tgt * N + c;
-    for (int tt = 0; tt < n_tgt; tt++) {
-        const ConvTarget t = sm_t[tt];
-        if (t.q < kFpPrimeLimit) {
-            const FpMod f = sm_f[tt];
-            double acc = 0.0;
+
+    // 60-bit targets
+    if constexpr (NARROW) {
+        double y0[NS], y1[NS];
 #pragma unroll
-            for (int s = 0; s < NS; s++) {
-                // a wide source residue first drops to [0, 2t)
-                double ys = narrow[s] ? yd[s] : u2d(y[s] - __umul64hi(y[s], t.one_shoup) * t.q);
-                acc = __dadd_rn(acc, fp_mulmod_s(ys, sm_md[s * kConvMaxTargets + tt], f));
-            }
-            o[(size_t)tt * N] = d2u(fp_canon(acc, f));
-        } else if (all_narrow) {
+        for (int s = 0; s < NS; s++) {
+            y0[s] = (double)(y[s] & ((1ull << 21) - 1));
+            y1[s] = (double)(y[s] >> 21);  // < 2^20
+        }
+        for (int g = 0; g < n_int; g++) {
             double v0 = 0, v1 = 0, v2 = 0, v3 = 0;
 #pragma unroll
             for (int s = 0; s < NS; s++) {
-                const int k = s * kConvMaxTargets + tt;
-                const double m0 = sm_m0[k], m1 = sm_m1[k], m2 = sm_m2[k];
-                v0 = __fma_rn(y0[s], m0, v0);
-                v1 = __fma_rn(y0[s], m1, __fma_rn(y1[s], m0, v1));
-                v2 = __fma_rn(y0[s], m2, __fma_rn(y1[s], m1, v2));
+                const double2 m01 = sm_i01[s * kConvMaxInt + g];
+                const double m2 = sm_i2[s * kConvMaxInt + g];
+                v0 = __fma_rn(y0[s], m01.x, v0);
+                v1 = __fma_rn(y0[s], m01.y, __fma_rn(y1[s], m01.x, v1));
+                v2 = __fma_rn(y0[s], m2, __fma_rn(y1[s], m01.y, v2));
                 v3 = __fma_rn(y1[s], m2, v3);
             }
             const uint64_t w0 = d2u(v0), w1 = d2u(v1), w2 = d2u(v2), w3 = d2u(v3);
@@ -179,13 +199,39 @@ __global__ void __launch_bounds__(256)
             add128(acc, w1 << 21, w1 >> 43);
             add128(acc, w2 << 42, w2 >> 22);
             add128(acc, w3 << 63, w3 >> 1);
-            o[(size_t)tt * N] = redc_t(acc, t);
-        } else {
+            o[(size_t)sm_itt[g] * N] = redc_t(acc, sm_it[g]);
+        }
+    } else {
+        for (int g = 0; g < n_int; g++) {
             U128 acc = {0, 0};
 #pragma unroll
-            for (int s = 0; s < NS; s++) mac128(acc, y[s], sm_m[s * kConvMaxTargets + tt]);
-            o[(size_t)tt * N] = redc_t(acc, t);
+            for (int s = 0; s < NS; s++) mac128(acc, y[s], sm_im[s * kConvMaxInt + g]);
+            o[(size_t)sm_itt[g] * N] = redc_t(acc, sm_it[g]);
         }
+    }
+
+    // targets below 2^41, two at a time
+    for (int f = 0; f < n_fp; f += 2) {
+        const bool two = f + 1 < n_fp;
+        const int f1 = two ? f + 1 : f;
+        const FpMod F0 = sm_ff[f], F1 = sm_ff[f1];
+        double acc0 = 0.0, acc1 = 0.0;
+#pragma unroll
+        for (int s = 0; s < NS; s++) {
+            double m0 = sm_fm[s * kConvMaxTargets + f], m1 = sm_fm[s * kConvMaxTargets + f1];
+            double y0 = yd[s], y1 = yd[s];
+            if constexpr (!NARROW) {
+                if (pr[s0 + s].q >= kFpPrimeLimit) {  // a wide source residue first drops to [0, 2t)
+                    const ConvTarget t0 = sm_ft[f], t1 = sm_ft[f1];
+                    y0 = u2d(y[s] - __umul64hi(y[s], t0.one_shoup) * t0.q);
+                    y1 = u2d(y[s] - __umul64hi(y[s], t1.one_shoup) * t1.q);
+                }
+            }
+            acc0 = __dadd_rn(acc0, fp_mulmod_s(y0, m0, F0));
+            acc1 = __dadd_rn(acc1, fp_mulmod_s(y1, m1, F1));
+        }
+        o[(size_t)sm_ftt[f] * N] = d2u(fp_canon(acc0, F0));
+        if (two) o[(size_t)sm_ftt[f1] * N] = d2u(fp_canon(acc1, F1));
     }
 }
 
@@ -536,21 +582,37 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     prof_begin(c, HE_PROF_MODUP);
     for (int j = 0; j < nd; j++) {
         uint64_t* ext_j = ext + (size_t)ma.ext_off[j] * n * N;
-        const int s0 = ma.src_row[j];
-        int narrow_j = 1;  // every source prime of the digit below 2^41
-        for (int s = 0; s < ma.n_src[j]; s++) narrow_j &= fp_prime(c, s0 + s);
-        switch (ma.n_src[j]) {
-#define HE_MU_CASE(S)                                                                                       \
-    case S:                                                                                                 \
-        k_modup_conv<S><<<dim3(gx, n), blk, 0, c->stream>>>(coef, ext_j, ma.src[j], ma.mat[j], ma, c->d_prime, \
-                                                            c->d_fpmod, level, n_rows, s0, narrow_j, c->log_n); \
+        const int s0 = ma.src_row[j], ns = ma.n_src[j];
+        bool narrow_j = true;  // every source prime of the digit below 2^41
+        for (int s = 0; s < ns; s++) narrow_j = narrow_j && fp_prime(c, s0 + s);
+        ConvLists cl;
+        cl.n_fp = cl.n_int = 0;
+        for (int tt = 0; tt < n_rows - ns; tt++) {
+            const int t = tt < s0 ? tt : tt + ns;
+            if (fp_prime(c, ep[t]))
+                cl.fp_tt[cl.n_fp++] = (uint8_t)tt;
+            else
+                cl.int_tt[cl.n_int++] = (uint8_t)tt;
+        }
+        if (cl.n_int > kConvMaxInt) return set_err(c, HE_EINVAL, "key switch: %d wide targets unsupported", cl.n_int);
+        switch (ns * 2 + (narrow_j ? 1 : 0)) {
+#define HE_MU_CASE(S)                                                                                             \
+    case 2 * S:                                                                                                   \
+        k_modup_conv<S, false><<<dim3(gx, n), blk, 0, c->stream>>>(coef, ext_j, ma.src[j], ma.mat[j], ma, cl,       \
+                                                                   c->d_prime, c->d_fpmod, level, n_rows, s0,     \
+                                                                   c->log_n);                                     \
+        break;                                                                                                    \
+    case 2 * S + 1:                                                                                               \
+        k_modup_conv<S, true><<<dim3(gx, n), blk, 0, c->stream>>>(coef, ext_j, ma.src[j], ma.mat[j], ma, cl,        \
+                                                                  c->d_prime, c->d_fpmod, level, n_rows, s0,      \
+                                                                  c->log_n);                                      \
         break;
             HE_MU_CASE(1) HE_MU_CASE(2) HE_MU_CASE(3) HE_MU_CASE(4) HE_MU_CASE(5) HE_MU_CASE(6) HE_MU_CASE(7)
             HE_MU_CASE(8) HE_MU_CASE(9) HE_MU_CASE(10) HE_MU_CASE(11) HE_MU_CASE(12) HE_MU_CASE(13)
             HE_MU_CASE(14) HE_MU_CASE(15) HE_MU_CASE(16)
 #undef HE_MU_CASE
             default:
-                return set_err(c, HE_EINVAL, "key switch: digit of %d primes unsupported", ma.n_src[j]);
+                return set_err(c, HE_EINVAL, "key switch: digit of %d primes unsupported", ns);
         }
         if ((rc = lc(c, "modup_conv"))) return rc;
     }
