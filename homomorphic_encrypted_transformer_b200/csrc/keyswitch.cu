@@ -251,53 +251,62 @@ __global__ void __launch_bounds__(256)
                int n_rows, int level, int L, int LK, int n_cts, const DevPrime* __restrict__ pr,
                const FpMod* __restrict__ fpm, ModupArgs a, int logn) {
     const int N = 1 << logn;
-    int i = blockIdx.x, t = blockIdx.z;
-    int c = blockIdx.y * blockDim.x + threadIdx.x;
+    const int i = blockIdx.x, t = blockIdx.z;
+    const int c = 2 * (blockIdx.y * blockDim.x + threadIdx.x);  // positions c, c+1
     if (c >= N) return;
     const uint64_t* key = keys.p[i];
-    const int own = automorph_src(c, logn, gal.g[i]);
+    const int own = automorph_src(c, logn, gal.g[i]);  // the pair maps onto {own & ~1, own | 1}
+    const bool own_sw = own & 1;
     const int krow = t < level ? t : L + (t - level);
     const int pidx = a.tprime[t];
     const DevPrime p = pr[pidx];
     const bool fp = p.q < kFpPrimeLimit;
-    uint64_t xs[ND], kbs[ND], kas[ND];
+    ulonglong2 xs[ND], kbs[ND], kas[ND];
 #pragma unroll
     for (int j = 0; j < ND; j++) {
         const int s0 = a.src_row[j], ns = a.n_src[j];
         if (t >= s0 && t < s0 + ns) {
-            xs[j] = __ldg(din.p[i] + (size_t)t * N + own);
+            const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2*>(din.p[i] + (size_t)t * N + (own & ~1)));
+            xs[j] = own_sw ? make_ulonglong2(v.y, v.x) : v;
         } else {
             int pos = t < s0 ? t : t - ns;
-            xs[j] = ext[((size_t)a.ext_off[j] * n_cts + (size_t)i * (n_rows - ns) + pos) * N + c];
+            xs[j] = __ldg(reinterpret_cast<const ulonglong2*>(
+                ext + ((size_t)a.ext_off[j] * n_cts + (size_t)i * (n_rows - ns) + pos) * N + c));
         }
-        kbs[j] = key[(((size_t)j * 2 + 0) * LK + krow) * N + c];
-        kas[j] = key[(((size_t)j * 2 + 1) * LK + krow) * N + c];
+        kbs[j] = __ldg(reinterpret_cast<const ulonglong2*>(key + (((size_t)j * 2 + 0) * LK + krow) * N + c));
+        kas[j] = __ldg(reinterpret_cast<const ulonglong2*>(key + (((size_t)j * 2 + 1) * LK + krow) * N + c));
     }
-    U128 acc0 = {0, 0}, acc1 = {0, 0};
-    double f0 = 0.0, f1 = 0.0;
-    const FpMod m = fpm[pidx];
+    ulonglong2 ob, oa;
     if (fp) {
+        const FpMod m = fpm[pidx];
+        double b0 = 0.0, b1 = 0.0, a0 = 0.0, a1 = 0.0;
 #pragma unroll
         for (int j = 0; j < ND; j++) {
-            const double xd = u2d(xs[j]);
-            f0 = __dadd_rn(f0, fp_mulmod_s(xd, __longlong_as_double((long long)kbs[j]), m));
-            f1 = __dadd_rn(f1, fp_mulmod_s(xd, __longlong_as_double((long long)kas[j]), m));
+            const double x0 = u2d(xs[j].x), x1 = u2d(xs[j].y);
+            b0 = __dadd_rn(b0, fp_mulmod_s(x0, __longlong_as_double((long long)kbs[j].x), m));
+            b1 = __dadd_rn(b1, fp_mulmod_s(x1, __longlong_as_double((long long)kbs[j].y), m));
+            a0 = __dadd_rn(a0, fp_mulmod_s(x0, __longlong_as_double((long long)kas[j].x), m));
+            a1 = __dadd_rn(a1, fp_mulmod_s(x1, __longlong_as_double((long long)kas[j].y), m));
         }
+        ob = make_ulonglong2(d2u(fp_canon(b0, m)), d2u(fp_canon(b1, m)));
+        oa = make_ulonglong2(d2u(fp_canon(a0, m)), d2u(fp_canon(a1, m)));
     } else {
+        U128 b0 = {0, 0}, b1 = {0, 0}, a0 = {0, 0}, a1 = {0, 0};
 #pragma unroll
         for (int j = 0; j < ND; j++) {
-            mac128(acc0, xs[j], kbs[j]);
-            mac128(acc1, xs[j], kas[j]);
+            mac128(b0, xs[j].x, kbs[j].x);
+            mac128(b1, xs[j].y, kbs[j].y);
+            mac128(a0, xs[j].x, kas[j].x);
+            mac128(a1, xs[j].y, kas[j].y);
         }
+        ob = make_ulonglong2(csub(redc_lazy(b0.hi, b0.lo, p.q, p.qinv_neg), p.q),
+                             csub(redc_lazy(b1.hi, b1.lo, p.q, p.qinv_neg), p.q));
+        oa = make_ulonglong2(csub(redc_lazy(a0.hi, a0.lo, p.q, p.qinv_neg), p.q),
+                             csub(redc_lazy(a1.hi, a1.lo, p.q, p.qinv_neg), p.q));
     }
     uint64_t* o = u + ((size_t)i * 2 * n_rows) * N + c;
-    if (fp) {
-        o[(size_t)t * N] = d2u(fp_canon(f0, m));
-        o[(size_t)(n_rows + t) * N] = d2u(fp_canon(f1, m));
-    } else {
-        o[(size_t)t * N] = csub(redc_lazy(acc0.hi, acc0.lo, p.q, p.qinv_neg), p.q);
-        o[(size_t)(n_rows + t) * N] = csub(redc_lazy(acc1.hi, acc1.lo, p.q, p.qinv_neg), p.q);
-    }
+    *reinterpret_cast<ulonglong2*>(o + (size_t)t * N) = ob;
+    *reinterpret_cast<ulonglong2*>(o + (size_t)(n_rows + t) * N) = oa;
 }
 
 // tmp[i][poly][r][c] = sum_k y'_k (P/p_k mod q_r), y_k = [x_k (P/p_k)^-1]_{p_k},
@@ -641,10 +650,11 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     }
 
     prof_begin(c, HE_PROF_KS_INNER);
+    const int gx2 = (N / 2 + TB - 1) / TB;  // two positions per thread
     switch (nd) {
 #define HE_KS_CASE(D)                                                                                             \
     case D:                                                                                                       \
-        k_ks_inner<D><<<dim3(n, gx, n_rows), blk, 0, c->stream>>>(ext, din, gal, keys, u, n_rows, level, L, LK, n, \
+        k_ks_inner<D><<<dim3(n, gx2, n_rows), blk, 0, c->stream>>>(ext, din, gal, keys, u, n_rows, level, L, LK, n, \
                                                                   c->d_prime, c->d_fpmod, ma, c->log_n);         \
         break;
         HE_KS_CASE(1) HE_KS_CASE(2) HE_KS_CASE(3) HE_KS_CASE(4) HE_KS_CASE(5) HE_KS_CASE(6) HE_KS_CASE(7)
