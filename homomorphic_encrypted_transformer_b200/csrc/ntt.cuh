@@ -385,6 +385,19 @@ __device__ __forceinline__ void row_load_strided(T (&x)[16], const uint64_t* row
     for (int k = 0; k < 16; k++) x[k] = raw_in(row[p + CS * k], T());
 }
 
+// Brings the twiddles of the last four stages of row r, which thread p uses
+// after the exchange, towards L1 while the first four stages run: one
+// prefetch per stage (its twiddles span at most 128 bytes, line-aligned).
+template <int LOGN, typename TW>
+__device__ __forceinline__ void prefetch_row_tw(const TW* tw, int r, int p) {
+    constexpr int S = NttCfg<LOGN>::S1 + 4, H = NttCfg<LOGN>::S2 - 4;
+#pragma unroll
+    for (int u = 0; u < H; u++) {
+        const TW* a = tw + (1 << (S + u)) + ((r << 4) << u) + ((16 * p) >> (H - u));
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(a));
+    }
+}
+
 // Forward row pass (stages S1..LOGN-1) on registers loaded from columns
 // p + CS k of row r; returns columns 16 p + k in [0, 4q).
 template <int LOGN, typename T, typename TW, typename M>
@@ -393,6 +406,7 @@ __device__ __forceinline__ void fwd_rows_core(T (&x)[16], T* sm, int r, const TW
     constexpr int CS = Cf::C / 16;
     const int p = threadIdx.x % CS, rr = threadIdx.x / CS;
     T* s = sm + rr * Cf::ROW_PITCH;
+    prefetch_row_tw<LOGN>(tw, r, p);
     fwd_stages<4>(x, tw, Cf::S1, r, 0, m);
 #pragma unroll
     for (int k = 0; k < 16; k++) s[padded(p + CS * k)] = x[k];
