@@ -46,9 +46,11 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--case", default="rotation", choices=["rotation", "ntt", "rot_small"],
-                    help="ntt / rot_small: kernel cases for profiler captures (no JSON metric line): "
-                         "NTT of 512 limbs, or 8 rotations with 2 keys")
+    ap.add_argument("--case", default="rotation",
+                    choices=["rotation", "ntt", "rot_small", "ffn128", "ffn2048", "ps15", "tiny"],
+                    help="rotation: the headline workload (default). ffn128 / ffn2048 / ps15 / tiny: the other "
+                         "workloads, one JSON line each. ntt / rot_small: kernel cases for profiler captures "
+                         "(NTT of 512 limbs, or 8 rotations with 2 keys)")
     return ap.parse_args()
 
 
@@ -233,6 +235,183 @@ def run_rot_small_case(args, local_rank):
     print(json.dumps({"case": "rot_small", "rotations": 8 * (args.warmup + args.steps)}))
 
 
+# ------------------------------------------------------------------ other workloads
+
+FFN = {"n_feat": 256, "n_tok": 128, "bs": 16, "gs": 16, "n_in": 3, "n_out": 12, "level": 12}
+
+
+def device_residues(torch, shape_lead, primes, N, gen, dev):
+    """Seeded uniform canonical residues generated on the device:
+    [*shape_lead][len(primes)][N] int64 (the kernels' work does not depend on
+    the values; parity tests use real encodings and encryptions)."""
+    t = torch.empty(tuple(shape_lead) + (len(primes), N), dtype=torch.int64, device=dev)
+    for r, q in enumerate(primes):
+        t[..., r, :] = torch.randint(0, int(q), tuple(shape_lead) + (N,), dtype=torch.int64, device=dev,
+                                     generator=gen)
+    return t
+
+
+def run_workload_case(args, local_rank):
+    """Throughput of the other workloads on one GPU, one JSON line each:
+    ffn128 (FFN1 768->3072, 128 tokens: 3 x 12 blocks by BSGS at level 12),
+    ffn2048 (the same product for 16 token groups sharing the weights),
+    ps15 (degree-15 Paterson-Stockmeyer on 64 ciphertexts from level 24),
+    tiny (N=2^12 NTT round trip, 3 rotations and one HMult-relin-rescale).
+    Inputs are seeded uniform residues on the device; the rotation and
+    relinearisation keys are computed by the library from seeded draws."""
+    import torch
+
+    from homomorphic_encrypted_transformer_b200 import he
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    case = args.case
+    widx = {"tiny": 0, "ffn128": 2, "ffn2048": 3, "ps15": 4}[case]
+    master = S.master_seed(widx)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(master)
+    if case == "tiny":
+        ctx = he.he_ctx_create(12, 3, 1, 3, stream=stream)
+    else:
+        ctx = he.he_ctx_create(LOG_N, L, K, DNUM, stream=stream)
+    N = ctx.N
+    s_key = S.secret(master, N)
+
+    def upload(kind, step):
+        kid = 2 if kind == he.HE_KEY_RELIN else pow(5, step % (N // 2), 2 * N)  # Galois elements are odd
+        a, e = S.key_draws(master, kid, ctx.primes, N, ctx.dnum)
+        he.he_keygen_upload(ctx, kind, step, s_key, a, e)
+
+    if case in ("ffn128", "ffn2048"):
+        f = FFN
+        n_groups = 1 if case == "ffn128" else 16
+        lvl = f["level"]
+        steps = sorted({f["n_tok"] * b for b in range(1, f["bs"])} |
+                       {f["n_tok"] * f["bs"] * g for g in range(1, f["gs"])})
+        for st in steps:
+            upload(he.HE_KEY_ROTATION, st)
+        pt = device_residues(torch, (f["n_out"], f["n_in"], f["gs"], f["bs"]), ctx.primes[:lvl], N, gen, dev)
+        x = device_residues(torch, (n_groups * f["n_in"], 2), ctx.primes[:lvl], N, gen, dev)
+        y = torch.empty((n_groups * f["n_out"], 2, lvl, N), dtype=torch.int64, device=dev)
+        xs = [he.Ciphertext(x[i], lvl, 2.0 ** 40) for i in range(n_groups * f["n_in"])]
+
+        def step():
+            ys = [he.Ciphertext(y[i], lvl, 2.0 ** 40) for i in range(n_groups * f["n_out"])]
+            he.he_pmult_accum_bsgs(ctx, xs, f["n_in"], pt, 2.0 ** 40, f["n_out"], f["bs"], f["gs"], f["n_tok"],
+                                   n_groups, ys)
+
+        metric, unit = ("FFN1 768->3072 products/s (128 tokens)" if n_groups == 1 else
+                        "FFN1 768->3072 products/s (2048 tokens, 16 groups)"), "products/s"
+        per_step = 1
+        cfg = {"workload": case, "N": N, "level": lvl, "tokens": f["n_tok"] * n_groups, "bs": f["bs"], "gs": f["gs"],
+               "rotations_per_step": n_groups * f["n_in"] * (f["bs"] - 1) + n_groups * f["n_out"] * (f["gs"] - 1),
+               "weights_gb": pt.numel() * 8 / 1e9}
+    elif case == "ps15":
+        upload(he.HE_KEY_RELIN, 0)
+        n = 64
+        coeffs = S.poly_coeffs(master, 15)
+        x = device_residues(torch, (n, 2), ctx.primes[:L], N, gen, dev)
+        y = torch.empty_like(x)
+        xs = [he.Ciphertext(x[i], L, 2.0 ** 40) for i in range(n)]
+
+        def step():
+            ys = [he.Ciphertext(y[i], L, 2.0 ** 40) for i in range(n)]
+            he.he_poly_eval_ps15(ctx, xs, coeffs, 2.0 ** 62, ys)
+
+        metric, unit, per_step = "degree-15 polynomial evaluations/s (64 ciphertexts, level 24)", "evals/s", n
+        cfg = {"workload": case, "N": N, "level": L, "n_ciphertexts": n, "hmrr_per_eval": 3 + 3}
+    else:
+        for st in (1, 2, -1):
+            upload(he.HE_KEY_ROTATION, st)
+        upload(he.HE_KEY_RELIN, 0)
+        x = device_residues(torch, (2,), ctx.primes, N, gen, dev)[:, :3].contiguous()
+        d = device_residues(torch, (1,), ctx.primes[:3], N, gen, dev)
+        r = torch.empty_like(x)
+        xc = he.Ciphertext(x, 3, 2.0 ** 40)
+
+        def step():
+            he.he_ntt_inv(ctx, d, 1, 3, 0)
+            he.he_ntt_fwd(ctx, d, 1, 3, 0)
+            for st in (1, 2, -1):
+                he.he_rotate(ctx, xc, st, he.Ciphertext(r, 3, 2.0 ** 40))
+            he.he_hmult_relin_rescale(ctx, xc, xc, he.Ciphertext(r, 3, 2.0 ** 40))
+
+        metric, unit, per_step = "tiny-config operation sequences/s (N=2^12)", "sequences/s", 1
+        cfg = {"workload": case, "N": N, "ops": "NTT round trip, 3 rotations, 1 HMult-relin-rescale"}
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    copy_gbs, int_modmul_s, fp_modmul_s = run_probes(he, ctx, dev, stream)
+    pk, pk_kind = peaks()
+    hbm_peak = float(pk.get("hbm_gbs", 6650.0))
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    clk = clocks.stop()
+    he.he_profile_enable(ctx, True)
+    for _ in range(args.steps):
+        step()
+    prof = {name: he.he_profile_read(ctx, cls) + (he.he_profile_read_fp(ctx, cls),) for name, cls in he.PROF.items()}
+    he.he_profile_enable(ctx, False)
+    dom = max(prof, key=lambda k: prof[k][0])
+    alu_ideal = sum(((v[3] - v[4]) / int_modmul_s + v[4] / fp_modmul_s) * 1e3 for v in prof.values()) / args.steps
+    line = {"case": case, "metric": metric, "value": per_step * args.steps / (ms * 1e-3), "unit": unit,
+            "ms_per_step": ms / args.steps, "steps": args.steps, "warmup": args.warmup, "n_gpus": 1,
+            "higher_is_better": True, "dtype": "u64", "data": "synthetic (seeded uniform residues, seeded keys)",
+            "config": cfg, "roofline": roofline_for(dom, prof[dom], int_modmul_s, fp_modmul_s, hbm_peak, pk_kind),
+            "alu_ideal_ms_per_step": alu_ideal,
+            "kernel_ms_per_step": {k: round(v[0] / args.steps, 4) for k, v in prof.items() if v[1]},
+            "kernel_roofline_frac": {k: round(roofline_for(k, v, int_modmul_s, fp_modmul_s, hbm_peak,
+                                                           pk_kind)["frac"], 3) for k, v in prof.items() if v[1]},
+            "probes": {"copy_gbs": copy_gbs, "int_shoup_modmul_per_s": int_modmul_s,
+                       "fp64_modmul_per_s": fp_modmul_s},
+            "clocks": clk}
+    print(json.dumps(line), flush=True)
+
+
+def run_probes(he, ctx, dev, stream):
+    """HBM copy, integer and FP64 modular-product probes in the same run:
+    (copy GB/s, integer products/s, FP64 products/s)."""
+    import torch
+
+    probe_words = 1 << 28  # 2 GiB each way
+    pa = torch.empty(probe_words, dtype=torch.int64, device=dev)
+    pb = torch.empty_like(pa)
+    pa.fill_(1)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    best = 1e9
+    for _ in range(5):
+        ev0.record(stream)
+        he.he_probe_copy(ctx, pb, pa, probe_words)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        best = min(best, ev0.elapsed_time(ev1))
+    copy_gbs = 2 * probe_words * 8 / (best * 1e-3) / 1e9
+    del pa, pb
+    sink = torch.empty(he.he_probe_int_threads(ctx), dtype=torch.int64, device=dev)
+    iters = 4096
+    rates = []
+    for fn in (he.he_probe_int, he.he_probe_fp):
+        best = 1e9
+        for _ in range(3):
+            ev0.record(stream)
+            fn(ctx, iters, sink)
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            best = min(best, ev0.elapsed_time(ev1))
+        rates.append(he.he_probe_int_threads(ctx) * iters * he.he_probe_int_mults_per_iter() / (best * 1e-3))
+    return copy_gbs, rates[0], rates[1]
+
+
 def run_native(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -270,39 +449,7 @@ def run_native(args, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
 
-    # HBM and integer probes in the same run
-    probe_words = 1 << 28  # 2 GiB each way
-    pa = torch.empty(probe_words, dtype=torch.int64, device=dev)
-    pb = torch.empty_like(pa)
-    pa.fill_(1)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    best = 1e9
-    for _ in range(5):
-        ev0.record(stream)
-        he.he_probe_copy(ctx, pb, pa, probe_words)
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        best = min(best, ev0.elapsed_time(ev1))
-    copy_gbs = 2 * probe_words * 8 / (best * 1e-3) / 1e9
-    del pa, pb
-    sink = torch.empty(he.he_probe_int_threads(ctx), dtype=torch.int64, device=dev)
-    iters = 4096
-    best = 1e9
-    for _ in range(3):
-        ev0.record(stream)
-        he.he_probe_int(ctx, iters, sink)
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        best = min(best, ev0.elapsed_time(ev1))
-    int_modmul_s = he.he_probe_int_threads(ctx) * iters * he.he_probe_int_mults_per_iter() / (best * 1e-3)
-    best = 1e9
-    for _ in range(3):
-        ev0.record(stream)
-        he.he_probe_fp(ctx, iters, sink)
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        best = min(best, ev0.elapsed_time(ev1))
-    fp_modmul_s = he.he_probe_int_threads(ctx) * iters * he.he_probe_int_mults_per_iter() / (best * 1e-3)
+    copy_gbs, int_modmul_s, fp_modmul_s = run_probes(he, ctx, dev, stream)
 
     # timed region (the headline number): K steps, no profiling events
     clocks = ClockSampler(local_rank)
@@ -459,6 +606,8 @@ def main():
             run_ntt_case(args, local_rank)
         elif args.case == "rot_small":
             run_rot_small_case(args, local_rank)
+        elif args.case in ("ffn128", "ffn2048", "ps15", "tiny"):
+            run_workload_case(args, local_rank)
         else:
             run_native(args, rank, world, local_rank)
     finally:

@@ -5,37 +5,136 @@
 #include <algorithm>
 
 #include "he_internal.h"
+#include "ntt.cuh"
 
 namespace he {
 
 int add_raw(he_ctx* c, const uint64_t* a, const uint64_t* b, uint64_t* out, int level);
 
-// Z[t][g][poly][r][c] = sum_{j,b} pt[i][j][g][b][r][c] * B[t][j][b][poly][r][c]
-// (128-bit accumulation, one reduction per output).  One thread per (r, c).
-__global__ void k_pmult_accum(const uint64_t* __restrict__ pt_i, const uint64_t* __restrict__ B,
-                              uint64_t* __restrict__ Z, int n_groups, int n_in, int gs, int bs, int level,
-                              const DevPrime* __restrict__ pr, int logn) {
+// Z[t][g][poly][r][c] = sum_{k < KB} pt[i][j][g][b][r][c] * B[t][k][poly][r][c],  k = j bs + b,
+// a small modular matrix product per coefficient ([g x k] weights times
+// [k x t] rotated inputs).  A block covers kPmCols columns of limb r and
+// kPmG giant steps; the rotated inputs of up to TCH token groups for those
+// columns are staged in shared memory once and read by all kPmG giant-step
+// warps, while each thread streams its own weights.  Limbs of primes below
+// 2^41 sum signed FP64 products (|.| < 5q/8 each, one reduction per output);
+// the others accumulate 128-bit products and reduce once.
+constexpr int kPmThreadsX = 32, kPmG = 8;
+
+// Element of the staged tile: the residue as a double (FP64 limbs) or as is.
+__device__ __forceinline__ void stage_put(uint64_t* dst, uint64_t v, bool fp) {
+    *dst = fp ? (uint64_t)__double_as_longlong(u2d(v)) : v;
+}
+
+// TCH token groups staged per pass, CPT adjacent columns per thread
+// (kPmThreadsX * CPT columns per block).
+template <int TCH, int CPT>
+__global__ void __launch_bounds__(kPmThreadsX* kPmG)
+    k_pmult_accum(const uint64_t* __restrict__ pt_i, const uint64_t* __restrict__ B, uint64_t* __restrict__ Z,
+                  int n_groups, int n_in, int gs, int bs, int level, const DevPrime* __restrict__ pr,
+                  const FpMod* __restrict__ fpm, int logn) {
+    constexpr int COLS = kPmThreadsX * CPT;
+    extern __shared__ uint64_t sB[];  // [TCH][KB][2][COLS]
     const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y;
-    if (c >= N) return;
+    const int KB = n_in * bs;
+    const int tx = threadIdx.x % kPmThreadsX, tg = threadIdx.x / kPmThreadsX;
+    // giant-step blocks of one column tile are neighbours: the second finds the tile in L2
+    const int c0 = blockIdx.y * COLS, r = blockIdx.z, g = blockIdx.x * kPmG + tg;
     const DevPrime p = pr[r];
+    const bool fp = p.q < kFpPrimeLimit;
+    const FpMod m = fpm[r];
     const size_t limb = (size_t)level * N, ctw = 2 * limb;
-    const size_t off = (size_t)r * N + c;
-    for (int g = 0; g < gs; g++) {
-        for (int t = 0; t < n_groups; t++) {
-            U128 a0 = {0, 0}, a1 = {0, 0};
-            for (int j = 0; j < n_in; j++) {
-                const uint64_t* ptj = pt_i + ((size_t)(j * gs + g) * bs) * limb + off;
-                const uint64_t* bj = B + ((size_t)(t * n_in + j) * bs) * ctw + off;
-                for (int b = 0; b < bs; b++) {
-                    uint64_t w = ptj[(size_t)b * limb];
-                    mac128(a0, w, bj[(size_t)b * ctw]);
-                    mac128(a1, w, bj[(size_t)b * ctw + limb]);
+    const size_t col = (size_t)r * N + c0;
+    for (int t0 = 0; t0 < n_groups; t0 += TCH) {
+        const int nt = min(TCH, n_groups - t0);
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < nt * KB * 2 * COLS; idx += blockDim.x) {
+            const int cc = idx % COLS, rest = idx / COLS;  // rest = (t KB + k) 2 + poly
+            const int poly = rest & 1, tk = rest >> 1, t = tk / KB, k = tk - t * KB;
+            stage_put(sB + idx, B[((size_t)(t0 + t) * KB + k) * ctw + poly * limb + col + cc], fp);
+        }
+        __syncthreads();
+        if (g >= gs) continue;
+        const uint64_t* w_g = pt_i + col + CPT * tx;
+        if (fp) {
+            double acc[TCH][2][CPT];
+#pragma unroll
+            for (int t = 0; t < TCH; t++)
+#pragma unroll
+                for (int e = 0; e < CPT; e++) acc[t][0][e] = acc[t][1][e] = 0.0;
+#pragma unroll 8
+            for (int k = 0; k < KB; k++) {
+                const int j = k / bs, b = k - j * bs;
+                const uint64_t* wp = w_g + ((size_t)(j * gs + g) * bs + b) * limb;
+                double w[CPT];
+                if constexpr (CPT == 2) {
+                    const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2*>(wp));
+                    w[0] = u2d(v.x);
+                    w[1] = u2d(v.y);
+                } else {
+                    w[0] = u2d(__ldg(wp));
+                }
+                const double* sk = reinterpret_cast<const double*>(sB) + (size_t)k * 2 * COLS + CPT * tx;
+#pragma unroll
+                for (int t = 0; t < TCH; t++) {
+                    if (t < nt) {
+                        const double* st = sk + (size_t)t * KB * 2 * COLS;
+#pragma unroll
+                        for (int e = 0; e < CPT; e++) {
+                            acc[t][0][e] = __dadd_rn(acc[t][0][e], fp_mulmod_s(w[e], st[e], m));
+                            acc[t][1][e] = __dadd_rn(acc[t][1][e], fp_mulmod_s(w[e], st[COLS + e], m));
+                        }
+                    }
                 }
             }
-            uint64_t* z = Z + (size_t)(t * gs + g) * ctw + off;
-            z[0] = reduce128(a0, p);
-            z[limb] = reduce128(a1, p);
+#pragma unroll
+            for (int t = 0; t < TCH; t++) {
+                if (t < nt) {
+                    uint64_t* z = Z + ((size_t)(t0 + t) * gs + g) * ctw + col + CPT * tx;
+#pragma unroll
+                    for (int e = 0; e < CPT; e++) {
+                        z[e] = d2u(fp_canon(acc[t][0][e], m));
+                        z[limb + e] = d2u(fp_canon(acc[t][1][e], m));
+                    }
+                }
+            }
+        } else {
+            U128 acc[TCH][2][CPT];
+#pragma unroll
+            for (int t = 0; t < TCH; t++)
+#pragma unroll
+                for (int e = 0; e < CPT; e++) acc[t][0][e] = acc[t][1][e] = U128{0, 0};
+#pragma unroll 4
+            for (int k = 0; k < KB; k++) {
+                const int j = k / bs, b = k - j * bs;
+                const uint64_t* wp = w_g + ((size_t)(j * gs + g) * bs + b) * limb;
+                uint64_t w[CPT];
+#pragma unroll
+                for (int e = 0; e < CPT; e++) w[e] = __ldg(wp + e);
+                const uint64_t* sk = sB + (size_t)k * 2 * COLS + CPT * tx;
+#pragma unroll
+                for (int t = 0; t < TCH; t++) {
+                    if (t < nt) {
+                        const uint64_t* st = sk + (size_t)t * KB * 2 * COLS;
+#pragma unroll
+                        for (int e = 0; e < CPT; e++) {
+                            mac128(acc[t][0][e], w[e], st[e]);
+                            mac128(acc[t][1][e], w[e], st[COLS + e]);
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < TCH; t++) {
+                if (t < nt) {
+                    uint64_t* z = Z + ((size_t)(t0 + t) * gs + g) * ctw + col + CPT * tx;
+#pragma unroll
+                    for (int e = 0; e < CPT; e++) {
+                        z[e] = reduce128(acc[t][0][e], p);
+                        z[limb + e] = reduce128(acc[t][1][e], p);
+                    }
+                }
+            }
         }
     }
 }
@@ -92,15 +191,35 @@ extern "C" int he_pmult_accum_bsgs(he_ctx* c, const he_ct* x, int n_in, const ui
         }
     if (!bin.empty() && (rc = rotate_many(c, bin.data(), bsteps.data(), bout.data(), (int)bin.size()))) return rc;
 
-    const int gx = (N + 255) / 256;
     const size_t pt_block = (size_t)n_in * gs * bs * level * N;
+    // one token group: 2 columns per thread; several: 4 groups staged per pass
+    const int tch = n_groups == 1 ? 1 : 4, cpt = n_groups == 1 ? 2 : 1;
+    const int smem = tch * n_in * bs * 2 * kPmThreadsX * cpt * 8;
+    if (smem > 200 * 1024) return set_err(c, HE_EINVAL, "he_pmult_accum_bsgs: n_in*bs = %d too large", n_in * bs);
+    const dim3 pgrid((gs + kPmG - 1) / kPmG, N / (kPmThreadsX * cpt), level);
     for (int i = 0; i < n_out; i++) {
         prof_begin(c, HE_PROF_PMULT);
-        k_pmult_accum<<<dim3(gx, level), 256, 0, c->stream>>>(d_pt + pt_block * i, B, Z, n_groups, n_in, gs, bs,
-                                                              level, c->d_prime, c->log_n);
+        if (tch == 1) {
+            cudaFuncSetAttribute(k_pmult_accum<1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            k_pmult_accum<1, 2><<<pgrid, kPmThreadsX * kPmG, smem, c->stream>>>(
+                d_pt + pt_block * i, B, Z, n_groups, n_in, gs, bs, level, c->d_prime, c->d_fpmod, c->log_n);
+        } else {
+            cudaFuncSetAttribute(k_pmult_accum<4, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            k_pmult_accum<4, 1><<<pgrid, kPmThreadsX * kPmG, smem, c->stream>>>(
+                d_pt + pt_block * i, B, Z, n_groups, n_in, gs, bs, level, c->d_prime, c->d_fpmod, c->log_n);
+        }
         c->launches++;
         if ((rc = check_cuda(c, cudaGetLastError(), "pmult_accum"))) return rc;
-        prof_end(c, HE_PROF_PMULT);
+        // weights of block i once per staged pass of token groups, the rotated
+        // inputs once, the sums written once
+        {
+            const double passes = (n_groups + tch - 1) / tch;
+            int fp_l = 0;
+            for (int r = 0; r < level; r++) fp_l += fp_prime(c, r);
+            const double macs_per_limb = 2.0 * N * (double)gs * n_groups * n_in * bs;
+            prof_end(c, HE_PROF_PMULT, 8.0 * ((double)pt_block * passes + (double)ctw * nB + (double)ctw * nZ),
+                     macs_per_limb * level, macs_per_limb * fp_l);
+        }
         // giant steps
         std::vector<he_ct> gin, gout;
         std::vector<int32_t> gsteps;
