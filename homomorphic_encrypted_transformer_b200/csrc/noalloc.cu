@@ -28,9 +28,19 @@ namespace he {
 
 __global__ void k_rescale_lift(const uint64_t* __restrict__ last, uint64_t* __restrict__ out, int lm1, uint64_t ql,
                                const uint64_t* __restrict__ qmod, const DevPrime* __restrict__ pr, int logn);
-__global__ void k_rescale_combine(const uint64_t* __restrict__ in, const uint64_t* __restrict__ lift,
-                                  uint64_t* __restrict__ out, int level, const ulonglong2* __restrict__ qinv,
-                                  const DevPrime* __restrict__ pr, int logn);
+
+// out[r] = (in[r] - lift[r]) q_l^-1 for the limbs of one chunk (pointers and
+// tables offset to the chunk's first limb)
+__global__ void k_noalloc_combine(const uint64_t* __restrict__ in, const uint64_t* __restrict__ lift,
+                                  uint64_t* __restrict__ out, const ulonglong2* __restrict__ qinv,
+                                  const DevPrime* __restrict__ pr, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y;
+    if (c >= N) return;
+    const uint64_t q = pr[r].q;
+    const ulonglong2 w = qinv[r];
+    out[(size_t)r * N + c] = mul_shoup(in[(size_t)r * N + c] + q - lift[(size_t)r * N + c], w.x, w.y, q);
+}
 
 static __device__ __align__(256) uint64_t g_noalloc_scratch[HE_NOALLOC_SCRATCH_WORDS];
 
@@ -100,8 +110,8 @@ extern "C" int he_rescale_noalloc(he_ctx* c, const he_ct* in, he_ct* out) {
             c->launches++;
             if ((rc = check_cuda(c, cudaGetLastError(), "he_rescale_noalloc: lift"))) return rc;
             if ((rc = ntt_fwd_set(c, rowset_contig(lift, m, N, prime_range(i0, m)), m))) return rc;
-            k_rescale_combine<<<dim3(gx, m, 1), 256, 0, c->stream>>>(
-                in->data + ((size_t)poly * level + i0) * N, lift, out->data + ((size_t)poly * lm1 + i0) * N, level,
+            k_noalloc_combine<<<dim3(gx, m, 1), 256, 0, c->stream>>>(
+                in->data + ((size_t)poly * level + i0) * N, lift, out->data + ((size_t)poly * lm1 + i0) * N,
                 c->d_rs_inv + (size_t)lm1 * c->L + i0, c->d_prime + i0, c->log_n);
             c->launches++;
             if ((rc = check_cuda(c, cudaGetLastError(), "he_rescale_noalloc: combine"))) return rc;

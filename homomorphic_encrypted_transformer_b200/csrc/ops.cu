@@ -89,12 +89,107 @@ __global__ void k_key_canonical(const uint64_t* __restrict__ in, uint64_t* __res
     out[k] = p.q < kFpPrimeLimit ? (uint64_t)__longlong_as_double((long long)in[k]) : mont_mul(in[k], 1, p);
 }
 
-// d[i] = (a0 b0, a0 b1 + a1 b0, a1 b1), each [level][N]
-__global__ void k_tensor(const uint64_t* __restrict__ a, const uint64_t* __restrict__ b, uint64_t* __restrict__ d,
-                         int level, const DevPrime* __restrict__ pr, int logn) {
+
+// Rescale, step 1 (batched): last[i][poly] = in_i[poly][level-1] (still in the
+// evaluation domain; an inverse NTT follows).
+__global__ void k_rescale_gather_last(PtrList in, uint64_t* __restrict__ last, int level, int logn) {
     const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y;
+    int c = blockIdx.x * blockDim.x + threadIdx.x, poly = blockIdx.y, i = blockIdx.z;
     if (c >= N) return;
+    last[((size_t)i * 2 + poly) * N + c] = in.p[i][((size_t)poly * level + level - 1) * N + c];
+}
+
+// Rescale, step 2: the centred last limb x (coefficients mod q_l) onto every
+// q_r, r < l: lift[i][poly][r] = [x]_{q_r} - (x > q_l/2 ? q_l : 0).
+__global__ void k_rescale_lift(const uint64_t* __restrict__ last, uint64_t* __restrict__ lift, int lm1, uint64_t ql,
+                               const uint64_t* __restrict__ qmod, const DevPrime* __restrict__ pr, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y, ip = blockIdx.z;  // ip = i 2 + poly
+    if (c >= N) return;
+    uint64_t x = last[(size_t)ip * N + c];
+    DevPrime p = pr[r];
+    uint64_t v = reduce64(x, p);
+    if (x > (ql >> 1)) v = sub_mod(v, qmod[r], p.q);  // x - q_l
+    lift[((size_t)ip * lm1 + r) * N + c] = v;
+}
+
+// Rescale, step 3: out_i[poly][r] = (in_i[poly][r] - lift[i][poly][r]) q_l^-1.
+// out_i = in_i is not allowed here (the limb shift of c1 would overwrite
+// unread input); callers route in-place rescales through a staging buffer.
+__global__ void k_rescale_combine(PtrList in, const uint64_t* __restrict__ lift, MutPtrList out, int level,
+                                  const ulonglong2* __restrict__ qinv, const DevPrime* __restrict__ pr, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y, ip = blockIdx.z;
+    if (c >= N) return;
+    const int lm1 = level - 1, i = ip >> 1, poly = ip & 1;
+    uint64_t q = pr[r].q;
+    uint64_t x = in.p[i][((size_t)poly * level + r) * N + c];
+    uint64_t y = lift[((size_t)ip * lm1 + r) * N + c];
+    ulonglong2 w = qinv[r];
+    out.p[i][((size_t)poly * lm1 + r) * N + c] = mul_shoup(x + q - y, w.x, w.y, q);
+}
+
+// dst_i[k] = src_i[k], k < words (16-byte copies)
+__global__ void k_copy_many(PtrList src, MutPtrList dst, size_t words2) {
+    const int i = blockIdx.y;
+    const ulonglong2* s = reinterpret_cast<const ulonglong2*>(src.p[i]);
+    ulonglong2* d = reinterpret_cast<ulonglong2*>(dst.p[i]);
+    for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < words2; k += (size_t)gridDim.x * blockDim.x)
+        d[k] = s[k];
+}
+
+
+
+
+// Batched helpers over n <= kMaxBatch ciphertexts (grid z = ciphertext).
+// out_i[poly][r] = K_r in_i[poly][r] for r < lv, in_i at level lin >= lv
+// (limbs lv..lin-1 dropped on the way).
+__global__ void k_mul_const_many(PtrList in, MutPtrList out, RowConst kc, int lin, int lv,
+                                 const DevPrime* __restrict__ pr, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x, y = blockIdx.y, i = blockIdx.z;
+    if (c >= N) return;
+    const int poly = y / lv, r = y - poly * lv;
+    const uint64_t x = in.p[i][((size_t)poly * lin + r) * N + c];
+    out.p[i][((size_t)poly * lv + r) * N + c] = mul_shoup(x, kc.v[r].x, kc.v[r].y, pr[r].q);
+}
+
+// out_i = in_i keeping limbs r < lv of both polynomials (out_i != in_i)
+__global__ void k_drop_many(PtrList in, MutPtrList out, int lin, int lv, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x, y = blockIdx.y, i = blockIdx.z;
+    if (c >= N) return;
+    const int poly = y / lv, r = y - poly * lv;
+    out.p[i][((size_t)poly * lv + r) * N + c] = in.p[i][((size_t)poly * lin + r) * N + c];
+}
+
+// o_i = a_i + b_i (level lv)
+__global__ void k_add_many(PtrList a, PtrList b, MutPtrList o, int lv, const DevPrime* __restrict__ pr, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x, y = blockIdx.y, i = blockIdx.z;
+    if (c >= N) return;
+    const size_t k = (size_t)y * N + c;
+    o.p[i][k] = add_mod(a.p[i][k], b.p[i][k], pr[y % lv].q);
+}
+
+// c0 of io_i gains the constant polynomial K (every evaluation equals K)
+__global__ void k_add_const_many(MutPtrList io, RowConst kc, const DevPrime* __restrict__ pr, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y, i = blockIdx.z;
+    if (c >= N) return;
+    uint64_t* a = io.p[i] + (size_t)r * N + c;
+    *a = add_mod(*a, kc.v[r].x, pr[r].q);
+}
+
+// d_i = (a0 b0, a0 b1 + a1 b0, a1 b1) of the pairs (a_i, b_i), [3][level][N]
+__global__ void k_tensor_many(PtrList pa, PtrList pb, MutPtrList pd, int level, const DevPrime* __restrict__ pr,
+                              int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y, i = blockIdx.z;
+    if (c >= N) return;
+    const uint64_t* a = pa.p[i];
+    const uint64_t* b = pb.p[i];
+    uint64_t* d = pd.p[i];
     DevPrime p = pr[r];
     size_t k0 = (size_t)r * N + c, k1 = (size_t)(level + r) * N + c;
     uint64_t a0 = a[k0], a1 = a[k1], b0 = b[k0], b1 = b[k1];
@@ -105,64 +200,6 @@ __global__ void k_tensor(const uint64_t* __restrict__ a, const uint64_t* __restr
     d[k0] = mont_mul(m00, p.r2, p);
     d[(size_t)(level + r) * N + c] = mont_mul(add_mod(m01, m10, p.q), p.r2, p);
     d[(size_t)(2 * level + r) * N + c] = mont_mul(m11, p.r2, p);
-}
-
-// Rescale, step 1: lift the (inverse-transformed) last limb x (coefficients
-// mod q_l, l = level-1) to every q_i, i < l, as its centred representative.
-__global__ void k_rescale_lift(const uint64_t* __restrict__ last, uint64_t* __restrict__ out, int lm1, uint64_t ql,
-                               const uint64_t* __restrict__ qmod, const DevPrime* __restrict__ pr, int logn) {
-    const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y, poly = blockIdx.z;  // r < lm1
-    if (c >= N) return;
-    uint64_t x = last[(size_t)poly * N + c];
-    DevPrime p = pr[r];
-    uint64_t v = reduce64(x, p);
-    if (x > (ql >> 1)) v = sub_mod(v, qmod[r], p.q);  // x - q_l
-    out[((size_t)poly * lm1 + r) * N + c] = v;
-}
-
-// Rescale, step 2: out[poly][r] = (in[poly][r] - lift[poly][r]) q_l^-1
-__global__ void k_rescale_combine(const uint64_t* __restrict__ in, const uint64_t* __restrict__ lift,
-                                  uint64_t* __restrict__ out, int level, const ulonglong2* __restrict__ qinv,
-                                  const DevPrime* __restrict__ pr, int logn) {
-    const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y, poly = blockIdx.z;
-    if (c >= N) return;
-    const int lm1 = level - 1;
-    uint64_t q = pr[r].q;
-    uint64_t x = in[((size_t)poly * level + r) * N + c];
-    uint64_t y = lift[((size_t)poly * lm1 + r) * N + c];
-    ulonglong2 w = qinv[r];
-    out[((size_t)poly * lm1 + r) * N + c] = mul_shoup(x + q - y, w.x, w.y, q);
-}
-
-__global__ void k_add_ct(const uint64_t* __restrict__ a, const uint64_t* __restrict__ b, uint64_t* __restrict__ o,
-                         int level, const DevPrime* __restrict__ pr, int logn) {
-    const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y;  // r < 2 level
-    if (c >= N) return;
-    uint64_t q = pr[r % level].q;
-    size_t k = (size_t)r * N + c;
-    o[k] = add_mod(a[k], b[k], q);
-}
-
-__global__ void k_mul_const(const uint64_t* __restrict__ a, uint64_t* __restrict__ o, RowConst kc, int level,
-                            const DevPrime* __restrict__ pr, int logn) {
-    const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y;
-    if (c >= N) return;
-    int rr = r % level;
-    uint64_t q = pr[rr].q;
-    size_t k = (size_t)r * N + c;
-    o[k] = mul_shoup(a[k], kc.v[rr].x, kc.v[rr].y, q);
-}
-
-__global__ void k_add_const(uint64_t* __restrict__ a, RowConst kc, const DevPrime* __restrict__ pr, int logn) {
-    const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y;  // rows of c0
-    if (c >= N) return;
-    size_t k = (size_t)r * N + c;
-    a[k] = add_mod(a[k], kc.v[r].x, pr[r].q);
 }
 
 // --------------------------------------------------------------- host side
@@ -192,41 +229,55 @@ static int ct_ok(he_ctx* c, const he_ct* x, const char* what) {
 int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int level) {
     const int N = c->N, n = (int)in.size(), lm1 = level - 1;
     if (level < 2) return set_err(c, HE_ELEVEL, "rescale: level %d has no prime to drop", level);
-    uint64_t* base;
-    // per ciphertext: last limbs [2][N], lifts [2][lm1][N], output [2][lm1][N]
-    size_t per = (size_t)N * (2 + 4 * lm1);
-    int rc = scratch_slot(c, 1, per * n, &base);
-    if (rc) return rc;
     const int gx = (N + TB - 1) / TB;
     const uint64_t ql = c->primes[level - 1];
-    for (int i = 0; i < n; i++) {
-        uint64_t* last = base + per * i;
-        uint64_t* lift = last + 2 * N;
-        uint64_t* res = lift + (size_t)2 * lm1 * N;
-        for (int poly = 0; poly < 2; poly++) {
-            rc = check_cuda(c, cudaMemcpyAsync(last + (size_t)poly * N, in[i] + ((size_t)poly * level + lm1) * N,
-                                               (size_t)N * 8, cudaMemcpyDeviceToDevice, c->stream), "rescale copy");
-            if (rc) return rc;
+    const double limbB = 8.0 * N;
+    for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
+        const int m = std::min(kMaxBatch, n - i0);
+        // per ciphertext: last limbs [2][N], lifts [2][lm1][N], staging of in-place outputs [2][lm1][N]
+        const size_t per = (size_t)N * (2 + 4 * lm1);
+        uint64_t* base;
+        int rc = scratch_slot(c, 1, per * m, &base);
+        if (rc) return rc;
+        uint64_t* last = base;
+        uint64_t* lift = last + (size_t)2 * m * N;
+        uint64_t* stage = lift + (size_t)2 * m * lm1 * N;
+        PtrList pin, sback;
+        MutPtrList pout, dback;
+        int n_back = 0;
+        for (int i = 0; i < m; i++) {
+            pin.p[i] = in[i0 + i];
+            const bool inplace = out[i0 + i] == in[i0 + i];
+            pout.p[i] = inplace ? stage + (size_t)i * 2 * lm1 * N : out[i0 + i];
+            if (inplace) {
+                sback.p[n_back] = pout.p[i];
+                dback.p[n_back++] = out[i0 + i];
+            }
         }
+        prof_begin(c, HE_PROF_RESCALE);
+        k_rescale_gather_last<<<dim3(gx, 2, m), TB, 0, c->stream>>>(pin, last, level, c->log_n);
+        if ((rc = lc(c, "rescale_gather"))) return rc;
+        prof_end(c, HE_PROF_RESCALE, 4.0 * m * limbB);
         std::vector<int> pl(1, level - 1);
-        if ((rc = ntt_inv_set(c, rowset_contig(last, 1, N, pl), 2))) return rc;
+        if ((rc = ntt_inv_set(c, rowset_contig(last, 1, N, pl), 2 * m))) return rc;
         prof_begin(c, HE_PROF_RESCALE);
-        k_rescale_lift<<<dim3(gx, lm1, 2), TB, 0, c->stream>>>(last, lift, lm1, ql, c->d_rs_qmod + (size_t)lm1 * c->L,
-                                                               c->d_prime, c->log_n);
+        k_rescale_lift<<<dim3(gx, lm1, 2 * m), TB, 0, c->stream>>>(last, lift, lm1, ql,
+                                                                   c->d_rs_qmod + (size_t)lm1 * c->L, c->d_prime,
+                                                                   c->log_n);
         if ((rc = lc(c, "rescale_lift"))) return rc;
-        prof_end(c, HE_PROF_RESCALE);
-        if ((rc = ntt_fwd_set(c, rowset_contig(lift, lm1, N, prime_range(0, lm1)), 2 * lm1))) return rc;
-        uint64_t* dst = (out[i] == in[i]) ? res : out[i];
+        prof_end(c, HE_PROF_RESCALE, (2.0 * m + 2.0 * m * lm1) * limbB, 2.0 * m * lm1 * N);
+        if ((rc = ntt_fwd_set(c, rowset_contig(lift, lm1, N, prime_range(0, lm1)), 2 * m * lm1))) return rc;
         prof_begin(c, HE_PROF_RESCALE);
-        k_rescale_combine<<<dim3(gx, lm1, 2), TB, 0, c->stream>>>(in[i], lift, dst, level,
-                                                                  c->d_rs_inv + (size_t)lm1 * c->L, c->d_prime,
-                                                                  c->log_n);
+        k_rescale_combine<<<dim3(gx, lm1, 2 * m), TB, 0, c->stream>>>(pin, lift, pout, level,
+                                                                      c->d_rs_inv + (size_t)lm1 * c->L, c->d_prime,
+                                                                      c->log_n);
         if ((rc = lc(c, "rescale_combine"))) return rc;
-        prof_end(c, HE_PROF_RESCALE);
-        if (dst != out[i]) {
-            rc = check_cuda(c, cudaMemcpyAsync(out[i], dst, (size_t)2 * lm1 * N * 8, cudaMemcpyDeviceToDevice,
-                                               c->stream), "rescale copy back");
-            if (rc) return rc;
+        prof_end(c, HE_PROF_RESCALE, 6.0 * m * lm1 * limbB, 2.0 * m * lm1 * N);
+        if (n_back) {
+            prof_begin(c, HE_PROF_RESCALE);
+            k_copy_many<<<dim3(c->sm_count * 4, n_back), TB, 0, c->stream>>>(sback, dback, (size_t)lm1 * N);
+            if ((rc = lc(c, "rescale_copy"))) return rc;
+            prof_end(c, HE_PROF_RESCALE, 4.0 * n_back * lm1 * limbB);
         }
     }
     return HE_OK;
@@ -247,12 +298,19 @@ int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vecto
         int rc = scratch_slot(c, 2, per * m, &base);
         if (rc) return rc;
         KsIoList io;
+        PtrList pa, pb;
+        MutPtrList pd;
+        for (int i = 0; i < m; i++) {
+            pa.p[i] = a[i0 + i];
+            pb.p[i] = b[i0 + i];
+            pd.p[i] = base + per * i;
+        }
+        prof_begin(c, HE_PROF_ELEMENTWISE);
+        k_tensor_many<<<dim3(gx, level, m), TB, 0, c->stream>>>(pa, pb, pd, level, c->d_prime, c->log_n);
+        if ((rc = lc(c, "tensor"))) return rc;
+        prof_end(c, HE_PROF_ELEMENTWISE, 7.0 * m * level * 8.0 * N, 7.0 * m * level * N);
         for (int i = 0; i < m; i++) {
             uint64_t* d = base + per * i;
-            prof_begin(c, HE_PROF_ELEMENTWISE);
-            k_tensor<<<dim3(gx, level), TB, 0, c->stream>>>(a[i0 + i], b[i0 + i], d, level, c->d_prime, c->log_n);
-            if ((rc = lc(c, "tensor"))) return rc;
-            prof_end(c, HE_PROF_ELEMENTWISE);
             io.galois.push_back(0);
             io.key.push_back(c->relin.d);
             io.d.push_back(d + (size_t)2 * level * N);
@@ -268,54 +326,121 @@ int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vecto
     return HE_OK;
 }
 
-int mul_const_raw(he_ctx* c, const uint64_t* in, uint64_t* out, int level, int64_t K) {
+// ---- batched helpers: n ciphertexts, kMaxBatch per launch
+
+static RowConst row_const_shoup(const he_ctx* c, int level, int64_t K) {
     RowConst kc;
     for (int r = 0; r < level; r++) {
         uint64_t q = c->primes[r], v = int_mod(K, q);
         kc.v[r] = make_ulonglong2(v, h_shoup(v, q));
     }
-    prof_begin(c, HE_PROF_ELEMENTWISE);
-    k_mul_const<<<dim3((c->N + TB - 1) / TB, 2 * level), TB, 0, c->stream>>>(in, out, kc, level, c->d_prime,
-                                                                             c->log_n);
-    int rc = lc(c, "mul_const");
-    prof_end(c, HE_PROF_ELEMENTWISE);
-    return rc;
+    return kc;
 }
 
-int add_const_raw(he_ctx* c, uint64_t* inout, int level, int64_t K) {
-    RowConst kc;
-    for (int r = 0; r < level; r++) kc.v[r] = make_ulonglong2(int_mod(K, c->primes[r]), 0);
-    prof_begin(c, HE_PROF_ELEMENTWISE);
-    k_add_const<<<dim3((c->N + TB - 1) / TB, level), TB, 0, c->stream>>>(inout, kc, c->d_prime, c->log_n);
-    int rc = lc(c, "add_const");
-    prof_end(c, HE_PROF_ELEMENTWISE);
-    return rc;
+// out_i = K in_i at level lv (in_i at level lin >= lv; out_i may equal in_i only when lin == lv)
+int mul_const_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int lin,
+                   int lv, int64_t K) {
+    const RowConst kc = row_const_shoup(c, lv, K);
+    const int n = (int)in.size(), gx = (c->N + TB - 1) / TB;
+    for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
+        const int m = std::min(kMaxBatch, n - i0);
+        PtrList pi;
+        MutPtrList po;
+        for (int i = 0; i < m; i++) {
+            pi.p[i] = in[i0 + i];
+            po.p[i] = out[i0 + i];
+        }
+        prof_begin(c, HE_PROF_ELEMENTWISE);
+        k_mul_const_many<<<dim3(gx, 2 * lv, m), TB, 0, c->stream>>>(pi, po, kc, lin, lv, c->d_prime, c->log_n);
+        int rc = lc(c, "mul_const");
+        if (rc) return rc;
+        prof_end(c, HE_PROF_ELEMENTWISE, 4.0 * m * lv * 8.0 * c->N, 2.0 * m * lv * c->N);
+    }
+    return HE_OK;
 }
+
+// out_i = in_i keeping limbs < lv (out_i != in_i)
+int drop_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int lin, int lv) {
+    const int n = (int)in.size(), gx = (c->N + TB - 1) / TB;
+    for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
+        const int m = std::min(kMaxBatch, n - i0);
+        PtrList pi;
+        MutPtrList po;
+        for (int i = 0; i < m; i++) {
+            pi.p[i] = in[i0 + i];
+            po.p[i] = out[i0 + i];
+        }
+        prof_begin(c, HE_PROF_ELEMENTWISE);
+        k_drop_many<<<dim3(gx, 2 * lv, m), TB, 0, c->stream>>>(pi, po, lin, lv, c->log_n);
+        int rc = lc(c, "drop");
+        if (rc) return rc;
+        prof_end(c, HE_PROF_ELEMENTWISE, 4.0 * m * lv * 8.0 * c->N);
+    }
+    return HE_OK;
+}
+
+// o_i = a_i + b_i at level lv (o_i may equal a_i or b_i)
+int add_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector<const uint64_t*>& b,
+             const std::vector<uint64_t*>& o, int lv) {
+    const int n = (int)a.size(), gx = (c->N + TB - 1) / TB;
+    for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
+        const int m = std::min(kMaxBatch, n - i0);
+        PtrList pa, pb;
+        MutPtrList po;
+        for (int i = 0; i < m; i++) {
+            pa.p[i] = a[i0 + i];
+            pb.p[i] = b[i0 + i];
+            po.p[i] = o[i0 + i];
+        }
+        prof_begin(c, HE_PROF_ELEMENTWISE);
+        k_add_many<<<dim3(gx, 2 * lv, m), TB, 0, c->stream>>>(pa, pb, po, lv, c->d_prime, c->log_n);
+        int rc = lc(c, "add");
+        if (rc) return rc;
+        prof_end(c, HE_PROF_ELEMENTWISE, 6.0 * m * lv * 8.0 * c->N);
+    }
+    return HE_OK;
+}
+
+// io_i gains K/scale in every slot: K added to c0's constant polynomial
+int add_const_many(he_ctx* c, const std::vector<uint64_t*>& io, int lv, int64_t K) {
+    RowConst kc;
+    for (int r = 0; r < lv; r++) kc.v[r] = make_ulonglong2(int_mod(K, c->primes[r]), 0);
+    const int n = (int)io.size(), gx = (c->N + TB - 1) / TB;
+    for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
+        const int m = std::min(kMaxBatch, n - i0);
+        MutPtrList po;
+        for (int i = 0; i < m; i++) po.p[i] = io[i0 + i];
+        prof_begin(c, HE_PROF_ELEMENTWISE);
+        k_add_const_many<<<dim3(gx, lv, m), TB, 0, c->stream>>>(po, kc, c->d_prime, c->log_n);
+        int rc = lc(c, "add_const");
+        if (rc) return rc;
+        prof_end(c, HE_PROF_ELEMENTWISE, 2.0 * m * lv * 8.0 * c->N);
+    }
+    return HE_OK;
+}
+
+int mul_const_raw(he_ctx* c, const uint64_t* in, uint64_t* out, int level, int64_t K) {
+    return mul_const_many(c, {in}, {out}, level, level, K);
+}
+
+int add_const_raw(he_ctx* c, uint64_t* inout, int level, int64_t K) { return add_const_many(c, {inout}, level, K); }
 
 int add_raw(he_ctx* c, const uint64_t* a, const uint64_t* b, uint64_t* out, int level) {
-    prof_begin(c, HE_PROF_ELEMENTWISE);
-    k_add_ct<<<dim3((c->N + TB - 1) / TB, 2 * level), TB, 0, c->stream>>>(a, b, out, level, c->d_prime, c->log_n);
-    int rc = lc(c, "add");
-    prof_end(c, HE_PROF_ELEMENTWISE);
-    return rc;
+    return add_many(c, {a}, {b}, {out}, level);
 }
 
 // Keep limbs 0..new_level-1 of both polynomials: out = [2][new_level][N].
 int drop_raw(he_ctx* c, const uint64_t* in, int level, uint64_t* out, int new_level) {
     const size_t N = c->N;
-    int rc;
-    if (out != in) {
-        rc = check_cuda(c, cudaMemcpyAsync(out, in, new_level * N * 8, cudaMemcpyDeviceToDevice, c->stream), "drop");
-        if (rc) return rc;
-    }
-    if (out != in || new_level != level) {
-        // c1 rows move from offset level*N to new_level*N; ascending row copies never
-        // overwrite a source row that is still to be read (the shift is >= one row).
-        for (int r = 0; r < new_level; r++) {
-            rc = check_cuda(c, cudaMemcpyAsync(out + (new_level + r) * N, in + (level + r) * N, N * 8,
+    if (out != in) return drop_many(c, {in}, {out}, level, new_level);
+    if (new_level == level) return HE_OK;
+    // in place: c1 rows move from offset level*N to new_level*N; ascending row
+    // copies never overwrite a source row that is still to be read (the shift
+    // is >= one row)
+    for (int r = 0; r < new_level; r++) {
+        int rc = check_cuda(c, cudaMemcpyAsync(out + (new_level + r) * N, in + (level + r) * N, N * 8,
                                                cudaMemcpyDeviceToDevice, c->stream), "drop");
-            if (rc) return rc;
-        }
+        if (rc) return rc;
     }
     return HE_OK;
 }
@@ -539,90 +664,66 @@ extern "C" int he_poly_eval_ps15(he_ctx* c, const he_ct* x, int n, const double*
     int rc = scratch_slot(c, 3, ctw * nbuf * n, &pool);
     if (rc) return rc;
     auto buf = [&](int k, int i) { return pool + ctw * ((size_t)k * n + i); };
+    auto bufs = [&](int k) {
+        std::vector<uint64_t*> v(n);
+        for (int i = 0; i < n; i++) v[i] = buf(k, i);
+        return v;
+    };
+    auto cbufs = [&](int k) {
+        std::vector<const uint64_t*> v(n);
+        for (int i = 0; i < n; i++) v[i] = buf(k, i);
+        return v;
+    };
     enum { X2, X3, X4, ACC, PROD, TERM, QSUM, TMP };
-    std::vector<const uint64_t*> vx(n), va(n), vb(n);
-    std::vector<uint64_t*> vo(n);
-    auto run_hmrr = [&](int level) { return hmrr_many(c, va, vb, vo, level); };
+    std::vector<const uint64_t*> xd(n);
+    for (int i = 0; i < n; i++) xd[i] = x[i].data;
     double sx = x[0].scale;
     // x2 = HMRR(x, x)
-    for (int i = 0; i < n; i++) {
-        va[i] = x[i].data;
-        vb[i] = x[i].data;
-        vo[i] = buf(X2, i);
-    }
-    if ((rc = run_hmrr(l0))) goto done;
+    if ((rc = hmrr_many(c, xd, xd, bufs(X2), l0))) goto done;
     {
         double s2 = (sx * sx) / (double)c->primes[l0 - 1];
         // x3 = HMRR(x2, drop(x, l0-1))
-        for (int i = 0; i < n; i++) {
-            if ((rc = drop_raw(c, x[i].data, l0, buf(TMP, i), l0 - 1))) goto done;
-            va[i] = buf(X2, i);
-            vb[i] = buf(TMP, i);
-            vo[i] = buf(X3, i);
-        }
-        if ((rc = run_hmrr(l0 - 1))) goto done;
+        if ((rc = drop_many(c, xd, bufs(TMP), l0, l0 - 1))) goto done;
+        if ((rc = hmrr_many(c, cbufs(X2), cbufs(TMP), bufs(X3), l0 - 1))) goto done;
         double s3 = (s2 * sx) / (double)c->primes[l0 - 2];
-        for (int i = 0; i < n; i++) {
-            va[i] = buf(X2, i);
-            vb[i] = buf(X2, i);
-            vo[i] = buf(X4, i);
-        }
-        if ((rc = run_hmrr(l0 - 1))) goto done;
+        // x4 = HMRR(x2, x2)
+        if ((rc = hmrr_many(c, cbufs(X2), cbufs(X2), bufs(X4), l0 - 1))) goto done;
         double s4 = (s2 * s2) / (double)c->primes[l0 - 2];
-        const uint64_t* pw_data[4] = {nullptr, nullptr, nullptr, nullptr};
         int pw_level[4] = {0, l0, l0 - 1, l0 - 2};
         double pw_scale[4] = {0, sx, s2, s3};
 
-        // q_blk(x) at (lam, T) into dst buffers (level lam)
+        // q_blk(x) at (lam, T) into dst buffers (level lam): each x^j dropped
+        // to lam+1 and multiplied by its integer constant in one pass, then
+        // rescaled; the constant term added last
         auto build_q = [&](int blk, int lam, double T, int dst) -> int {
             int r;
             for (int j = 1; j <= 3; j++) {
                 double cj = coeffs[4 * blk + j];
                 double v = cj * T * (double)c->primes[lam] / pw_scale[j];
                 int64_t K = (int64_t)round_half_away(v);
-                for (int i = 0; i < n; i++) {
-                    const uint64_t* src = j == 1 ? x[i].data : (j == 2 ? buf(X2, i) : buf(X3, i));
-                    if ((r = drop_raw(c, src, pw_level[j], buf(TMP, i), lam + 1))) return r;
-                    if ((r = mul_const_raw(c, buf(TMP, i), buf(TMP, i), lam + 1, K))) return r;
-                }
-                std::vector<const uint64_t*> rin(n);
-                std::vector<uint64_t*> rout(n);
-                for (int i = 0; i < n; i++) {
-                    rin[i] = buf(TMP, i);
-                    rout[i] = j == 1 ? buf(dst, i) : buf(TERM, i);
-                }
-                if ((r = rescale_many(c, rin, rout, lam + 1))) return r;
-                if (j > 1)
-                    for (int i = 0; i < n; i++)
-                        if ((r = add_raw(c, buf(dst, i), buf(TERM, i), buf(dst, i), lam))) return r;
+                const std::vector<const uint64_t*> src = j == 1 ? xd : cbufs(j == 2 ? X2 : X3);
+                if ((r = mul_const_many(c, src, bufs(TMP), pw_level[j], lam + 1, K))) return r;
+                if ((r = rescale_many(c, cbufs(TMP), bufs(j == 1 ? dst : TERM), lam + 1))) return r;
+                if (j > 1 && (r = add_many(c, cbufs(dst), cbufs(TERM), bufs(dst), lam))) return r;
             }
             int64_t K0 = (int64_t)round_half_away(coeffs[4 * blk] * T);
-            for (int i = 0; i < n; i++)
-                if ((r = add_const_raw(c, buf(dst, i), lam, K0))) return r;
-            return HE_OK;
+            return add_const_many(c, bufs(dst), lam, K0);
         };
-        (void)pw_data;
         int lev = l0 - 3;
         double T = top_scale;
         if ((rc = build_q(3, lev, T, ACC))) goto done;
         for (int blk = 2; blk >= 0; blk--) {
-            for (int i = 0; i < n; i++) {
-                if ((rc = drop_raw(c, buf(X4, i), l0 - 2, buf(TMP, i), lev))) goto done;
-                va[i] = buf(ACC, i);
-                vb[i] = buf(TMP, i);
-                vo[i] = buf(PROD, i);
-            }
-            if ((rc = run_hmrr(lev))) goto done;
+            if ((rc = drop_many(c, cbufs(X4), bufs(TMP), l0 - 2, lev))) goto done;
+            if ((rc = hmrr_many(c, cbufs(ACC), cbufs(TMP), bufs(PROD), lev))) goto done;
             T = (T * s4) / (double)c->primes[lev - 1];
             lev -= 1;
             if ((rc = build_q(blk, lev, T, QSUM))) goto done;
-            for (int i = 0; i < n; i++)
-                if ((rc = add_raw(c, buf(PROD, i), buf(QSUM, i), buf(ACC, i), lev))) goto done;
+            if ((rc = add_many(c, cbufs(PROD), cbufs(QSUM), bufs(ACC), lev))) goto done;
         }
+        std::vector<uint64_t*> od(n);
+        for (int i = 0; i < n; i++) od[i] = out[i].data;
+        if ((rc = drop_many(c, cbufs(ACC), od, lev, lev))) goto done;
         for (int i = 0; i < n; i++) {
-            rc = check_cuda(c, cudaMemcpyAsync(out[i].data, buf(ACC, i), (size_t)2 * lev * N * 8,
-                                               cudaMemcpyDeviceToDevice, c->stream), "ps15 out");
-            if (rc) goto done;
             out[i].level = lev;
             out[i].scale = T;
             out[i].is_ntt = 1;
