@@ -9,7 +9,6 @@
 
 namespace he {
 
-int add_raw(he_ctx* c, const uint64_t* a, const uint64_t* b, uint64_t* out, int level);
 
 // Z[t][g][poly][r][c] = sum_{k < KB} pt[i][j][g][b][r][c] * B[t][k][poly][r][c],  k = j bs + b,
 // a small modular matrix product per coefficient ([g x k] weights times
@@ -20,6 +19,9 @@ int add_raw(he_ctx* c, const uint64_t* a, const uint64_t* b, uint64_t* out, int 
 // 2^41 sum signed FP64 products (|.| < 5q/8 each, one reduction per output);
 // the others accumulate 128-bit products and reduce once.
 constexpr int kPmThreadsX = 32, kPmG = 8;
+
+// Scratch words of sums and rotated sums a wave of output blocks may hold (8 GiB).
+constexpr size_t kBsgsWaveWords = (size_t)1 << 30;
 
 // Element of the staged tile: the residue as a double (FP64 limbs) or as is.
 __device__ __forceinline__ void stage_put(uint64_t* dst, uint64_t v, bool fp) {
@@ -139,6 +141,22 @@ __global__ void __launch_bounds__(kPmThreadsX* kPmG)
     }
 }
 
+// Y_u = Z_u[0] + sum_{g=1}^{gs-1} R_u[g] for the outputs u of one launch:
+// Z_u = zbase + u gs ctw (gs ciphertexts), R_u = rbase + u gs ctw (entry 0 unused).
+__global__ void k_sum_giant(const uint64_t* __restrict__ zbase, const uint64_t* __restrict__ rbase, MutPtrList y,
+                            int gs, int level, const DevPrime* __restrict__ pr, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x, row = blockIdx.y, u = blockIdx.z;  // row < 2 level
+    if (c >= N) return;
+    const size_t ctw = (size_t)2 * level * N, k = (size_t)row * N + c;
+    const uint64_t q = pr[row % level].q;
+    const uint64_t* z = zbase + (size_t)u * gs * ctw + k;
+    const uint64_t* r = rbase + (size_t)u * gs * ctw + k;
+    uint64_t acc = z[0];
+    for (int g = 1; g < gs; g++) acc = add_mod(acc, r[(size_t)g * ctw], q);
+    y.p[u][k] = acc;
+}
+
 }  // namespace he
 
 using namespace he;
@@ -165,13 +183,18 @@ extern "C" int he_pmult_accum_bsgs(he_ctx* c, const he_ct* x, int n_in, const ui
             return set_err(c, HE_ENOKEY, "he_pmult_accum_bsgs: no key for giant step %d", stride * bs * g);
 
     const size_t ctw = (size_t)2 * level * N;
-    const size_t nB = (size_t)n_groups * n_in * bs, nZ = (size_t)n_groups * gs;
+    const size_t nB = (size_t)n_groups * n_in * bs;
+    // output blocks run in waves: each block needs n_groups gs ciphertexts of
+    // sums Z and as many of rotated sums; a wave holds as many blocks as fit
+    // in kBsgsWaveWords (at least one)
+    const size_t per_block = (size_t)2 * n_groups * gs * ctw;
+    const int wave = std::max(1, std::min(n_out, (int)(kBsgsWaveWords / per_block)));
     uint64_t* buf;
-    int rc = scratch_slot(c, 3, ctw * (nB + 2 * nZ), &buf);
+    int rc = scratch_slot(c, 3, ctw * nB + per_block * wave, &buf);
     if (rc) return rc;
     uint64_t* B = buf;
-    uint64_t* Z = B + ctw * nB;
-    uint64_t* Rg = Z + ctw * nZ;
+    uint64_t* Z = B + ctw * nB;                                 // [wave][n_groups][gs]
+    uint64_t* Rg = Z + (size_t)wave * n_groups * gs * ctw;      // same layout (entries g >= 1)
 
     // baby steps: B[t][j][b] = rot_{stride b}(X[t][j])
     std::vector<he_ct> bin, bout;
@@ -197,55 +220,62 @@ extern "C" int he_pmult_accum_bsgs(he_ctx* c, const he_ct* x, int n_in, const ui
     const int smem = tch * n_in * bs * 2 * kPmThreadsX * cpt * 8;
     if (smem > 200 * 1024) return set_err(c, HE_EINVAL, "he_pmult_accum_bsgs: n_in*bs = %d too large", n_in * bs);
     const dim3 pgrid((gs + kPmG - 1) / kPmG, N / (kPmThreadsX * cpt), level);
-    for (int i = 0; i < n_out; i++) {
-        prof_begin(c, HE_PROF_PMULT);
-        if (tch == 1) {
-            cudaFuncSetAttribute(k_pmult_accum<1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            k_pmult_accum<1, 2><<<pgrid, kPmThreadsX * kPmG, smem, c->stream>>>(
-                d_pt + pt_block * i, B, Z, n_groups, n_in, gs, bs, level, c->d_prime, c->d_fpmod, c->log_n);
-        } else {
-            cudaFuncSetAttribute(k_pmult_accum<4, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            k_pmult_accum<4, 1><<<pgrid, kPmThreadsX * kPmG, smem, c->stream>>>(
-                d_pt + pt_block * i, B, Z, n_groups, n_in, gs, bs, level, c->d_prime, c->d_fpmod, c->log_n);
-        }
-        c->launches++;
-        if ((rc = check_cuda(c, cudaGetLastError(), "pmult_accum"))) return rc;
-        // weights of block i once per staged pass of token groups, the rotated
-        // inputs once, the sums written once
-        {
+    int fp_l = 0;
+    for (int r = 0; r < level; r++) fp_l += fp_prime(c, r);
+    for (int i0 = 0; i0 < n_out; i0 += wave) {
+        const int w = std::min(wave, n_out - i0);
+        for (int ii = 0; ii < w; ii++) {
+            uint64_t* Zi = Z + (size_t)ii * n_groups * gs * ctw;
+            const uint64_t* pti = d_pt + pt_block * (i0 + ii);
+            prof_begin(c, HE_PROF_PMULT);
+            if (tch == 1) {
+                cudaFuncSetAttribute(k_pmult_accum<1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+                k_pmult_accum<1, 2><<<pgrid, kPmThreadsX * kPmG, smem, c->stream>>>(
+                    pti, B, Zi, n_groups, n_in, gs, bs, level, c->d_prime, c->d_fpmod, c->log_n);
+            } else {
+                cudaFuncSetAttribute(k_pmult_accum<4, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+                k_pmult_accum<4, 1><<<pgrid, kPmThreadsX * kPmG, smem, c->stream>>>(
+                    pti, B, Zi, n_groups, n_in, gs, bs, level, c->d_prime, c->d_fpmod, c->log_n);
+            }
+            c->launches++;
+            if ((rc = check_cuda(c, cudaGetLastError(), "pmult_accum"))) return rc;
+            // weights of the block once per staged pass of token groups, the
+            // rotated inputs once, the sums written once
             const double passes = (n_groups + tch - 1) / tch;
-            int fp_l = 0;
-            for (int r = 0; r < level; r++) fp_l += fp_prime(c, r);
             const double macs_per_limb = 2.0 * N * (double)gs * n_groups * n_in * bs;
-            prof_end(c, HE_PROF_PMULT, 8.0 * ((double)pt_block * passes + (double)ctw * nB + (double)ctw * nZ),
+            prof_end(c, HE_PROF_PMULT, 8.0 * ((double)pt_block * passes + (double)ctw * nB +
+                                              (double)ctw * n_groups * gs),
                      macs_per_limb * level, macs_per_limb * fp_l);
         }
-        // giant steps
+        // giant steps of the whole wave in one batch
         std::vector<he_ct> gin, gout;
         std::vector<int32_t> gsteps;
-        for (int t = 0; t < n_groups; t++)
+        for (int u = 0; u < w * n_groups; u++)
             for (int g = 1; g < gs; g++) {
-                gin.push_back(he_ct{Z + (size_t)(t * gs + g) * ctw, level, 1.0, 1});
-                gout.push_back(he_ct{Rg + (size_t)(t * gs + g) * ctw, level, 1.0, 1});
+                gin.push_back(he_ct{Z + ((size_t)u * gs + g) * ctw, level, 1.0, 1});
+                gout.push_back(he_ct{Rg + ((size_t)u * gs + g) * ctw, level, 1.0, 1});
                 gsteps.push_back(stride * bs * g);
             }
         if (!gin.empty() && (rc = rotate_many(c, gin.data(), gsteps.data(), gout.data(), (int)gin.size())))
             return rc;
+        // Y = Z_0 + sum_g rotated Z_g, then one rescale for the wave
         std::vector<const uint64_t*> rin;
         std::vector<uint64_t*> rout;
-        for (int t = 0; t < n_groups; t++) {
-            uint64_t* dst = y[t * n_out + i].data;
-            const uint64_t* z0 = Z + (size_t)(t * gs) * ctw;
-            if (gs == 1) {
-                rc = check_cuda(c, cudaMemcpyAsync(dst, z0, ctw * 8, cudaMemcpyDeviceToDevice, c->stream), "bsgs");
-                if (rc) return rc;
+        for (int u0 = 0; u0 < w * n_groups; u0 += kMaxBatch) {
+            const int m = std::min(kMaxBatch, w * n_groups - u0);
+            MutPtrList py;
+            for (int u = 0; u < m; u++) {
+                const int ii = (u0 + u) / n_groups, t = (u0 + u) - ii * n_groups;
+                py.p[u] = y[t * n_out + i0 + ii].data;
+                rin.push_back(py.p[u]);
+                rout.push_back(py.p[u]);
             }
-            for (int g = 1; g < gs; g++) {
-                const uint64_t* src = g == 1 ? z0 : dst;
-                if ((rc = add_raw(c, src, Rg + (size_t)(t * gs + g) * ctw, dst, level))) return rc;
-            }
-            rin.push_back(dst);
-            rout.push_back(dst);
+            prof_begin(c, HE_PROF_ELEMENTWISE);
+            k_sum_giant<<<dim3((N + 255) / 256, 2 * level, m), 256, 0, c->stream>>>(
+                Z + (size_t)u0 * gs * ctw, Rg + (size_t)u0 * gs * ctw, py, gs, level, c->d_prime, c->log_n);
+            c->launches++;
+            if ((rc = check_cuda(c, cudaGetLastError(), "bsgs sum"))) return rc;
+            prof_end(c, HE_PROF_ELEMENTWISE, 8.0 * m * (double)(gs + 1) * ctw);
         }
         if ((rc = rescale_many(c, rin, rout, level))) return rc;
     }
