@@ -125,6 +125,24 @@ class ClockSampler:
 
 # ------------------------------------------------------------ cpu baseline
 
+def max_over_ranks(values, world, device):
+    """Element-wise maximum of a list of floats over all ranks (the ranks'
+    device times: the job's time is its slowest rank's)."""
+    if world == 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def rank_seed(master, rank):
+    """Seed of a rank's own ciphertexts (every rank rotates different inputs)."""
+    return master + 7919 * rank
+
+
 def cpu_baseline(seconds):
     """The oracle, as it stands, rotating full-size ciphertexts of this workload
     on the host cores until about `seconds` of rotation work has run."""
@@ -432,7 +450,7 @@ def run_native(args, rank, world, local_rank):
         he.he_keygen_upload(ctx, he.HE_KEY_ROTATION, st, s, a, e)
     # inputs: uniform residues (a fresh encryption is computationally
     # indistinguishable from them); per-rank stream of draws
-    h_in = S.uniform_residues(master + 7919 * rank, "ct_residues", ctx.primes[:L], N, lead=(N_CTS, 2))
+    h_in = S.uniform_residues(rank_seed(master, rank), "ct_residues", ctx.primes[:L], N, lead=(N_CTS, 2))
     x = torch.from_numpy(h_in.view(np.int64)).to(dev)
     y = torch.empty_like(x)
     xs = [he.Ciphertext(x[i], LEVEL, 2.0 ** 40) for i in range(N_CTS)]
@@ -483,10 +501,7 @@ def run_native(args, rank, world, local_rank):
     prof = {name: he.he_profile_read(ctx, cls) + (he.he_profile_read_fp(ctx, cls),) for name, cls in he.PROF.items()}
     he.he_profile_enable(ctx, False)
 
-    if world > 1:
-        tt = torch.tensor([ms_plain, ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_plain, ms = float(tt[0]), float(tt[1])
+    ms_plain, ms = max_over_ranks([ms_plain, ms], world, dev)
 
     # end to end through the host-buffer entry point (pinned host memory)
     h_pin = torch.from_numpy(h_in.view(np.int64)).pin_memory()
@@ -498,10 +513,7 @@ def run_native(args, rank, world, local_rank):
     for _ in range(e2e_steps):
         he.he_rotate_batch_host(ctx, h_pin, LEVEL, ct_steps, h_out)
     e2e_s = time.perf_counter() - te
-    if world > 1:
-        tt = torch.tensor([e2e_s], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_s = float(tt[0])
+    (e2e_s,) = max_over_ranks([e2e_s], world, dev)
 
     if rank != 0:
         return
