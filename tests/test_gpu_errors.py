@@ -1,0 +1,91 @@
+"""GPU: argument and state errors of the C ABI come back as codes (nothing is
+launched), and the context stays usable after each of them."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import ckks as C
+import seeded_inputs as S
+from tests.helpers import Setup, lib
+
+pytestmark = pytest.mark.gpu
+
+
+def _code(fn, *args):
+    he = lib()
+    with pytest.raises(he.HEError) as ei:
+        fn(*args)
+    return ei.value.code
+
+
+def test_forced_allocation_failure_is_enomem():
+    """HE_FAIL_ALLOC=1 makes every device allocation of the library fail:
+    context creation reports HE_ENOMEM and leaks nothing observable."""
+    he = lib()
+    os.environ["HE_FAIL_ALLOC"] = "1"
+    try:
+        with pytest.raises(he.HEError) as ei:
+            he.he_ctx_create(12, 3, 1, 3)
+        assert ei.value.code == he.HE_ENOMEM
+    finally:
+        del os.environ["HE_FAIL_ALLOC"]
+    ctx = he.he_ctx_create(12, 3, 1, 3)  # and works again without it
+    he.he_ctx_destroy(ctx)
+
+
+def test_unaligned_ciphertexts_are_rejected():
+    he = lib()
+    st = Setup(12, 3, 1, 3, seed=61)
+    st.upload_rot(1)
+    st.upload_relin()
+    z = S.complex_slots(st.seed, st.P.n_slots, -1, 1)
+    x = st.to_gpu(st.encrypt(z, 3))
+    raw = torch.zeros(2 * 3 * st.P.N + 1, dtype=torch.int64, device="cuda")
+    bad = he.Ciphertext(raw[1:], 3, 1.0)  # 8 bytes past a 16-byte boundary
+    y = st.empty_gpu(3)
+    assert _code(he.he_rotate, st.ctx, bad, 1, y) == he.HE_EINVAL
+    assert _code(he.he_rotate, st.ctx, x, 1, bad) == he.HE_EINVAL
+    assert _code(he.he_hmult_relin_rescale, st.ctx, x, x, bad) == he.HE_EINVAL
+    # the context still rotates correctly
+    he.he_rotate(st.ctx, x, 1, y)
+    he.he_sync(st.ctx)
+    want = C.rotate(st.encrypt(z, 3), 1, st.oracle_rot_key(1), st.P)
+    assert np.array_equal(st.from_gpu(y), want["c"])
+
+
+def test_host_buffer_entry_errors():
+    he = lib()
+    st = Setup(12, 3, 1, 3, seed=62)
+    st.upload_rot(1)
+    h = np.zeros((2, 2, 3, st.P.N), dtype=np.uint64)
+    out = np.zeros_like(h)
+    assert _code(he.he_rotate_batch_host, st.ctx, h, 3, [1, 5], out) == he.HE_ENOKEY
+    assert _code(he.he_rotate_batch_host, st.ctx, h, 9, [1, 1], out) == he.HE_EINVAL
+    he.he_rotate_batch_host(st.ctx, h, 3, [1, 1], out)  # zero ciphertexts rotate to zero
+    assert not out.any()
+
+
+def test_bsgs_and_polynomial_errors():
+    he = lib()
+    st = Setup(12, 3, 1, 3, seed=63)
+    z = S.complex_slots(st.seed, st.P.n_slots, -1, 1)
+    x3 = st.to_gpu(st.encrypt(z, 3))
+    ys = [st.empty_gpu(3)]
+    pt = torch.zeros((1, 1, 2, 2, 3, st.P.N), dtype=torch.int64, device="cuda")
+    # keys for the baby step (stride 1) and the giant step (stride 2) missing
+    assert _code(he.he_pmult_accum_bsgs, st.ctx, [x3], 1, pt, 2.0 ** 40, 1, 2, 2, 1, 1, ys) == he.HE_ENOKEY
+    # n_in * bs above 255
+    assert _code(he.he_pmult_accum_bsgs, st.ctx, [x3], 1, pt, 2.0 ** 40, 1, 256, 1, 1, 1, ys) == he.HE_EINVAL
+    # mixed input levels
+    x2 = st.to_gpu(st.encrypt(z, 2), room=3)
+    st.upload_rot(1)
+    assert _code(he.he_pmult_accum_bsgs, st.ctx, [x3, x2], 2, pt, 2.0 ** 40, 1, 2, 1, 1, 1, ys) == he.HE_ELEVEL
+    # the polynomial needs level 7 and the relinearisation key
+    coeffs = S.poly_coeffs(st.seed, 15)
+    assert _code(he.he_poly_eval_ps15, st.ctx, [x3], coeffs, 2.0 ** 62, [st.empty_gpu(3)]) in (he.HE_ELEVEL,
+                                                                                              he.HE_ENOKEY)
+    st7 = Setup(12, 8, 3, 3, seed=64)
+    x7 = st7.to_gpu(st7.encrypt(z, 8))
+    assert _code(he.he_poly_eval_ps15, st7.ctx, [x7], coeffs, 2.0 ** 62, [st7.empty_gpu(8)]) == he.HE_ENOKEY
