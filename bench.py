@@ -269,6 +269,83 @@ def device_residues(torch, shape_lead, primes, N, gen, dev):
     return t
 
 
+def workload_cpu_baseline(case, seconds):
+    """The oracle, as it stands, on a bounded sample of a workload (host cores).
+    tiny: whole operation sequences at N=2^12.  ps15: whole degree-15
+    evaluations of single full-size ciphertexts.  ffn128 / ffn2048: one
+    full-size rotation and plaintext products at level 12, timed, scaled by
+    the product's operation counts (the key generation is outside every
+    timing)."""
+    from oracle import ckks as C
+
+    widx = {"tiny": 0, "ffn128": 2, "ffn2048": 3, "ps15": 4}[case]
+    master = S.master_seed(widx)
+    t_end = time.perf_counter() + seconds
+    if case == "tiny":
+        P = C.Params(12, 3, 1, 3)
+        s = S.secret(master, P.N)
+        keys = {}
+        for st in (1, 2, -1):
+            a, e = S.key_draws(master, P.galois_elt(st), P.mods, P.N, P.dnum)
+            keys[st] = C.rotation_key(s, st, a, e, P)
+        a, e = S.key_draws(master, 2, P.mods, P.N, P.dnum)
+        rlk = C.relin_key(s, a, e, P)
+        ct = C.make_ct(S.uniform_residues(master, "ct_residues", P.q, P.N, lead=(2,)), 3, 2.0 ** 40)
+        done, t = 0, 0.0
+        while done < 2 or time.perf_counter() < t_end:
+            t0 = time.perf_counter()
+            C.ntt_rows(C.intt_rows(ct["c"][0], P.q, P), P.q, P)
+            for st in (1, 2, -1):
+                C.rotate(ct, st, keys[st], P)
+            C.hmult_relin_rescale(ct, ct, rlk, P)
+            t += time.perf_counter() - t0
+            done += 1
+        return {"value": done / t, "unit": "sequences/s", "cores": C.n_threads(), "kind": "oracle",
+                "sample": "%d whole sequences (NTT round trip, 3 rotations, 1 HMult-relin-rescale), N=2^12" % done}
+    P = C.Params(LOG_N, L, K, DNUM)
+    s = S.secret(master, P.N)
+    if case == "ps15":
+        a, e = S.key_draws(master, 2, P.mods, P.N, P.dnum)
+        rlk = C.relin_key(s, a, e, P)
+        coeffs = S.poly_coeffs(master, 15)
+        ct = C.make_ct(S.uniform_residues(master, "ct_residues", P.q, P.N, lead=(2,)), L, 2.0 ** 40)
+        done, t = 0, 0.0
+        while done < 1 or time.perf_counter() < t_end:
+            t0 = time.perf_counter()
+            C.ps_eval_deg15(ct, coeffs, rlk, P)
+            t += time.perf_counter() - t0
+            done += 1
+        return {"value": done / t, "unit": "evals/s", "cores": C.n_threads(), "kind": "oracle",
+                "sample": "%d whole degree-15 evaluations of single full-size ciphertexts (level 24)" % done}
+    f = FFN
+    n_groups = 1 if case == "ffn128" else 16
+    lvl = f["level"]
+    st = f["n_tok"]
+    a, e = S.key_draws(master, P.galois_elt(st), P.mods, P.N, P.dnum)
+    key = C.rotation_key(s, st, a, e, P)
+    ct = C.make_ct(S.uniform_residues(master, "ct_residues", P.q[:lvl], P.N, lead=(2,)), lvl, 2.0 ** 40)
+    pt = S.uniform_residues(master, "pt_residues", P.q[:lvl], P.N, lead=(1,))[0]
+    t0 = time.perf_counter()
+    C.rotate(ct, st, key, P)
+    t_rot = time.perf_counter() - t0
+    n_pm, t_pm = 0, 0.0
+    while n_pm < 4 or time.perf_counter() < t_end:
+        t0 = time.perf_counter()
+        C.pmult_accum([ct], [pt], lvl, P)
+        t_pm += time.perf_counter() - t0
+        n_pm += 1
+    t0 = time.perf_counter()
+    C.rescale(ct, P)
+    t_rs = time.perf_counter() - t0
+    rot = n_groups * f["n_in"] * (f["bs"] - 1) + n_groups * f["n_out"] * (f["gs"] - 1)
+    pms = n_groups * f["n_out"] * f["n_in"] * f["gs"] * f["bs"]
+    per_product = rot * t_rot + pms * t_pm / n_pm + n_groups * f["n_out"] * t_rs
+    return {"value": 1.0 / per_product, "unit": "products/s", "cores": C.n_threads(), "kind": "oracle",
+            "sample": "1 full-size rotation, %d plaintext products and 1 rescale at level 12, scaled to the "
+                      "product's %d rotations, %d plaintext products and %d rescales (%.1f s per product)"
+                      % (n_pm, rot, pms, n_groups * f["n_out"], per_product)}
+
+
 def run_workload_case(args, local_rank):
     """Throughput of the other workloads on one GPU, one JSON line each:
     ffn128 (FFN1 768->3072, 128 tokens: 3 x 12 blocks by BSGS at level 12),
@@ -393,6 +470,8 @@ def run_workload_case(args, local_rank):
             "probes": {"copy_gbs": copy_gbs, "int_shoup_modmul_per_s": int_modmul_s,
                        "fp64_modmul_per_s": fp_modmul_s},
             "clocks": clk}
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = workload_cpu_baseline(case, args.cpu_seconds)
     print(json.dumps(line), flush=True)
 
 
