@@ -28,9 +28,10 @@ __device__ __forceinline__ void stage_put(uint64_t* dst, uint64_t v, bool fp) {
     *dst = fp ? (uint64_t)__double_as_longlong(u2d(v)) : v;
 }
 
-// TCH token groups staged per pass, CPT adjacent columns per thread
-// (kPmThreadsX * CPT columns per block).
-template <int TCH, int CPT>
+// TCH token groups staged per pass, CPT adjacent columns and GPT giant steps
+// per thread (kPmThreadsX * CPT columns and kPmG * GPT giant steps per block):
+// each staged input feeds GPT products, each weight TCH * 2.
+template <int TCH, int CPT, int GPT>
 __global__ void __launch_bounds__(kPmThreadsX* kPmG)
     k_pmult_accum(const uint64_t* __restrict__ pt_i, const uint64_t* __restrict__ B, uint64_t* __restrict__ Z,
                   int n_groups, int n_in, int gs, int bs, int level, const DevPrime* __restrict__ pr,
@@ -40,8 +41,8 @@ __global__ void __launch_bounds__(kPmThreadsX* kPmG)
     const int N = 1 << logn;
     const int KB = n_in * bs;
     const int tx = threadIdx.x % kPmThreadsX, tg = threadIdx.x / kPmThreadsX;
-    // giant-step blocks of one column tile are neighbours: the second finds the tile in L2
-    const int c0 = blockIdx.y * COLS, r = blockIdx.z, g = blockIdx.x * kPmG + tg;
+    // giant-step blocks of one column tile are neighbours: a second finds the tile in L2
+    const int c0 = blockIdx.y * COLS, r = blockIdx.z, g0 = (blockIdx.x * kPmG + tg) * GPT;
     const DevPrime p = pr[r];
     const bool fp = p.q < kFpPrimeLimit;
     const FpMod m = fpm[r];
@@ -56,25 +57,32 @@ __global__ void __launch_bounds__(kPmThreadsX* kPmG)
             stage_put(sB + idx, B[((size_t)(t0 + t) * KB + k) * ctw + poly * limb + col + cc], fp);
         }
         __syncthreads();
-        if (g >= gs) continue;
-        const uint64_t* w_g = pt_i + col + CPT * tx;
+        if (g0 >= gs) continue;
+        const bool g1ok = GPT > 1 && g0 + 1 < gs;
+        const uint64_t* w_base = pt_i + col + CPT * tx;
         if (fp) {
-            double acc[TCH][2][CPT];
+            double acc[GPT][TCH][2][CPT];
 #pragma unroll
-            for (int t = 0; t < TCH; t++)
+            for (int h = 0; h < GPT; h++)
 #pragma unroll
-                for (int e = 0; e < CPT; e++) acc[t][0][e] = acc[t][1][e] = 0.0;
-#pragma unroll 8
+                for (int t = 0; t < TCH; t++)
+#pragma unroll
+                    for (int e = 0; e < CPT; e++) acc[h][t][0][e] = acc[h][t][1][e] = 0.0;
+#pragma unroll 4
             for (int k = 0; k < KB; k++) {
                 const int j = k / bs, b = k - j * bs;
-                const uint64_t* wp = w_g + ((size_t)(j * gs + g) * bs + b) * limb;
-                double w[CPT];
-                if constexpr (CPT == 2) {
-                    const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2*>(wp));
-                    w[0] = u2d(v.x);
-                    w[1] = u2d(v.y);
-                } else {
-                    w[0] = u2d(__ldg(wp));
+                double w[GPT][CPT];
+#pragma unroll
+                for (int h = 0; h < GPT; h++) {
+                    const int g = (h == 0 || g1ok) ? g0 + h : g0;
+                    const uint64_t* wp = w_base + ((size_t)(j * gs + g) * bs + b) * limb;
+                    if constexpr (CPT == 2) {
+                        const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2*>(wp));
+                        w[h][0] = u2d(v.x);
+                        w[h][1] = u2d(v.y);
+                    } else {
+                        w[h][0] = u2d(__ldg(wp));
+                    }
                 }
                 const double* sk = reinterpret_cast<const double*>(sB) + (size_t)k * 2 * COLS + CPT * tx;
 #pragma unroll
@@ -83,57 +91,69 @@ __global__ void __launch_bounds__(kPmThreadsX* kPmG)
                         const double* st = sk + (size_t)t * KB * 2 * COLS;
 #pragma unroll
                         for (int e = 0; e < CPT; e++) {
-                            acc[t][0][e] = __dadd_rn(acc[t][0][e], fp_mulmod_s(w[e], st[e], m));
-                            acc[t][1][e] = __dadd_rn(acc[t][1][e], fp_mulmod_s(w[e], st[COLS + e], m));
+                            const double b0 = st[e], b1 = st[COLS + e];
+#pragma unroll
+                            for (int h = 0; h < GPT; h++) {
+                                acc[h][t][0][e] = __dadd_rn(acc[h][t][0][e], fp_mulmod_s(w[h][e], b0, m));
+                                acc[h][t][1][e] = __dadd_rn(acc[h][t][1][e], fp_mulmod_s(w[h][e], b1, m));
+                            }
                         }
                     }
                 }
             }
 #pragma unroll
-            for (int t = 0; t < TCH; t++) {
-                if (t < nt) {
-                    uint64_t* z = Z + ((size_t)(t0 + t) * gs + g) * ctw + col + CPT * tx;
+            for (int h = 0; h < GPT; h++) {
+                if (h > 0 && !g1ok) break;
 #pragma unroll
-                    for (int e = 0; e < CPT; e++) {
-                        z[e] = d2u(fp_canon(acc[t][0][e], m));
-                        z[limb + e] = d2u(fp_canon(acc[t][1][e], m));
+                for (int t = 0; t < TCH; t++) {
+                    if (t < nt) {
+                        uint64_t* z = Z + ((size_t)(t0 + t) * gs + g0 + h) * ctw + col + CPT * tx;
+#pragma unroll
+                        for (int e = 0; e < CPT; e++) {
+                            z[e] = d2u(fp_canon(acc[h][t][0][e], m));
+                            z[limb + e] = d2u(fp_canon(acc[h][t][1][e], m));
+                        }
                     }
                 }
             }
         } else {
-            U128 acc[TCH][2][CPT];
+            for (int h = 0; h < GPT; h++) {
+                if (h > 0 && !g1ok) break;
+                const int g = g0 + h;
+                U128 acc[TCH][2][CPT];
 #pragma unroll
-            for (int t = 0; t < TCH; t++)
+                for (int t = 0; t < TCH; t++)
 #pragma unroll
-                for (int e = 0; e < CPT; e++) acc[t][0][e] = acc[t][1][e] = U128{0, 0};
+                    for (int e = 0; e < CPT; e++) acc[t][0][e] = acc[t][1][e] = U128{0, 0};
 #pragma unroll 4
-            for (int k = 0; k < KB; k++) {
-                const int j = k / bs, b = k - j * bs;
-                const uint64_t* wp = w_g + ((size_t)(j * gs + g) * bs + b) * limb;
-                uint64_t w[CPT];
+                for (int k = 0; k < KB; k++) {
+                    const int j = k / bs, b = k - j * bs;
+                    const uint64_t* wp = w_base + ((size_t)(j * gs + g) * bs + b) * limb;
+                    uint64_t w[CPT];
 #pragma unroll
-                for (int e = 0; e < CPT; e++) w[e] = __ldg(wp + e);
-                const uint64_t* sk = sB + (size_t)k * 2 * COLS + CPT * tx;
+                    for (int e = 0; e < CPT; e++) w[e] = __ldg(wp + e);
+                    const uint64_t* sk = sB + (size_t)k * 2 * COLS + CPT * tx;
 #pragma unroll
-                for (int t = 0; t < TCH; t++) {
-                    if (t < nt) {
-                        const uint64_t* st = sk + (size_t)t * KB * 2 * COLS;
+                    for (int t = 0; t < TCH; t++) {
+                        if (t < nt) {
+                            const uint64_t* st = sk + (size_t)t * KB * 2 * COLS;
 #pragma unroll
-                        for (int e = 0; e < CPT; e++) {
-                            mac128(acc[t][0][e], w[e], st[e]);
-                            mac128(acc[t][1][e], w[e], st[COLS + e]);
+                            for (int e = 0; e < CPT; e++) {
+                                mac128(acc[t][0][e], w[e], st[e]);
+                                mac128(acc[t][1][e], w[e], st[COLS + e]);
+                            }
                         }
                     }
                 }
-            }
 #pragma unroll
-            for (int t = 0; t < TCH; t++) {
-                if (t < nt) {
-                    uint64_t* z = Z + ((size_t)(t0 + t) * gs + g) * ctw + col + CPT * tx;
+                for (int t = 0; t < TCH; t++) {
+                    if (t < nt) {
+                        uint64_t* z = Z + ((size_t)(t0 + t) * gs + g) * ctw + col + CPT * tx;
 #pragma unroll
-                    for (int e = 0; e < CPT; e++) {
-                        z[e] = reduce128(acc[t][0][e], p);
-                        z[limb + e] = reduce128(acc[t][1][e], p);
+                        for (int e = 0; e < CPT; e++) {
+                            z[e] = reduce128(acc[t][0][e], p);
+                            z[limb + e] = reduce128(acc[t][1][e], p);
+                        }
                     }
                 }
             }
@@ -219,7 +239,8 @@ extern "C" int he_pmult_accum_bsgs(he_ctx* c, const he_ct* x, int n_in, const ui
     const int tch = n_groups == 1 ? 1 : 4, cpt = n_groups == 1 ? 2 : 1;
     const int smem = tch * n_in * bs * 2 * kPmThreadsX * cpt * 8;
     if (smem > 200 * 1024) return set_err(c, HE_EINVAL, "he_pmult_accum_bsgs: n_in*bs = %d too large", n_in * bs);
-    const dim3 pgrid((gs + kPmG - 1) / kPmG, N / (kPmThreadsX * cpt), level);
+    const int gpt = 2;  // giant steps per thread
+    const dim3 pgrid((gs + kPmG * gpt - 1) / (kPmG * gpt), N / (kPmThreadsX * cpt), level);
     int fp_l = 0;
     for (int r = 0; r < level; r++) fp_l += fp_prime(c, r);
     for (int i0 = 0; i0 < n_out; i0 += wave) {
@@ -229,12 +250,12 @@ extern "C" int he_pmult_accum_bsgs(he_ctx* c, const he_ct* x, int n_in, const ui
             const uint64_t* pti = d_pt + pt_block * (i0 + ii);
             prof_begin(c, HE_PROF_PMULT);
             if (tch == 1) {
-                cudaFuncSetAttribute(k_pmult_accum<1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-                k_pmult_accum<1, 2><<<pgrid, kPmThreadsX * kPmG, smem, c->stream>>>(
+                cudaFuncSetAttribute(k_pmult_accum<1, 2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+                k_pmult_accum<1, 2, 2><<<pgrid, kPmThreadsX * kPmG, smem, c->stream>>>(
                     pti, B, Zi, n_groups, n_in, gs, bs, level, c->d_prime, c->d_fpmod, c->log_n);
             } else {
-                cudaFuncSetAttribute(k_pmult_accum<4, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-                k_pmult_accum<4, 1><<<pgrid, kPmThreadsX * kPmG, smem, c->stream>>>(
+                cudaFuncSetAttribute(k_pmult_accum<4, 1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+                k_pmult_accum<4, 1, 2><<<pgrid, kPmThreadsX * kPmG, smem, c->stream>>>(
                     pti, B, Zi, n_groups, n_in, gs, bs, level, c->d_prime, c->d_fpmod, c->log_n);
             }
             c->launches++;
