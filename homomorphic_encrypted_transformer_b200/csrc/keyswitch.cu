@@ -109,9 +109,17 @@ struct ConvLists {
 //    are exact doubles below 2^47 (NS <= 16); the 128-bit value
 //    V0 + V1 2^21 + V2 2^42 + V3 2^63 = S y m' is assembled on the integer
 //    pipe and one REDC gives S y m mod t;
-//  - 60-bit targets of a digit with a 60-bit source: 128-bit accumulation of
-//    the NS products, one REDC.
-template <int NS, bool NARROW>
+//  - 60-bit targets of a digit whose first source alone is 60-bit (WIDE0,
+//    the digit holding q_0): that residue splits in three 21-bit parts
+//    (y = y2 2^42 + y1 2^21 + y0), adding V2 += y2 m0, V3 += y2 m1 and
+//    V4 = y2 m2, all still exact (each sum below 2^48), and
+//    V0 + V1 2^21 + V2 2^42 + V3 2^63 + V4 2^84 = S y m' (< 2^124);
+//  - 60-bit targets of any other digit: 128-bit accumulation of the NS
+//    products, one REDC.
+// MODE: kConvNarrow, kConvWide0 or kConvGeneric.
+constexpr int kConvGeneric = 0, kConvNarrow = 1, kConvWide0 = 2;
+
+template <int NS, int MODE>
 __global__ void __launch_bounds__(256)
     k_modup_conv(const uint64_t* __restrict__ coef, uint64_t* __restrict__ ext_j, const ulonglong2* __restrict__ src,
                  const ulonglong2* __restrict__ mat, ModupArgs a, const __grid_constant__ ConvLists cl,
@@ -120,9 +128,10 @@ __global__ void __launch_bounds__(256)
     __shared__ double sm_fm[NS * kConvMaxTargets];  // [s][f]: FP64 targets in list order
     __shared__ FpMod sm_ff[kConvMaxTargets];
     __shared__ ConvTarget sm_ft[kConvMaxTargets];  // (wide sources: reduction into [0, 2t))
-    __shared__ double2 sm_i01[NARROW ? NS * kConvMaxInt : 1];
-    __shared__ double sm_i2[NARROW ? NS * kConvMaxInt : 1];
-    __shared__ uint64_t sm_im[NARROW ? 1 : NS * kConvMaxInt];
+    constexpr bool SPLIT = MODE != kConvGeneric;  // 60-bit targets from exact FP64 partial sums
+    __shared__ double2 sm_i01[SPLIT ? NS * kConvMaxInt : 1];
+    __shared__ double sm_i2[SPLIT ? NS * kConvMaxInt : 1];
+    __shared__ uint64_t sm_im[SPLIT ? 1 : NS * kConvMaxInt];
     __shared__ ConvTarget sm_it[kConvMaxInt];
     __shared__ int sm_ftt[kConvMaxTargets], sm_itt[kConvMaxInt];  // output rows, list order
     const int N = 1 << logn;
@@ -140,7 +149,7 @@ __global__ void __launch_bounds__(256)
         int s = idx / n_int, g = idx - s * n_int;
         int tt = sm_itt[g], t = tt < s0 ? tt : tt + NS;
         uint64_t m = mat[(size_t)s * n_rows + t].x;
-        if constexpr (NARROW) {
+        if constexpr (SPLIT) {
             sm_i01[s * kConvMaxInt + g] =
                 make_double2((double)(m & ((1ull << 21) - 1)), (double)((m >> 21) & ((1ull << 21) - 1)));
             sm_i2[s * kConvMaxInt + g] = (double)(m >> 42);
@@ -176,15 +185,16 @@ __global__ void __launch_bounds__(256)
     uint64_t* o = ext_j + (size_t)i * n_tgt * N + c;
 
     // 60-bit targets
-    if constexpr (NARROW) {
+    if constexpr (SPLIT) {
         double y0[NS], y1[NS];
 #pragma unroll
         for (int s = 0; s < NS; s++) {
             y0[s] = (double)(y[s] & ((1ull << 21) - 1));
-            y1[s] = (double)(y[s] >> 21);  // < 2^20
+            y1[s] = (double)((y[s] >> 21) & ((1ull << 21) - 1));  // all of the rest when narrow
         }
+        const double y2w = MODE == kConvWide0 ? (double)(y[0] >> 42) : 0.0;  // < 2^18
         for (int g = 0; g < n_int; g++) {
-            double v0 = 0, v1 = 0, v2 = 0, v3 = 0;
+            double v0 = 0, v1 = 0, v2 = 0, v3 = 0, v4 = 0;
 #pragma unroll
             for (int s = 0; s < NS; s++) {
                 const double2 m01 = sm_i01[s * kConvMaxInt + g];
@@ -193,12 +203,18 @@ __global__ void __launch_bounds__(256)
                 v1 = __fma_rn(y0[s], m01.y, __fma_rn(y1[s], m01.x, v1));
                 v2 = __fma_rn(y0[s], m2, __fma_rn(y1[s], m01.y, v2));
                 v3 = __fma_rn(y1[s], m2, v3);
+                if (MODE == kConvWide0 && s == 0) {
+                    v2 = __fma_rn(y2w, m01.x, v2);
+                    v3 = __fma_rn(y2w, m01.y, v3);
+                    v4 = __fma_rn(y2w, m2, v4);
+                }
             }
             const uint64_t w0 = d2u(v0), w1 = d2u(v1), w2 = d2u(v2), w3 = d2u(v3);
             U128 acc = {w0, 0};
             add128(acc, w1 << 21, w1 >> 43);
             add128(acc, w2 << 42, w2 >> 22);
             add128(acc, w3 << 63, w3 >> 1);
+            if constexpr (MODE == kConvWide0) add128(acc, 0, d2u(v4) << 20);
             o[(size_t)sm_itt[g] * N] = redc_t(acc, sm_it[g]);
         }
     } else {
@@ -220,8 +236,9 @@ __global__ void __launch_bounds__(256)
         for (int s = 0; s < NS; s++) {
             double m0 = sm_fm[s * kConvMaxTargets + f], m1 = sm_fm[s * kConvMaxTargets + f1];
             double y0 = yd[s], y1 = yd[s];
-            if constexpr (!NARROW) {
-                if (pr[s0 + s].q >= kFpPrimeLimit) {  // a wide source residue first drops to [0, 2t)
+            if constexpr (MODE != kConvNarrow) {
+                if ((MODE == kConvGeneric || s == 0) && pr[s0 + s].q >= kFpPrimeLimit) {
+                    // a wide source residue first drops to [0, 2t)
                     const ConvTarget t0 = sm_ft[f], t1 = sm_ft[f1];
                     y0 = u2d(y[s] - __umul64hi(y[s], t0.one_shoup) * t0.q);
                     y1 = u2d(y[s] - __umul64hi(y[s], t1.one_shoup) * t1.q);
@@ -604,22 +621,29 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
                 cl.int_tt[cl.n_int++] = (uint8_t)tt;
         }
         if (cl.n_int > kConvMaxInt) return set_err(c, HE_EINVAL, "key switch: %d wide targets unsupported", cl.n_int);
-        switch (ns * 2 + (narrow_j ? 1 : 0)) {
-#define HE_MU_CASE(S)                                                                                             \
-    case 2 * S:                                                                                                   \
-        k_modup_conv<S, false><<<dim3(gx, n), blk, 0, c->stream>>>(coef, ext_j, ma.src[j], ma.mat[j], ma, cl,       \
-                                                                   c->d_prime, c->d_fpmod, level, n_rows, s0,     \
-                                                                   c->log_n);                                     \
-        break;                                                                                                    \
-    case 2 * S + 1:                                                                                               \
-        k_modup_conv<S, true><<<dim3(gx, n), blk, 0, c->stream>>>(coef, ext_j, ma.src[j], ma.mat[j], ma, cl,        \
-                                                                  c->d_prime, c->d_fpmod, level, n_rows, s0,      \
-                                                                  c->log_n);                                      \
+        // only the first source 60-bit (the digit holding q_0)?
+        bool wide0 = !narrow_j && !fp_prime(c, s0);
+        for (int s = 1; s < ns && wide0; s++) wide0 = fp_prime(c, s0 + s);
+        const int mode = narrow_j ? kConvNarrow : (wide0 ? kConvWide0 : kConvGeneric);
+        switch (ns * 3 + mode) {
+#define HE_MU_LAUNCH(S, MD)                                                                                        \
+    k_modup_conv<S, MD><<<dim3(gx, n), blk, 0, c->stream>>>(coef, ext_j, ma.src[j], ma.mat[j], ma, cl, c->d_prime, \
+                                                           c->d_fpmod, level, n_rows, s0, c->log_n)
+#define HE_MU_CASE(S)                      \
+    case 3 * S + kConvGeneric:             \
+        HE_MU_LAUNCH(S, kConvGeneric);     \
+        break;                             \
+    case 3 * S + kConvNarrow:              \
+        HE_MU_LAUNCH(S, kConvNarrow);      \
+        break;                             \
+    case 3 * S + kConvWide0:               \
+        HE_MU_LAUNCH(S, kConvWide0);       \
         break;
             HE_MU_CASE(1) HE_MU_CASE(2) HE_MU_CASE(3) HE_MU_CASE(4) HE_MU_CASE(5) HE_MU_CASE(6) HE_MU_CASE(7)
             HE_MU_CASE(8) HE_MU_CASE(9) HE_MU_CASE(10) HE_MU_CASE(11) HE_MU_CASE(12) HE_MU_CASE(13)
             HE_MU_CASE(14) HE_MU_CASE(15) HE_MU_CASE(16)
 #undef HE_MU_CASE
+#undef HE_MU_LAUNCH
             default:
                 return set_err(c, HE_EINVAL, "key switch: digit of %d primes unsupported", ns);
         }
@@ -631,8 +655,10 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
             prods += (double)ma.n_src[j] * (1 + n_rows - ma.n_src[j]);
             // FP64 pipe: 40-bit targets, and every target of a digit of 40-bit
             // sources (exact FP64 partial sums, six FMAs per product)
-            int narrow_j = 1;
+            int narrow_j = 1, wide0 = !fp_prime(c, ma.src_row[j]);  // digit all 40-bit / only its first source 60-bit
             for (int s = 0; s < ma.n_src[j]; s++) narrow_j &= fp_prime(c, ma.src_row[j] + s);
+            for (int s = 1; s < ma.n_src[j]; s++) wide0 &= fp_prime(c, ma.src_row[j] + s);
+            narrow_j |= wide0;
             for (int t = 0; t < n_rows; t++)
                 if ((t < ma.src_row[j] || t >= ma.src_row[j] + ma.n_src[j]) && (narrow_j || fp_prime(c, ep[t])))
                     prods_fp += ma.n_src[j];
