@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(256)
 // ND = number of digits (compile time, so that every load of a thread is in
 // flight at once).
 template <int ND>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 5)  // 5 blocks per SM: more loads in flight than at 4
     k_ks_inner(const uint64_t* __restrict__ ext, PtrList din, GalList gal, PtrList keys, uint64_t* __restrict__ u,
                int n_rows, int level, int L, int LK, int n_cts, const DevPrime* __restrict__ pr,
                const FpMod* __restrict__ fpm, ModupArgs a, int logn) {
