@@ -120,7 +120,7 @@ struct ConvLists {
 constexpr int kConvGeneric = 0, kConvNarrow = 1, kConvWide0 = 2;
 
 template <int NS, int MODE>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)  // measured: better than 3 blocks per SM despite small spills
     k_modup_conv(const uint64_t* __restrict__ coef, uint64_t* __restrict__ ext_j, const ulonglong2* __restrict__ src,
                  const ulonglong2* __restrict__ mat, ModupArgs a, const __grid_constant__ ConvLists cl,
                  const DevPrime* __restrict__ pr,
