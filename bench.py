@@ -636,11 +636,14 @@ def run_native(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
-# ncu dram bytes (read + write) over algorithmic bytes, per kernel class, from
-# the committed capture in profiles/ (rotation of 8 ciphertexts at level 24;
-# the ratio carries over to the benchmark's launches, which move the same
-# rows per ciphertext).  Remove an entry when its kernel changes.
-NCU_TRAFFIC_RATIO = {}
+# ncu dram bytes (read + write) over algorithmic bytes per launch, per kernel
+# class, from the committed capture of that kernel (profiles/
+# ntt_passes_n65536_512limbs_full.md: 512 limbs, 268.4 MB each way).  Reads
+# grow in proportion to the limbs a launch transforms; the small case leaves
+# some written lines in L2 at its end, so the ratio slightly undercounts
+# writes.  Remove an entry when its kernel changes.
+NCU_TRAFFIC_RATIO = {"ntt_fwd_cols": (268.57344 + 220.00768) / 536.870912,
+                     "ntt_inv_cols": (268.57728 + 217.766912) / 536.870912}
 
 
 def roofline_for(name, prof_entry, int_modmul_s, fp_modmul_s, hbm_peak, pk_kind):
