@@ -23,6 +23,14 @@ constexpr int kPmThreadsX = 32, kPmG = 8;
 // Scratch words of sums and rotated sums a wave of output blocks may hold (8 GiB).
 constexpr size_t kBsgsWaveWords = (size_t)1 << 30;
 
+// 16-byte asynchronous copy global -> shared (both 16-byte aligned)
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+                 "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Element of the staged tile: the residue as a double (FP64 limbs) or as is.
 __device__ __forceinline__ void stage_put(uint64_t* dst, uint64_t v, bool fp) {
     *dst = fp ? (uint64_t)__double_as_longlong(u2d(v)) : v;
@@ -37,7 +45,7 @@ __global__ void __launch_bounds__(kPmThreadsX* kPmG)
                   int n_groups, int n_in, int gs, int bs, int level, const DevPrime* __restrict__ pr,
                   const FpMod* __restrict__ fpm, int logn) {
     constexpr int COLS = kPmThreadsX * CPT;
-    extern __shared__ uint64_t sB[];  // [TCH][KB][2][COLS]
+    extern __shared__ __align__(16) uint64_t sB[];  // [TCH][KB][2][COLS]
     const int N = 1 << logn;
     const int KB = n_in * bs;
     const int tx = threadIdx.x % kPmThreadsX, tg = threadIdx.x / kPmThreadsX;
@@ -51,12 +59,20 @@ __global__ void __launch_bounds__(kPmThreadsX* kPmG)
     for (int t0 = 0; t0 < n_groups; t0 += TCH) {
         const int nt = min(TCH, n_groups - t0);
         __syncthreads();
-        for (int idx = threadIdx.x; idx < nt * KB * 2 * COLS; idx += blockDim.x) {
-            const int cc = idx % COLS, rest = idx / COLS;  // rest = (t KB + k) 2 + poly
+        // stage the rotated inputs with asynchronous 16-byte copies (all of a
+        // thread's copies in flight at once), then convert FP64 limbs in place
+        for (int idx = threadIdx.x; idx < nt * KB * COLS; idx += blockDim.x) {
+            const int cc2 = idx % (COLS / 2), rest = idx / (COLS / 2);  // rest = (t KB + k) 2 + poly
             const int poly = rest & 1, tk = rest >> 1, t = tk / KB, k = tk - t * KB;
-            stage_put(sB + idx, B[((size_t)(t0 + t) * KB + k) * ctw + poly * limb + col + cc], fp);
+            cp_async16(sB + (size_t)rest * COLS + 2 * cc2,
+                       B + ((size_t)(t0 + t) * KB + k) * ctw + poly * limb + col + 2 * cc2);
         }
+        cp_async_wait_all();
         __syncthreads();
+        if (fp) {
+            for (int idx = threadIdx.x; idx < nt * KB * 2 * COLS; idx += blockDim.x) stage_put(sB + idx, sB[idx], true);
+            __syncthreads();
+        }
         if (g0 >= gs) continue;
         const bool g1ok = GPT > 1 && g0 + 1 < gs;
         const uint64_t* w_base = pt_i + col + CPT * tx;
