@@ -22,7 +22,9 @@ follows the textbook method it names:
     Homomorphic Encryption", SAC 2018 (CHKKS);
   * hybrid key switching with dnum digits: Han, Ki, "Better Bootstrapping for
     Approximate Homomorphic Encryption", CT-RSA 2020, section 3 (HK);
-  * Paterson-Stockmeyer polynomial evaluation (1973).
+  * Paterson-Stockmeyer polynomial evaluation (1973);
+  * hoisted rotations: Halevi, Shoup, "Faster Homomorphic Linear
+    Transformations in HElib", CRYPTO 2018, section 5.
 Readings taken where the pages are silent are marked "Reading:" below.
 
 Parity pins for every function live in tests/test_oracle_*.py.
@@ -563,6 +565,45 @@ def rotate(ct, step, evk, params):
     return make_ct(np.stack([add_rows(c0, u0, qm), u1]), level, ct["scale"])
 
 
+def rotate_hoisted(ct, steps, keys, params):
+    """Hoisted rotations of one ciphertext (Halevi-Shoup, "Faster
+    homomorphic linear transformations in HElib", section 5): the digits of
+    c1 are raised to Q_level and P once, and each rotation applies sigma_k to
+    the raised digits in the evaluation domain before its inner product:
+
+        rot_step(ct) = (sigma_k(c0) + ModDown(sum_j sigma_k(ModUp_j(c1)) (.) evk_j.b),
+                                      ModDown(sum_j sigma_k(ModUp_j(c1)) (.) evk_j.a)).
+
+    sigma_k is a signed permutation of coefficients and the fast base
+    conversion maps -x to -Conv(x) only up to a multiple of the digit's
+    modulus, so the residues differ from rotate()'s: sigma_k(ModUp_j(c1)) and
+    ModUp_j(sigma_k(c1)) agree on the digit's own rows and differ by
+    m Q_{D_j} (|m| <= |D_j|) per coefficient on the others.  Both are
+    lifts of sigma_k(c1)'s digit, so the result decrypts to the same rotated
+    slots.  keys: step -> switching key.  Returns one ciphertext per step."""
+    level = ct["level"]
+    qm = params.q[:level]
+    ext_mods = qm + params.p
+    key_rows = list(range(level)) + list(range(params.L, params.L + params.K))
+    c1 = ct["c"][1]
+    c1_coeff = intt_rows(c1, qm, params)
+    raised = [modup(c1_coeff, c1, D, level, params) for D in params.digits(level)]
+    out = []
+    for step in steps:
+        k = params.galois_elt(step)
+        b, a = keys[step]
+        u0 = np.zeros((level + params.K, params.N), dtype=np.uint64)
+        u1 = np.zeros_like(u0)
+        for j, ext in enumerate(raised):
+            ext_k = automorph_ntt_rows(ext, k, ext_mods, params)
+            u0 = add_rows(u0, mul_rows(ext_k, b[j][key_rows], ext_mods), ext_mods)
+            u1 = add_rows(u1, mul_rows(ext_k, a[j][key_rows], ext_mods), ext_mods)
+        c0 = automorph_ntt_rows(ct["c"][0], k, qm, params)
+        out.append(make_ct(np.stack([add_rows(c0, moddown(u0, level, params), qm), moddown(u1, level, params)]),
+                           level, ct["scale"]))
+    return out
+
+
 # --------------------------------------------------------------------------
 # Multiplication, rescale, helpers
 # --------------------------------------------------------------------------
@@ -682,20 +723,25 @@ def pmult_accum(xs, pts, level, params):
     return acc
 
 
-def bsgs_matvec(X, pt, bs, gs, slot_stride, keys, params, outputs, pt_scale):
+def bsgs_matvec(X, pt, bs, gs, slot_stride, keys, params, outputs, pt_scale, hoisted=False):
     """Y_i = rescale( sum_g rot_{slot_stride bs g}( sum_{j,b} pt[i][j][g][b] (.) rot_{slot_stride b}(X_j) ) ).
 
     X: list of n_in ciphertexts at one level; pt: callable (i, j, g, b) ->
     evaluation-domain plaintext rows at that level, encoded at pt_scale;
     keys: step -> switching key.
-    Baby-step rotations are plain rotations of each X_j; the giant-step sum
-    is over rotated partial sums, followed by one rescale.
+    Baby-step rotations of each X_j are plain rotations, or with hoisted=True
+    the hoisted rotations of rotate_hoisted (one ModUp per X_j); the
+    giant-step sum is over rotated partial sums, followed by one rescale.
     Reading: one rescale after the whole accumulation."""
     level = X[0]["level"]
     qm = params.q[:level]
     n_in = len(X)
-    baby = [[X[j] if b == 0 else rotate(X[j], slot_stride * b, keys[slot_stride * b], params)
-             for b in range(bs)] for j in range(n_in)]
+    if hoisted:
+        steps = [slot_stride * b for b in range(1, bs)]
+        baby = [[X[j]] + rotate_hoisted(X[j], steps, keys, params) for j in range(n_in)]
+    else:
+        baby = [[X[j] if b == 0 else rotate(X[j], slot_stride * b, keys[slot_stride * b], params)
+                 for b in range(bs)] for j in range(n_in)]
     Y = {}
     for i in outputs:
         acc = None

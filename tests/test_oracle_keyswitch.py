@@ -201,3 +201,100 @@ def test_mutation_rotation_direction_is_caught():
     a, e = S.key_draws(seed, P.galois_elt(bad), P.mods, P.N, P.dnum)
     r = C.rotate(ct, bad, C.rotation_key(s, bad, a, e, P), P)
     assert np.max(np.abs(C.decrypt_decode(r, s, P) - np.roll(z, -step))) > 1e-2
+
+
+def _encrypted(P, seed, level):
+    s = S.secret(seed, P.N)
+    pa, pe = S.public_key_draws(seed, P.q, P.N)
+    pk = C.public_key(s, pa, pe, P)
+    z = S.complex_slots(seed, P.n_slots, -1, 1)
+    v, e0, e1 = S.encryption_draws(seed, 0, P.N)
+    ct = C.make_ct(C.encrypt(pk, C.encode(z, 2.0 ** 40, level, P), v, e0, e1, level, P), level, 2.0 ** 40)
+    return s, z, ct
+
+
+def _rot_keys(P, seed, s, steps):
+    keys = {}
+    for st in steps:
+        a, e = S.key_draws(seed, P.galois_elt(st), P.mods, P.N, P.dnum)
+        keys[st] = C.rotation_key(s, st, a, e, P)
+    return keys
+
+
+@pytest.mark.parametrize("mk,level", [("tiny", 3), ("mid", 7), ("mid", 5)])
+def test_hoisted_rotations_decrypt_to_rolled_slots(mk, level):
+    """Every hoisted rotation of one ciphertext decrypts to the input's
+    slots rolled left by its step."""
+    P = _tiny() if mk == "tiny" else _mid()
+    seed = S.master_seed(7)
+    s, z, ct = _encrypted(P, seed, level)
+    steps = [1, 2, -1, 5, 37]
+    keys = _rot_keys(P, seed, s, steps)
+    for st, r in zip(steps, C.rotate_hoisted(ct, steps, keys, P)):
+        assert r["level"] == level and r["scale"] == ct["scale"]
+        assert np.max(np.abs(C.decrypt_decode(r, s, P) - np.roll(z, -st))) < 1e-5
+
+
+@pytest.mark.parametrize("mk,level", [("tiny", 3), ("mid", 6)])
+def test_hoisted_rotation_by_identity_is_the_plain_rotation(mk, level):
+    """sigma_1 is the identity, so hoisting changes nothing: a hoisted
+    rotation by step 0 (Galois element 1) equals rotate() residue for residue."""
+    P = _tiny() if mk == "tiny" else _mid()
+    seed = S.master_seed(8)
+    s, _, ct = _encrypted(P, seed, level)
+    assert P.galois_elt(0) == 1
+    keys = _rot_keys(P, seed, s, [0])
+    got = C.rotate_hoisted(ct, [0], keys, P)[0]
+    want = C.rotate(ct, 0, keys[0], P)
+    assert np.array_equal(got["c"], want["c"])
+
+
+def test_hoisted_raised_digits_differ_by_multiples_of_the_digit_modulus():
+    """sigma_k(ModUp_j(d)) and ModUp_j(sigma_k(d)): equal on the digit's own
+    rows; elsewhere every coefficient differs by m Q_{D_j}, one integer m with
+    |m| <= |D_j| for all the target rows of that coefficient."""
+    P = _mid()
+    level = 7
+    qm = P.q[:level]
+    ext_mods = qm + P.p
+    rng = np.random.default_rng(3)
+    d = np.stack([rng.integers(0, m, size=P.N, dtype=np.uint64) for m in qm])
+    d_coeff = C.intt_rows(d, qm, P)
+    k = P.galois_elt(3)
+    d_rot = C.automorph_ntt_rows(d, k, qm, P)
+    d_rot_coeff = C.intt_rows(d_rot, qm, P)
+    for D in P.digits(level):
+        hoisted = C.intt_rows(C.automorph_ntt_rows(C.modup(d_coeff, d, D, level, P), k, ext_mods, P), ext_mods, P)
+        plain = C.intt_rows(C.modup(d_rot_coeff, d_rot, D, level, P), ext_mods, P)
+        QD = math.prod(qm[i] for i in D)
+        m_ref = None
+        for r, mod in enumerate(ext_mods):
+            diff = (hoisted[r].astype(object) - plain[r].astype(object)) % mod
+            if r in D:
+                assert not diff.any()
+                continue
+            m = C.centered(diff * pow(QD, -1, mod), mod)
+            assert max(abs(int(v)) for v in m) <= len(D)
+            if m_ref is None:
+                m_ref = m
+                assert any(int(v) != 0 for v in m)  # the two lifts do differ
+            else:
+                assert np.array_equal(m, m_ref)
+
+
+def test_mutation_hoisted_digits_left_unpermuted_is_caught(monkeypatch):
+    """Planting a hoisted rotation that permutes c0 but not the raised digits
+    fails the slot pin."""
+    P = _tiny()
+    seed = S.master_seed(9)
+    s, z, ct = _encrypted(P, seed, 3)
+    keys = _rot_keys(P, seed, s, [1])
+    real = C.automorph_ntt_rows
+    n_ext = 3 + P.K
+
+    def planted(a, k, mods, params):
+        return np.array(a, copy=True) if len(mods) == n_ext else real(a, k, mods, params)
+
+    monkeypatch.setattr(C, "automorph_ntt_rows", planted)
+    r = C.rotate_hoisted(ct, [1], keys, P)[0]
+    assert np.max(np.abs(C.decrypt_decode(r, s, P) - np.roll(z, -1))) > 1e-2
