@@ -47,7 +47,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--case", default="rotation",
-                    choices=["rotation", "ntt", "rot_small", "ffn128", "ffn2048", "ps15", "tiny"],
+                    choices=["rotation", "ntt", "rot_small", "ffn128", "ffn2048", "ps15", "tiny", "hoisted"],
                     help="rotation: the headline workload (default). ffn128 / ffn2048 / ps15 / tiny: the other "
                          "workloads, one JSON line each. ntt / rot_small: kernel cases for profiler captures "
                          "(NTT of 512 limbs, or 8 rotations with 2 keys)")
@@ -278,7 +278,7 @@ def workload_cpu_baseline(case, seconds):
     timing)."""
     from oracle import ckks as C
 
-    widx = {"tiny": 0, "ffn128": 2, "ffn2048": 3, "ps15": 4}[case]
+    widx = {"tiny": 0, "hoisted": 1, "ffn128": 2, "ffn2048": 3, "ps15": 4}[case]
     master = S.master_seed(widx)
     t_end = time.perf_counter() + seconds
     if case == "tiny":
@@ -304,6 +304,22 @@ def workload_cpu_baseline(case, seconds):
                 "sample": "%d whole sequences (NTT round trip, 3 rotations, 1 HMult-relin-rescale), N=2^12" % done}
     P = C.Params(LOG_N, L, K, DNUM)
     s = S.secret(master, P.N)
+    if case == "hoisted":
+        steps = workload_inputs(master, P.q, N_CTS)[0][:2]
+        keys = {}
+        for st in steps:
+            a, e = S.key_draws(master, P.galois_elt(st), P.mods, P.N, P.dnum)
+            keys[st] = C.rotation_key(s, st, a, e, P)
+        ct = C.make_ct(S.uniform_residues(master, "ct_residues", P.q, P.N, lead=(2,)), L, 2.0 ** 40)
+        done, t = 0, 0.0
+        while done < 2 or time.perf_counter() < t_end:
+            t0 = time.perf_counter()
+            C.rotate_hoisted(ct, steps, keys, P)
+            t += time.perf_counter() - t0
+            done += len(steps)
+        return {"value": done / t, "unit": "rotations/s", "cores": C.n_threads(), "kind": "oracle",
+                "sample": "%d full-size hoisted rotations (level 24), one ciphertext by 2 steps per call, so one "
+                          "ModUp per 2 rotations; key generation excluded" % done}
     if case == "ps15":
         a, e = S.key_draws(master, 2, P.mods, P.N, P.dnum)
         rlk = C.relin_key(s, a, e, P)
@@ -351,7 +367,9 @@ def run_workload_case(args, local_rank):
     ffn128 (FFN1 768->3072, 128 tokens: 3 x 12 blocks by BSGS at level 12),
     ffn2048 (the same product for 16 token groups sharing the weights),
     ps15 (degree-15 Paterson-Stockmeyer on 64 ciphertexts from level 24),
-    tiny (N=2^12 NTT round trip, 3 rotations and one HMult-relin-rescale).
+    tiny (N=2^12 NTT round trip, 3 rotations and one HMult-relin-rescale),
+    hoisted (4 ciphertexts at level 24 each rotated by the rotation batch's
+    16 steps through one ModUp per ciphertext: 64 hoisted rotations).
     Inputs are seeded uniform residues on the device; the rotation and
     relinearisation keys are computed by the library from seeded draws."""
     import torch
@@ -362,7 +380,7 @@ def run_workload_case(args, local_rank):
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream()
     case = args.case
-    widx = {"tiny": 0, "ffn128": 2, "ffn2048": 3, "ps15": 4}[case]
+    widx = {"tiny": 0, "hoisted": 1, "ffn128": 2, "ffn2048": 3, "ps15": 4}[case]
     master = S.master_seed(widx)
     gen = torch.Generator(device=dev)
     gen.manual_seed(master)
@@ -402,6 +420,23 @@ def run_workload_case(args, local_rank):
         cfg = {"workload": case, "N": N, "level": lvl, "tokens": f["n_tok"] * n_groups, "bs": f["bs"], "gs": f["gs"],
                "rotations_per_step": n_groups * f["n_in"] * (f["bs"] - 1) + n_groups * f["n_out"] * (f["gs"] - 1),
                "weights_gb": pt.numel() * 8 / 1e9}
+    elif case == "hoisted":
+        steps, _ = workload_inputs(master, ctx.primes[:L], N_CTS)
+        for st in steps:
+            upload(he.HE_KEY_ROTATION, st)
+        n_in = N_CTS // N_KEYS
+        x = device_residues(torch, (n_in, 2), ctx.primes[:L], N, gen, dev)
+        y = torch.empty((n_in * N_KEYS, 2, L, N), dtype=torch.int64, device=dev)
+        xs = [he.Ciphertext(x[i], L, 2.0 ** 40) for i in range(n_in)]
+
+        def step():
+            ys = [he.Ciphertext(y[i], L, 2.0 ** 40) for i in range(n_in * N_KEYS)]
+            he.he_rotate_hoisted(ctx, xs, steps, ys)
+
+        metric, unit, per_step = "hoisted rotations/s (4 ciphertexts x 16 steps, N=2^16, level 24)", "rotations/s", \
+            n_in * N_KEYS
+        cfg = {"workload": case, "N": N, "L": L, "K": K, "dnum": DNUM, "level": L, "n_ciphertexts": n_in,
+               "n_steps": N_KEYS, "l2": "inputs and keys larger than L2 (1.6 GB of keys per step)"}
     elif case == "ps15":
         upload(he.HE_KEY_RELIN, 0)
         n = 64
@@ -700,7 +735,7 @@ def main():
             run_ntt_case(args, local_rank)
         elif args.case == "rot_small":
             run_rot_small_case(args, local_rank)
-        elif args.case in ("ffn128", "ffn2048", "ps15", "tiny"):
+        elif args.case in ("ffn128", "ffn2048", "ps15", "tiny", "hoisted"):
             run_workload_case(args, local_rank)
         else:
             run_native(args, rank, world, local_rank)

@@ -232,9 +232,11 @@ extern "C" int he_pmult_accum_bsgs(he_ctx* c, const he_ct* x, int n_in, const ui
     uint64_t* Z = B + ctw * nB;                                 // [wave][n_groups][gs]
     uint64_t* Rg = Z + (size_t)wave * n_groups * gs * ctw;      // same layout (entries g >= 1)
 
-    // baby steps: B[t][j][b] = rot_{stride b}(X[t][j])
-    std::vector<he_ct> bin, bout;
+    // baby steps: B[t][j][b] = rot_{stride b}(X[t][j]), the rotations b >= 1
+    // hoisted (one ModUp per input X[t][j])
+    std::vector<he_ct> bout;
     std::vector<int32_t> bsteps;
+    for (int b = 1; b < bs; b++) bsteps.push_back(stride * b);
     for (int t = 0; t < n_groups; t++)
         for (int j = 0; j < n_in; j++) {
             const he_ct& xi = x[t * n_in + j];
@@ -242,13 +244,9 @@ extern "C" int he_pmult_accum_bsgs(he_ctx* c, const he_ct* x, int n_in, const ui
             rc = check_cuda(c, cudaMemcpyAsync(dst0, xi.data, ctw * 8, cudaMemcpyDeviceToDevice, c->stream),
                             "bsgs copy");
             if (rc) return rc;
-            for (int b = 1; b < bs; b++) {
-                bin.push_back(xi);
-                bout.push_back(he_ct{dst0 + (size_t)b * ctw, level, xi.scale, 1});
-                bsteps.push_back(stride * b);
-            }
+            for (int b = 1; b < bs; b++) bout.push_back(he_ct{dst0 + (size_t)b * ctw, level, xi.scale, 1});
         }
-    if (!bin.empty() && (rc = rotate_many(c, bin.data(), bsteps.data(), bout.data(), (int)bin.size()))) return rc;
+    if (bs > 1 && (rc = rotate_hoisted_many(c, x, n_groups * n_in, bsteps.data(), bs - 1, bout.data()))) return rc;
 
     const size_t pt_block = (size_t)n_in * gs * bs * level * N;
     // one token group: 2 columns per thread; several: 4 groups staged per pass

@@ -141,10 +141,18 @@ struct KsIoList {
     std::vector<uint64_t*> out;
     std::vector<const uint64_t*> add0;
     std::vector<const uint64_t*> add1;
+    // Hoisted mode (non-empty hoist_d): ModUp runs once on each hoist_d[m]
+    // (evaluation rows, no automorphism) and output i takes the raised digits
+    // of hoist_d[hoist_src[i]] through sigma_{galois[i]}; d[i] must then be
+    // hoist_d[hoist_src[i]].
+    std::vector<const uint64_t*> hoist_d;
+    std::vector<int> hoist_src;
 };
 int key_switch(he_ctx* c, int level, const KsIoList& io);
-size_t key_switch_scratch_words(const he_ctx* c, int n, int level);
+int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io);
+size_t key_switch_scratch_words(const he_ctx* c, int n_raised, int n, int level);
 int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, int n);
+int rotate_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t* steps, int n_steps, he_ct* out);
 
 // Scratch slots: 0 = key switching internals, 1 = rescale temporaries,
 // 2 = HMult temporaries and key generation, 3 = driver buffers (polynomial

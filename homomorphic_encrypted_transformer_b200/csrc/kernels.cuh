@@ -43,6 +43,9 @@ struct MutPtrList {
 struct GalList {
     uint64_t g[kMaxBatch];
 };
+struct IdxList {
+    int i[kMaxBatch];
+};
 
 // Evaluation-domain index whose value sigma_k moves to index j (k = 0: j):
 // storage j is the point psi^(2 brev(j)+1); sigma_k(a) there is a(psi^((2 brev(j)+1) k)).

@@ -7,6 +7,7 @@
 //            in the centred range, so the result is round(x/P) - v, |v| <= K/2.
 //   rot_r(ct) = (sigma_k(c0), 0) + KS_{evk_r}(sigma_k(c1)),  k = 5^r mod 2N.
 #include <algorithm>
+#include <set>
 
 #include "he_internal.h"
 #include "ntt.cuh"
@@ -261,12 +262,14 @@ __global__ void __launch_bounds__(256, 4)  // measured: better than 3 blocks per
 // The ciphertext index is the fastest grid dimension: neighbouring blocks
 // that share a key read the same key tile, which DRAM then serves once.
 // ND = number of digits (compile time, so that every load of a thread is in
-// flight at once).
-template <int ND>
+// flight at once).  HOIST: the raised digits belong to ciphertext xsrc[i] of
+// ext (n_ext of them) and are read through sigma_{g_i} as well: the
+// automorphism of a hoisted rotation, applied after ModUp.
+template <int ND, bool HOIST>
 __global__ void __launch_bounds__(256, 5)  // 5 blocks per SM: more loads in flight than at 4
-    k_ks_inner(const uint64_t* __restrict__ ext, PtrList din, GalList gal, PtrList keys, uint64_t* __restrict__ u,
-               int n_rows, int level, int L, int LK, int n_cts, const DevPrime* __restrict__ pr,
-               const FpMod* __restrict__ fpm, ModupArgs a, int logn) {
+    k_ks_inner(const uint64_t* __restrict__ ext, PtrList din, GalList gal, PtrList keys, IdxList xsrc,
+               uint64_t* __restrict__ u, int n_rows, int level, int L, int LK, int n_ext,
+               const DevPrime* __restrict__ pr, const FpMod* __restrict__ fpm, ModupArgs a, int logn) {
     const int N = 1 << logn;
     const int i = blockIdx.x, t = blockIdx.z;
     const int c = 2 * (blockIdx.y * blockDim.x + threadIdx.x);  // positions c, c+1
@@ -286,9 +289,15 @@ __global__ void __launch_bounds__(256, 5)  // 5 blocks per SM: more loads in fli
             const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2*>(din.p[i] + (size_t)t * N + (own & ~1)));
             xs[j] = own_sw ? make_ulonglong2(v.y, v.x) : v;
         } else {
-            int pos = t < s0 ? t : t - ns;
-            xs[j] = __ldg(reinterpret_cast<const ulonglong2*>(
-                ext + ((size_t)a.ext_off[j] * n_cts + (size_t)i * (n_rows - ns) + pos) * N + c));
+            const int pos = t < s0 ? t : t - ns;
+            const uint64_t* e =
+                ext + ((size_t)a.ext_off[j] * n_ext + (size_t)(HOIST ? xsrc.i[i] : i) * (n_rows - ns) + pos) * N;
+            if (HOIST) {
+                const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2*>(e + (own & ~1)));
+                xs[j] = own_sw ? make_ulonglong2(v.y, v.x) : v;
+            } else {
+                xs[j] = __ldg(reinterpret_cast<const ulonglong2*>(e + c));
+            }
         }
         kbs[j] = __ldg(reinterpret_cast<const ulonglong2*>(key + (((size_t)j * 2 + 0) * LK + krow) * N + c));
         kas[j] = __ldg(reinterpret_cast<const ulonglong2*>(key + (((size_t)j * 2 + 1) * LK + krow) * N + c));
@@ -519,11 +528,12 @@ static int lc(he_ctx* c, const char* what) {
     return check_cuda(c, cudaGetLastError(), what);
 }
 
-// coef [n][level], ext [n][sum_j (level+K-|D_j|)], u [n][2][level+K], tmp [n][2][level]
-size_t key_switch_scratch_words(const he_ctx* c, int n, int level) {
+// coef [nm][level], ext [nm][sum_j (level+K-|D_j|)], u [n][2][level+K],
+// tmp [n][2][level]: nm ciphertexts raised by ModUp, n key-switched.
+size_t key_switch_scratch_words(const he_ctx* c, int nm, int n, int level) {
     size_t nd = (level + c->alpha - 1) / c->alpha, nr = level + c->K;
     size_t ext_rows = nd * nr - level;
-    return (size_t)c->N * n * (level + ext_rows + 2 * nr + 2 * level);
+    return (size_t)c->N * ((size_t)nm * (level + ext_rows) + (size_t)n * (2 * nr + 2 * level));
 }
 
 // Launches of the transform-fused kernels for the context's ring degree.
@@ -560,17 +570,24 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     const int n_rows = level + K;
     ModupArgs ma = modup_args(c, level);
     const int nd = ma.n_digits;
+    // hoisted: ModUp raises the nm inputs hoist_d once (no automorphism) and
+    // the inner product reads them through each output's sigma
+    const bool hoist = !io.hoist_d.empty();
+    const int nm = hoist ? (int)io.hoist_d.size() : n;
+    if (nm > kMaxBatch || (hoist && (int)io.hoist_src.size() != n))
+        return set_err(c, HE_EINVAL, "key switch: bad hoisting lists");
     uint64_t* base;
-    int rc = scratch_slot(c, 0, key_switch_scratch_words(c, n, level), &base);
+    int rc = scratch_slot(c, 0, key_switch_scratch_words(c, nm, n, level), &base);
     if (rc) return rc;
     const int ext_rows = nd * n_rows - level;  // sum over digits of the target rows
     uint64_t* coef = base;
-    uint64_t* ext = coef + (size_t)n * level * N;
-    uint64_t* u = ext + (size_t)n * ext_rows * N;
+    uint64_t* ext = coef + (size_t)nm * level * N;
+    uint64_t* u = ext + (size_t)nm * ext_rows * N;
     uint64_t* tmp = u + (size_t)n * 2 * n_rows * N;
 
-    PtrList din, keys;
-    GalList gal;
+    PtrList din, keys, mdin;
+    GalList gal, mgal;
+    IdxList xsrc;
     MdOut mo;
     mo.sig_add0 = io.sig_add0 ? 1 : 0;
     for (int i = 0; i < kMaxBatch; i++) {
@@ -580,6 +597,11 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
         mo.out.p[i] = i < n ? io.out[i] : nullptr;
         mo.add0.p[i] = i < n ? io.add0[i] : nullptr;
         mo.add1.p[i] = i < n ? io.add1[i] : nullptr;
+        mdin.p[i] = hoist ? (i < nm ? io.hoist_d[i] : nullptr) : din.p[i];
+        mgal.g[i] = hoist ? 0 : gal.g[i];
+        xsrc.i[i] = hoist && i < n ? io.hoist_src[i] : i;
+        if (hoist && i < n && (xsrc.i[i] < 0 || xsrc.i[i] >= nm || io.hoist_d[xsrc.i[i]] != io.d[i]))
+            return set_err(c, HE_EINVAL, "key switch: output %d has no raised input", i);
     }
     mo.gal = gal;
     const int TB = 256;
@@ -594,20 +616,21 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     int fp_q = 0;  // primes of Q_level on the FP64 path
     for (int t = 0; t < level; t++) fp_q += fp_prime(c, t);
 
-    // sigma(d) back to coefficients: gathered row pass, then the column pass
+    // sigma(d) (hoisted: d) back to coefficients: gathered row pass, then the
+    // column pass
     prof_begin(c, HE_PROF_NTT_INV_ROWS);
-#define HE_IRG(LN) launch_inv_rows_gather<LN>(c, din, gal, coef, n, level)
+#define HE_IRG(LN) launch_inv_rows_gather<LN>(c, mdin, mgal, coef, nm, level)
     HE_LOGN_SWITCH(c, HE_IRG)
 #undef HE_IRG
     if ((rc = lc(c, "inv_rows_gather"))) return rc;
-    prof_end(c, HE_PROF_NTT_INV_ROWS, 2.0 * n * level * limbB, 0.5 * N * n * level * sh.s2,
-             0.5 * N * n * fp_q * sh.s2);
+    prof_end(c, HE_PROF_NTT_INV_ROWS, 2.0 * nm * level * limbB, 0.5 * N * nm * level * sh.s2,
+             0.5 * N * nm * fp_q * sh.s2);
     std::vector<int> qp = prime_range(0, level);
-    if ((rc = ntt_inv_cols_set(c, rowset_contig(coef, level, N, qp), n * level))) return rc;
+    if ((rc = ntt_inv_cols_set(c, rowset_contig(coef, level, N, qp), nm * level))) return rc;
 
     prof_begin(c, HE_PROF_MODUP);
     for (int j = 0; j < nd; j++) {
-        uint64_t* ext_j = ext + (size_t)ma.ext_off[j] * n * N;
+        uint64_t* ext_j = ext + (size_t)ma.ext_off[j] * nm * N;
         const int s0 = ma.src_row[j], ns = ma.n_src[j];
         bool narrow_j = true;  // every source prime of the digit below 2^41
         for (int s = 0; s < ns; s++) narrow_j = narrow_j && fp_prime(c, s0 + s);
@@ -627,7 +650,7 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
         const int mode = narrow_j ? kConvNarrow : (wide0 ? kConvWide0 : kConvGeneric);
         switch (ns * 3 + mode) {
 #define HE_MU_LAUNCH(S, MD)                                                                                        \
-    k_modup_conv<S, MD><<<dim3(gx, n), blk, 0, c->stream>>>(coef, ext_j, ma.src[j], ma.mat[j], ma, cl, c->d_prime, \
+    k_modup_conv<S, MD><<<dim3(gx, nm), blk, 0, c->stream>>>(coef, ext_j, ma.src[j], ma.mat[j], ma, cl, c->d_prime, \
                                                            c->d_fpmod, level, n_rows, s0, c->log_n)
 #define HE_MU_CASE(S)                      \
     case 3 * S + kConvGeneric:             \
@@ -663,16 +686,16 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
                 if ((t < ma.src_row[j] || t >= ma.src_row[j] + ma.n_src[j]) && (narrow_j || fp_prime(c, ep[t])))
                     prods_fp += ma.n_src[j];
         }
-        prof_end(c, HE_PROF_MODUP, (double)n * (sum_src + ext_rows) * limbB, (double)n * N * prods,
-                 (double)n * N * prods_fp);
+        prof_end(c, HE_PROF_MODUP, (double)nm * (sum_src + ext_rows) * limbB, (double)nm * N * prods,
+                 (double)nm * N * prods_fp);
     }
     for (int j = 0; j < nd; j++) {
         std::vector<int> tp;
         for (int t = 0; t < n_rows; t++)
             if (t < ma.src_row[j] || t >= ma.src_row[j] + ma.n_src[j]) tp.push_back(ep[t]);
         const int nt = (int)tp.size();
-        RowSet rs = rowset_contig(ext + (size_t)ma.ext_off[j] * n * N, nt, N, tp);
-        if ((rc = ntt_fwd_set(c, rs, n * nt))) return rc;
+        RowSet rs = rowset_contig(ext + (size_t)ma.ext_off[j] * nm * N, nt, N, tp);
+        if ((rc = ntt_fwd_set(c, rs, nm * nt))) return rc;
     }
 
     prof_begin(c, HE_PROF_KS_INNER);
@@ -680,8 +703,12 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     switch (nd) {
 #define HE_KS_CASE(D)                                                                                             \
     case D:                                                                                                       \
-        k_ks_inner<D><<<dim3(n, gx2, n_rows), blk, 0, c->stream>>>(ext, din, gal, keys, u, n_rows, level, L, LK, n, \
-                                                                  c->d_prime, c->d_fpmod, ma, c->log_n);         \
+        if (hoist)                                                                                                \
+            k_ks_inner<D, true><<<dim3(n, gx2, n_rows), blk, 0, c->stream>>>(                                     \
+                ext, din, gal, keys, xsrc, u, n_rows, level, L, LK, nm, c->d_prime, c->d_fpmod, ma, c->log_n);    \
+        else                                                                                                      \
+            k_ks_inner<D, false><<<dim3(n, gx2, n_rows), blk, 0, c->stream>>>(                                    \
+                ext, din, gal, keys, xsrc, u, n_rows, level, L, LK, nm, c->d_prime, c->d_fpmod, ma, c->log_n);    \
         break;
         HE_KS_CASE(1) HE_KS_CASE(2) HE_KS_CASE(3) HE_KS_CASE(4) HE_KS_CASE(5) HE_KS_CASE(6) HE_KS_CASE(7)
         HE_KS_CASE(8) HE_KS_CASE(9) HE_KS_CASE(10) HE_KS_CASE(11) HE_KS_CASE(12) HE_KS_CASE(13) HE_KS_CASE(14)
@@ -692,9 +719,15 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     }
     if ((rc = lc(c, "ks_inner"))) return rc;
     {
+        // raised digits of each raised input once, each distinct key once,
+        // the products written once
         int fp_rows_ks = 0;
         for (int t = 0; t < n_rows; t++) fp_rows_ks += fp_prime(c, ep[t]);
-        prof_end(c, HE_PROF_KS_INNER, ((double)n * nd * n_rows + 2.0 * nd * n_rows + 2.0 * n * n_rows) * limbB,
+        std::vector<const uint64_t*> kd(io.key.begin(), io.key.begin() + n);
+        std::sort(kd.begin(), kd.end());
+        const double n_keys = (double)(std::unique(kd.begin(), kd.end()) - kd.begin());
+        prof_end(c, HE_PROF_KS_INNER,
+                 ((double)nm * nd * n_rows + n_keys * 2.0 * nd * n_rows + 2.0 * n * n_rows) * limbB,
                  (double)n * n_rows * N * 2.0 * nd, (double)n * fp_rows_ks * N * 2.0 * nd);
     }
 
@@ -823,9 +856,93 @@ int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, in
     return HE_OK;
 }
 
+// Hoisted rotations (Halevi-Shoup, CRYPTO 2018, section 5):
+// out[i n_steps + s] = (sigma_k(c0) + ModDown(sum_j sigma_k(ModUp_j(c1)) (.) evk_j.b),
+//                        ModDown(sum_j sigma_k(ModUp_j(c1)) (.) evk_j.a)),  k = 5^steps[s],
+// for the inputs in[i] = (c0, c1).  ModUp runs once per input and chunk of
+// steps; each output reads the raised digits through its automorphism inside
+// the inner product.  Outputs are ordered step-major within a chunk, so
+// neighbouring inner-product blocks share a key tile.  Steps whose Galois
+// element is 1 are copies.
+int rotate_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t* steps, int n_steps, he_ct* out) {
+    if (n_in < 0 || n_steps < 0) return set_err(c, HE_EINVAL, "rotate_hoisted: negative count");
+    if (n_in == 0 || n_steps == 0) return HE_OK;
+    if (!in || !out || !steps) return set_err(c, HE_EINVAL, "rotate_hoisted: null argument");
+    const int level = in[0].level;
+    std::set<const uint64_t*> ins;
+    for (int i = 0; i < n_in; i++) {
+        int rc = ct_ok(c, &in[i], "rotate_hoisted");
+        if (rc) return rc;
+        if (in[i].level != level) return set_err(c, HE_ELEVEL, "rotate_hoisted: mixed levels");
+        ins.insert(in[i].data);
+    }
+    for (long long o = 0; o < (long long)n_in * n_steps; o++) {
+        if (!out[o].data || ((uintptr_t)out[o].data & 15))
+            return set_err(c, HE_EINVAL, "rotate_hoisted: null or unaligned output %lld", o);
+        if (ins.count(out[o].data)) return set_err(c, HE_EINVAL, "rotate_hoisted: output %lld aliases an input", o);
+    }
+    std::vector<int> eff;  // steps that key-switch
+    std::vector<uint64_t> gal(n_steps);
+    for (int s = 0; s < n_steps; s++) {
+        gal[s] = galois_elt(c, steps[s]);
+        if (gal[s] == 1) continue;
+        if (!c->rot_keys.count(gal[s]))
+            return set_err(c, HE_ENOKEY, "rotate_hoisted: no key for step %d (galois %llu)", steps[s],
+                           (unsigned long long)gal[s]);
+        eff.push_back(s);
+    }
+    const size_t N = c->N, ct_words = (size_t)2 * level * N;
+    for (int s = 0; s < n_steps; s++)
+        if (gal[s] == 1)
+            for (int i = 0; i < n_in; i++) {
+                int rc = check_cuda(c, cudaMemcpyAsync(out[(size_t)i * n_steps + s].data, in[i].data, ct_words * 8,
+                                                       cudaMemcpyDeviceToDevice, c->stream), "rotate_hoisted copy");
+                if (rc) return rc;
+            }
+    // chunks of ms steps x mi inputs, at most kMaxBatch outputs each
+    const int ne = (int)eff.size();
+    const int ms = std::min(ne, kMaxBatch), mi = ne ? std::max(1, kMaxBatch / ms) : 1;
+    for (int e0 = 0; e0 < ne; e0 += ms)
+        for (int i0 = 0; i0 < n_in; i0 += mi) {
+            const int se = std::min(ne, e0 + ms), ie = std::min(n_in, i0 + mi);
+            KsIoList io;
+            io.sig_add0 = true;
+            for (int i = i0; i < ie; i++) io.hoist_d.push_back(in[i].data + (size_t)level * N);
+            for (int e = e0; e < se; e++) {
+                const int s = eff[e];
+                const uint64_t* key = c->rot_keys[gal[s]].d;
+                for (int i = i0; i < ie; i++) {
+                    io.galois.push_back(gal[s]);
+                    io.key.push_back(key);
+                    io.d.push_back(in[i].data + (size_t)level * N);
+                    io.out.push_back(out[(size_t)i * n_steps + s].data);
+                    io.add0.push_back(in[i].data);
+                    io.add1.push_back(nullptr);
+                    io.hoist_src.push_back(i - i0);
+                }
+            }
+            int rc = key_switch_chunk(c, (int)io.d.size(), level, io);
+            if (rc) return rc;
+        }
+    for (int i = 0; i < n_in; i++)
+        for (int s = 0; s < n_steps; s++) {
+            he_ct& o = out[(size_t)i * n_steps + s];
+            o.level = level;
+            o.scale = in[i].scale;
+            o.is_ntt = 1;
+        }
+    return HE_OK;
+}
+
 }  // namespace he
 
 using namespace he;
+
+extern "C" int he_rotate_hoisted(he_ctx* c, const he_ct* in, int n_in, const int32_t* steps, int n_steps,
+                                 he_ct* out) {
+    if (!c) return HE_EINVAL;
+    return rotate_hoisted_many(c, in, n_in, steps, n_steps, out);
+}
 
 extern "C" int he_rotate(he_ctx* c, const he_ct* in, int32_t step, he_ct* out) {
     if (!c) return HE_EINVAL;

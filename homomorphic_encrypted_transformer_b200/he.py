@@ -81,6 +81,7 @@ _sig("he_ntt_fwd", _i, _vp, _vp, _i, _i, _i)
 _sig("he_ntt_inv", _i, _vp, _vp, _i, _i, _i)
 _sig("he_rotate", _i, _vp, ctypes.POINTER(he_ct), ctypes.c_int32, ctypes.POINTER(he_ct))
 _sig("he_rotate_batch", _i, _vp, ctypes.POINTER(he_ct), _vp, ctypes.POINTER(he_ct), _i)
+_sig("he_rotate_hoisted", _i, _vp, ctypes.POINTER(he_ct), _i, _vp, _i, ctypes.POINTER(he_ct))
 _sig("he_rotate_batch_host", _i, _vp, _vp, _i, _vp, _vp, _i)
 _sig("he_hmult_relin_rescale", _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct), ctypes.POINTER(he_ct))
 _sig("he_rescale", _i, _vp, ctypes.POINTER(he_ct))
@@ -263,6 +264,19 @@ def he_rotate_batch(ctx, cts_in, steps, cts_out):
     ao = (he_ct * n)(*[c._c() for c in cts_out])
     st = np.ascontiguousarray(steps, dtype=np.int32)
     _check(ctx, _lib.he_rotate_batch(ctx.ptr, ai, _ptr(st), ao, n))
+    for c, o in zip(cts_out, ao):
+        c._update(o)
+
+
+def he_rotate_hoisted(ctx, cts_in, steps, cts_out):
+    """cts_out[i * len(steps) + s] = hoisted rotation of cts_in[i] by steps[s]."""
+    n_in, n_steps = len(cts_in), len(steps)
+    if len(cts_out) != n_in * n_steps:
+        raise ValueError("he_rotate_hoisted: need len(cts_in) * len(steps) outputs")
+    ai = (he_ct * max(1, n_in))(*[c._c() for c in cts_in])
+    ao = (he_ct * max(1, len(cts_out)))(*[c._c() for c in cts_out])
+    st = np.ascontiguousarray(steps, dtype=np.int32)
+    _check(ctx, _lib.he_rotate_hoisted(ctx.ptr, ai, n_in, _ptr(st), n_steps, ao))
     for c, o in zip(cts_out, ao):
         c._update(o)
 

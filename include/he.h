@@ -163,6 +163,25 @@ int he_rotate_batch(he_ctx* ctx, const he_ct* in, const int32_t* steps, he_ct* o
  * not overlap h_in.  Synchronous. */
 int he_rotate_batch_host(he_ctx* ctx, const uint64_t* h_in, int level, const int32_t* steps,
                          uint64_t* h_out, int n);
+/*
+ * Hoisted rotations (Halevi-Shoup, "Faster Homomorphic Linear Transformations
+ * in HElib", CRYPTO 2018, section 5): every input rotated by every step, with
+ * one ModUp per input shared by all its steps.  For in[i] = (c0, c1) and
+ * k = 5^(steps[s] mod N/2) mod 2N,
+ *   out[i*n_steps + s] = (sigma_k(c0) + ModDown(sum_j sigma_k(ModUp_j(c1)) (.) evk_j.b),
+ *                                       ModDown(sum_j sigma_k(ModUp_j(c1)) (.) evk_j.a)),
+ * sigma_k applied to the raised digits in the evaluation domain.  The
+ * residues differ from he_rotate's (the fast base conversion commutes with
+ * sigma_k only up to multiples of each digit's modulus), the decrypted slots
+ * do not: slot j of out[i*n_steps + s] = slot j + steps[s] of in[i].
+ * in: n_in device ciphertexts at one level, 16-byte aligned; out: n_in *
+ * n_steps device ciphertexts, none overlapping an input, each given in[i]'s
+ * level and scale.  A step whose Galois element is 1 copies.  Errors:
+ * HE_EINVAL (null, unaligned, aliasing, negative counts), HE_ELEVEL (mixed or
+ * out-of-range levels), HE_EDOMAIN (an input not in the evaluation domain),
+ * HE_ENOKEY (a step without a rotation key); nothing is launched then.
+ */
+int he_rotate_hoisted(he_ctx* ctx, const he_ct* in, int n_in, const int32_t* steps, int n_steps, he_ct* out);
 
 /* Tensor, relinearise (key switch of d2 with the s^2 key), rescale.
  * a and b at the same level l >= 2; out at level l-1, scale (sa*sb)/q_{l-1}.
@@ -209,6 +228,9 @@ int he_drop_level(he_ctx* ctx, const he_ct* in, int level, he_ct* out);
  *       encoded at pt_scale.
  * y: n_groups*n_out ciphertexts (group-major) with room for level l; they
  *    come back at level l-1, scale x.scale*pt_scale/q_{l-1}.
+ * The baby-step rotations rot_{stride*b}(X[t][j]) are the hoisted rotations of
+ * he_rotate_hoisted (one ModUp per input); the giant-step rotations are
+ * he_rotate_batch's.
  * Needs rotation keys for stride*b (0<b<bs) and stride*bs*g (0<g<gs).
  */
 int he_pmult_accum_bsgs(he_ctx* ctx, const he_ct* x, int n_in, const uint64_t* d_pt, double pt_scale,

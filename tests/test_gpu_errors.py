@@ -89,3 +89,23 @@ def test_bsgs_and_polynomial_errors():
     st7 = Setup(12, 8, 3, 3, seed=64)
     x7 = st7.to_gpu(st7.encrypt(z, 8))
     assert _code(he.he_poly_eval_ps15, st7.ctx, [x7], coeffs, 2.0 ** 62, [st7.empty_gpu(8)]) == he.HE_ENOKEY
+
+
+def test_hoisted_rotation_errors():
+    he = lib()
+    st = Setup(12, 3, 1, 3, seed=65)
+    st.upload_rot(1)
+    z = S.complex_slots(st.seed, st.P.n_slots, -1, 1)
+    x3 = st.to_gpu(st.encrypt(z, 3))
+    x2 = st.to_gpu(st.encrypt(z, 2), room=3)
+    y = [st.empty_gpu(3), st.empty_gpu(3)]
+    assert _code(he.he_rotate_hoisted, st.ctx, [x3], [1, 4], y) == he.HE_ENOKEY
+    assert _code(he.he_rotate_hoisted, st.ctx, [x3, x2], [1], y) == he.HE_ELEVEL
+    assert _code(he.he_rotate_hoisted, st.ctx, [x3], [1, 1], [y[0], x3]) == he.HE_EINVAL  # aliases the input
+    raw = torch.zeros(2 * 3 * st.P.N + 1, dtype=torch.int64, device="cuda")
+    assert _code(he.he_rotate_hoisted, st.ctx, [x3], [1], [he.Ciphertext(raw[1:], 3, 1.0)]) == he.HE_EINVAL
+    # the context still rotates correctly afterwards
+    he.he_rotate_hoisted(st.ctx, [x3], [1], y[:1])
+    he.he_sync(st.ctx)
+    want = C.rotate_hoisted(st.encrypt(z, 3), [1], {1: st.oracle_rot_key(1)}, st.P)[0]
+    assert np.array_equal(st.from_gpu(y[0]), want["c"])

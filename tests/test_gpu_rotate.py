@@ -178,3 +178,59 @@ def test_rotation_batch_host_buffers_pipelined():
     h_out2 = np.zeros_like(h_in)
     he.he_rotate_batch_host(st.ctx, h_in, 3, steps, h_out2)
     assert np.array_equal(h_out2, h_out)
+
+
+def _hoisted_case(st, level, n_in, steps):
+    """he_rotate_hoisted of n_in encrypted inputs by `steps` against the
+    oracle's rotate_hoisted, residue for residue; Galois element 1 copies."""
+    he = lib()
+    P = st.P
+    eff = [s for s in steps if P.galois_elt(s) != 1]
+    for s in sorted(set(eff)):
+        st.upload_rot(s)
+    keys = {s: st.oracle_rot_key(s) for s in eff}
+    cts = [st.encrypt(S.complex_slots(st.seed, P.n_slots, -1, 1, i), level, ct_id=i) for i in range(n_in)]
+    xs = [st.to_gpu(ct) for ct in cts]
+    ys = [st.empty_gpu(level) for _ in range(n_in * len(steps))]
+    he.he_rotate_hoisted(st.ctx, xs, steps, ys)
+    he.he_sync(st.ctx)
+    for i, ct in enumerate(cts):
+        want = dict(zip(eff, C.rotate_hoisted(ct, eff, keys, P)))
+        for k, s in enumerate(steps):
+            y = ys[i * len(steps) + k]
+            assert y.level == level and y.scale == ct["scale"]
+            got = st.from_gpu(y)
+            if P.galois_elt(s) == 1:
+                assert np.array_equal(got, ct["c"])
+            else:
+                assert np.array_equal(got, want[s]["c"]), (i, s)
+    return cts, ys
+
+
+def test_rotation_hoisted_tiny():
+    """Two inputs, steps {1, 2, -1, 0}: step 0 (Galois element 1) copies;
+    every output also decrypts to the rolled slots."""
+    st = Setup(12, 3, 1, 3, seed=S.master_seed(0))
+    steps = [1, 2, -1, 0]
+    cts, ys = _hoisted_case(st, 3, 2, steps)
+    for i, ct in enumerate(cts):
+        z = S.complex_slots(st.seed, st.P.n_slots, -1, 1, i)
+        for k, s in enumerate(steps):
+            got = C.make_ct(st.from_gpu(ys[i * len(steps) + k]), 3, ct["scale"])
+            assert np.max(np.abs(C.decrypt_decode(got, st.s, st.P) - np.roll(z, -s))) < 1e-5
+
+
+@pytest.mark.parametrize("level", [7, 5, 1])
+def test_rotation_hoisted_mid_levels(level):
+    """Several primes per digit (alpha = 3, 60-bit and 40-bit rows), partial
+    last digits, level 1."""
+    st = Setup(11, 7, 3, 3, seed=45)
+    _hoisted_case(st, level, 3, [5, -3, 17])
+
+
+def test_rotation_hoisted_chunks():
+    """More outputs than one launch holds: 5 inputs x 20 steps (chunks of
+    3 and 2 inputs), and 1 input x 70 steps (chunks of 64 and 6 steps)."""
+    st = Setup(11, 3, 1, 3, seed=46)
+    _hoisted_case(st, 3, 5, list(range(1, 21)))
+    _hoisted_case(st, 2, 1, list(range(-35, 0)) + list(range(1, 36)))
