@@ -24,7 +24,10 @@ follows the textbook method it names:
     Approximate Homomorphic Encryption", CT-RSA 2020, section 3 (HK);
   * Paterson-Stockmeyer polynomial evaluation (1973);
   * hoisted rotations: Halevi, Shoup, "Faster Homomorphic Linear
-    Transformations in HElib", CRYPTO 2018, section 5.
+    Transformations in HElib", CRYPTO 2018, section 5;
+  * one ModDown for a sum of rotations: Bossuat, Mouchet, Troncoso-Pastoriza,
+    Hubaux, "Efficient Bootstrapping for Approximate Homomorphic Encryption
+    with Non-Sparse Keys", EUROCRYPT 2021, section 4.
 Readings taken where the pages are silent are marked "Reading:" below.
 
 Parity pins for every function live in tests/test_oracle_*.py.
@@ -604,6 +607,40 @@ def rotate_hoisted(ct, steps, keys, params):
     return out
 
 
+def rotate_sum(zs, steps, keys, params):
+    """sum_g rot_{steps[g]}(zs[g]) with a single ModDown per polynomial
+    (the ModDown hoisting of Bossuat, Mouchet, Troncoso-Pastoriza, Hubaux,
+    "Efficient Bootstrapping for Approximate Homomorphic Encryption with
+    Non-Sparse Keys", EUROCRYPT 2021, section 4): each rotation's key inner
+    product stays in Q_level and P, the products are summed there, and
+
+        result = (sum_g sigma_g(z0_g) + ModDown(sum_g u0_g),  ModDown(sum_g u1_g)),
+        u_g = sum_j ModUp_j(sigma_g(z1_g)) (.) evk_{g,j}.
+
+    ModDown rounds once instead of once per rotation, so the residues differ
+    from the sum of rotate() results by the rounding of the sum; with one
+    rotation they are rotate()'s.  keys: step -> switching key."""
+    level = zs[0]["level"]
+    qm = params.q[:level]
+    ext_mods = qm + params.p
+    key_rows = list(range(level)) + list(range(params.L, params.L + params.K))
+    u0 = np.zeros((level + params.K, params.N), dtype=np.uint64)
+    u1 = np.zeros_like(u0)
+    c0 = np.zeros((level, params.N), dtype=np.uint64)
+    for z, step in zip(zs, steps):
+        k = params.galois_elt(step)
+        b, a = keys[step]
+        c0 = add_rows(c0, automorph_ntt_rows(z["c"][0], k, qm, params), qm)
+        d = automorph_ntt_rows(z["c"][1], k, qm, params)
+        d_coeff = intt_rows(d, qm, params)
+        for j, D in enumerate(params.digits(level)):
+            ext = modup(d_coeff, d, D, level, params)
+            u0 = add_rows(u0, mul_rows(ext, b[j][key_rows], ext_mods), ext_mods)
+            u1 = add_rows(u1, mul_rows(ext, a[j][key_rows], ext_mods), ext_mods)
+    return make_ct(np.stack([add_rows(c0, moddown(u0, level, params), qm), moddown(u1, level, params)]),
+                   level, zs[0]["scale"])
+
+
 # --------------------------------------------------------------------------
 # Multiplication, rescale, helpers
 # --------------------------------------------------------------------------
@@ -723,15 +760,17 @@ def pmult_accum(xs, pts, level, params):
     return acc
 
 
-def bsgs_matvec(X, pt, bs, gs, slot_stride, keys, params, outputs, pt_scale, hoisted=False):
+def bsgs_matvec(X, pt, bs, gs, slot_stride, keys, params, outputs, pt_scale, hoisted=False, one_moddown=False):
     """Y_i = rescale( sum_g rot_{slot_stride bs g}( sum_{j,b} pt[i][j][g][b] (.) rot_{slot_stride b}(X_j) ) ).
 
     X: list of n_in ciphertexts at one level; pt: callable (i, j, g, b) ->
     evaluation-domain plaintext rows at that level, encoded at pt_scale;
     keys: step -> switching key.
     Baby-step rotations of each X_j are plain rotations, or with hoisted=True
-    the hoisted rotations of rotate_hoisted (one ModUp per X_j); the
-    giant-step sum is over rotated partial sums, followed by one rescale.
+    the hoisted rotations of rotate_hoisted (one ModUp per X_j).  The
+    giant-step sum is over rotated partial sums Z_g: plain rotations added
+    one by one, or with one_moddown=True Z_0 + rotate_sum(Z_1..Z_{gs-1}) (one
+    ModDown per output).  One rescale follows.
     Reading: one rescale after the whole accumulation."""
     level = X[0]["level"]
     qm = params.q[:level]
@@ -744,18 +783,23 @@ def bsgs_matvec(X, pt, bs, gs, slot_stride, keys, params, outputs, pt_scale, hoi
                  for b in range(bs)] for j in range(n_in)]
     Y = {}
     for i in outputs:
-        acc = None
+        zs = []
         for g in range(gs):
             xs, pts = [], []
             for j in range(n_in):
                 for b in range(bs):
                     xs.append(baby[j][b])
                     pts.append(pt(i, j, g, b))
-            z = make_ct(pmult_accum(xs, pts, level, params), level, X[0]["scale"] * pt_scale)
-            if g > 0:
-                z = rotate(z, slot_stride * bs * g, keys[slot_stride * bs * g], params)
-            acc = z if acc is None else make_ct(np.stack([add_rows(acc["c"][c], z["c"][c], qm) for c in range(2)]),
-                                                level, acc["scale"])
+            zs.append(make_ct(pmult_accum(xs, pts, level, params), level, X[0]["scale"] * pt_scale))
+        giant = [slot_stride * bs * g for g in range(1, gs)]
+        if one_moddown and gs > 1:
+            r = rotate_sum(zs[1:], giant, keys, params)
+            parts = [zs[0], r]
+        else:
+            parts = [zs[0]] + [rotate(z, st, keys[st], params) for z, st in zip(zs[1:], giant)]
+        acc = parts[0]
+        for z in parts[1:]:
+            acc = make_ct(np.stack([add_rows(acc["c"][c], z["c"][c], qm) for c in range(2)]), level, acc["scale"])
         Y[i] = acc
     return Y
 

@@ -298,3 +298,79 @@ def test_mutation_hoisted_digits_left_unpermuted_is_caught(monkeypatch):
     monkeypatch.setattr(C, "automorph_ntt_rows", planted)
     r = C.rotate_hoisted(ct, [1], keys, P)[0]
     assert np.max(np.abs(C.decrypt_decode(r, s, P) - np.roll(z, -1))) > 1e-2
+
+
+def _several(P, seed, level, n):
+    s = S.secret(seed, P.N)
+    pa, pe = S.public_key_draws(seed, P.q, P.N)
+    pk = C.public_key(s, pa, pe, P)
+    zs, cts = [], []
+    for i in range(n):
+        z = S.complex_slots(seed, P.n_slots, -1, 1, i)
+        v, e0, e1 = S.encryption_draws(seed, i, P.N)
+        zs.append(z)
+        cts.append(C.make_ct(C.encrypt(pk, C.encode(z, 2.0 ** 40, level, P), v, e0, e1, level, P), level, 2.0 ** 40))
+    return s, zs, cts
+
+
+@pytest.mark.parametrize("mk,level", [("tiny", 3), ("mid", 7), ("mid", 4)])
+def test_rotate_sum_decrypts_to_sum_of_rolled_slots(mk, level):
+    P = _tiny() if mk == "tiny" else _mid()
+    seed = S.master_seed(10)
+    steps = [3, -7, 64, 1]
+    s, zs, cts = _several(P, seed, level, len(steps))
+    keys = _rot_keys(P, seed, s, steps)
+    r = C.rotate_sum(cts, steps, keys, P)
+    want = sum(np.roll(z, -st) for z, st in zip(zs, steps))
+    assert r["level"] == level and r["scale"] == cts[0]["scale"]
+    assert np.max(np.abs(C.decrypt_decode(r, s, P) - want)) < 1e-5
+
+
+@pytest.mark.parametrize("mk,level", [("tiny", 3), ("mid", 5)])
+def test_rotate_sum_of_one_rotation_is_the_rotation(mk, level):
+    """With one term there is nothing to share: rotate_sum == rotate, residue
+    for residue."""
+    P = _tiny() if mk == "tiny" else _mid()
+    seed = S.master_seed(11)
+    s, _, cts = _several(P, seed, level, 1)
+    keys = _rot_keys(P, seed, s, [5])
+    assert np.array_equal(C.rotate_sum(cts, [5], keys, P)["c"], C.rotate(cts[0], 5, keys[5], P)["c"])
+
+
+def test_rotate_sum_differs_from_summed_rotations_by_moddown_rounding_only():
+    """ModDown(x) = (x - [x]_P)/P - v with [x]_P centred and |v| <= K/2, so
+    ModDown(sum_g u_g) - sum_g ModDown(u_g) is an integer polynomial with
+    coefficients of magnitude at most (G+1)(K+1)/2, for both polynomials."""
+    P = _mid()
+    level = 6
+    seed = S.master_seed(12)
+    steps = [1, 2, 3, -4, 9]
+    s, _, cts = _several(P, seed, level, len(steps))
+    keys = _rot_keys(P, seed, s, steps)
+    lazy = C.rotate_sum(cts, steps, keys, P)["c"]
+    qm = P.q[:level]
+    summed = None
+    for ct, st in zip(cts, steps):
+        r = C.rotate(ct, st, keys[st], P)["c"]
+        summed = r if summed is None else np.stack([C.add_rows(summed[c], r[c], qm) for c in range(2)])
+    bound = (len(steps) + 1) * (P.K + 1) / 2
+    Q = math.prod(qm)
+    worst = 0
+    for c in range(2):
+        diff = C.intt_rows(C.sub_rows(lazy[c], summed[c], qm), qm, P)
+        cen = C.centered(C.crt(diff, qm), Q)
+        worst = max(worst, max(abs(int(v)) for v in cen))
+    assert 0 < worst <= bound
+
+
+def test_mutation_rotate_sum_one_key_for_all_is_caught():
+    """Planting the first rotation's key and automorphism for every term fails
+    the slot pin."""
+    P = _tiny()
+    seed = S.master_seed(13)
+    steps = [1, 2]
+    s, zs, cts = _several(P, seed, 3, 2)
+    keys = _rot_keys(P, seed, s, steps)
+    r = C.rotate_sum(cts, [1, 1], keys, P)  # planted: step 1 for both terms
+    want = sum(np.roll(z, -st) for z, st in zip(zs, steps))
+    assert np.max(np.abs(C.decrypt_decode(r, s, P) - want)) > 1e-2

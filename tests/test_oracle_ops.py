@@ -82,12 +82,12 @@ def test_helpers():
     assert np.max(np.abs(C.decrypt_decode(d, s, P) - z)) < 1e-5
 
 
-@pytest.mark.parametrize("hoisted", [False, True])
-def test_bsgs_matvec_small(hoisted):
+@pytest.mark.parametrize("hoisted,one_moddown", [(False, False), (True, False), (True, True)])
+def test_bsgs_matvec_small(hoisted, one_moddown):
     """Feature-major packed block product y = W x by diagonals with BSGS:
     n_feat = 16 features x 64 tokens on N = 2^11, 4 baby x 4 giant steps,
     two input blocks and two output blocks; baby steps as plain or hoisted
-    rotations."""
+    rotations, giant steps summed with one ModDown per rotation or per output."""
     P = C.Params(11, 3, 1, 3)
     seed = 21
     n_feat, n_tok, bs, gs = 16, 64, 4, 4
@@ -114,7 +114,8 @@ def test_bsgs_matvec_small(hoisted):
             Wij = W[i * n_feat:(i + 1) * n_feat, j * n_feat:(j + 1) * n_feat]
             slots[(i, j)] = C.bsgs_plaintext_slots(Wij, n_feat, n_tok, bs, gs)
     pt = lambda i, j, g, b: C.encode(slots[(i, j)][g, b], 2.0 ** 40, level, P)
-    Y = C.bsgs_matvec(cts, pt, bs, gs, n_tok, keys, P, list(range(n_out)), 2.0 ** 40, hoisted=hoisted)
+    Y = C.bsgs_matvec(cts, pt, bs, gs, n_tok, keys, P, list(range(n_out)), 2.0 ** 40, hoisted=hoisted,
+                      one_moddown=one_moddown)
     want = W @ X
     for i in range(n_out):
         y = C.rescale(Y[i], P)
