@@ -177,22 +177,6 @@ __global__ void __launch_bounds__(kPmThreadsX* kPmG)
     }
 }
 
-// Y_u = Z_u[0] + sum_{g=1}^{gs-1} R_u[g] for the outputs u of one launch:
-// Z_u = zbase + u gs ctw (gs ciphertexts), R_u = rbase + u gs ctw (entry 0 unused).
-__global__ void k_sum_giant(const uint64_t* __restrict__ zbase, const uint64_t* __restrict__ rbase, MutPtrList y,
-                            int gs, int level, const DevPrime* __restrict__ pr, int logn) {
-    const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, row = blockIdx.y, u = blockIdx.z;  // row < 2 level
-    if (c >= N) return;
-    const size_t ctw = (size_t)2 * level * N, k = (size_t)row * N + c;
-    const uint64_t q = pr[row % level].q;
-    const uint64_t* z = zbase + (size_t)u * gs * ctw + k;
-    const uint64_t* r = rbase + (size_t)u * gs * ctw + k;
-    uint64_t acc = z[0];
-    for (int g = 1; g < gs; g++) acc = add_mod(acc, r[(size_t)g * ctw], q);
-    y.p[u][k] = acc;
-}
-
 }  // namespace he
 
 using namespace he;
@@ -221,16 +205,15 @@ extern "C" int he_pmult_accum_bsgs(he_ctx* c, const he_ct* x, int n_in, const ui
     const size_t ctw = (size_t)2 * level * N;
     const size_t nB = (size_t)n_groups * n_in * bs;
     // output blocks run in waves: each block needs n_groups gs ciphertexts of
-    // sums Z and as many of rotated sums; a wave holds as many blocks as fit
-    // in kBsgsWaveWords (at least one)
-    const size_t per_block = (size_t)2 * n_groups * gs * ctw;
+    // sums Z; a wave holds as many blocks as fit in kBsgsWaveWords (at least
+    // one)
+    const size_t per_block = (size_t)n_groups * gs * ctw;
     const int wave = std::max(1, std::min(n_out, (int)(kBsgsWaveWords / per_block)));
     uint64_t* buf;
     int rc = scratch_slot(c, 3, ctw * nB + per_block * wave, &buf);
     if (rc) return rc;
     uint64_t* B = buf;
-    uint64_t* Z = B + ctw * nB;                                 // [wave][n_groups][gs]
-    uint64_t* Rg = Z + (size_t)wave * n_groups * gs * ctw;      // same layout (entries g >= 1)
+    uint64_t* Z = B + ctw * nB;  // [wave][n_groups][gs]
 
     // baby steps: B[t][j][b] = rot_{stride b}(X[t][j]), the rotations b >= 1
     // hoisted (one ModUp per input X[t][j])
@@ -282,36 +265,23 @@ extern "C" int he_pmult_accum_bsgs(he_ctx* c, const he_ct* x, int n_in, const ui
                                               (double)ctw * n_groups * gs),
                      macs_per_limb * level, macs_per_limb * fp_l);
         }
-        // giant steps of the whole wave in one batch
-        std::vector<he_ct> gin, gout;
+        // Y = Z_0 + sum_{g>=1} rot_{stride bs g}(Z_g) for every output of the
+        // wave, one ModDown per output, then one rescale for the wave
+        std::vector<he_ct> zg, z0, yo;
         std::vector<int32_t> gsteps;
-        for (int u = 0; u < w * n_groups; u++)
-            for (int g = 1; g < gs; g++) {
-                gin.push_back(he_ct{Z + ((size_t)u * gs + g) * ctw, level, 1.0, 1});
-                gout.push_back(he_ct{Rg + ((size_t)u * gs + g) * ctw, level, 1.0, 1});
-                gsteps.push_back(stride * bs * g);
-            }
-        if (!gin.empty() && (rc = rotate_many(c, gin.data(), gsteps.data(), gout.data(), (int)gin.size())))
-            return rc;
-        // Y = Z_0 + sum_g rotated Z_g, then one rescale for the wave
         std::vector<const uint64_t*> rin;
         std::vector<uint64_t*> rout;
-        for (int u0 = 0; u0 < w * n_groups; u0 += kMaxBatch) {
-            const int m = std::min(kMaxBatch, w * n_groups - u0);
-            MutPtrList py;
-            for (int u = 0; u < m; u++) {
-                const int ii = (u0 + u) / n_groups, t = (u0 + u) - ii * n_groups;
-                py.p[u] = y[t * n_out + i0 + ii].data;
-                rin.push_back(py.p[u]);
-                rout.push_back(py.p[u]);
-            }
-            prof_begin(c, HE_PROF_ELEMENTWISE);
-            k_sum_giant<<<dim3((N + 255) / 256, 2 * level, m), 256, 0, c->stream>>>(
-                Z + (size_t)u0 * gs * ctw, Rg + (size_t)u0 * gs * ctw, py, gs, level, c->d_prime, c->log_n);
-            c->launches++;
-            if ((rc = check_cuda(c, cudaGetLastError(), "bsgs sum"))) return rc;
-            prof_end(c, HE_PROF_ELEMENTWISE, 8.0 * m * (double)(gs + 1) * ctw);
+        for (int g = 1; g < gs; g++) gsteps.push_back(stride * bs * g);
+        for (int u = 0; u < w * n_groups; u++) {
+            const int ii = u / n_groups, t = u - ii * n_groups;
+            z0.push_back(he_ct{Z + (size_t)u * gs * ctw, level, 1.0, 1});
+            for (int g = 1; g < gs; g++) zg.push_back(he_ct{Z + ((size_t)u * gs + g) * ctw, level, 1.0, 1});
+            yo.push_back(he_ct{y[t * n_out + i0 + ii].data, level, 1.0, 1});
+            rin.push_back(yo.back().data);
+            rout.push_back(yo.back().data);
         }
+        if ((rc = rotate_sum_many(c, zg.data(), w * n_groups, gs - 1, gsteps.data(), z0.data(), yo.data())))
+            return rc;
         if ((rc = rescale_many(c, rin, rout, level))) return rc;
     }
     for (int i = 0; i < n_groups * n_out; i++) {

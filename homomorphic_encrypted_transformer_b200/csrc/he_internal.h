@@ -147,12 +147,19 @@ struct KsIoList {
     // hoist_d[hoist_src[i]].
     std::vector<const uint64_t*> hoist_d;
     std::vector<int> hoist_src;
+    // Summed mode (sum_terms > 0): the key switches o*sum_terms ..
+    // o*sum_terms + sum_terms - 1 share output o: their inner products are
+    // added in Q_level and P and brought down by one ModDown; out, add0 and
+    // add1 then hold one entry per output.
+    int sum_terms = 0;
 };
 int key_switch(he_ctx* c, int level, const KsIoList& io);
 int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io);
 size_t key_switch_scratch_words(const he_ctx* c, int n_raised, int n, int level);
 int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, int n);
 int rotate_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t* steps, int n_steps, he_ct* out);
+int rotate_sum_many(he_ctx* c, const he_ct* z, int n_out, int n_terms, const int32_t* steps, const he_ct* base,
+                    he_ct* out);
 
 // Scratch slots: 0 = key switching internals, 1 = rescale temporaries,
 // 2 = HMult temporaries and key generation, 3 = driver buffers (polynomial

@@ -335,6 +335,88 @@ __global__ void __launch_bounds__(256, 5)  // 5 blocks per SM: more loads in fli
     *reinterpret_cast<ulonglong2*>(o + (size_t)(n_rows + t) * N) = oa;
 }
 
+// Sum of G key inner products per output, for one ModDown of the sum:
+// u[o][0/1][t][c] = sum_{g<G} sum_j x_{r,j}[t][c] * key_r,j[b/a][row(t)][c],
+// r = o G + g, x_{r,j} as in k_ks_inner for key switch r (its own sigma on
+// the digit's own rows, its raised digits elsewhere).  FP64 rows add the
+// signed products of all G switches (|sum| <= G ND 5q/8 < 2^51 for G <= 64,
+// ND <= 15); integer rows reduce each switch's 128-bit sum once and add the
+// results, kept in [0, 2q).
+template <int ND>
+__global__ void __launch_bounds__(256, 4)
+    k_ks_inner_sum(const uint64_t* __restrict__ ext, PtrList din, GalList gal, PtrList keys, int G,
+                   uint64_t* __restrict__ u, int n_rows, int level, int L, int LK, int n_ext,
+                   const DevPrime* __restrict__ pr, const FpMod* __restrict__ fpm, ModupArgs a, int logn) {
+    const int N = 1 << logn;
+    const int o = blockIdx.x, t = blockIdx.z;
+    const int c = 2 * (blockIdx.y * blockDim.x + threadIdx.x);  // positions c, c+1
+    if (c >= N) return;
+    const int krow = t < level ? t : L + (t - level);
+    const int pidx = a.tprime[t];
+    const DevPrime p = pr[pidx];
+    const bool fp = p.q < kFpPrimeLimit;
+    const FpMod m = fpm[pidx];
+    double fb0 = 0.0, fb1 = 0.0, fa0 = 0.0, fa1 = 0.0;
+    uint64_t ib0 = 0, ib1 = 0, ia0 = 0, ia1 = 0;
+    for (int g = 0; g < G; g++) {
+        const int r = o * G + g;
+        const uint64_t* key = keys.p[r];
+        const int own = automorph_src(c, logn, gal.g[r]);
+        const bool own_sw = own & 1;
+        ulonglong2 xs[ND], kbs[ND], kas[ND];
+#pragma unroll
+        for (int j = 0; j < ND; j++) {
+            const int s0 = a.src_row[j], ns = a.n_src[j];
+            if (t >= s0 && t < s0 + ns) {
+                const ulonglong2 v =
+                    __ldg(reinterpret_cast<const ulonglong2*>(din.p[r] + (size_t)t * N + (own & ~1)));
+                xs[j] = own_sw ? make_ulonglong2(v.y, v.x) : v;
+            } else {
+                const int pos = t < s0 ? t : t - ns;
+                xs[j] = __ldg(reinterpret_cast<const ulonglong2*>(
+                    ext + ((size_t)a.ext_off[j] * n_ext + (size_t)r * (n_rows - ns) + pos) * N + c));
+            }
+            kbs[j] = __ldg(reinterpret_cast<const ulonglong2*>(key + (((size_t)j * 2 + 0) * LK + krow) * N + c));
+            kas[j] = __ldg(reinterpret_cast<const ulonglong2*>(key + (((size_t)j * 2 + 1) * LK + krow) * N + c));
+        }
+        if (fp) {
+#pragma unroll
+            for (int j = 0; j < ND; j++) {
+                const double x0 = u2d(xs[j].x), x1 = u2d(xs[j].y);
+                fb0 = __dadd_rn(fb0, fp_mulmod_s(x0, __longlong_as_double((long long)kbs[j].x), m));
+                fb1 = __dadd_rn(fb1, fp_mulmod_s(x1, __longlong_as_double((long long)kbs[j].y), m));
+                fa0 = __dadd_rn(fa0, fp_mulmod_s(x0, __longlong_as_double((long long)kas[j].x), m));
+                fa1 = __dadd_rn(fa1, fp_mulmod_s(x1, __longlong_as_double((long long)kas[j].y), m));
+            }
+        } else {
+            U128 b0 = {0, 0}, b1 = {0, 0}, a0 = {0, 0}, a1 = {0, 0};
+#pragma unroll
+            for (int j = 0; j < ND; j++) {
+                mac128(b0, xs[j].x, kbs[j].x);
+                mac128(b1, xs[j].y, kbs[j].y);
+                mac128(a0, xs[j].x, kas[j].x);
+                mac128(a1, xs[j].y, kas[j].y);
+            }
+            const uint64_t q2 = 2 * p.q;
+            ib0 = csub(ib0 + redc_lazy(b0.hi, b0.lo, p.q, p.qinv_neg), q2);
+            ib1 = csub(ib1 + redc_lazy(b1.hi, b1.lo, p.q, p.qinv_neg), q2);
+            ia0 = csub(ia0 + redc_lazy(a0.hi, a0.lo, p.q, p.qinv_neg), q2);
+            ia1 = csub(ia1 + redc_lazy(a1.hi, a1.lo, p.q, p.qinv_neg), q2);
+        }
+    }
+    ulonglong2 ob, oa;
+    if (fp) {
+        ob = make_ulonglong2(d2u(fp_canon(fb0, m)), d2u(fp_canon(fb1, m)));
+        oa = make_ulonglong2(d2u(fp_canon(fa0, m)), d2u(fp_canon(fa1, m)));
+    } else {
+        ob = make_ulonglong2(csub(ib0, p.q), csub(ib1, p.q));
+        oa = make_ulonglong2(csub(ia0, p.q), csub(ia1, p.q));
+    }
+    uint64_t* out = u + ((size_t)o * 2 * n_rows) * N + c;
+    *reinterpret_cast<ulonglong2*>(out + (size_t)t * N) = ob;
+    *reinterpret_cast<ulonglong2*>(out + (size_t)(n_rows + t) * N) = oa;
+}
+
 // tmp[i][poly][r][c] = sum_k y'_k (P/p_k mod q_r), y_k = [x_k (P/p_k)^-1]_{p_k},
 // y'_k = y_k or y_k - p_k (centred, |y'_k| < 2^59).  Two arithmetic paths:
 //  - FP64 (targets below 2^41): with y'_k = a_k 2^40 + b_k 2^20 + c_k
@@ -576,14 +658,19 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     const int nm = hoist ? (int)io.hoist_d.size() : n;
     if (nm > kMaxBatch || (hoist && (int)io.hoist_src.size() != n))
         return set_err(c, HE_EINVAL, "key switch: bad hoisting lists");
+    // summed: n_md = n / G outputs, each the sum of G key switches
+    const int G = io.sum_terms;
+    const bool summed = G > 0;
+    if (summed && (hoist || n % G)) return set_err(c, HE_EINVAL, "key switch: bad summed lists");
+    const int n_md = summed ? n / G : n;
     uint64_t* base;
-    int rc = scratch_slot(c, 0, key_switch_scratch_words(c, nm, n, level), &base);
+    int rc = scratch_slot(c, 0, key_switch_scratch_words(c, nm, n_md, level), &base);
     if (rc) return rc;
     const int ext_rows = nd * n_rows - level;  // sum over digits of the target rows
     uint64_t* coef = base;
     uint64_t* ext = coef + (size_t)nm * level * N;
     uint64_t* u = ext + (size_t)nm * ext_rows * N;
-    uint64_t* tmp = u + (size_t)n * 2 * n_rows * N;
+    uint64_t* tmp = u + (size_t)n_md * 2 * n_rows * N;
 
     PtrList din, keys, mdin;
     GalList gal, mgal;
@@ -594,9 +681,9 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
         gal.g[i] = i < n ? io.galois[i] : 0;
         keys.p[i] = i < n ? io.key[i] : nullptr;
         din.p[i] = i < n ? io.d[i] : nullptr;
-        mo.out.p[i] = i < n ? io.out[i] : nullptr;
-        mo.add0.p[i] = i < n ? io.add0[i] : nullptr;
-        mo.add1.p[i] = i < n ? io.add1[i] : nullptr;
+        mo.out.p[i] = i < n_md ? io.out[i] : nullptr;
+        mo.add0.p[i] = i < n_md ? io.add0[i] : nullptr;
+        mo.add1.p[i] = i < n_md ? io.add1[i] : nullptr;
         mdin.p[i] = hoist ? (i < nm ? io.hoist_d[i] : nullptr) : din.p[i];
         mgal.g[i] = hoist ? 0 : gal.g[i];
         xsrc.i[i] = hoist && i < n ? io.hoist_src[i] : i;
@@ -703,7 +790,10 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     switch (nd) {
 #define HE_KS_CASE(D)                                                                                             \
     case D:                                                                                                       \
-        if (hoist)                                                                                                \
+        if (summed)                                                                                               \
+            k_ks_inner_sum<D><<<dim3(n_md, gx2, n_rows), blk, 0, c->stream>>>(                                    \
+                ext, din, gal, keys, G, u, n_rows, level, L, LK, nm, c->d_prime, c->d_fpmod, ma, c->log_n);       \
+        else if (hoist)                                                                                           \
             k_ks_inner<D, true><<<dim3(n, gx2, n_rows), blk, 0, c->stream>>>(                                     \
                 ext, din, gal, keys, xsrc, u, n_rows, level, L, LK, nm, c->d_prime, c->d_fpmod, ma, c->log_n);    \
         else                                                                                                      \
@@ -727,19 +817,19 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
         std::sort(kd.begin(), kd.end());
         const double n_keys = (double)(std::unique(kd.begin(), kd.end()) - kd.begin());
         prof_end(c, HE_PROF_KS_INNER,
-                 ((double)nm * nd * n_rows + n_keys * 2.0 * nd * n_rows + 2.0 * n * n_rows) * limbB,
+                 ((double)nm * nd * n_rows + n_keys * 2.0 * nd * n_rows + 2.0 * n_md * n_rows) * limbB,
                  (double)n * n_rows * N * 2.0 * nd, (double)n * fp_rows_ks * N * 2.0 * nd);
     }
 
     std::vector<int> pp = prime_range(L, K);
     RowSet prs = rowset(u + (size_t)level * N, (long long)n_rows * N, K, pp.data());
-    if ((rc = ntt_inv_set(c, prs, n * 2 * K))) return rc;
+    if ((rc = ntt_inv_set(c, prs, n_md * 2 * K))) return rc;
 
     prof_begin(c, HE_PROF_MODDOWN_CONV);
     switch (K) {
 #define HE_MD_CASE(KK)                                                                                          \
     case KK:                                                                                                    \
-        k_moddown_conv<KK><<<dim3(gx, 2, n), blk, 0, c->stream>>>(u, tmp, level, L, c->d_prime, c->d_fpmod,    \
+        k_moddown_conv<KK><<<dim3(gx, 2, n_md), blk, 0, c->stream>>>(u, tmp, level, L, c->d_prime, c->d_fpmod, \
                                                                   c->d_md_pcoef, c->d_md_mat, c->d_md_negP,    \
                                                                   c->log_n);                                   \
         break;
@@ -754,23 +844,24 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     {
         int fp_t = 0;
         for (int r = 0; r < level; r++) fp_t += fp_prime(c, r);
-        prof_end(c, HE_PROF_MODDOWN_CONV, 2.0 * n * (K + level) * limbB,
-                 2.0 * n * N * (K + (double)K * (level - fp_t) + 2.0 * K * fp_t), 2.0 * n * N * 2.0 * K * fp_t);
+        prof_end(c, HE_PROF_MODDOWN_CONV, 2.0 * n_md * (K + level) * limbB,
+                 2.0 * n_md * N * (K + (double)K * (level - fp_t) + 2.0 * K * fp_t),
+                 2.0 * n_md * N * 2.0 * K * fp_t);
     }
 
     // back to the evaluation domain: column pass, then the row pass fused
     // with (u - tmp) P^-1 + add
-    if ((rc = ntt_fwd_cols_set(c, rowset_contig(tmp, level, N, qp), n * 2 * level))) return rc;
+    if ((rc = ntt_fwd_cols_set(c, rowset_contig(tmp, level, N, qp), n_md * 2 * level))) return rc;
     prof_begin(c, HE_PROF_MODDOWN_COMBINE);
-#define HE_FRM(LN) launch_fwd_rows_moddown<LN>(c, tmp, u, mo, n, level)
+#define HE_FRM(LN) launch_fwd_rows_moddown<LN>(c, tmp, u, mo, n_md, level)
     HE_LOGN_SWITCH(c, HE_FRM)
 #undef HE_FRM
     if ((rc = lc(c, "fwd_rows_moddown"))) return rc;
     {
         int n_add = 0;
-        for (int i = 0; i < n; i++) n_add += (io.add0[i] != nullptr) + (io.add1[i] != nullptr);
-        prof_end(c, HE_PROF_MODDOWN_COMBINE, (6.0 * n + n_add) * level * limbB,
-                 2.0 * n * level * N * (1.0 + 0.5 * sh.s2), 2.0 * n * fp_q * N * 0.5 * sh.s2);
+        for (int i = 0; i < n_md; i++) n_add += (io.add0[i] != nullptr) + (io.add1[i] != nullptr);
+        prof_end(c, HE_PROF_MODDOWN_COMBINE, (6.0 * n_md + n_add) * level * limbB,
+                 2.0 * n_md * level * N * (1.0 + 0.5 * sh.s2), 2.0 * n_md * fp_q * N * 0.5 * sh.s2);
     }
     return HE_OK;
 }
@@ -934,9 +1025,143 @@ int rotate_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t* ste
     return HE_OK;
 }
 
+// First part of a sum of rotations: s_o = base_o + sum_g (sigma_g(z0_{o,g}), 0)
+// over the key-switched terms (gal != 0) + z_{o,g} over the identity terms
+// (gal == 0, both polynomials); the key switches' ModDown adds the rest.
+// Term r = o G + g.  Grid (ceil(N/256), 2 level, outputs).
+__global__ void k_rot_presum(PtrList z, GalList gal, PtrList base, MutPtrList s, int G, int level,
+                             const DevPrime* __restrict__ pr, int logn) {
+    const int N = 1 << logn;
+    const int c = blockIdx.x * blockDim.x + threadIdx.x, row = blockIdx.y, o = blockIdx.z;
+    if (c >= N) return;
+    const int poly = row / level, t = row - poly * level;
+    const uint64_t q = pr[t].q;
+    const size_t k = (size_t)row * N;  // this limb within a ciphertext
+    uint64_t acc = base.p[o] ? base.p[o][k + c] : 0;
+    for (int g = 0; g < G; g++) {
+        const int r = o * G + g;
+        const uint64_t gl = gal.g[r];
+        if (gl == 0)
+            acc = add_mod(acc, z.p[r][k + c], q);
+        else if (poly == 0)
+            acc = add_mod(acc, z.p[r][k + automorph_src(c, logn, gl)], q);
+    }
+    s.p[o][k + c] = acc;
+}
+
+// Sums of rotations with one ModDown per output (the ModDown hoisting of
+// Bossuat, Mouchet, Troncoso-Pastoriza, Hubaux, EUROCRYPT 2021, section 4):
+//   out[o] = base[o] + sum_g rot_{steps[g]}(z[o n_terms + g])
+//          = (base0 + sum_g sigma_g(z0_g) + ModDown(sum_g u0_g),  base1 + ModDown(sum_g u1_g)),
+//   u_g = sum_j ModUp_j(sigma_g(z1_g)) (.) evk_{g,j}.
+// base may be null.  Terms whose Galois element is 1 are added as they are.
+// Outputs go in chunks of floor(64 / n_terms): one pre-sum launch, then one
+// key-switching pass of the chunk's terms in summed mode.
+int rotate_sum_many(he_ctx* c, const he_ct* z, int n_out, int n_terms, const int32_t* steps, const he_ct* base,
+                    he_ct* out) {
+    if (n_out < 0 || n_terms < 0) return set_err(c, HE_EINVAL, "rotate_sum: negative count");
+    if (n_out == 0) return HE_OK;
+    if (n_terms > kMaxBatch) return set_err(c, HE_EINVAL, "rotate_sum: at most %d terms", kMaxBatch);
+    if (!out || (n_terms && (!z || !steps)) || (!n_terms && !base))
+        return set_err(c, HE_EINVAL, "rotate_sum: null argument");
+    const int level = n_terms ? z[0].level : base[0].level;
+    const double scale = n_terms ? z[0].scale : base[0].scale;
+    std::set<const uint64_t*> ins;
+    for (long long i = 0; i < (long long)n_out * n_terms; i++) {
+        int rc = ct_ok(c, &z[i], "rotate_sum");
+        if (rc) return rc;
+        if (z[i].level != level || z[i].scale != scale) return set_err(c, HE_ELEVEL, "rotate_sum: mixed levels or scales");
+        ins.insert(z[i].data);
+    }
+    for (int o = 0; base && o < n_out; o++) {
+        int rc = ct_ok(c, &base[o], "rotate_sum");
+        if (rc) return rc;
+        if (base[o].level != level || base[o].scale != scale)
+            return set_err(c, HE_ELEVEL, "rotate_sum: base level or scale differs");
+        ins.insert(base[o].data);
+    }
+    for (int o = 0; o < n_out; o++) {
+        if (!out[o].data || ((uintptr_t)out[o].data & 15))
+            return set_err(c, HE_EINVAL, "rotate_sum: null or unaligned output %d", o);
+        if (ins.count(out[o].data)) return set_err(c, HE_EINVAL, "rotate_sum: output %d aliases an input", o);
+    }
+    std::vector<uint64_t> gal(n_terms);
+    int g_eff = 0;
+    for (int g = 0; g < n_terms; g++) {
+        gal[g] = galois_elt(c, steps[g]);
+        if (gal[g] == 1) continue;
+        if (!c->rot_keys.count(gal[g]))
+            return set_err(c, HE_ENOKEY, "rotate_sum: no key for step %d (galois %llu)", steps[g],
+                           (unsigned long long)gal[g]);
+        g_eff++;
+    }
+    const size_t N = c->N, ctw = (size_t)2 * level * N;
+    const int G = n_terms, mc = std::max(1, kMaxBatch / std::max(1, G));
+    uint64_t* S = nullptr;
+    if (g_eff) {
+        int rc = scratch_slot(c, 2, ctw * std::min(mc, n_out), &S);
+        if (rc) return rc;
+    }
+    for (int o0 = 0; o0 < n_out; o0 += mc) {
+        const int m = std::min(mc, n_out - o0);
+        PtrList zp, bp;
+        GalList gl;
+        MutPtrList sp;
+        for (int i = 0; i < kMaxBatch; i++) {
+            zp.p[i] = nullptr;
+            gl.g[i] = 0;
+            bp.p[i] = nullptr;
+            sp.p[i] = nullptr;
+        }
+        for (int o = 0; o < m; o++) {
+            for (int g = 0; g < G; g++) {
+                zp.p[o * G + g] = z[(size_t)(o0 + o) * G + g].data;
+                gl.g[o * G + g] = gal[g] == 1 ? 0 : gal[g];
+            }
+            bp.p[o] = base ? base[o0 + o].data : nullptr;
+            sp.p[o] = g_eff ? S + (size_t)o * ctw : out[o0 + o].data;
+        }
+        prof_begin(c, HE_PROF_ELEMENTWISE);
+        k_rot_presum<<<dim3((unsigned)((N + 255) / 256), 2 * level, m), 256, 0, c->stream>>>(
+            zp, gl, bp, sp, G, level, c->d_prime, c->log_n);
+        int rc = lc(c, "rot_presum");
+        if (rc) return rc;
+        prof_end(c, HE_PROF_ELEMENTWISE,
+                 8.0 * m * ((double)(base ? 2 : 1) * ctw + (double)(G - g_eff) * ctw + (double)g_eff * ctw / 2));
+        if (!g_eff) continue;
+        KsIoList io;
+        io.sig_add0 = false;
+        io.sum_terms = g_eff;
+        for (int o = 0; o < m; o++) {
+            for (int g = 0; g < G; g++) {
+                if (gal[g] == 1) continue;
+                io.galois.push_back(gal[g]);
+                io.key.push_back(c->rot_keys[gal[g]].d);
+                io.d.push_back(z[(size_t)(o0 + o) * G + g].data + (size_t)level * N);
+            }
+            io.out.push_back(out[o0 + o].data);
+            io.add0.push_back(S + (size_t)o * ctw);
+            io.add1.push_back(S + (size_t)o * ctw + (size_t)level * N);
+        }
+        if ((rc = key_switch_chunk(c, m * g_eff, level, io))) return rc;
+    }
+    for (int o = 0; o < n_out; o++) {
+        out[o].level = level;
+        out[o].scale = scale;
+        out[o].is_ntt = 1;
+    }
+    return HE_OK;
+}
+
 }  // namespace he
 
 using namespace he;
+
+extern "C" int he_rotate_sum(he_ctx* c, const he_ct* z, int n_out, int n_terms, const int32_t* steps,
+                             const he_ct* base, he_ct* out) {
+    if (!c) return HE_EINVAL;
+    return rotate_sum_many(c, z, n_out, n_terms, steps, base, out);
+}
 
 extern "C" int he_rotate_hoisted(he_ctx* c, const he_ct* in, int n_in, const int32_t* steps, int n_steps,
                                  he_ct* out) {

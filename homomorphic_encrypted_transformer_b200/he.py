@@ -82,6 +82,7 @@ _sig("he_ntt_inv", _i, _vp, _vp, _i, _i, _i)
 _sig("he_rotate", _i, _vp, ctypes.POINTER(he_ct), ctypes.c_int32, ctypes.POINTER(he_ct))
 _sig("he_rotate_batch", _i, _vp, ctypes.POINTER(he_ct), _vp, ctypes.POINTER(he_ct), _i)
 _sig("he_rotate_hoisted", _i, _vp, ctypes.POINTER(he_ct), _i, _vp, _i, ctypes.POINTER(he_ct))
+_sig("he_rotate_sum", _i, _vp, ctypes.POINTER(he_ct), _i, _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct))
 _sig("he_rotate_batch_host", _i, _vp, _vp, _i, _vp, _vp, _i)
 _sig("he_hmult_relin_rescale", _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct), ctypes.POINTER(he_ct))
 _sig("he_rescale", _i, _vp, ctypes.POINTER(he_ct))
@@ -277,6 +278,21 @@ def he_rotate_hoisted(ctx, cts_in, steps, cts_out):
     ao = (he_ct * max(1, len(cts_out)))(*[c._c() for c in cts_out])
     st = np.ascontiguousarray(steps, dtype=np.int32)
     _check(ctx, _lib.he_rotate_hoisted(ctx.ptr, ai, n_in, _ptr(st), n_steps, ao))
+    for c, o in zip(cts_out, ao):
+        c._update(o)
+
+
+def he_rotate_sum(ctx, z, steps, base, cts_out):
+    """cts_out[o] = base[o] + sum_g rot_{steps[g]}(z[o * len(steps) + g]), one
+    ModDown per output; base may be None."""
+    n_out, n_terms = len(cts_out), len(steps)
+    if len(z) != n_out * n_terms or (base is not None and len(base) != n_out):
+        raise ValueError("he_rotate_sum: need len(cts_out) * len(steps) terms and one base per output")
+    az = (he_ct * max(1, len(z)))(*[c._c() for c in z])
+    ab = (he_ct * n_out)(*[c._c() for c in base]) if base is not None else None
+    ao = (he_ct * max(1, n_out))(*[c._c() for c in cts_out])
+    st = np.ascontiguousarray(steps, dtype=np.int32)
+    _check(ctx, _lib.he_rotate_sum(ctx.ptr, az, n_out, n_terms, _ptr(st), ab, ao))
     for c, o in zip(cts_out, ao):
         c._update(o)
 

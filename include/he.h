@@ -182,6 +182,28 @@ int he_rotate_batch_host(he_ctx* ctx, const uint64_t* h_in, int level, const int
  * HE_ENOKEY (a step without a rotation key); nothing is launched then.
  */
 int he_rotate_hoisted(he_ctx* ctx, const he_ct* in, int n_in, const int32_t* steps, int n_steps, he_ct* out);
+/*
+ * Sums of rotations with one ModDown per sum (the ModDown hoisting of
+ * Bossuat, Mouchet, Troncoso-Pastoriza, Hubaux, "Efficient Bootstrapping for
+ * Approximate Homomorphic Encryption with Non-Sparse Keys", EUROCRYPT 2021,
+ * section 4).  For o < n_out, with z_g = z[o*n_terms + g] = (z0_g, z1_g) and
+ * k_g = 5^(steps[g] mod N/2) mod 2N:
+ *   out[o] = base[o] + sum_g rot_{steps[g]}(z_g)
+ *          = (b0 + sum_g sigma_g(z0_g) + ModDown(sum_g u0_g),  b1 + ModDown(sum_g u1_g)),
+ *   u_g = sum_j ModUp_j(sigma_g(z1_g)) (.) evk_{g,j}   (kept over Q_level and P).
+ * ModDown rounds once per sum, so the residues differ from adding he_rotate
+ * results (by at most (n_terms+1)(K+1)/2 per coefficient) while the slots
+ * agree.  Terms whose Galois element is 1 are added unchanged.
+ * z: n_out*n_terms device ciphertexts (output-major), base: n_out ciphertexts
+ * or NULL (then n_terms >= 1), all at one level and scale, 16-byte aligned;
+ * n_terms <= 64.  out: n_out device ciphertexts with room for that level,
+ * none overlapping an input; each gets the level and scale.  Errors:
+ * HE_EINVAL (null, unaligned, aliasing, counts), HE_ELEVEL (mixed levels or
+ * scales), HE_EDOMAIN, HE_ENOKEY (a step without a rotation key); nothing is
+ * launched then.
+ */
+int he_rotate_sum(he_ctx* ctx, const he_ct* z, int n_out, int n_terms, const int32_t* steps, const he_ct* base,
+                  he_ct* out);
 
 /* Tensor, relinearise (key switch of d2 with the s^2 key), rescale.
  * a and b at the same level l >= 2; out at level l-1, scale (sa*sb)/q_{l-1}.
@@ -229,8 +251,8 @@ int he_drop_level(he_ctx* ctx, const he_ct* in, int level, he_ct* out);
  * y: n_groups*n_out ciphertexts (group-major) with room for level l; they
  *    come back at level l-1, scale x.scale*pt_scale/q_{l-1}.
  * The baby-step rotations rot_{stride*b}(X[t][j]) are the hoisted rotations of
- * he_rotate_hoisted (one ModUp per input); the giant-step rotations are
- * he_rotate_batch's.
+ * he_rotate_hoisted (one ModUp per input); the giant-step sum of each output
+ * is he_rotate_sum's (one ModDown per output).
  * Needs rotation keys for stride*b (0<b<bs) and stride*bs*g (0<g<gs).
  */
 int he_pmult_accum_bsgs(he_ctx* ctx, const he_ct* x, int n_in, const uint64_t* d_pt, double pt_scale,

@@ -109,3 +109,22 @@ def test_hoisted_rotation_errors():
     he.he_sync(st.ctx)
     want = C.rotate_hoisted(st.encrypt(z, 3), [1], {1: st.oracle_rot_key(1)}, st.P)[0]
     assert np.array_equal(st.from_gpu(y[0]), want["c"])
+
+
+def test_rotation_sum_errors():
+    he = lib()
+    st = Setup(12, 3, 1, 3, seed=66)
+    st.upload_rot(1)
+    z = S.complex_slots(st.seed, st.P.n_slots, -1, 1)
+    x3 = st.to_gpu(st.encrypt(z, 3))
+    x3b = st.to_gpu(st.encrypt(z, 3, scale=2.0 ** 30))
+    y = [st.empty_gpu(3)]
+    assert _code(he.he_rotate_sum, st.ctx, [x3, x3], [1, 4], None, y) == he.HE_ENOKEY
+    assert _code(he.he_rotate_sum, st.ctx, [x3, x3b], [1, 1], None, y) == he.HE_ELEVEL  # scales differ
+    assert _code(he.he_rotate_sum, st.ctx, [x3], [1], None, [x3]) == he.HE_EINVAL  # output aliases a term
+    assert _code(he.he_rotate_sum, st.ctx, [x3] * 65, [1] * 65, None, y) == he.HE_EINVAL  # more than 64 terms
+    assert _code(he.he_rotate_sum, st.ctx, [], [], None, y) == he.HE_EINVAL  # no terms and no base
+    he.he_rotate_sum(st.ctx, [x3], [1], None, y)  # and still works
+    he.he_sync(st.ctx)
+    want = C.rotate_sum([st.encrypt(z, 3)], [1], {1: st.oracle_rot_key(1)}, st.P)
+    assert np.array_equal(st.from_gpu(y[0]), want["c"])

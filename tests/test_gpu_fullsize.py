@@ -93,7 +93,8 @@ def _ffn_case(n_groups, check_groups, workload_index):
     he.he_sync(st.ctx)
     keys = {s_: st.oracle_rot_key(s_) for s_ in steps}
     for t in check_groups:
-        Y = C.bsgs_matvec(cts[t * N_IN:(t + 1) * N_IN], pt, BS, GS, N_TOK, keys, P, [0], 2.0 ** 40, hoisted=True)
+        Y = C.bsgs_matvec(cts[t * N_IN:(t + 1) * N_IN], pt, BS, GS, N_TOK, keys, P, [0], 2.0 ** 40, hoisted=True,
+                          one_moddown=True)
         want = C.rescale(Y[0], P)
         got = ys[t]
         assert got.level == LEVEL - 1 and got.scale == want["scale"]

@@ -157,7 +157,7 @@ def test_bsgs_small():
     pt = lambda i, j, g, b: pts[i, j, g, b]
     for t in range(n_grp):
         Y = C.bsgs_matvec(cts[t * n_in:(t + 1) * n_in], pt, bs, gs, n_tok, keys, P, list(range(n_out)), 2.0 ** 40,
-                          hoisted=True)
+                          hoisted=True, one_moddown=True)
         want_plain = W @ X[t]
         for i in range(n_out):
             want = C.rescale(Y[i], P)

@@ -234,3 +234,65 @@ def test_rotation_hoisted_chunks():
     st = Setup(11, 3, 1, 3, seed=46)
     _hoisted_case(st, 3, 5, list(range(1, 21)))
     _hoisted_case(st, 2, 1, list(range(-35, 0)) + list(range(1, 36)))
+
+
+def _sum_case(st, level, n_out, steps, with_base=True):
+    """he_rotate_sum against the oracle: base + identity terms + rotate_sum of
+    the key-switched terms, residue for residue."""
+    he = lib()
+    P = st.P
+    G = len(steps)
+    eff = [s for s in steps if P.galois_elt(s) != 1]
+    for s in sorted(set(eff)):
+        st.upload_rot(s)
+    keys = {s: st.oracle_rot_key(s) for s in eff}
+    slots = lambda i: S.complex_slots(st.seed, P.n_slots, -1, 1, i)
+    zs = [st.encrypt(slots(100 + i), level, ct_id=100 + i) for i in range(n_out * G)]
+    bs = [st.encrypt(slots(300 + o), level, ct_id=300 + o) for o in range(n_out)] if with_base else None
+    ys = [st.empty_gpu(level) for _ in range(n_out)]
+    he.he_rotate_sum(st.ctx, [st.to_gpu(z) for z in zs], steps, [st.to_gpu(b) for b in bs] if with_base else None,
+                     ys)
+    he.he_sync(st.ctx)
+    qm = P.q[:level]
+    for o in range(n_out):
+        terms = zs[o * G:(o + 1) * G]
+        ks = [(z, s) for z, s in zip(terms, steps) if P.galois_elt(s) != 1]
+        parts = [z for z, s in zip(terms, steps) if P.galois_elt(s) == 1]
+        if ks:
+            parts.append(C.rotate_sum([z for z, _ in ks], [s for _, s in ks], keys, P))
+        if with_base:
+            parts.append(bs[o])
+        want = parts[0]["c"]
+        for p_ in parts[1:]:
+            want = np.stack([C.add_rows(want[c], p_["c"][c], qm) for c in range(2)])
+        assert ys[o].level == level and ys[o].scale == zs[0]["scale"]
+        assert np.array_equal(st.from_gpu(ys[o]), want), o
+    return zs, bs, ys
+
+
+def test_rotation_sum_tiny():
+    """Two sums of 3 rotations plus a base; the sums decrypt to the base plus
+    the rolled slots.  Then an identity term (step 0) without a base."""
+    st = Setup(12, 3, 1, 3, seed=S.master_seed(0))
+    steps = [1, 2, -1]
+    zs, bs, ys = _sum_case(st, 3, 2, steps)
+    for o in range(2):
+        want = S.complex_slots(st.seed, st.P.n_slots, -1, 1, 300 + o)
+        for g, s in enumerate(steps):
+            want = want + np.roll(S.complex_slots(st.seed, st.P.n_slots, -1, 1, 100 + o * 3 + g), -s)
+        got = C.make_ct(st.from_gpu(ys[o]), 3, 2.0 ** 40)
+        assert np.max(np.abs(C.decrypt_decode(got, st.s, st.P) - want)) < 1e-5
+    _sum_case(st, 3, 2, [3, 0], with_base=False)
+
+
+@pytest.mark.parametrize("level", [7, 4, 1])
+def test_rotation_sum_mid_levels(level):
+    st = Setup(11, 7, 3, 3, seed=47)
+    _sum_case(st, level, 2, [5, -3, 17, 2])
+
+
+def test_rotation_sum_chunks():
+    """5 sums of 20 rotations: chunks of 3 and 2 outputs (60 and 40 key
+    switches in summed mode)."""
+    st = Setup(11, 3, 1, 3, seed=48)
+    _sum_case(st, 3, 5, list(range(1, 21)))
