@@ -641,6 +641,40 @@ def rotate_sum(zs, steps, keys, params):
                    level, zs[0]["scale"])
 
 
+def rotate_sum_hoisted(ct, steps, keys, params):
+    """sum_s rot_{steps[s]}(ct) of one ciphertext with one ModUp and one
+    ModDown: the raised digits of c1 are shared by every step (as in
+    rotate_hoisted) and the inner products are added over Q_level and P
+    before a single ModDown (as in rotate_sum):
+
+        result = (sum_s sigma_s(c0) + ModDown(sum_s sum_j sigma_s(ModUp_j(c1)) (.) evk_{s,j}.b),
+                                      ModDown(sum_s sum_j sigma_s(ModUp_j(c1)) (.) evk_{s,j}.a)).
+
+    With one step it is rotate_hoisted's; against the sum of rotate_hoisted
+    results it differs by the rounding of one ModDown instead of several.
+    keys: step -> switching key."""
+    level = ct["level"]
+    qm = params.q[:level]
+    ext_mods = qm + params.p
+    key_rows = list(range(level)) + list(range(params.L, params.L + params.K))
+    c1 = ct["c"][1]
+    c1_coeff = intt_rows(c1, qm, params)
+    raised = [modup(c1_coeff, c1, D, level, params) for D in params.digits(level)]
+    u0 = np.zeros((level + params.K, params.N), dtype=np.uint64)
+    u1 = np.zeros_like(u0)
+    c0 = np.zeros((level, params.N), dtype=np.uint64)
+    for step in steps:
+        k = params.galois_elt(step)
+        b, a = keys[step]
+        c0 = add_rows(c0, automorph_ntt_rows(ct["c"][0], k, qm, params), qm)
+        for j, ext in enumerate(raised):
+            ext_k = automorph_ntt_rows(ext, k, ext_mods, params)
+            u0 = add_rows(u0, mul_rows(ext_k, b[j][key_rows], ext_mods), ext_mods)
+            u1 = add_rows(u1, mul_rows(ext_k, a[j][key_rows], ext_mods), ext_mods)
+    return make_ct(np.stack([add_rows(c0, moddown(u0, level, params), qm), moddown(u1, level, params)]),
+                   level, ct["scale"])
+
+
 # --------------------------------------------------------------------------
 # Multiplication, rescale, helpers
 # --------------------------------------------------------------------------

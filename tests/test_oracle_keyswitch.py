@@ -374,3 +374,61 @@ def test_mutation_rotate_sum_one_key_for_all_is_caught():
     r = C.rotate_sum(cts, [1, 1], keys, P)  # planted: step 1 for both terms
     want = sum(np.roll(z, -st) for z, st in zip(zs, steps))
     assert np.max(np.abs(C.decrypt_decode(r, s, P) - want)) > 1e-2
+
+
+@pytest.mark.parametrize("mk,level", [("tiny", 3), ("mid", 7), ("mid", 4)])
+def test_rotate_sum_hoisted_decrypts_to_sum_of_rolled_slots(mk, level):
+    P = _tiny() if mk == "tiny" else _mid()
+    seed = S.master_seed(14)
+    s, z, ct = _encrypted(P, seed, level)
+    steps = [1, 2, 4, -8, 64]
+    keys = _rot_keys(P, seed, s, steps)
+    r = C.rotate_sum_hoisted(ct, steps, keys, P)
+    want = sum(np.roll(z, -st) for st in steps)
+    assert r["level"] == level and r["scale"] == ct["scale"]
+    assert np.max(np.abs(C.decrypt_decode(r, s, P) - want)) < 1e-5
+
+
+@pytest.mark.parametrize("mk,level", [("tiny", 3), ("mid", 5)])
+def test_rotate_sum_hoisted_of_one_step_is_the_hoisted_rotation(mk, level):
+    P = _tiny() if mk == "tiny" else _mid()
+    seed = S.master_seed(15)
+    s, _, ct = _encrypted(P, seed, level)
+    keys = _rot_keys(P, seed, s, [3])
+    want = C.rotate_hoisted(ct, [3], keys, P)[0]["c"]
+    assert np.array_equal(C.rotate_sum_hoisted(ct, [3], keys, P)["c"], want)
+
+
+def test_rotate_sum_hoisted_differs_from_summed_hoisted_rotations_by_moddown_rounding_only():
+    """Against the sum of rotate_hoisted results (one ModDown each): an
+    integer polynomial of magnitude at most (G+1)(K+1)/2 per coefficient, in
+    both polynomials."""
+    P = _mid()
+    level = 6
+    seed = S.master_seed(16)
+    s, _, ct = _encrypted(P, seed, level)
+    steps = [1, 2, 3, -4, 9]
+    keys = _rot_keys(P, seed, s, steps)
+    lazy = C.rotate_sum_hoisted(ct, steps, keys, P)["c"]
+    qm = P.q[:level]
+    summed = None
+    for r in C.rotate_hoisted(ct, steps, keys, P):
+        summed = r["c"] if summed is None else np.stack([C.add_rows(summed[c], r["c"][c], qm) for c in range(2)])
+    Q = math.prod(qm)
+    worst = 0
+    for c in range(2):
+        cen = C.centered(C.crt(C.intt_rows(C.sub_rows(lazy[c], summed[c], qm), qm, P), qm), Q)
+        worst = max(worst, max(abs(int(v)) for v in cen))
+    assert 0 < worst <= (len(steps) + 1) * (P.K + 1) / 2
+
+
+def test_mutation_rotate_sum_hoisted_dropped_step_is_caught():
+    """Planting a sum that skips its last step fails the slot pin."""
+    P = _tiny()
+    seed = S.master_seed(17)
+    s, z, ct = _encrypted(P, seed, 3)
+    steps = [1, 2, 4]
+    keys = _rot_keys(P, seed, s, steps)
+    r = C.rotate_sum_hoisted(ct, steps[:-1], keys, P)  # planted: last step dropped
+    want = sum(np.roll(z, -st) for st in steps)
+    assert np.max(np.abs(C.decrypt_decode(r, s, P) - want)) > 1e-2
