@@ -47,7 +47,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--case", default="rotation",
-                    choices=["rotation", "ntt", "rot_small", "ffn128", "ffn2048", "ps15", "tiny", "hoisted"],
+                    choices=["rotation", "ntt", "rot_small", "ffn128", "ffn2048", "ps15", "tiny", "hoisted",
+                             "rotsum"],
                     help="rotation: the headline workload (default). ffn128 / ffn2048 / ps15 / tiny: the other "
                          "workloads, one JSON line each. ntt / rot_small: kernel cases for profiler captures "
                          "(NTT of 512 limbs, or 8 rotations with 2 keys)")
@@ -278,7 +279,7 @@ def workload_cpu_baseline(case, seconds):
     timing)."""
     from oracle import ckks as C
 
-    widx = {"tiny": 0, "hoisted": 1, "ffn128": 2, "ffn2048": 3, "ps15": 4}[case]
+    widx = {"tiny": 0, "hoisted": 1, "rotsum": 1, "ffn128": 2, "ffn2048": 3, "ps15": 4}[case]
     master = S.master_seed(widx)
     t_end = time.perf_counter() + seconds
     if case == "tiny":
@@ -304,7 +305,7 @@ def workload_cpu_baseline(case, seconds):
                 "sample": "%d whole sequences (NTT round trip, 3 rotations, 1 HMult-relin-rescale), N=2^12" % done}
     P = C.Params(LOG_N, L, K, DNUM)
     s = S.secret(master, P.N)
-    if case == "hoisted":
+    if case in ("hoisted", "rotsum"):
         steps = workload_inputs(master, P.q, N_CTS)[0][:2]
         keys = {}
         for st in steps:
@@ -314,12 +315,16 @@ def workload_cpu_baseline(case, seconds):
         done, t = 0, 0.0
         while done < 2 or time.perf_counter() < t_end:
             t0 = time.perf_counter()
-            C.rotate_hoisted(ct, steps, keys, P)
+            if case == "hoisted":
+                C.rotate_hoisted(ct, steps, keys, P)
+            else:
+                C.rotate_sum_hoisted(ct, steps, keys, P)
             t += time.perf_counter() - t0
             done += len(steps)
+        what = "hoisted rotations" if case == "hoisted" else "rotations summed with one ModUp and one ModDown"
         return {"value": done / t, "unit": "rotations/s", "cores": C.n_threads(), "kind": "oracle",
-                "sample": "%d full-size hoisted rotations (level 24), one ciphertext by 2 steps per call, so one "
-                          "ModUp per 2 rotations; key generation excluded" % done}
+                "sample": "%d full-size %s (level 24), one ciphertext by 2 steps per call; key generation "
+                          "excluded" % (done, what)}
     if case == "ps15":
         a, e = S.key_draws(master, 2, P.mods, P.N, P.dnum)
         rlk = C.relin_key(s, a, e, P)
@@ -369,7 +374,9 @@ def run_workload_case(args, local_rank):
     ps15 (degree-15 Paterson-Stockmeyer on 64 ciphertexts from level 24),
     tiny (N=2^12 NTT round trip, 3 rotations and one HMult-relin-rescale),
     hoisted (4 ciphertexts at level 24 each rotated by the rotation batch's
-    16 steps through one ModUp per ciphertext: 64 hoisted rotations).
+    16 steps through one ModUp per ciphertext: 64 hoisted rotations),
+    rotsum (the same 4 ciphertexts each summed over its 16 rotations with
+    one ModUp and one ModDown: 64 rotations into 4 sums).
     Inputs are seeded uniform residues on the device; the rotation and
     relinearisation keys are computed by the library from seeded draws."""
     import torch
@@ -380,7 +387,7 @@ def run_workload_case(args, local_rank):
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream()
     case = args.case
-    widx = {"tiny": 0, "hoisted": 1, "ffn128": 2, "ffn2048": 3, "ps15": 4}[case]
+    widx = {"tiny": 0, "hoisted": 1, "rotsum": 1, "ffn128": 2, "ffn2048": 3, "ps15": 4}[case]
     master = S.master_seed(widx)
     gen = torch.Generator(device=dev)
     gen.manual_seed(master)
@@ -437,6 +444,22 @@ def run_workload_case(args, local_rank):
             n_in * N_KEYS
         cfg = {"workload": case, "N": N, "L": L, "K": K, "dnum": DNUM, "level": L, "n_ciphertexts": n_in,
                "n_steps": N_KEYS, "l2": "inputs and keys larger than L2 (1.6 GB of keys per step)"}
+    elif case == "rotsum":
+        steps, _ = workload_inputs(master, ctx.primes[:L], N_CTS)
+        for st in steps:
+            upload(he.HE_KEY_ROTATION, st)
+        n_in = N_CTS // N_KEYS
+        x = device_residues(torch, (n_in, 2), ctx.primes[:L], N, gen, dev)
+        y = torch.empty_like(x)
+        xs = [he.Ciphertext(x[i], L, 2.0 ** 40) for i in range(n_in)]
+
+        def step():
+            he.he_rotate_sum_hoisted(ctx, xs, steps, [he.Ciphertext(y[i], L, 2.0 ** 40) for i in range(n_in)])
+
+        metric, unit, per_step = ("summed rotations/s (4 ciphertexts x 16 steps into 4 sums, N=2^16, level 24)",
+                                  "rotations/s", n_in * N_KEYS)
+        cfg = {"workload": case, "N": N, "L": L, "K": K, "dnum": DNUM, "level": L, "n_ciphertexts": n_in,
+               "n_steps": N_KEYS, "l2": "keys larger than L2 (1.6 GB of keys per step)"}
     elif case == "ps15":
         upload(he.HE_KEY_RELIN, 0)
         n = 64
@@ -735,7 +758,7 @@ def main():
             run_ntt_case(args, local_rank)
         elif args.case == "rot_small":
             run_rot_small_case(args, local_rank)
-        elif args.case in ("ffn128", "ffn2048", "ps15", "tiny", "hoisted"):
+        elif args.case in ("ffn128", "ffn2048", "ps15", "tiny", "hoisted", "rotsum"):
             run_workload_case(args, local_rank)
         else:
             run_native(args, rank, world, local_rank)

@@ -160,6 +160,7 @@ int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, in
 int rotate_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t* steps, int n_steps, he_ct* out);
 int rotate_sum_many(he_ctx* c, const he_ct* z, int n_out, int n_terms, const int32_t* steps, const he_ct* base,
                     he_ct* out);
+int rotate_sum_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t* steps, int n_steps, he_ct* out);
 
 // Scratch slots: 0 = key switching internals, 1 = rescale temporaries,
 // 2 = HMult temporaries and key generation, 3 = driver buffers (polynomial

@@ -338,13 +338,14 @@ __global__ void __launch_bounds__(256, 5)  // 5 blocks per SM: more loads in fli
 // Sum of G key inner products per output, for one ModDown of the sum:
 // u[o][0/1][t][c] = sum_{g<G} sum_j x_{r,j}[t][c] * key_r,j[b/a][row(t)][c],
 // r = o G + g, x_{r,j} as in k_ks_inner for key switch r (its own sigma on
-// the digit's own rows, its raised digits elsewhere).  FP64 rows add the
+// the digit's own rows, its raised digits elsewhere; HOIST: the raised
+// digits of ciphertext xsrc[r], read through sigma_r).  FP64 rows add the
 // signed products of all G switches (|sum| <= G ND 5q/8 < 2^51 for G <= 64,
 // ND <= 15); integer rows reduce each switch's 128-bit sum once and add the
 // results, kept in [0, 2q).
-template <int ND>
+template <int ND, bool HOIST>
 __global__ void __launch_bounds__(256, 4)
-    k_ks_inner_sum(const uint64_t* __restrict__ ext, PtrList din, GalList gal, PtrList keys, int G,
+    k_ks_inner_sum(const uint64_t* __restrict__ ext, PtrList din, GalList gal, PtrList keys, IdxList xsrc, int G,
                    uint64_t* __restrict__ u, int n_rows, int level, int L, int LK, int n_ext,
                    const DevPrime* __restrict__ pr, const FpMod* __restrict__ fpm, ModupArgs a, int logn) {
     const int N = 1 << logn;
@@ -373,8 +374,14 @@ __global__ void __launch_bounds__(256, 4)
                 xs[j] = own_sw ? make_ulonglong2(v.y, v.x) : v;
             } else {
                 const int pos = t < s0 ? t : t - ns;
-                xs[j] = __ldg(reinterpret_cast<const ulonglong2*>(
-                    ext + ((size_t)a.ext_off[j] * n_ext + (size_t)r * (n_rows - ns) + pos) * N + c));
+                const uint64_t* e =
+                    ext + ((size_t)a.ext_off[j] * n_ext + (size_t)(HOIST ? xsrc.i[r] : r) * (n_rows - ns) + pos) * N;
+                if (HOIST) {
+                    const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2*>(e + (own & ~1)));
+                    xs[j] = own_sw ? make_ulonglong2(v.y, v.x) : v;
+                } else {
+                    xs[j] = __ldg(reinterpret_cast<const ulonglong2*>(e + c));
+                }
             }
             kbs[j] = __ldg(reinterpret_cast<const ulonglong2*>(key + (((size_t)j * 2 + 0) * LK + krow) * N + c));
             kas[j] = __ldg(reinterpret_cast<const ulonglong2*>(key + (((size_t)j * 2 + 1) * LK + krow) * N + c));
@@ -661,7 +668,7 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     // summed: n_md = n / G outputs, each the sum of G key switches
     const int G = io.sum_terms;
     const bool summed = G > 0;
-    if (summed && (hoist || n % G)) return set_err(c, HE_EINVAL, "key switch: bad summed lists");
+    if (summed && n % G) return set_err(c, HE_EINVAL, "key switch: bad summed lists");
     const int n_md = summed ? n / G : n;
     uint64_t* base;
     int rc = scratch_slot(c, 0, key_switch_scratch_words(c, nm, n_md, level), &base);
@@ -790,9 +797,12 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     switch (nd) {
 #define HE_KS_CASE(D)                                                                                             \
     case D:                                                                                                       \
-        if (summed)                                                                                               \
-            k_ks_inner_sum<D><<<dim3(n_md, gx2, n_rows), blk, 0, c->stream>>>(                                    \
-                ext, din, gal, keys, G, u, n_rows, level, L, LK, nm, c->d_prime, c->d_fpmod, ma, c->log_n);       \
+        if (summed && hoist)                                                                                      \
+            k_ks_inner_sum<D, true><<<dim3(n_md, gx2, n_rows), blk, 0, c->stream>>>(                              \
+                ext, din, gal, keys, xsrc, G, u, n_rows, level, L, LK, nm, c->d_prime, c->d_fpmod, ma, c->log_n); \
+        else if (summed)                                                                                          \
+            k_ks_inner_sum<D, false><<<dim3(n_md, gx2, n_rows), blk, 0, c->stream>>>(                             \
+                ext, din, gal, keys, xsrc, G, u, n_rows, level, L, LK, nm, c->d_prime, c->d_fpmod, ma, c->log_n); \
         else if (hoist)                                                                                           \
             k_ks_inner<D, true><<<dim3(n, gx2, n_rows), blk, 0, c->stream>>>(                                     \
                 ext, din, gal, keys, xsrc, u, n_rows, level, L, LK, nm, c->d_prime, c->d_fpmod, ma, c->log_n);    \
@@ -1153,9 +1163,111 @@ int rotate_sum_many(he_ctx* c, const he_ct* z, int n_out, int n_terms, const int
     return HE_OK;
 }
 
+// Rotate-and-sum of single ciphertexts with one ModUp and one ModDown each
+// (the hoisting of Halevi-Shoup combined with the ModDown hoisting of
+// Bossuat et al.):
+//   out[i] = sum_s rot_{steps[s]}(in[i])
+//          = (sum_s sigma_s(c0) + ModDown(sum_s sum_j sigma_s(ModUp_j(c1)) (.) evk_{s,j}.b),
+//                                 ModDown(sum_s sum_j sigma_s(ModUp_j(c1)) (.) evk_{s,j}.a)).
+// Steps whose Galois element is 1 add in[i] unchanged.  Inputs go in chunks
+// of floor(64 / n_steps): one pre-sum launch, then one key-switching pass in
+// hoisted and summed mode.
+int rotate_sum_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t* steps, int n_steps, he_ct* out) {
+    if (n_in < 0 || n_steps < 0) return set_err(c, HE_EINVAL, "rotate_sum_hoisted: negative count");
+    if (n_in == 0) return HE_OK;
+    if (n_steps < 1 || n_steps > kMaxBatch)
+        return set_err(c, HE_EINVAL, "rotate_sum_hoisted: 1 to %d steps", kMaxBatch);
+    if (!in || !out || !steps) return set_err(c, HE_EINVAL, "rotate_sum_hoisted: null argument");
+    const int level = in[0].level;
+    std::set<const uint64_t*> ins;
+    for (int i = 0; i < n_in; i++) {
+        int rc = ct_ok(c, &in[i], "rotate_sum_hoisted");
+        if (rc) return rc;
+        if (in[i].level != level) return set_err(c, HE_ELEVEL, "rotate_sum_hoisted: mixed levels");
+        ins.insert(in[i].data);
+    }
+    for (int i = 0; i < n_in; i++) {
+        if (!out[i].data || ((uintptr_t)out[i].data & 15))
+            return set_err(c, HE_EINVAL, "rotate_sum_hoisted: null or unaligned output %d", i);
+        if (ins.count(out[i].data)) return set_err(c, HE_EINVAL, "rotate_sum_hoisted: output %d aliases an input", i);
+    }
+    std::vector<uint64_t> gal(n_steps);
+    int g_eff = 0;
+    for (int s = 0; s < n_steps; s++) {
+        gal[s] = galois_elt(c, steps[s]);
+        if (gal[s] == 1) continue;
+        if (!c->rot_keys.count(gal[s]))
+            return set_err(c, HE_ENOKEY, "rotate_sum_hoisted: no key for step %d (galois %llu)", steps[s],
+                           (unsigned long long)gal[s]);
+        g_eff++;
+    }
+    const size_t N = c->N, ctw = (size_t)2 * level * N;
+    const int G = n_steps, mc = std::max(1, kMaxBatch / G);
+    uint64_t* S = nullptr;
+    if (g_eff) {
+        int rc = scratch_slot(c, 2, ctw * std::min(mc, n_in), &S);
+        if (rc) return rc;
+    }
+    for (int i0 = 0; i0 < n_in; i0 += mc) {
+        const int m = std::min(mc, n_in - i0);
+        PtrList zp, bp;
+        GalList gl;
+        MutPtrList sp;
+        for (int k = 0; k < kMaxBatch; k++) {
+            zp.p[k] = nullptr;
+            gl.g[k] = 0;
+            bp.p[k] = nullptr;
+            sp.p[k] = nullptr;
+        }
+        for (int o = 0; o < m; o++) {
+            for (int g = 0; g < G; g++) {
+                zp.p[o * G + g] = in[i0 + o].data;
+                gl.g[o * G + g] = gal[g] == 1 ? 0 : gal[g];
+            }
+            sp.p[o] = g_eff ? S + (size_t)o * ctw : out[i0 + o].data;
+        }
+        prof_begin(c, HE_PROF_ELEMENTWISE);
+        k_rot_presum<<<dim3((unsigned)((N + 255) / 256), 2 * level, m), 256, 0, c->stream>>>(
+            zp, gl, bp, sp, G, level, c->d_prime, c->log_n);
+        int rc = lc(c, "rot_presum");
+        if (rc) return rc;
+        prof_end(c, HE_PROF_ELEMENTWISE, 8.0 * m * ((double)(G - g_eff) * ctw + (double)g_eff * ctw / 2 + ctw));
+        if (!g_eff) continue;
+        KsIoList io;
+        io.sig_add0 = false;
+        io.sum_terms = g_eff;
+        for (int o = 0; o < m; o++) {
+            io.hoist_d.push_back(in[i0 + o].data + (size_t)level * N);
+            for (int g = 0; g < G; g++) {
+                if (gal[g] == 1) continue;
+                io.galois.push_back(gal[g]);
+                io.key.push_back(c->rot_keys[gal[g]].d);
+                io.d.push_back(in[i0 + o].data + (size_t)level * N);
+                io.hoist_src.push_back(o);
+            }
+            io.out.push_back(out[i0 + o].data);
+            io.add0.push_back(S + (size_t)o * ctw);
+            io.add1.push_back(S + (size_t)o * ctw + (size_t)level * N);
+        }
+        if ((rc = key_switch_chunk(c, m * g_eff, level, io))) return rc;
+    }
+    for (int i = 0; i < n_in; i++) {
+        out[i].level = level;
+        out[i].scale = in[i].scale;
+        out[i].is_ntt = 1;
+    }
+    return HE_OK;
+}
+
 }  // namespace he
 
 using namespace he;
+
+extern "C" int he_rotate_sum_hoisted(he_ctx* c, const he_ct* in, int n_in, const int32_t* steps, int n_steps,
+                                     he_ct* out) {
+    if (!c) return HE_EINVAL;
+    return rotate_sum_hoisted_many(c, in, n_in, steps, n_steps, out);
+}
 
 extern "C" int he_rotate_sum(he_ctx* c, const he_ct* z, int n_out, int n_terms, const int32_t* steps,
                              const he_ct* base, he_ct* out) {

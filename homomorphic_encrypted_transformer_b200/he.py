@@ -83,6 +83,7 @@ _sig("he_rotate", _i, _vp, ctypes.POINTER(he_ct), ctypes.c_int32, ctypes.POINTER
 _sig("he_rotate_batch", _i, _vp, ctypes.POINTER(he_ct), _vp, ctypes.POINTER(he_ct), _i)
 _sig("he_rotate_hoisted", _i, _vp, ctypes.POINTER(he_ct), _i, _vp, _i, ctypes.POINTER(he_ct))
 _sig("he_rotate_sum", _i, _vp, ctypes.POINTER(he_ct), _i, _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct))
+_sig("he_rotate_sum_hoisted", _i, _vp, ctypes.POINTER(he_ct), _i, _vp, _i, ctypes.POINTER(he_ct))
 _sig("he_rotate_batch_host", _i, _vp, _vp, _i, _vp, _vp, _i)
 _sig("he_hmult_relin_rescale", _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct), ctypes.POINTER(he_ct))
 _sig("he_rescale", _i, _vp, ctypes.POINTER(he_ct))
@@ -293,6 +294,19 @@ def he_rotate_sum(ctx, z, steps, base, cts_out):
     ao = (he_ct * max(1, n_out))(*[c._c() for c in cts_out])
     st = np.ascontiguousarray(steps, dtype=np.int32)
     _check(ctx, _lib.he_rotate_sum(ctx.ptr, az, n_out, n_terms, _ptr(st), ab, ao))
+    for c, o in zip(cts_out, ao):
+        c._update(o)
+
+
+def he_rotate_sum_hoisted(ctx, cts_in, steps, cts_out):
+    """cts_out[i] = sum_s rot_{steps[s]}(cts_in[i]), one ModUp and one ModDown each."""
+    if len(cts_out) != len(cts_in):
+        raise ValueError("he_rotate_sum_hoisted: one output per input")
+    n_in = len(cts_in)
+    ai = (he_ct * max(1, n_in))(*[c._c() for c in cts_in])
+    ao = (he_ct * max(1, n_in))(*[c._c() for c in cts_out])
+    st = np.ascontiguousarray(steps, dtype=np.int32)
+    _check(ctx, _lib.he_rotate_sum_hoisted(ctx.ptr, ai, n_in, _ptr(st), len(st), ao))
     for c, o in zip(cts_out, ao):
         c._update(o)
 

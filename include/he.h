@@ -204,6 +204,23 @@ int he_rotate_hoisted(he_ctx* ctx, const he_ct* in, int n_in, const int32_t* ste
  */
 int he_rotate_sum(he_ctx* ctx, const he_ct* z, int n_out, int n_terms, const int32_t* steps, const he_ct* base,
                   he_ct* out);
+/*
+ * Rotate-and-sum of single ciphertexts with one ModUp and one ModDown each:
+ * the hoisting of he_rotate_hoisted and the single ModDown of he_rotate_sum
+ * together.  For in[i] = (c0, c1) and k_s = 5^(steps[s] mod N/2) mod 2N,
+ *   out[i] = sum_s rot_{steps[s]}(in[i])
+ *          = (sum_s sigma_s(c0) + ModDown(sum_s sum_j sigma_s(ModUp_j(c1)) (.) evk_{s,j}.b),
+ *                                 ModDown(sum_s sum_j sigma_s(ModUp_j(c1)) (.) evk_{s,j}.a)).
+ * Residues differ from adding he_rotate_hoisted results by the rounding of
+ * one ModDown instead of n_steps (at most (n_steps+1)(K+1)/2 per
+ * coefficient); the slots agree.  A step whose Galois element is 1 adds
+ * in[i] unchanged.  in: n_in device ciphertexts at one level, 16-byte
+ * aligned; 1 <= n_steps <= 64; out: n_in device ciphertexts with room for
+ * that level, none overlapping an input, each given in[i]'s level and scale.
+ * Errors: HE_EINVAL, HE_ELEVEL, HE_EDOMAIN, HE_ENOKEY as he_rotate_hoisted;
+ * nothing is launched then.
+ */
+int he_rotate_sum_hoisted(he_ctx* ctx, const he_ct* in, int n_in, const int32_t* steps, int n_steps, he_ct* out);
 
 /* Tensor, relinearise (key switch of d2 with the s^2 key), rescale.
  * a and b at the same level l >= 2; out at level l-1, scale (sa*sb)/q_{l-1}.

@@ -128,3 +128,22 @@ def test_rotation_sum_errors():
     he.he_sync(st.ctx)
     want = C.rotate_sum([st.encrypt(z, 3)], [1], {1: st.oracle_rot_key(1)}, st.P)
     assert np.array_equal(st.from_gpu(y[0]), want["c"])
+
+
+def test_rotation_sum_hoisted_errors():
+    he = lib()
+    st = Setup(12, 3, 1, 3, seed=67)
+    st.upload_rot(1)
+    z = S.complex_slots(st.seed, st.P.n_slots, -1, 1)
+    x3 = st.to_gpu(st.encrypt(z, 3))
+    x2 = st.to_gpu(st.encrypt(z, 2), room=3)
+    y = [st.empty_gpu(3), st.empty_gpu(3)]
+    assert _code(he.he_rotate_sum_hoisted, st.ctx, [x3], [1, 4], y[:1]) == he.HE_ENOKEY
+    assert _code(he.he_rotate_sum_hoisted, st.ctx, [x3, x2], [1], y) == he.HE_ELEVEL
+    assert _code(he.he_rotate_sum_hoisted, st.ctx, [x3], [1], [x3]) == he.HE_EINVAL  # aliases the input
+    assert _code(he.he_rotate_sum_hoisted, st.ctx, [x3], [], y[:1]) == he.HE_EINVAL  # no steps
+    assert _code(he.he_rotate_sum_hoisted, st.ctx, [x3], [1] * 65, y[:1]) == he.HE_EINVAL  # above 64 steps
+    he.he_rotate_sum_hoisted(st.ctx, [x3], [1, 1], y[:1])  # and still works
+    he.he_sync(st.ctx)
+    want = C.rotate_sum_hoisted(st.encrypt(z, 3), [1, 1], {1: st.oracle_rot_key(1)}, st.P)
+    assert np.array_equal(st.from_gpu(y[0]), want["c"])

@@ -296,3 +296,55 @@ def test_rotation_sum_chunks():
     switches in summed mode)."""
     st = Setup(11, 3, 1, 3, seed=48)
     _sum_case(st, 3, 5, list(range(1, 21)))
+
+
+def _sum_hoisted_case(st, level, n_in, steps):
+    """he_rotate_sum_hoisted against the oracle: identity steps add the input,
+    the others go through rotate_sum_hoisted; residue for residue."""
+    he = lib()
+    P = st.P
+    eff = [s for s in steps if P.galois_elt(s) != 1]
+    for s in sorted(set(eff)):
+        st.upload_rot(s)
+    keys = {s: st.oracle_rot_key(s) for s in eff}
+    cts = [st.encrypt(S.complex_slots(st.seed, P.n_slots, -1, 1, 500 + i), level, ct_id=500 + i)
+           for i in range(n_in)]
+    ys = [st.empty_gpu(level) for _ in range(n_in)]
+    he.he_rotate_sum_hoisted(st.ctx, [st.to_gpu(c) for c in cts], steps, ys)
+    he.he_sync(st.ctx)
+    qm = P.q[:level]
+    for i, ct in enumerate(cts):
+        parts = [ct] * (len(steps) - len(eff))
+        if eff:
+            parts.append(C.rotate_sum_hoisted(ct, eff, keys, P))
+        want = parts[0]["c"]
+        for p_ in parts[1:]:
+            want = np.stack([C.add_rows(want[c], p_["c"][c], qm) for c in range(2)])
+        assert ys[i].level == level and ys[i].scale == ct["scale"]
+        assert np.array_equal(st.from_gpu(ys[i]), want), i
+    return cts, ys
+
+
+def test_rotation_sum_hoisted_tiny():
+    """Rotate-and-sum of two ciphertexts over {1, 2, -1, 4}: bit-exact and
+    decrypting to the summed rolled slots; then an identity step."""
+    st = Setup(12, 3, 1, 3, seed=S.master_seed(0))
+    steps = [1, 2, -1, 4]
+    cts, ys = _sum_hoisted_case(st, 3, 2, steps)
+    for i in range(2):
+        z = S.complex_slots(st.seed, st.P.n_slots, -1, 1, 500 + i)
+        got = C.make_ct(st.from_gpu(ys[i]), 3, 2.0 ** 40)
+        assert np.max(np.abs(C.decrypt_decode(got, st.s, st.P) - sum(np.roll(z, -s) for s in steps))) < 1e-5
+    _sum_hoisted_case(st, 3, 1, [0, 3])
+
+
+@pytest.mark.parametrize("level", [7, 4, 1])
+def test_rotation_sum_hoisted_mid_levels(level):
+    st = Setup(11, 7, 3, 3, seed=49)
+    _sum_hoisted_case(st, level, 2, [5, -3, 17])
+
+
+def test_rotation_sum_hoisted_chunks():
+    """5 ciphertexts x 20 steps: chunks of 3 and 2 inputs."""
+    st = Setup(11, 3, 1, 3, seed=50)
+    _sum_hoisted_case(st, 3, 5, list(range(1, 21)))
