@@ -163,8 +163,9 @@ int rotate_sum_many(he_ctx* c, const he_ct* z, int n_out, int n_terms, const int
 int rotate_sum_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t* steps, int n_steps, he_ct* out);
 
 // Scratch slots: 0 = key switching internals, 1 = rescale temporaries,
-// 2 = HMult temporaries and key generation, 3 = driver buffers (polynomial
-// evaluation, BSGS).  A call only uses slots below the ones its callers hold.
+// 2 = HMult temporaries, key generation and the pre-sums of the summed
+// rotations, 3 = driver buffers (polynomial evaluation, BSGS).  A call only
+// uses slots below the ones its callers hold.
 constexpr int kScratchSlots = 4;
 int scratch_slot(he_ctx* c, int slot, size_t words, uint64_t** out);
 

@@ -79,3 +79,12 @@ def test_reference_arm_two_ranks_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_oracle_baselines_of_the_rotation_cases():
+    """The reference leg of the hoisted and rotate-and-sum cases: the oracle
+    on a bounded full-size sample, reported as rotations/s."""
+    for case in ("hoisted", "rotsum"):
+        r = bench.workload_cpu_baseline(case, 0.5)
+        assert r["kind"] == "oracle" and r["unit"] == "rotations/s" and r["value"] > 0 and r["cores"] >= 1
+        assert "key generation excluded" in r["sample"]
