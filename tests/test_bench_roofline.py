@@ -1,0 +1,42 @@
+"""Host arithmetic of bench.py's roofline on CPU: which ceiling binds a
+kernel class, and the achieved/peak figures of each case."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+INT_S, FP_S, HBM = 1.0e12, 3.0e12, 6000.0  # products/s, products/s, GB/s
+
+
+def test_hbm_bound_class():
+    # 12 GB take 2 ms at 6 TB/s, 1e9 integer products 1 ms at 1e12/s: bytes bind
+    ms, launches, nbytes, mults, mults_fp = 2.0, 1, 12e9, 1e9, 0.0
+    r = bench.roofline_for("x", (ms, launches, nbytes, mults, mults_fp), INT_S, FP_S, HBM, "measured")
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(12e9 / 2e-3 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / HBM)
+    assert r["traffic"] is None
+
+
+def test_alu_bound_class_weights_the_two_pipes():
+    # 3e9 products, 2e9 of them FP64: ideal 1e9/1e12 + 2e9/3e12 = 1.667 ms; bytes small
+    ms, launches, nbytes, mults, mults_fp = 4.0, 2, 1e6, 6e9, 4e9  # per launch: 2 ms, 3e9 products
+    r = bench.roofline_for("x", (ms, launches, nbytes, mults, mults_fp), INT_S, FP_S, HBM, "measured")
+    assert r["bound"] == "alu" and r["unit"] == "Gmodmul/s"
+    ideal = 1e9 / INT_S + 2e9 / FP_S
+    assert r["peak"] == pytest.approx(3e9 / ideal / 1e9)
+    assert r["achieved"] == pytest.approx(3e9 / 2e-3 / 1e9)
+    assert r["frac"] == pytest.approx(ideal / 2e-3)
+    assert r["fp64_share"] == pytest.approx(2.0 / 3.0)
+
+
+def test_traffic_is_scaled_from_the_committed_capture():
+    name = next(iter(bench.NCU_TRAFFIC_RATIO))
+    r = bench.roofline_for(name, (1.0, 1, 1e9, 1.0, 0.0), INT_S, FP_S, HBM, "measured")
+    assert r["traffic"] == pytest.approx(bench.NCU_TRAFFIC_RATIO[name] * 1e9)
+    assert 0.8 < bench.NCU_TRAFFIC_RATIO[name] < 1.3  # DRAM bytes near the algorithmic bytes
