@@ -41,6 +41,7 @@ STREAMS = {
     "pt_residues": 15,
     "ntt_residues": 16,
     "groups": 17,
+    "normal_slots": 18,
 }
 
 SIGMA = 3.2
@@ -95,6 +96,12 @@ def real_slots(master, n_slots, lo, hi, *sub):
     """n_slots real values iid U[lo, hi] (as complex with zero imaginary part)."""
     g = rng(master, "slots", *sub)
     return g.uniform(lo, hi, size=n_slots).astype(np.complex128)
+
+
+def normal_slots(master, n_slots, mean, std, lo, hi, *sub):
+    """n_slots real values iid N(mean, std^2) clipped to [lo, hi] (as complex)."""
+    g = rng(master, "normal_slots", *sub)
+    return np.clip(g.normal(mean, std, size=n_slots), lo, hi).astype(np.complex128)
 
 
 def weights(master, shape, lo, hi, *sub):

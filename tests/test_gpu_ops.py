@@ -121,6 +121,28 @@ def test_ps15_small():
         assert np.array_equal(st.from_gpu(outs[i]), want["c"])
 
 
+def test_ps15_gelu_coefficients():
+    """The distribution-fitted GELU coefficients (zeros above degree 8) on the
+    same engine: 3 ciphertexts of normal inputs, residue for residue."""
+    from homomorphic_encrypted_transformer_b200 import gelu as G
+
+    he = lib()
+    st = Setup(12, 8, 3, 3, seed=34)
+    P = st.P
+    coeffs = G.fit()
+    st.upload_relin()
+    cts = [st.encrypt(S.normal_slots(st.seed, P.n_slots, G.input_mean(), 1.0, G.LO, G.HI, i), 8, ct_id=i)
+           for i in range(3)]
+    xs = [st.to_gpu(c) for c in cts]
+    outs = [st.empty_gpu(8) for _ in cts]
+    he.he_poly_eval_ps15(st.ctx, xs, coeffs, C.PS_TOP_SCALE, outs)
+    he.he_sync(st.ctx)
+    for i, c in enumerate(cts):
+        want = C.ps_eval_deg15(c, coeffs, st.oracle_relin_key(), P)
+        assert outs[i].level == want["level"] and outs[i].scale == want["scale"]
+        assert np.array_equal(st.from_gpu(outs[i]), want["c"])
+
+
 def test_bsgs_small():
     """y = W x by diagonals with BSGS on N=2^11: 16 features x 64 tokens,
     4 baby x 4 giant steps, 2 input / 2 output blocks, 2 token groups."""
