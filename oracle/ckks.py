@@ -839,6 +839,64 @@ def bsgs_matvec(X, pt, bs, gs, slot_stride, keys, params, outputs, pt_scale, hoi
 
 
 # --------------------------------------------------------------------------
+# One encrypted attention head (AEGIS summary section 2.3: Q x K^T, a
+# polynomial Softmax, A x V).  The pages name the three stages only.
+# Reading: token-duplicated feature-major packing, d features x n tokens with
+# d 2n = N/2; scores by token offset (the diagonal method over the token
+# axis); the feature sum by log2(d) rotations; Softmax's exponential by the
+# degree-15 polynomial, without the division by the row sums.
+# --------------------------------------------------------------------------
+
+def attention_pack(X, dup):
+    """Slot vector of a d x n matrix X, feature-major with stride 2n:
+    slot f 2n + t holds X[f][t mod n] for every t < 2n (dup: the token axis
+    twice, so that a slot rotation by delta < n shifts every feature's tokens
+    cyclically), or X[f][t] for t < n and 0 for t >= n."""
+    d, n = X.shape
+    out = np.zeros((d, 2 * n), dtype=np.complex128)
+    out[:, :n] = X
+    if dup:
+        out[:, n:] = X
+    return out.reshape(-1)
+
+
+def attention_scores(q, k, n_tok, d, offsets, keys, rlk, params):
+    """S_delta for each token offset delta (0 <= delta < n):
+        P = HMRR(q, rot_delta(k)),  rot_delta(k) hoisted (one ModUp of k; delta = 0: k),
+        S <- S + rot_{2n 2^i}(S) for i < log2(d), starting from S = P.
+    q packs Q with zeros on t >= n, k packs K token-duplicated; then every
+    feature block of S_delta holds sum_f Q[f][t] K[f][(t + delta) mod n] at
+    t < n and 0 at t >= n (the sum wraps around the d 2n = N/2 slots)."""
+    assert d * 2 * n_tok == params.n_slots and d & (d - 1) == 0
+    nz = [o for o in offsets if o % params.n_slots]
+    rot = dict(zip(nz, rotate_hoisted(k, nz, keys, params)))
+    out = []
+    for o in offsets:
+        acc = hmult_relin_rescale(q, rot[o] if o in rot else k, rlk, params)
+        for i in range(d.bit_length() - 1):
+            st = 2 * n_tok * (1 << i)
+            acc = add(acc, rotate(acc, st, keys[st], params), params)
+        out.append(acc)
+    return out
+
+
+def attention_av(a, v, offsets, keys, rlk, params):
+    """O = sum_delta HMRR(a_delta, drop(rot_delta(v))) over the offsets,
+    rot_delta(v) hoisted (one ModUp of v; delta = 0: v) and dropped to
+    a_delta's level.  With a_delta = p(S_delta) replicated over the feature
+    blocks and v token-duplicated, slot f 2n + t of O holds
+    sum_delta p(S_delta[t]) V[f][(t + delta) mod n] for t < n."""
+    nz = [o for o in offsets if o % params.n_slots]
+    rot = dict(zip(nz, rotate_hoisted(v, nz, keys, params)))
+    out = None
+    for ad, o in zip(a, offsets):
+        vv = drop_level(rot[o] if o in rot else v, ad["level"])
+        t = hmult_relin_rescale(ad, vv, rlk, params)
+        out = t if out is None else add(out, t, params)
+    return out
+
+
+# --------------------------------------------------------------------------
 # Paterson-Stockmeyer evaluation of a degree-15 polynomial
 # (AEGIS summary section 2.3: Softmax by polynomial approximation)
 # --------------------------------------------------------------------------
