@@ -171,6 +171,14 @@ int scratch_slot(he_ctx* c, int slot, size_t words, uint64_t** out);
 
 // out[i] = rescale(in[i]) for n ciphertexts at `level` (out may equal in).
 int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int level);
+// Batched helpers of the drivers (ops.cu): HMult + relinearisation + rescale
+// of pairs at `level`; out_i = a_i + b_i at lv limbs (out may equal a);
+// out_i = in_i keeping limbs < lv (out != in).
+int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector<const uint64_t*>& b,
+              const std::vector<uint64_t*>& out, int level);
+int add_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector<const uint64_t*>& b,
+             const std::vector<uint64_t*>& o, int lv);
+int drop_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int lin, int lv);
 
 int elementwise_setup(he_ctx* c);
 

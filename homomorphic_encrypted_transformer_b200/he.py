@@ -84,6 +84,9 @@ _sig("he_rotate_batch", _i, _vp, ctypes.POINTER(he_ct), _vp, ctypes.POINTER(he_c
 _sig("he_rotate_hoisted", _i, _vp, ctypes.POINTER(he_ct), _i, _vp, _i, ctypes.POINTER(he_ct))
 _sig("he_rotate_sum", _i, _vp, ctypes.POINTER(he_ct), _i, _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct))
 _sig("he_rotate_sum_hoisted", _i, _vp, ctypes.POINTER(he_ct), _i, _vp, _i, ctypes.POINTER(he_ct))
+_sig("he_attention_scores", _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct), _i, _i, _vp, _i,
+     ctypes.POINTER(he_ct))
+_sig("he_attention_output", _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct), _i, _vp, _i, ctypes.POINTER(he_ct))
 _sig("he_rotate_batch_host", _i, _vp, _vp, _i, _vp, _vp, _i)
 _sig("he_hmult_relin_rescale", _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct), ctypes.POINTER(he_ct))
 _sig("he_rescale", _i, _vp, ctypes.POINTER(he_ct))
@@ -309,6 +312,29 @@ def he_rotate_sum_hoisted(ctx, cts_in, steps, cts_out):
     _check(ctx, _lib.he_rotate_sum_hoisted(ctx.ptr, ai, n_in, _ptr(st), len(st), ao))
     for c, o in zip(cts_out, ao):
         c._update(o)
+
+
+def he_attention_scores(ctx, q, k, n_tok, d, offsets, s_out):
+    """s_out[i] = the scores of token offset offsets[i] (see he.h)."""
+    if len(s_out) != len(offsets):
+        raise ValueError("he_attention_scores: one output per offset")
+    cq, ck = q._c(), k._c()
+    ao = (he_ct * max(1, len(s_out)))(*[c._c() for c in s_out])
+    off = np.ascontiguousarray(offsets, dtype=np.int32)
+    _check(ctx, _lib.he_attention_scores(ctx.ptr, ctypes.byref(cq), ctypes.byref(ck), n_tok, d, _ptr(off), len(off), ao))
+    for c, o in zip(s_out, ao):
+        c._update(o)
+
+
+def he_attention_output(ctx, a, v, n_tok, offsets, out):
+    """out = sum_i HMRR(a[i], drop(rot_{offsets[i]}(v))) (see he.h)."""
+    if len(a) != len(offsets):
+        raise ValueError("he_attention_output: one weight ciphertext per offset")
+    aa = (he_ct * max(1, len(a)))(*[c._c() for c in a])
+    cv, co = v._c(), out._c()
+    off = np.ascontiguousarray(offsets, dtype=np.int32)
+    _check(ctx, _lib.he_attention_output(ctx.ptr, aa, ctypes.byref(cv), n_tok, _ptr(off), len(off), ctypes.byref(co)))
+    out._update(co)
 
 
 def he_rotate_batch_host(ctx, h_in, level, steps, h_out):

@@ -276,6 +276,37 @@ int he_pmult_accum_bsgs(he_ctx* ctx, const he_ct* x, int n_in, const uint64_t* d
                         int n_out, int bs, int gs, int slot_stride, int n_groups, he_ct* y);
 
 /*
+ * One encrypted attention head (AEGIS section 2.3: Q x K^T, a polynomial
+ * Softmax, A x V; the pages give no packing, this one is the engine's).
+ * d features x n_tok tokens with d a power of two and d * 2 * n_tok = N/2,
+ * feature-major with stride 2 n_tok: q holds Q[f][t] at slot f*2n + t for
+ * t < n (zeros at t >= n); k and v are token-duplicated (slot f*2n + t holds
+ * X[f][t mod n] for every t < 2n).
+ * he_attention_scores: for each offset delta = offsets[i] in [0, n_tok),
+ *   s[i] = HMRR(q, rot_delta(k)), then s[i] += rot_{2n*h}(s[i]) for
+ *   h = 1, 2, .., d/2, so that every feature block of s[i] holds
+ *   sum_f Q[f][t] K[f][(t + delta) mod n] at t < n (0 at t >= n).
+ *   The rotations of k are hoisted (he_rotate_hoisted).  q and k at one
+ *   level l >= 2; s[i] come back at level l-1, scale q.scale*k.scale/q_{l-1}.
+ *   Needs rotation keys for the non-zero offsets and for 2n*h, and the
+ *   relinearisation key.
+ * Softmax between the two calls is the caller's: shift each s[i] by a known
+ * bound (he_add_const) and evaluate the exponential by he_poly_eval_ps15.
+ * he_attention_output: out = sum_i HMRR(a[i], drop(rot_{offsets[i]}(v))),
+ *   a[i] the n_off weights at one level la >= 2 and scale, v at level
+ *   >= la; the rotations of v are hoisted.  Slot f*2n + t of out holds
+ *   sum_i A_i[t] V[f][(t + offsets[i]) mod n] for t < n.  out at la-1,
+ *   scale a.scale*v.scale/q_{la-1}.
+ * Scratch (context-owned): the rotated copies and one ciphertext per offset.
+ * Errors: HE_EINVAL (shape, offsets, null, unaligned, aliasing), HE_ELEVEL,
+ * HE_EDOMAIN, HE_ENOKEY; nothing is launched then.
+ */
+int he_attention_scores(he_ctx* ctx, const he_ct* q, const he_ct* k, int n_tok, int d, const int32_t* offsets,
+                        int n_off, he_ct* s);
+int he_attention_output(he_ctx* ctx, const he_ct* a, const he_ct* v, int n_tok, const int32_t* offsets, int n_off,
+                        he_ct* out);
+
+/*
  * Degree-15 polynomial sum_k c_k x^k by Paterson-Stockmeyer with 4 baby
  * powers (AEGIS section 2.3: Softmax by polynomial approximation):
  *   x2 = HMRR(x,x); x3 = HMRR(x2, drop(x)); x4 = HMRR(x2,x2);

@@ -31,7 +31,7 @@ def test_header_declares_the_hot_path_calls():
     names = set(declared_functions())
     for n in ["he_keygen_upload", "he_ntt_fwd", "he_ntt_inv", "he_rotate", "he_hmult_relin_rescale",
               "he_pmult_accum_bsgs", "he_rescale", "he_rotate_hoisted", "he_rotate_sum",
-              "he_rotate_sum_hoisted"]:
+              "he_rotate_sum_hoisted", "he_attention_scores", "he_attention_output"]:
         assert n in names
 
 

@@ -1,0 +1,99 @@
+"""GPU parity of one encrypted attention head against the oracle, residue
+for residue: the scores of 4 token offsets, their shifted exponentials by the
+degree-15 engine, and A x V (N = 2^11, 16 features x 32 tokens)."""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import ckks as C
+import seeded_inputs as S
+from tests.helpers import Setup, lib
+
+pytestmark = pytest.mark.gpu
+
+D, NT = 16, 32
+EXP = [1.0 / math.factorial(k) for k in range(16)]
+
+
+def test_attention_head_small():
+    he = lib()
+    st = Setup(11, 10, 4, 3, seed=S.master_seed(5))
+    P = st.P
+    Q = S.weights(st.seed, (D, NT), -0.25, 0.25, 1)
+    K = S.weights(st.seed, (D, NT), -0.25, 0.25, 2)
+    V = S.weights(st.seed, (D, NT), -0.25, 0.25, 3)
+    q = st.encrypt(C.attention_pack(Q, False), P.L, ct_id=0)
+    k = st.encrypt(C.attention_pack(K, True), P.L, ct_id=1)
+    v = st.encrypt(C.attention_pack(V, True), P.L, ct_id=2)
+    offsets = [0, 1, 5, 31]
+    steps = sorted({o for o in offsets if o} | {2 * NT * h for h in (1, 2, 4, 8)})
+    for s_ in steps:
+        st.upload_rot(s_)
+    st.upload_relin()
+    keys = {s_: st.oracle_rot_key(s_) for s_ in steps}
+    rlk = st.oracle_relin_key()
+    gq, gk, gv = st.to_gpu(q), st.to_gpu(k), st.to_gpu(v)
+
+    # scores
+    sc = [st.empty_gpu(P.L) for _ in offsets]
+    he.he_attention_scores(st.ctx, gq, gk, NT, D, offsets, sc)
+    he.he_sync(st.ctx)
+    want_s = C.attention_scores(q, k, NT, D, offsets, keys, rlk, P)
+    for g, w in zip(sc, want_s):
+        assert g.level == w["level"] == P.L - 1 and g.scale == w["scale"]
+        assert np.array_equal(st.from_gpu(g), w["c"])
+
+    # Softmax's exponential on scores shifted by -1 (|scores| <= 1 here)
+    Ks = [int(C.round_half_away(np.float64(-1.0 * w["scale"]))) for w in want_s]
+    for g, kk in zip(sc, Ks):
+        he.he_add_const(st.ctx, g, kk)
+    A = [st.empty_gpu(P.L) for _ in offsets]
+    he.he_poly_eval_ps15(st.ctx, sc, EXP, C.PS_TOP_SCALE, A)
+    he.he_sync(st.ctx)
+    want_a = [C.ps_eval_deg15(C.add_const(w, kk, P), EXP, rlk, P) for w, kk in zip(want_s, Ks)]
+    for g, w in zip(A, want_a):
+        assert g.level == w["level"] and g.scale == w["scale"]
+        assert np.array_equal(st.from_gpu(g), w["c"])
+
+    # A x V
+    out = st.empty_gpu(P.L)
+    he.he_attention_output(st.ctx, A, gv, NT, offsets, out)
+    he.he_sync(st.ctx)
+    want_o = C.attention_av(want_a, v, offsets, keys, rlk, P)
+    assert out.level == want_o["level"] and out.scale == want_o["scale"]
+    assert np.array_equal(st.from_gpu(out), want_o["c"])
+    # and the slots: sum over the 4 offsets of exp(score - 1) V
+    got = C.decrypt_decode(want_o, st.s, P).real.reshape(D, 2 * NT)[:, :NT]
+    Sc = Q.T @ K
+    want = np.zeros((D, NT))
+    for o in offsets:
+        for t in range(NT):
+            want[:, t] += np.exp(Sc[t, (t + o) % NT] - 1.0) * V[:, (t + o) % NT]
+    assert np.max(np.abs(got - want)) < 1e-4
+
+
+def test_attention_errors():
+    he = lib()
+    st = Setup(11, 10, 4, 3, seed=68)
+    P = st.P
+    z = S.complex_slots(st.seed, P.n_slots, -1, 1)
+    x = st.to_gpu(st.encrypt(z, P.L))
+    y = st.to_gpu(st.encrypt(z, P.L, ct_id=1))
+    out = [st.empty_gpu(P.L)]
+    with pytest.raises(he.HEError) as ei:  # d * 2 * n_tok must be N/2
+        he.he_attention_scores(st.ctx, x, y, 32, 8, [0], out)
+    assert ei.value.code == he.HE_EINVAL
+    with pytest.raises(he.HEError) as ei:  # no relinearisation key yet
+        he.he_attention_scores(st.ctx, x, y, 32, 16, [0], out)
+    assert ei.value.code == he.HE_ENOKEY
+    st.upload_relin()
+    with pytest.raises(he.HEError) as ei:  # offset outside [0, n_tok)
+        he.he_attention_scores(st.ctx, x, y, 32, 16, [32], out)
+    assert ei.value.code == he.HE_EINVAL
+    with pytest.raises(he.HEError) as ei:  # no key for offset 3 nor the feature-sum steps
+        he.he_attention_scores(st.ctx, x, y, 32, 16, [3], out)
+    assert ei.value.code == he.HE_ENOKEY
+    with pytest.raises(he.HEError) as ei:  # output aliases an input
+        he.he_attention_output(st.ctx, [x], y, 32, [0], x)
+    assert ei.value.code == he.HE_EINVAL
