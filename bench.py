@@ -16,6 +16,7 @@ host cores on a bounded sample of the same workload.
 """
 import argparse
 import json
+import math
 import os
 import subprocess
 import sys
@@ -48,7 +49,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--case", default="rotation",
                     choices=["rotation", "ntt", "rot_small", "ffn128", "ffn2048", "ps15", "tiny", "hoisted",
-                             "rotsum"],
+                             "rotsum", "attention"],
                     help="rotation: the headline workload (default). ffn128 / ffn2048 / ps15 / tiny: the other "
                          "workloads, one JSON line each. ntt / rot_small: kernel cases for profiler captures "
                          "(NTT of 512 limbs, or 8 rotations with 2 keys)")
@@ -257,6 +258,9 @@ def run_rot_small_case(args, local_rank):
 # ------------------------------------------------------------------ other workloads
 
 FFN = {"n_feat": 256, "n_tok": 128, "bs": 16, "gs": 16, "n_in": 3, "n_out": 12, "level": 12}
+# one attention head: d features x n_tok tokens with d 2 n_tok = N/2 at N = 2^16;
+# scores shifted by `shift` before the exponential
+ATT = {"d": 64, "n_tok": 256, "shift": 1.0}
 
 
 def device_residues(torch, shape_lead, primes, N, gen, dev):
@@ -279,7 +283,7 @@ def workload_cpu_baseline(case, seconds):
     timing)."""
     from oracle import ckks as C
 
-    widx = {"tiny": 0, "hoisted": 1, "rotsum": 1, "ffn128": 2, "ffn2048": 3, "ps15": 4}[case]
+    widx = {"tiny": 0, "hoisted": 1, "rotsum": 1, "ffn128": 2, "ffn2048": 3, "ps15": 4, "attention": 5}[case]
     master = S.master_seed(widx)
     t_end = time.perf_counter() + seconds
     if case == "tiny":
@@ -305,6 +309,29 @@ def workload_cpu_baseline(case, seconds):
                 "sample": "%d whole sequences (NTT round trip, 3 rotations, 1 HMult-relin-rescale), N=2^12" % done}
     P = C.Params(LOG_N, L, K, DNUM)
     s = S.secret(master, P.N)
+    if case == "attention":
+        d, n_tok = ATT["d"], ATT["n_tok"]
+        steps = [1] + [2 * n_tok * (1 << i) for i in range(d.bit_length() - 1)]
+        keys = {}
+        for st in steps:
+            a, e = S.key_draws(master, P.galois_elt(st), P.mods, P.N, P.dnum)
+            keys[st] = C.rotation_key(s, st, a, e, P)
+        a, e = S.key_draws(master, 2, P.mods, P.N, P.dnum)
+        rlk = C.relin_key(s, a, e, P)
+        q, k, v = (C.make_ct(S.uniform_residues(master, "ct_residues", P.q, P.N, i, lead=(2,)), L, 2.0 ** 40)
+                   for i in range(3))
+        exp_c = [1.0 / math.factorial(j) for j in range(16)]
+        done, t = 0, 0.0
+        while done < 1 or time.perf_counter() < t_end:
+            t0 = time.perf_counter()
+            sc = C.attention_scores(q, k, n_tok, d, [1], keys, rlk, P)
+            a_ = [C.ps_eval_deg15(x, exp_c, rlk, P) for x in sc]
+            C.attention_av(a_, v, [1], keys, rlk, P)
+            t += time.perf_counter() - t0
+            done += 1
+        return {"value": done / (t * n_tok), "unit": "heads/s", "cores": C.n_threads(), "kind": "oracle",
+                "sample": "%d full-size token offsets of one head (scores, exponential, output at level 24), "
+                          "scaled to the head's %d offsets; key generation excluded" % (done, n_tok)}
     if case in ("hoisted", "rotsum"):
         steps = workload_inputs(master, P.q, N_CTS)[0][:2]
         keys = {}
@@ -376,7 +403,9 @@ def run_workload_case(args, local_rank):
     hoisted (4 ciphertexts at level 24 each rotated by the rotation batch's
     16 steps through one ModUp per ciphertext: 64 hoisted rotations),
     rotsum (the same 4 ciphertexts each summed over its 16 rotations with
-    one ModUp and one ModDown: 64 rotations into 4 sums).
+    one ModUp and one ModDown: 64 rotations into 4 sums),
+    attention (one encrypted head at level 24: 64 features x 256 tokens, all
+    256 token offsets: scores, the degree-15 exponential, A x V).
     Inputs are seeded uniform residues on the device; the rotation and
     relinearisation keys are computed by the library from seeded draws."""
     import torch
@@ -387,7 +416,7 @@ def run_workload_case(args, local_rank):
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream()
     case = args.case
-    widx = {"tiny": 0, "hoisted": 1, "rotsum": 1, "ffn128": 2, "ffn2048": 3, "ps15": 4}[case]
+    widx = {"tiny": 0, "hoisted": 1, "rotsum": 1, "ffn128": 2, "ffn2048": 3, "ps15": 4, "attention": 5}[case]
     master = S.master_seed(widx)
     gen = torch.Generator(device=dev)
     gen.manual_seed(master)
@@ -460,6 +489,33 @@ def run_workload_case(args, local_rank):
                                   "rotations/s", n_in * N_KEYS)
         cfg = {"workload": case, "N": N, "L": L, "K": K, "dnum": DNUM, "level": L, "n_ciphertexts": n_in,
                "n_steps": N_KEYS, "l2": "keys larger than L2 (1.6 GB of keys per step)"}
+    elif case == "attention":
+        d, n_tok = ATT["d"], ATT["n_tok"]
+        offsets = list(range(n_tok))
+        for st in sorted(set(offsets[1:]) | {2 * n_tok * h for h in (1 << i for i in range(d.bit_length() - 1))}):
+            upload(he.HE_KEY_ROTATION, st)
+        upload(he.HE_KEY_RELIN, 0)
+        qkv = device_residues(torch, (3, 2), ctx.primes[:L], N, gen, dev)
+        q, k, v = (he.Ciphertext(qkv[i], L, 2.0 ** 40) for i in range(3))
+        sbuf = torch.empty((n_tok, 2, L, N), dtype=torch.int64, device=dev)
+        abuf = torch.empty_like(sbuf)
+        obuf = torch.empty((2, L, N), dtype=torch.int64, device=dev)
+        exp_c = [1.0 / math.factorial(j) for j in range(16)]
+
+        def step():
+            sc = [he.Ciphertext(sbuf[i], L, 2.0 ** 40) for i in range(n_tok)]
+            he.he_attention_scores(ctx, q, k, n_tok, d, offsets, sc)
+            kk = int(round(-ATT["shift"] * sc[0].scale))
+            for x in sc:
+                he.he_add_const(ctx, x, kk)
+            a = [he.Ciphertext(abuf[i], L, 2.0 ** 40) for i in range(n_tok)]
+            he.he_poly_eval_ps15(ctx, sc, exp_c, 2.0 ** 62, a)
+            he.he_attention_output(ctx, a, v, n_tok, offsets, he.Ciphertext(obuf, L, 2.0 ** 40))
+
+        metric, unit, per_step = "attention heads/s (64 features x 256 tokens, N=2^16, level 24)", "heads/s", 1
+        cfg = {"workload": case, "N": N, "level": L, "d": d, "tokens": n_tok, "offsets": n_tok,
+               "ops_per_head": {"hoisted_rotations": 2 * (n_tok - 1), "rotations": n_tok * (d.bit_length() - 1),
+                                "hmult_relin_rescale": 2 * n_tok, "degree15_evals": n_tok}}
     elif case == "ps15":
         upload(he.HE_KEY_RELIN, 0)
         n = 64
@@ -758,7 +814,7 @@ def main():
             run_ntt_case(args, local_rank)
         elif args.case == "rot_small":
             run_rot_small_case(args, local_rank)
-        elif args.case in ("ffn128", "ffn2048", "ps15", "tiny", "hoisted", "rotsum"):
+        elif args.case in ("ffn128", "ffn2048", "ps15", "tiny", "hoisted", "rotsum", "attention"):
             run_workload_case(args, local_rank)
         else:
             run_native(args, rank, world, local_rank)

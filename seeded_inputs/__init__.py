@@ -49,7 +49,7 @@ ERR_BOUND = 19
 
 # Master seed of each workload: 0xAE615000 + workload index (0 = tiny CKKS,
 # 1 = rotation batch, 2 = FFN1 128 tokens, 3 = FFN1 2048 tokens,
-# 4 = degree-15 polynomial).
+# 4 = degree-15 polynomial, 5 = attention head).
 MASTER_BASE = 0xAE615000
 
 
