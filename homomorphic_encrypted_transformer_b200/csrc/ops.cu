@@ -204,7 +204,6 @@ __global__ void k_tensor_many(PtrList pa, PtrList pb, MutPtrList pd, int level, 
 
 // --------------------------------------------------------------- host side
 
-static uint64_t h_mulmod(uint64_t a, uint64_t b, uint64_t m) { return (uint64_t)((unsigned __int128)a * b % m); }
 static uint64_t h_shoup(uint64_t w, uint64_t q) { return (uint64_t)(((unsigned __int128)w << 64) / q); }
 
 static uint64_t int_mod(int64_t K, uint64_t q) {
