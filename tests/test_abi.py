@@ -70,3 +70,23 @@ def test_explicit_primes_checked(he):
         he.he_derive_primes(12, 3, 1, 3, q=[P.q[0], P.q[1], 1000003], p=P.p)
     with pytest.raises(he.HEError):  # repeated prime
         he.he_derive_primes(12, 3, 1, 3, q=[P.q[0], P.q[1], P.q[1]], p=P.p)
+
+
+def test_bindings_check_list_lengths_before_calling(he):
+    """The list-taking bindings reject mismatched lengths on the host, before
+    any call into the library (no context needed)."""
+    import torch
+
+    x = he.Ciphertext(torch.zeros(16, dtype=torch.int64), 1, 1.0)
+    with pytest.raises(ValueError):
+        he.he_rotate_hoisted(None, [x, x], [1, 2], [x, x, x])  # needs 2 x 2 outputs
+    with pytest.raises(ValueError):
+        he.he_rotate_sum(None, [x, x, x], [1, 2], None, [x, x])  # needs 2 x 2 terms
+    with pytest.raises(ValueError):
+        he.he_rotate_sum(None, [x, x], [1, 2], [x, x], [x])  # one base per output
+    with pytest.raises(ValueError):
+        he.he_rotate_sum_hoisted(None, [x, x], [1], [x])  # one output per input
+    with pytest.raises(ValueError):
+        he.he_attention_scores(None, x, x, 32, 16, [0, 1], [x])  # one output per offset
+    with pytest.raises(ValueError):
+        he.he_attention_output(None, [x], x, 32, [0, 1], x)  # one weight per offset
