@@ -348,3 +348,73 @@ def test_rotation_sum_hoisted_chunks():
     """5 ciphertexts x 20 steps: chunks of 3 and 2 inputs."""
     st = Setup(11, 3, 1, 3, seed=50)
     _sum_hoisted_case(st, 3, 5, list(range(1, 21)))
+
+
+def _full_size_inputs(n_in):
+    """The hoisted and rotate-and-sum cases of the benchmark: N = 2^16,
+    level 24, K = 8, dnum = 3; n_in encrypted inputs and the rotation batch's
+    16 seeded steps, with their keys uploaded."""
+    st = Setup(16, 24, 8, 3, seed=S.master_seed(1))
+    P = st.P
+    steps = S.rotation_steps(st.seed, 16, 1, P.n_slots - 1)
+    for s_ in steps:
+        st.upload_rot(s_)
+    zs = [S.complex_slots(st.seed, P.n_slots, -1, 1, 700 + i) for i in range(n_in)]
+    cts = [st.encrypt(z, 24, ct_id=700 + i) for i, z in enumerate(zs)]
+    return st, steps, zs, cts
+
+
+def test_rotation_hoisted_full_size_sampled():
+    """he_rotate_hoisted in the launch configuration of the hoisted benchmark
+    case (4 ciphertexts x the 16 steps of the rotation batch: one chunk of 64
+    outputs, 4 raised inputs, 3 digits); two (ciphertext, step) outputs chosen
+    by seed are recomputed by the oracle, residue for residue, and decrypt to
+    the rolled slots."""
+    he = lib()
+    n_in = 4
+    st, steps, zs, cts = _full_size_inputs(n_in)
+    P = st.P
+    xs = [st.to_gpu(c) for c in cts]
+    ys = [st.empty_gpu(24) for _ in range(n_in * len(steps))]
+    he.he_rotate_hoisted(st.ctx, xs, steps, ys)
+    he.he_sync(st.ctx)
+    for o in S.choose_groups(st.seed + 11, n_in * len(steps), 2):
+        i, k = divmod(o, len(steps))
+        s_ = steps[k]
+        want = C.rotate_hoisted(cts[i], [s_], {s_: st.oracle_rot_key(s_)}, P)[0]
+        assert ys[o].level == 24 and ys[o].scale == cts[i]["scale"]
+        assert np.array_equal(st.from_gpu(ys[o]), want["c"]), (i, s_)
+        assert np.max(np.abs(C.decrypt_decode(want, st.s, P) - np.roll(zs[i], -s_))) < 1e-5
+    q = np.array(P.q, dtype=np.uint64)[None, :, None]
+    for y in ys:
+        assert np.all(st.from_gpu(y) < q)
+
+
+def test_rotation_sum_hoisted_full_size_sampled():
+    """he_rotate_sum_hoisted in the launch configuration of the rotate-and-sum
+    benchmark case (4 ciphertexts, each summed over the 16 steps of the
+    rotation batch: 64 key switches in summed and hoisted mode); one output
+    chosen by seed is recomputed by the oracle residue for residue.  Its slots
+    are within 1e-5 of the summed rolled slots of the decrypted input (the
+    key-switching noise of one ModDown); against the encoded plaintext the
+    fresh-encryption noise of the input enters 16 times, so that comparison
+    takes 1e-4."""
+    he = lib()
+    n_in = 4
+    st, steps, zs, cts = _full_size_inputs(n_in)
+    P = st.P
+    ys = [st.empty_gpu(24) for _ in range(n_in)]
+    he.he_rotate_sum_hoisted(st.ctx, [st.to_gpu(c) for c in cts], steps, ys)
+    he.he_sync(st.ctx)
+    (i,) = S.choose_groups(st.seed + 12, n_in, 1)
+    keys = {s_: st.oracle_rot_key(s_) for s_ in steps}
+    want = C.rotate_sum_hoisted(cts[i], steps, keys, P)
+    assert ys[i].level == 24 and ys[i].scale == cts[i]["scale"]
+    assert np.array_equal(st.from_gpu(ys[i]), want["c"])
+    got = C.decrypt_decode(want, st.s, P)
+    dec_in = C.decrypt_decode(cts[i], st.s, P)
+    assert np.max(np.abs(got - sum(np.roll(dec_in, -s_) for s_ in steps))) < 1e-5
+    assert np.max(np.abs(got - sum(np.roll(zs[i], -s_) for s_ in steps))) < 1e-4
+    q = np.array(P.q, dtype=np.uint64)[None, :, None]
+    for y in ys:
+        assert np.all(st.from_gpu(y) < q)
