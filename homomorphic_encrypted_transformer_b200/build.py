@@ -21,7 +21,8 @@ FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-ffp-contract=of
 
 
 def sources():
-    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cu"))
+    """CUDA sources (nvcc) and host-only C++ sources (nvcc hands them to the host compiler)."""
+    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cpp")))
 
 
 def _headers_mtime():
@@ -35,7 +36,7 @@ def build(force=False, verbose=False):
     hdr = _headers_mtime()
     objs, jobs = [], []
     for src in sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(BUILD, os.path.splitext(os.path.basename(src))[0] + ".o")
         objs.append(obj)
         if force or not os.path.exists(obj) or os.path.getmtime(obj) < max(os.path.getmtime(src), hdr):
             jobs.append((src, obj))
@@ -54,7 +55,7 @@ def build(force=False, verbose=False):
                 print("== %s\n%s" % (os.path.basename(src), log))
     if force or jobs or not os.path.exists(LIB):
         tmp = LIB + ".%d.tmp" % os.getpid()
-        cmd = [NVCC] + ARCH + ["-shared", "-o", tmp] + objs
+        cmd = [NVCC] + ARCH + ["-shared", "-o", tmp] + objs + ["-lquadmath"]
         subprocess.check_call(cmd)
         os.replace(tmp, LIB)
     return LIB

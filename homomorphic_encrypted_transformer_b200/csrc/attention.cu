@@ -47,6 +47,29 @@ static int split_offsets(he_ctx* c, const int32_t* offsets, int n_off, int n_tok
     return HE_OK;
 }
 
+// Ranges [p, p + words) of two device buffers intersect.
+static bool overlap(const uint64_t* a, size_t a_words, const uint64_t* b, size_t b_words) {
+    return a < b + b_words && b < a + a_words;
+}
+
+// Rejects outputs (each `out_words` long) that overlap one another or one of
+// the inputs (ins[i] with in_words[i] words).
+static int check_outputs(he_ctx* c, const he_ct* out, int n_out, size_t out_words,
+                         const std::vector<std::pair<const uint64_t*, size_t>>& ins, const char* what) {
+    std::vector<const uint64_t*> o(n_out);
+    for (int i = 0; i < n_out; i++) {
+        o[i] = out[i].data;
+        for (const auto& in : ins)
+            if (overlap(o[i], out_words, in.first, in.second))
+                return set_err(c, HE_EINVAL, "%s: output %d overlaps an input", what, i);
+    }
+    std::sort(o.begin(), o.end());
+    for (int i = 1; i < n_out; i++)
+        if (overlap(o[i - 1], out_words, o[i], out_words))
+            return set_err(c, HE_EINVAL, "%s: outputs overlap one another", what);
+    return HE_OK;
+}
+
 }  // namespace he
 
 using namespace he;
@@ -69,12 +92,10 @@ extern "C" int he_attention_scores(he_ctx* c, const he_ct* q, const he_ct* k, in
     if ((rc = split_offsets(c, offsets, n_off, n_tok, nz, pos, what))) return rc;
     for (int h = 1; h < d; h <<= 1)
         if ((rc = need_key(c, 2 * n_tok * h, what))) return rc;
-    for (int i = 0; i < n_off; i++) {
-        if (!s[i].data || ((uintptr_t)s[i].data & 15)) return set_err(c, HE_EINVAL, "%s: null or unaligned output", what);
-        if (s[i].data == q->data || s[i].data == k->data) return set_err(c, HE_EINVAL, "%s: output aliases an input", what);
-    }
-
     const size_t N = c->N, ctw = (size_t)2 * l * N, ctw1 = (size_t)2 * (l - 1) * N;
+    for (int i = 0; i < n_off; i++)
+        if (!s[i].data || ((uintptr_t)s[i].data & 15)) return set_err(c, HE_EINVAL, "%s: null or unaligned output", what);
+    if ((rc = check_outputs(c, s, n_off, ctw1, {{q->data, ctw}, {k->data, ctw}}, what))) return rc;
     uint64_t* pool;
     if ((rc = scratch_slot(c, 3, ctw * nz.size() + ctw1 * n_off, &pool))) return rc;
     // rot_delta(k) for the non-zero offsets, hoisted
@@ -126,10 +147,15 @@ extern "C" int he_attention_output(he_ctx* c, const he_ct* a, const he_ct* v, in
         if ((rc = ct_check(c, &a[i], what))) return rc;
         if (a[i].level != la || a[i].scale != a[0].scale)
             return set_err(c, HE_ELEVEL, "%s: mixed levels or scales among the weights", what);
-        if (out->data == a[i].data) return set_err(c, HE_EINVAL, "%s: output aliases an input", what);
     }
-    if (out->data == v->data) return set_err(c, HE_EINVAL, "%s: output aliases an input", what);
     if (la < 2 || lv < la) return set_err(c, HE_ELEVEL, "%s: weights at level %d, values at %d", what, la, lv);
+    {
+        const size_t n = c->N;
+        std::vector<std::pair<const uint64_t*, size_t>> ins;
+        for (int i = 0; i < n_off; i++) ins.push_back({a[i].data, (size_t)2 * la * n});
+        ins.push_back({v->data, (size_t)2 * lv * n});
+        if ((rc = check_outputs(c, out, 1, (size_t)2 * (la - 1) * n, ins, what))) return rc;
+    }
     if (!c->relin.d) return set_err(c, HE_ENOKEY, "%s: no relinearisation key", what);
     std::vector<int32_t> nz;
     std::vector<int> pos;

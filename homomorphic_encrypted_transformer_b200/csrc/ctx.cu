@@ -496,8 +496,15 @@ extern "C" int he_ctx_create(const he_params* prm, void* stream, he_ctx** out) {
 
     int rc = check_cuda(c, cudaGetDevice(&c->device), "cudaGetDevice");
     if (!rc) rc = build_tables(c);
-    if (!rc) rc = ntt_setup(c);
-    if (!rc) rc = elementwise_setup(c);
+    if (!rc) rc = noalloc_setup(c);
+    if (!rc) rc = check_cuda(c, cudaMalloc(&c->d_err, sizeof(int)), "error word");
+    if (!rc) rc = check_cuda(c, cudaMemset(c->d_err, 0, sizeof(int)), "error word");
+    if (!rc) rc = moddown_tc_setup(c);
+    if (!rc) {
+        // the FP64 conversion kernel unless "tc" selects the tensor-core one
+        const char* v = getenv("HE_MODDOWN_CONV");
+        c->tc_moddown = moddown_tc_available(c) && v && strcmp(v, "tc") == 0;
+    }
     if (rc) {
         fprintf(stderr, "he_ctx_create: %s\n", c->err.c_str());
         he_ctx_destroy(c);
@@ -524,6 +531,9 @@ extern "C" int he_ctx_destroy(he_ctx* c) {
     cudaFree(c->d_md_pinv);
     cudaFree(c->d_rs_inv);
     cudaFree(c->d_rs_qmod);
+    cudaFree(c->d_err);
+    cudaFree(c->d_tc_btab);
+    cudaFree(c->d_tc_tgt);
     for (auto& kv : c->rot_keys) cudaFree(kv.second.d);
     cudaFree(c->relin.d);
     for (int i = 0; i < kScratchSlots; i++) cudaFree(c->scratch[i]);
@@ -549,7 +559,15 @@ extern "C" int he_set_stream(he_ctx* c, void* s) {
 
 extern "C" int he_sync(he_ctx* c) {
     if (!c) return HE_EINVAL;
-    return check_cuda(c, cudaStreamSynchronize(c->stream), "he_sync");
+    int rc = check_cuda(c, cudaStreamSynchronize(c->stream), "he_sync");
+    if (rc || !c->d_err) return rc;
+    int e = 0;
+    if ((rc = check_cuda(c, cudaMemcpy(&e, c->d_err, sizeof(int), cudaMemcpyDeviceToHost), "he_sync"))) return rc;
+    if (e) {
+        cudaMemset(c->d_err, 0, sizeof(int));
+        return set_err(c, HE_ETIMEOUT, "he_sync: a bounded device wait gave up (its results are not valid)");
+    }
+    return HE_OK;
 }
 
 extern "C" const char* he_last_error(const he_ctx* c) { return c ? c->err.c_str() : "null context"; }

@@ -81,6 +81,11 @@ struct he_ctx {
 
     uint64_t* scratch[4] = {nullptr, nullptr, nullptr, nullptr};
     size_t scratch_words[4] = {0, 0, 0, 0};
+    uint64_t* noalloc_scratch = nullptr;  // device address of he_rescale_noalloc's fixed array
+    int* d_err = nullptr;                 // device error word: a bounded device wait gave up (he_sync reports it)
+    void* d_tc_btab = nullptr;            // tensor-core ModDown conversion: byte matrix B (moddown_tc.cu)
+    void* d_tc_tgt = nullptr;             // and its per-target recombination constants
+    bool tc_moddown = false;              // ModDown conversion on the tensor cores
     uint64_t* io_buf = nullptr;  // device staging of the host-buffer entry point
     size_t io_words = 0;
     cudaStream_t io_h2d = nullptr, io_d2h = nullptr;  // its copy streams (one per direction)
@@ -116,7 +121,6 @@ std::vector<int> prime_range(int first, int count);
 // Rows of Q_level then all of P: 0..level-1, L..L+K-1
 std::vector<int> ext_primes(const he_ctx* c, int level);
 
-int ntt_setup(he_ctx* c);
 int ntt_fwd_set(he_ctx* c, const RowSet& rs, int n_rows);
 int ntt_inv_set(he_ctx* c, const RowSet& rs, int n_rows);
 // Single passes, for callers that fuse the other pass with their own work:
@@ -180,6 +184,18 @@ int add_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector
              const std::vector<uint64_t*>& o, int lv);
 int drop_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int lin, int lv);
 
-int elementwise_setup(he_ctx* c);
+// Set-up of he_rescale_noalloc at context creation (noalloc.cu): looks up
+// the device address of its fixed scratch array on the context's device and
+// loads every kernel that entry point launches, so that its calls allocate
+// nothing, the first one included.
+int noalloc_setup(he_ctx* c);
+// ModDown base conversion as a split-integer GEMM on the tensor cores
+// (moddown_tc.cu): tables at context creation, then one launch per key switch
+// writing the same canonical residues as k_moddown_conv.
+int moddown_tc_setup(he_ctx* c);
+bool moddown_tc_available(const he_ctx* c);
+int moddown_conv_tc(he_ctx* c, const uint64_t* u, uint64_t* tmp, int n_md, int level);
+// Loads the transform kernels of the context's ring degree (cudaFuncGetAttributes).
+int ntt_preload(he_ctx* c);
 
 }  // namespace he

@@ -836,19 +836,24 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     if ((rc = ntt_inv_set(c, prs, n_md * 2 * K))) return rc;
 
     prof_begin(c, HE_PROF_MODDOWN_CONV);
-    switch (K) {
+    if (c->tc_moddown) {
+        if ((rc = moddown_conv_tc(c, u, tmp, n_md, level))) return rc;
+        c->launches--;  // counted once below
+    } else {
+        switch (K) {
 #define HE_MD_CASE(KK)                                                                                          \
     case KK:                                                                                                    \
         k_moddown_conv<KK><<<dim3(gx, 2, n_md), blk, 0, c->stream>>>(u, tmp, level, L, c->d_prime, c->d_fpmod, \
                                                                   c->d_md_pcoef, c->d_md_mat, c->d_md_negP,    \
                                                                   c->log_n);                                   \
         break;
-        HE_MD_CASE(1) HE_MD_CASE(2) HE_MD_CASE(3) HE_MD_CASE(4) HE_MD_CASE(5) HE_MD_CASE(6) HE_MD_CASE(7)
-        HE_MD_CASE(8) HE_MD_CASE(9) HE_MD_CASE(10) HE_MD_CASE(11) HE_MD_CASE(12) HE_MD_CASE(13) HE_MD_CASE(14)
-        HE_MD_CASE(15) HE_MD_CASE(16)
+            HE_MD_CASE(1) HE_MD_CASE(2) HE_MD_CASE(3) HE_MD_CASE(4) HE_MD_CASE(5) HE_MD_CASE(6) HE_MD_CASE(7)
+            HE_MD_CASE(8) HE_MD_CASE(9) HE_MD_CASE(10) HE_MD_CASE(11) HE_MD_CASE(12) HE_MD_CASE(13) HE_MD_CASE(14)
+            HE_MD_CASE(15) HE_MD_CASE(16)
 #undef HE_MD_CASE
-        default:
-            return set_err(c, HE_EINVAL, "key switch: K = %d unsupported", K);
+            default:
+                return set_err(c, HE_EINVAL, "key switch: K = %d unsupported", K);
+        }
     }
     if ((rc = lc(c, "moddown_conv"))) return rc;
     {

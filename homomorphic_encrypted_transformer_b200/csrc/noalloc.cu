@@ -16,12 +16,14 @@
 // clearing between calls.
 //
 // Host code cannot use the array's name as a device address (in host code
-// the symbol is a stand-in, not device memory), so the first call on each
-// device looks its address up with cudaGetSymbolAddress while that device is
-// current and caches it.  That first call should come before any stream
-// capture begins.
-#include <mutex>
-
+// the symbol is a stand-in, not device memory).  he_ctx_create therefore
+// looks the address up with cudaGetSymbolAddress on the context's device
+// (current during creation) and keeps it in the context.  CUDA loads a
+// module and its device arrays lazily, on first use; the lookup does that
+// load for this file, and the set-up also loads every kernel the entry point
+// launches, so the entry point's first call allocates nothing either.  A
+// context does not survive a reset of its device (cudaDeviceReset frees all
+// of its memory); contexts created after a reset look the address up again.
 #include "he_internal.h"
 
 namespace he {
@@ -44,27 +46,16 @@ __global__ void k_noalloc_combine(const uint64_t* __restrict__ in, const uint64_
 
 static __device__ __align__(256) uint64_t g_noalloc_scratch[HE_NOALLOC_SCRATCH_WORDS];
 
-static std::mutex g_noalloc_mu;
-static uint64_t* g_noalloc_ptr[kMaxDevices] = {nullptr};
-
-// Device address of the scratch array on c's device (looked up once per device).
-static int noalloc_scratch(he_ctx* c, uint64_t** out) {
-    if (c->device < 0 || c->device >= kMaxDevices)
-        return set_err(c, HE_EINVAL, "he_rescale_noalloc: device %d out of range", c->device);
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[c->device]) {
-        int prev = -1;
-        int rc = check_cuda(c, cudaGetDevice(&prev), "he_rescale_noalloc: cudaGetDevice");
-        if (rc) return rc;
-        if (prev != c->device && (rc = check_cuda(c, cudaSetDevice(c->device), "he_rescale_noalloc: cudaSetDevice")))
-            return rc;
-        void* p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (prev != c->device) cudaSetDevice(prev);
-        if ((rc = check_cuda(c, e, "he_rescale_noalloc: cudaGetSymbolAddress"))) return rc;
-        g_noalloc_ptr[c->device] = (uint64_t*)p;
-    }
-    *out = g_noalloc_ptr[c->device];
+int noalloc_setup(he_ctx* c) {
+    void* p = nullptr;
+    int rc = check_cuda(c, cudaGetSymbolAddress(&p, g_noalloc_scratch), "he_rescale_noalloc set-up: cudaGetSymbolAddress");
+    if (rc) return rc;
+    cudaFuncAttributes a;
+    rc = check_cuda(c, cudaFuncGetAttributes(&a, k_noalloc_combine), "he_rescale_noalloc set-up: combine kernel");
+    if (!rc) rc = check_cuda(c, cudaFuncGetAttributes(&a, k_rescale_lift), "he_rescale_noalloc set-up: lift kernel");
+    if (!rc) rc = ntt_preload(c);
+    if (rc) return rc;
+    c->noalloc_scratch = (uint64_t*)p;
     return HE_OK;
 }
 
@@ -88,9 +79,9 @@ extern "C" int he_rescale_noalloc(he_ctx* c, const he_ct* in, he_ct* out) {
         return set_err(c, HE_EINVAL, "he_rescale_noalloc: N = %d needs %zu scratch words, the maximum is %u", N,
                        (size_t)2 * N, (unsigned)HE_NOALLOC_SCRATCH_WORDS);
     if (c->prof_on) return set_err(c, HE_EINVAL, "he_rescale_noalloc: not available while profiling is enabled");
-    uint64_t* scratch;
-    int rc = noalloc_scratch(c, &scratch);
-    if (rc) return rc;
+    uint64_t* scratch = c->noalloc_scratch;
+    if (!scratch) return set_err(c, HE_EINVAL, "he_rescale_noalloc: context has no scratch address");
+    int rc;
     const int chunk = (int)(HE_NOALLOC_SCRATCH_WORDS / N) - 1;
     uint64_t* last = scratch;
     uint64_t* lift = scratch + N;

@@ -219,6 +219,31 @@ static int ntt_pass(he_ctx* c, const RowSet& rs, int n_rows, bool fwd, int which
     return prof_end(c, cls, bytes, half * stages, 0.5 * c->N * fp_rows(c, rs, n_rows) * stages);
 }
 
+template <int LOGN>
+static cudaError_t preload_kernels() {
+    cudaFuncAttributes a;
+    cudaError_t e = cudaFuncGetAttributes(&a, k_ntt_fwd_cols<LOGN>);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, k_ntt_fwd_rows<LOGN>);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, k_ntt_inv_rows<LOGN>);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&a, k_ntt_inv_cols<LOGN>);
+    return e;
+}
+
+int ntt_preload(he_ctx* c) {
+    cudaError_t e = cudaErrorInvalidValue;
+    switch (c->log_n) {
+        case 10: e = preload_kernels<10>(); break;
+        case 11: e = preload_kernels<11>(); break;
+        case 12: e = preload_kernels<12>(); break;
+        case 13: e = preload_kernels<13>(); break;
+        case 14: e = preload_kernels<14>(); break;
+        case 15: e = preload_kernels<15>(); break;
+        case 16: e = preload_kernels<16>(); break;
+        default: break;
+    }
+    return check_cuda(c, e, "transform kernels");
+}
+
 int ntt_fwd_set(he_ctx* c, const RowSet& rs, int n_rows) {
     int rc = ntt_pass(c, rs, n_rows, true, 0);
     return rc ? rc : ntt_pass(c, rs, n_rows, true, 1);
@@ -232,11 +257,6 @@ int ntt_inv_set(he_ctx* c, const RowSet& rs, int n_rows) {
 int ntt_fwd_cols_set(he_ctx* c, const RowSet& rs, int n_rows) { return ntt_pass(c, rs, n_rows, true, 0); }
 
 int ntt_inv_cols_set(he_ctx* c, const RowSet& rs, int n_rows) { return ntt_pass(c, rs, n_rows, false, 1); }
-
-int ntt_setup(he_ctx* c) {
-    (void)c;
-    return HE_OK;
-}
 
 }  // namespace he
 

@@ -212,11 +212,6 @@ static uint64_t int_mod(int64_t K, uint64_t q) {
     return (q - 1 - m) % q;                 // K = -(m'+1) => q - 1 - m' mod q
 }
 
-int elementwise_setup(he_ctx* c) {
-    (void)c;
-    return HE_OK;
-}
-
 static int ct_ok(he_ctx* c, const he_ct* x, const char* what) {
     if (!x || !x->data) return set_err(c, HE_EINVAL, "%s: null ciphertext", what);
     if ((uintptr_t)x->data & 15) return set_err(c, HE_EINVAL, "%s: ciphertext not 16-byte aligned", what);
@@ -530,6 +525,29 @@ extern "C" int he_keygen_upload(he_ctx* c, int kind, int32_t step, const int8_t*
     Key* slot = galois ? &c->rot_keys[galois] : &c->relin;
     if (slot->d) cudaFree(slot->d);
     *slot = key;
+    return HE_OK;
+}
+
+extern "C" int he_keygen_seeded(he_ctx* c, uint64_t seed, const int32_t* rot_steps, int n_steps, int with_relin) {
+    if (!c) return HE_EINVAL;
+    if (n_steps < 0 || (n_steps > 0 && !rot_steps)) return set_err(c, HE_EINVAL, "he_keygen_seeded: bad step list");
+    for (int i = 0; i < n_steps; i++)
+        if (galois_elt(c, rot_steps[i]) == 1)
+            return set_err(c, HE_EINVAL, "he_keygen_seeded: step %d is the identity rotation", rot_steps[i]);
+    const int N = c->N, LK = c->L + c->K, nd = he_key_digits(c);
+    std::vector<int8_t> s(N);
+    std::vector<uint64_t> a((size_t)nd * LK * N);
+    std::vector<int32_t> e((size_t)nd * N);
+    int rc = he_sample_secret(seed, c->log_n, s.data());
+    if (rc) return set_err(c, rc, "he_keygen_seeded: secret");
+    auto one = [&](int kind, int32_t step, uint64_t key_id) {
+        int r = he_sample_key_draws(seed, key_id, c->log_n, c->primes.data(), LK, nd, a.data(), e.data());
+        if (r) return set_err(c, r, "he_keygen_seeded: key draws");
+        return he_keygen_upload(c, kind, step, s.data(), a.data(), e.data());
+    };
+    for (int i = 0; i < n_steps; i++)
+        if ((rc = one(HE_KEY_ROTATION, rot_steps[i], galois_elt(c, rot_steps[i])))) return rc;
+    if (with_relin && (rc = one(HE_KEY_RELIN, 0, 2))) return rc;
     return HE_OK;
 }
 

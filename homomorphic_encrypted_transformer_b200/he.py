@@ -76,6 +76,10 @@ _sig("he_get_primes", _i, _vp, _u64p)
 _sig("he_get_psi", _i, _vp, _u64p)
 _sig("he_keygen_upload", _i, _vp, _i, ctypes.c_int32, _vp, _vp, _vp)
 _sig("he_key_download", _i, _vp, _i, ctypes.c_int32, _vp)
+_sig("he_keygen_seeded", _i, _vp, ctypes.c_uint64, _vp, _i, _i)
+_sig("he_sample_secret", _i, ctypes.c_uint64, _i, _vp)
+_sig("he_sample_key_draws", _i, ctypes.c_uint64, ctypes.c_uint64, _i, _vp, _i, _i, _vp, _vp)
+_sig("he_gaussian_cdt", _i, _vp)
 _sig("he_key_digits", _i, _vp)
 _sig("he_ntt_fwd", _i, _vp, _vp, _i, _i, _i)
 _sig("he_ntt_inv", _i, _vp, _vp, _i, _i, _i)
@@ -240,6 +244,42 @@ def he_keygen_upload(ctx, kind, step, s, a, e):
     a = np.ascontiguousarray(a, dtype=np.uint64)
     e = np.ascontiguousarray(e, dtype=np.int32)
     _check(ctx, _lib.he_keygen_upload(ctx.ptr, kind, int(step), _ptr(s), _ptr(a), _ptr(e)))
+
+
+def he_keygen_seeded(ctx, seed, rot_steps, with_relin):
+    st = np.ascontiguousarray(list(rot_steps), dtype=np.int32)
+    _check(ctx, _lib.he_keygen_seeded(ctx.ptr, int(seed), _ptr(st), len(st), 1 if with_relin else 0))
+
+
+def he_sample_secret(seed, log_n):
+    """Host-only: the ternary secret of a seed (int8[2^log_n])."""
+    out = np.empty(1 << log_n, dtype=np.int8)
+    rc = _lib.he_sample_secret(int(seed), int(log_n), _ptr(out))
+    if rc != HE_OK:
+        raise HEError(rc, "he_sample_secret: bad arguments")
+    return out
+
+
+def he_sample_key_draws(seed, key_id, log_n, primes, digits):
+    """Host-only: (a [digits][len(primes)][N] uint64, e [digits][N] int32) of one key."""
+    pr = np.ascontiguousarray(primes, dtype=np.uint64)
+    n = 1 << log_n
+    a = np.empty((digits, len(pr), n), dtype=np.uint64)
+    e = np.empty((digits, n), dtype=np.int32)
+    rc = _lib.he_sample_key_draws(int(seed), int(key_id), int(log_n), _ptr(pr), len(pr), int(digits), _ptr(a),
+                                  _ptr(e))
+    if rc != HE_OK:
+        raise HEError(rc, "he_sample_key_draws: bad arguments")
+    return a, e
+
+
+def he_gaussian_cdt():
+    """Host-only: the error sampler's 38 thresholds."""
+    out = np.empty(38, dtype=np.uint64)
+    rc = _lib.he_gaussian_cdt(_ptr(out))
+    if rc != HE_OK:
+        raise HEError(rc, "he_gaussian_cdt")
+    return [int(v) for v in out]
 
 
 def he_key_download(ctx, kind, step):

@@ -125,6 +125,44 @@ int he_get_psi(const he_ctx* ctx, uint64_t* out);
  */
 int he_keygen_upload(he_ctx* ctx, int kind, int32_t step, const int8_t* s, const uint64_t* a,
                      const int32_t* e);
+/*
+ * Key generation from a seed (host sampling, then he_keygen_upload's device
+ * computation): the secret and every key's random parts are drawn from
+ * SplitMix64 streams of `seed` by the rule below, one rotation key per
+ * entry of rot_steps (HE_EINVAL for a step whose Galois element is 1) and
+ * the relinearisation key when with_relin != 0.  The context keeps the keys;
+ * the caller keeps the seed, from which he_sample_secret gives the secret
+ * for encryption and decryption.  Synchronous.
+ *
+ * Sampling rule (the pages name only the distributions; this fixes them so
+ * that a seed determines every key):
+ *  - SplitMix64 (Steele, Lea, Flood, "Fast splittable pseudorandom number
+ *    generators", OOPSLA 2014): state += 0x9E3779B97F4A7C15, output
+ *    mix64(state); one stream per object with initial state
+ *    mix64(seed + 0x9E3779B97F4A7C15 (1 + obj)),
+ *    obj = tag 2^56 + key_id 2^24 + digit 2^8 + prime_index, where
+ *    tag 1 = the secret (other fields 0), 2 = the uniform half a of digit
+ *    `digit` of a key on prime `prime_index`, 3 = the error of digit `digit`
+ *    (prime_index 0); key_id = the Galois element 5^(step mod N/2) mod 2N of
+ *    a rotation key, 2 for the relinearisation key.
+ *  - uniform residue mod q: draws x >> (64 - bitlen(q)) until one is < q;
+ *  - ternary secret coefficient: draws x until x != 2^64 - 1, then (x mod 3) - 1;
+ *  - error coefficient: discrete Gaussian with sigma = 3.2 on [-19, 19]:
+ *    -19 + the number of thresholds T_i <= x (he_gaussian_cdt).
+ * The key itself is he_keygen_upload's: s' = sigma_k(s) or s^2,
+ * b_j = -a_j s + e_j + P [prime in digit j] s'.
+ */
+int he_keygen_seeded(he_ctx* ctx, uint64_t seed, const int32_t* rot_steps, int n_steps, int with_relin);
+/* Host only (no context, no device): the ternary secret of a seed, int8[N] (N = 2^log_n). */
+int he_sample_secret(uint64_t seed, int log_n, int8_t* s_out);
+/* Host only: the random parts of one switching key as he_keygen_seeded draws
+ * them: a uint64 [digits][n_primes][N] (uniform mod primes[r] on row r) and
+ * e int32 [digits][N].  key_id < 2^32. */
+int he_sample_key_draws(uint64_t seed, uint64_t key_id, int log_n, const uint64_t* primes, int n_primes, int digits,
+                        uint64_t* a_out, int32_t* e_out);
+/* Host only: the 38 thresholds T_i = floor(2^64 C_i) of the error sampler,
+ * C_i = P(e <= -19 + i) for the discrete Gaussian of sigma 3.2 on [-19, 19]. */
+int he_gaussian_cdt(uint64_t* out);
 /* Copies a key back in canonical residues: host uint64 [digits][2][n_q+n_p][N] (b then a). */
 int he_key_download(he_ctx* ctx, int kind, int32_t step, uint64_t* host_out);
 /* Number of key-switching digits at the top level, ceil(L / alpha). */
@@ -239,11 +277,14 @@ int he_rescale(he_ctx* ctx, he_ct* inout);
  * It calls no cudaMalloc/cudaFree and no allocating routine.  Its scratch is
  * a fixed device array of HE_NOALLOC_SCRATCH_WORDS uint64 (4.5 MiB) inside
  * libhe.so, held by every GPU that loads the library until the process exits.
- * The first call on a device looks that array's address up (do it before any
- * stream capture starts).  All calls share the array, so calls that overlap
- * on the GPU race.  N must satisfy 2N <= HE_NOALLOC_SCRATCH_WORDS (always
- * true for log_n <= 16).  out must not overlap in; it receives level-1 and
- * scale/q_{level-1}.  Returns HE_EINVAL while profiling is enabled.
+ * he_ctx_create looks that array's address up on the context's device and
+ * loads every kernel this call launches (CUDA otherwise loads them lazily,
+ * on first use), so no call allocates, the first one included.  A context
+ * does not survive cudaDeviceReset of its device.  All calls share the
+ * array, so calls that overlap on the GPU race.  N must satisfy
+ * 2N <= HE_NOALLOC_SCRATCH_WORDS (always true for log_n <= 16).  out must not
+ * overlap in; it receives level-1 and scale/q_{level-1}.  Returns HE_EINVAL
+ * while profiling is enabled.
  */
 #define HE_NOALLOC_SCRATCH_WORDS 589824u
 int he_rescale_noalloc(he_ctx* ctx, const he_ct* in, he_ct* out);
@@ -297,9 +338,11 @@ int he_pmult_accum_bsgs(he_ctx* ctx, const he_ct* x, int n_in, const uint64_t* d
  *   >= la; the rotations of v are hoisted.  Slot f*2n + t of out holds
  *   sum_i A_i[t] V[f][(t + offsets[i]) mod n] for t < n.  out at la-1,
  *   scale a.scale*v.scale/q_{la-1}.
+ * Outputs: s[i] each [2][l-1][N] words, out [2][la-1][N]; an output may not
+ * overlap another output or any input.
  * Scratch (context-owned): the rotated copies and one ciphertext per offset.
- * Errors: HE_EINVAL (shape, offsets, null, unaligned, aliasing), HE_ELEVEL,
- * HE_EDOMAIN, HE_ENOKEY; nothing is launched then.
+ * Errors: HE_EINVAL (shape, offsets, null, unaligned, overlapping
+ * buffers), HE_ELEVEL, HE_EDOMAIN, HE_ENOKEY; nothing is launched then.
  */
 int he_attention_scores(he_ctx* ctx, const he_ct* q, const he_ct* k, int n_tok, int d, const int32_t* offsets,
                         int n_off, he_ct* s);

@@ -90,3 +90,20 @@ def test_bindings_check_list_lengths_before_calling(he):
         he.he_attention_scores(None, x, x, 32, 16, [0, 1], [x])  # one output per offset
     with pytest.raises(ValueError):
         he.he_attention_output(None, [x], x, 32, [0, 1], x)  # one weight per offset
+
+
+def test_library_sampler_matches_the_oracle_sampler(he):
+    """The host sampler of he_keygen_seeded against the oracle's independent
+    implementation of the same rule: threshold table, secret, key draws."""
+    from oracle import sampler as R
+
+    assert he.he_gaussian_cdt() == R.gaussian_cdt()
+    for seed in (0, 0xAE615000, (1 << 64) - 5):
+        assert (he.he_sample_secret(seed, 12) == R.secret(seed, 1 << 12)).all()
+    P = C.Params(11, 4, 2, 2)
+    for key_id in (2, P.galois_elt(3), P.galois_elt(-1)):
+        a, e = he.he_sample_key_draws(77, key_id, 11, P.mods, 2)
+        ra, re_ = R.key_draws(77, key_id, P.mods, P.N, 2)
+        assert (a == ra).all() and (e == re_).all()
+    with pytest.raises(he.HEError):
+        he.he_sample_key_draws(1, 1 << 32, 11, P.mods, 2)  # key id beyond 32 bits

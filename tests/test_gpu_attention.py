@@ -97,3 +97,89 @@ def test_attention_errors():
     with pytest.raises(he.HEError) as ei:  # output aliases an input
         he.he_attention_output(st.ctx, [x], y, 32, [0], x)
     assert ei.value.code == he.HE_EINVAL
+    # outputs that share storage only in part: views into one buffer (keys of
+    # the feature sum present, so that only the overlap is wrong)
+    for h in (1, 2, 4, 8):
+        st.upload_rot(2 * 32 * h)
+    big = st.empty_gpu(2 * P.L)
+    half = (P.L - 1) * P.N  # less than one output's [2][L-1][N] words
+    s0 = he.Ciphertext(big.data[:2 * P.L * P.N], P.L, 1.0)
+    s1 = he.Ciphertext(big.data[half:half + 2 * P.L * P.N], P.L, 1.0)
+    with pytest.raises(he.HEError) as ei:  # two score outputs overlap
+        he.he_attention_scores(st.ctx, x, y, 32, 16, [0, 0], [s0, s1])
+    assert ei.value.code == he.HE_EINVAL
+    xin = he.Ciphertext(big.data[:2 * P.L * P.N], P.L, 2.0 ** 40)
+    xin.data[:2 * P.L * P.N].copy_(x.data[:2 * P.L * P.N])
+    part = he.Ciphertext(big.data[2 * P.L * P.N - 2 * P.N:], P.L, 1.0)  # tail of the input
+    with pytest.raises(he.HEError) as ei:  # a score output overlaps the tail of q
+        he.he_attention_scores(st.ctx, xin, y, 32, 16, [0], [part])
+    assert ei.value.code == he.HE_EINVAL
+    with pytest.raises(he.HEError) as ei:  # the output overlaps the tail of v
+        he.he_attention_output(st.ctx, [y], xin, 32, [0], part)
+    assert ei.value.code == he.HE_EINVAL
+
+
+def test_attention_head_full_size_sampled():
+    """One head in the launch configuration of the attention benchmark case:
+    N = 2^16, level 24, d = 64 features x 256 tokens, all 256 token offsets
+    (255 hoisted key rotations, 6 feature-sum rotations per offset, 256
+    exponentials, A x V over every offset).  Two offsets chosen by seed are
+    recomputed by the oracle: their scores and exponentials residue for
+    residue.  The head's output sums all 256 offsets, more than the oracle
+    recomputes in a test, so it is checked by its slots: within 1e-4 of fp64
+    arithmetic on the plaintext matrices (the encryption noise of Q, K and V
+    enters through the 64-feature sums and the 256-term output sum, about
+    1e-5; the degree-15 Taylor exponential on [-2, 0] is within 1e-7)."""
+    he = lib()
+    d, n_tok = 64, 256
+    st = Setup(16, 24, 8, 3, seed=S.master_seed(5))
+    P = st.P
+    assert d * 2 * n_tok == P.n_slots
+    Q = S.weights(st.seed, (d, n_tok), -0.25, 0.25, 1)
+    K = S.weights(st.seed, (d, n_tok), -0.25, 0.25, 2)
+    V = S.weights(st.seed, (d, n_tok), -0.25, 0.25, 3)
+    q = st.encrypt(C.attention_pack(Q, False), P.L, ct_id=0)
+    k = st.encrypt(C.attention_pack(K, True), P.L, ct_id=1)
+    v = st.encrypt(C.attention_pack(V, True), P.L, ct_id=2)
+    offsets = list(range(n_tok))
+    sum_steps = [2 * n_tok * (1 << i) for i in range(d.bit_length() - 1)]
+    for s_ in sorted(set(offsets[1:]) | set(sum_steps)):
+        st.upload_rot(s_)
+    st.upload_relin()
+    gq, gk, gv = st.to_gpu(q), st.to_gpu(k), st.to_gpu(v)
+    sc = [st.empty_gpu(P.L) for _ in offsets]
+    he.he_attention_scores(st.ctx, gq, gk, n_tok, d, offsets, sc)
+    he.he_sync(st.ctx)
+    shift = [int(C.round_half_away(np.float64(-1.0 * x.scale))) for x in sc]
+    for g, kk in zip(sc, shift):
+        he.he_add_const(st.ctx, g, kk)
+    A = [st.empty_gpu(P.L) for _ in offsets]
+    he.he_poly_eval_ps15(st.ctx, sc, EXP, C.PS_TOP_SCALE, A)
+    out = st.empty_gpu(P.L)
+    he.he_attention_output(st.ctx, A, gv, n_tok, offsets, out)
+    he.he_sync(st.ctx)
+
+    rlk = st.oracle_relin_key()
+    for o in S.choose_groups(st.seed + 13, n_tok, 2):
+        keys = {s_: st.oracle_rot_key(s_) for s_ in ([o] if o else []) + sum_steps}
+        (ws,) = C.attention_scores(q, k, n_tok, d, [o], keys, rlk, P)
+        kk = int(C.round_half_away(np.float64(-1.0 * ws["scale"])))
+        assert kk == shift[o]
+        ws = C.add_const(ws, kk, P)
+        assert sc[o].level == ws["level"] and sc[o].scale == ws["scale"]
+        assert np.array_equal(st.from_gpu(sc[o]), ws["c"]), o
+        wa = C.ps_eval_deg15(ws, EXP, rlk, P)
+        assert A[o].level == wa["level"] and A[o].scale == wa["scale"]
+        assert np.array_equal(st.from_gpu(A[o]), wa["c"]), o
+        plain = np.array([Q[:, t] @ K[:, (t + o) % n_tok] for t in range(n_tok)])
+        dec = C.decrypt_decode(wa, st.s, P).real.reshape(d, 2 * n_tok)[:, :n_tok]
+        assert np.max(np.abs(dec - np.exp(plain - 1.0)[None, :])) < 1e-4
+
+    got = C.decrypt_decode(C.make_ct(st.from_gpu(out), out.level, out.scale), st.s, P)
+    got = got.real.reshape(d, 2 * n_tok)[:, :n_tok]
+    Sc = Q.T @ K
+    want = np.zeros((d, n_tok))
+    for o in offsets:
+        idx = (np.arange(n_tok) + o) % n_tok
+        want += np.exp(Sc[np.arange(n_tok), idx] - 1.0)[None, :] * V[:, idx]
+    assert np.max(np.abs(got - want)) < 1e-4

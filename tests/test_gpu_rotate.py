@@ -418,3 +418,65 @@ def test_rotation_sum_hoisted_full_size_sampled():
     q = np.array(P.q, dtype=np.uint64)[None, :, None]
     for y in ys:
         assert np.all(st.from_gpu(y) < q)
+
+
+def test_seeded_keygen_matches_oracle():
+    """he_keygen_seeded: the library samples the secret and every key's
+    random parts from the seed on the host; the keys equal the oracle's keys
+    built from the oracle sampler's draws of the same seed, residue for
+    residue, and a rotation with them decrypts under the seed's secret."""
+    from oracle import sampler as R
+
+    he = lib()
+    P = C.Params(12, 3, 1, 3)
+    ctx = he.he_ctx_create(12, 3, 1, 3)
+    seed = 0x5EED0001
+    steps = [1, 2, -1]
+    he.he_keygen_seeded(ctx, seed, steps, True)
+    s = R.secret(seed, P.N)
+    assert (he.he_sample_secret(seed, 12) == s).all()
+    for st in steps:
+        a, e = R.key_draws(seed, P.galois_elt(st), P.mods, P.N, P.dnum)
+        b_, a_ = C.rotation_key(s, st, a, e, P)
+        got = he.he_key_download(ctx, he.HE_KEY_ROTATION, st)
+        assert np.array_equal(got[:, 0], b_) and np.array_equal(got[:, 1], a_)
+    a, e = R.key_draws(seed, 2, P.mods, P.N, P.dnum)
+    b_, a_ = C.relin_key(s, a, e, P)
+    got = he.he_key_download(ctx, he.HE_KEY_RELIN, 0)
+    assert np.array_equal(got[:, 0], b_) and np.array_equal(got[:, 1], a_)
+    # a ciphertext under the seed's secret rotates correctly with these keys
+    pa, pe = S.public_key_draws(seed, P.q, P.N)
+    pk = C.public_key(s, pa, pe, P)
+    z = S.complex_slots(seed, P.n_slots, -1, 1)
+    v, e0, e1 = S.encryption_draws(seed, 0, P.N)
+    ct = C.make_ct(C.encrypt(pk, C.encode(z, 2.0 ** 40, 3, P), v, e0, e1, 3, P), 3, 2.0 ** 40)
+    x = he.Ciphertext(torch.from_numpy(ct["c"].view(np.int64).copy()).cuda(), 3, 2.0 ** 40)
+    y = he.Ciphertext(torch.empty_like(x.data), 3, 1.0)
+    he.he_rotate(ctx, x, 2, y)
+    he.he_sync(ctx)
+    got = C.make_ct(host(y.data, (2, 3, P.N)), 3, y.scale)
+    assert np.max(np.abs(C.decrypt_decode(got, s, P) - np.roll(z, -2))) < 1e-5
+    with pytest.raises(he.HEError) as ei:  # the identity rotation has no key
+        he.he_keygen_seeded(ctx, seed, [P.n_slots], False)
+    assert ei.value.code == he.HE_EINVAL
+
+
+def test_seeded_keygen_full_size():
+    """One seeded rotation key and the relinearisation key at N = 2^16,
+    L = 24, K = 8, dnum = 3 against the oracle."""
+    from oracle import sampler as R
+
+    he = lib()
+    P = C.Params(16, 24, 8, 3)
+    ctx = he.he_ctx_create(16, 24, 8, 3)
+    seed = S.master_seed(1)
+    he.he_keygen_seeded(ctx, seed, [12345], True)
+    s = R.secret(seed, P.N)
+    a, e = R.key_draws(seed, P.galois_elt(12345), P.mods, P.N, P.dnum)
+    b_, a_ = C.rotation_key(s, 12345, a, e, P)
+    got = he.he_key_download(ctx, he.HE_KEY_ROTATION, 12345)
+    assert np.array_equal(got[:, 0], b_) and np.array_equal(got[:, 1], a_)
+    a, e = R.key_draws(seed, 2, P.mods, P.N, P.dnum)
+    b_, a_ = C.relin_key(s, a, e, P)
+    got = he.he_key_download(ctx, he.HE_KEY_RELIN, 0)
+    assert np.array_equal(got[:, 0], b_) and np.array_equal(got[:, 1], a_)
