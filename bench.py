@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="default run: the rotation-batch line only, without the other workloads' entries")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--case", default="rotation",
                     choices=["rotation", "ntt", "rot_small", "ffn128", "ffn2048", "ps15", "tiny", "hoisted",
@@ -73,18 +75,46 @@ def workload_inputs(master, primes_q, n_cts):
 
 
 class ClockSampler:
-    """nvidia-smi clocks during the timed region (SM MHz and throttle reasons)."""
+    """SM clocks and clock-event reasons of this rank's GPU during the timed
+    region, sampled every 20 ms through NVML (query only; nothing is set),
+    or every 200 ms through nvidia-smi when NVML is unavailable.  The GPU is
+    found by its PCI bus id, so the sample follows CUDA's device numbering
+    whatever CUDA_VISIBLE_DEVICES holds."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.samples = []  # (sm MHz, max MHz, reasons bitmask) from NVML
+        self.nvml = None
+        self.stop_flag = threading.Event()
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+
+        pynvml.nvmlInit()
+        pr = torch.cuda.get_device_properties(self.gpu)
+        try:
+            bus = "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
 
     def start(self):
+        try:
+            nv, h = self._nvml_handle()
+            self.nvml = (nv, h)
+            self.t = threading.Thread(target=self._poll, daemon=True)
+            self.t.start()
+            return
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
                                           "--format=csv,noheader,nounits", "-lms", "200"],
@@ -94,13 +124,37 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
+    def _poll(self):
+        nv, h = self.nvml
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+            except Exception:
+                pass
+            self.stop_flag.wait(0.02)
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
     def stop(self):
+        if self.nvml:
+            self.stop_flag.set()
+            self.t.join(timeout=2)
+            nv = self.nvml[0]
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            sm = [x[0] for x in self.samples]
+            reasons = sorted({nm for x in self.samples for nm, b in bits.items() if x[2] & b})
+            return {"sm_mhz": float(np.median(sm)) if sm else None,
+                    "sm_max_mhz": float(self.samples[-1][1]) if self.samples else None,
+                    "reasons": reasons, "samples": len(sm), "source": "nvml, 20 ms"}
         if not self.proc:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -108,7 +162,6 @@ class ClockSampler:
             self.proc.kill()
         self.t.join(timeout=2)
         sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 8:
@@ -118,11 +171,11 @@ class ClockSampler:
                 mx = float(parts[1])
             except ValueError:
                 continue
-            for nm, v in zip(names, parts[4:8]):
+            for nm, v in zip(self.NAMES, parts[4:8]):
                 if v.lower() == "active":
                     reasons.add(nm)
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi, 200 ms"}
 
 
 # ------------------------------------------------------------ cpu baseline
@@ -145,52 +198,97 @@ def rank_seed(master, rank):
     return master + 7919 * rank
 
 
-def cpu_baseline(seconds):
-    """The oracle, as it stands, rotating full-size ciphertexts of this workload
-    on the host cores until about `seconds` of rotation work has run."""
-    from oracle import ckks as C
+class OracleRotations:
+    """The oracle, as it stands, rotating full-size ciphertexts of the
+    rotation-batch workload (uniform-residue ciphertexts at level 24, the
+    workload's seeded steps and keys).  Keys are generated on first use,
+    outside every timing."""
 
-    master = S.master_seed(1)
-    P = C.Params(LOG_N, L, K, DNUM)
-    steps, ct_steps = workload_inputs(master, P.q, N_CTS)
-    s = S.secret(master, P.N)
-    uni = S.uniform_residues(master, "ct_residues", P.q, P.N, lead=(4, 2))
-    keys = {}
-    done, t_rot, i = 0, 0.0, 0
-    while (t_rot < seconds and done < 64) or done < 2:
-        st = ct_steps[i % N_CTS]
-        if st not in keys:
-            k = P.galois_elt(st)
-            a, e = S.key_draws(master, k, P.mods, P.N, P.dnum)
-            keys[st] = C.rotation_key(s, st, a, e, P)
-        ct = C.make_ct(uni[i % 4], LEVEL, 2.0 ** 40)
+    def __init__(self):
+        from oracle import ckks as C
+
+        self.C = C
+        master = S.master_seed(1)
+        self.master = master
+        self.P = C.Params(LOG_N, L, K, DNUM)
+        _, self.ct_steps = workload_inputs(master, self.P.q, N_CTS)
+        self.s = S.secret(master, self.P.N)
+        self.uni = S.uniform_residues(master, "ct_residues", self.P.q, self.P.N, lead=(4, 2))
+        self.keys = {}
+
+    def key(self, st):
+        if st not in self.keys:
+            a, e = S.key_draws(self.master, self.P.galois_elt(st), self.P.mods, self.P.N, self.P.dnum)
+            self.keys[st] = self.C.rotation_key(self.s, st, a, e, self.P)
+        return self.keys[st]
+
+    def rotate(self, i):
+        """Rotation i of the batch (ciphertext i mod 64 with its step); returns seconds."""
+        st = self.ct_steps[i % N_CTS]
+        key = self.key(st)
+        ct = self.C.make_ct(self.uni[i % 4], LEVEL, 2.0 ** 40)
         t0 = time.perf_counter()
-        C.rotate(ct, st, keys[st], P)
-        t_rot += time.perf_counter() - t0
+        self.C.rotate(ct, st, key, self.P)
+        return time.perf_counter() - t0
+
+
+def cpu_baseline(seconds):
+    """The oracle rotating full-size ciphertexts of this workload on the host
+    cores until about `seconds` of rotation work has run (at least 2)."""
+    o = OracleRotations()
+    done, t_rot = 0, 0.0
+    while (t_rot < seconds and done < 64) or done < 2:
+        t_rot += o.rotate(done)
         done += 1
-        i += 1
-    return {"value": done / t_rot, "unit": "rotations/s", "cores": C.n_threads(), "kind": "oracle",
+    return {"value": done / t_rot, "unit": "rotations/s", "cores": o.C.n_threads(), "kind": "oracle",
             "sample": "%d full-size rotations (N=2^16, level 24, K=8, dnum=3) of uniform-residue ciphertexts, "
                       "key generation excluded; oracle threads over limbs" % done}
 
 
+def line_config(world):
+    """The `config` of the rotation-batch line, identical on both arms."""
+    return dict(WORKLOAD, parallelism="replicas%d" % world if world > 1 else "single")
+
+
+# rotations of the batch that one step of the reference arm times
+REF_ROTATIONS_PER_STEP = 2
+
+
 def run_reference(args, rank, world):
+    """The reference arm: the oracle on the host cores, rank 0 only.  Each
+    step is a bounded sample of the workload, REF_ROTATIONS_PER_STEP of its 64
+    rotations (in batch order), timed with the host clock; value is the
+    rotations timed over the time they took, ms_per_step the time of one
+    such step."""
     if rank != 0:
         return
-    steps = args.steps
     t0 = time.perf_counter()
-    per = []
-    for _ in range(args.warmup + steps):
-        r = cpu_baseline(max(1.0, args.cpu_seconds / max(1, steps + args.warmup)))
-        per.append(r)
-    timed = per[args.warmup:]
-    v = float(np.mean([r["value"] for r in timed]))
+    o = OracleRotations()
+    R = REF_ROTATIONS_PER_STEP
+    for i in range(R * (args.warmup + args.steps)):  # keys outside the timing
+        o.key(o.ct_steps[i % N_CTS])
+    i = 0
+    for _ in range(args.warmup):
+        for _ in range(R):
+            o.rotate(i)
+            i += 1
+    t_steps = []
+    for _ in range(args.steps):
+        t = 0.0
+        for _ in range(R):
+            t += o.rotate(i)
+            i += 1
+        t_steps.append(t)
+    total = float(sum(t_steps))
+    v = R * args.steps / total
+    sample = ("%d full-size rotations of the batch per step (N=2^16, level 24, K=8, dnum=3), uniform-residue "
+              "ciphertexts, key generation excluded; oracle threads over limbs" % R)
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "rotations/s", "n_gpus": args.gpus,
-            "steps": steps, "warmup": args.warmup, "ms_per_step": 1000.0 * 64 / v, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "u64", "data": "synthetic",
-            "config": WORKLOAD,
-            "cpu_baseline": {"value": v, "unit": "rotations/s", "cores": timed[0]["cores"], "kind": "oracle",
-                             "sample": timed[0]["sample"] + " (per step)"},
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * total / args.steps,
+            "rotations_per_step": R, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "u64", "data": "synthetic", "config": line_config(world),
+            "cpu_baseline": {"value": v, "unit": "rotations/s", "cores": o.C.n_threads(), "kind": "oracle",
+                             "sample": sample},
             "e2e": {"value": v, "unit": "rotations/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "wall_s": time.perf_counter() - t0}
     print(json.dumps(line), flush=True)
@@ -198,32 +296,73 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------------------ native
 
-def run_ntt_case(args, local_rank):
-    """Kernel case for profiler captures: forward and inverse NTT of 512
-    limbs of 2^16 words (256 MiB, larger than L2), all 32 primes cycled."""
+def ntt_case(steps, warmup, local_rank, probes=None):
+    """The NTT sub-metric: forward and inverse NTT of 512 limbs of 2^16 words
+    (256 MiB, larger than L2; 16 polynomials x all 32 primes), device-timed
+    per pass.  Butterflies/s per pass against two ceilings: the mixed one
+    (integer-path butterflies at the integer probe's rate plus FP64-path
+    butterflies at the FP64 probe's rate) and the integer probe's rate alone
+    (every butterfly as a 64-bit Shoup product on the integer pipe)."""
     import torch
 
     from homomorphic_encrypted_transformer_b200 import he
 
     torch.cuda.set_device(local_rank)
-    ctx = he.he_ctx_create(LOG_N, L, K, DNUM, stream=torch.cuda.current_stream())
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    ctx = he.he_ctx_create(LOG_N, L, K, DNUM, stream=stream)
     n_polys, n_limbs = 16, L + K
     h = S.uniform_residues(S.master_seed(1), "ntt_residues", ctx.primes, ctx.N, lead=(n_polys,))
-    d = torch.from_numpy(h.view(np.int64)).cuda()
-    for i in range(args.warmup + args.steps):
-        if i == args.warmup:
-            he.he_profile_enable(ctx, True)
+    d = torch.from_numpy(h.view(np.int64)).to(dev)
+    if probes is None:
+        probes = run_probes(he, ctx, dev, stream)
+    copy_gbs, int_s, fp_s = probes
+    pk, pk_kind = peaks()
+    hbm_peak = float(pk.get("hbm_gbs", 6650.0))
+
+    def step():
         he.he_ntt_fwd(ctx, d, n_polys, n_limbs, 0)
         he.he_ntt_inv(ctx, d, n_polys, n_limbs, 0)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    clk = clocks.stop()
+    he.he_profile_enable(ctx, True)
+    for _ in range(steps):
+        step()
     torch.cuda.synchronize()
     ok = np.array_equal(d.cpu().numpy().view(np.uint64), h)
-    res = {"case": "ntt", "rows": n_polys * n_limbs, "roundtrip_ok": bool(ok)}
-    for name in ("ntt_fwd_cols", "ntt_fwd_rows", "ntt_inv_rows", "ntt_inv_cols"):
-        ms, n, _, mults = he.he_profile_read(ctx, he.PROF[name])
-        if n:
-            res[name + "_us"] = round(1e3 * ms / n, 2)
-            res[name + "_Gbfly_s"] = round(mults / (ms * 1e-3) / 1e9, 1)
-    print(json.dumps(res))
+    prof = {name: he.he_profile_read(ctx, he.PROF[name]) + (he.he_profile_read_fp(ctx, he.PROF[name]),)
+            for name in ("ntt_fwd_cols", "ntt_fwd_rows", "ntt_inv_rows", "ntt_inv_cols")}
+    he.he_profile_enable(ctx, False)
+    passes = {}
+    for name, (pms, n, nbytes, mults, mults_fp) in prof.items():
+        if not n:
+            continue
+        t = pms * 1e-3
+        bfly_s = mults / t
+        mixed = mults / ((mults - mults_fp) / int_s + mults_fp / fp_s)
+        passes[name] = {"us_per_launch": 1e3 * pms / n, "bfly_per_s": bfly_s, "fp64_share": mults_fp / mults,
+                        "frac_of_mixed_ceiling": bfly_s / mixed, "frac_of_int_probe": bfly_s / int_s,
+                        "hbm_frac": nbytes / t / 1e9 / hbm_peak}
+    dom = max(prof, key=lambda k: prof[k][0])
+    bfly_step = sum(v[3] for v in prof.values()) / steps
+    return {"case": "ntt", "metric": "NTT butterflies/s (N=2^16, 512 limbs: 16 polynomials x 32 primes, forward "
+                                     "and inverse)", "value": bfly_step * steps / (ms * 1e-3), "unit": "butterflies/s",
+            "ms_per_step": ms / steps, "steps": steps, "warmup": warmup, "roundtrip_ok": bool(ok),
+            "roofline": roofline_for(dom, prof[dom], int_s, fp_s, hbm_peak, pk_kind), "passes": passes,
+            "probes": {"int_shoup_modmul_per_s": int_s, "fp64_modmul_per_s": fp_s, "copy_gbs": copy_gbs},
+            "clocks": clk, "l2": "256 MiB of limbs per transform (larger than L2)"}
 
 
 def run_rot_small_case(args, local_rank):
@@ -394,8 +533,8 @@ def workload_cpu_baseline(case, seconds):
                       % (n_pm, rot, pms, n_groups * f["n_out"], per_product)}
 
 
-def run_workload_case(args, local_rank):
-    """Throughput of the other workloads on one GPU, one JSON line each:
+def workload_case(case, n_steps, n_warmup, cpu_seconds, local_rank, probes=None, with_cpu=True):
+    """Throughput of one of the other workloads on one GPU, as a dict:
     ffn128 (FFN1 768->3072, 128 tokens: 3 x 12 blocks by BSGS at level 12),
     ffn2048 (the same product for 16 token groups sharing the weights),
     ps15 (degree-15 Paterson-Stockmeyer on 64 ciphertexts from level 24),
@@ -415,7 +554,6 @@ def run_workload_case(args, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream()
-    case = args.case
     widx = {"tiny": 0, "hoisted": 1, "rotsum": 1, "ffn128": 2, "ffn2048": 3, "ps15": 4, "attention": 5}[case]
     master = S.master_seed(widx)
     gen = torch.Generator(device=dev)
@@ -549,10 +687,10 @@ def run_workload_case(args, local_rank):
         metric, unit, per_step = "tiny-config operation sequences/s (N=2^12)", "sequences/s", 1
         cfg = {"workload": case, "N": N, "ops": "NTT round trip, 3 rotations, 1 HMult-relin-rescale"}
 
-    for _ in range(args.warmup):
+    for _ in range(n_warmup):
         step()
     torch.cuda.synchronize()
-    copy_gbs, int_modmul_s, fp_modmul_s = run_probes(he, ctx, dev, stream)
+    copy_gbs, int_modmul_s, fp_modmul_s = probes if probes is not None else run_probes(he, ctx, dev, stream)
     pk, pk_kind = peaks()
     hbm_peak = float(pk.get("hbm_gbs", 6650.0))
     clocks = ClockSampler(local_rank)
@@ -560,33 +698,62 @@ def run_workload_case(args, local_rank):
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     t0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(n_steps):
         step()
     t1.record(stream)
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1)
     clk = clocks.stop()
     he.he_profile_enable(ctx, True)
-    for _ in range(args.steps):
+    for _ in range(n_steps):
         step()
     prof = {name: he.he_profile_read(ctx, cls) + (he.he_profile_read_fp(ctx, cls),) for name, cls in he.PROF.items()}
     he.he_profile_enable(ctx, False)
     dom = max(prof, key=lambda k: prof[k][0])
-    alu_ideal = sum(((v[3] - v[4]) / int_modmul_s + v[4] / fp_modmul_s) * 1e3 for v in prof.values()) / args.steps
-    line = {"case": case, "metric": metric, "value": per_step * args.steps / (ms * 1e-3), "unit": unit,
-            "ms_per_step": ms / args.steps, "steps": args.steps, "warmup": args.warmup, "n_gpus": 1,
+    alu_ideal = sum(((v[3] - v[4]) / int_modmul_s + v[4] / fp_modmul_s) * 1e3 for v in prof.values()) / n_steps
+    line = {"case": case, "metric": metric, "value": per_step * n_steps / (ms * 1e-3), "unit": unit,
+            "ms_per_step": ms / n_steps, "steps": n_steps, "warmup": n_warmup, "n_gpus": 1,
             "higher_is_better": True, "dtype": "u64", "data": "synthetic (seeded uniform residues, seeded keys)",
             "config": cfg, "roofline": roofline_for(dom, prof[dom], int_modmul_s, fp_modmul_s, hbm_peak, pk_kind),
             "alu_ideal_ms_per_step": alu_ideal,
-            "kernel_ms_per_step": {k: round(v[0] / args.steps, 4) for k, v in prof.items() if v[1]},
+            "kernel_ms_per_step": {k: round(v[0] / n_steps, 4) for k, v in prof.items() if v[1]},
             "kernel_roofline_frac": {k: round(roofline_for(k, v, int_modmul_s, fp_modmul_s, hbm_peak,
                                                            pk_kind)["frac"], 3) for k, v in prof.items() if v[1]},
             "probes": {"copy_gbs": copy_gbs, "int_shoup_modmul_per_s": int_modmul_s,
                        "fp64_modmul_per_s": fp_modmul_s},
             "clocks": clk}
-    if not args.no_cpu_baseline:
-        line["cpu_baseline"] = workload_cpu_baseline(case, args.cpu_seconds)
-    print(json.dumps(line), flush=True)
+    if with_cpu:
+        line["cpu_baseline"] = workload_cpu_baseline(case, cpu_seconds)
+    return line
+
+
+# the other workloads of the default run: (warm-up steps, timed steps) each
+WORKLOAD_STEPS = {"ntt": (3, 10), "tiny": (3, 20), "hoisted": (3, 10), "rotsum": (3, 10), "ps15": (3, 5),
+                  "ffn128": (3, 4), "ffn2048": (3, 2), "attention": (3, 2)}
+# seconds of oracle work per workload's cpu_baseline in the default run
+WORKLOAD_CPU_SECONDS = 3.0
+
+
+def all_workloads(local_rank, probes):
+    """Every other workload, one after the other in this process, as
+    {case: dict}; each frees its device memory before the next."""
+    import gc
+
+    import torch
+
+    out = {}
+    for case, (w, k) in WORKLOAD_STEPS.items():
+        t0 = time.perf_counter()
+        if case == "ntt":
+            r = ntt_case(k, w, local_rank, probes)
+        else:
+            r = workload_case(case, k, w, WORKLOAD_CPU_SECONDS, local_rank, probes)
+        r["wall_s"] = time.perf_counter() - t0
+        out[case] = r
+        gc.collect()
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_probes(he, ctx, dev, stream):
@@ -709,7 +876,7 @@ def run_native(args, rank, world, local_rank):
     (e2e_s,) = max_over_ranks([e2e_s], world, dev)
 
     if rank != 0:
-        return
+        return None
     total_rot = N_CTS * args.steps * world
     value = total_rot / (ms_plain * 1e-3)
     pk, pk_kind = peaks()
@@ -728,7 +895,7 @@ def run_native(args, rank, world, local_rank):
     line = {"metric": METRIC, "value": value, "unit": "rotations/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_plain / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u64", "data": "synthetic",
-            "config": dict(WORKLOAD, parallelism="replicas%d" % world if world > 1 else "single"),
+            "config": line_config(world),
             "hbm_roofline_frac_of_step": hbm_frac_step,
             "alu_ideal_ms_per_step": alu_ideal_ms,
             "alu_roofline_frac_of_step": alu_ideal_ms / (ms_plain / args.steps),
@@ -747,17 +914,44 @@ def run_native(args, rank, world, local_rank):
                     "h2d_bytes_per_step": int(h_in.nbytes), "d2h_bytes_per_step": int(h_in.nbytes)}}
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
-    print(json.dumps(line), flush=True)
+    line["_probes"] = (copy_gbs, int_modmul_s, fp_modmul_s)
+    return line
 
 
-# ncu dram bytes (read + write) over algorithmic bytes per launch, per kernel
-# class, from the committed capture of that kernel (profiles/
-# ntt_passes_n65536_512limbs_full.md: 512 limbs, 268.4 MB each way).  Reads
-# grow in proportion to the limbs a launch transforms; the small case leaves
-# some written lines in L2 at its end, so the ratio slightly undercounts
-# writes.  Remove an entry when its kernel changes.
-NCU_TRAFFIC_RATIO = {"ntt_fwd_cols": (268.57344 + 220.00768) / 536.870912,
-                     "ntt_inv_cols": (268.57728 + 217.766912) / 536.870912}
+# ncu DRAM bytes (read + write) of one launch over that launch's algorithmic
+# bytes, per kernel class, from one capture of the kernel.  `sources` are the
+# files the kernel is built from and `sha256` their digest (source_digest)
+# when the counters were taken: a ratio whose sources have changed since is
+# not used, and `traffic` is then null.  Reads grow in proportion to the limbs
+# a launch transforms; a small capture leaves some written lines in L2 at its
+# end, so the ratio slightly undercounts writes.
+NCU_TRAFFIC = {}
+
+
+def source_digest(files):
+    """sha256 over the named repository files (path and contents, in order)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in files:
+        h.update(f.encode())
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def traffic_ratio(name, table=None):
+    """The stored ncu traffic ratio of a kernel class, or None when there is
+    none or its sources changed after the capture."""
+    e = (NCU_TRAFFIC if table is None else table).get(name)
+    if not e:
+        return None
+    try:
+        if source_digest(e["sources"]) != e["sha256"]:
+            return None
+    except OSError:
+        return None
+    return e["ratio"]
 
 
 def roofline_for(name, prof_entry, int_modmul_s, fp_modmul_s, hbm_peak, pk_kind):
@@ -774,7 +968,8 @@ def roofline_for(name, prof_entry, int_modmul_s, fp_modmul_s, hbm_peak, pk_kind)
     b, m, m_fp = nbytes / launches, mults / launches, mults_fp / launches
     t_hbm = b / (hbm_peak * 1e9)
     t_alu = (m - m_fp) / int_modmul_s + (m_fp / fp_modmul_s if fp_modmul_s > 0 else 0.0)
-    traffic = NCU_TRAFFIC_RATIO[name] * b if name in NCU_TRAFFIC_RATIO else None
+    ratio = traffic_ratio(name)
+    traffic = ratio * b if ratio is not None else None
     if t_hbm >= t_alu:
         ach = b / t / 1e9
         return {"kernel": name, "bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
@@ -811,13 +1006,21 @@ def main():
         if args.impl == "reference":
             run_reference(args, rank, world)
         elif args.case == "ntt":
-            run_ntt_case(args, local_rank)
+            print(json.dumps(ntt_case(args.steps, args.warmup, local_rank)), flush=True)
         elif args.case == "rot_small":
             run_rot_small_case(args, local_rank)
         elif args.case in ("ffn128", "ffn2048", "ps15", "tiny", "hoisted", "rotsum", "attention"):
-            run_workload_case(args, local_rank)
+            print(json.dumps(workload_case(args.case, args.steps, args.warmup, args.cpu_seconds, local_rank,
+                                           with_cpu=not args.no_cpu_baseline)), flush=True)
         else:
-            run_native(args, rank, world, local_rank)
+            line = run_native(args, rank, world, local_rank)
+            if line is not None:
+                probes = line.pop("_probes")
+                # the other workloads on one GPU (the scaling runs time the
+                # rotation batch alone)
+                if world == 1 and not args.no_workloads:
+                    line["workloads"] = all_workloads(local_rank, probes)
+                print(json.dumps(line), flush=True)
     finally:
         if world > 1:
             import torch.distributed as dist

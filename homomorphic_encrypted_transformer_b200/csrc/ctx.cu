@@ -495,6 +495,8 @@ extern "C" int he_ctx_create(const he_params* prm, void* stream, he_ctx** out) {
     c->psi = psi;
 
     int rc = check_cuda(c, cudaGetDevice(&c->device), "cudaGetDevice");
+    if (!rc) rc = check_cuda(c, cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device),
+                             "multiprocessor count");
     if (!rc) rc = build_tables(c);
     if (!rc) rc = noalloc_setup(c);
     if (!rc) rc = check_cuda(c, cudaMalloc(&c->d_err, sizeof(int)), "error word");

@@ -156,25 +156,32 @@ __device__ __forceinline__ uint64_t tc_combine_int(const uint32_t (&v)[16], cons
     return add_mod(r, reduce64(w, p), t.q);
 }
 
-// Grid (N / 128, 2, outputs); 128 threads, thread = coefficient, warp w reads
-// tensor-memory lanes 32 w .. 32 w + 31.
-__global__ void __launch_bounds__(kTcM) k_moddown_conv_tc(const uint64_t* __restrict__ u, uint64_t* __restrict__ tmp,
-                                                         int level, int L, int K, const DevPrime* __restrict__ pr,
-                                                         const ulonglong2* __restrict__ pcoef,
-                                                         const uint8_t* __restrict__ btab,
-                                                         const TcTarget* __restrict__ tcon, int* __restrict__ err,
-                                                         int logn) {
+// Persistent: each CTA loads the byte matrix B and the target constants
+// once, then loops over work items (128-coefficient tile, polynomial,
+// output).  256 threads: for the staging, thread t takes coefficient t % 128
+// and sources 4 (t / 128) .. +3; in the epilogue warp w reads tensor-memory
+// lanes 32 (w % 4) .. +31 (its coefficients) and recombines the targets of
+// its half, t = w / 4 (mod 2), two targets' columns loaded per wait.
+constexpr int kTcThreads = 256;
+
+__global__ void __launch_bounds__(kTcThreads) k_moddown_conv_tc(const uint64_t* __restrict__ u,
+                                                               uint64_t* __restrict__ tmp, int level, int L, int K,
+                                                               int n_md, const DevPrime* __restrict__ pr,
+                                                               const ulonglong2* __restrict__ pcoef,
+                                                               const uint8_t* __restrict__ btab,
+                                                               const TcTarget* __restrict__ tcon,
+                                                               int* __restrict__ err, int logn) {
     __shared__ __align__(1024) uint8_t sA[kTcM * kTcK];
     extern __shared__ __align__(1024) uint8_t dyn[];
     uint8_t* sB = dyn;  // [level x 16 rows][64 bytes], K-major interleaved
     TcTarget* sT = reinterpret_cast<TcTarget*>(dyn + (size_t)level * kTcCols * kTcK);
     __shared__ uint64_t mbar;
     __shared__ uint32_t tmem_base;
+    __shared__ uint32_t s_neg[2][kTcM];
     const int N = 1 << logn;
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int poly = blockIdx.y, i = blockIdx.z;
-    const int c = blockIdx.x * kTcM + tid;
     const int n_rows = level + K;
+    const int tiles = N / kTcM, items = tiles * 2 * n_md;
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base)),
@@ -186,60 +193,86 @@ __global__ void __launch_bounds__(kTcM) k_moddown_conv_tc(const uint64_t* __rest
         mbar_init(&mbar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // B rows of the level's targets and their constants
     {
         const uint4* src = reinterpret_cast<const uint4*>(btab);
         uint4* dst = reinterpret_cast<uint4*>(sB);
-        for (int idx = tid; idx < level * kTcCols * kTcK / 16; idx += kTcM) dst[idx] = src[idx];
-        for (int r = tid; r < level; r += kTcM) sT[r] = tcon[r];
+        for (int idx = tid; idx < level * kTcCols * kTcK / 16; idx += kTcThreads) dst[idx] = src[idx];
+        for (int r = tid; r < level; r += kTcThreads) sT[r] = tcon[r];
     }
-    // A: y_k of this coefficient, and the number of negative centred terms
-    uint32_t n_neg = 0;
-    {
-        const uint64_t* x = u + (((size_t)i * 2 + poly) * n_rows + level) * N + c;
-        for (int k = 0; k < K; k++) {
-            const uint64_t p = pr[L + k].q;
-            const ulonglong2 w = pcoef[k];
-            const uint64_t y = mul_shoup(x[(size_t)k * N], w.x, w.y, p);
-            n_neg += y > (p >> 1) ? 1u : 0u;
-            *reinterpret_cast<uint64_t*>(sA + umma_off(tid, k >> 1) + (k & 1) * 8) = y;
-        }
-        for (int k = K; k < 8; k++) *reinterpret_cast<uint64_t*>(sA + umma_off(tid, k >> 1) + (k & 1) * 8) = 0;
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // stores visible to the tensor cores
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = tmem_base;
-    const uint32_t lane_addr = tbase + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_addr = tbase + ((uint32_t)((warp & 3) * 32) << 16);
+    const int half = warp >> 2, row = tid & (kTcM - 1), shalf = tid / kTcM;
+    uint32_t phase = 0;
     bool ok = true;
-    uint64_t* out = tmp + (((size_t)i * 2 + poly) * level) * N + c;
-    const int rounds = (level + kTcTgtRound - 1) / kTcTgtRound;
-    for (int rd = 0; rd < rounds; rd++) {
-        const int r0 = rd * kTcTgtRound, nt = min(kTcTgtRound, level - r0);
-        if (tid == 0 && ok) {
-            const uint32_t idesc = umma_idesc_u8(kTcM, nt * kTcCols);
-            for (int ks = 0; ks < 2; ks++) {
-                const uint64_t ad = umma_desc(smem_u32(sA) + ks * 2 * 128, 128, 512);
-                const uint64_t bd = umma_desc(smem_u32(sB) + (r0 * kTcCols / 8) * 512 + ks * 2 * 128, 128, 512);
-                mma_i8(tbase, ad, bd, idesc, ks);
+    for (int it = blockIdx.x; it < items && ok; it += gridDim.x) {
+        const int tile = it % tiles, rest = it / tiles, poly = rest & 1, i = rest >> 1;
+        // A: sources 4 shalf .. 4 shalf + 3 of coefficient `row`
+        {
+            const int c = tile * kTcM + row;
+            const uint64_t* x = u + (((size_t)i * 2 + poly) * n_rows + level) * N + c;
+            uint32_t neg = 0;
+#pragma unroll
+            for (int kk = 0; kk < 4; kk++) {
+                const int k = 4 * shalf + kk;
+                uint64_t y = 0;
+                if (k < K) {
+                    const uint64_t p = pr[L + k].q;
+                    const ulonglong2 w = pcoef[k];
+                    y = mul_shoup(x[(size_t)k * N], w.x, w.y, p);
+                    neg += y > (p >> 1) ? 1u : 0u;
+                }
+                *reinterpret_cast<uint64_t*>(sA + umma_off(row, k >> 1) + (k & 1) * 8) = y;
             }
-            mma_commit(&mbar);
+            s_neg[shalf][row] = neg;
         }
-        ok = ok && mbar_wait(&mbar, rd & 1);
-        tc_fence_after();
-        if (ok) {
-            for (int t = 0; t < nt; t++) {
-                uint32_t v[16];
-                tmem_ld16(lane_addr + t * kTcCols, v);
-                tmem_ld_wait();
-                const TcTarget& T = sT[r0 + t];
-                out[(size_t)(r0 + t) * N] = T.use_int ? tc_combine_int(v, T, n_neg) : d2u(tc_combine_fp(v, T, n_neg));
-            }
-        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // stores visible to the tensor cores
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        const uint32_t n_neg = s_neg[0][(warp & 3) * 32 + (tid & 31)] + s_neg[1][(warp & 3) * 32 + (tid & 31)];
+        uint64_t* out = tmp + (((size_t)i * 2 + poly) * level) * N + tile * kTcM + (warp & 3) * 32 + (tid & 31);
+        const int rounds = (level + kTcTgtRound - 1) / kTcTgtRound;
+        for (int rd = 0; rd < rounds; rd++) {
+            const int r0 = rd * kTcTgtRound, nt = min(kTcTgtRound, level - r0);
+            if (tid == 0) {
+                const uint32_t idesc = umma_idesc_u8(kTcM, nt * kTcCols);
+                for (int ks = 0; ks < 2; ks++) {
+                    const uint64_t ad = umma_desc(smem_u32(sA) + ks * 2 * 128, 128, 512);
+                    const uint64_t bd = umma_desc(smem_u32(sB) + (r0 * kTcCols / 8) * 512 + ks * 2 * 128, 128, 512);
+                    mma_i8(tbase, ad, bd, idesc, ks);
+                }
+                mma_commit(&mbar);
+            }
+            ok = mbar_wait(&mbar, phase);
+            phase ^= 1;
+            tc_fence_after();
+            if (ok) {
+                // this half's targets of the round: t = half, half + 2, ...
+                for (int t = half; t < nt; t += 4) {
+                    uint32_t v[16], w2[16];
+                    const bool two = t + 2 < nt;
+                    tmem_ld16(lane_addr + t * kTcCols, v);
+                    if (two) tmem_ld16(lane_addr + (t + 2) * kTcCols, w2);
+                    tmem_ld_wait();
+                    const TcTarget& T = sT[r0 + t];
+                    out[(size_t)(r0 + t) * N] =
+                        T.use_int ? tc_combine_int(v, T, n_neg) : d2u(tc_combine_fp(v, T, n_neg));
+                    if (two) {
+                        const TcTarget& T2 = sT[r0 + t + 2];
+                        out[(size_t)(r0 + t + 2) * N] =
+                            T2.use_int ? tc_combine_int(w2, T2, n_neg) : d2u(tc_combine_fp(w2, T2, n_neg));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncthreads();  // tensor memory and A free again
+            tc_fence_after();
+            ok = __syncthreads_and(ok);
+            if (!ok) break;
+        }
     }
     if (!ok && tid == 0) atomicExch(err, 1);
     __syncthreads();
@@ -307,9 +340,12 @@ int moddown_conv_tc(he_ctx* c, const uint64_t* u, uint64_t* tmp, int n_md, int l
     const size_t smem = (size_t)level * kTcCols * kTcK + (size_t)level * sizeof(TcTarget);
     cudaFuncSetAttribute(k_moddown_conv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)((size_t)kTcMaxTargets * (kTcCols * kTcK + sizeof(TcTarget))));
-    k_moddown_conv_tc<<<dim3(c->N / kTcM, 2, n_md), kTcM, smem, c->stream>>>(
-        u, tmp, level, c->L, c->K, c->d_prime, c->d_md_pcoef, (const uint8_t*)c->d_tc_btab,
-        (const TcTarget*)c->d_tc_tgt, c->d_err, c->log_n);
+    // persistent CTAs: four per SM (tensor memory: 128 of 512 columns each)
+    const int items = (c->N / kTcM) * 2 * n_md;
+    const int grid = items < 4 * c->sm_count ? items : 4 * c->sm_count;
+    k_moddown_conv_tc<<<grid, kTcThreads, smem, c->stream>>>(u, tmp, level, c->L, c->K, n_md, c->d_prime,
+                                                            c->d_md_pcoef, (const uint8_t*)c->d_tc_btab,
+                                                            (const TcTarget*)c->d_tc_tgt, c->d_err, c->log_n);
     c->launches++;
     return check_cuda(c, cudaGetLastError(), "moddown_conv_tc");
 }

@@ -35,8 +35,25 @@ def test_alu_bound_class_weights_the_two_pipes():
     assert r["fp64_share"] == pytest.approx(2.0 / 3.0)
 
 
-def test_traffic_is_scaled_from_the_committed_capture():
-    name = next(iter(bench.NCU_TRAFFIC_RATIO))
-    r = bench.roofline_for(name, (1.0, 1, 1e9, 1.0, 0.0), INT_S, FP_S, HBM, "measured")
-    assert r["traffic"] == pytest.approx(bench.NCU_TRAFFIC_RATIO[name] * 1e9)
-    assert 0.8 < bench.NCU_TRAFFIC_RATIO[name] < 1.3  # DRAM bytes near the algorithmic bytes
+def test_traffic_is_scaled_from_a_capture_of_unchanged_sources(tmp_path, monkeypatch):
+    """A stored ratio is used only while the digest of its kernel's sources
+    matches the one recorded with the capture."""
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    table = {"x": {"ratio": 0.91, "sources": ["k.cu"], "sha256": bench.source_digest(["k.cu"])}}
+    monkeypatch.setattr(bench, "NCU_TRAFFIC", table)
+    r = bench.roofline_for("x", (1.0, 1, 1e9, 1.0, 0.0), INT_S, FP_S, HBM, "measured")
+    assert r["traffic"] == pytest.approx(0.91e9)
+    src.write_text("kernel v2")  # the kernel changed after the capture
+    r = bench.roofline_for("x", (1.0, 1, 1e9, 1.0, 0.0), INT_S, FP_S, HBM, "measured")
+    assert r["traffic"] is None
+    assert bench.traffic_ratio("y") is None
+
+
+def test_stored_traffic_ratios_are_current():
+    """Every committed ratio still matches its kernel's sources and lies near
+    the algorithmic bytes (no class is re-reading what it should not)."""
+    for name, e in bench.NCU_TRAFFIC.items():
+        assert bench.traffic_ratio(name) is not None, name
+        assert 0.8 < e["ratio"] < 1.3, name
