@@ -925,7 +925,19 @@ def run_native(args, rank, world, local_rank):
 # not used, and `traffic` is then null.  Reads grow in proportion to the limbs
 # a launch transforms; a small capture leaves some written lines in L2 at its
 # end, so the ratio slightly undercounts writes.
-NCU_TRAFFIC = {}
+NTT_SOURCES = ["homomorphic_encrypted_transformer_b200/csrc/ntt.cu", "homomorphic_encrypted_transformer_b200/csrc/ntt.cuh",
+               "homomorphic_encrypted_transformer_b200/csrc/modarith.cuh",
+               "homomorphic_encrypted_transformer_b200/csrc/kernels.cuh"]
+# one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the four
+# transform passes on 512 limbs of 2^16 words (bench.py --case ntt; each pass
+# reads and writes 268.4 MB of limbs), taken with the sources of this digest
+NTT_SHA256 = "478a41ef306750bed1e66e57a1c2ba3effdc31a1ca75c4a7a4e9080bad334180"
+NCU_TRAFFIC = {
+    "ntt_fwd_cols": {"ratio": (268578304 + 217961984) / 536870912.0, "sources": NTT_SOURCES, "sha256": NTT_SHA256},
+    "ntt_fwd_rows": {"ratio": (314841600 + 217830144) / 536870912.0, "sources": NTT_SOURCES, "sha256": NTT_SHA256},
+    "ntt_inv_rows": {"ratio": (311631104 + 212199424) / 536870912.0, "sources": NTT_SOURCES, "sha256": NTT_SHA256},
+    "ntt_inv_cols": {"ratio": (268576512 + 214450432) / 536870912.0, "sources": NTT_SOURCES, "sha256": NTT_SHA256},
+}
 
 
 def source_digest(files):

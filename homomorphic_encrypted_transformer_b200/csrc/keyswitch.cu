@@ -173,27 +173,61 @@ __global__ void __launch_bounds__(256, 4)  // measured: better than 3 blocks per
     int c = blockIdx.x * blockDim.x + threadIdx.x;
     int i = blockIdx.y;
     if (c >= N) return;
-    uint64_t y[NS];
-    double yd[NS];  // y as a double (sources below 2^41)
-#pragma unroll
-    for (int s = 0; s < NS; s++) {
-        uint64_t q = pr[s0 + s].q;
-        uint64_t x = coef[((size_t)i * level + s0 + s) * N + c];
-        ulonglong2 w = src[s];
-        y[s] = mul_shoup(x, w.x, w.y, q);
-        yd[s] = u2d(q < kFpPrimeLimit ? y[s] : 0);
-    }
     uint64_t* o = ext_j + (size_t)i * n_tgt * N + c;
-
-    // 60-bit targets
     if constexpr (SPLIT) {
+        // Sources below 2^41 live as doubles only (the 60-bit source of a
+        // WIDE0 digit as an integer); the targets below 2^41 go first, then
+        // the 21-bit splits of the 60-bit targets are derived from the
+        // doubles, so at most two forms of a source are live at a time.
+        double yd[NS];
+        uint64_t yw = 0;
+#pragma unroll
+        for (int s = 0; s < NS; s++) {
+            const uint64_t q = pr[s0 + s].q;
+            const ulonglong2 w = src[s];
+            const uint64_t y = mul_shoup(coef[((size_t)i * level + s0 + s) * N + c], w.x, w.y, q);
+            if (MODE == kConvWide0 && s == 0) {
+                yw = y;
+                yd[0] = 0.0;
+            } else {
+                yd[s] = u2d(y);
+            }
+        }
+        // targets below 2^41, two at a time
+        for (int f = 0; f < n_fp; f += 2) {
+            const bool two = f + 1 < n_fp;
+            const int f1 = two ? f + 1 : f;
+            const FpMod F0 = sm_ff[f], F1 = sm_ff[f1];
+            double acc0 = 0.0, acc1 = 0.0;
+#pragma unroll
+            for (int s = 0; s < NS; s++) {
+                const double m0 = sm_fm[s * kConvMaxTargets + f], m1 = sm_fm[s * kConvMaxTargets + f1];
+                double y0 = yd[s], y1 = yd[s];
+                if (MODE == kConvWide0 && s == 0) {  // the 60-bit residue first drops to [0, 2t)
+                    const ConvTarget t0 = sm_ft[f], t1 = sm_ft[f1];
+                    y0 = u2d(yw - __umul64hi(yw, t0.one_shoup) * t0.q);
+                    y1 = u2d(yw - __umul64hi(yw, t1.one_shoup) * t1.q);
+                }
+                acc0 = __dadd_rn(acc0, fp_mulmod_s(y0, m0, F0));
+                acc1 = __dadd_rn(acc1, fp_mulmod_s(y1, m1, F1));
+            }
+            o[(size_t)sm_ftt[f] * N] = d2u(fp_canon(acc0, F0));
+            if (two) o[(size_t)sm_ftt[f1] * N] = d2u(fp_canon(acc1, F1));
+        }
+        // 60-bit targets: y = y1 2^21 + y0 (y0 < 2^21, y1 < 2^20), and for the
+        // WIDE0 source y = y2 2^42 + y1 2^21 + y0
         double y0[NS], y1[NS];
 #pragma unroll
         for (int s = 0; s < NS; s++) {
-            y0[s] = (double)(y[s] & ((1ull << 21) - 1));
-            y1[s] = (double)((y[s] >> 21) & ((1ull << 21) - 1));  // all of the rest when narrow
+            if (MODE == kConvWide0 && s == 0) {
+                y0[0] = (double)(yw & ((1ull << 21) - 1));
+                y1[0] = (double)((yw >> 21) & ((1ull << 21) - 1));
+            } else {
+                y1[s] = trunc(__dmul_rn(yd[s], 4.76837158203125e-07));  // exact: times 2^-21
+                y0[s] = __fma_rn(-y1[s], 2097152.0, yd[s]);
+            }
         }
-        const double y2w = MODE == kConvWide0 ? (double)(y[0] >> 42) : 0.0;  // < 2^18
+        const double y2w = MODE == kConvWide0 ? (double)(yw >> 42) : 0.0;  // < 2^18
         for (int g = 0; g < n_int; g++) {
             double v0 = 0, v1 = 0, v2 = 0, v3 = 0, v4 = 0;
 #pragma unroll
@@ -219,37 +253,42 @@ __global__ void __launch_bounds__(256, 4)  // measured: better than 3 blocks per
             o[(size_t)sm_itt[g] * N] = redc_t(acc, sm_it[g]);
         }
     } else {
+        uint64_t y[NS];
+        double yd[NS];  // y as a double (sources below 2^41)
+#pragma unroll
+        for (int s = 0; s < NS; s++) {
+            const uint64_t q = pr[s0 + s].q;
+            const ulonglong2 w = src[s];
+            y[s] = mul_shoup(coef[((size_t)i * level + s0 + s) * N + c], w.x, w.y, q);
+            yd[s] = u2d(q < kFpPrimeLimit ? y[s] : 0);
+        }
         for (int g = 0; g < n_int; g++) {
             U128 acc = {0, 0};
 #pragma unroll
             for (int s = 0; s < NS; s++) mac128(acc, y[s], sm_im[s * kConvMaxInt + g]);
             o[(size_t)sm_itt[g] * N] = redc_t(acc, sm_it[g]);
         }
-    }
-
-    // targets below 2^41, two at a time
-    for (int f = 0; f < n_fp; f += 2) {
-        const bool two = f + 1 < n_fp;
-        const int f1 = two ? f + 1 : f;
-        const FpMod F0 = sm_ff[f], F1 = sm_ff[f1];
-        double acc0 = 0.0, acc1 = 0.0;
+        // targets below 2^41, two at a time
+        for (int f = 0; f < n_fp; f += 2) {
+            const bool two = f + 1 < n_fp;
+            const int f1 = two ? f + 1 : f;
+            const FpMod F0 = sm_ff[f], F1 = sm_ff[f1];
+            double acc0 = 0.0, acc1 = 0.0;
 #pragma unroll
-        for (int s = 0; s < NS; s++) {
-            double m0 = sm_fm[s * kConvMaxTargets + f], m1 = sm_fm[s * kConvMaxTargets + f1];
-            double y0 = yd[s], y1 = yd[s];
-            if constexpr (MODE != kConvNarrow) {
-                if ((MODE == kConvGeneric || s == 0) && pr[s0 + s].q >= kFpPrimeLimit) {
-                    // a wide source residue first drops to [0, 2t)
+            for (int s = 0; s < NS; s++) {
+                const double m0 = sm_fm[s * kConvMaxTargets + f], m1 = sm_fm[s * kConvMaxTargets + f1];
+                double y0 = yd[s], y1 = yd[s];
+                if (pr[s0 + s].q >= kFpPrimeLimit) {  // a wide source residue first drops to [0, 2t)
                     const ConvTarget t0 = sm_ft[f], t1 = sm_ft[f1];
                     y0 = u2d(y[s] - __umul64hi(y[s], t0.one_shoup) * t0.q);
                     y1 = u2d(y[s] - __umul64hi(y[s], t1.one_shoup) * t1.q);
                 }
+                acc0 = __dadd_rn(acc0, fp_mulmod_s(y0, m0, F0));
+                acc1 = __dadd_rn(acc1, fp_mulmod_s(y1, m1, F1));
             }
-            acc0 = __dadd_rn(acc0, fp_mulmod_s(y0, m0, F0));
-            acc1 = __dadd_rn(acc1, fp_mulmod_s(y1, m1, F1));
+            o[(size_t)sm_ftt[f] * N] = d2u(fp_canon(acc0, F0));
+            if (two) o[(size_t)sm_ftt[f1] * N] = d2u(fp_canon(acc1, F1));
         }
-        o[(size_t)sm_ftt[f] * N] = d2u(fp_canon(acc0, F0));
-        if (two) o[(size_t)sm_ftt[f1] * N] = d2u(fp_canon(acc1, F1));
     }
 }
 

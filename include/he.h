@@ -97,7 +97,10 @@ int he_derive_primes(const he_params* params, uint64_t* primes_out, uint64_t* ps
 
 /* Builds the RNS tables on the host (primes, roots, twiddles, conversion
  * constants) and uploads them.  cuda_stream: a cudaStream_t or NULL for the
- * legacy default stream.  Synchronous.  *out receives the context. */
+ * legacy default stream.  Synchronous.  *out receives the context.
+ * Environment: HE_MODDOWN_CONV=tc makes the context's key switches run the
+ * ModDown base conversion as a split-integer GEMM on the tensor cores
+ * (identical residues; slower than the default FP64 kernel on B200). */
 int he_ctx_create(const he_params* params, void* cuda_stream, he_ctx** out);
 int he_ctx_destroy(he_ctx* ctx);
 int he_set_stream(he_ctx* ctx, void* cuda_stream);
