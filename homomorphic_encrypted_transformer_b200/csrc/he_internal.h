@@ -79,8 +79,12 @@ struct he_ctx {
     std::map<uint64_t, he::Key> rot_keys;  // by Galois element
     he::Key relin;
 
-    uint64_t* scratch[4] = {nullptr, nullptr, nullptr, nullptr};
-    size_t scratch_words[4] = {0, 0, 0, 0};
+    uint64_t* scratch[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+    size_t scratch_words[5] = {0, 0, 0, 0, 0};
+    int ks_slot = 0;                    // scratch slot of key switching (4 on the auxiliary stream)
+    cudaStream_t aux = nullptr;         // second stream of a split rotation batch
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr, ev_mid = nullptr;
+    bool stagger = false, ev_mid_pending = false;  // second half starts after the first half's ModUp
     uint64_t* noalloc_scratch = nullptr;  // device address of he_rescale_noalloc's fixed array
     int* d_err = nullptr;                 // device error word: a bounded device wait gave up (he_sync reports it)
     void* d_tc_btab = nullptr;            // tensor-core ModDown conversion: byte matrix B (moddown_tc.cu)
@@ -158,6 +162,9 @@ struct KsIoList {
     int sum_terms = 0;
 };
 int key_switch(he_ctx* c, int level, const KsIoList& io);
+// key_switch of a plain (not hoisted, not summed) batch in two halves on two
+// streams, forked from and joined back into the context's stream.
+int key_switch_split(he_ctx* c, int level, const KsIoList& io);
 int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io);
 size_t key_switch_scratch_words(const he_ctx* c, int n_raised, int n, int level);
 int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, int n);
@@ -168,9 +175,10 @@ int rotate_sum_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t*
 
 // Scratch slots: 0 = key switching internals, 1 = rescale temporaries,
 // 2 = HMult temporaries, key generation and the pre-sums of the summed
-// rotations, 3 = driver buffers (polynomial evaluation, BSGS).  A call only
-// uses slots below the ones its callers hold.
-constexpr int kScratchSlots = 4;
+// rotations, 3 = driver buffers (polynomial evaluation, BSGS), 4 = key
+// switching on the auxiliary stream (the second half of a split rotation
+// batch).  A call only uses slots below the ones its callers hold.
+constexpr int kScratchSlots = 5;
 int scratch_slot(he_ctx* c, int slot, size_t words, uint64_t** out);
 
 // out[i] = rescale(in[i]) for n ciphertexts at `level` (out may equal in).

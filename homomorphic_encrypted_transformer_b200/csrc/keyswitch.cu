@@ -710,7 +710,7 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     if (summed && n % G) return set_err(c, HE_EINVAL, "key switch: bad summed lists");
     const int n_md = summed ? n / G : n;
     uint64_t* base;
-    int rc = scratch_slot(c, 0, key_switch_scratch_words(c, nm, n_md, level), &base);
+    int rc = scratch_slot(c, c->ks_slot, key_switch_scratch_words(c, nm, n_md, level), &base);
     if (rc) return rc;
     const int ext_rows = nd * n_rows - level;  // sum over digits of the target rows
     uint64_t* coef = base;
@@ -831,6 +831,11 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
         if ((rc = ntt_fwd_set(c, rs, nm * nt))) return rc;
     }
 
+    // the ModUp of this chunk is enqueued: a staggered split starts its second half here
+    if (c->ev_mid_pending) {
+        if ((rc = check_cuda(c, cudaEventRecord(c->ev_mid, c->stream), "stagger"))) return rc;
+        c->ev_mid_pending = false;
+    }
     prof_begin(c, HE_PROF_KS_INNER);
     const int gx2 = (N / 2 + TB - 1) / TB;  // two positions per thread
     switch (nd) {
@@ -938,6 +943,69 @@ int key_switch(he_ctx* c, int level, const KsIoList& io) {
     return HE_OK;
 }
 
+// Key switching of a batch split in two halves on two streams: the first
+// half on the context's stream, the second on an auxiliary stream with its
+// own scratch, forked from and joined back into the context's stream by
+// events.  Each half is a chain of ALU-heavy and memory-heavy kernels; run
+// side by side, one half's key inner product streams keys while the other
+// converts or transforms.  The split falls on a key boundary (entries that
+// share a key are adjacent), so each key is still read once per half at
+// most (a batch with a single key, as in relinearisation, splits in the
+// middle and each half reads the key once).  Results are the same as
+// key_switch's.  With profiling on, or for small batches, one stream does
+// everything in order.
+int key_switch_split(he_ctx* c, int level, const KsIoList& io) {
+    const int n = (int)io.d.size();
+    if (c->prof_on || n < 16) return key_switch(c, level, io);
+    int k = n / 2;
+    while (k < n && io.key[k] == io.key[k - 1]) k++;  // next key boundary at or after n/2
+    if (k == n) {                                      // else the last one before it
+        k = n / 2;
+        while (k > 0 && io.key[k] == io.key[k - 1]) k--;
+    }
+    if (k == 0) k = n / 2;  // one key for all
+    int rc;
+    if (!c->aux && (rc = check_cuda(c, cudaStreamCreateWithFlags(&c->aux, cudaStreamNonBlocking), "aux stream")))
+        return rc;
+    if (!c->ev_fork && (rc = check_cuda(c, cudaEventCreateWithFlags(&c->ev_fork, cudaEventDisableTiming), "event")))
+        return rc;
+    if (!c->ev_join && (rc = check_cuda(c, cudaEventCreateWithFlags(&c->ev_join, cudaEventDisableTiming), "event")))
+        return rc;
+    auto part = [&](int a, int b) {
+        KsIoList h;
+        h.sig_add0 = io.sig_add0;
+        h.galois.assign(io.galois.begin() + a, io.galois.begin() + b);
+        h.key.assign(io.key.begin() + a, io.key.begin() + b);
+        h.d.assign(io.d.begin() + a, io.d.begin() + b);
+        h.out.assign(io.out.begin() + a, io.out.begin() + b);
+        h.add0.assign(io.add0.begin() + a, io.add0.begin() + b);
+        h.add1.assign(io.add1.begin() + a, io.add1.begin() + b);
+        return h;
+    };
+    if (c->stagger && !c->ev_mid &&
+        (rc = check_cuda(c, cudaEventCreateWithFlags(&c->ev_mid, cudaEventDisableTiming), "event")))
+        return rc;
+    if ((rc = check_cuda(c, cudaEventRecord(c->ev_fork, c->stream), "fork")) ||
+        (rc = check_cuda(c, cudaStreamWaitEvent(c->aux, c->ev_fork, 0), "fork")))
+        return rc;
+    c->ev_mid_pending = c->stagger;
+    rc = key_switch(c, level, part(0, k));
+    c->ev_mid_pending = false;
+    if (!rc && c->stagger) rc = check_cuda(c, cudaStreamWaitEvent(c->aux, c->ev_mid, 0), "stagger");
+    cudaStream_t main = c->stream;
+    if (!rc) {
+        c->stream = c->aux;
+        c->ks_slot = 4;
+        rc = key_switch(c, level, part(k, n));
+        c->stream = main;
+        c->ks_slot = 0;
+    }
+    // join whatever was enqueued on the auxiliary stream, also after an error
+    int rj = check_cuda(c, cudaEventRecord(c->ev_join, c->aux), "join");
+    if (!rj) rj = check_cuda(c, cudaStreamWaitEvent(c->stream, c->ev_join, 0), "join");
+    return rc ? rc : rj;
+}
+
 static int ct_ok(he_ctx* c, const he_ct* x, const char* what) {
     if (!x || !x->data) return set_err(c, HE_EINVAL, "%s: null ciphertext", what);
     if ((uintptr_t)x->data & 15) return set_err(c, HE_EINVAL, "%s: ciphertext not 16-byte aligned", what);
@@ -990,7 +1058,7 @@ int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, in
         }
     }
     if (!io.d.empty()) {
-        int rc = key_switch(c, level, io);
+        int rc = key_switch_split(c, level, io);
         if (rc) return rc;
     }
     for (int i = 0; i < n; i++) {

@@ -312,7 +312,7 @@ int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vecto
             io.add0.push_back(d);
             io.add1.push_back(d + (size_t)level * N);
         }
-        if ((rc = key_switch(c, level, io))) return rc;
+        if ((rc = key_switch_split(c, level, io))) return rc;
         std::vector<const uint64_t*> rin(io.out.begin(), io.out.end());
         std::vector<uint64_t*> rout(out.begin() + i0, out.begin() + i0 + m);
         if ((rc = rescale_many(c, rin, rout, level))) return rc;
