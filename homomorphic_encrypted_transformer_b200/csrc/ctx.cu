@@ -506,8 +506,6 @@ extern "C" int he_ctx_create(const he_params* prm, void* stream, he_ctx** out) {
         // the FP64 conversion kernel unless "tc" selects the tensor-core one
         const char* v = getenv("HE_MODDOWN_CONV");
         c->tc_moddown = moddown_tc_available(c) && v && strcmp(v, "tc") == 0;
-        const char* st = getenv("HE_KS_STAGGER");
-        c->stagger = st && st[0] == '1';
     }
     if (rc) {
         fprintf(stderr, "he_ctx_create: %s\n", c->err.c_str());
@@ -524,7 +522,6 @@ extern "C" int he_ctx_destroy(he_ctx* c) {
     if (c->aux) cudaStreamSynchronize(c->aux), cudaStreamDestroy(c->aux);
     if (c->ev_fork) cudaEventDestroy(c->ev_fork);
     if (c->ev_join) cudaEventDestroy(c->ev_join);
-    if (c->ev_mid) cudaEventDestroy(c->ev_mid);
     cudaFree(c->d_prime);
     cudaFree(c->d_tw_fwd);
     cudaFree(c->d_tw_inv);

@@ -83,8 +83,7 @@ struct he_ctx {
     size_t scratch_words[5] = {0, 0, 0, 0, 0};
     int ks_slot = 0;                    // scratch slot of key switching (4 on the auxiliary stream)
     cudaStream_t aux = nullptr;         // second stream of a split rotation batch
-    cudaEvent_t ev_fork = nullptr, ev_join = nullptr, ev_mid = nullptr;
-    bool stagger = false, ev_mid_pending = false;  // second half starts after the first half's ModUp
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
     uint64_t* noalloc_scratch = nullptr;  // device address of he_rescale_noalloc's fixed array
     int* d_err = nullptr;                 // device error word: a bounded device wait gave up (he_sync reports it)
     void* d_tc_btab = nullptr;            // tensor-core ModDown conversion: byte matrix B (moddown_tc.cu)

@@ -831,11 +831,6 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
         if ((rc = ntt_fwd_set(c, rs, nm * nt))) return rc;
     }
 
-    // the ModUp of this chunk is enqueued: a staggered split starts its second half here
-    if (c->ev_mid_pending) {
-        if ((rc = check_cuda(c, cudaEventRecord(c->ev_mid, c->stream), "stagger"))) return rc;
-        c->ev_mid_pending = false;
-    }
     prof_begin(c, HE_PROF_KS_INNER);
     const int gx2 = (N / 2 + TB - 1) / TB;  // two positions per thread
     switch (nd) {
@@ -982,16 +977,10 @@ int key_switch_split(he_ctx* c, int level, const KsIoList& io) {
         h.add1.assign(io.add1.begin() + a, io.add1.begin() + b);
         return h;
     };
-    if (c->stagger && !c->ev_mid &&
-        (rc = check_cuda(c, cudaEventCreateWithFlags(&c->ev_mid, cudaEventDisableTiming), "event")))
-        return rc;
     if ((rc = check_cuda(c, cudaEventRecord(c->ev_fork, c->stream), "fork")) ||
         (rc = check_cuda(c, cudaStreamWaitEvent(c->aux, c->ev_fork, 0), "fork")))
         return rc;
-    c->ev_mid_pending = c->stagger;
     rc = key_switch(c, level, part(0, k));
-    c->ev_mid_pending = false;
-    if (!rc && c->stagger) rc = check_cuda(c, cudaStreamWaitEvent(c->aux, c->ev_mid, 0), "stagger");
     cudaStream_t main = c->stream;
     if (!rc) {
         c->stream = c->aux;
