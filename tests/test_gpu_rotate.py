@@ -180,6 +180,27 @@ def test_rotation_batch_host_buffers_pipelined():
     assert np.array_equal(h_out2, h_out)
 
 
+def test_rotation_batch_host_buffers_full_size():
+    """The host-buffer entry on the rotation batch (64 ciphertexts at
+    N=2^16, level 24, 16 keys; chunks of 8 ordered by step) gives the device
+    entry's residues, ciphertext for ciphertext."""
+    he = lib()
+    st = Setup(16, 24, 8, 3, seed=S.master_seed(1))
+    P = st.P
+    steps, ct_steps = _rotation_batch_inputs(st, 64, 16)
+    for s_ in steps:
+        st.upload_rot(s_)
+    h_in = S.uniform_residues(st.seed, "ct_residues", P.q, P.N, lead=(64, 2))
+    x = torch.from_numpy(h_in.view(np.int64)).cuda()
+    y = torch.empty_like(x)
+    he.he_rotate_batch(st.ctx, [he.Ciphertext(x[i], 24, 2.0 ** 40) for i in range(64)], ct_steps,
+                       [he.Ciphertext(y[i], 24, 2.0 ** 40) for i in range(64)])
+    he.he_sync(st.ctx)
+    h_out = np.zeros_like(h_in)
+    he.he_rotate_batch_host(st.ctx, h_in, 24, ct_steps, h_out)
+    assert np.array_equal(h_out, host(y).reshape(h_in.shape))
+
+
 def _hoisted_case(st, level, n_in, steps):
     """he_rotate_hoisted of n_in encrypted inputs by `steps` against the
     oracle's rotate_hoisted, residue for residue; Galois element 1 copies."""
