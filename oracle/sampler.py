@@ -18,11 +18,17 @@ from the published definitions; no code is shared with the library.
     T_i = floor(2^64 C_i), C_i = P(e <= -19 + i) with
     P(k) proportional to exp(-k^2 / (2 sigma^2)) = exp(-25 k^2 / 512),
     computed in exact decimal arithmetic; a draw x gives -19 + #{i: T_i <= x}.
+  * Seeded a-halves (keys that store only b and regenerate a where it is
+    used): tag 4, one stream per digit and prime; coefficient i of the row
+    takes outputs 1 + i + t N, t = 0, 1, ..., 63 (so any coefficient is
+    computed alone), the first whose top bitlen(q) bits are < q; if none of
+    the 64 is, the last one's top bits minus q.
 
 Parity pinned: SplitMix64's published first outputs (tests/golden), the
 threshold table's symmetry and its agreement with an independent float
-computation to 2^-40, the samplers' value ranges and frequencies
-(tests/test_oracle_sampler.py).
+computation to 2^-40, the samplers' value ranges and frequencies, and the
+seeded a-halves against the generator stepped one state at a time with
+rejections forced (tests/test_oracle_sampler.py).
 """
 from decimal import Decimal, getcontext
 
@@ -31,7 +37,8 @@ import numpy as np
 GAMMA = 0x9E3779B97F4A7C15
 M64 = (1 << 64) - 1
 ERR_BOUND = 19
-TAG_SECRET, TAG_KEY_A, TAG_KEY_E = 1, 2, 3
+TAG_SECRET, TAG_KEY_A, TAG_KEY_E, TAG_KEY_A_SEEDED = 1, 2, 3, 4
+A_SEEDED_TRIES = 64
 
 
 def mix64(z):
@@ -126,3 +133,39 @@ def key_draws(seed, key_id, moduli, n, digits):
             a[j, r] = uniform(seed, obj_id(TAG_KEY_A, key_id, j, r), q, n)
         e[j] = gaussian(seed, obj_id(TAG_KEY_E, key_id, j, 0), n)
     return a, e
+
+
+def a_seeded_row(seed, obj, q, n, tries=A_SEEDED_TRIES):
+    """One row of a seeded a-half: uint64[n], coefficient i from outputs
+    1 + i + t n of the stream of obj (t < tries), by the rule above."""
+    sh = np.uint64(64 - int(q).bit_length())
+    qq = np.uint64(q)
+    s0 = stream_start(seed, obj)
+    out = np.zeros(n, dtype=np.uint64)
+    todo = np.arange(n)
+    for t in range(tries):
+        x = outputs(s0, t * n, n)[todo] >> sh
+        ok = x < qq
+        out[todo[ok]] = x[ok]
+        if t == tries - 1:
+            out[todo[~ok]] = x[~ok] - qq
+        todo = todo[~ok]
+        if len(todo) == 0:
+            break
+    return out
+
+
+def key_a_seeded(seed, key_id, moduli, n, digits):
+    """The a-half of one switching key with seeded a: uint64
+    [digits][len(moduli)][n], row r of digit j uniform mod moduli[r]."""
+    a = np.empty((digits, len(moduli), n), dtype=np.uint64)
+    for j in range(digits):
+        for r, q in enumerate(moduli):
+            a[j, r] = a_seeded_row(seed, obj_id(TAG_KEY_A_SEEDED, key_id, j, r), q, n)
+    return a
+
+
+def key_errors(seed, key_id, n, digits):
+    """The errors of one switching key, int32 [digits][n] (the same draws as
+    key_draws')."""
+    return np.stack([gaussian(seed, obj_id(TAG_KEY_E, key_id, j, 0), n) for j in range(digits)])

@@ -106,3 +106,58 @@ def test_streams_differ_by_object_and_seed():
     c = R.uniform(2, R.obj_id(R.TAG_KEY_A, 5, 0, 0), 97, 64)
     assert not np.array_equal(a, b) and not np.array_equal(a, c)
     assert math.isclose(np.mean(a), 48, abs_tol=15)
+
+
+def _a_seeded_brute(seed, obj, q, n, tries):
+    """Coefficient i from the generator stepped one state at a time: output
+    number 1 + i + t n is raw[i + t n]."""
+    sh = 64 - q.bit_length()
+    raw = _sequential(R.stream_start(seed, obj), tries * n)
+    out = []
+    for i in range(n):
+        for t in range(tries):
+            x = raw[i + t * n] >> sh
+            if x < q:
+                out.append(x)
+                break
+        else:
+            out.append(x - q)
+    return out
+
+
+def test_seeded_a_row_against_the_stepped_generator():
+    # q = 5 keeps 5 of the 8 values of the top three bits: many coefficients
+    # need a second or third try
+    seed, obj = 0xA5EED, R.obj_id(R.TAG_KEY_A_SEEDED, 7, 2, 3)
+    want = _a_seeded_brute(seed, obj, 5, 24, R.A_SEEDED_TRIES)
+    assert R.a_seeded_row(seed, obj, 5, 24).tolist() == want
+    assert max(want) < 5
+
+
+def test_seeded_a_row_fallback_after_the_last_try():
+    # two tries only: about 14% of the coefficients reject both and take the
+    # last draw minus q
+    seed, obj = 11, R.obj_id(R.TAG_KEY_A_SEEDED, 3, 0, 1)
+    sh = 61
+    raw = _sequential(R.stream_start(seed, obj), 2 * 64)
+    fell = [i for i in range(64) if (raw[i] >> sh) >= 5 and (raw[i + 64] >> sh) >= 5]
+    assert fell, "the seed must exercise the fallback"
+    got = R.a_seeded_row(seed, obj, 5, 64, tries=2).tolist()
+    assert got == _a_seeded_brute(seed, obj, 5, 64, 2)
+    assert all(got[i] == (raw[i + 64] >> sh) - 5 for i in fell)
+
+
+def test_seeded_a_ranges_frequencies_and_streams():
+    n = 1 << 16
+    q = 0xffffe80001  # a 40-bit prime of the chain
+    a = R.a_seeded_row(5, R.obj_id(R.TAG_KEY_A_SEEDED, 9, 1, 4), q, n)
+    assert a.max() < q
+    h = np.bincount((a.astype(np.float64) / q * 16).astype(np.int64), minlength=16)
+    assert ((h - n / 16) ** 2 / (n / 16)).sum() < 40
+    # distinct from the stored-key stream of the same key, digit and prime
+    b = R.uniform(5, R.obj_id(R.TAG_KEY_A, 9, 1, 4), q, n)
+    assert np.mean(a == b) < 1e-3
+    A = R.key_a_seeded(5, 9, [97, q], 256, 2)
+    assert A.shape == (2, 2, 256) and A[:, 0].max() < 97
+    assert np.array_equal(A[1, 1], R.a_seeded_row(5, R.obj_id(R.TAG_KEY_A_SEEDED, 9, 1, 1), q, 256))
+    assert np.array_equal(R.key_errors(5, 9, 256, 2), R.key_draws(5, 9, [97], 256, 2)[1])
