@@ -49,6 +49,9 @@ def parse():
     ap.add_argument("--no-workloads", action="store_true",
                     help="default run: the rotation-batch line only, without the other workloads' entries")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--seeded-a", action="store_true",
+                    help="keys with seeded a-halves (he_keygen_seeded_ex, HE_KEYGEN_SEEDED_A): only b stored, a "
+                         "regenerated inside the key-switching kernels (rotation, hoisted, rotsum)")
     ap.add_argument("--case", default="rotation",
                     choices=["rotation", "ntt", "rot_small", "ffn128", "ffn2048", "ps15", "tiny", "hoisted",
                              "rotsum", "attention"],
@@ -245,9 +248,12 @@ def cpu_baseline(seconds):
                       "key generation excluded; oracle threads over limbs" % done}
 
 
-def line_config(world):
+def line_config(world, seeded_a=False):
     """The `config` of the rotation-batch line, identical on both arms."""
-    return dict(WORKLOAD, parallelism="replicas%d" % world if world > 1 else "single")
+    cfg = dict(WORKLOAD, parallelism="replicas%d" % world if world > 1 else "single")
+    if seeded_a:
+        cfg["keys"] = "seeded a-halves: b stored (0.8 GB per step), a regenerated in the key inner product"
+    return cfg
 
 
 # rotations of the batch that one step of the reference arm times
@@ -533,7 +539,7 @@ def workload_cpu_baseline(case, seconds):
                       % (n_pm, rot, pms, n_groups * f["n_out"], per_product)}
 
 
-def workload_case(case, n_steps, n_warmup, cpu_seconds, local_rank, probes=None, with_cpu=True):
+def workload_case(case, n_steps, n_warmup, cpu_seconds, local_rank, probes=None, with_cpu=True, seeded_a=False):
     """Throughput of one of the other workloads on one GPU, as a dict:
     ffn128 (FFN1 768->3072, 128 tokens: 3 x 12 blocks by BSGS at level 12),
     ffn2048 (the same product for 16 token groups sharing the weights),
@@ -543,6 +549,7 @@ def workload_case(case, n_steps, n_warmup, cpu_seconds, local_rank, probes=None,
     16 steps through one ModUp per ciphertext: 64 hoisted rotations),
     rotsum (the same 4 ciphertexts each summed over its 16 rotations with
     one ModUp and one ModDown: 64 rotations into 4 sums),
+    rotation (the rotation batch of the headline, for its seeded-a form),
     attention (one encrypted head at level 24: 64 features x 256 tokens, all
     256 token offsets: scores, the degree-15 exponential, A x V).
     Inputs are seeded uniform residues on the device; the rotation and
@@ -554,7 +561,8 @@ def workload_case(case, n_steps, n_warmup, cpu_seconds, local_rank, probes=None,
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream()
-    widx = {"tiny": 0, "hoisted": 1, "rotsum": 1, "ffn128": 2, "ffn2048": 3, "ps15": 4, "attention": 5}[case]
+    widx = {"tiny": 0, "rotation": 1, "hoisted": 1, "rotsum": 1, "ffn128": 2, "ffn2048": 3, "ps15": 4,
+            "attention": 5}[case]
     master = S.master_seed(widx)
     gen = torch.Generator(device=dev)
     gen.manual_seed(master)
@@ -569,6 +577,13 @@ def workload_case(case, n_steps, n_warmup, cpu_seconds, local_rank, probes=None,
         kid = 2 if kind == he.HE_KEY_RELIN else pow(5, step % (N // 2), 2 * N)  # Galois elements are odd
         a, e = S.key_draws(master, kid, ctx.primes, N, ctx.dnum)
         he.he_keygen_upload(ctx, kind, step, s_key, a, e)
+
+    def rotation_keys(steps):
+        if seeded_a:
+            he.he_keygen_seeded_ex(ctx, master, steps, False, he.HE_KEYGEN_SEEDED_A)
+        else:
+            for st in steps:
+                upload(he.HE_KEY_ROTATION, st)
 
     if case in ("ffn128", "ffn2048"):
         f = FFN
@@ -594,10 +609,22 @@ def workload_case(case, n_steps, n_warmup, cpu_seconds, local_rank, probes=None,
         cfg = {"workload": case, "N": N, "level": lvl, "tokens": f["n_tok"] * n_groups, "bs": f["bs"], "gs": f["gs"],
                "rotations_per_step": n_groups * f["n_in"] * (f["bs"] - 1) + n_groups * f["n_out"] * (f["gs"] - 1),
                "weights_gb": pt.numel() * 8 / 1e9}
+    elif case == "rotation":
+        steps, ct_steps = workload_inputs(master, ctx.primes[:L], N_CTS)
+        rotation_keys(steps)
+        x = device_residues(torch, (N_CTS, 2), ctx.primes[:L], N, gen, dev)
+        y = torch.empty_like(x)
+        xs = [he.Ciphertext(x[i], L, 2.0 ** 40) for i in range(N_CTS)]
+        ys = [he.Ciphertext(y[i], L, 2.0 ** 40) for i in range(N_CTS)]
+
+        def step():
+            he.he_rotate_batch(ctx, xs, ct_steps, ys)
+
+        metric, unit, per_step = METRIC, "rotations/s", N_CTS
+        cfg = dict(WORKLOAD)
     elif case == "hoisted":
         steps, _ = workload_inputs(master, ctx.primes[:L], N_CTS)
-        for st in steps:
-            upload(he.HE_KEY_ROTATION, st)
+        rotation_keys(steps)
         n_in = N_CTS // N_KEYS
         x = device_residues(torch, (n_in, 2), ctx.primes[:L], N, gen, dev)
         y = torch.empty((n_in * N_KEYS, 2, L, N), dtype=torch.int64, device=dev)
@@ -613,8 +640,7 @@ def workload_case(case, n_steps, n_warmup, cpu_seconds, local_rank, probes=None,
                "n_steps": N_KEYS, "l2": "inputs and keys larger than L2 (1.6 GB of keys per step)"}
     elif case == "rotsum":
         steps, _ = workload_inputs(master, ctx.primes[:L], N_CTS)
-        for st in steps:
-            upload(he.HE_KEY_ROTATION, st)
+        rotation_keys(steps)
         n_in = N_CTS // N_KEYS
         x = device_residues(torch, (n_in, 2), ctx.primes[:L], N, gen, dev)
         y = torch.empty_like(x)
@@ -722,14 +748,21 @@ def workload_case(case, n_steps, n_warmup, cpu_seconds, local_rank, probes=None,
             "probes": {"copy_gbs": copy_gbs, "int_shoup_modmul_per_s": int_modmul_s,
                        "fp64_modmul_per_s": fp_modmul_s},
             "clocks": clk}
+    if seeded_a:
+        cfg["keys"] = "seeded a-halves: b stored, a regenerated in the key inner product"
     if with_cpu:
         line["cpu_baseline"] = workload_cpu_baseline(case, cpu_seconds)
     return line
 
 
-# the other workloads of the default run: (warm-up steps, timed steps) each
+# the other workloads of the default run: (warm-up steps, timed steps) each.
+# A name ending in _seeded_a is its workload with seeded a-halves in every
+# key (HE_KEYGEN_SEEDED_A); its oracle baseline is the stored-key entry's
+# (the oracle's work does not depend on how the key is kept).
 WORKLOAD_STEPS = {"ntt": (3, 10), "tiny": (3, 20), "hoisted": (3, 10), "rotsum": (3, 10), "ps15": (3, 5),
-                  "ffn128": (3, 4), "ffn2048": (3, 2), "attention": (3, 2)}
+                  "ffn128": (3, 4), "ffn2048": (3, 2), "attention": (3, 2), "rotation_seeded_a": (3, 10),
+                  "hoisted_seeded_a": (3, 10)}
+SEEDED_A_SUFFIX = "_seeded_a"
 # seconds of oracle work per workload's cpu_baseline in the default run
 WORKLOAD_CPU_SECONDS = 3.0
 
@@ -746,6 +779,9 @@ def all_workloads(local_rank, probes):
         t0 = time.perf_counter()
         if case == "ntt":
             r = ntt_case(k, w, local_rank, probes)
+        elif case.endswith(SEEDED_A_SUFFIX):
+            r = workload_case(case[:-len(SEEDED_A_SUFFIX)], k, w, WORKLOAD_CPU_SECONDS, local_rank, probes,
+                              with_cpu=False, seeded_a=True)
         else:
             r = workload_case(case, k, w, WORKLOAD_CPU_SECONDS, local_rank, probes)
         r["wall_s"] = time.perf_counter() - t0
@@ -803,11 +839,14 @@ def run_native(args, rank, world, local_rank):
     N = ctx.N
     master = S.master_seed(1)
     steps, ct_steps = workload_inputs(master, ctx.primes[:L], N_CTS)
-    s = S.secret(master, N)
-    for st in steps:
-        k = pow(5, st % (N // 2), 2 * N)
-        a, e = S.key_draws(master, k, ctx.primes, N, DNUM)
-        he.he_keygen_upload(ctx, he.HE_KEY_ROTATION, st, s, a, e)
+    if args.seeded_a:
+        he.he_keygen_seeded_ex(ctx, master, steps, False, he.HE_KEYGEN_SEEDED_A)
+    else:
+        s = S.secret(master, N)
+        for st in steps:
+            k = pow(5, st % (N // 2), 2 * N)
+            a, e = S.key_draws(master, k, ctx.primes, N, DNUM)
+            he.he_keygen_upload(ctx, he.HE_KEY_ROTATION, st, s, a, e)
     # inputs: uniform residues (a fresh encryption is computationally
     # indistinguishable from them); per-rank stream of draws
     h_in = S.uniform_residues(rank_seed(master, rank), "ct_residues", ctx.primes[:L], N, lead=(N_CTS, 2))
@@ -884,7 +923,7 @@ def run_native(args, rank, world, local_rank):
     # dominant kernel class by device time in the profiled pass
     dom_name = max(prof, key=lambda k: prof[k][0])
     ct_bytes = 2 * LEVEL * N * 8
-    key_bytes = 3 * 2 * (L + K) * N * 8
+    key_bytes = 3 * (1 if args.seeded_a else 2) * (L + K) * N * 8  # digits x stored halves x rows
     # algorithmic bytes of one rotation batch (keys read once per key group)
     batch_bytes = N_KEYS * key_bytes + N_CTS * 2 * ct_bytes
     hbm_frac_step = (batch_bytes / (ms_plain * 1e-3 / args.steps)) / 1e9 / hbm_peak
@@ -895,7 +934,7 @@ def run_native(args, rank, world, local_rank):
     line = {"metric": METRIC, "value": value, "unit": "rotations/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_plain / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u64", "data": "synthetic",
-            "config": line_config(world),
+            "config": line_config(world, args.seeded_a),
             "hbm_roofline_frac_of_step": hbm_frac_step,
             "alu_ideal_ms_per_step": alu_ideal_ms,
             "alu_roofline_frac_of_step": alu_ideal_ms / (ms_plain / args.steps),
@@ -1023,7 +1062,7 @@ def main():
             run_rot_small_case(args, local_rank)
         elif args.case in ("ffn128", "ffn2048", "ps15", "tiny", "hoisted", "rotsum", "attention"):
             print(json.dumps(workload_case(args.case, args.steps, args.warmup, args.cpu_seconds, local_rank,
-                                           with_cpu=not args.no_cpu_baseline)), flush=True)
+                                           with_cpu=not args.no_cpu_baseline, seeded_a=args.seeded_a)), flush=True)
         else:
             line = run_native(args, rank, world, local_rank)
             if line is not None:

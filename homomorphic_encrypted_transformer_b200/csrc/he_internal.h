@@ -30,10 +30,20 @@ struct ConvTable {
 struct FpMod;  // FP64 constants of a prime below 2^41 (ntt.cuh)
 
 struct Key {
-    // [digits][2][L+K][N]: rows of primes below 2^41 as doubles, the others in
-    // Montgomery form (value * 2^64 mod p)
+    // [digits][2][L+K][N] (b then a): rows of primes below 2^41 as doubles,
+    // the others in Montgomery form (value * 2^64 mod p).  With seeded_a:
+    // [digits][L+K][N] b-halves only, followed by the a-halves' stream starts
+    // s0 [digits][L+K] (keyseed.cuh), from which the kernels regenerate a.
     uint64_t* d = nullptr;
+    bool seeded_a = false;
 };
+
+// Do the context's keys store only b-halves?  (All keys of a context have
+// one form.)
+bool keys_seeded_a(const he_ctx* c);
+
+// Stream start of row prime_index of digit `digit` of a seeded a-half (sampler.cpp).
+uint64_t seeded_a_stream_start(uint64_t seed, uint64_t key_id, int digit, int prime_index);
 
 struct ProfSlot {
     double ms = 0;

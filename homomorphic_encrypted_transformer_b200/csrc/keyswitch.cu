@@ -10,6 +10,7 @@
 #include <set>
 
 #include "he_internal.h"
+#include "keyseed.cuh"
 #include "ntt.cuh"
 
 namespace he {
@@ -65,6 +66,11 @@ __global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
 // src_row..src_row+n_src-1 and its targets are all the other rows, stored
 // compactly: target row t sits at position t (t < src_row) or t - n_src.
 // ext layout: [digit][ciphertext][n_rows - n_src][N].
+// Entries per group of k_ks_inner_grp (one thread applies its key words to
+// each in turn): 16 measured best, by a little, for the rotation batch,
+// hoisted rotations and relinearisation batches (caps of 1 to 16 tried).
+constexpr int kKsGroupMax = 16;
+
 struct ModupArgs {
     int n_digits;
     int n_src[kMaxDigits];
@@ -303,11 +309,58 @@ __global__ void __launch_bounds__(256, 4)  // measured: better than 3 blocks per
 // ND = number of digits (compile time, so that every load of a thread is in
 // flight at once).  HOIST: the raised digits belong to ciphertext xsrc[i] of
 // ext (n_ext of them) and are read through sigma_{g_i} as well: the
-// automorphism of a hoisted rotation, applied after ModUp.
-template <int ND, bool HOIST>
+// automorphism of a hoisted rotation, applied after ModUp.  SA: the keys
+// store only their b-halves (key_digits of them); the a-halves are
+// regenerated from their stream starts (keyseed.cuh) as canonical residues,
+// and integer rows reduce their a-sums with reduce128 instead of REDC.
+template <int ND, bool SA>
+__device__ __forceinline__ void load_key_halves(const uint64_t* key, int j, int krow, int LK, int N, int c,
+                                                ulonglong2& kb, ulonglong2& ka) {
+    if constexpr (SA) {
+        kb = __ldg(reinterpret_cast<const ulonglong2*>(key + ((size_t)j * LK + krow) * N + c));
+    } else {
+        kb = __ldg(reinterpret_cast<const ulonglong2*>(key + (((size_t)j * 2 + 0) * LK + krow) * N + c));
+        ka = __ldg(reinterpret_cast<const ulonglong2*>(key + (((size_t)j * 2 + 1) * LK + krow) * N + c));
+    }
+}
+
+// The a-halves of a seeded key at positions c, c + 1 of row krow, digits < ND.
+template <int ND>
+__device__ __forceinline__ void seeded_a_halves(const uint64_t* key, int key_digits, int krow, int LK, int N, int c,
+                                                uint64_t q, ulonglong2 (&ka)[ND]) {
+    const uint64_t* s0p = key + (size_t)key_digits * LK * N + krow;
+    const int sh = __clzll(q);
+#pragma unroll
+    for (int j = 0; j < ND; j++) {
+        const uint64_t s0 = __ldg(s0p + (size_t)j * LK);
+        ka[j] = make_ulonglong2(seeded_a(s0, c, N, q, sh), seeded_a(s0, c + 1, N, q, sh));
+    }
+}
+
+// An a-half word as the FP64 path multiplies it: stored keys hold the bits
+// of a double, seeded ones the canonical residue.
+template <bool SA>
+__device__ __forceinline__ double key_a_fp(uint64_t w) {
+    if constexpr (SA)
+        return u2d(w);
+    else
+        return __longlong_as_double((long long)w);
+}
+
+// sum of the a-products mod q, [0, q): REDC of Montgomery-form stored keys,
+// plain 128-bit reduction of canonical seeded ones
+template <bool SA>
+__device__ __forceinline__ uint64_t reduce_a_sum(const U128& x, const DevPrime& p) {
+    if constexpr (SA)
+        return reduce128(x, p);
+    else
+        return csub(redc_lazy(x.hi, x.lo, p.q, p.qinv_neg), p.q);
+}
+
+template <int ND, bool HOIST, bool SA>
 __global__ void __launch_bounds__(256, 5)  // 5 blocks per SM: more loads in flight than at 4
     k_ks_inner(const uint64_t* __restrict__ ext, PtrList din, GalList gal, PtrList keys, IdxList xsrc,
-               uint64_t* __restrict__ u, int n_rows, int level, int L, int LK, int n_ext,
+               uint64_t* __restrict__ u, int n_rows, int level, int L, int LK, int n_ext, int key_digits,
                const DevPrime* __restrict__ pr, const FpMod* __restrict__ fpm, ModupArgs a, int logn) {
     const int N = 1 << logn;
     const int i = blockIdx.x, t = blockIdx.z;
@@ -338,9 +391,9 @@ __global__ void __launch_bounds__(256, 5)  // 5 blocks per SM: more loads in fli
                 xs[j] = __ldg(reinterpret_cast<const ulonglong2*>(e + c));
             }
         }
-        kbs[j] = __ldg(reinterpret_cast<const ulonglong2*>(key + (((size_t)j * 2 + 0) * LK + krow) * N + c));
-        kas[j] = __ldg(reinterpret_cast<const ulonglong2*>(key + (((size_t)j * 2 + 1) * LK + krow) * N + c));
+        load_key_halves<ND, SA>(key, j, krow, LK, N, c, kbs[j], kas[j]);
     }
+    if constexpr (SA) seeded_a_halves<ND>(key, key_digits, krow, LK, N, c, p.q, kas);
     ulonglong2 ob, oa;
     if (fp) {
         const FpMod m = fpm[pidx];
@@ -350,8 +403,8 @@ __global__ void __launch_bounds__(256, 5)  // 5 blocks per SM: more loads in fli
             const double x0 = u2d(xs[j].x), x1 = u2d(xs[j].y);
             b0 = __dadd_rn(b0, fp_mulmod_s(x0, __longlong_as_double((long long)kbs[j].x), m));
             b1 = __dadd_rn(b1, fp_mulmod_s(x1, __longlong_as_double((long long)kbs[j].y), m));
-            a0 = __dadd_rn(a0, fp_mulmod_s(x0, __longlong_as_double((long long)kas[j].x), m));
-            a1 = __dadd_rn(a1, fp_mulmod_s(x1, __longlong_as_double((long long)kas[j].y), m));
+            a0 = __dadd_rn(a0, fp_mulmod_s(x0, key_a_fp<SA>(kas[j].x), m));
+            a1 = __dadd_rn(a1, fp_mulmod_s(x1, key_a_fp<SA>(kas[j].y), m));
         }
         ob = make_ulonglong2(d2u(fp_canon(b0, m)), d2u(fp_canon(b1, m)));
         oa = make_ulonglong2(d2u(fp_canon(a0, m)), d2u(fp_canon(a1, m)));
@@ -366,12 +419,92 @@ __global__ void __launch_bounds__(256, 5)  // 5 blocks per SM: more loads in fli
         }
         ob = make_ulonglong2(csub(redc_lazy(b0.hi, b0.lo, p.q, p.qinv_neg), p.q),
                              csub(redc_lazy(b1.hi, b1.lo, p.q, p.qinv_neg), p.q));
-        oa = make_ulonglong2(csub(redc_lazy(a0.hi, a0.lo, p.q, p.qinv_neg), p.q),
-                             csub(redc_lazy(a1.hi, a1.lo, p.q, p.qinv_neg), p.q));
+        oa = make_ulonglong2(reduce_a_sum<SA>(a0, p), reduce_a_sum<SA>(a1, p));
     }
     uint64_t* o = u + ((size_t)i * 2 * n_rows) * N + c;
     *reinterpret_cast<ulonglong2*>(o + (size_t)t * N) = ob;
     *reinterpret_cast<ulonglong2*>(o + (size_t)(n_rows + t) * N) = oa;
+}
+
+// The inner product of k_ks_inner for a group of key switches that share one
+// key (and so one Galois element): block x covers entries grp[x] ..
+// grp[x + 1] - 1 (the last group ends at n).  Each thread reads (or, SA,
+// regenerates) its key words once and applies them to every entry of the
+// group in turn, instead of once per entry.
+template <int ND, bool HOIST, bool SA>
+__global__ void __launch_bounds__(256, 4)
+    k_ks_inner_grp(const uint64_t* __restrict__ ext, PtrList din, GalList gal, PtrList keys, IdxList xsrc,
+                   IdxList grp, int n_grp, int n, uint64_t* __restrict__ u, int n_rows, int level, int L, int LK,
+                   int n_ext, int key_digits, const DevPrime* __restrict__ pr, const FpMod* __restrict__ fpm,
+                   ModupArgs a, int logn) {
+    const int N = 1 << logn;
+    const int g = blockIdx.x, t = blockIdx.z;
+    const int c = 2 * (blockIdx.y * blockDim.x + threadIdx.x);  // positions c, c+1
+    if (c >= N) return;
+    const int i0 = grp.i[g], i1 = g + 1 < n_grp ? grp.i[g + 1] : n;
+    const uint64_t* key = keys.p[i0];
+    const int own = automorph_src(c, logn, gal.g[i0]);  // the pair maps onto {own & ~1, own | 1}
+    const bool own_sw = own & 1;
+    const int krow = t < level ? t : L + (t - level);
+    const int pidx = a.tprime[t];
+    const DevPrime p = pr[pidx];
+    const bool fp = p.q < kFpPrimeLimit;
+    ulonglong2 kbs[ND], kas[ND];
+#pragma unroll
+    for (int j = 0; j < ND; j++) load_key_halves<ND, SA>(key, j, krow, LK, N, c, kbs[j], kas[j]);
+    if constexpr (SA) seeded_a_halves<ND>(key, key_digits, krow, LK, N, c, p.q, kas);
+    for (int i = i0; i < i1; i++) {
+        ulonglong2 xs[ND];
+#pragma unroll
+        for (int j = 0; j < ND; j++) {
+            const int s0 = a.src_row[j], ns = a.n_src[j];
+            if (t >= s0 && t < s0 + ns) {
+                const ulonglong2 v =
+                    __ldg(reinterpret_cast<const ulonglong2*>(din.p[i] + (size_t)t * N + (own & ~1)));
+                xs[j] = own_sw ? make_ulonglong2(v.y, v.x) : v;
+            } else {
+                const int pos = t < s0 ? t : t - ns;
+                const uint64_t* e =
+                    ext + ((size_t)a.ext_off[j] * n_ext + (size_t)(HOIST ? xsrc.i[i] : i) * (n_rows - ns) + pos) * N;
+                if (HOIST) {
+                    const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2*>(e + (own & ~1)));
+                    xs[j] = own_sw ? make_ulonglong2(v.y, v.x) : v;
+                } else {
+                    xs[j] = __ldg(reinterpret_cast<const ulonglong2*>(e + c));
+                }
+            }
+        }
+        ulonglong2 ob, oa;
+        if (fp) {
+            const FpMod m = fpm[pidx];
+            double b0 = 0.0, b1 = 0.0, a0 = 0.0, a1 = 0.0;
+#pragma unroll
+            for (int j = 0; j < ND; j++) {
+                const double x0 = u2d(xs[j].x), x1 = u2d(xs[j].y);
+                b0 = __dadd_rn(b0, fp_mulmod_s(x0, __longlong_as_double((long long)kbs[j].x), m));
+                b1 = __dadd_rn(b1, fp_mulmod_s(x1, __longlong_as_double((long long)kbs[j].y), m));
+                a0 = __dadd_rn(a0, fp_mulmod_s(x0, key_a_fp<SA>(kas[j].x), m));
+                a1 = __dadd_rn(a1, fp_mulmod_s(x1, key_a_fp<SA>(kas[j].y), m));
+            }
+            ob = make_ulonglong2(d2u(fp_canon(b0, m)), d2u(fp_canon(b1, m)));
+            oa = make_ulonglong2(d2u(fp_canon(a0, m)), d2u(fp_canon(a1, m)));
+        } else {
+            U128 b0 = {0, 0}, b1 = {0, 0}, a0 = {0, 0}, a1 = {0, 0};
+#pragma unroll
+            for (int j = 0; j < ND; j++) {
+                mac128(b0, xs[j].x, kbs[j].x);
+                mac128(b1, xs[j].y, kbs[j].y);
+                mac128(a0, xs[j].x, kas[j].x);
+                mac128(a1, xs[j].y, kas[j].y);
+            }
+            ob = make_ulonglong2(csub(redc_lazy(b0.hi, b0.lo, p.q, p.qinv_neg), p.q),
+                                 csub(redc_lazy(b1.hi, b1.lo, p.q, p.qinv_neg), p.q));
+            oa = make_ulonglong2(reduce_a_sum<SA>(a0, p), reduce_a_sum<SA>(a1, p));
+        }
+        uint64_t* o = u + ((size_t)i * 2 * n_rows) * N + c;
+        *reinterpret_cast<ulonglong2*>(o + (size_t)t * N) = ob;
+        *reinterpret_cast<ulonglong2*>(o + (size_t)(n_rows + t) * N) = oa;
+    }
 }
 
 // Sum of G key inner products per output, for one ModDown of the sum:
@@ -382,10 +515,10 @@ __global__ void __launch_bounds__(256, 5)  // 5 blocks per SM: more loads in fli
 // signed products of all G switches (|sum| <= G ND 5q/8 < 2^51 for G <= 64,
 // ND <= 15); integer rows reduce each switch's 128-bit sum once and add the
 // results, kept in [0, 2q).
-template <int ND, bool HOIST>
+template <int ND, bool HOIST, bool SA>
 __global__ void __launch_bounds__(256, 4)
     k_ks_inner_sum(const uint64_t* __restrict__ ext, PtrList din, GalList gal, PtrList keys, IdxList xsrc, int G,
-                   uint64_t* __restrict__ u, int n_rows, int level, int L, int LK, int n_ext,
+                   uint64_t* __restrict__ u, int n_rows, int level, int L, int LK, int n_ext, int key_digits,
                    const DevPrime* __restrict__ pr, const FpMod* __restrict__ fpm, ModupArgs a, int logn) {
     const int N = 1 << logn;
     const int o = blockIdx.x, t = blockIdx.z;
@@ -422,17 +555,17 @@ __global__ void __launch_bounds__(256, 4)
                     xs[j] = __ldg(reinterpret_cast<const ulonglong2*>(e + c));
                 }
             }
-            kbs[j] = __ldg(reinterpret_cast<const ulonglong2*>(key + (((size_t)j * 2 + 0) * LK + krow) * N + c));
-            kas[j] = __ldg(reinterpret_cast<const ulonglong2*>(key + (((size_t)j * 2 + 1) * LK + krow) * N + c));
+            load_key_halves<ND, SA>(key, j, krow, LK, N, c, kbs[j], kas[j]);
         }
+        if constexpr (SA) seeded_a_halves<ND>(key, key_digits, krow, LK, N, c, p.q, kas);
         if (fp) {
 #pragma unroll
             for (int j = 0; j < ND; j++) {
                 const double x0 = u2d(xs[j].x), x1 = u2d(xs[j].y);
                 fb0 = __dadd_rn(fb0, fp_mulmod_s(x0, __longlong_as_double((long long)kbs[j].x), m));
                 fb1 = __dadd_rn(fb1, fp_mulmod_s(x1, __longlong_as_double((long long)kbs[j].y), m));
-                fa0 = __dadd_rn(fa0, fp_mulmod_s(x0, __longlong_as_double((long long)kas[j].x), m));
-                fa1 = __dadd_rn(fa1, fp_mulmod_s(x1, __longlong_as_double((long long)kas[j].y), m));
+                fa0 = __dadd_rn(fa0, fp_mulmod_s(x0, key_a_fp<SA>(kas[j].x), m));
+                fa1 = __dadd_rn(fa1, fp_mulmod_s(x1, key_a_fp<SA>(kas[j].y), m));
             }
         } else {
             U128 b0 = {0, 0}, b1 = {0, 0}, a0 = {0, 0}, a1 = {0, 0};
@@ -446,8 +579,8 @@ __global__ void __launch_bounds__(256, 4)
             const uint64_t q2 = 2 * p.q;
             ib0 = csub(ib0 + redc_lazy(b0.hi, b0.lo, p.q, p.qinv_neg), q2);
             ib1 = csub(ib1 + redc_lazy(b1.hi, b1.lo, p.q, p.qinv_neg), q2);
-            ia0 = csub(ia0 + redc_lazy(a0.hi, a0.lo, p.q, p.qinv_neg), q2);
-            ia1 = csub(ia1 + redc_lazy(a1.hi, a1.lo, p.q, p.qinv_neg), q2);
+            ia0 = csub(ia0 + reduce_a_sum<SA>(a0, p), q2);
+            ia1 = csub(ia1 + reduce_a_sum<SA>(a1, p), q2);
         }
     }
     ulonglong2 ob, oa;
@@ -833,26 +966,49 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
 
     prof_begin(c, HE_PROF_KS_INNER);
     const int gx2 = (N / 2 + TB - 1) / TB;  // two positions per thread
-    switch (nd) {
-#define HE_KS_CASE(D)                                                                                             \
-    case D:                                                                                                       \
-        if (summed && hoist)                                                                                      \
-            k_ks_inner_sum<D, true><<<dim3(n_md, gx2, n_rows), blk, 0, c->stream>>>(                              \
-                ext, din, gal, keys, xsrc, G, u, n_rows, level, L, LK, nm, c->d_prime, c->d_fpmod, ma, c->log_n); \
-        else if (summed)                                                                                          \
-            k_ks_inner_sum<D, false><<<dim3(n_md, gx2, n_rows), blk, 0, c->stream>>>(                             \
-                ext, din, gal, keys, xsrc, G, u, n_rows, level, L, LK, nm, c->d_prime, c->d_fpmod, ma, c->log_n); \
-        else if (hoist)                                                                                           \
-            k_ks_inner<D, true><<<dim3(n, gx2, n_rows), blk, 0, c->stream>>>(                                     \
-                ext, din, gal, keys, xsrc, u, n_rows, level, L, LK, nm, c->d_prime, c->d_fpmod, ma, c->log_n);    \
-        else                                                                                                      \
-            k_ks_inner<D, false><<<dim3(n, gx2, n_rows), blk, 0, c->stream>>>(                                    \
-                ext, din, gal, keys, xsrc, u, n_rows, level, L, LK, nm, c->d_prime, c->d_fpmod, ma, c->log_n);    \
+    const int kd = he_key_digits(c);
+    // groups of adjacent entries that share a key, at most kKsGroupMax each
+    IdxList grp;
+    int n_grp = 0;
+    for (int i = 0; i < n; i++)
+        if (i == 0 || io.key[i] != io.key[i - 1] || i - grp.i[n_grp - 1] >= kKsGroupMax) grp.i[n_grp++] = i;
+    // single entries keep the lighter per-entry kernel (48 registers, five
+    // blocks per SM against four)
+    const bool grouped = !summed && n_grp < n;
+    switch (nd * 2 + (keys_seeded_a(c) ? 1 : 0)) {
+#define HE_KS_LAUNCH(D, SA)                                                                                        \
+    if (summed && hoist)                                                                                           \
+        k_ks_inner_sum<D, true, SA><<<dim3(n_md, gx2, n_rows), blk, 0, c->stream>>>(                               \
+            ext, din, gal, keys, xsrc, G, u, n_rows, level, L, LK, nm, kd, c->d_prime, c->d_fpmod, ma, c->log_n);  \
+    else if (summed)                                                                                               \
+        k_ks_inner_sum<D, false, SA><<<dim3(n_md, gx2, n_rows), blk, 0, c->stream>>>(                              \
+            ext, din, gal, keys, xsrc, G, u, n_rows, level, L, LK, nm, kd, c->d_prime, c->d_fpmod, ma, c->log_n);  \
+    else if (grouped && hoist)                                                                                     \
+        k_ks_inner_grp<D, true, SA><<<dim3(n_grp, gx2, n_rows), blk, 0, c->stream>>>(                              \
+            ext, din, gal, keys, xsrc, grp, n_grp, n, u, n_rows, level, L, LK, nm, kd, c->d_prime, c->d_fpmod, ma, \
+            c->log_n);                                                                                             \
+    else if (grouped)                                                                                              \
+        k_ks_inner_grp<D, false, SA><<<dim3(n_grp, gx2, n_rows), blk, 0, c->stream>>>(                             \
+            ext, din, gal, keys, xsrc, grp, n_grp, n, u, n_rows, level, L, LK, nm, kd, c->d_prime, c->d_fpmod, ma, \
+            c->log_n);                                                                                             \
+    else if (hoist)                                                                                                \
+        k_ks_inner<D, true, SA><<<dim3(n, gx2, n_rows), blk, 0, c->stream>>>(                                      \
+            ext, din, gal, keys, xsrc, u, n_rows, level, L, LK, nm, kd, c->d_prime, c->d_fpmod, ma, c->log_n);     \
+    else                                                                                                           \
+        k_ks_inner<D, false, SA><<<dim3(n, gx2, n_rows), blk, 0, c->stream>>>(                                     \
+            ext, din, gal, keys, xsrc, u, n_rows, level, L, LK, nm, kd, c->d_prime, c->d_fpmod, ma, c->log_n);
+#define HE_KS_CASE(D)         \
+    case 2 * D:               \
+        HE_KS_LAUNCH(D, false) \
+        break;                \
+    case 2 * D + 1:           \
+        HE_KS_LAUNCH(D, true)  \
         break;
         HE_KS_CASE(1) HE_KS_CASE(2) HE_KS_CASE(3) HE_KS_CASE(4) HE_KS_CASE(5) HE_KS_CASE(6) HE_KS_CASE(7)
         HE_KS_CASE(8) HE_KS_CASE(9) HE_KS_CASE(10) HE_KS_CASE(11) HE_KS_CASE(12) HE_KS_CASE(13) HE_KS_CASE(14)
         HE_KS_CASE(15)
 #undef HE_KS_CASE
+#undef HE_KS_LAUNCH
         default:
             return set_err(c, HE_EINVAL, "key switch: %d digits unsupported", nd);
     }
@@ -865,8 +1021,9 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
         std::vector<const uint64_t*> kd(io.key.begin(), io.key.begin() + n);
         std::sort(kd.begin(), kd.end());
         const double n_keys = (double)(std::unique(kd.begin(), kd.end()) - kd.begin());
+        const double key_halves = keys_seeded_a(c) ? 1.0 : 2.0;  // a-halves regenerated, not read
         prof_end(c, HE_PROF_KS_INNER,
-                 ((double)nm * nd * n_rows + n_keys * 2.0 * nd * n_rows + 2.0 * n_md * n_rows) * limbB,
+                 ((double)nm * nd * n_rows + n_keys * key_halves * nd * n_rows + 2.0 * n_md * n_rows) * limbB,
                  (double)n * n_rows * N * 2.0 * nd, (double)n * fp_rows_ks * N * 2.0 * nd);
     }
 

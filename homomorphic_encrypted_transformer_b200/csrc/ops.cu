@@ -5,6 +5,7 @@
 #include <algorithm>
 
 #include "he_internal.h"
+#include "keyseed.cuh"
 #include "ntt.cuh"
 
 namespace he {
@@ -75,7 +76,7 @@ __global__ void k_keygen_digit(const uint64_t* __restrict__ a, const uint64_t* _
     uint64_t b = sub_mod(e[k], as, p.q);
     if (g.v[r].x) b = add_mod(b, mul_shoup(sp[k], g.v[r].x, g.v[r].y, p.q), p.q);
     kb[k] = key_store_form(b, p);
-    ka[k] = key_store_form(av, p);
+    if (ka) ka[k] = key_store_form(av, p);
 }
 
 // canonical residues of a stored key
@@ -87,6 +88,26 @@ __global__ void k_key_canonical(const uint64_t* __restrict__ in, uint64_t* __res
     DevPrime p = pr[r % rows_per_poly];
     size_t k = (size_t)r * N + c;
     out[k] = p.q < kFpPrimeLimit ? (uint64_t)__longlong_as_double((long long)in[k]) : mont_mul(in[k], 1, p);
+}
+
+// canonical residues of a key with seeded a-halves, out [digits][2][LK][N]:
+// b from its stored rows, a regenerated from the stream starts after them
+__global__ void k_key_canonical_seeded(const uint64_t* __restrict__ in, uint64_t* __restrict__ out, int LK, int nd,
+                                       const DevPrime* __restrict__ pr, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x, R = blockIdx.y;
+    if (c >= N) return;
+    const int r = R % LK, half = (R / LK) & 1, j = R / (2 * LK);
+    const DevPrime p = pr[r];
+    uint64_t v;
+    if (half == 0) {
+        const uint64_t w = in[((size_t)j * LK + r) * N + c];
+        v = p.q < kFpPrimeLimit ? (uint64_t)__longlong_as_double((long long)w) : mont_mul(w, 1, p);
+    } else {
+        const uint64_t s0 = in[(size_t)nd * LK * N + (size_t)j * LK + r];
+        v = seeded_a(s0, c, N, p.q, __clzll(p.q));
+    }
+    out[(size_t)R * N + c] = v;
 }
 
 
@@ -451,14 +472,33 @@ using namespace he;
 
 extern "C" int he_key_digits(const he_ctx* c) { return c ? (c->L + c->alpha - 1) / c->alpha : HE_EINVAL; }
 
-extern "C" int he_keygen_upload(he_ctx* c, int kind, int32_t step, const int8_t* s, const uint64_t* a,
-                                const int32_t* e) {
+namespace he {
+bool keys_seeded_a(const he_ctx* c) {
+    if (c->relin.d) return c->relin.seeded_a;
+    return !c->rot_keys.empty() && c->rot_keys.begin()->second.seeded_a;
+}
+}  // namespace he
+
+// Does the context hold keys of the other form than seeded_a?
+static bool key_form_clash(const he_ctx* c, bool seeded_a) {
+    if (c->relin.d && c->relin.seeded_a != seeded_a) return true;
+    for (const auto& kv : c->rot_keys)
+        if (kv.second.seeded_a != seeded_a) return true;
+    return false;
+}
+
+// One switching key from host draws.  s0 (host [nd][LK], or null): the key
+// keeps only its b-halves and these stream starts of its seeded a-halves.
+static int keygen_one(he_ctx* c, int kind, int32_t step, const int8_t* s, const uint64_t* a, const int32_t* e,
+                      const uint64_t* s0) {
     if (!c) return HE_EINVAL;
     if (!s || !a || !e || (kind != HE_KEY_ROTATION && kind != HE_KEY_RELIN))
         return set_err(c, HE_EINVAL, "he_keygen_upload: bad arguments");
     const int N = c->N, LK = c->L + c->K, nd = he_key_digits(c);
     const uint64_t galois = kind == HE_KEY_ROTATION ? galois_elt(c, step) : 0;
     if (kind == HE_KEY_ROTATION && galois == 1) return set_err(c, HE_EINVAL, "he_keygen_upload: identity rotation");
+    if (key_form_clash(c, s0 != nullptr))
+        return set_err(c, HE_EINVAL, "keygen: the context holds keys with %s a-halves", s0 ? "stored" : "seeded");
     for (int i = 0; i < N; i++)
         if (s[i] < -1 || s[i] > 1) return set_err(c, HE_EINVAL, "he_keygen_upload: secret not ternary");
     for (int j = 0; j < nd; j++)
@@ -495,7 +535,16 @@ extern "C" int he_keygen_upload(he_ctx* c, int kind, int32_t step, const int8_t*
     }
     if ((rc = lc(c, "keygen s'"))) return rc;
     Key key;
-    if ((rc = check_cuda(c, cudaMalloc(&key.d, (size_t)nd * 2 * LK * N * 8), "key allocation"))) return rc;
+    key.seeded_a = s0 != nullptr;
+    const int kw = key.seeded_a ? 1 : 2;  // stored halves per digit
+    const size_t key_words = (size_t)nd * kw * LK * N + (key.seeded_a ? (size_t)nd * LK : 0);
+    if ((rc = check_cuda(c, cudaMalloc(&key.d, key_words * 8), "key allocation"))) return rc;
+    if (key.seeded_a &&
+        (rc = check_cuda(c, cudaMemcpyAsync(key.d + (size_t)nd * LK * N, s0, (size_t)nd * LK * 8,
+                                            cudaMemcpyHostToDevice, c->stream), "key stream starts"))) {
+        cudaFree(key.d);
+        return rc;
+    }
     for (int j = 0; j < nd; j++) {
         RowSet rs_e = rowset_contig(e_ntt, LK, N, all);
         k_signed_to_res<<<dim3(gx, LK), TB, 0, c->stream>>>(e32 + (size_t)j * N, e_ntt, rs_e, c->d_prime, c->log_n);
@@ -510,9 +559,9 @@ extern "C" int he_keygen_upload(he_ctx* c, int kind, int32_t step, const int8_t*
             uint64_t v = in_digit ? c->h_Pmod[r] : 0;
             g.v[r] = make_ulonglong2(v, v ? h_shoup(v, c->primes[r]) : 0);
         }
-        k_keygen_digit<<<dim3(gx, LK), TB, 0, c->stream>>>(a_d, s_ntt, e_ntt, sp, g, key.d + (size_t)(2 * j) * LK * N,
-                                                           key.d + (size_t)(2 * j + 1) * LK * N, c->d_prime,
-                                                           c->log_n);
+        k_keygen_digit<<<dim3(gx, LK), TB, 0, c->stream>>>(
+            a_d, s_ntt, e_ntt, sp, g, key.d + (size_t)(kw * j) * LK * N,
+            key.seeded_a ? nullptr : key.d + (size_t)(kw * j + 1) * LK * N, c->d_prime, c->log_n);
         if ((rc = lc(c, "keygen digit"))) break;
         // the host arrays are read by the copies above: wait before reusing a_d
         if ((rc = check_cuda(c, cudaStreamSynchronize(c->stream), "keygen sync"))) break;
@@ -528,9 +577,24 @@ extern "C" int he_keygen_upload(he_ctx* c, int kind, int32_t step, const int8_t*
     return HE_OK;
 }
 
+extern "C" int he_keygen_upload(he_ctx* c, int kind, int32_t step, const int8_t* s, const uint64_t* a,
+                                const int32_t* e) {
+    return keygen_one(c, kind, step, s, a, e, nullptr);
+}
+
 extern "C" int he_keygen_seeded(he_ctx* c, uint64_t seed, const int32_t* rot_steps, int n_steps, int with_relin) {
+    return he_keygen_seeded_ex(c, seed, rot_steps, n_steps, with_relin, 0);
+}
+
+extern "C" int he_keygen_seeded_ex(he_ctx* c, uint64_t seed, const int32_t* rot_steps, int n_steps, int with_relin,
+                                   int flags) {
     if (!c) return HE_EINVAL;
+    if (flags & ~HE_KEYGEN_SEEDED_A) return set_err(c, HE_EINVAL, "he_keygen_seeded: unknown flags %d", flags);
+    const bool seeded_a = flags & HE_KEYGEN_SEEDED_A;
     if (n_steps < 0 || (n_steps > 0 && !rot_steps)) return set_err(c, HE_EINVAL, "he_keygen_seeded: bad step list");
+    if (key_form_clash(c, seeded_a))
+        return set_err(c, HE_EINVAL, "he_keygen_seeded: the context holds keys with %s a-halves",
+                       seeded_a ? "stored" : "seeded");
     for (int i = 0; i < n_steps; i++)
         if (galois_elt(c, rot_steps[i]) == 1)
             return set_err(c, HE_EINVAL, "he_keygen_seeded: step %d is the identity rotation", rot_steps[i]);
@@ -540,10 +604,15 @@ extern "C" int he_keygen_seeded(he_ctx* c, uint64_t seed, const int32_t* rot_ste
     std::vector<int32_t> e((size_t)nd * N);
     int rc = he_sample_secret(seed, c->log_n, s.data());
     if (rc) return set_err(c, rc, "he_keygen_seeded: secret");
+    std::vector<uint64_t> s0(seeded_a ? (size_t)nd * LK : 0);
     auto one = [&](int kind, int32_t step, uint64_t key_id) {
         int r = he_sample_key_draws(seed, key_id, c->log_n, c->primes.data(), LK, nd, a.data(), e.data());
+        if (!r && seeded_a) r = he_sample_key_a_seeded(seed, key_id, c->log_n, c->primes.data(), LK, nd, a.data());
         if (r) return set_err(c, r, "he_keygen_seeded: key draws");
-        return he_keygen_upload(c, kind, step, s.data(), a.data(), e.data());
+        if (seeded_a)
+            for (int j = 0; j < nd; j++)
+                for (int p = 0; p < LK; p++) s0[(size_t)j * LK + p] = seeded_a_stream_start(seed, key_id, j, p);
+        return keygen_one(c, kind, step, s.data(), a.data(), e.data(), seeded_a ? s0.data() : nullptr);
     };
     for (int i = 0; i < n_steps; i++)
         if ((rc = one(HE_KEY_ROTATION, rot_steps[i], galois_elt(c, rot_steps[i])))) return rc;
@@ -569,8 +638,12 @@ extern "C" int he_key_download(he_ctx* c, int kind, int32_t step, uint64_t* host
     uint64_t* tmp;
     int rc = scratch_slot(c, 2, words, &tmp);
     if (rc) return rc;
-    k_key_canonical<<<dim3((N + TB - 1) / TB, nd * 2 * LK), TB, 0, c->stream>>>(k->d, tmp, LK, c->d_prime,
-                                                                            c->log_n);
+    if (k->seeded_a)
+        k_key_canonical_seeded<<<dim3((N + TB - 1) / TB, nd * 2 * LK), TB, 0, c->stream>>>(k->d, tmp, LK, nd,
+                                                                                       c->d_prime, c->log_n);
+    else
+        k_key_canonical<<<dim3((N + TB - 1) / TB, nd * 2 * LK), TB, 0, c->stream>>>(k->d, tmp, LK, c->d_prime,
+                                                                                c->log_n);
     if ((rc = lc(c, "key download"))) return rc;
     rc = check_cuda(c, cudaMemcpyAsync(host_out, tmp, words * 8, cudaMemcpyDeviceToHost, c->stream), "key D2H");
     if (rc) return rc;

@@ -24,6 +24,11 @@
 //    number of T_i <= x.  The table is computed in quad precision; the
 //    oracle computes it with exact decimal arithmetic and a test compares
 //    the two.
+//  * Seeded a-halves (keys that store only b): tag 4, one stream per digit
+//    and prime; coefficient i takes outputs 1 + i + t N, t = 0..63, the
+//    first whose top bitlen(q) bits are < q (if none, the last one's top bits
+//    minus q).  Any coefficient is computed alone, so the kernels regenerate
+//    a where they use it (keyseed.cuh).
 #include <quadmath.h>
 #include <stdint.h>
 
@@ -59,6 +64,25 @@ static uint64_t obj_id(uint64_t tag, uint64_t key_id, uint64_t digit, uint64_t p
 }
 
 static int bitlen(uint64_t q) { return 64 - __builtin_clzll(q); }
+
+constexpr uint64_t kTagSeededA = 4;
+constexpr int kSeededTries = 64;
+
+// Output k (k >= 1) of the stream that starts at state s0.
+static uint64_t output_at(uint64_t s0, uint64_t k) { return mix64(s0 + kGamma * k); }
+
+static void seeded_a_row(uint64_t s0, uint64_t q, uint64_t* out, int n) {
+    const int sh = 64 - bitlen(q);
+    for (int i = 0; i < n; i++) {
+        uint64_t x = 0;
+        bool ok = false;
+        for (int t = 0; t < kSeededTries && !ok; t++) {
+            x = output_at(s0, 1 + (uint64_t)i + (uint64_t)t * n) >> sh;
+            ok = x < q;
+        }
+        out[i] = ok ? x : x - q;
+    }
+}
 
 static void uniform(Stream& st, uint64_t q, uint64_t* out, int n) {
     const int sh = 64 - bitlen(q);
@@ -116,6 +140,12 @@ static void gaussian(Stream& st, int32_t* out, int n) {
 
 using namespace he_sampler;
 
+namespace he {
+uint64_t seeded_a_stream_start(uint64_t seed, uint64_t key_id, int digit, int prime_index) {
+    return stream(seed, obj_id(kTagSeededA, key_id, digit, prime_index)).state;
+}
+}  // namespace he
+
 extern "C" int he_gaussian_cdt(uint64_t* out) {
     if (!out) return HE_EINVAL;
     const uint64_t* t = cdt_table();
@@ -146,5 +176,20 @@ extern "C" int he_sample_key_draws(uint64_t seed, uint64_t key_id, int log_n, co
         Stream se = stream(seed, obj_id(3, key_id, j, 0));
         gaussian(se, e_out + (size_t)j * N, N);
     }
+    return HE_OK;
+}
+
+extern "C" int he_sample_key_a_seeded(uint64_t seed, uint64_t key_id, int log_n, const uint64_t* primes, int n_primes,
+                                      int digits, uint64_t* a_out) {
+    if (!primes || !a_out || log_n < 1 || log_n > 20 || n_primes < 1 || n_primes > 255 || digits < 1 ||
+        digits > 255 || key_id >= (1ull << 32))
+        return HE_EINVAL;
+    for (int r = 0; r < n_primes; r++)
+        if (primes[r] < 2) return HE_EINVAL;
+    const int N = 1 << log_n;
+    for (int j = 0; j < digits; j++)
+        for (int r = 0; r < n_primes; r++)
+            seeded_a_row(stream(seed, obj_id(kTagSeededA, key_id, j, r)).state, primes[r],
+                         a_out + ((size_t)j * n_primes + r) * N, N);
     return HE_OK;
 }

@@ -29,6 +29,7 @@ HE_ECUDA = -6
 HE_ETIMEOUT = -7
 HE_KEY_ROTATION = 0
 HE_KEY_RELIN = 1
+HE_KEYGEN_SEEDED_A = 1
 
 PROF = {"ntt_fwd_cols": 0, "ntt_fwd_rows": 1, "ntt_inv_rows": 2, "ntt_inv_cols": 3, "modup": 4, "ks_inner": 5,
         "moddown_conv": 6, "moddown_combine": 7, "automorph": 8, "elementwise": 9, "rescale": 10, "pmult": 11}
@@ -77,6 +78,8 @@ _sig("he_get_psi", _i, _vp, _u64p)
 _sig("he_keygen_upload", _i, _vp, _i, ctypes.c_int32, _vp, _vp, _vp)
 _sig("he_key_download", _i, _vp, _i, ctypes.c_int32, _vp)
 _sig("he_keygen_seeded", _i, _vp, ctypes.c_uint64, _vp, _i, _i)
+_sig("he_keygen_seeded_ex", _i, _vp, ctypes.c_uint64, _vp, _i, _i, _i)
+_sig("he_sample_key_a_seeded", _i, ctypes.c_uint64, ctypes.c_uint64, _i, _vp, _i, _i, _vp)
 _sig("he_sample_secret", _i, ctypes.c_uint64, _i, _vp)
 _sig("he_sample_key_draws", _i, ctypes.c_uint64, ctypes.c_uint64, _i, _vp, _i, _i, _vp, _vp)
 _sig("he_gaussian_cdt", _i, _vp)
@@ -251,6 +254,12 @@ def he_keygen_seeded(ctx, seed, rot_steps, with_relin):
     _check(ctx, _lib.he_keygen_seeded(ctx.ptr, int(seed), _ptr(st), len(st), 1 if with_relin else 0))
 
 
+def he_keygen_seeded_ex(ctx, seed, rot_steps, with_relin, flags):
+    st = np.ascontiguousarray(list(rot_steps), dtype=np.int32)
+    _check(ctx, _lib.he_keygen_seeded_ex(ctx.ptr, int(seed), _ptr(st), len(st), 1 if with_relin else 0,
+                                         int(flags)))
+
+
 def he_sample_secret(seed, log_n):
     """Host-only: the ternary secret of a seed (int8[2^log_n])."""
     out = np.empty(1 << log_n, dtype=np.int8)
@@ -271,6 +280,16 @@ def he_sample_key_draws(seed, key_id, log_n, primes, digits):
     if rc != HE_OK:
         raise HEError(rc, "he_sample_key_draws: bad arguments")
     return a, e
+
+
+def he_sample_key_a_seeded(seed, key_id, log_n, primes, digits):
+    """Host-only: the seeded a-half of one key, [digits][len(primes)][N] uint64."""
+    pr = np.ascontiguousarray(primes, dtype=np.uint64)
+    a = np.empty((digits, len(pr), 1 << log_n), dtype=np.uint64)
+    rc = _lib.he_sample_key_a_seeded(int(seed), int(key_id), int(log_n), _ptr(pr), len(pr), int(digits), _ptr(a))
+    if rc != HE_OK:
+        raise HEError(rc, "he_sample_key_a_seeded: bad arguments")
+    return a
 
 
 def he_gaussian_cdt():

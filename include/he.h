@@ -156,6 +156,26 @@ int he_keygen_upload(he_ctx* ctx, int kind, int32_t step, const int8_t* s, const
  * b_j = -a_j s + e_j + P [prime in digit j] s'.
  */
 int he_keygen_seeded(he_ctx* ctx, uint64_t seed, const int32_t* rot_steps, int n_steps, int with_relin);
+/*
+ * he_keygen_seeded with flags.  HE_KEYGEN_SEEDED_A: every key keeps only its
+ * b-half (plus one 8-byte stream start per digit and prime) and the
+ * key-switching kernels regenerate the uniform a-half where they read it
+ * (the optional seeded a-halves of the hoisted-rotation design: half the key
+ * bytes in HBM and per key switch).  a_j is then drawn by the counter rule
+ * below instead of the sequential stream of tag 2; s and e are drawn as
+ * above, and b_j = -a_j s + e_j + P [prime in digit j] s' as before.
+ *  - stream start s0 = mix64(seed + 0x9E3779B97F4A7C15 (1 + obj)),
+ *    obj = 4 2^56 + key_id 2^24 + digit 2^8 + prime_index;
+ *  - coefficient i (evaluation-domain storage index) of that row is the
+ *    first x_t = mix64(s0 + 0x9E3779B97F4A7C15 (1 + i + t N)) >> (64 -
+ *    bitlen(q)), t = 0..63, with x_t < q, or x_63 - q if there is none.
+ * All keys of a context have one form: HE_EINVAL if the context already
+ * holds keys of the other form (he_keygen_upload makes stored-a keys).
+ * he_key_download returns such a key whole (a regenerated on the device).
+ */
+#define HE_KEYGEN_SEEDED_A 1
+int he_keygen_seeded_ex(he_ctx* ctx, uint64_t seed, const int32_t* rot_steps, int n_steps, int with_relin,
+                        int flags);
 /* Host only (no context, no device): the ternary secret of a seed, int8[N] (N = 2^log_n). */
 int he_sample_secret(uint64_t seed, int log_n, int8_t* s_out);
 /* Host only: the random parts of one switching key as he_keygen_seeded draws
@@ -163,6 +183,11 @@ int he_sample_secret(uint64_t seed, int log_n, int8_t* s_out);
  * e int32 [digits][N].  key_id < 2^32. */
 int he_sample_key_draws(uint64_t seed, uint64_t key_id, int log_n, const uint64_t* primes, int n_primes, int digits,
                         uint64_t* a_out, int32_t* e_out);
+/* Host only: the a-half of one key as HE_KEYGEN_SEEDED_A defines it,
+ * uint64 [digits][n_primes][N] (row r uniform mod primes[r], prime_index r).
+ * key_id < 2^32. */
+int he_sample_key_a_seeded(uint64_t seed, uint64_t key_id, int log_n, const uint64_t* primes, int n_primes,
+                           int digits, uint64_t* a_out);
 /* Host only: the 38 thresholds T_i = floor(2^64 C_i) of the error sampler,
  * C_i = P(e <= -19 + i) for the discrete Gaussian of sigma 3.2 on [-19, 19]. */
 int he_gaussian_cdt(uint64_t* out);

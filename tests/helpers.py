@@ -95,3 +95,49 @@ class Setup:
 def random_rows(seed, mods, n_polys, N):
     """[n_polys][len(mods)][N] canonical residues."""
     return S.uniform_residues(seed, "ntt_residues", mods, N, lead=(n_polys,))
+
+
+class SeededASetup(Setup):
+    """Setup whose keys come from he_keygen_seeded_ex(HE_KEYGEN_SEEDED_A):
+    the secret and key errors of the library's stated sampler, a-halves by
+    its counter rule (the keys store only b).  The oracle builds the same
+    keys from oracle/sampler.py."""
+
+    def __init__(self, log_n, L, K, dnum, seed):
+        from oracle import sampler as R
+
+        super().__init__(log_n, L, K, dnum, seed)
+        self.s = R.secret(seed, self.P.N)
+        pa, pe = S.public_key_draws(seed, self.P.q, self.P.N)
+        self.pk = C.public_key(self.s, pa, pe, self.P)
+
+    def key_draws(self, key_id):
+        from oracle import sampler as R
+
+        P = self.P
+        return (R.key_a_seeded(self.seed, key_id, P.mods, P.N, P.dnum),
+                R.key_errors(self.seed, key_id, P.N, P.dnum))
+
+    def upload_rot(self, step):
+        he = lib()
+        he.he_keygen_seeded_ex(self.ctx, self.seed, [step], False, he.HE_KEYGEN_SEEDED_A)
+
+    def upload_relin(self):
+        he = lib()
+        he.he_keygen_seeded_ex(self.ctx, self.seed, [], True, he.HE_KEYGEN_SEEDED_A)
+
+    def stored_twin(self):
+        """A second context holding the same keys in stored form (both halves
+        uploaded through he_keygen_upload): its key switches must give the
+        same residues."""
+        he = lib()
+        twin = Setup.__new__(Setup)
+        twin.__dict__.update(self.__dict__)
+        twin.ctx = he.he_ctx_create(self.P.log_n, self.P.L, self.P.K, self.P.dnum)
+        twin._ok = self._ok
+        return twin
+
+    def upload_rot_stored(self, twin, step):
+        he = lib()
+        a, e = self.key_draws(self.P.galois_elt(step))
+        he.he_keygen_upload(twin.ctx, he.HE_KEY_ROTATION, step, self.s, a, e)

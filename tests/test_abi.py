@@ -107,3 +107,19 @@ def test_library_sampler_matches_the_oracle_sampler(he):
         assert (a == ra).all() and (e == re_).all()
     with pytest.raises(he.HEError):
         he.he_sample_key_draws(1, 1 << 32, 11, P.mods, 2)  # key id beyond 32 bits
+
+
+def test_library_seeded_a_matches_the_oracle(he):
+    """The seeded a-halves (HE_KEYGEN_SEEDED_A) of the library's host sampler
+    against the oracle's counter rule, including a modulus that forces
+    rejections (5 of the 8 values of its top three bits kept)."""
+    from oracle import sampler as R
+
+    P = C.Params(11, 4, 2, 2)
+    for key_id in (2, P.galois_elt(5)):
+        a = he.he_sample_key_a_seeded(0xC0FFEE, key_id, 11, P.mods, 2)
+        assert (a == R.key_a_seeded(0xC0FFEE, key_id, P.mods, P.N, 2)).all()
+    a = he.he_sample_key_a_seeded(9, 4, 8, [5, 97], 3)
+    assert (a == R.key_a_seeded(9, 4, [5, 97], 256, 3)).all()
+    with pytest.raises(he.HEError):
+        he.he_sample_key_a_seeded(1, 1 << 32, 11, P.mods, 2)
