@@ -70,6 +70,8 @@ __global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
 // each in turn): 16 measured best, by a little, for the rotation batch,
 // hoisted rotations and relinearisation batches (caps of 1 to 16 tried).
 constexpr int kKsGroupMax = 16;
+// Outputs per thread of k_ks_inner_sum_mo.
+constexpr int kKsSumMo = 4;
 
 struct ModupArgs {
     int n_digits;
@@ -596,6 +598,118 @@ __global__ void __launch_bounds__(256, 4)
     *reinterpret_cast<ulonglong2*>(out + (size_t)(n_rows + t) * N) = oa;
 }
 
+// The hoisted k_ks_inner_sum for MO outputs whose G terms use the same keys
+// term by term (key of term g of output o = key of term g of output o0, as
+// in the rotate-and-sum of several ciphertexts over one step list): one
+// position per thread; each key word (or, SA, its regeneration) and each
+// automorphism index serves all MO outputs of a term.  Block x covers
+// outputs MO x .. MO x + MO - 1.  Measured against k_ks_inner_sum, this
+// form wins for hoisted sums, whose terms gather from shared raised digits,
+// and loses for plain sums (BSGS giant steps), whose per-term digits are
+// the bulk of the reads and lose their 16-byte pair loads here.
+template <int ND, bool SA, int MO>
+__global__ void __launch_bounds__(256, 4)
+    k_ks_inner_sum_mo(const uint64_t* __restrict__ ext, PtrList din, GalList gal, PtrList keys, IdxList xsrc, int G,
+                      uint64_t* __restrict__ u, int n_rows, int level, int L, int LK, int n_ext, int key_digits,
+                      const DevPrime* __restrict__ pr, const FpMod* __restrict__ fpm, ModupArgs a, int logn) {
+    const int N = 1 << logn;
+    const int o0 = blockIdx.x * MO, t = blockIdx.z;
+    const int c = blockIdx.y * blockDim.x + threadIdx.x;
+    if (c >= N) return;
+    const int krow = t < level ? t : L + (t - level);
+    const int pidx = a.tprime[t];
+    const DevPrime p = pr[pidx];
+    constexpr int KW = SA ? 1 : 2;  // stored halves per digit
+    // x_{r,j} at this thread's position (digit j's own rows through sigma_r)
+    auto load_x = [&](int r, int own, int j) -> uint64_t {
+        const int s0 = a.src_row[j], ns = a.n_src[j];
+        if (t >= s0 && t < s0 + ns) return __ldg(din.p[r] + (size_t)t * N + own);
+        const int pos = t < s0 ? t : t - ns;
+        return __ldg(ext + ((size_t)a.ext_off[j] * n_ext + (size_t)xsrc.i[r] * (n_rows - ns) + pos) * N + own);
+    };
+    uint64_t* out0 = u + ((size_t)o0 * 2 * n_rows) * N + c;
+    const size_t ostride = (size_t)2 * n_rows * N;
+    if (p.q < kFpPrimeLimit) {
+        const FpMod m = fpm[pidx];
+        double fb[MO], fa[MO];
+#pragma unroll
+        for (int o = 0; o < MO; o++) fb[o] = fa[o] = 0.0;
+        for (int g = 0; g < G; g++) {
+            const int r0 = o0 * G + g;
+            const uint64_t* key = keys.p[r0];
+            const int own = automorph_src(c, logn, gal.g[r0]);
+            double kb[ND], ka[ND];
+#pragma unroll
+            for (int j = 0; j < ND; j++) {
+                kb[j] = __longlong_as_double((long long)__ldg(key + ((size_t)j * KW * LK + krow) * N + c));
+                if constexpr (!SA)
+                    ka[j] = __longlong_as_double((long long)__ldg(key + ((size_t)(j * KW + 1) * LK + krow) * N + c));
+            }
+            if constexpr (SA) {
+                const uint64_t* s0p = key + (size_t)key_digits * LK * N + krow;
+                const int sh = __clzll(p.q);
+#pragma unroll
+                for (int j = 0; j < ND; j++) ka[j] = u2d(seeded_a(__ldg(s0p + (size_t)j * LK), c, N, p.q, sh));
+            }
+#pragma unroll
+            for (int o = 0; o < MO; o++) {
+                const int r = r0 + o * G;
+#pragma unroll
+                for (int j = 0; j < ND; j++) {
+                    const double x = u2d(load_x(r, own, j));
+                    fb[o] = __dadd_rn(fb[o], fp_mulmod_s(x, kb[j], m));
+                    fa[o] = __dadd_rn(fa[o], fp_mulmod_s(x, ka[j], m));
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 0; o < MO; o++) {
+            out0[o * ostride + (size_t)t * N] = d2u(fp_canon(fb[o], m));
+            out0[o * ostride + (size_t)(n_rows + t) * N] = d2u(fp_canon(fa[o], m));
+        }
+    } else {
+        const uint64_t q2 = 2 * p.q;
+        uint64_t ib[MO], ia[MO];
+#pragma unroll
+        for (int o = 0; o < MO; o++) ib[o] = ia[o] = 0;
+        for (int g = 0; g < G; g++) {
+            const int r0 = o0 * G + g;
+            const uint64_t* key = keys.p[r0];
+            const int own = automorph_src(c, logn, gal.g[r0]);
+            uint64_t kb[ND], ka[ND];
+#pragma unroll
+            for (int j = 0; j < ND; j++) {
+                kb[j] = __ldg(key + ((size_t)j * KW * LK + krow) * N + c);
+                if constexpr (!SA) ka[j] = __ldg(key + ((size_t)(j * KW + 1) * LK + krow) * N + c);
+            }
+            if constexpr (SA) {
+                const uint64_t* s0p = key + (size_t)key_digits * LK * N + krow;
+                const int sh = __clzll(p.q);
+#pragma unroll
+                for (int j = 0; j < ND; j++) ka[j] = seeded_a(__ldg(s0p + (size_t)j * LK), c, N, p.q, sh);
+            }
+#pragma unroll
+            for (int o = 0; o < MO; o++) {
+                const int r = r0 + o * G;
+                U128 b = {0, 0}, aa = {0, 0};
+#pragma unroll
+                for (int j = 0; j < ND; j++) {
+                    const uint64_t x = load_x(r, own, j);
+                    mac128(b, x, kb[j]);
+                    mac128(aa, x, ka[j]);
+                }
+                ib[o] = csub(ib[o] + redc_lazy(b.hi, b.lo, p.q, p.qinv_neg), q2);
+                ia[o] = csub(ia[o] + reduce_a_sum<SA>(aa, p), q2);
+            }
+        }
+#pragma unroll
+        for (int o = 0; o < MO; o++) {
+            out0[o * ostride + (size_t)t * N] = csub(ib[o], p.q);
+            out0[o * ostride + (size_t)(n_rows + t) * N] = csub(ia[o], p.q);
+        }
+    }
+}
+
 // tmp[i][poly][r][c] = sum_k y'_k (P/p_k mod q_r), y_k = [x_k (P/p_k)^-1]_{p_k},
 // y'_k = y_k or y_k - p_k (centred, |y'_k| < 2^59).  Two arithmetic paths:
 //  - FP64 (targets below 2^41): with y'_k = a_k 2^40 + b_k 2^20 + c_k
@@ -975,9 +1089,18 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     // single entries keep the lighter per-entry kernel (48 registers, five
     // blocks per SM against four)
     const bool grouped = !summed && n_grp < n;
+    // hoisted sums whose outputs, kKsSumMo at a time, use the same key term
+    // by term (rotate-and-sum of several ciphertexts over one step list)
+    bool sum_mo = summed && hoist && n_md % kKsSumMo == 0;
+    for (int o = 0; sum_mo && o < n_md; o++)
+        for (int g = 0; g < G && sum_mo; g++)
+            sum_mo = io.key[(size_t)o * G + g] == io.key[(size_t)(o - o % kKsSumMo) * G + g];
     switch (nd * 2 + (keys_seeded_a(c) ? 1 : 0)) {
 #define HE_KS_LAUNCH(D, SA)                                                                                        \
-    if (summed && hoist)                                                                                           \
+    if (sum_mo)                                                                                                    \
+        k_ks_inner_sum_mo<D, SA, kKsSumMo><<<dim3(n_md / kKsSumMo, gx, n_rows), blk, 0, c->stream>>>(             \
+            ext, din, gal, keys, xsrc, G, u, n_rows, level, L, LK, nm, kd, c->d_prime, c->d_fpmod, ma, c->log_n);  \
+    else if (summed && hoist)                                                                                      \
         k_ks_inner_sum<D, true, SA><<<dim3(n_md, gx2, n_rows), blk, 0, c->stream>>>(                               \
             ext, din, gal, keys, xsrc, G, u, n_rows, level, L, LK, nm, kd, c->d_prime, c->d_fpmod, ma, c->log_n);  \
     else if (summed)                                                                                               \
