@@ -1085,7 +1085,9 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     IdxList grp;
     int n_grp = 0;
     for (int i = 0; i < n; i++)
-        if (i == 0 || io.key[i] != io.key[i - 1] || i - grp.i[n_grp - 1] >= kKsGroupMax) grp.i[n_grp++] = i;
+        if (i == 0 || io.key[i] != io.key[i - 1] || io.galois[i] != io.galois[i - 1] ||
+            i - grp.i[n_grp - 1] >= kKsGroupMax)
+            grp.i[n_grp++] = i;
     // single entries keep the lighter per-entry kernel (48 registers, five
     // blocks per SM against four)
     const bool grouped = !summed && n_grp < n;
@@ -1093,8 +1095,10 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     // by term (rotate-and-sum of several ciphertexts over one step list)
     bool sum_mo = summed && hoist && n_md % kKsSumMo == 0;
     for (int o = 0; sum_mo && o < n_md; o++)
-        for (int g = 0; g < G && sum_mo; g++)
-            sum_mo = io.key[(size_t)o * G + g] == io.key[(size_t)(o - o % kKsSumMo) * G + g];
+        for (int g = 0; g < G && sum_mo; g++) {
+            const size_t r = (size_t)o * G + g, r0 = (size_t)(o - o % kKsSumMo) * G + g;
+            sum_mo = io.key[r] == io.key[r0] && io.galois[r] == io.galois[r0];
+        }
     switch (nd * 2 + (keys_seeded_a(c) ? 1 : 0)) {
 #define HE_KS_LAUNCH(D, SA)                                                                                        \
     if (sum_mo)                                                                                                    \
