@@ -711,7 +711,8 @@ def workload_case(case, n_steps, n_warmup, cpu_seconds, local_rank, probes=None,
             he.he_hmult_relin_rescale(ctx, xc, xc, he.Ciphertext(r, 3, 2.0 ** 40))
 
         metric, unit, per_step = "tiny-config operation sequences/s (N=2^12)", "sequences/s", 1
-        cfg = {"workload": case, "N": N, "ops": "NTT round trip, 3 rotations, 1 HMult-relin-rescale"}
+        cfg = {"workload": case, "N": N, "ops": "NTT round trip, 3 rotations, 1 HMult-relin-rescale",
+               "l2": "inputs L2-resident (a latency-bound sequence of small launches)"}
 
     for _ in range(n_warmup):
         step()
@@ -729,6 +730,22 @@ def workload_case(case, n_steps, n_warmup, cpu_seconds, local_rank, probes=None,
     t1.record(stream)
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1)
+    if case == "tiny":
+        # launch-bound: the same sequence captured once as a CUDA graph and
+        # replayed (the eager calls above sized the scratch); value = replay
+        ms_eager = ms
+        graph = capture_graph(he, ctx, step, stream)
+        graph.replay()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(n_steps):
+            graph.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1)
+        del graph
+        cfg["cuda_graph"] = "value: one captured sequence replayed per step; eager_value: the calls issued one by one"
+        cfg["eager_value"] = per_step * n_steps / (ms_eager * 1e-3)
     clk = clocks.stop()
     he.he_profile_enable(ctx, True)
     for _ in range(n_steps):
@@ -753,6 +770,28 @@ def workload_case(case, n_steps, n_warmup, cpu_seconds, local_rank, probes=None,
     if with_cpu:
         line["cpu_baseline"] = workload_cpu_baseline(case, cpu_seconds)
     return line
+
+
+def capture_graph(he, ctx, step, stream):
+    """step() captured as one CUDA graph on a side stream (the context's
+    calls enqueue there during the capture), for replay on `stream`."""
+    import torch
+
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    he.he_set_stream(ctx, cap)
+    try:
+        with torch.cuda.stream(cap):
+            g.capture_begin()
+            try:
+                step()
+            finally:
+                g.capture_end()
+    finally:
+        he.he_set_stream(ctx, stream)
+    stream.wait_stream(cap)
+    return g
 
 
 # the other workloads of the default run: (warm-up steps, timed steps) each.

@@ -154,6 +154,13 @@ static int upload(he_ctx* c, T** p, const std::vector<T>& h, const char* what) {
 
 int scratch_slot(he_ctx* c, int slot, size_t words, uint64_t** out) {
     if (words > c->scratch_words[slot]) {
+        // growing synchronises and allocates, which a stream capture cannot hold
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(c->stream, &cs) == cudaSuccess && cs != cudaStreamCaptureStatusNone)
+            return set_err(c, HE_EINVAL,
+                           "scratch slot %d must grow to %zu words during a stream capture: run the call once "
+                           "before capturing it",
+                           slot, words);
         if (c->scratch[slot]) {
             cudaStreamSynchronize(c->stream);
             cudaFree(c->scratch[slot]);

@@ -103,6 +103,18 @@ int he_derive_primes(const he_params* params, uint64_t* primes_out, uint64_t* ps
  * (identical residues; slower than the default FP64 kernel on B200). */
 int he_ctx_create(const he_params* params, void* cuda_stream, he_ctx** out);
 int he_ctx_destroy(he_ctx* ctx);
+/*
+ * Later calls enqueue on cuda_stream.  CUDA graph capture: the operation
+ * calls (transforms, rotations, HMult, rescale, the BSGS product, the
+ * degree-15 evaluation, attention, the helpers) launch kernels and record
+ * events only, so a sequence of them can be captured on the context's
+ * stream and replayed, provided each call already ran once eagerly with
+ * the same sizes (that run sizes the context's scratch).  A call that would
+ * have to grow its scratch while the stream is being captured returns
+ * HE_EINVAL before any CUDA work, leaving the capture intact.  Key
+ * generation, key download, the host-buffer entry point, he_sync and
+ * profiling synchronise and cannot be captured.
+ */
 int he_set_stream(he_ctx* ctx, void* cuda_stream);
 /* Blocks until the context's stream is idle; returns HE_ECUDA on a pending error. */
 int he_sync(he_ctx* ctx);
