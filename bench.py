@@ -767,6 +767,8 @@ def workload_case(case, n_steps, n_warmup, cpu_seconds, local_rank, probes=None,
             "clocks": clk}
     if seeded_a:
         cfg["keys"] = "seeded a-halves: b stored, a regenerated in the key inner product"
+    if case == "ps15":
+        line["hmrr_per_s"] = line["value"] * cfg["hmrr_per_eval"]
     if with_cpu:
         line["cpu_baseline"] = workload_cpu_baseline(case, cpu_seconds)
     return line
@@ -975,6 +977,9 @@ def run_native(args, rank, world, local_rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "u64", "data": "synthetic",
             "config": line_config(world, args.seeded_a),
             "hbm_roofline_frac_of_step": hbm_frac_step,
+            # the same with every rotation reading its own key (no reuse across the batch)
+            "hbm_roofline_frac_no_key_reuse": (N_CTS * (key_bytes + 2 * ct_bytes) / (ms_plain * 1e-3 / args.steps))
+            / 1e9 / hbm_peak,
             "alu_ideal_ms_per_step": alu_ideal_ms,
             "alu_roofline_frac_of_step": alu_ideal_ms / (ms_plain / args.steps),
             "roofline": roof,
