@@ -232,8 +232,11 @@ extern "C" int he_pmult_accum_bsgs(he_ctx* c, const he_ct* x, int n_in, const ui
     if (bs > 1 && (rc = rotate_hoisted_many(c, x, n_groups * n_in, bsteps.data(), bs - 1, bout.data()))) return rc;
 
     const size_t pt_block = (size_t)n_in * gs * bs * level * N;
-    // one token group: 2 columns per thread; several: 4 groups staged per pass
-    const int tch = n_groups == 1 ? 1 : 4, cpt = n_groups == 1 ? 2 : 1;
+    // one token group: 2 columns per thread.  Several: 2 groups staged per
+    // pass, measured against 1, 3 and 4 for FFN1 at 2048 tokens (190 ms of
+    // products against 225, 193 and 214): with 4 the 98 KB of staging leaves
+    // 2 blocks per SM; with 1 the weights are re-read 16 times and bind.
+    const int tch = n_groups == 1 ? 1 : 2, cpt = tch == 1 ? 2 : 1;
     const int smem = tch * n_in * bs * 2 * kPmThreadsX * cpt * 8;
     if (smem > 200 * 1024) return set_err(c, HE_EINVAL, "he_pmult_accum_bsgs: n_in*bs = %d too large", n_in * bs);
     const int gpt = 2;  // giant steps per thread
@@ -251,8 +254,8 @@ extern "C" int he_pmult_accum_bsgs(he_ctx* c, const he_ct* x, int n_in, const ui
                 k_pmult_accum<1, 2, 2><<<pgrid, kPmThreadsX * kPmG, smem, c->stream>>>(
                     pti, B, Zi, n_groups, n_in, gs, bs, level, c->d_prime, c->d_fpmod, c->log_n);
             } else {
-                cudaFuncSetAttribute(k_pmult_accum<4, 1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-                k_pmult_accum<4, 1, 2><<<pgrid, kPmThreadsX * kPmG, smem, c->stream>>>(
+                cudaFuncSetAttribute(k_pmult_accum<2, 1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+                k_pmult_accum<2, 1, 2><<<pgrid, kPmThreadsX * kPmG, smem, c->stream>>>(
                     pti, B, Zi, n_groups, n_in, gs, bs, level, c->d_prime, c->d_fpmod, c->log_n);
             }
             c->launches++;
