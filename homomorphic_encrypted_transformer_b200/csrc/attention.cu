@@ -163,29 +163,21 @@ extern "C" int he_attention_output(he_ctx* c, const he_ct* a, const he_ct* v, in
 
     const size_t N = c->N, ctv = (size_t)2 * lv * N, cta = (size_t)2 * la * N;
     uint64_t* pool;
-    if ((rc = scratch_slot(c, 3, ctv * nz.size() + cta * n_off * 2, &pool))) return rc;
-    uint64_t* dropped = pool + ctv * nz.size();
-    uint64_t* prod = dropped + cta * n_off;
-    // rot_delta(v) for the non-zero offsets, hoisted, then dropped to the weights' level
+    if ((rc = scratch_slot(c, 3, ctv * nz.size() + cta * n_off, &pool))) return rc;
+    uint64_t* prod = pool + ctv * nz.size();
+    // rot_delta(v) for the non-zero offsets, hoisted; the products read them
+    // at the weights' level in place
     std::vector<he_ct> rv(nz.size());
     for (size_t j = 0; j < nz.size(); j++) rv[j] = he_ct{pool + j * ctv, lv, v->scale, 1};
     if (!nz.empty() && (rc = rotate_hoisted_many(c, v, 1, nz.data(), (int)nz.size(), rv.data()))) return rc;
-    std::vector<const uint64_t*> src, A, B;
-    std::vector<uint64_t*> dst, P;
+    std::vector<const uint64_t*> A, B;
+    std::vector<uint64_t*> P;
     for (int i = 0; i < n_off; i++) {
-        const uint64_t* vi = pos[i] < 0 ? v->data : rv[pos[i]].data;
-        if (lv > la) {
-            src.push_back(vi);
-            dst.push_back(dropped + cta * i);
-            B.push_back(dropped + cta * i);
-        } else {
-            B.push_back(vi);
-        }
+        B.push_back(pos[i] < 0 ? v->data : rv[pos[i]].data);
         A.push_back(a[i].data);
         P.push_back(prod + cta * i);
     }
-    if (!src.empty() && (rc = drop_many(c, src, dst, lv, la))) return rc;
-    if ((rc = hmrr_many(c, A, B, P, la))) return rc;
+    if ((rc = hmrr_many(c, A, B, P, la, la, lv))) return rc;
     // sum of the products, halving the list each round
     int m = n_off;
     while (m > 1) {

@@ -190,13 +190,19 @@ int rotate_sum_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t*
 constexpr int kScratchSlots = 5;
 int scratch_slot(he_ctx* c, int slot, size_t words, uint64_t** out);
 
-// out[i] = rescale(in[i]) for n ciphertexts at `level` (out may equal in).
-int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int level);
+// out[i] = rescale(in[i]) for n ciphertexts at `level` (out may equal in),
+// plus addend[i] (a ciphertext at level - 1) when addend is not empty.
+int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int level,
+                 const std::vector<const uint64_t*>& addend = {});
 // Batched helpers of the drivers (ops.cu): HMult + relinearisation + rescale
-// of pairs at `level`; out_i = a_i + b_i at lv limbs (out may equal a);
-// out_i = in_i keeping limbs < lv (out != in).
+// of pairs at `level` (a_i, b_i with at least `level` limbs per polynomial:
+// their c1 starts at limb room_a / room_b, 0 = level; out_i may be a_i or
+// b_i of the same i; plus addend_i at level - 1 when addend is not empty); out_i = a_i +
+// b_i at lv limbs (out may equal a); out_i = in_i keeping limbs < lv (out !=
+// in).
 int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector<const uint64_t*>& b,
-              const std::vector<uint64_t*>& out, int level);
+              const std::vector<uint64_t*>& out, int level, int room_a = 0, int room_b = 0,
+              const std::vector<const uint64_t*>& addend = {});
 int add_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector<const uint64_t*>& b,
              const std::vector<uint64_t*>& o, int lv);
 int drop_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int lin, int lv);

@@ -137,8 +137,10 @@ __global__ void k_rescale_lift(const uint64_t* __restrict__ last, uint64_t* __re
 // Rescale, step 3: out_i[poly][r] = (in_i[poly][r] - lift[i][poly][r]) q_l^-1.
 // out_i = in_i is not allowed here (the limb shift of c1 would overwrite
 // unread input); callers route in-place rescales through a staging buffer.
+// (with_add: plus addend_i, a ciphertext at level - 1, added after the rescale)
 __global__ void k_rescale_combine(PtrList in, const uint64_t* __restrict__ lift, MutPtrList out, int level,
-                                  const ulonglong2* __restrict__ qinv, const DevPrime* __restrict__ pr, int logn) {
+                                  const ulonglong2* __restrict__ qinv, PtrList addend, int with_add,
+                                  const DevPrime* __restrict__ pr, int logn) {
     const int N = 1 << logn;
     int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y, ip = blockIdx.z;
     if (c >= N) return;
@@ -147,7 +149,44 @@ __global__ void k_rescale_combine(PtrList in, const uint64_t* __restrict__ lift,
     uint64_t x = in.p[i][((size_t)poly * level + r) * N + c];
     uint64_t y = lift[((size_t)ip * lm1 + r) * N + c];
     ulonglong2 w = qinv[r];
-    out.p[i][((size_t)poly * lm1 + r) * N + c] = mul_shoup(x + q - y, w.x, w.y, q);
+    const size_t k = ((size_t)poly * lm1 + r) * N + c;
+    uint64_t v = mul_shoup(x + q - y, w.x, w.y, q);
+    if (with_add) v = add_mod(addend.p[i][k], v, q);
+    out.p[i][k] = v;
+}
+
+// The rescale of K x (x at level lin dropped to lv limbs), optionally added
+// into out and with an integer constant added to c0, in the launches of one
+// rescale: the gather multiplies the last limb by K and the combine each
+// limb, then adds.  The same modular operations in the same order as
+// mul_const_many, rescale_many, add_many and add_const_many one after the
+// other, without the intermediate ciphertexts in HBM.
+__global__ void k_rescale_gather_last_k(PtrList in, uint64_t* __restrict__ last, int lin, int lv, RowConst kc,
+                                        const DevPrime* __restrict__ pr, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x, poly = blockIdx.y, i = blockIdx.z;
+    if (c >= N) return;
+    const int r = lv - 1;
+    const uint64_t x = in.p[i][((size_t)poly * lin + r) * N + c];
+    last[((size_t)i * 2 + poly) * N + c] = mul_shoup(x, kc.v[r].x, kc.v[r].y, pr[r].q);
+}
+
+__global__ void k_rescale_combine_k(PtrList in, const uint64_t* __restrict__ lift, MutPtrList out, int lin, int lv,
+                                    RowConst kc, const ulonglong2* __restrict__ qinv, int accumulate, RowConst k0,
+                                    int add_k0, const DevPrime* __restrict__ pr, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y, ip = blockIdx.z;
+    if (c >= N) return;
+    const int lm1 = lv - 1, i = ip >> 1, poly = ip & 1;
+    const uint64_t q = pr[r].q;
+    const uint64_t x = mul_shoup(in.p[i][((size_t)poly * lin + r) * N + c], kc.v[r].x, kc.v[r].y, q);
+    const uint64_t y = lift[((size_t)ip * lm1 + r) * N + c];
+    const ulonglong2 w = qinv[r];
+    uint64_t v = mul_shoup(x + q - y, w.x, w.y, q);
+    uint64_t* o = out.p[i] + ((size_t)poly * lm1 + r) * N + c;
+    if (accumulate) v = add_mod(*o, v, q);
+    if (add_k0 && poly == 0) v = add_mod(v, k0.v[r].x, q);
+    *o = v;
 }
 
 // dst_i[k] = src_i[k], k < words (16-byte copies)
@@ -203,8 +242,10 @@ __global__ void k_add_const_many(MutPtrList io, RowConst kc, const DevPrime* __r
 }
 
 // d_i = (a0 b0, a0 b1 + a1 b0, a1 b1) of the pairs (a_i, b_i), [3][level][N]
-__global__ void k_tensor_many(PtrList pa, PtrList pb, MutPtrList pd, int level, const DevPrime* __restrict__ pr,
-                              int logn) {
+// a_i and b_i hold level or more limbs per polynomial: their c1 starts at
+// limb room_a / room_b (the first `level` limbs of each polynomial are read)
+__global__ void k_tensor_many(PtrList pa, PtrList pb, MutPtrList pd, int level, int room_a, int room_b,
+                              const DevPrime* __restrict__ pr, int logn) {
     const int N = 1 << logn;
     int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y, i = blockIdx.z;
     if (c >= N) return;
@@ -212,8 +253,8 @@ __global__ void k_tensor_many(PtrList pa, PtrList pb, MutPtrList pd, int level, 
     const uint64_t* b = pb.p[i];
     uint64_t* d = pd.p[i];
     DevPrime p = pr[r];
-    size_t k0 = (size_t)r * N + c, k1 = (size_t)(level + r) * N + c;
-    uint64_t a0 = a[k0], a1 = a[k1], b0 = b[k0], b1 = b[k1];
+    size_t k0 = (size_t)r * N + c;
+    uint64_t a0 = a[k0], a1 = a[(size_t)(room_a + r) * N + c], b0 = b[k0], b1 = b[(size_t)(room_b + r) * N + c];
     // Montgomery products a0 b0 R^-1 etc.; the sum is taken before the final
     // correction by R^2 R^-1.
     uint64_t m00 = mont_mul(a0, b0, p), m01 = mont_mul(a0, b1, p), m10 = mont_mul(a1, b0, p),
@@ -241,9 +282,12 @@ static int ct_ok(he_ctx* c, const he_ct* x, const char* what) {
     return HE_OK;
 }
 
-int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int level) {
+int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int level,
+                 const std::vector<const uint64_t*>& addend) {
     const int N = c->N, n = (int)in.size(), lm1 = level - 1;
     if (level < 2) return set_err(c, HE_ELEVEL, "rescale: level %d has no prime to drop", level);
+    const bool with_add = !addend.empty();
+    if (with_add && (int)addend.size() != n) return set_err(c, HE_EINVAL, "rescale: addend list length");
     const int gx = (N + TB - 1) / TB;
     const uint64_t ql = c->primes[level - 1];
     const double limbB = 8.0 * N;
@@ -257,11 +301,12 @@ int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::v
         uint64_t* last = base;
         uint64_t* lift = last + (size_t)2 * m * N;
         uint64_t* stage = lift + (size_t)2 * m * lm1 * N;
-        PtrList pin, sback;
+        PtrList pin, sback, padd;
         MutPtrList pout, dback;
         int n_back = 0;
         for (int i = 0; i < m; i++) {
             pin.p[i] = in[i0 + i];
+            padd.p[i] = with_add ? addend[i0 + i] : nullptr;
             const bool inplace = out[i0 + i] == in[i0 + i];
             pout.p[i] = inplace ? stage + (size_t)i * 2 * lm1 * N : out[i0 + i];
             if (inplace) {
@@ -284,10 +329,10 @@ int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::v
         if ((rc = ntt_fwd_set(c, rowset_contig(lift, lm1, N, prime_range(0, lm1)), 2 * m * lm1))) return rc;
         prof_begin(c, HE_PROF_RESCALE);
         k_rescale_combine<<<dim3(gx, lm1, 2 * m), TB, 0, c->stream>>>(pin, lift, pout, level,
-                                                                      c->d_rs_inv + (size_t)lm1 * c->L, c->d_prime,
-                                                                      c->log_n);
+                                                                      c->d_rs_inv + (size_t)lm1 * c->L, padd,
+                                                                      with_add ? 1 : 0, c->d_prime, c->log_n);
         if ((rc = lc(c, "rescale_combine"))) return rc;
-        prof_end(c, HE_PROF_RESCALE, 6.0 * m * lm1 * limbB, 2.0 * m * lm1 * N);
+        prof_end(c, HE_PROF_RESCALE, (with_add ? 8.0 : 6.0) * m * lm1 * limbB, 2.0 * m * lm1 * N);
         if (n_back) {
             prof_begin(c, HE_PROF_RESCALE);
             k_copy_many<<<dim3(c->sm_count * 4, n_back), TB, 0, c->stream>>>(sback, dback, (size_t)lm1 * N);
@@ -300,10 +345,14 @@ int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::v
 
 // HMult + relinearisation + rescale of n pairs at one level.
 int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector<const uint64_t*>& b,
-              const std::vector<uint64_t*>& out, int level) {
+              const std::vector<uint64_t*>& out, int level, int room_a, int room_b,
+              const std::vector<const uint64_t*>& addend) {
     const int N = c->N, n = (int)a.size();
     if (!c->relin.d) return set_err(c, HE_ENOKEY, "hmult: no relinearisation key");
     if (level < 2) return set_err(c, HE_ELEVEL, "hmult: level %d cannot be rescaled", level);
+    if (room_a == 0) room_a = level;
+    if (room_b == 0) room_b = level;
+    if (room_a < level || room_b < level) return set_err(c, HE_ELEVEL, "hmult: input room below level %d", level);
     const int gx = (N + TB - 1) / TB;
     const size_t per = (size_t)5 * level * N;  // d0 d1 d2 | relinearised [2][level]
     const int chunk = 64;
@@ -321,7 +370,8 @@ int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vecto
             pd.p[i] = base + per * i;
         }
         prof_begin(c, HE_PROF_ELEMENTWISE);
-        k_tensor_many<<<dim3(gx, level, m), TB, 0, c->stream>>>(pa, pb, pd, level, c->d_prime, c->log_n);
+        k_tensor_many<<<dim3(gx, level, m), TB, 0, c->stream>>>(pa, pb, pd, level, room_a, room_b, c->d_prime,
+                                                                c->log_n);
         if ((rc = lc(c, "tensor"))) return rc;
         prof_end(c, HE_PROF_ELEMENTWISE, 7.0 * m * level * 8.0 * N, 7.0 * m * level * N);
         for (int i = 0; i < m; i++) {
@@ -336,7 +386,9 @@ int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vecto
         if ((rc = key_switch_split(c, level, io))) return rc;
         std::vector<const uint64_t*> rin(io.out.begin(), io.out.end());
         std::vector<uint64_t*> rout(out.begin() + i0, out.begin() + i0 + m);
-        if ((rc = rescale_many(c, rin, rout, level))) return rc;
+        std::vector<const uint64_t*> radd;
+        if (!addend.empty()) radd.assign(addend.begin() + i0, addend.begin() + i0 + m);
+        if ((rc = rescale_many(c, rin, rout, level, radd))) return rc;
     }
     return HE_OK;
 }
@@ -370,6 +422,58 @@ int mul_const_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std:
         int rc = lc(c, "mul_const");
         if (rc) return rc;
         prof_end(c, HE_PROF_ELEMENTWISE, 4.0 * m * lv * 8.0 * c->N, 2.0 * m * lv * c->N);
+    }
+    return HE_OK;
+}
+
+// out_i (+)= rescale(K in_i dropped to lv limbs) at level lv - 1, and, with
+// add_k0, K0 added to c0 after that; in_i at level lin >= lv, out_i apart
+// from every in_i.  Equal, residue for residue, to mul_const_many into a
+// temporary, rescale_many of it, add_many into out_i (accumulate) and
+// add_const_many (add_k0), and two full passes over HBM cheaper.
+int mul_const_rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, int lin, int lv, int64_t K,
+                           const std::vector<uint64_t*>& out, bool accumulate, bool add_k0, int64_t K0) {
+    const int N = c->N, n = (int)in.size(), lm1 = lv - 1;
+    if (lv < 2 || lin < lv) return set_err(c, HE_ELEVEL, "rescale: level %d from %d", lv, lin);
+    const RowConst kc = row_const_shoup(c, lv, K);
+    RowConst k0;
+    for (int r = 0; r < lm1; r++) k0.v[r] = make_ulonglong2(add_k0 ? int_mod(K0, c->primes[r]) : 0, 0);
+    const int gx = (N + TB - 1) / TB;
+    const uint64_t ql = c->primes[lv - 1];
+    const double limbB = 8.0 * N;
+    for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
+        const int m = std::min(kMaxBatch, n - i0);
+        // per ciphertext: last limbs [2][N], lifts [2][lm1][N]
+        uint64_t* base;
+        int rc = scratch_slot(c, 1, (size_t)N * (2 + 2 * lm1) * m, &base);
+        if (rc) return rc;
+        uint64_t* last = base;
+        uint64_t* lift = last + (size_t)2 * m * N;
+        PtrList pin;
+        MutPtrList pout;
+        for (int i = 0; i < m; i++) {
+            pin.p[i] = in[i0 + i];
+            pout.p[i] = out[i0 + i];
+        }
+        prof_begin(c, HE_PROF_RESCALE);
+        k_rescale_gather_last_k<<<dim3(gx, 2, m), TB, 0, c->stream>>>(pin, last, lin, lv, kc, c->d_prime, c->log_n);
+        if ((rc = lc(c, "rescale_gather"))) return rc;
+        prof_end(c, HE_PROF_RESCALE, 4.0 * m * limbB, 2.0 * m * N);
+        std::vector<int> pl(1, lv - 1);
+        if ((rc = ntt_inv_set(c, rowset_contig(last, 1, N, pl), 2 * m))) return rc;
+        prof_begin(c, HE_PROF_RESCALE);
+        k_rescale_lift<<<dim3(gx, lm1, 2 * m), TB, 0, c->stream>>>(last, lift, lm1, ql,
+                                                                   c->d_rs_qmod + (size_t)lm1 * c->L, c->d_prime,
+                                                                   c->log_n);
+        if ((rc = lc(c, "rescale_lift"))) return rc;
+        prof_end(c, HE_PROF_RESCALE, (2.0 * m + 2.0 * m * lm1) * limbB, 2.0 * m * lm1 * N);
+        if ((rc = ntt_fwd_set(c, rowset_contig(lift, lm1, N, prime_range(0, lm1)), 2 * m * lm1))) return rc;
+        prof_begin(c, HE_PROF_RESCALE);
+        k_rescale_combine_k<<<dim3(gx, lm1, 2 * m), TB, 0, c->stream>>>(
+            pin, lift, pout, lin, lv, kc, c->d_rs_inv + (size_t)lm1 * c->L, accumulate ? 1 : 0, k0, add_k0 ? 1 : 0,
+            c->d_prime, c->log_n);
+        if ((rc = lc(c, "rescale_combine"))) return rc;
+        prof_end(c, HE_PROF_RESCALE, (accumulate ? 8.0 : 6.0) * m * lm1 * limbB, 4.0 * m * lm1 * N);
     }
     return HE_OK;
 }
@@ -748,8 +852,8 @@ extern "C" int he_poly_eval_ps15(he_ctx* c, const he_ct* x, int n, const double*
     if (l0 < 7) return set_err(c, HE_ELEVEL, "ps15: needs level >= 7, got %d", l0);
     if (!c->relin.d) return set_err(c, HE_ENOKEY, "ps15: no relinearisation key");
     const size_t ctw = (size_t)2 * l0 * N;  // room of one ciphertext at the top level
-    // per ciphertext: x2 x3 x4 acc prod term qsum tmp
-    const int nbuf = 8;
+    // per ciphertext: x2 x3 x4 acc qsum
+    const int nbuf = 5;
     uint64_t* pool = nullptr;
     int rc = scratch_slot(c, 3, ctw * nbuf * n, &pool);
     if (rc) return rc;
@@ -764,7 +868,7 @@ extern "C" int he_poly_eval_ps15(he_ctx* c, const he_ct* x, int n, const double*
         for (int i = 0; i < n; i++) v[i] = buf(k, i);
         return v;
     };
-    enum { X2, X3, X4, ACC, PROD, TERM, QSUM, TMP };
+    enum { X2, X3, X4, ACC, QSUM };
     std::vector<const uint64_t*> xd(n);
     for (int i = 0; i < n; i++) xd[i] = x[i].data;
     double sx = x[0].scale;
@@ -772,9 +876,8 @@ extern "C" int he_poly_eval_ps15(he_ctx* c, const he_ct* x, int n, const double*
     if ((rc = hmrr_many(c, xd, xd, bufs(X2), l0))) goto done;
     {
         double s2 = (sx * sx) / (double)c->primes[l0 - 1];
-        // x3 = HMRR(x2, drop(x, l0-1))
-        if ((rc = drop_many(c, xd, bufs(TMP), l0, l0 - 1))) goto done;
-        if ((rc = hmrr_many(c, cbufs(X2), cbufs(TMP), bufs(X3), l0 - 1))) goto done;
+        // x3 = HMRR(x2, drop(x, l0-1)): x read at level l0-1 in place
+        if ((rc = hmrr_many(c, cbufs(X2), xd, bufs(X3), l0 - 1, l0 - 1, l0))) goto done;
         double s3 = (s2 * sx) / (double)c->primes[l0 - 2];
         // x4 = HMRR(x2, x2)
         if ((rc = hmrr_many(c, cbufs(X2), cbufs(X2), bufs(X4), l0 - 1))) goto done;
@@ -785,34 +888,38 @@ extern "C" int he_poly_eval_ps15(he_ctx* c, const he_ct* x, int n, const double*
         // q_blk(x) at (lam, T) into dst buffers (level lam): each x^j dropped
         // to lam+1 and multiplied by its integer constant in one pass, then
         // rescaled; the constant term added last
+        // (the multiply, rescale, sum and constant of each term in the
+        // launches of one rescale: mul_const_rescale_many)
         auto build_q = [&](int blk, int lam, double T, int dst) -> int {
             int r;
+            const int64_t K0 = (int64_t)round_half_away(coeffs[4 * blk] * T);
             for (int j = 1; j <= 3; j++) {
                 double cj = coeffs[4 * blk + j];
                 double v = cj * T * (double)c->primes[lam] / pw_scale[j];
                 int64_t K = (int64_t)round_half_away(v);
                 const std::vector<const uint64_t*> src = j == 1 ? xd : cbufs(j == 2 ? X2 : X3);
-                if ((r = mul_const_many(c, src, bufs(TMP), pw_level[j], lam + 1, K))) return r;
-                if ((r = rescale_many(c, cbufs(TMP), bufs(j == 1 ? dst : TERM), lam + 1))) return r;
-                if (j > 1 && (r = add_many(c, cbufs(dst), cbufs(TERM), bufs(dst), lam))) return r;
+                if ((r = mul_const_rescale_many(c, src, pw_level[j], lam + 1, K, bufs(dst), j > 1, j == 3, K0)))
+                    return r;
             }
-            int64_t K0 = (int64_t)round_half_away(coeffs[4 * blk] * T);
-            return add_const_many(c, bufs(dst), lam, K0);
+            return HE_OK;
         };
         int lev = l0 - 3;
         double T = top_scale;
         if ((rc = build_q(3, lev, T, ACC))) goto done;
+        std::vector<uint64_t*> od(n);
+        for (int i = 0; i < n; i++) od[i] = out[i].data;
+        // acc <- HMRR(acc, drop(x4)) + q_blk: q_blk built first, x4 read at
+        // the accumulator's level in place, the sum taken in the rescale of
+        // the product, the last one written to the outputs
         for (int blk = 2; blk >= 0; blk--) {
-            if ((rc = drop_many(c, cbufs(X4), bufs(TMP), l0 - 2, lev))) goto done;
-            if ((rc = hmrr_many(c, cbufs(ACC), cbufs(TMP), bufs(PROD), lev))) goto done;
+            const int lev_in = lev;
             T = (T * s4) / (double)c->primes[lev - 1];
             lev -= 1;
             if ((rc = build_q(blk, lev, T, QSUM))) goto done;
-            if ((rc = add_many(c, cbufs(PROD), cbufs(QSUM), bufs(ACC), lev))) goto done;
+            if ((rc = hmrr_many(c, cbufs(ACC), cbufs(X4), blk == 0 ? od : bufs(ACC), lev_in, lev_in, l0 - 2,
+                                cbufs(QSUM))))
+                goto done;
         }
-        std::vector<uint64_t*> od(n);
-        for (int i = 0; i < n; i++) od[i] = out[i].data;
-        if ((rc = drop_many(c, cbufs(ACC), od, lev, lev))) goto done;
         for (int i = 0; i < n; i++) {
             out[i].level = lev;
             out[i].scale = T;
