@@ -1014,12 +1014,12 @@ NTT_SOURCES = ["homomorphic_encrypted_transformer_b200/csrc/ntt.cu", "homomorphi
 # one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the four
 # transform passes on 512 limbs of 2^16 words (bench.py --case ntt; each pass
 # reads and writes 268.4 MB of limbs), taken with the sources of this digest
-NTT_SHA256 = "478a41ef306750bed1e66e57a1c2ba3effdc31a1ca75c4a7a4e9080bad334180"
+NTT_SHA256 = "0eeb6e0dc51e6a7f1939d8cfd007c567a91aea1a08579ff357f1f62e1633ac71"
 NCU_TRAFFIC = {
-    "ntt_fwd_cols": {"ratio": (268578304 + 217961984) / 536870912.0, "sources": NTT_SOURCES, "sha256": NTT_SHA256},
-    "ntt_fwd_rows": {"ratio": (314841600 + 217830144) / 536870912.0, "sources": NTT_SOURCES, "sha256": NTT_SHA256},
-    "ntt_inv_rows": {"ratio": (311631104 + 212199424) / 536870912.0, "sources": NTT_SOURCES, "sha256": NTT_SHA256},
-    "ntt_inv_cols": {"ratio": (268576512 + 214450432) / 536870912.0, "sources": NTT_SOURCES, "sha256": NTT_SHA256},
+    "ntt_fwd_cols": {"ratio": (268579072 + 218044416) / 536870912.0, "sources": NTT_SOURCES, "sha256": NTT_SHA256},
+    "ntt_fwd_rows": {"ratio": (311915776 + 216503296) / 536870912.0, "sources": NTT_SOURCES, "sha256": NTT_SHA256},
+    "ntt_inv_rows": {"ratio": (313877760 + 213612800) / 536870912.0, "sources": NTT_SOURCES, "sha256": NTT_SHA256},
+    "ntt_inv_cols": {"ratio": (268575744 + 214055424) / 536870912.0, "sources": NTT_SOURCES, "sha256": NTT_SHA256},
 }
 
 

@@ -20,7 +20,7 @@ namespace he {
 
 static int ct_check(he_ctx* c, const he_ct* x, const char* what) {
     if (!x || !x->data) return set_err(c, HE_EINVAL, "%s: null ciphertext", what);
-    if ((uintptr_t)x->data & 15) return set_err(c, HE_EINVAL, "%s: ciphertext not 16-byte aligned", what);
+    if ((uintptr_t)x->data & 31) return set_err(c, HE_EINVAL, "%s: ciphertext not 32-byte aligned", what);
     if (x->level < 1 || x->level > c->L) return set_err(c, HE_ELEVEL, "%s: level %d out of range", what, x->level);
     if (!x->is_ntt) return set_err(c, HE_EDOMAIN, "%s: ciphertext not in the evaluation domain", what);
     return HE_OK;
@@ -94,7 +94,7 @@ extern "C" int he_attention_scores(he_ctx* c, const he_ct* q, const he_ct* k, in
         if ((rc = need_key(c, 2 * n_tok * h, what))) return rc;
     const size_t N = c->N, ctw = (size_t)2 * l * N, ctw1 = (size_t)2 * (l - 1) * N;
     for (int i = 0; i < n_off; i++)
-        if (!s[i].data || ((uintptr_t)s[i].data & 15)) return set_err(c, HE_EINVAL, "%s: null or unaligned output", what);
+        if (!s[i].data || ((uintptr_t)s[i].data & 31)) return set_err(c, HE_EINVAL, "%s: null or unaligned output", what);
     if ((rc = check_outputs(c, s, n_off, ctw1, {{q->data, ctw}, {k->data, ctw}}, what))) return rc;
     uint64_t* pool;
     if ((rc = scratch_slot(c, 3, ctw * nz.size() + ctw1 * n_off, &pool))) return rc;
@@ -141,7 +141,7 @@ extern "C" int he_attention_output(he_ctx* c, const he_ct* a, const he_ct* v, in
     if (!a || !out || !offsets || n_off < 1 || n_tok < 1) return set_err(c, HE_EINVAL, "%s: bad arguments", what);
     int rc;
     if ((rc = ct_check(c, v, what))) return rc;
-    if (!out->data || ((uintptr_t)out->data & 15)) return set_err(c, HE_EINVAL, "%s: null or unaligned output", what);
+    if (!out->data || ((uintptr_t)out->data & 31)) return set_err(c, HE_EINVAL, "%s: null or unaligned output", what);
     const int la = a[0].level, lv = v->level;
     for (int i = 0; i < n_off; i++) {
         if ((rc = ct_check(c, &a[i], what))) return rc;

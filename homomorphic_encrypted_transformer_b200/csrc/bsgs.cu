@@ -189,7 +189,7 @@ extern "C" int he_pmult_accum_bsgs(he_ctx* c, const he_ct* x, int n_in, const ui
         return set_err(c, HE_EINVAL, "he_pmult_accum_bsgs: bad arguments");
     const int level = x[0].level, N = c->N;
     for (int i = 0; i < n_groups * n_in; i++) {
-        if (!x[i].data || ((uintptr_t)x[i].data & 15) || !x[i].is_ntt) return set_err(c, HE_EINVAL, "he_pmult_accum_bsgs: bad input %d", i);
+        if (!x[i].data || ((uintptr_t)x[i].data & 31) || !x[i].is_ntt) return set_err(c, HE_EINVAL, "he_pmult_accum_bsgs: bad input %d", i);
         if (x[i].level != level) return set_err(c, HE_ELEVEL, "he_pmult_accum_bsgs: mixed levels");
     }
     for (int i = 0; i < n_groups * n_out; i++)

@@ -1281,7 +1281,7 @@ int key_switch_split(he_ctx* c, int level, const KsIoList& io) {
 
 static int ct_ok(he_ctx* c, const he_ct* x, const char* what) {
     if (!x || !x->data) return set_err(c, HE_EINVAL, "%s: null ciphertext", what);
-    if ((uintptr_t)x->data & 15) return set_err(c, HE_EINVAL, "%s: ciphertext not 16-byte aligned", what);
+    if ((uintptr_t)x->data & 31) return set_err(c, HE_EINVAL, "%s: ciphertext not 32-byte aligned", what);
     if (x->level < 1 || x->level > c->L) return set_err(c, HE_ELEVEL, "%s: level %d out of range", what, x->level);
     if (!x->is_ntt) return set_err(c, HE_EDOMAIN, "%s: ciphertext not in the evaluation domain", what);
     return HE_OK;
@@ -1296,7 +1296,7 @@ int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, in
         int rc = ct_ok(c, &in[i], "rotate");
         if (rc) return rc;
         if (in[i].level != level) return set_err(c, HE_ELEVEL, "rotate: mixed levels in a batch");
-        if (!out[i].data || ((uintptr_t)out[i].data & 15)) return set_err(c, HE_EINVAL, "rotate: null or unaligned output");
+        if (!out[i].data || ((uintptr_t)out[i].data & 31)) return set_err(c, HE_EINVAL, "rotate: null or unaligned output");
         if (out[i].data == in[i].data) return set_err(c, HE_EINVAL, "rotate: output aliases input");
     }
     // group by Galois element so that each key is streamed once per group
@@ -1363,7 +1363,7 @@ int rotate_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t* ste
         ins.insert(in[i].data);
     }
     for (long long o = 0; o < (long long)n_in * n_steps; o++) {
-        if (!out[o].data || ((uintptr_t)out[o].data & 15))
+        if (!out[o].data || ((uintptr_t)out[o].data & 31))
             return set_err(c, HE_EINVAL, "rotate_hoisted: null or unaligned output %lld", o);
         if (ins.count(out[o].data)) return set_err(c, HE_EINVAL, "rotate_hoisted: output %lld aliases an input", o);
     }
@@ -1476,7 +1476,7 @@ int rotate_sum_many(he_ctx* c, const he_ct* z, int n_out, int n_terms, const int
         ins.insert(base[o].data);
     }
     for (int o = 0; o < n_out; o++) {
-        if (!out[o].data || ((uintptr_t)out[o].data & 15))
+        if (!out[o].data || ((uintptr_t)out[o].data & 31))
             return set_err(c, HE_EINVAL, "rotate_sum: null or unaligned output %d", o);
         if (ins.count(out[o].data)) return set_err(c, HE_EINVAL, "rotate_sum: output %d aliases an input", o);
     }
@@ -1572,7 +1572,7 @@ int rotate_sum_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t*
         ins.insert(in[i].data);
     }
     for (int i = 0; i < n_in; i++) {
-        if (!out[i].data || ((uintptr_t)out[i].data & 15))
+        if (!out[i].data || ((uintptr_t)out[i].data & 31))
             return set_err(c, HE_EINVAL, "rotate_sum_hoisted: null or unaligned output %d", i);
         if (ins.count(out[i].data)) return set_err(c, HE_EINVAL, "rotate_sum_hoisted: output %d aliases an input", i);
     }

@@ -28,8 +28,20 @@
 
 namespace he {
 
+// The centred last limb x (coefficients mod q_l) onto every q_r of a chunk:
+// out[r] = [x]_{q_r} - (x > q_l/2 ? q_l : 0)  (pointers and tables offset to
+// the chunk's first limb)
 __global__ void k_rescale_lift(const uint64_t* __restrict__ last, uint64_t* __restrict__ out, int lm1, uint64_t ql,
-                               const uint64_t* __restrict__ qmod, const DevPrime* __restrict__ pr, int logn);
+                               const uint64_t* __restrict__ qmod, const DevPrime* __restrict__ pr, int logn) {
+    const int N = 1 << logn;
+    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y, ip = blockIdx.z;
+    if (c >= N) return;
+    const uint64_t x = last[(size_t)ip * N + c];
+    const DevPrime p = pr[r];
+    uint64_t v = reduce64(x, p);
+    if (x > (ql >> 1)) v = sub_mod(v, qmod[r], p.q);  // x - q_l
+    out[((size_t)ip * lm1 + r) * N + c] = v;
+}
 
 // out[r] = (in[r] - lift[r]) q_l^-1 for the limbs of one chunk (pointers and
 // tables offset to the chunk's first limb)
@@ -66,6 +78,8 @@ using namespace he;
 extern "C" int he_rescale_noalloc(he_ctx* c, const he_ct* in, he_ct* out) {
     if (!c) return HE_EINVAL;
     if (!in || !in->data || !out || !out->data) return set_err(c, HE_EINVAL, "he_rescale_noalloc: null argument");
+    if (((uintptr_t)in->data | (uintptr_t)out->data) & 31)
+        return set_err(c, HE_EINVAL, "he_rescale_noalloc: ciphertext not 32-byte aligned");
     if (!in->is_ntt) return set_err(c, HE_EDOMAIN, "he_rescale_noalloc: input not in the evaluation domain");
     const int level = in->level, N = c->N, lm1 = level - 1;
     if (level < 2 || level > c->L)

@@ -265,7 +265,7 @@ using namespace he;
 extern "C" int he_ntt_fwd(he_ctx* c, uint64_t* d, int n_polys, int n_limbs, int first_prime) {
     if (!c) return HE_EINVAL;
     if (!d || n_polys < 0 || n_limbs < 0 || first_prime < 0 || first_prime + n_limbs > c->L + c->K ||
-        ((uintptr_t)d & 15))
+        ((uintptr_t)d & 31))
         return set_err(c, HE_EINVAL, "he_ntt_fwd: bad arguments");
     RowSet rs = rowset_contig(d, n_limbs, c->N, prime_range(first_prime, n_limbs));
     return ntt_fwd_set(c, rs, n_polys * n_limbs);
@@ -274,7 +274,7 @@ extern "C" int he_ntt_fwd(he_ctx* c, uint64_t* d, int n_polys, int n_limbs, int 
 extern "C" int he_ntt_inv(he_ctx* c, uint64_t* d, int n_polys, int n_limbs, int first_prime) {
     if (!c) return HE_EINVAL;
     if (!d || n_polys < 0 || n_limbs < 0 || first_prime < 0 || first_prime + n_limbs > c->L + c->K ||
-        ((uintptr_t)d & 15))
+        ((uintptr_t)d & 31))
         return set_err(c, HE_EINVAL, "he_ntt_inv: bad arguments");
     RowSet rs = rowset_contig(d, n_limbs, c->N, prime_range(first_prime, n_limbs));
     return ntt_inv_set(c, rs, n_polys * n_limbs);

@@ -21,6 +21,18 @@ struct RowConst {
     ulonglong2 v[kMaxPrimes];  // {value, shoup} per row
 };
 
+#define HE_NTT_LOGN_SWITCH(c, CALL)       \
+    switch ((c)->log_n) {                 \
+        case 10: CALL(10); break;         \
+        case 11: CALL(11); break;         \
+        case 12: CALL(12); break;         \
+        case 13: CALL(13); break;         \
+        case 14: CALL(14); break;         \
+        case 15: CALL(15); break;         \
+        case 16: CALL(16); break;         \
+        default: break;                   \
+    }
+
 // ------------------------------------------------------------------ kernels
 
 // out[r][c] = src[c] mod prime(r)   (src: signed 32-bit coefficients)
@@ -111,82 +123,140 @@ __global__ void k_key_canonical_seeded(const uint64_t* __restrict__ in, uint64_t
 }
 
 
-// Rescale, step 1 (batched): last[i][poly] = in_i[poly][level-1] (still in the
-// evaluation domain; an inverse NTT follows).
-__global__ void k_rescale_gather_last(PtrList in, uint64_t* __restrict__ last, int level, int logn) {
-    const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, poly = blockIdx.y, i = blockIdx.z;
-    if (c >= N) return;
-    last[((size_t)i * 2 + poly) * N + c] = in.p[i][((size_t)poly * level + level - 1) * N + c];
-}
+// Rescale of x (level lin, its first lv limbs kept, optionally times an
+// integer K) by q_l = q_{lv-1}, in the layout of the key switch's ModDown:
+//   last   = INTT((K) x_{lv-1})                              (coefficients)
+//   lift_r = [last]_{q_r} - (last > q_l/2 ? q_l : 0)          (r < lv-1, centred)
+//   out_r  = ((K) x_r - NTT(lift_r)) q_l^-1 mod q_r  (+ addend_r) (+ K0 on c0)
+// k_rescale_gather_last picks (K) x_{lv-1}; the forward column pass of
+// NTT(lift_r) computes the lift as it loads `last`, and the row pass ends
+// with the combine, so no lifted limb crosses HBM and the rescale takes two
+// transform launches where the unfused form took a lift, two passes and a
+// combine.  Residue for residue the same values.
 
-// Rescale, step 2: the centred last limb x (coefficients mod q_l) onto every
-// q_r, r < l: lift[i][poly][r] = [x]_{q_r} - (x > q_l/2 ? q_l : 0).
-__global__ void k_rescale_lift(const uint64_t* __restrict__ last, uint64_t* __restrict__ lift, int lm1, uint64_t ql,
-                               const uint64_t* __restrict__ qmod, const DevPrime* __restrict__ pr, int logn) {
-    const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y, ip = blockIdx.z;  // ip = i 2 + poly
-    if (c >= N) return;
-    uint64_t x = last[(size_t)ip * N + c];
-    DevPrime p = pr[r];
-    uint64_t v = reduce64(x, p);
-    if (x > (ql >> 1)) v = sub_mod(v, qmod[r], p.q);  // x - q_l
-    lift[((size_t)ip * lm1 + r) * N + c] = v;
-}
-
-// Rescale, step 3: out_i[poly][r] = (in_i[poly][r] - lift[i][poly][r]) q_l^-1.
-// out_i = in_i is not allowed here (the limb shift of c1 would overwrite
-// unread input); callers route in-place rescales through a staging buffer.
-// (with_add: plus addend_i, a ciphertext at level - 1, added after the rescale)
-__global__ void k_rescale_combine(PtrList in, const uint64_t* __restrict__ lift, MutPtrList out, int level,
-                                  const ulonglong2* __restrict__ qinv, PtrList addend, int with_add,
-                                  const DevPrime* __restrict__ pr, int logn) {
-    const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y, ip = blockIdx.z;
-    if (c >= N) return;
-    const int lm1 = level - 1, i = ip >> 1, poly = ip & 1;
-    uint64_t q = pr[r].q;
-    uint64_t x = in.p[i][((size_t)poly * level + r) * N + c];
-    uint64_t y = lift[((size_t)ip * lm1 + r) * N + c];
-    ulonglong2 w = qinv[r];
-    const size_t k = ((size_t)poly * lm1 + r) * N + c;
-    uint64_t v = mul_shoup(x + q - y, w.x, w.y, q);
-    if (with_add) v = add_mod(addend.p[i][k], v, q);
-    out.p[i][k] = v;
-}
-
-// The rescale of K x (x at level lin dropped to lv limbs), optionally added
-// into out and with an integer constant added to c0, in the launches of one
-// rescale: the gather multiplies the last limb by K and the combine each
-// limb, then adds.  The same modular operations in the same order as
-// mul_const_many, rescale_many, add_many and add_const_many one after the
-// other, without the intermediate ciphertexts in HBM.
-__global__ void k_rescale_gather_last_k(PtrList in, uint64_t* __restrict__ last, int lin, int lv, RowConst kc,
-                                        const DevPrime* __restrict__ pr, int logn) {
+// last[i][poly] = (K) in_i[poly][lv-1] (still in the evaluation domain)
+__global__ void k_rescale_gather_last(PtrList in, uint64_t* __restrict__ last, int lin, int lv, RowConst kc,
+                                      int with_k, const DevPrime* __restrict__ pr, int logn) {
     const int N = 1 << logn;
     int c = blockIdx.x * blockDim.x + threadIdx.x, poly = blockIdx.y, i = blockIdx.z;
     if (c >= N) return;
     const int r = lv - 1;
     const uint64_t x = in.p[i][((size_t)poly * lin + r) * N + c];
-    last[((size_t)i * 2 + poly) * N + c] = mul_shoup(x, kc.v[r].x, kc.v[r].y, pr[r].q);
+    last[((size_t)i * 2 + poly) * N + c] = with_k ? mul_shoup(x, kc.v[r].x, kc.v[r].y, pr[r].q) : x;
 }
 
-__global__ void k_rescale_combine_k(PtrList in, const uint64_t* __restrict__ lift, MutPtrList out, int lin, int lv,
-                                    RowConst kc, const ulonglong2* __restrict__ qinv, int accumulate, RowConst k0,
-                                    int add_k0, const DevPrime* __restrict__ pr, int logn) {
-    const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y, ip = blockIdx.z;
-    if (c >= N) return;
-    const int lm1 = lv - 1, i = ip >> 1, poly = ip & 1;
-    const uint64_t q = pr[r].q;
-    const uint64_t x = mul_shoup(in.p[i][((size_t)poly * lin + r) * N + c], kc.v[r].x, kc.v[r].y, q);
-    const uint64_t y = lift[((size_t)ip * lm1 + r) * N + c];
-    const ulonglong2 w = qinv[r];
-    uint64_t v = mul_shoup(x + q - y, w.x, w.y, q);
-    uint64_t* o = out.p[i] + ((size_t)poly * lm1 + r) * N + c;
-    if (accumulate) v = add_mod(*o, v, q);
-    if (add_k0 && poly == 0) v = add_mod(v, k0.v[r].x, q);
-    *o = v;
+// Column pass of NTT(lift_r), the lift taken as the limb loads: rows
+// y = ip (lv-1) + r of tmp receive the pass's raw state.
+template <int LOGN, typename T, typename TW, typename M>
+__device__ __forceinline__ void rescale_cols_body(T* sm, const uint64_t* last, uint64_t* a, const TW* tw,
+                                                  const M& m, uint64_t q, uint64_t one_shoup, uint64_t ql,
+                                                  uint64_t qlmod) {
+    using Cf = NttCfg<LOGN>;
+    const int cc = threadIdx.x % Cf::TC, g = threadIdx.x / Cf::TC;
+    constexpr int RS = Cf::R / 16;
+    T x[16];
+#pragma unroll
+    for (int k = 0; k < 16; k++) {
+        const uint64_t v = last[(size_t)(g + RS * k) * Cf::C + cc];
+        uint64_t w = csub(v - __umul64hi(v, one_shoup) * q, q);  // v mod q_r
+        if (v > (ql >> 1)) w = sub_mod(w, qlmod, q);             // v - q_l
+        x[k] = to_elem(w, T());
+    }
+    fwd_stages<4>(x, tw, 0, 0, 0, m);
+#pragma unroll
+    for (int k = 0; k < 16; k++) sm[(g + RS * k) * Cf::TC + cc] = x[k];
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 16; k++) x[k] = sm[(16 * g + k) * Cf::TC + cc];
+    fwd_stages<Cf::S1 - 4>(x, tw, 4, 0, 16 * g, m);
+#pragma unroll
+    for (int k = 0; k < 16; k++) a[(size_t)(16 * g + k) * Cf::C + cc] = raw_out(x[k]);
+}
+
+template <int LOGN>
+__global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS, NTT_COL_MIN_BLOCKS)
+    k_rescale_cols_lift(const uint64_t* __restrict__ last, uint64_t* __restrict__ tmp, int lm1, uint64_t ql,
+                        const uint64_t* __restrict__ qmod, const DevPrime* __restrict__ pr,
+                        const ulonglong2* __restrict__ tw_all, const double* __restrict__ twd_all,
+                        const FpMod* __restrict__ fpm) {
+    using Cf = NttCfg<LOGN>;
+    __shared__ uint64_t sm[Cf::R * Cf::TC];
+    const int y = blockIdx.y, ip = y / lm1, r = y - ip * lm1;
+    const uint64_t q = pr[r].q, os = pr[r].one_shoup, qm = qmod[r];
+    const uint64_t* l = last + (size_t)ip * Cf::N + blockIdx.x * Cf::TC;
+    uint64_t* a = tmp + (size_t)y * Cf::N + blockIdx.x * Cf::TC;
+    if (q < kFpPrimeLimit)
+        rescale_cols_body<LOGN>(reinterpret_cast<double*>(sm), l, a, twd_all + (size_t)r * Cf::N, fpm[r], q, os,
+                                ql, qm);
+    else
+        rescale_cols_body<LOGN>(sm, l, a, tw_all + (size_t)r * Cf::N, q, q, os, ql, qm);
+}
+
+struct RescaleIo {
+    PtrList in;      // x_i at level lin
+    MutPtrList out;  // [2][lv-1][N]
+    PtrList add;     // addend_i at level lv-1, or unused
+};
+
+// Row pass of NTT(lift_r), then the combine.
+template <int LOGN>
+__global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
+    k_rescale_rows_combine(const uint64_t* __restrict__ tmp, const RescaleIo io, int lin, int lm1, const RowConst kc,
+                           int with_k, const RowConst k0, int add_k0, int with_add,
+                           const ulonglong2* __restrict__ qinv, const DevPrime* __restrict__ pr,
+                           const ulonglong2* __restrict__ tw_all, const double* __restrict__ twd_all,
+                           const FpMod* __restrict__ fpm) {
+    using Cf = NttCfg<LOGN>;
+    __shared__ uint64_t sm[Cf::TR * Cf::ROW_PITCH];
+    const int y = blockIdx.y, ip = y / lm1, t = y - ip * lm1, i = ip >> 1, poly = ip & 1;
+    const uint64_t q = pr[t].q;
+    const int r = blockIdx.x * Cf::TR + threadIdx.x / (Cf::C / 16);
+    const int j0 = r * Cf::C + 16 * row_lane<LOGN>();
+    const uint64_t* a = tmp + (size_t)y * Cf::N + (size_t)r * Cf::C;
+    uint64_t v[16];
+    if (q < kFpPrimeLimit) {
+        const FpMod m = fpm[t];
+        double x[16];
+        row_load_strided<LOGN>(x, a);
+        fwd_rows_core<LOGN>(x, reinterpret_cast<double*>(sm), r, twd_all + (size_t)t * Cf::N, m);
+#pragma unroll
+        for (int k = 0; k < 16; k++) v[k] = fwd_canon(x[k], m);
+    } else {
+        uint64_t x[16];
+        row_load_strided<LOGN>(x, a);
+        fwd_rows_core<LOGN>(x, sm, r, tw_all + (size_t)t * Cf::N, q);
+#pragma unroll
+        for (int k = 0; k < 16; k++) v[k] = fwd_canon(x[k], q);
+    }
+    const uint64_t* xp = io.in.p[i] + ((size_t)poly * lin + t) * Cf::N + j0;
+    uint64_t* op = io.out.p[i] + ((size_t)poly * lm1 + t) * Cf::N + j0;
+    const uint64_t* ap = with_add ? io.add.p[i] + ((size_t)poly * lm1 + t) * Cf::N + j0 : nullptr;
+    const ulonglong2 w = qinv[t], kk = kc.v[t];
+    const bool k0_here = add_k0 && poly == 0;
+    const uint64_t kv = k0.v[t].x;
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        uint64_t z[4];
+        ldg256_ro(xp + 4 * k, z[0], z[1], z[2], z[3]);
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const uint64_t xv = with_k ? mul_shoup(z[e], kk.x, kk.y, q) : z[e];
+            z[e] = mul_shoup(xv + q - v[4 * k + e], w.x, w.y, q);
+        }
+        if (ap) {  // the addend may be the output itself: a coherent load
+            uint64_t s0, s1, s2, s3;
+            ldg256(ap + 4 * k, s0, s1, s2, s3);
+            z[0] = add_mod(s0, z[0], q);
+            z[1] = add_mod(s1, z[1], q);
+            z[2] = add_mod(s2, z[2], q);
+            z[3] = add_mod(s3, z[3], q);
+        }
+        if (k0_here) {
+#pragma unroll
+            for (int e = 0; e < 4; e++) z[e] = add_mod(z[e], kv, q);
+        }
+        stg256(op + 4 * k, z[0], z[1], z[2], z[3]);
+    }
 }
 
 // dst_i[k] = src_i[k], k < words (16-byte copies)
@@ -276,63 +346,81 @@ static uint64_t int_mod(int64_t K, uint64_t q) {
 
 static int ct_ok(he_ctx* c, const he_ct* x, const char* what) {
     if (!x || !x->data) return set_err(c, HE_EINVAL, "%s: null ciphertext", what);
-    if ((uintptr_t)x->data & 15) return set_err(c, HE_EINVAL, "%s: ciphertext not 16-byte aligned", what);
+    if ((uintptr_t)x->data & 31) return set_err(c, HE_EINVAL, "%s: ciphertext not 32-byte aligned", what);
     if (x->level < 1 || x->level > c->L) return set_err(c, HE_ELEVEL, "%s: level %d out of range", what, x->level);
     if (!x->is_ntt) return set_err(c, HE_EDOMAIN, "%s: ciphertext not in the evaluation domain", what);
     return HE_OK;
 }
 
-int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int level,
-                 const std::vector<const uint64_t*>& addend) {
-    const int N = c->N, n = (int)in.size(), lm1 = level - 1;
-    if (level < 2) return set_err(c, HE_ELEVEL, "rescale: level %d has no prime to drop", level);
+// The rescale path above for n ciphertexts: out_i = rescale((K) in_i) (+
+// addend_i) (+ K0 on c0), in_i at level lin, its first lv limbs kept.
+// out_i = in_i (in place) goes through a staging buffer: c1's limbs move
+// down, which would overwrite input another block has still to read.
+static int rescale_fused(he_ctx* c, const std::vector<const uint64_t*>& in, int lin, int lv, const RowConst* kc,
+                         const std::vector<uint64_t*>& out, const std::vector<const uint64_t*>& addend, bool add_k0,
+                         int64_t K0) {
+    const int N = c->N, n = (int)in.size(), lm1 = lv - 1;
+    if (lv < 2 || lin < lv) return set_err(c, HE_ELEVEL, "rescale: level %d of %d has no prime to drop", lv, lin);
     const bool with_add = !addend.empty();
     if (with_add && (int)addend.size() != n) return set_err(c, HE_EINVAL, "rescale: addend list length");
+    RowConst k1, k0;
+    if (kc) k1 = *kc;
+    for (int r = 0; r < lm1; r++) k0.v[r] = make_ulonglong2(add_k0 ? int_mod(K0, c->primes[r]) : 0, 0);
     const int gx = (N + TB - 1) / TB;
-    const uint64_t ql = c->primes[level - 1];
+    const uint64_t ql = c->primes[lv - 1];
     const double limbB = 8.0 * N;
+    const NttShape sh = ntt_shape(c->log_n);
     for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
         const int m = std::min(kMaxBatch, n - i0);
-        // per ciphertext: last limbs [2][N], lifts [2][lm1][N], staging of in-place outputs [2][lm1][N]
+        // per ciphertext: last limbs [2][N], transform rows [2][lm1][N], staging of in-place outputs [2][lm1][N]
         const size_t per = (size_t)N * (2 + 4 * lm1);
         uint64_t* base;
         int rc = scratch_slot(c, 1, per * m, &base);
         if (rc) return rc;
         uint64_t* last = base;
-        uint64_t* lift = last + (size_t)2 * m * N;
-        uint64_t* stage = lift + (size_t)2 * m * lm1 * N;
-        PtrList pin, sback, padd;
-        MutPtrList pout, dback;
-        int n_back = 0;
+        uint64_t* tmp = last + (size_t)2 * m * N;
+        uint64_t* stage = tmp + (size_t)2 * m * lm1 * N;
+        RescaleIo io;
+        PtrList sback;
+        MutPtrList dback;
+        int n_back = 0, fp_rows_n = 0;
+        for (int r = 0; r < lm1; r++) fp_rows_n += fp_prime(c, r);
         for (int i = 0; i < m; i++) {
-            pin.p[i] = in[i0 + i];
-            padd.p[i] = with_add ? addend[i0 + i] : nullptr;
+            io.in.p[i] = in[i0 + i];
+            io.add.p[i] = with_add ? addend[i0 + i] : nullptr;
             const bool inplace = out[i0 + i] == in[i0 + i];
-            pout.p[i] = inplace ? stage + (size_t)i * 2 * lm1 * N : out[i0 + i];
+            io.out.p[i] = inplace ? stage + (size_t)i * 2 * lm1 * N : out[i0 + i];
             if (inplace) {
-                sback.p[n_back] = pout.p[i];
+                sback.p[n_back] = io.out.p[i];
                 dback.p[n_back++] = out[i0 + i];
             }
         }
         prof_begin(c, HE_PROF_RESCALE);
-        k_rescale_gather_last<<<dim3(gx, 2, m), TB, 0, c->stream>>>(pin, last, level, c->log_n);
+        k_rescale_gather_last<<<dim3(gx, 2, m), TB, 0, c->stream>>>(io.in, last, lin, lv, k1, kc ? 1 : 0,
+                                                                    c->d_prime, c->log_n);
         if ((rc = lc(c, "rescale_gather"))) return rc;
-        prof_end(c, HE_PROF_RESCALE, 4.0 * m * limbB);
-        std::vector<int> pl(1, level - 1);
+        prof_end(c, HE_PROF_RESCALE, 4.0 * m * limbB, kc ? 2.0 * m * N : 0);
+        std::vector<int> pl(1, lv - 1);
         if ((rc = ntt_inv_set(c, rowset_contig(last, 1, N, pl), 2 * m))) return rc;
+        const double rows = 2.0 * m * lm1, rows_fp = 2.0 * m * fp_rows_n;
+        prof_begin(c, HE_PROF_NTT_FWD_COLS);
+#define HE_RS_COLS(LN)                                                                                             \
+    k_rescale_cols_lift<LN><<<dim3(NttCfg<LN>::COL_TILES, 2 * m * lm1), NttCfg<LN>::COL_THREADS, 0, c->stream>>>( \
+        last, tmp, lm1, ql, c->d_rs_qmod + (size_t)lm1 * c->L, c->d_prime, c->d_tw_fwd, c->d_twd_fwd, c->d_fpmod)
+        HE_NTT_LOGN_SWITCH(c, HE_RS_COLS)
+#undef HE_RS_COLS
+        if ((rc = lc(c, "rescale_cols"))) return rc;
+        prof_end(c, HE_PROF_NTT_FWD_COLS, (rows + 2.0 * m) * limbB, 0.5 * N * rows * sh.s1, 0.5 * N * rows_fp * sh.s1);
         prof_begin(c, HE_PROF_RESCALE);
-        k_rescale_lift<<<dim3(gx, lm1, 2 * m), TB, 0, c->stream>>>(last, lift, lm1, ql,
-                                                                   c->d_rs_qmod + (size_t)lm1 * c->L, c->d_prime,
-                                                                   c->log_n);
-        if ((rc = lc(c, "rescale_lift"))) return rc;
-        prof_end(c, HE_PROF_RESCALE, (2.0 * m + 2.0 * m * lm1) * limbB, 2.0 * m * lm1 * N);
-        if ((rc = ntt_fwd_set(c, rowset_contig(lift, lm1, N, prime_range(0, lm1)), 2 * m * lm1))) return rc;
-        prof_begin(c, HE_PROF_RESCALE);
-        k_rescale_combine<<<dim3(gx, lm1, 2 * m), TB, 0, c->stream>>>(pin, lift, pout, level,
-                                                                      c->d_rs_inv + (size_t)lm1 * c->L, padd,
-                                                                      with_add ? 1 : 0, c->d_prime, c->log_n);
-        if ((rc = lc(c, "rescale_combine"))) return rc;
-        prof_end(c, HE_PROF_RESCALE, (with_add ? 8.0 : 6.0) * m * lm1 * limbB, 2.0 * m * lm1 * N);
+#define HE_RS_ROWS(LN)                                                                                              \
+    k_rescale_rows_combine<LN><<<dim3(NttCfg<LN>::ROW_TILES, 2 * m * lm1), NttCfg<LN>::ROW_THREADS, 0, c->stream>>>( \
+        tmp, io, lin, lm1, k1, kc ? 1 : 0, k0, add_k0 ? 1 : 0, with_add ? 1 : 0, c->d_rs_inv + (size_t)lm1 * c->L,   \
+        c->d_prime, c->d_tw_fwd, c->d_twd_fwd, c->d_fpmod)
+        HE_NTT_LOGN_SWITCH(c, HE_RS_ROWS)
+#undef HE_RS_ROWS
+        if ((rc = lc(c, "rescale_rows"))) return rc;
+        prof_end(c, HE_PROF_RESCALE, (with_add ? 4.0 : 3.0) * rows * limbB,
+                 0.5 * N * rows * sh.s2 + (kc ? 2.0 : 1.0) * N * rows, 0.5 * N * rows_fp * sh.s2);
         if (n_back) {
             prof_begin(c, HE_PROF_RESCALE);
             k_copy_many<<<dim3(c->sm_count * 4, n_back), TB, 0, c->stream>>>(sback, dback, (size_t)lm1 * N);
@@ -341,6 +429,11 @@ int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::v
         }
     }
     return HE_OK;
+}
+
+int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int level,
+                 const std::vector<const uint64_t*>& addend) {
+    return rescale_fused(c, in, level, level, nullptr, out, addend, false, 0);
 }
 
 // HMult + relinearisation + rescale of n pairs at one level.
@@ -430,52 +523,13 @@ int mul_const_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std:
 // add_k0, K0 added to c0 after that; in_i at level lin >= lv, out_i apart
 // from every in_i.  Equal, residue for residue, to mul_const_many into a
 // temporary, rescale_many of it, add_many into out_i (accumulate) and
-// add_const_many (add_k0), and two full passes over HBM cheaper.
+// add_const_many (add_k0), without the intermediate ciphertexts in HBM.
 int mul_const_rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, int lin, int lv, int64_t K,
                            const std::vector<uint64_t*>& out, bool accumulate, bool add_k0, int64_t K0) {
-    const int N = c->N, n = (int)in.size(), lm1 = lv - 1;
-    if (lv < 2 || lin < lv) return set_err(c, HE_ELEVEL, "rescale: level %d from %d", lv, lin);
     const RowConst kc = row_const_shoup(c, lv, K);
-    RowConst k0;
-    for (int r = 0; r < lm1; r++) k0.v[r] = make_ulonglong2(add_k0 ? int_mod(K0, c->primes[r]) : 0, 0);
-    const int gx = (N + TB - 1) / TB;
-    const uint64_t ql = c->primes[lv - 1];
-    const double limbB = 8.0 * N;
-    for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
-        const int m = std::min(kMaxBatch, n - i0);
-        // per ciphertext: last limbs [2][N], lifts [2][lm1][N]
-        uint64_t* base;
-        int rc = scratch_slot(c, 1, (size_t)N * (2 + 2 * lm1) * m, &base);
-        if (rc) return rc;
-        uint64_t* last = base;
-        uint64_t* lift = last + (size_t)2 * m * N;
-        PtrList pin;
-        MutPtrList pout;
-        for (int i = 0; i < m; i++) {
-            pin.p[i] = in[i0 + i];
-            pout.p[i] = out[i0 + i];
-        }
-        prof_begin(c, HE_PROF_RESCALE);
-        k_rescale_gather_last_k<<<dim3(gx, 2, m), TB, 0, c->stream>>>(pin, last, lin, lv, kc, c->d_prime, c->log_n);
-        if ((rc = lc(c, "rescale_gather"))) return rc;
-        prof_end(c, HE_PROF_RESCALE, 4.0 * m * limbB, 2.0 * m * N);
-        std::vector<int> pl(1, lv - 1);
-        if ((rc = ntt_inv_set(c, rowset_contig(last, 1, N, pl), 2 * m))) return rc;
-        prof_begin(c, HE_PROF_RESCALE);
-        k_rescale_lift<<<dim3(gx, lm1, 2 * m), TB, 0, c->stream>>>(last, lift, lm1, ql,
-                                                                   c->d_rs_qmod + (size_t)lm1 * c->L, c->d_prime,
-                                                                   c->log_n);
-        if ((rc = lc(c, "rescale_lift"))) return rc;
-        prof_end(c, HE_PROF_RESCALE, (2.0 * m + 2.0 * m * lm1) * limbB, 2.0 * m * lm1 * N);
-        if ((rc = ntt_fwd_set(c, rowset_contig(lift, lm1, N, prime_range(0, lm1)), 2 * m * lm1))) return rc;
-        prof_begin(c, HE_PROF_RESCALE);
-        k_rescale_combine_k<<<dim3(gx, lm1, 2 * m), TB, 0, c->stream>>>(
-            pin, lift, pout, lin, lv, kc, c->d_rs_inv + (size_t)lm1 * c->L, accumulate ? 1 : 0, k0, add_k0 ? 1 : 0,
-            c->d_prime, c->log_n);
-        if ((rc = lc(c, "rescale_combine"))) return rc;
-        prof_end(c, HE_PROF_RESCALE, (accumulate ? 8.0 : 6.0) * m * lm1 * limbB, 4.0 * m * lm1 * N);
-    }
-    return HE_OK;
+    std::vector<const uint64_t*> addend;
+    if (accumulate) addend.assign(out.begin(), out.end());
+    return rescale_fused(c, in, lin, lv, &kc, out, addend, add_k0, K0);
 }
 
 // out_i = in_i keeping limbs < lv (out_i != in_i)
@@ -774,7 +828,7 @@ extern "C" int he_hmult_relin_rescale(he_ctx* c, const he_ct* a, const he_ct* b,
     if (!c) return HE_EINVAL;
     int rc;
     if ((rc = ct_ok(c, a, "hmult")) || (rc = ct_ok(c, b, "hmult"))) return rc;
-    if (!out || !out->data || ((uintptr_t)out->data & 15)) return set_err(c, HE_EINVAL, "hmult: null or unaligned output");
+    if (!out || !out->data || ((uintptr_t)out->data & 31)) return set_err(c, HE_EINVAL, "hmult: null or unaligned output");
     if (a->level != b->level) return set_err(c, HE_ELEVEL, "hmult: levels %d and %d differ", a->level, b->level);
     if (out->data == a->data || out->data == b->data) return set_err(c, HE_EINVAL, "hmult: output aliases an input");
     const int level = a->level;

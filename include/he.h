@@ -79,9 +79,9 @@ typedef struct {
     const uint64_t* p; /* optional host array of n_p primes, or NULL */
 } he_params;
 
-/* A ciphertext: data is a device pointer to [2][level][N] uint64, 16-byte
- * aligned (kernels move residues in pairs); calls reject other pointers
- * with HE_EINVAL. */
+/* A ciphertext: data is a device pointer to [2][level][N] uint64, 32-byte
+ * aligned (the transform passes move residues four at a time with 256-bit
+ * accesses); calls reject other pointers with HE_EINVAL. */
 typedef struct {
     uint64_t* data;
     int level;
@@ -213,8 +213,9 @@ int he_key_digits(const he_ctx* ctx);
 /*
  * In-place batched negacyclic NTT (coefficients -> evaluation values, storage
  * index j = value at psi^(2 brev(j)+1)) / its inverse (including N^-1).
- * d: device [n_polys][n_limbs][N]; limb i of every poly uses prime index
- * first_prime + i.  Inputs must be canonical; outputs are canonical.
+ * d: device [n_polys][n_limbs][N], 32-byte aligned; limb i of every poly
+ * uses prime index first_prime + i.  Inputs must be canonical; outputs are
+ * canonical.
  */
 int he_ntt_fwd(he_ctx* ctx, uint64_t* d, int n_polys, int n_limbs, int first_prime);
 int he_ntt_inv(he_ctx* ctx, uint64_t* d, int n_polys, int n_limbs, int first_prime);
@@ -252,7 +253,7 @@ int he_rotate_batch_host(he_ctx* ctx, const uint64_t* h_in, int level, const int
  * residues differ from he_rotate's (the fast base conversion commutes with
  * sigma_k only up to multiples of each digit's modulus), the decrypted slots
  * do not: slot j of out[i*n_steps + s] = slot j + steps[s] of in[i].
- * in: n_in device ciphertexts at one level, 16-byte aligned; out: n_in *
+ * in: n_in device ciphertexts at one level, 32-byte aligned; out: n_in *
  * n_steps device ciphertexts, none overlapping an input, each given in[i]'s
  * level and scale.  A step whose Galois element is 1 copies.  Errors:
  * HE_EINVAL (null, unaligned, aliasing, negative counts), HE_ELEVEL (mixed or
@@ -273,7 +274,7 @@ int he_rotate_hoisted(he_ctx* ctx, const he_ct* in, int n_in, const int32_t* ste
  * results (by at most (n_terms+1)(K+1)/2 per coefficient) while the slots
  * agree.  Terms whose Galois element is 1 are added unchanged.
  * z: n_out*n_terms device ciphertexts (output-major), base: n_out ciphertexts
- * or NULL (then n_terms >= 1), all at one level and scale, 16-byte aligned;
+ * or NULL (then n_terms >= 1), all at one level and scale, 32-byte aligned;
  * n_terms <= 64.  out: n_out device ciphertexts with room for that level,
  * none overlapping an input; each gets the level and scale.  Errors:
  * HE_EINVAL (null, unaligned, aliasing, counts), HE_ELEVEL (mixed levels or
@@ -292,7 +293,7 @@ int he_rotate_sum(he_ctx* ctx, const he_ct* z, int n_out, int n_terms, const int
  * Residues differ from adding he_rotate_hoisted results by the rounding of
  * one ModDown instead of n_steps (at most (n_steps+1)(K+1)/2 per
  * coefficient); the slots agree.  A step whose Galois element is 1 adds
- * in[i] unchanged.  in: n_in device ciphertexts at one level, 16-byte
+ * in[i] unchanged.  in: n_in device ciphertexts at one level, 32-byte
  * aligned; 1 <= n_steps <= 64; out: n_in device ciphertexts with room for
  * that level, none overlapping an input, each given in[i]'s level and scale.
  * Errors: HE_EINVAL, HE_ELEVEL, HE_EDOMAIN, HE_ENOKEY as he_rotate_hoisted;

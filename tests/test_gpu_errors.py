@@ -42,12 +42,17 @@ def test_unaligned_ciphertexts_are_rejected():
     st.upload_relin()
     z = S.complex_slots(st.seed, st.P.n_slots, -1, 1)
     x = st.to_gpu(st.encrypt(z, 3))
-    raw = torch.zeros(2 * 3 * st.P.N + 1, dtype=torch.int64, device="cuda")
-    bad = he.Ciphertext(raw[1:], 3, 1.0)  # 8 bytes past a 16-byte boundary
+    raw = torch.zeros(2 * 3 * st.P.N + 2, dtype=torch.int64, device="cuda")
     y = st.empty_gpu(3)
-    assert _code(he.he_rotate, st.ctx, bad, 1, y) == he.HE_EINVAL
-    assert _code(he.he_rotate, st.ctx, x, 1, bad) == he.HE_EINVAL
-    assert _code(he.he_hmult_relin_rescale, st.ctx, x, x, bad) == he.HE_EINVAL
+    # 8 bytes past a 16-byte boundary, and 16 bytes past a 32-byte one (the
+    # transform passes move four residues per 256-bit access)
+    for off in (1, 2):
+        bad = he.Ciphertext(raw[off:off + 2 * 3 * st.P.N], 3, 1.0)
+        assert _code(he.he_rotate, st.ctx, bad, 1, y) == he.HE_EINVAL
+        assert _code(he.he_rotate, st.ctx, x, 1, bad) == he.HE_EINVAL
+        assert _code(he.he_hmult_relin_rescale, st.ctx, x, x, bad) == he.HE_EINVAL
+        assert _code(he.he_rescale, st.ctx, bad) == he.HE_EINVAL
+        assert _code(he.he_ntt_fwd, st.ctx, raw[off:off + 3 * st.P.N], 1, 3, 0) == he.HE_EINVAL
     # the context still rotates correctly
     he.he_rotate(st.ctx, x, 1, y)
     he.he_sync(st.ctx)
