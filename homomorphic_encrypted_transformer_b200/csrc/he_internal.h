@@ -190,6 +190,13 @@ int rotate_sum_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t*
 constexpr int kScratchSlots = 5;
 int scratch_slot(he_ctx* c, int slot, size_t words, uint64_t** out);
 
+// Packed wire format of ciphertexts (wire.cu): bytes of one ciphertext at
+// `level`; device unpacking of n packed ciphertexts into ct_i and packing
+// back (wire: device, 8-byte aligned, ciphertexts back to back).
+size_t wire_bytes(const he_ctx* c, int level);
+int wire_unpack_many(he_ctx* c, const uint8_t* wire, int level, const std::vector<uint64_t*>& ct);
+int wire_pack_many(he_ctx* c, const std::vector<const uint64_t*>& ct, int level, uint8_t* wire);
+
 // out[i] = rescale(in[i]) for n ciphertexts at `level` (out may equal in),
 // plus addend[i] (a ciphertext at level - 1) when addend is not empty.
 int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int level,

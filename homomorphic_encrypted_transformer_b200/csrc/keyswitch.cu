@@ -1708,25 +1708,30 @@ static int io_drain(he_ctx* c, int rc) {
     return rc;
 }
 
-extern "C" int he_rotate_batch_host(he_ctx* c, const uint64_t* h_in, int level, const int32_t* steps,
-                                    uint64_t* h_out, int n) {
+// The host-buffer pipeline; wire: the host buffers hold ciphertexts in the
+// packed wire format (wire.cu), unpacked and packed on the device, so only
+// the packed bytes cross the host link.
+static int rotate_batch_host(he_ctx* c, const uint8_t* h_in, int level, const int32_t* steps, uint8_t* h_out, int n,
+                             bool wire, const char* what) {
     if (!c) return HE_EINVAL;
     if (!h_in || !h_out || !steps || n < 0 || level < 1 || level > c->L)
-        return set_err(c, HE_EINVAL, "he_rotate_batch_host: bad arguments");
+        return set_err(c, HE_EINVAL, "%s: bad arguments", what);
     if (n == 0) return HE_OK;
     std::vector<uint64_t> gal(n);
     for (int i = 0; i < n; i++) {
         gal[i] = galois_elt(c, steps[i]);
         if (gal[i] != 1 && !c->rot_keys.count(gal[i]))
-            return set_err(c, HE_ENOKEY, "he_rotate_batch_host: no key for step %d", steps[i]);
+            return set_err(c, HE_ENOKEY, "%s: no key for step %d", what, steps[i]);
     }
     std::vector<int> order(n);
     for (int i = 0; i < n; i++) order[i] = i;
     std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return gal[x] < gal[y]; });
 
-    const size_t ct_words = (size_t)2 * level * c->N, ct_bytes = ct_words * 8;
+    const size_t ct_words = (size_t)2 * level * c->N;
+    const size_t link_bytes = wire ? wire_bytes(c, level) : ct_words * 8;  // per ciphertext across the link
+    const size_t link_words = (link_bytes + 7) / 8;
     const int chunk = std::min(kIoChunk, n);
-    int rc = io_setup(c, 4 * (size_t)chunk * ct_words);
+    int rc = io_setup(c, 4 * (size_t)chunk * ct_words + (wire ? 4 * (size_t)chunk * link_words : 0));
     if (rc) return rc;
     cudaEvent_t* up = c->io_ev;        // [2] upload of buffer b done
     cudaEvent_t* done = c->io_ev + 2;  // [2] rotation of buffer b done
@@ -1736,11 +1741,15 @@ extern "C" int he_rotate_batch_host(he_ctx* c, const uint64_t* h_in, int level, 
         const int b = k & 1, i0 = k * chunk, m = std::min(chunk, n - i0);
         uint64_t* din = c->io_buf + (size_t)b * chunk * ct_words;
         uint64_t* dout = c->io_buf + (size_t)(2 + b) * chunk * ct_words;
+        uint64_t* wbase = c->io_buf + 4 * (size_t)chunk * ct_words;
+        uint8_t* lin = reinterpret_cast<uint8_t*>(wire ? wbase + (size_t)b * chunk * link_words : din);
+        uint8_t* lout = reinterpret_cast<uint8_t*>(wire ? wbase + (size_t)(2 + b) * chunk * link_words : dout);
+        const size_t lstride = wire ? link_words * 8 : ct_words * 8;  // bytes between staged ciphertexts
         // upload, once chunk k-2 no longer reads this buffer
         if (k >= 2) cudaStreamWaitEvent(c->io_h2d, done[b], 0);
         for (int j = 0; j < m; j++) {
-            rc = check_cuda(c, cudaMemcpyAsync(din + j * ct_words, h_in + (size_t)order[i0 + j] * ct_words, ct_bytes,
-                                               cudaMemcpyHostToDevice, c->io_h2d), "H2D");
+            rc = check_cuda(c, cudaMemcpyAsync(lin + j * lstride, h_in + (size_t)order[i0 + j] * link_bytes,
+                                               link_bytes, cudaMemcpyHostToDevice, c->io_h2d), "H2D");
             if (rc) return io_drain(c, rc);
         }
         cudaEventRecord(up[b], c->io_h2d);
@@ -1749,19 +1758,26 @@ extern "C" int he_rotate_batch_host(he_ctx* c, const uint64_t* h_in, int level, 
         if (k >= 2) cudaStreamWaitEvent(c->stream, down[b], 0);
         std::vector<he_ct> in(m), out(m);
         std::vector<int32_t> st(m);
+        std::vector<uint64_t*> dins(m);
+        std::vector<const uint64_t*> douts(m);
         for (int j = 0; j < m; j++) {
             in[j] = he_ct{din + j * ct_words, level, 1.0, 1};
             out[j] = he_ct{dout + j * ct_words, level, 1.0, 1};
             st[j] = steps[order[i0 + j]];
+            dins[j] = in[j].data;
+            douts[j] = out[j].data;
         }
+        if (wire && lstride != link_bytes) return io_drain(c, set_err(c, HE_EINVAL, "%s: wire size", what));
+        if (wire && (rc = wire_unpack_many(c, lin, level, dins))) return io_drain(c, rc);
         rc = rotate_many(c, in.data(), st.data(), out.data(), m);
         if (rc) return io_drain(c, rc);
+        if (wire && (rc = wire_pack_many(c, douts, level, lout))) return io_drain(c, rc);
         cudaEventRecord(done[b], c->stream);
         // download
         cudaStreamWaitEvent(c->io_d2h, done[b], 0);
         for (int j = 0; j < m; j++) {
-            rc = check_cuda(c, cudaMemcpyAsync(h_out + (size_t)order[i0 + j] * ct_words, dout + j * ct_words, ct_bytes,
-                                               cudaMemcpyDeviceToHost, c->io_d2h), "D2H");
+            rc = check_cuda(c, cudaMemcpyAsync(h_out + (size_t)order[i0 + j] * link_bytes, lout + j * lstride,
+                                               link_bytes, cudaMemcpyDeviceToHost, c->io_d2h), "D2H");
             if (rc) return io_drain(c, rc);
         }
         cudaEventRecord(down[b], c->io_d2h);
@@ -1769,4 +1785,15 @@ extern "C" int he_rotate_batch_host(he_ctx* c, const uint64_t* h_in, int level, 
     rc = check_cuda(c, cudaStreamSynchronize(c->io_d2h), "D2H sync");
     if (rc) return io_drain(c, rc);
     return he_sync(c);
+}
+
+extern "C" int he_rotate_batch_host(he_ctx* c, const uint64_t* h_in, int level, const int32_t* steps,
+                                    uint64_t* h_out, int n) {
+    return rotate_batch_host(c, reinterpret_cast<const uint8_t*>(h_in), level, steps,
+                             reinterpret_cast<uint8_t*>(h_out), n, false, "he_rotate_batch_host");
+}
+
+extern "C" int he_rotate_batch_host_wire(he_ctx* c, const uint8_t* h_in, int level, const int32_t* steps,
+                                         uint8_t* h_out, int n) {
+    return rotate_batch_host(c, h_in, level, steps, h_out, n, true, "he_rotate_batch_host_wire");
 }

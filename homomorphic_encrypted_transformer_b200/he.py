@@ -95,6 +95,10 @@ _sig("he_attention_scores", _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct
      ctypes.POINTER(he_ct))
 _sig("he_attention_output", _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct), _i, _vp, _i, ctypes.POINTER(he_ct))
 _sig("he_rotate_batch_host", _i, _vp, _vp, _i, _vp, _vp, _i)
+_sig("he_rotate_batch_host_wire", _i, _vp, _vp, _i, _vp, _vp, _i)
+_sig("he_ct_wire_bytes", ctypes.c_longlong, _vp, _i, _i)
+_sig("he_ct_pack", _i, _vp, _i, _i, _vp, _i, _vp)
+_sig("he_ct_unpack", _i, _vp, _i, _i, _vp, _i, _vp)
 _sig("he_hmult_relin_rescale", _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct), ctypes.POINTER(he_ct))
 _sig("he_rescale", _i, _vp, ctypes.POINTER(he_ct))
 _sig("he_rescale_noalloc", _i, _vp, ctypes.POINTER(he_ct), ctypes.POINTER(he_ct))
@@ -400,6 +404,57 @@ def he_rotate_batch_host(ctx, h_in, level, steps, h_out):
     """h_in, h_out: host arrays (numpy or pinned torch CPU tensors) of [n][2][level][N] uint64."""
     st = np.ascontiguousarray(steps, dtype=np.int32)
     _check(ctx, _lib.he_rotate_batch_host(ctx.ptr, _ptr(h_in), level, _ptr(st), _ptr(h_out), len(st)))
+
+
+def _nbytes(a):
+    return a.nbytes if isinstance(a, np.ndarray) else a.numel() * a.element_size()
+
+
+def he_ct_wire_bytes(primes, level, log_n):
+    """Bytes of one ciphertext at `level` in the packed wire format (host only)."""
+    pr = np.ascontiguousarray(primes[:level], dtype=np.uint64)
+    v = _lib.he_ct_wire_bytes(_ptr(pr), int(level), int(log_n))
+    if v < 0:
+        raise HEError(int(v), "he_ct_wire_bytes: bad arguments")
+    return int(v)
+
+
+def he_ct_pack(primes, level, log_n, cts):
+    """Host [n][2][level][N] uint64 -> n packed ciphertexts (uint8, back to back)."""
+    pr = np.ascontiguousarray(primes[:level], dtype=np.uint64)
+    a = np.ascontiguousarray(cts, dtype=np.uint64)
+    per = 2 * level << log_n
+    n = a.size // per
+    if a.size != n * per:
+        raise ValueError("he_ct_pack: expected [n][2][level][N] residues")
+    out = np.empty(n * he_ct_wire_bytes(primes, level, log_n), dtype=np.uint8)
+    rc = _lib.he_ct_pack(_ptr(pr), int(level), int(log_n), _ptr(a), n, _ptr(out))
+    if rc != HE_OK:
+        raise HEError(rc, "he_ct_pack: bad arguments or a residue not below its prime")
+    return out
+
+
+def he_ct_unpack(primes, level, log_n, packed, n):
+    """n packed ciphertexts -> host [n][2][level][N] uint64."""
+    pr = np.ascontiguousarray(primes[:level], dtype=np.uint64)
+    p = np.ascontiguousarray(packed, dtype=np.uint8)
+    if p.size < n * he_ct_wire_bytes(primes, level, log_n):
+        raise ValueError("he_ct_unpack: buffer shorter than n packed ciphertexts")
+    out = np.empty((n, 2, level, 1 << log_n), dtype=np.uint64)
+    rc = _lib.he_ct_unpack(_ptr(pr), int(level), int(log_n), _ptr(p), int(n), _ptr(out))
+    if rc != HE_OK:
+        raise HEError(rc, "he_ct_unpack: bad arguments")
+    return out
+
+
+def he_rotate_batch_host_wire(ctx, h_in, level, steps, h_out):
+    """h_in, h_out: host buffers (numpy or pinned torch CPU uint8 tensors) of
+    len(steps) packed ciphertexts each (he_ct_wire_bytes apiece)."""
+    st = np.ascontiguousarray(steps, dtype=np.int32)
+    need = len(st) * he_ct_wire_bytes(ctx.primes, level, ctx.log_n)
+    if _nbytes(h_in) < need or _nbytes(h_out) < need:
+        raise ValueError("he_rotate_batch_host_wire: buffers shorter than %d bytes" % need)
+    _check(ctx, _lib.he_rotate_batch_host_wire(ctx.ptr, _ptr(h_in), level, _ptr(st), _ptr(h_out), len(st)))
 
 
 def he_hmult_relin_rescale(ctx, a, b, out):

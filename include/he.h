@@ -243,6 +243,29 @@ int he_rotate_batch(he_ctx* ctx, const he_ct* in, const int32_t* steps, he_ct* o
 int he_rotate_batch_host(he_ctx* ctx, const uint64_t* h_in, int level, const int32_t* steps,
                          uint64_t* h_out, int n);
 /*
+ * Packed wire format of ciphertexts, for host transfers: a residue mod q_r
+ * takes b_r = ceil(bitlen(q_r) / 8) bytes, little-endian (5 for the 40-bit
+ * primes of the chain, 8 for a 60-bit one); a ciphertext at `level` is, for
+ * poly 0 then 1 and limb r = 0..level-1, its N residues of b_r bytes each:
+ * he_ct_wire_bytes = 2 N sum_{r<level} b_r bytes (64% of 2 level N 8 at
+ * N = 2^16, level 24).  Exact for canonical residues.  Host only (no
+ * context, no device work): primes = q_0..q_{level-1} (he_get_primes or
+ * he_derive_primes), N = 2^log_n.  he_ct_pack / he_ct_unpack convert n
+ * ciphertexts between host [n][2][level][N] uint64 and n packed ciphertexts
+ * back to back; he_ct_pack returns HE_EINVAL for a residue not below its
+ * prime.  he_ct_wire_bytes returns HE_EINVAL (negative) for bad arguments.
+ */
+long long he_ct_wire_bytes(const uint64_t* primes, int level, int log_n);
+int he_ct_pack(const uint64_t* primes, int level, int log_n, const uint64_t* in, int n, uint8_t* out);
+int he_ct_unpack(const uint64_t* primes, int level, int log_n, const uint8_t* in, int n, uint64_t* out);
+/* he_rotate_batch_host on packed host buffers: h_in / h_out hold n packed
+ * ciphertexts each (he_ct_wire_bytes bytes apiece at the context's primes,
+ * canonical
+ * residues); they are unpacked and packed on the device, so only the packed
+ * bytes cross the host link.  Same pipeline, staging and rules otherwise. */
+int he_rotate_batch_host_wire(he_ctx* ctx, const uint8_t* h_in, int level, const int32_t* steps,
+                              uint8_t* h_out, int n);
+/*
  * Hoisted rotations (Halevi-Shoup, "Faster Homomorphic Linear Transformations
  * in HElib", CRYPTO 2018, section 5): every input rotated by every step, with
  * one ModUp per input shared by all its steps.  For in[i] = (c0, c1) and

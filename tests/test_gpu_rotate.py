@@ -201,6 +201,59 @@ def test_rotation_batch_host_buffers_full_size():
     assert np.array_equal(h_out, host(y).reshape(h_in.shape))
 
 
+def test_rotation_batch_host_wire():
+    """The packed wire entry (he_rotate_batch_host_wire): 21 packed
+    ciphertexts in three chunks, steps unsorted and repeated and one identity
+    rotation; unpacked, the outputs equal the oracle's rotations, and the
+    packed output equals the host packing of the unpacked entry's output."""
+    he = lib()
+    st = Setup(12, 3, 1, 3, seed=7)
+    P = st.P
+    n = 21
+    steps = [3, 1, 2, 1, 7, 3, 2, P.n_slots, 1, 7, 2, 3, 1, 1, 2, 7, 3, 2, 1, 7, 3]
+    for s_ in set(steps):
+        if s_ != P.n_slots:
+            st.upload_rot(s_)
+    cts = [st.encrypt(S.complex_slots(st.seed, P.n_slots, -1, 1, i), 3, ct_id=i) for i in range(n)]
+    h_in = np.stack([c["c"] for c in cts])
+    w_in = he.he_ct_pack(P.q, 3, P.log_n, h_in)
+    w_out = np.zeros_like(w_in)
+    he.he_rotate_batch_host_wire(st.ctx, w_in, 3, steps, w_out)
+    got = he.he_ct_unpack(P.q, 3, P.log_n, w_out, n)
+    for i in range(n):
+        if steps[i] == P.n_slots:
+            assert np.array_equal(got[i], h_in[i])
+            continue
+        want = C.rotate(cts[i], steps[i], st.oracle_rot_key(steps[i]), P)
+        assert np.array_equal(got[i], want["c"]), i
+    h_out = np.zeros_like(h_in)
+    he.he_rotate_batch_host(st.ctx, h_in, 3, steps, h_out)
+    assert np.array_equal(w_out, he.he_ct_pack(P.q, 3, P.log_n, h_out))
+
+
+def test_rotation_batch_host_wire_full_size():
+    """The packed wire entry on the rotation batch (64 ciphertexts at
+    N = 2^16, level 24, 16 keys): 64% of the bytes cross the host link, and
+    the unpacked outputs equal the device entry's, ciphertext for ciphertext."""
+    he = lib()
+    st = Setup(16, 24, 8, 3, seed=S.master_seed(1))
+    P = st.P
+    steps, ct_steps = _rotation_batch_inputs(st, 64, 16)
+    for s_ in steps:
+        st.upload_rot(s_)
+    h_in = S.uniform_residues(st.seed, "ct_residues", P.q, P.N, lead=(64, 2))
+    x = torch.from_numpy(h_in.view(np.int64)).cuda()
+    y = torch.empty_like(x)
+    he.he_rotate_batch(st.ctx, [he.Ciphertext(x[i], 24, 2.0 ** 40) for i in range(64)], ct_steps,
+                       [he.Ciphertext(y[i], 24, 2.0 ** 40) for i in range(64)])
+    he.he_sync(st.ctx)
+    w_in = he.he_ct_pack(P.q, 24, 16, h_in)
+    assert w_in.nbytes == 64 * 2 * (1 << 16) * (8 + 23 * 5)
+    w_out = np.zeros_like(w_in)
+    he.he_rotate_batch_host_wire(st.ctx, w_in, 24, ct_steps, w_out)
+    assert np.array_equal(he.he_ct_unpack(P.q, 24, 16, w_out, 64), host(y).reshape(h_in.shape))
+
+
 def _hoisted_case(st, level, n_in, steps):
     """he_rotate_hoisted of n_in encrypted inputs by `steps` against the
     oracle's rotate_hoisted, residue for residue; Galois element 1 copies."""
