@@ -193,7 +193,9 @@ extern "C" int he_pmult_accum_bsgs(he_ctx* c, const he_ct* x, int n_in, const ui
         if (x[i].level != level) return set_err(c, HE_ELEVEL, "he_pmult_accum_bsgs: mixed levels");
     }
     for (int i = 0; i < n_groups * n_out; i++)
-        if (!y[i].data) return set_err(c, HE_EINVAL, "he_pmult_accum_bsgs: null output %d", i);
+        if (!y[i].data || ((uintptr_t)y[i].data & 31))
+            return set_err(c, HE_EINVAL, "he_pmult_accum_bsgs: null or unaligned output %d", i);
+    if ((uintptr_t)d_pt & 31) return set_err(c, HE_EINVAL, "he_pmult_accum_bsgs: plaintexts not 32-byte aligned");
     if (level < 2) return set_err(c, HE_ELEVEL, "he_pmult_accum_bsgs: level %d cannot be rescaled", level);
     for (int b = 1; b < bs; b++)
         if (!c->rot_keys.count(galois_elt(c, stride * b)) && galois_elt(c, stride * b) != 1)

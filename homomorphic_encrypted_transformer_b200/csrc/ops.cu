@@ -901,7 +901,7 @@ extern "C" int he_poly_eval_ps15(he_ctx* c, const he_ct* x, int n, const double*
         if (rc) return rc;
         if (x[i].level != l0) return set_err(c, HE_ELEVEL, "ps15: mixed levels");
         if (x[i].scale != x[0].scale) return set_err(c, HE_ELEVEL, "ps15: mixed scales");
-        if (!out[i].data) return set_err(c, HE_EINVAL, "ps15: null output");
+        if (!out[i].data || ((uintptr_t)out[i].data & 31)) return set_err(c, HE_EINVAL, "ps15: null or unaligned output");
     }
     if (l0 < 7) return set_err(c, HE_ELEVEL, "ps15: needs level >= 7, got %d", l0);
     if (!c->relin.d) return set_err(c, HE_ENOKEY, "ps15: no relinearisation key");

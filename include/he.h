@@ -369,7 +369,7 @@ int he_drop_level(he_ctx* ctx, const he_ct* in, int level, he_ct* out);
  *   Y[t][i] = rescale( sum_g rot_{stride*bs*g}( sum_{j,b} pt[i][j][g][b] (.) rot_{stride*b}(X[t][j]) ) )
  * x: n_groups*n_in ciphertexts (group-major) at one level l >= 2.
  * d_pt: device [n_out][n_in][gs][bs][l][N] evaluation-domain plaintexts,
- *       encoded at pt_scale.
+ *       encoded at pt_scale, 32-byte aligned.
  * y: n_groups*n_out ciphertexts (group-major) with room for level l; they
  *    come back at level l-1, scale x.scale*pt_scale/q_{l-1}.
  * The baby-step rotations rot_{stride*b}(X[t][j]) are the hoisted rotations of

@@ -83,6 +83,12 @@ def test_bsgs_and_polynomial_errors():
     assert _code(he.he_pmult_accum_bsgs, st.ctx, [x3], 1, pt, 2.0 ** 40, 1, 2, 2, 1, 1, ys) == he.HE_ENOKEY
     # n_in * bs above 255
     assert _code(he.he_pmult_accum_bsgs, st.ctx, [x3], 1, pt, 2.0 ** 40, 1, 256, 1, 1, 1, ys) == he.HE_EINVAL
+    # outputs and plaintexts 16 bytes past a 32-byte boundary
+    raw = torch.zeros(2 * 3 * st.P.N + 2, dtype=torch.int64, device="cuda")
+    bad = [he.Ciphertext(raw[2:], 3, 1.0)]
+    assert _code(he.he_pmult_accum_bsgs, st.ctx, [x3], 1, pt, 2.0 ** 40, 1, 2, 2, 1, 1, bad) == he.HE_EINVAL
+    pt_raw = torch.zeros(pt.numel() + 2, dtype=torch.int64, device="cuda")
+    assert _code(he.he_pmult_accum_bsgs, st.ctx, [x3], 1, pt_raw[2:], 2.0 ** 40, 1, 2, 2, 1, 1, ys) == he.HE_EINVAL
     # mixed input levels
     x2 = st.to_gpu(st.encrypt(z, 2), room=3)
     st.upload_rot(1)
@@ -94,6 +100,9 @@ def test_bsgs_and_polynomial_errors():
     st7 = Setup(12, 8, 3, 3, seed=64)
     x7 = st7.to_gpu(st7.encrypt(z, 8))
     assert _code(he.he_poly_eval_ps15, st7.ctx, [x7], coeffs, 2.0 ** 62, [st7.empty_gpu(8)]) == he.HE_ENOKEY
+    raw7 = torch.zeros(2 * 8 * st7.P.N + 2, dtype=torch.int64, device="cuda")
+    assert _code(he.he_poly_eval_ps15, st7.ctx, [x7], coeffs, 2.0 ** 62,
+                 [he.Ciphertext(raw7[2:], 8, 1.0)]) == he.HE_EINVAL  # output 16 bytes off
 
 
 def test_hoisted_rotation_errors():
