@@ -418,6 +418,15 @@ def test_rotation_sum_hoisted_mid_levels(level):
     _sum_hoisted_case(st, level, 2, [5, -3, 17])
 
 
+@pytest.mark.parametrize("level,n_in", [(7, 4), (4, 8), (1, 4)])
+def test_rotation_sum_hoisted_four_outputs_per_thread(level, n_in):
+    """Rotate-and-sum of 4 or 8 ciphertexts over one step list: outputs in
+    blocks of four share each key word (k_ks_inner_sum_mo), with 60-bit and
+    40-bit rows, partial digits and level 1; residue for residue."""
+    st = Setup(11, 7, 3, 3, seed=51)
+    _sum_hoisted_case(st, level, n_in, [5, -3, 17, 0, 9])
+
+
 def test_rotation_sum_hoisted_chunks():
     """5 ciphertexts x 20 steps: chunks of 3 and 2 inputs."""
     st = Setup(11, 3, 1, 3, seed=50)
