@@ -103,13 +103,12 @@ extern "C" int he_attention_scores(he_ctx* c, const he_ct* q, const he_ct* k, in
     for (size_t j = 0; j < nz.size(); j++) rk[j] = he_ct{pool + j * ctw, l, k->scale, 1};
     if (!nz.empty() && (rc = rotate_hoisted_many(c, k, 1, nz.data(), (int)nz.size(), rk.data()))) return rc;
     // P_delta = HMRR(q, rot_delta(k)) into the outputs
-    std::vector<const uint64_t*> A, B, Sc;
+    std::vector<const uint64_t*> A, B;
     std::vector<uint64_t*> So, Tm;
     for (int i = 0; i < n_off; i++) {
         A.push_back(q->data);
         B.push_back(pos[i] < 0 ? k->data : rk[pos[i]].data);
         So.push_back(s[i].data);
-        Sc.push_back(s[i].data);
         Tm.push_back(pool + ctw * nz.size() + ctw1 * i);
     }
     if ((rc = hmrr_many(c, A, B, So, l))) return rc;
@@ -120,12 +119,20 @@ extern "C" int he_attention_scores(he_ctx* c, const he_ct* q, const he_ct* k, in
         sc[i] = he_ct{s[i].data, l - 1, scale, 1};
         tc[i] = he_ct{Tm[i], l - 1, scale, 1};
     }
-    std::vector<const uint64_t*> Tc(Tm.begin(), Tm.end());
-    for (int h = 1; h < d; h <<= 1) {
+    // each round: dst = rot(src) + src, the sum taken in the rotation's
+    // ModDown; src and dst alternate between the outputs and the scratch
+    int rounds = 0;
+    for (int h = 1; h < d; h <<= 1, rounds++) {
         std::vector<int32_t> st(n_off, 2 * n_tok * h);
-        if ((rc = rotate_many(c, sc.data(), st.data(), tc.data(), n_off))) return rc;
-        if ((rc = add_many(c, Sc, Tc, So, l - 1))) return rc;
+        const std::vector<he_ct>& src = rounds % 2 ? tc : sc;
+        std::vector<he_ct>& dst = rounds % 2 ? sc : tc;
+        if ((rc = rotate_many(c, src.data(), st.data(), dst.data(), n_off, src.data()))) return rc;
     }
+    if (rounds % 2)  // an odd number of rounds ends in the scratch
+        for (int i = 0; i < n_off; i++)
+            if ((rc = check_cuda(c, cudaMemcpyAsync(s[i].data, Tm[i], (size_t)2 * (l - 1) * c->N * 8,
+                                                    cudaMemcpyDeviceToDevice, c->stream), "attention copy")))
+                return rc;
     for (int i = 0; i < n_off; i++) {
         s[i].level = l - 1;
         s[i].scale = scale;
