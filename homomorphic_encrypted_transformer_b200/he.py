@@ -410,9 +410,16 @@ def _nbytes(a):
     return a.nbytes if isinstance(a, np.ndarray) else a.numel() * a.element_size()
 
 
+def _wire_primes(primes, level):
+    pr = np.ascontiguousarray(list(primes)[:max(int(level), 0)], dtype=np.uint64)
+    if len(pr) != level:
+        raise ValueError("wire format: level %d needs %d primes, got %d" % (level, level, len(pr)))
+    return pr
+
+
 def he_ct_wire_bytes(primes, level, log_n):
     """Bytes of one ciphertext at `level` in the packed wire format (host only)."""
-    pr = np.ascontiguousarray(primes[:level], dtype=np.uint64)
+    pr = _wire_primes(primes, level)
     v = _lib.he_ct_wire_bytes(_ptr(pr), int(level), int(log_n))
     if v < 0:
         raise HEError(int(v), "he_ct_wire_bytes: bad arguments")
@@ -421,7 +428,7 @@ def he_ct_wire_bytes(primes, level, log_n):
 
 def he_ct_pack(primes, level, log_n, cts):
     """Host [n][2][level][N] uint64 -> n packed ciphertexts (uint8, back to back)."""
-    pr = np.ascontiguousarray(primes[:level], dtype=np.uint64)
+    pr = _wire_primes(primes, level)
     a = np.ascontiguousarray(cts, dtype=np.uint64)
     per = 2 * level << log_n
     n = a.size // per
@@ -436,7 +443,7 @@ def he_ct_pack(primes, level, log_n, cts):
 
 def he_ct_unpack(primes, level, log_n, packed, n):
     """n packed ciphertexts -> host [n][2][level][N] uint64."""
-    pr = np.ascontiguousarray(primes[:level], dtype=np.uint64)
+    pr = _wire_primes(primes, level)
     p = np.ascontiguousarray(packed, dtype=np.uint8)
     if p.size < n * he_ct_wire_bytes(primes, level, log_n):
         raise ValueError("he_ct_unpack: buffer shorter than n packed ciphertexts")

@@ -70,6 +70,27 @@ def test_host_buffer_entry_errors():
     assert _code(he.he_rotate_batch_host, st.ctx, h, 9, [1, 1], out) == he.HE_EINVAL
     he.he_rotate_batch_host(st.ctx, h, 3, [1, 1], out)  # zero ciphertexts rotate to zero
     assert not out.any()
+    # the packed wire entry: the same checks, and zero packs to zero
+    w = he.he_ct_pack(st.P.q, 3, st.P.log_n, h)
+    wout = np.full_like(w, 7)
+    assert _code(he.he_rotate_batch_host_wire, st.ctx, w, 3, [1, 5], wout) == he.HE_ENOKEY
+    with pytest.raises(ValueError):  # level beyond the chain: no wire size
+        he.he_rotate_batch_host_wire(st.ctx, w, 9, [1, 1], wout)
+    with pytest.raises(ValueError):  # buffers shorter than the ciphertexts
+        he.he_rotate_batch_host_wire(st.ctx, w[:-1], 3, [1, 1], wout)
+    he.he_rotate_batch_host_wire(st.ctx, w, 3, [1, 1], wout)
+    assert not wout.any()
+    he.he_rotate_batch_host_wire(st.ctx, w, 3, [], wout)  # no ciphertexts: nothing to do
+
+
+def test_seeded_keygen_edge_cases():
+    he = lib()
+    st = Setup(11, 3, 1, 3, seed=66)
+    he.he_keygen_seeded_ex(st.ctx, 5, [], False, he.HE_KEYGEN_SEEDED_A)  # no keys asked for: nothing made
+    with pytest.raises(he.HEError) as ei:
+        he.he_key_download(st.ctx, he.HE_KEY_RELIN, 0)
+    assert ei.value.code == he.HE_ENOKEY
+    assert _code(he.he_keygen_seeded_ex, st.ctx, 5, [st.P.n_slots], False, he.HE_KEYGEN_SEEDED_A) == he.HE_EINVAL
 
 
 def test_bsgs_and_polynomial_errors():

@@ -62,5 +62,7 @@ def test_wire_argument_checks(he):
         he.he_ct_pack(P.q, 4, 11, cts)
     with pytest.raises(he.HEError):
         he.he_ct_wire_bytes(P.q, 0, 11)
+    with pytest.raises(ValueError):  # more limbs than primes given
+        he.he_ct_wire_bytes(P.q[:2], 3, 11)
     with pytest.raises(ValueError):
         he.he_ct_unpack(P.q, 4, 11, np.zeros(10, dtype=np.uint8), 1)
