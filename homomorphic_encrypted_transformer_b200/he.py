@@ -250,6 +250,9 @@ def he_keygen_upload(ctx, kind, step, s, a, e):
     s = np.ascontiguousarray(s, dtype=np.int8)
     a = np.ascontiguousarray(a, dtype=np.uint64)
     e = np.ascontiguousarray(e, dtype=np.int32)
+    nd = he_key_digits(ctx)
+    if s.size < ctx.N or a.size < nd * len(ctx.primes) * ctx.N or e.size < nd * ctx.N:
+        raise ValueError("he_keygen_upload: s needs N, a digits*(L+K)*N and e digits*N entries")
     _check(ctx, _lib.he_keygen_upload(ctx.ptr, kind, int(step), _ptr(s), _ptr(a), _ptr(e)))
 
 
@@ -403,6 +406,9 @@ def he_attention_output(ctx, a, v, n_tok, offsets, out):
 def he_rotate_batch_host(ctx, h_in, level, steps, h_out):
     """h_in, h_out: host arrays (numpy or pinned torch CPU tensors) of [n][2][level][N] uint64."""
     st = np.ascontiguousarray(steps, dtype=np.int32)
+    need = len(st) * 2 * int(level) * ctx.N * 8
+    if 1 <= level <= ctx.L and (_nbytes(h_in) < need or _nbytes(h_out) < need):  # (a bad level: the library's error)
+        raise ValueError("he_rotate_batch_host: buffers shorter than %d bytes" % need)
     _check(ctx, _lib.he_rotate_batch_host(ctx.ptr, _ptr(h_in), level, _ptr(st), _ptr(h_out), len(st)))
 
 
