@@ -141,7 +141,8 @@ class Context:
         self.psi = [int(v) for v in ps]
 
     def __del__(self):
-        if getattr(self, "ptr", None):
+        # at interpreter exit the module's globals may already be gone
+        if getattr(self, "ptr", None) and _lib is not None:
             _lib.he_ctx_destroy(self.ptr)
             self.ptr = None
 
