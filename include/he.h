@@ -29,9 +29,9 @@
  *    limb-major, c0 then c1, in the evaluation (NTT) domain: storage index j
  *    holds the value at psi^(2*brev(j)+1), psi the smallest primitive 2N-th
  *    root of unity mod the limb's prime.
- *  - Ciphertext and plaintext buffers are device memory owned by the caller.
- *    The context owns its tables, keys and scratch, and frees them in
- *    he_ctx_destroy().
+ *  - Ciphertext and plaintext buffers are device memory owned by the caller,
+ *    32-byte aligned.  The context owns its tables, keys and scratch, and
+ *    frees them in he_ctx_destroy().
  *  - A context is not thread-safe: one host thread at a time.
  */
 #ifndef HE_B200_H
@@ -51,7 +51,7 @@ extern "C" {
 #define HE_EDOMAIN (-4)  /* operand not in the evaluation (NTT) domain */
 #define HE_ENOMEM (-5)   /* device allocation failed */
 #define HE_ECUDA (-6)    /* CUDA runtime error (message in he_last_error) */
-#define HE_ETIMEOUT (-7) /* reserved: a bounded device wait gave up */
+#define HE_ETIMEOUT (-7) /* a bounded device wait gave up (reported by he_sync) */
 
 #define HE_KEY_ROTATION 0
 #define HE_KEY_RELIN 1
@@ -112,11 +112,12 @@ int he_ctx_destroy(he_ctx* ctx);
  * the same sizes (that run sizes the context's scratch).  A call that would
  * have to grow its scratch while the stream is being captured returns
  * HE_EINVAL before any CUDA work, leaving the capture intact.  Key
- * generation, key download, the host-buffer entry point, he_sync and
+ * generation, key download, the host-buffer entry points, he_sync and
  * profiling synchronise and cannot be captured.
  */
 int he_set_stream(he_ctx* ctx, void* cuda_stream);
-/* Blocks until the context's stream is idle; returns HE_ECUDA on a pending error. */
+/* Blocks until the context's stream is idle; returns HE_ECUDA on a pending
+ * CUDA error, HE_ETIMEOUT if a bounded device wait gave up. */
 int he_sync(he_ctx* ctx);
 const char* he_last_error(const he_ctx* ctx);
 /* Host copies of the n_q + n_p primes / of their psi (smallest primitive 2N-th roots). */
