@@ -143,13 +143,19 @@ def test_ps15_gelu_coefficients():
         assert np.array_equal(st.from_gpu(outs[i]), want["c"])
 
 
-def test_bsgs_small():
+BSGS_SMALL = [(4, 4, 2, 2), (4, 4, 2, 3), (8, 2, 13, 2)]
+
+
+@pytest.mark.parametrize("bs,gs,n_in,n_grp", BSGS_SMALL, ids=["-".join(map(str, c)) for c in BSGS_SMALL])
+def test_bsgs_small(bs, gs, n_in, n_grp):
     """y = W x by diagonals with BSGS on N=2^11: 16 features x 64 tokens,
-    4 baby x 4 giant steps, 2 input / 2 output blocks, 2 token groups."""
+    bs baby x gs giant steps, n_in input / 2 output blocks, n_grp token
+    groups: two groups per staged pass, an odd group count (a last pass of
+    one group), and 104 (input, baby step) terms per output."""
     he = lib()
     st = Setup(11, 3, 1, 3, seed=21)
     P = st.P
-    n_feat, n_tok, bs, gs, n_in, n_out, n_grp = 16, 64, 4, 4, 2, 2, 2
+    n_feat, n_tok, n_out = 16, 64, 2
     level = 3
     W = S.weights(st.seed, (n_out * n_feat, n_in * n_feat), -0.05, 0.05)
     steps = sorted({n_tok * b for b in range(1, bs)} | {n_tok * bs * g for g in range(1, gs)})
