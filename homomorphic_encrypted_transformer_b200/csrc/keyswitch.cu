@@ -1698,9 +1698,28 @@ extern "C" int he_rotate_batch(he_ctx* c, const he_ct* in, const int32_t* steps,
 
 // Host-buffer rotation, pipelined: the ciphertexts, ordered by Galois element
 // (so that a chunk holds few distinct keys), go through the GPU in chunks of
-// kIoChunk.  Two staging buffers per direction let chunk k+1's upload and
-// chunk k-1's download (one copy engine each) overlap chunk k's rotation.
+// at most kIoChunk.  Two staging buffers per direction let chunk k+1's upload
+// and chunk k-1's download (one copy engine each) overlap chunk k's rotation.
 constexpr int kIoChunk = 8;
+
+// Chunk sizes of a pipeline of n ciphertexts: 2 and 4 first and last (when n
+// leaves at least one full chunk between them), so that the upload before the
+// first rotation and the download after the last, when one copy engine works
+// alone, are short; the rest in near-equal chunks of at most kIoChunk.
+static std::vector<int> io_plan(int n) {
+    std::vector<int> head;
+    int rem = n;
+    for (int r : {2, 4})
+        if (rem >= 2 * r + kIoChunk) {
+            head.push_back(r);
+            rem -= 2 * r;
+        }
+    std::vector<int> plan = head;
+    const int nm = (rem + kIoChunk - 1) / kIoChunk;
+    for (int k = 0; k < nm; k++) plan.push_back(rem / nm + (k < rem % nm ? 1 : 0));
+    plan.insert(plan.end(), head.rbegin(), head.rend());
+    return plan;
+}
 
 static int io_setup(he_ctx* c, size_t words) {
     int rc;
@@ -1756,9 +1775,9 @@ static int rotate_batch_host(he_ctx* c, const uint8_t* h_in, int level, const in
     cudaEvent_t* up = c->io_ev;        // [2] upload of buffer b done
     cudaEvent_t* done = c->io_ev + 2;  // [2] rotation of buffer b done
     cudaEvent_t* down = c->io_ev + 4;  // [2] download of buffer b done
-    const int n_chunks = (n + chunk - 1) / chunk;
-    for (int k = 0; k < n_chunks; k++) {
-        const int b = k & 1, i0 = k * chunk, m = std::min(chunk, n - i0);
+    const std::vector<int> plan = io_plan(n);
+    for (int k = 0, i0 = 0; k < (int)plan.size(); i0 += plan[k], k++) {
+        const int b = k & 1, m = plan[k];
         uint64_t* din = c->io_buf + (size_t)b * chunk * ct_words;
         uint64_t* dout = c->io_buf + (size_t)(2 + b) * chunk * ct_words;
         uint64_t* wbase = c->io_buf + 4 * (size_t)chunk * ct_words;

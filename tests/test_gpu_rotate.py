@@ -153,9 +153,10 @@ def test_rotation_batch_host_buffers():
 
 
 def test_rotation_batch_host_buffers_pipelined():
-    """21 ciphertexts pass the host-buffer entry in three chunks (both staging
-    buffers reused); steps unsorted, repeated, and one identity rotation
-    (step N/2, Galois element 1)."""
+    """21 ciphertexts pass the host-buffer entry in six chunks (2, 4, 5, 4,
+    4, 2: both staging buffers reused, chunks of every size the plan makes);
+    steps unsorted, repeated, and one identity rotation (step N/2, Galois
+    element 1)."""
     he = lib()
     st = Setup(12, 3, 1, 3, seed=6)
     P = st.P
@@ -182,7 +183,7 @@ def test_rotation_batch_host_buffers_pipelined():
 
 def test_rotation_batch_host_buffers_full_size():
     """The host-buffer entry on the rotation batch (64 ciphertexts at
-    N=2^16, level 24, 16 keys; chunks of 8 ordered by step) gives the device
+    N=2^16, level 24, 16 keys; chunks of 2 to 8 ordered by step) gives the device
     entry's residues, ciphertext for ciphertext."""
     he = lib()
     st = Setup(16, 24, 8, 3, seed=S.master_seed(1))
@@ -203,7 +204,7 @@ def test_rotation_batch_host_buffers_full_size():
 
 def test_rotation_batch_host_wire():
     """The packed wire entry (he_rotate_batch_host_wire): 21 packed
-    ciphertexts in three chunks, steps unsorted and repeated and one identity
+    ciphertexts in six chunks, steps unsorted and repeated and one identity
     rotation; unpacked, the outputs equal the oracle's rotations, and the
     packed output equals the host packing of the unpacked entry's output."""
     he = lib()
