@@ -53,11 +53,12 @@ def parse():
                     help="keys with seeded a-halves (he_keygen_seeded_ex, HE_KEYGEN_SEEDED_A): only b stored, a "
                          "regenerated inside the key-switching kernels (rotation, hoisted, rotsum)")
     ap.add_argument("--case", default="rotation",
-                    choices=["rotation", "ntt", "rot_small", "ffn128", "ffn2048", "ps15", "tiny", "hoisted",
-                             "rotsum", "attention"],
+                    choices=["rotation", "ntt", "rot_small", "ps15_small", "ffn128", "ffn2048", "ps15", "tiny",
+                             "hoisted", "rotsum", "attention"],
                     help="rotation: the headline workload (default). ffn128 / ffn2048 / ps15 / tiny: the other "
-                         "workloads, one JSON line each. ntt / rot_small: kernel cases for profiler captures "
-                         "(NTT of 512 limbs, or 8 rotations with 2 keys)")
+                         "workloads, one JSON line each. ntt / rot_small / ps15_small: kernel cases for profiler "
+                         "captures (NTT of 512 limbs, 8 rotations with 2 keys, or the degree-15 evaluation of 8 "
+                         "ciphertexts)")
     return ap.parse_args()
 
 
@@ -398,6 +399,33 @@ def run_rot_small_case(args, local_rank):
         he.he_rotate_batch(ctx, xs, cs, ys)
     torch.cuda.synchronize()
     print(json.dumps({"case": "rot_small", "rotations": 8 * (args.warmup + args.steps)}))
+
+
+def run_ps15_small_case(args, local_rank):
+    """Kernel case for profiler captures: the degree-15 evaluation of 8
+    ciphertexts at level 24 (the tensor, relinearisation, fused rescale and
+    constant-multiply rescale launches of the degree-15 workload at an eighth
+    of its batch, ~1.2 GB)."""
+    import torch
+
+    from homomorphic_encrypted_transformer_b200 import he
+
+    torch.cuda.set_device(local_rank)
+    ctx = he.he_ctx_create(LOG_N, L, K, DNUM, stream=torch.cuda.current_stream())
+    N = ctx.N
+    master = S.master_seed(4)
+    s = S.secret(master, N)
+    a, e = S.key_draws(master, 2, ctx.primes, N, DNUM)
+    he.he_keygen_upload(ctx, he.HE_KEY_RELIN, 0, s, a, e)
+    h = S.uniform_residues(master, "ct_residues", ctx.primes[:L], N, lead=(8, 2))
+    x = torch.from_numpy(h.view(np.int64)).cuda()
+    y = torch.empty_like(x)
+    coeffs = S.poly_coeffs(master, 15)
+    xs = [he.Ciphertext(x[i], LEVEL, 2.0 ** 40) for i in range(8)]
+    for _ in range(args.warmup + args.steps):
+        he.he_poly_eval_ps15(ctx, xs, coeffs, 2.0 ** 62, [he.Ciphertext(y[i], LEVEL, 2.0 ** 40) for i in range(8)])
+    torch.cuda.synchronize()
+    print(json.dumps({"case": "ps15_small", "evaluations": 8 * (args.warmup + args.steps)}))
 
 
 # ------------------------------------------------------------------ other workloads
@@ -1118,6 +1146,8 @@ def main():
             print(json.dumps(ntt_case(args.steps, args.warmup, local_rank)), flush=True)
         elif args.case == "rot_small":
             run_rot_small_case(args, local_rank)
+        elif args.case == "ps15_small":
+            run_ps15_small_case(args, local_rank)
         elif args.case in ("ffn128", "ffn2048", "ps15", "tiny", "hoisted", "rotsum", "attention"):
             print(json.dumps(workload_case(args.case, args.steps, args.warmup, args.cpu_seconds, local_rank,
                                            with_cpu=not args.no_cpu_baseline, seeded_a=args.seeded_a)), flush=True)

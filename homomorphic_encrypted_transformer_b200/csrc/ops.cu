@@ -313,25 +313,49 @@ __global__ void k_add_const_many(MutPtrList io, RowConst kc, const DevPrime* __r
 
 // d_i = (a0 b0, a0 b1 + a1 b0, a1 b1) of the pairs (a_i, b_i), [3][level][N]
 // a_i and b_i hold level or more limbs per polynomial: their c1 starts at
-// limb room_a / room_b (the first `level` limbs of each polynomial are read)
+// limb room_a / room_b (the first `level` limbs of each polynomial are read).
+// Two adjacent coefficients per thread (16-byte accesses).  Limbs of primes
+// below 2^41 take signed FP64 rounded-quotient products (four per
+// coefficient, one canonicalisation per output); the others Montgomery
+// products, corrected by R^2 R^-1 after the sum.
 __global__ void k_tensor_many(PtrList pa, PtrList pb, MutPtrList pd, int level, int room_a, int room_b,
-                              const DevPrime* __restrict__ pr, int logn) {
+                              const DevPrime* __restrict__ pr, const FpMod* __restrict__ fpm, int logn) {
     const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y, i = blockIdx.z;
+    const int c = 2 * (blockIdx.x * blockDim.x + threadIdx.x), r = blockIdx.y, i = blockIdx.z;
     if (c >= N) return;
     const uint64_t* a = pa.p[i];
     const uint64_t* b = pb.p[i];
     uint64_t* d = pd.p[i];
-    DevPrime p = pr[r];
-    size_t k0 = (size_t)r * N + c;
-    uint64_t a0 = a[k0], a1 = a[(size_t)(room_a + r) * N + c], b0 = b[k0], b1 = b[(size_t)(room_b + r) * N + c];
-    // Montgomery products a0 b0 R^-1 etc.; the sum is taken before the final
-    // correction by R^2 R^-1.
-    uint64_t m00 = mont_mul(a0, b0, p), m01 = mont_mul(a0, b1, p), m10 = mont_mul(a1, b0, p),
-             m11 = mont_mul(a1, b1, p);
-    d[k0] = mont_mul(m00, p.r2, p);
-    d[(size_t)(level + r) * N + c] = mont_mul(add_mod(m01, m10, p.q), p.r2, p);
-    d[(size_t)(2 * level + r) * N + c] = mont_mul(m11, p.r2, p);
+    const DevPrime p = pr[r];
+    const size_t k0 = (size_t)r * N + c;
+    const ulonglong2 A0 = __ldg(reinterpret_cast<const ulonglong2*>(a + k0));
+    const ulonglong2 A1 = __ldg(reinterpret_cast<const ulonglong2*>(a + (size_t)(room_a + r) * N + c));
+    const ulonglong2 B0 = __ldg(reinterpret_cast<const ulonglong2*>(b + k0));
+    const ulonglong2 B1 = __ldg(reinterpret_cast<const ulonglong2*>(b + (size_t)(room_b + r) * N + c));
+    const uint64_t a0[2] = {A0.x, A0.y}, a1[2] = {A1.x, A1.y}, b0[2] = {B0.x, B0.y}, b1[2] = {B1.x, B1.y};
+    uint64_t o0[2], o1[2], o2[2];
+    if (p.q < kFpPrimeLimit) {
+        const FpMod m = fpm[r];
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            const double x0 = u2d(a0[e]), x1 = u2d(a1[e]), y0 = u2d(b0[e]), y1 = u2d(b1[e]);
+            o0[e] = d2u(fp_modmul(x0, y0, m));
+            o1[e] = d2u(fp_canon(__dadd_rn(fp_mulmod_s(x0, y1, m), fp_mulmod_s(x1, y0, m)), m));
+            o2[e] = d2u(fp_modmul(x1, y1, m));
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            const uint64_t m00 = mont_mul(a0[e], b0[e], p), m01 = mont_mul(a0[e], b1[e], p),
+                           m10 = mont_mul(a1[e], b0[e], p), m11 = mont_mul(a1[e], b1[e], p);
+            o0[e] = mont_mul(m00, p.r2, p);
+            o1[e] = mont_mul(add_mod(m01, m10, p.q), p.r2, p);
+            o2[e] = mont_mul(m11, p.r2, p);
+        }
+    }
+    *reinterpret_cast<ulonglong2*>(d + k0) = make_ulonglong2(o0[0], o0[1]);
+    *reinterpret_cast<ulonglong2*>(d + (size_t)(level + r) * N + c) = make_ulonglong2(o1[0], o1[1]);
+    *reinterpret_cast<ulonglong2*>(d + (size_t)(2 * level + r) * N + c) = make_ulonglong2(o2[0], o2[1]);
 }
 
 // --------------------------------------------------------------- host side
@@ -446,7 +470,9 @@ int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vecto
     if (room_a == 0) room_a = level;
     if (room_b == 0) room_b = level;
     if (room_a < level || room_b < level) return set_err(c, HE_ELEVEL, "hmult: input room below level %d", level);
-    const int gx = (N + TB - 1) / TB;
+    const int gx2 = (N / 2 + TB - 1) / TB;
+    int fp_l = 0;
+    for (int r = 0; r < level; r++) fp_l += fp_prime(c, r);
     const size_t per = (size_t)5 * level * N;  // d0 d1 d2 | relinearised [2][level]
     const int chunk = 64;
     for (int i0 = 0; i0 < n; i0 += chunk) {
@@ -463,10 +489,12 @@ int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vecto
             pd.p[i] = base + per * i;
         }
         prof_begin(c, HE_PROF_ELEMENTWISE);
-        k_tensor_many<<<dim3(gx, level, m), TB, 0, c->stream>>>(pa, pb, pd, level, room_a, room_b, c->d_prime,
-                                                                c->log_n);
+        k_tensor_many<<<dim3(gx2, level, m), TB, 0, c->stream>>>(pa, pb, pd, level, room_a, room_b, c->d_prime,
+                                                                 c->d_fpmod, c->log_n);
         if ((rc = lc(c, "tensor"))) return rc;
-        prof_end(c, HE_PROF_ELEMENTWISE, 7.0 * m * level * 8.0 * N, 7.0 * m * level * N);
+        // 4 products per coefficient on FP64 limbs, 7 (with the corrections) on the others
+        prof_end(c, HE_PROF_ELEMENTWISE, 7.0 * m * level * 8.0 * N, (7.0 * level - 3.0 * fp_l) * m * N,
+                 4.0 * fp_l * m * N);
         for (int i = 0; i < m; i++) {
             uint64_t* d = base + per * i;
             io.galois.push_back(0);
