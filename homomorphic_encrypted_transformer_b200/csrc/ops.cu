@@ -213,6 +213,7 @@ __global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
     const int r = blockIdx.x * Cf::TR + threadIdx.x / (Cf::C / 16);
     const int j0 = r * Cf::C + 16 * row_lane<LOGN>();
     const uint64_t* a = tmp + (size_t)y * Cf::N + (size_t)r * Cf::C;
+    prefetch_l2(io.in.p[i] + ((size_t)poly * lin + t) * Cf::N + j0);  // read after the stages
     uint64_t v[16];
     if (q < kFpPrimeLimit) {
         const FpMod m = fpm[t];
