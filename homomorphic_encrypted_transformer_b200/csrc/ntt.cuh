@@ -385,10 +385,6 @@ __device__ __forceinline__ void row_load_strided(T (&x)[16], const uint64_t* row
     for (int k = 0; k < 16; k++) x[k] = raw_in(row[p + CS * k], T());
 }
 
-// Starts bringing the 128-byte line at p into L2 (a hint: nothing waits on
-// it); for the inputs a fused row pass reads only after its stages.
-__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
-
 // Brings the twiddles of the last four stages of row r, which thread p uses
 // after the exchange, towards L1 while the first four stages run: one
 // prefetch per stage (its twiddles span at most 128 bytes, line-aligned).

@@ -198,6 +198,9 @@ struct RescaleIo {
     PtrList add;     // addend_i at level lv-1, or unused
 };
 
+// Starts bringing the 128-byte line at p into L2 (a hint: nothing waits on it).
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 // Row pass of NTT(lift_r), then the combine.
 template <int LOGN>
 __global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
