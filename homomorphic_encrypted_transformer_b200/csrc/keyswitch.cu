@@ -1443,25 +1443,33 @@ int rotate_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t* ste
 // First part of a sum of rotations: s_o = base_o + sum_g (sigma_g(z0_{o,g}), 0)
 // over the key-switched terms (gal != 0) + z_{o,g} over the identity terms
 // (gal == 0, both polynomials); the key switches' ModDown adds the rest.
-// Term r = o G + g.  Grid (ceil(N/256), 2 level, outputs).
+// Term r = o G + g.  Positions c, c + 1 per thread: sigma maps the aligned
+// pair onto an aligned pair, so every term is one 16-byte load.
+// Grid (ceil(N/512), 2 level, outputs).
 __global__ void k_rot_presum(PtrList z, GalList gal, PtrList base, MutPtrList s, int G, int level,
                              const DevPrime* __restrict__ pr, int logn) {
     const int N = 1 << logn;
-    const int c = blockIdx.x * blockDim.x + threadIdx.x, row = blockIdx.y, o = blockIdx.z;
+    const int c = 2 * (blockIdx.x * blockDim.x + threadIdx.x), row = blockIdx.y, o = blockIdx.z;
     if (c >= N) return;
     const int poly = row / level, t = row - poly * level;
     const uint64_t q = pr[t].q;
     const size_t k = (size_t)row * N;  // this limb within a ciphertext
-    uint64_t acc = base.p[o] ? base.p[o][k + c] : 0;
+    ulonglong2 acc = base.p[o] ? *reinterpret_cast<const ulonglong2*>(base.p[o] + k + c) : make_ulonglong2(0, 0);
     for (int g = 0; g < G; g++) {
         const int r = o * G + g;
         const uint64_t gl = gal.g[r];
-        if (gl == 0)
-            acc = add_mod(acc, z.p[r][k + c], q);
-        else if (poly == 0)
-            acc = add_mod(acc, z.p[r][k + automorph_src(c, logn, gl)], q);
+        if (gl == 0) {
+            // may be the output itself (sums of identity terms only): a coherent load
+            const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(z.p[r] + k + c);
+            acc = make_ulonglong2(add_mod(acc.x, v.x, q), add_mod(acc.y, v.y, q));
+        } else if (poly == 0) {
+            const int src = automorph_src(c, logn, gl);
+            const ulonglong2 v = __ldg(reinterpret_cast<const ulonglong2*>(z.p[r] + k + (src & ~1)));
+            const bool sw = src & 1;
+            acc = make_ulonglong2(add_mod(acc.x, sw ? v.y : v.x, q), add_mod(acc.y, sw ? v.x : v.y, q));
+        }
     }
-    s.p[o][k + c] = acc;
+    *reinterpret_cast<ulonglong2*>(s.p[o] + k + c) = acc;
 }
 
 // Sums of rotations with one ModDown per output (the ModDown hoisting of
@@ -1537,7 +1545,7 @@ int rotate_sum_many(he_ctx* c, const he_ct* z, int n_out, int n_terms, const int
             sp.p[o] = g_eff ? S + (size_t)o * ctw : out[o0 + o].data;
         }
         prof_begin(c, HE_PROF_ELEMENTWISE);
-        k_rot_presum<<<dim3((unsigned)((N + 255) / 256), 2 * level, m), 256, 0, c->stream>>>(
+        k_rot_presum<<<dim3((unsigned)((N / 2 + 255) / 256), 2 * level, m), 256, 0, c->stream>>>(
             zp, gl, bp, sp, G, level, c->d_prime, c->log_n);
         int rc = lc(c, "rot_presum");
         if (rc) return rc;
@@ -1632,7 +1640,7 @@ int rotate_sum_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t*
             sp.p[o] = g_eff ? S + (size_t)o * ctw : out[i0 + o].data;
         }
         prof_begin(c, HE_PROF_ELEMENTWISE);
-        k_rot_presum<<<dim3((unsigned)((N + 255) / 256), 2 * level, m), 256, 0, c->stream>>>(
+        k_rot_presum<<<dim3((unsigned)((N / 2 + 255) / 256), 2 * level, m), 256, 0, c->stream>>>(
             zp, gl, bp, sp, G, level, c->d_prime, c->log_n);
         int rc = lc(c, "rot_presum");
         if (rc) return rc;
