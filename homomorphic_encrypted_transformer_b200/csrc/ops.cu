@@ -275,44 +275,58 @@ __global__ void k_copy_many(PtrList src, MutPtrList dst, size_t words2) {
 
 
 
-// Batched helpers over n <= kMaxBatch ciphertexts (grid z = ciphertext).
+// Batched helpers over n <= kMaxBatch ciphertexts (grid z = ciphertext), two
+// adjacent coefficients per thread (16-byte accesses; limbs start on
+// 16-byte boundaries).
+__device__ __forceinline__ ulonglong2 ld2(const uint64_t* p) { return *reinterpret_cast<const ulonglong2*>(p); }
+__device__ __forceinline__ void st2(uint64_t* p, uint64_t a, uint64_t b) {
+    *reinterpret_cast<ulonglong2*>(p) = make_ulonglong2(a, b);
+}
+
 // out_i[poly][r] = K_r in_i[poly][r] for r < lv, in_i at level lin >= lv
 // (limbs lv..lin-1 dropped on the way).
 __global__ void k_mul_const_many(PtrList in, MutPtrList out, RowConst kc, int lin, int lv,
                                  const DevPrime* __restrict__ pr, int logn) {
     const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, y = blockIdx.y, i = blockIdx.z;
+    const int c = 2 * (blockIdx.x * blockDim.x + threadIdx.x), y = blockIdx.y, i = blockIdx.z;
     if (c >= N) return;
     const int poly = y / lv, r = y - poly * lv;
-    const uint64_t x = in.p[i][((size_t)poly * lin + r) * N + c];
-    out.p[i][((size_t)poly * lv + r) * N + c] = mul_shoup(x, kc.v[r].x, kc.v[r].y, pr[r].q);
+    const uint64_t q = pr[r].q;
+    const ulonglong2 x = ld2(in.p[i] + ((size_t)poly * lin + r) * N + c);
+    st2(out.p[i] + ((size_t)poly * lv + r) * N + c, mul_shoup(x.x, kc.v[r].x, kc.v[r].y, q),
+        mul_shoup(x.y, kc.v[r].x, kc.v[r].y, q));
 }
 
 // out_i = in_i keeping limbs r < lv of both polynomials (out_i != in_i)
 __global__ void k_drop_many(PtrList in, MutPtrList out, int lin, int lv, int logn) {
     const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, y = blockIdx.y, i = blockIdx.z;
+    const int c = 2 * (blockIdx.x * blockDim.x + threadIdx.x), y = blockIdx.y, i = blockIdx.z;
     if (c >= N) return;
     const int poly = y / lv, r = y - poly * lv;
-    out.p[i][((size_t)poly * lv + r) * N + c] = in.p[i][((size_t)poly * lin + r) * N + c];
+    const ulonglong2 x = ld2(in.p[i] + ((size_t)poly * lin + r) * N + c);
+    st2(out.p[i] + ((size_t)poly * lv + r) * N + c, x.x, x.y);
 }
 
 // o_i = a_i + b_i (level lv)
 __global__ void k_add_many(PtrList a, PtrList b, MutPtrList o, int lv, const DevPrime* __restrict__ pr, int logn) {
     const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, y = blockIdx.y, i = blockIdx.z;
+    const int c = 2 * (blockIdx.x * blockDim.x + threadIdx.x), y = blockIdx.y, i = blockIdx.z;
     if (c >= N) return;
     const size_t k = (size_t)y * N + c;
-    o.p[i][k] = add_mod(a.p[i][k], b.p[i][k], pr[y % lv].q);
+    const uint64_t q = pr[y % lv].q;
+    const ulonglong2 u = ld2(a.p[i] + k), v = ld2(b.p[i] + k);
+    st2(o.p[i] + k, add_mod(u.x, v.x, q), add_mod(u.y, v.y, q));
 }
 
 // c0 of io_i gains the constant polynomial K (every evaluation equals K)
 __global__ void k_add_const_many(MutPtrList io, RowConst kc, const DevPrime* __restrict__ pr, int logn) {
     const int N = 1 << logn;
-    int c = blockIdx.x * blockDim.x + threadIdx.x, r = blockIdx.y, i = blockIdx.z;
+    const int c = 2 * (blockIdx.x * blockDim.x + threadIdx.x), r = blockIdx.y, i = blockIdx.z;
     if (c >= N) return;
     uint64_t* a = io.p[i] + (size_t)r * N + c;
-    *a = add_mod(*a, kc.v[r].x, pr[r].q);
+    const uint64_t q = pr[r].q, kv = kc.v[r].x;
+    const ulonglong2 u = ld2(a);
+    st2(a, add_mod(u.x, kv, q), add_mod(u.y, kv, q));
 }
 
 // d_i = (a0 b0, a0 b1 + a1 b0, a1 b1) of the pairs (a_i, b_i), [3][level][N]
@@ -533,7 +547,7 @@ static RowConst row_const_shoup(const he_ctx* c, int level, int64_t K) {
 int mul_const_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int lin,
                    int lv, int64_t K) {
     const RowConst kc = row_const_shoup(c, lv, K);
-    const int n = (int)in.size(), gx = (c->N + TB - 1) / TB;
+    const int n = (int)in.size(), gx2 = (c->N / 2 + TB - 1) / TB;
     for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
         const int m = std::min(kMaxBatch, n - i0);
         PtrList pi;
@@ -543,7 +557,7 @@ int mul_const_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std:
             po.p[i] = out[i0 + i];
         }
         prof_begin(c, HE_PROF_ELEMENTWISE);
-        k_mul_const_many<<<dim3(gx, 2 * lv, m), TB, 0, c->stream>>>(pi, po, kc, lin, lv, c->d_prime, c->log_n);
+        k_mul_const_many<<<dim3(gx2, 2 * lv, m), TB, 0, c->stream>>>(pi, po, kc, lin, lv, c->d_prime, c->log_n);
         int rc = lc(c, "mul_const");
         if (rc) return rc;
         prof_end(c, HE_PROF_ELEMENTWISE, 4.0 * m * lv * 8.0 * c->N, 2.0 * m * lv * c->N);
@@ -566,7 +580,7 @@ int mul_const_rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, in
 
 // out_i = in_i keeping limbs < lv (out_i != in_i)
 int drop_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int lin, int lv) {
-    const int n = (int)in.size(), gx = (c->N + TB - 1) / TB;
+    const int n = (int)in.size(), gx2 = (c->N / 2 + TB - 1) / TB;
     for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
         const int m = std::min(kMaxBatch, n - i0);
         PtrList pi;
@@ -576,7 +590,7 @@ int drop_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vect
             po.p[i] = out[i0 + i];
         }
         prof_begin(c, HE_PROF_ELEMENTWISE);
-        k_drop_many<<<dim3(gx, 2 * lv, m), TB, 0, c->stream>>>(pi, po, lin, lv, c->log_n);
+        k_drop_many<<<dim3(gx2, 2 * lv, m), TB, 0, c->stream>>>(pi, po, lin, lv, c->log_n);
         int rc = lc(c, "drop");
         if (rc) return rc;
         prof_end(c, HE_PROF_ELEMENTWISE, 4.0 * m * lv * 8.0 * c->N);
@@ -587,7 +601,7 @@ int drop_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vect
 // o_i = a_i + b_i at level lv (o_i may equal a_i or b_i)
 int add_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector<const uint64_t*>& b,
              const std::vector<uint64_t*>& o, int lv) {
-    const int n = (int)a.size(), gx = (c->N + TB - 1) / TB;
+    const int n = (int)a.size(), gx2 = (c->N / 2 + TB - 1) / TB;
     for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
         const int m = std::min(kMaxBatch, n - i0);
         PtrList pa, pb;
@@ -598,7 +612,7 @@ int add_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector
             po.p[i] = o[i0 + i];
         }
         prof_begin(c, HE_PROF_ELEMENTWISE);
-        k_add_many<<<dim3(gx, 2 * lv, m), TB, 0, c->stream>>>(pa, pb, po, lv, c->d_prime, c->log_n);
+        k_add_many<<<dim3(gx2, 2 * lv, m), TB, 0, c->stream>>>(pa, pb, po, lv, c->d_prime, c->log_n);
         int rc = lc(c, "add");
         if (rc) return rc;
         prof_end(c, HE_PROF_ELEMENTWISE, 6.0 * m * lv * 8.0 * c->N);
@@ -610,13 +624,13 @@ int add_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector
 int add_const_many(he_ctx* c, const std::vector<uint64_t*>& io, int lv, int64_t K) {
     RowConst kc;
     for (int r = 0; r < lv; r++) kc.v[r] = make_ulonglong2(int_mod(K, c->primes[r]), 0);
-    const int n = (int)io.size(), gx = (c->N + TB - 1) / TB;
+    const int n = (int)io.size(), gx2 = (c->N / 2 + TB - 1) / TB;
     for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
         const int m = std::min(kMaxBatch, n - i0);
         MutPtrList po;
         for (int i = 0; i < m; i++) po.p[i] = io[i0 + i];
         prof_begin(c, HE_PROF_ELEMENTWISE);
-        k_add_const_many<<<dim3(gx, lv, m), TB, 0, c->stream>>>(po, kc, c->d_prime, c->log_n);
+        k_add_const_many<<<dim3(gx2, lv, m), TB, 0, c->stream>>>(po, kc, c->d_prime, c->log_n);
         int rc = lc(c, "add_const");
         if (rc) return rc;
         prof_end(c, HE_PROF_ELEMENTWISE, 2.0 * m * lv * 8.0 * c->N);
