@@ -920,9 +920,12 @@ def ps_eval_deg15(x, coeffs, rlk, params, top_scale=PS_TOP_SCALE):
       x3 = HMRR(x2, drop(x, l0-1))       level l0-2
       x4 = HMRR(x2, x2)                  level l0-2
       q_i(x) = sum_{j<4} c_{4i+j} x^j, built at (lambda, T): each x^j, j >= 1,
-        is dropped to lambda+1 limbs, multiplied by
-        K = round_half_away(c T q_lambda / S_j) and rescaled by q_lambda; the
-        constant adds round_half_away(c_{4i} T).  Its declared scale is T.
+        is dropped to lambda+1 limbs and multiplied by
+        K = round_half_away(c T q_lambda / S_j); the three products (all at
+        nominal scale T q_lambda) are summed and the sum rescaled once by
+        q_lambda; the constant adds round_half_away(c_{4i} T).  Its declared
+        scale is T.  (One rounding per block instead of one per term: the
+        pages fix no order, and rescaling is linear up to that rounding.)
       Horner: acc = q_3 at (l0-3, top_scale);
         acc = HMRR(acc, drop(x4)) + q_2;  acc = HMRR(acc, drop(x4)) + q_1;
         acc = HMRR(acc, drop(x4)) + q_0, each q_i built at the accumulator's
@@ -946,9 +949,11 @@ def ps_eval_deg15(x, coeffs, rlk, params, top_scale=PS_TOP_SCALE):
             c = float(coeffs[4 * i + j])
             xj = drop_level(pw[j], lam + 1)
             K = ps_const(c, T, params.q[lam], xj["scale"])
-            t = rescale(mul_const(xj, K, params), params)
+            t = mul_const(xj, K, params)
             acc = t if acc is None else make_ct(
-                np.stack([add_rows(acc["c"][k], t["c"][k], params.q[:lam]) for k in range(2)]), lam, T)
+                np.stack([add_rows(acc["c"][k], t["c"][k], params.q[:lam + 1]) for k in range(2)]), lam + 1,
+                T * float(params.q[lam]))
+        acc = rescale(make_ct(acc["c"], lam + 1, T * float(params.q[lam])), params)
         acc = add_const(acc, int(round_half_away(np.float64(float(coeffs[4 * i]) * T))), params)
         return make_ct(acc["c"], lam, T)
 
