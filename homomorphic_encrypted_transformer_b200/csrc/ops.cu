@@ -123,26 +123,52 @@ __global__ void k_key_canonical_seeded(const uint64_t* __restrict__ in, uint64_t
 }
 
 
-// Rescale of x (level lin, its first lv limbs kept, optionally times an
-// integer K) by q_l = q_{lv-1}, in the layout of the key switch's ModDown:
-//   last   = INTT((K) x_{lv-1})                              (coefficients)
+// Rescale of x (the sum of up to kRsTerms ciphertexts x_j, each at its own
+// level lin_j with its first lv limbs kept and optionally times an integer
+// K_j) by q_l = q_{lv-1}, in the layout of the key switch's ModDown:
+//   last   = INTT(x_{lv-1})                                  (coefficients)
 //   lift_r = [last]_{q_r} - (last > q_l/2 ? q_l : 0)          (r < lv-1, centred)
-//   out_r  = ((K) x_r - NTT(lift_r)) q_l^-1 mod q_r  (+ addend_r) (+ K0 on c0)
-// k_rescale_gather_last picks (K) x_{lv-1}; the forward column pass of
-// NTT(lift_r) computes the lift as it loads `last`, and the row pass ends
-// with the combine, so no lifted limb crosses HBM and the rescale takes two
-// transform launches where the unfused form took a lift, two passes and a
-// combine.  Residue for residue the same values.
+//   out_r  = (x_r - NTT(lift_r)) q_l^-1 mod q_r  (+ addend_r) (+ K0 on c0)
+// k_rescale_gather_last forms x_{lv-1}; the forward column pass of
+// NTT(lift_r) computes the lift as it loads `last`, and the row pass forms
+// x_r and ends with the combine, so neither the sum nor a lifted limb
+// crosses HBM and the rescale takes two transform launches where the
+// unfused form took a lift, two passes and a combine.  Residue for residue
+// the same values.
+constexpr int kRsTerms = 3;
 
-// last[i][poly] = (K) in_i[poly][lv-1] (still in the evaluation domain)
-__global__ void k_rescale_gather_last(PtrList in, uint64_t* __restrict__ last, int lin, int lv, RowConst kc,
-                                      int with_k, const DevPrime* __restrict__ pr, int logn) {
+struct RescaleIo {
+    PtrList in[kRsTerms];  // term j: x_{j,i} at level lin[j]
+    int lin[kRsTerms];
+    int nterm;             // 1..kRsTerms
+    int with_k;            // terms times their constants (else one term, as it is)
+    MutPtrList out;        // [2][lv-1][N]
+    PtrList add;           // addend_i at level lv-1, or unused
+};
+struct RescaleK {
+    RowConst k[kRsTerms];
+};
+
+// limb r of polynomial poly of the sum of the terms of ciphertext i at position c
+__device__ __forceinline__ uint64_t rs_term_sum(const RescaleIo& io, const RescaleK& kk, int i, int poly, int r,
+                                                size_t c, int N, uint64_t q) {
+    if (!io.with_k) return io.in[0].p[i][((size_t)poly * io.lin[0] + r) * N + c];
+    uint64_t acc = 0;
+    for (int j = 0; j < io.nterm; j++) {
+        const uint64_t x = io.in[j].p[i][((size_t)poly * io.lin[j] + r) * N + c];
+        acc = add_mod(acc, mul_shoup(x, kk.k[j].v[r].x, kk.k[j].v[r].y, q), q);
+    }
+    return acc;
+}
+
+// last[i][poly] = x_{lv-1} of ciphertext i (still in the evaluation domain)
+__global__ void k_rescale_gather_last(const RescaleIo io, const RescaleK kk, uint64_t* __restrict__ last, int lv,
+                                      const DevPrime* __restrict__ pr, int logn) {
     const int N = 1 << logn;
     int c = blockIdx.x * blockDim.x + threadIdx.x, poly = blockIdx.y, i = blockIdx.z;
     if (c >= N) return;
     const int r = lv - 1;
-    const uint64_t x = in.p[i][((size_t)poly * lin + r) * N + c];
-    last[((size_t)i * 2 + poly) * N + c] = with_k ? mul_shoup(x, kc.v[r].x, kc.v[r].y, pr[r].q) : x;
+    last[((size_t)i * 2 + poly) * N + c] = rs_term_sum(io, kk, i, poly, r, c, N, pr[r].q);
 }
 
 // Column pass of NTT(lift_r), the lift taken as the limb loads: rows
@@ -192,23 +218,16 @@ __global__ void __launch_bounds__(NttCfg<LOGN>::COL_THREADS, NTT_COL_MIN_BLOCKS)
         rescale_cols_body<LOGN>(sm, l, a, tw_all + (size_t)r * Cf::N, q, q, os, ql, qm);
 }
 
-struct RescaleIo {
-    PtrList in;      // x_i at level lin
-    MutPtrList out;  // [2][lv-1][N]
-    PtrList add;     // addend_i at level lv-1, or unused
-};
-
 // Starts bringing the 128-byte line at p into L2 (a hint: nothing waits on it).
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
 // Row pass of NTT(lift_r), then the combine.
 template <int LOGN>
 __global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
-    k_rescale_rows_combine(const uint64_t* __restrict__ tmp, const RescaleIo io, int lin, int lm1, const RowConst kc,
-                           int with_k, const RowConst k0, int add_k0, int with_add,
-                           const ulonglong2* __restrict__ qinv, const DevPrime* __restrict__ pr,
-                           const ulonglong2* __restrict__ tw_all, const double* __restrict__ twd_all,
-                           const FpMod* __restrict__ fpm) {
+    k_rescale_rows_combine(const uint64_t* __restrict__ tmp, const RescaleIo io, const RescaleK kk, int lm1,
+                           const RowConst k0, int add_k0, int with_add, const ulonglong2* __restrict__ qinv,
+                           const DevPrime* __restrict__ pr, const ulonglong2* __restrict__ tw_all,
+                           const double* __restrict__ twd_all, const FpMod* __restrict__ fpm) {
     using Cf = NttCfg<LOGN>;
     __shared__ uint64_t sm[Cf::TR * Cf::ROW_PITCH];
     const int y = blockIdx.y, ip = y / lm1, t = y - ip * lm1, i = ip >> 1, poly = ip & 1;
@@ -216,7 +235,8 @@ __global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
     const int r = blockIdx.x * Cf::TR + threadIdx.x / (Cf::C / 16);
     const int j0 = r * Cf::C + 16 * row_lane<LOGN>();
     const uint64_t* a = tmp + (size_t)y * Cf::N + (size_t)r * Cf::C;
-    prefetch_l2(io.in.p[i] + ((size_t)poly * lin + t) * Cf::N + j0);  // read after the stages
+    for (int j = 0; j < io.nterm; j++)  // read after the stages
+        prefetch_l2(io.in[j].p[i] + ((size_t)poly * io.lin[j] + t) * Cf::N + j0);
     uint64_t v[16];
     if (q < kFpPrimeLimit) {
         const FpMod m = fpm[t];
@@ -232,21 +252,29 @@ __global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
 #pragma unroll
         for (int k = 0; k < 16; k++) v[k] = fwd_canon(x[k], q);
     }
-    const uint64_t* xp = io.in.p[i] + ((size_t)poly * lin + t) * Cf::N + j0;
     uint64_t* op = io.out.p[i] + ((size_t)poly * lm1 + t) * Cf::N + j0;
     const uint64_t* ap = with_add ? io.add.p[i] + ((size_t)poly * lm1 + t) * Cf::N + j0 : nullptr;
-    const ulonglong2 w = qinv[t], kk = kc.v[t];
+    const ulonglong2 w = qinv[t];
     const bool k0_here = add_k0 && poly == 0;
     const uint64_t kv = k0.v[t].x;
 #pragma unroll
     for (int k = 0; k < 4; k++) {
         uint64_t z[4];
-        ldg256_ro(xp + 4 * k, z[0], z[1], z[2], z[3]);
+        if (io.with_k) {
+            z[0] = z[1] = z[2] = z[3] = 0;
+            for (int j = 0; j < io.nterm; j++) {
+                uint64_t e4[4];
+                ldg256_ro(io.in[j].p[i] + ((size_t)poly * io.lin[j] + t) * Cf::N + j0 + 4 * k, e4[0], e4[1], e4[2],
+                          e4[3]);
+                const ulonglong2 kj = kk.k[j].v[t];
 #pragma unroll
-        for (int e = 0; e < 4; e++) {
-            const uint64_t xv = with_k ? mul_shoup(z[e], kk.x, kk.y, q) : z[e];
-            z[e] = mul_shoup(xv + q - v[4 * k + e], w.x, w.y, q);
+                for (int e = 0; e < 4; e++) z[e] = add_mod(z[e], mul_shoup(e4[e], kj.x, kj.y, q), q);
+            }
+        } else {
+            ldg256_ro(io.in[0].p[i] + ((size_t)poly * io.lin[0] + t) * Cf::N + j0 + 4 * k, z[0], z[1], z[2], z[3]);
         }
+#pragma unroll
+        for (int e = 0; e < 4; e++) z[e] = mul_shoup(z[e] + q - v[4 * k + e], w.x, w.y, q);
         if (ap) {  // the addend may be the output itself: a coherent load
             uint64_t s0, s1, s2, s3;
             ldg256(ap + 4 * k, s0, s1, s2, s3);
@@ -394,20 +422,38 @@ static int ct_ok(he_ctx* c, const he_ct* x, const char* what) {
     return HE_OK;
 }
 
-// The rescale path above for n ciphertexts: out_i = rescale((K) in_i) (+
-// addend_i) (+ K0 on c0), in_i at level lin, its first lv limbs kept.
-// out_i = in_i (in place) goes through a staging buffer: c1's limbs move
-// down, which would overwrite input another block has still to read.
-static int rescale_fused(he_ctx* c, const std::vector<const uint64_t*>& in, int lin, int lv, const RowConst* kc,
-                         const std::vector<uint64_t*>& out, const std::vector<const uint64_t*>& addend, bool add_k0,
-                         int64_t K0) {
-    const int N = c->N, n = (int)in.size(), lm1 = lv - 1;
-    if (lv < 2 || lin < lv) return set_err(c, HE_ELEVEL, "rescale: level %d of %d has no prime to drop", lv, lin);
+// One term of a fused rescale: ciphertexts in[i] at level lin, their first
+// lv limbs kept, times the row constants *kc (or as they are: kc null).
+struct RsTerm {
+    const std::vector<const uint64_t*>* in;
+    int lin;
+    const RowConst* kc;
+};
+
+// The rescale path above for n ciphertexts: out_i = rescale(sum_j (K_j)
+// in_{j,i}) (+ addend_i) (+ K0 on c0), at most kRsTerms terms; several
+// terms need their constants.  An out_i equal to one of its inputs (in
+// place) goes through a staging buffer: c1's limbs move down, which would
+// overwrite input another block has still to read.
+static int rescale_fused(he_ctx* c, const RsTerm* terms, int nterm, int lv, const std::vector<uint64_t*>& out,
+                         const std::vector<const uint64_t*>& addend, bool add_k0, int64_t K0) {
+    const int N = c->N, n = (int)out.size(), lm1 = lv - 1;
+    if (nterm < 1 || nterm > kRsTerms || (nterm > 1 && !terms[0].kc))
+        return set_err(c, HE_EINVAL, "rescale: %d terms", nterm);
+    for (int j = 0; j < nterm; j++) {
+        if (lv < 2 || terms[j].lin < lv)
+            return set_err(c, HE_ELEVEL, "rescale: level %d of %d has no prime to drop", lv, terms[j].lin);
+        if ((int)terms[j].in->size() != n || (!terms[j].kc) != (!terms[0].kc))
+            return set_err(c, HE_EINVAL, "rescale: term lists");
+    }
     const bool with_add = !addend.empty();
     if (with_add && (int)addend.size() != n) return set_err(c, HE_EINVAL, "rescale: addend list length");
-    RowConst k1, k0;
-    if (kc) k1 = *kc;
+    RescaleK kk;
+    RowConst k0;
+    for (int j = 0; j < nterm; j++)
+        if (terms[j].kc) kk.k[j] = *terms[j].kc;
     for (int r = 0; r < lm1; r++) k0.v[r] = make_ulonglong2(add_k0 ? int_mod(K0, c->primes[r]) : 0, 0);
+    const bool with_k = terms[0].kc != nullptr;
     const int gx = (N + TB - 1) / TB;
     const uint64_t ql = c->primes[lv - 1];
     const double limbB = 8.0 * N;
@@ -423,14 +469,20 @@ static int rescale_fused(he_ctx* c, const std::vector<const uint64_t*>& in, int 
         uint64_t* tmp = last + (size_t)2 * m * N;
         uint64_t* stage = tmp + (size_t)2 * m * lm1 * N;
         RescaleIo io;
+        io.nterm = nterm;
+        io.with_k = with_k ? 1 : 0;
+        for (int j = 0; j < kRsTerms; j++) io.lin[j] = j < nterm ? terms[j].lin : 0;
         PtrList sback;
         MutPtrList dback;
         int n_back = 0, fp_rows_n = 0;
         for (int r = 0; r < lm1; r++) fp_rows_n += fp_prime(c, r);
         for (int i = 0; i < m; i++) {
-            io.in.p[i] = in[i0 + i];
+            bool inplace = false;
+            for (int j = 0; j < nterm; j++) {
+                io.in[j].p[i] = (*terms[j].in)[i0 + i];
+                inplace = inplace || out[i0 + i] == io.in[j].p[i];
+            }
             io.add.p[i] = with_add ? addend[i0 + i] : nullptr;
-            const bool inplace = out[i0 + i] == in[i0 + i];
             io.out.p[i] = inplace ? stage + (size_t)i * 2 * lm1 * N : out[i0 + i];
             if (inplace) {
                 sback.p[n_back] = io.out.p[i];
@@ -438,10 +490,9 @@ static int rescale_fused(he_ctx* c, const std::vector<const uint64_t*>& in, int 
             }
         }
         prof_begin(c, HE_PROF_RESCALE);
-        k_rescale_gather_last<<<dim3(gx, 2, m), TB, 0, c->stream>>>(io.in, last, lin, lv, k1, kc ? 1 : 0,
-                                                                    c->d_prime, c->log_n);
+        k_rescale_gather_last<<<dim3(gx, 2, m), TB, 0, c->stream>>>(io, kk, last, lv, c->d_prime, c->log_n);
         if ((rc = lc(c, "rescale_gather"))) return rc;
-        prof_end(c, HE_PROF_RESCALE, 4.0 * m * limbB, kc ? 2.0 * m * N : 0);
+        prof_end(c, HE_PROF_RESCALE, (2.0 + 2.0 * nterm) * m * limbB, with_k ? 2.0 * nterm * m * N : 0);
         std::vector<int> pl(1, lv - 1);
         if ((rc = ntt_inv_set(c, rowset_contig(last, 1, N, pl), 2 * m))) return rc;
         const double rows = 2.0 * m * lm1, rows_fp = 2.0 * m * fp_rows_n;
@@ -456,13 +507,13 @@ static int rescale_fused(he_ctx* c, const std::vector<const uint64_t*>& in, int 
         prof_begin(c, HE_PROF_RESCALE);
 #define HE_RS_ROWS(LN)                                                                                              \
     k_rescale_rows_combine<LN><<<dim3(NttCfg<LN>::ROW_TILES, 2 * m * lm1), NttCfg<LN>::ROW_THREADS, 0, c->stream>>>( \
-        tmp, io, lin, lm1, k1, kc ? 1 : 0, k0, add_k0 ? 1 : 0, with_add ? 1 : 0, c->d_rs_inv + (size_t)lm1 * c->L,   \
-        c->d_prime, c->d_tw_fwd, c->d_twd_fwd, c->d_fpmod)
+        tmp, io, kk, lm1, k0, add_k0 ? 1 : 0, with_add ? 1 : 0, c->d_rs_inv + (size_t)lm1 * c->L, c->d_prime,        \
+        c->d_tw_fwd, c->d_twd_fwd, c->d_fpmod)
         HE_NTT_LOGN_SWITCH(c, HE_RS_ROWS)
 #undef HE_RS_ROWS
         if ((rc = lc(c, "rescale_rows"))) return rc;
-        prof_end(c, HE_PROF_RESCALE, (with_add ? 4.0 : 3.0) * rows * limbB,
-                 0.5 * N * rows * sh.s2 + (kc ? 2.0 : 1.0) * N * rows, 0.5 * N * rows_fp * sh.s2);
+        prof_end(c, HE_PROF_RESCALE, ((with_add ? 3.0 : 2.0) + nterm) * rows * limbB,
+                 0.5 * N * rows * sh.s2 + (with_k ? 1.0 + nterm : 1.0) * N * rows, 0.5 * N * rows_fp * sh.s2);
         if (n_back) {
             prof_begin(c, HE_PROF_RESCALE);
             k_copy_many<<<dim3(c->sm_count * 4, n_back), TB, 0, c->stream>>>(sback, dback, (size_t)lm1 * N);
@@ -475,7 +526,8 @@ static int rescale_fused(he_ctx* c, const std::vector<const uint64_t*>& in, int 
 
 int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int level,
                  const std::vector<const uint64_t*>& addend) {
-    return rescale_fused(c, in, level, level, nullptr, out, addend, false, 0);
+    const RsTerm t{&in, level, nullptr};
+    return rescale_fused(c, &t, 1, level, out, addend, false, 0);
 }
 
 // HMult + relinearisation + rescale of n pairs at one level.
@@ -565,17 +617,25 @@ int mul_const_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std:
     return HE_OK;
 }
 
-// out_i (+)= rescale(K in_i dropped to lv limbs) at level lv - 1, and, with
-// add_k0, K0 added to c0 after that; in_i at level lin >= lv, out_i apart
-// from every in_i.  Equal, residue for residue, to mul_const_many into a
-// temporary, rescale_many of it, add_many into out_i (accumulate) and
-// add_const_many (add_k0), without the intermediate ciphertexts in HBM.
-int mul_const_rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, int lin, int lv, int64_t K,
-                           const std::vector<uint64_t*>& out, bool accumulate, bool add_k0, int64_t K0) {
-    const RowConst kc = row_const_shoup(c, lv, K);
-    std::vector<const uint64_t*> addend;
-    if (accumulate) addend.assign(out.begin(), out.end());
-    return rescale_fused(c, in, lin, lv, &kc, out, addend, add_k0, K0);
+// out_i = rescale(sum_j K_j in_{j,i}, each dropped to lv limbs) at level
+// lv - 1, and, with add_k0, K0 added to c0 after that; in_{j,i} at level
+// lin_j >= lv, out_i apart from every input; at most kRsTerms terms.  Equal,
+// residue for residue, to mul_const_many of each term into a temporary,
+// add_many of them, rescale_many of the sum and add_const_many (add_k0),
+// without the intermediate ciphertexts in HBM.
+int mul_const_sum_rescale_many(he_ctx* c, const std::vector<std::vector<const uint64_t*>>& in,
+                               const std::vector<int>& lin, int lv, const std::vector<int64_t>& K,
+                               const std::vector<uint64_t*>& out, bool add_k0, int64_t K0) {
+    const int nterm = (int)in.size();
+    if (nterm < 1 || nterm > kRsTerms || (int)lin.size() != nterm || (int)K.size() != nterm)
+        return set_err(c, HE_EINVAL, "mul_const_sum_rescale: %d terms", nterm);
+    RowConst kc[kRsTerms];
+    RsTerm t[kRsTerms];
+    for (int j = 0; j < nterm; j++) {
+        kc[j] = row_const_shoup(c, lv, K[j]);
+        t[j] = RsTerm{&in[j], lin[j], &kc[j]};
+    }
+    return rescale_fused(c, t, nterm, lv, out, {}, add_k0, K0);
 }
 
 // out_i = in_i keeping limbs < lv (out_i != in_i)
@@ -986,22 +1046,22 @@ extern "C" int he_poly_eval_ps15(he_ctx* c, const he_ct* x, int n, const double*
         double pw_scale[4] = {0, sx, s2, s3};
 
         // q_blk(x) at (lam, T) into dst buffers (level lam): each x^j dropped
-        // to lam+1 and multiplied by its integer constant in one pass, then
-        // rescaled; the constant term added last
-        // (the multiply, rescale, sum and constant of each term in the
-        // launches of one rescale: mul_const_rescale_many)
+        // to lam+1 and multiplied by its integer constant, the three summed
+        // and rescaled once, the constant term added last (all in the
+        // launches of one rescale: mul_const_sum_rescale_many)
         auto build_q = [&](int blk, int lam, double T, int dst) -> int {
-            int r;
             const int64_t K0 = (int64_t)round_half_away(coeffs[4 * blk] * T);
+            std::vector<std::vector<const uint64_t*>> src;
+            std::vector<int> lin;
+            std::vector<int64_t> K;
             for (int j = 1; j <= 3; j++) {
                 double cj = coeffs[4 * blk + j];
                 double v = cj * T * (double)c->primes[lam] / pw_scale[j];
-                int64_t K = (int64_t)round_half_away(v);
-                const std::vector<const uint64_t*> src = j == 1 ? xd : cbufs(j == 2 ? X2 : X3);
-                if ((r = mul_const_rescale_many(c, src, pw_level[j], lam + 1, K, bufs(dst), j > 1, j == 3, K0)))
-                    return r;
+                K.push_back((int64_t)round_half_away(v));
+                src.push_back(j == 1 ? xd : cbufs(j == 2 ? X2 : X3));
+                lin.push_back(pw_level[j]);
             }
-            return HE_OK;
+            return mul_const_sum_rescale_many(c, src, lin, lam + 1, K, bufs(dst), true, K0);
         };
         int lev = l0 - 3;
         double T = top_scale;

@@ -419,8 +419,9 @@ int he_attention_output(he_ctx* ctx, const he_ct* a, const he_ct* v, int n_tok, 
  * powers (AEGIS section 2.3: Softmax by polynomial approximation):
  *   x2 = HMRR(x,x); x3 = HMRR(x2, drop(x)); x4 = HMRR(x2,x2);
  *   q_i = sum_{j<4} c_{4i+j} x^j built at (level, T): each x^j is dropped to
- *         level+1, multiplied by K = round_half_away(c*T*q_level/S_j) (fp64,
- *         left to right) and rescaled; the constant adds round_half_away(c*T);
+ *         level+1 and multiplied by K = round_half_away(c*T*q_level/S_j)
+ *         (fp64, left to right); the three products are summed and the sum
+ *         rescaled once; the constant adds round_half_away(c*T);
  *   acc = q_3 at (l0-3, top_scale); acc = HMRR(acc, drop(x4)) + q_i, i = 2, 1, 0,
  *         each q_i at the accumulator's exact level and scale.
  * HMRR = he_hmult_relin_rescale.  x: n ciphertexts at level l0 >= 7;
