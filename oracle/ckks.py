@@ -881,19 +881,27 @@ def attention_scores(q, k, n_tok, d, offsets, keys, rlk, params):
 
 
 def attention_av(a, v, offsets, keys, rlk, params):
-    """O = sum_delta HMRR(a_delta, drop(rot_delta(v))) over the offsets,
-    rot_delta(v) hoisted (one ModUp of v; delta = 0: v) and dropped to
-    a_delta's level.  With a_delta = p(S_delta) replicated over the feature
-    blocks and v token-duplicated, slot f 2n + t of O holds
-    sum_delta p(S_delta[t]) V[f][(t + delta) mod n] for t < n."""
+    """O = rescale(relinearise(sum_delta a_delta (x) drop(rot_delta(v)))) over
+    the offsets: the tensors of the products summed, then one
+    relinearisation and one rescale; rot_delta(v) hoisted (one ModUp of v;
+    delta = 0: v) and dropped to a_delta's level.  With a_delta = p(S_delta)
+    replicated over the feature blocks and v token-duplicated, slot f 2n + t
+    of O holds sum_delta p(S_delta[t]) V[f][(t + delta) mod n] for t < n.
+    Reading: the pages give no order for relinearising and rescaling the
+    products; both maps are linear up to their noise and rounding, so the sum
+    is relinearised and rescaled once (every a_delta at one level and scale)."""
     nz = [o for o in offsets if o % params.n_slots]
     rot = dict(zip(nz, rotate_hoisted(v, nz, keys, params)))
-    out = None
+    level = a[0]["level"]
+    qm = params.q[:level]
+    d = None
     for ad, o in zip(a, offsets):
-        vv = drop_level(rot[o] if o in rot else v, ad["level"])
-        t = hmult_relin_rescale(ad, vv, rlk, params)
-        out = t if out is None else add(out, t, params)
-    return out
+        assert ad["level"] == level and ad["scale"] == a[0]["scale"]
+        vv = drop_level(rot[o] if o in rot else v, level)
+        t = tensor(ad, vv, params)
+        d = t if d is None else tuple(add_rows(d[k], t[k], qm) for k in range(3))
+    c = relinearize(d, level, rlk, params)
+    return rescale(make_ct(c, level, a[0]["scale"] * v["scale"]), params)
 
 
 # --------------------------------------------------------------------------
