@@ -10,7 +10,8 @@
 //            sum_f Q[f][t] K[f][(t + delta) mod n] at t < n (0 at t >= n);
 //   Softmax: the caller shifts S_delta by a known bound and evaluates its
 //            exponential with he_poly_eval_ps15 (no division by row sums);
-//   output:  O = sum_delta HMRR(A_delta, drop(rot_delta(V))).
+//   output:  O = rescale(relinearise(sum_delta A_delta (x) drop(rot_delta(V)))):
+//            the products' tensors summed, one relinearisation, one rescale.
 // The rotations of K and of V by the offsets are hoisted (one ModUp each).
 #include <algorithm>
 
@@ -168,35 +169,21 @@ extern "C" int he_attention_output(he_ctx* c, const he_ct* a, const he_ct* v, in
     std::vector<int> pos;
     if ((rc = split_offsets(c, offsets, n_off, n_tok, nz, pos, what))) return rc;
 
-    const size_t N = c->N, ctv = (size_t)2 * lv * N, cta = (size_t)2 * la * N;
-    uint64_t* pool;
-    if ((rc = scratch_slot(c, 3, ctv * nz.size() + cta * n_off, &pool))) return rc;
-    uint64_t* prod = pool + ctv * nz.size();
+    const size_t N = c->N, ctv = (size_t)2 * lv * N;
+    uint64_t* pool = nullptr;
+    if (!nz.empty() && (rc = scratch_slot(c, 3, ctv * nz.size(), &pool))) return rc;
     // rot_delta(v) for the non-zero offsets, hoisted; the products read them
     // at the weights' level in place
     std::vector<he_ct> rv(nz.size());
     for (size_t j = 0; j < nz.size(); j++) rv[j] = he_ct{pool + j * ctv, lv, v->scale, 1};
     if (!nz.empty() && (rc = rotate_hoisted_many(c, v, 1, nz.data(), (int)nz.size(), rv.data()))) return rc;
+    // the products' tensors summed, then one relinearisation and one rescale
     std::vector<const uint64_t*> A, B;
-    std::vector<uint64_t*> P;
     for (int i = 0; i < n_off; i++) {
         B.push_back(pos[i] < 0 ? v->data : rv[pos[i]].data);
         A.push_back(a[i].data);
-        P.push_back(prod + cta * i);
     }
-    if ((rc = hmrr_many(c, A, B, P, la, la, lv))) return rc;
-    // sum of the products, halving the list each round
-    int m = n_off;
-    while (m > 1) {
-        const int half = m / 2, keep = m - half;
-        std::vector<const uint64_t*> x(P.begin(), P.begin() + half), y(P.begin() + keep, P.begin() + m);
-        std::vector<uint64_t*> o(P.begin(), P.begin() + half);
-        if ((rc = add_many(c, x, y, o, la - 1))) return rc;
-        m = keep;
-    }
-    if ((rc = check_cuda(c, cudaMemcpyAsync(out->data, P[0], (size_t)2 * (la - 1) * N * 8, cudaMemcpyDeviceToDevice,
-                                            c->stream), "attention_output copy")))
-        return rc;
+    if ((rc = hmrr_sum(c, A, B, out->data, la, la, lv))) return rc;
     out->level = la - 1;
     out->scale = a[0].scale * v->scale / (double)c->primes[la - 1];
     out->is_ntt = 1;

@@ -214,6 +214,10 @@ int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::v
 int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector<const uint64_t*>& b,
               const std::vector<uint64_t*>& out, int level, int room_a = 0, int room_b = 0,
               const std::vector<const uint64_t*>& addend = {});
+// out = rescale(relinearise(sum_i tensor(a_i, b_i))) of the pairs at `level`
+// (a_i, b_i as in hmrr_many; out apart from every input).
+int hmrr_sum(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector<const uint64_t*>& b, uint64_t* out,
+             int level, int room_a = 0, int room_b = 0);
 int add_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector<const uint64_t*>& b,
              const std::vector<uint64_t*>& o, int lv);
 int drop_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::vector<uint64_t*>& out, int lin, int lv);

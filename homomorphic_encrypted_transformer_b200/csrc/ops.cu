@@ -404,6 +404,75 @@ __global__ void k_tensor_many(PtrList pa, PtrList pb, MutPtrList pd, int level, 
     *reinterpret_cast<ulonglong2*>(d + (size_t)(2 * level + r) * N + c) = make_ulonglong2(o2[0], o2[1]);
 }
 
+// d (+)= sum_i (a_i0 b_i0, a_i0 b_i1 + a_i1 b_i0, a_i1 b_i1) over the m pairs
+// (a_i, b_i), d = [3][level][N] (accumulate: d holds the sum of earlier
+// pairs, canonical); a_i / b_i as in k_tensor_many.  Two coefficients per
+// thread.  FP64 limbs sum signed rounded-quotient products (each |.| < 5q/8,
+// at most 2 kMaxBatch of them per output: below 2^48) and reduce once; q_0
+// sums Montgomery products and corrects once by R^2 R^-1.
+__global__ void k_tensor_sum(PtrList pa, PtrList pb, int m, uint64_t* __restrict__ d, int accumulate, int level,
+                             int room_a, int room_b, const DevPrime* __restrict__ pr, const FpMod* __restrict__ fpm,
+                             int logn) {
+    const int N = 1 << logn;
+    const int c = 2 * (blockIdx.x * blockDim.x + threadIdx.x), r = blockIdx.y;
+    if (c >= N) return;
+    const DevPrime p = pr[r];
+    const size_t k0 = (size_t)r * N + c, ka = (size_t)(room_a + r) * N + c, kb = (size_t)(room_b + r) * N + c;
+    uint64_t* dp[3] = {d + k0, d + (size_t)(level + r) * N + c, d + (size_t)(2 * level + r) * N + c};
+    uint64_t o[3][2];
+    if (p.q < kFpPrimeLimit) {
+        const FpMod fm = fpm[r];
+        double s[3][2] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
+        for (int i = 0; i < m; i++) {
+            const ulonglong2 A0 = __ldg(reinterpret_cast<const ulonglong2*>(pa.p[i] + k0));
+            const ulonglong2 A1 = __ldg(reinterpret_cast<const ulonglong2*>(pa.p[i] + ka));
+            const ulonglong2 B0 = __ldg(reinterpret_cast<const ulonglong2*>(pb.p[i] + k0));
+            const ulonglong2 B1 = __ldg(reinterpret_cast<const ulonglong2*>(pb.p[i] + kb));
+            const double x0[2] = {u2d(A0.x), u2d(A0.y)}, x1[2] = {u2d(A1.x), u2d(A1.y)};
+            const double y0[2] = {u2d(B0.x), u2d(B0.y)}, y1[2] = {u2d(B1.x), u2d(B1.y)};
+#pragma unroll
+            for (int e = 0; e < 2; e++) {
+                s[0][e] = __dadd_rn(s[0][e], fp_mulmod_s(x0[e], y0[e], fm));
+                s[1][e] = __dadd_rn(s[1][e], __dadd_rn(fp_mulmod_s(x0[e], y1[e], fm), fp_mulmod_s(x1[e], y0[e], fm)));
+                s[2][e] = __dadd_rn(s[2][e], fp_mulmod_s(x1[e], y1[e], fm));
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < 3; h++) {
+            if (accumulate) {
+                const ulonglong2 prev = *reinterpret_cast<const ulonglong2*>(dp[h]);
+                s[h][0] = __dadd_rn(s[h][0], u2d(prev.x));
+                s[h][1] = __dadd_rn(s[h][1], u2d(prev.y));
+            }
+            o[h][0] = d2u(fp_canon(s[h][0], fm));
+            o[h][1] = d2u(fp_canon(s[h][1], fm));
+        }
+    } else {
+        uint64_t s[3][2] = {{0, 0}, {0, 0}, {0, 0}};
+        for (int i = 0; i < m; i++) {
+            const ulonglong2 A0 = __ldg(reinterpret_cast<const ulonglong2*>(pa.p[i] + k0));
+            const ulonglong2 A1 = __ldg(reinterpret_cast<const ulonglong2*>(pa.p[i] + ka));
+            const ulonglong2 B0 = __ldg(reinterpret_cast<const ulonglong2*>(pb.p[i] + k0));
+            const ulonglong2 B1 = __ldg(reinterpret_cast<const ulonglong2*>(pb.p[i] + kb));
+            const uint64_t a0[2] = {A0.x, A0.y}, a1[2] = {A1.x, A1.y}, b0[2] = {B0.x, B0.y}, b1[2] = {B1.x, B1.y};
+#pragma unroll
+            for (int e = 0; e < 2; e++) {
+                s[0][e] = add_mod(s[0][e], mont_mul(a0[e], b0[e], p), p.q);
+                s[1][e] = add_mod(s[1][e], add_mod(mont_mul(a0[e], b1[e], p), mont_mul(a1[e], b0[e], p), p.q), p.q);
+                s[2][e] = add_mod(s[2][e], mont_mul(a1[e], b1[e], p), p.q);
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < 3; h++) {
+            const ulonglong2 prev = accumulate ? *reinterpret_cast<const ulonglong2*>(dp[h]) : make_ulonglong2(0, 0);
+            o[h][0] = add_mod(prev.x, mont_mul(s[h][0], p.r2, p), p.q);
+            o[h][1] = add_mod(prev.y, mont_mul(s[h][1], p.r2, p), p.q);
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < 3; h++) *reinterpret_cast<ulonglong2*>(dp[h]) = make_ulonglong2(o[h][0], o[h][1]);
+}
+
 // --------------------------------------------------------------- host side
 
 static uint64_t h_shoup(uint64_t w, uint64_t q) { return (uint64_t)(((unsigned __int128)w << 64) / q); }
@@ -582,6 +651,49 @@ int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vecto
         if ((rc = rescale_many(c, rin, rout, level, radd))) return rc;
     }
     return HE_OK;
+}
+
+// out = rescale(relinearise(sum_i tensor(a_i, b_i))) of n pairs at one level
+// (inputs as in hmrr_many; out apart from every input): the tensors summed
+// in kMaxBatch-pair launches, then one key switch and one rescale.
+int hmrr_sum(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector<const uint64_t*>& b, uint64_t* out,
+             int level, int room_a, int room_b) {
+    const int N = c->N, n = (int)a.size();
+    if (n < 1 || (int)b.size() != n) return set_err(c, HE_EINVAL, "hmult sum: %d pairs", n);
+    if (!c->relin.d) return set_err(c, HE_ENOKEY, "hmult: no relinearisation key");
+    if (level < 2) return set_err(c, HE_ELEVEL, "hmult: level %d cannot be rescaled", level);
+    if (room_a == 0) room_a = level;
+    if (room_b == 0) room_b = level;
+    if (room_a < level || room_b < level) return set_err(c, HE_ELEVEL, "hmult: input room below level %d", level);
+    uint64_t* d;
+    int rc = scratch_slot(c, 2, (size_t)5 * level * N, &d);  // d0 d1 d2 | relinearised [2][level]
+    if (rc) return rc;
+    int fp_l = 0;
+    for (int r = 0; r < level; r++) fp_l += fp_prime(c, r);
+    const int gx2 = (N / 2 + TB - 1) / TB;
+    for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
+        const int m = std::min(kMaxBatch, n - i0);
+        PtrList pa, pb;
+        for (int i = 0; i < m; i++) {
+            pa.p[i] = a[i0 + i];
+            pb.p[i] = b[i0 + i];
+        }
+        prof_begin(c, HE_PROF_ELEMENTWISE);
+        k_tensor_sum<<<dim3(gx2, level), TB, 0, c->stream>>>(pa, pb, m, d, i0 > 0 ? 1 : 0, level, room_a, room_b,
+                                                             c->d_prime, c->d_fpmod, c->log_n);
+        if ((rc = lc(c, "tensor_sum"))) return rc;
+        prof_end(c, HE_PROF_ELEMENTWISE, (4.0 * m + (i0 > 0 ? 6.0 : 3.0)) * level * 8.0 * N,
+                 4.0 * level * m * N + 3.0 * (level - fp_l) * N, 4.0 * fp_l * m * N);
+    }
+    KsIoList io;
+    io.galois.push_back(0);
+    io.key.push_back(c->relin.d);
+    io.d.push_back(d + (size_t)2 * level * N);
+    io.out.push_back(d + (size_t)3 * level * N);
+    io.add0.push_back(d);
+    io.add1.push_back(d + (size_t)level * N);
+    if ((rc = key_switch_split(c, level, io))) return rc;
+    return rescale_many(c, {d + (size_t)3 * level * N}, {out}, level);
 }
 
 // ---- batched helpers: n ciphertexts, kMaxBatch per launch

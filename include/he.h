@@ -398,14 +398,17 @@ int he_pmult_accum_bsgs(he_ctx* ctx, const he_ct* x, int n_in, const uint64_t* d
  *   relinearisation key.
  * Softmax between the two calls is the caller's: shift each s[i] by a known
  * bound (he_add_const) and evaluate the exponential by he_poly_eval_ps15.
- * he_attention_output: out = sum_i HMRR(a[i], drop(rot_{offsets[i]}(v))),
- *   a[i] the n_off weights at one level la >= 2 and scale, v at level
- *   >= la; the rotations of v are hoisted.  Slot f*2n + t of out holds
+ * he_attention_output: out = rescale(relinearise(sum_i a[i] (x)
+ *   drop(rot_{offsets[i]}(v)))): the products' tensors summed, then one
+ *   relinearisation and one rescale; a[i] the n_off weights at one level
+ *   la >= 2 and scale, v at level >= la; the rotations of v are hoisted
+ *   (he_rotate_hoisted).  Slot f*2n + t of out holds
  *   sum_i A_i[t] V[f][(t + offsets[i]) mod n] for t < n.  out at la-1,
  *   scale a.scale*v.scale/q_{la-1}.
  * Outputs: s[i] each [2][l-1][N] words, out [2][la-1][N]; an output may not
  * overlap another output or any input.
- * Scratch (context-owned): the rotated copies and one ciphertext per offset.
+ * Scratch (context-owned): the rotated copies, one ciphertext per offset
+ * (scores), and the summed tensor (output).
  * Errors: HE_EINVAL (shape, offsets, null, unaligned, overlapping
  * buffers), HE_ELEVEL, HE_EDOMAIN, HE_ENOKEY; nothing is launched then.
  */
