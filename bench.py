@@ -430,6 +430,13 @@ def run_ps15_small_case(args, local_rank):
 
 # ------------------------------------------------------------------ other workloads
 
+def attention_sum_steps(n_tok, d):
+    """Rotation steps the feature sum of he_attention_scores needs (include/he.h):
+    2 n b for 0 < b < d1 and 2 n d1 a for 0 < a < d / d1, d1 = 2^ceil(log2(d) / 2)."""
+    d1 = 1 << (((d.bit_length() - 1) + 1) // 2)
+    return [2 * n_tok * b for b in range(1, d1)] + [2 * n_tok * d1 * a for a in range(1, d // d1)]
+
+
 FFN = {"n_feat": 256, "n_tok": 128, "bs": 16, "gs": 16, "n_in": 3, "n_out": 12, "level": 12}
 # one attention head: d features x n_tok tokens with d 2 n_tok = N/2 at N = 2^16;
 # scores shifted by `shift` before the exponential
@@ -484,7 +491,7 @@ def workload_cpu_baseline(case, seconds):
     s = S.secret(master, P.N)
     if case == "attention":
         d, n_tok = ATT["d"], ATT["n_tok"]
-        steps = [1] + [2 * n_tok * (1 << i) for i in range(d.bit_length() - 1)]
+        steps = [1] + sorted({x for st in C.attention_sum_steps(n_tok, d) for x in st if x})
         keys = {}
         for st in steps:
             a, e = S.key_draws(master, P.galois_elt(st), P.mods, P.N, P.dnum)
@@ -684,7 +691,7 @@ def workload_case(case, n_steps, n_warmup, cpu_seconds, local_rank, probes=None,
     elif case == "attention":
         d, n_tok = ATT["d"], ATT["n_tok"]
         offsets = list(range(n_tok))
-        for st in sorted(set(offsets[1:]) | {2 * n_tok * h for h in (1 << i for i in range(d.bit_length() - 1))}):
+        for st in sorted(set(offsets[1:]) | set(attention_sum_steps(n_tok, d))):
             upload(he.HE_KEY_ROTATION, st)
         upload(he.HE_KEY_RELIN, 0)
         qkv = device_residues(torch, (3, 2), ctx.primes[:L], N, gen, dev)

@@ -860,22 +860,39 @@ def attention_pack(X, dup):
     return out.reshape(-1)
 
 
+def attention_sum_steps(n_tok, d):
+    """Steps of the feature sum sum_{h<d} rot_{2n h}(P), taken as two hoisted
+    rotate-and-sums: d = d1 d2 with d1 = 2^ceil(log2(d) / 2), first over
+    2n b (b < d1), then over 2n d1 a (a < d2); step 0 is the term itself."""
+    lg = d.bit_length() - 1
+    d1 = 1 << ((lg + 1) // 2)
+    d2 = d // d1
+    return [2 * n_tok * b for b in range(d1)], [2 * n_tok * d1 * a for a in range(d2)]
+
+
 def attention_scores(q, k, n_tok, d, offsets, keys, rlk, params):
     """S_delta for each token offset delta (0 <= delta < n):
         P = HMRR(q, rot_delta(k)),  rot_delta(k) hoisted (one ModUp of k; delta = 0: k),
-        S <- S + rot_{2n 2^i}(S) for i < log2(d), starting from S = P.
+        S = sum_{h<d} rot_{2n h}(P) as two hoisted rotate-and-sums,
+            T = sum_{b<d1} rot_{2n b}(P),  S = sum_{a<d2} rot_{2n d1 a}(T)
+        (attention_sum_steps; each: the term itself plus rotate_sum_hoisted
+        over the non-zero steps).
     q packs Q with zeros on t >= n, k packs K token-duplicated; then every
     feature block of S_delta holds sum_f Q[f][t] K[f][(t + delta) mod n] at
-    t < n and 0 at t >= n (the sum wraps around the d 2n = N/2 slots)."""
+    t < n and 0 at t >= n (the sum wraps around the d 2n = N/2 slots).
+    Reading: the pages give no schedule for the feature sum; two hoisted
+    sums take two ModUps and two ModDowns per offset where log2(d) doubling
+    rotations take log2(d) of each, and give the same slots."""
     assert d * 2 * n_tok == params.n_slots and d & (d - 1) == 0
     nz = [o for o in offsets if o % params.n_slots]
     rot = dict(zip(nz, rotate_hoisted(k, nz, keys, params)))
     out = []
     for o in offsets:
         acc = hmult_relin_rescale(q, rot[o] if o in rot else k, rlk, params)
-        for i in range(d.bit_length() - 1):
-            st = 2 * n_tok * (1 << i)
-            acc = add(acc, rotate(acc, st, keys[st], params), params)
+        for st in attention_sum_steps(n_tok, d):
+            nzs = [x for x in st if x]
+            if nzs:
+                acc = add(acc, rotate_sum_hoisted(acc, nzs, keys, params), params)
         out.append(acc)
     return out
 

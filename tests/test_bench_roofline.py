@@ -57,3 +57,14 @@ def test_stored_traffic_ratios_are_current():
     for name, e in bench.NCU_TRAFFIC.items():
         assert bench.traffic_ratio(name) is not None, name
         assert 0.8 < e["ratio"] < 1.3, name
+
+
+def test_attention_sum_steps_agree_with_the_oracle():
+    """The rotation keys the attention benchmark uploads for the feature sum
+    are the oracle's schedule's non-zero steps."""
+    import bench
+    from oracle import ckks as C
+
+    for n_tok, d in [(256, 64), (32, 16), (8, 2), (4, 128), (16, 1)]:
+        want = sorted({x for st in C.attention_sum_steps(n_tok, d) for x in st if x})
+        assert sorted(bench.attention_sum_steps(n_tok, d)) == want

@@ -27,7 +27,7 @@ def test_attention_head_small():
     k = st.encrypt(C.attention_pack(K, True), P.L, ct_id=1)
     v = st.encrypt(C.attention_pack(V, True), P.L, ct_id=2)
     offsets = [0, 1, 5, 31]
-    steps = sorted({o for o in offsets if o} | {2 * NT * h for h in (1, 2, 4, 8)})
+    steps = sorted({o for o in offsets if o} | {x for st_ in C.attention_sum_steps(NT, D) for x in st_ if x})
     for s_ in steps:
         st.upload_rot(s_)
     st.upload_relin()
@@ -142,7 +142,7 @@ def test_attention_head_full_size_sampled():
     k = st.encrypt(C.attention_pack(K, True), P.L, ct_id=1)
     v = st.encrypt(C.attention_pack(V, True), P.L, ct_id=2)
     offsets = list(range(n_tok))
-    sum_steps = [2 * n_tok * (1 << i) for i in range(d.bit_length() - 1)]
+    sum_steps = sorted({x for st_ in C.attention_sum_steps(n_tok, d) for x in st_ if x})
     for s_ in sorted(set(offsets[1:]) | set(sum_steps)):
         st.upload_rot(s_)
     st.upload_relin()

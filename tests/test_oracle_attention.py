@@ -31,7 +31,7 @@ def _head(seed):
     k = enc(C.attention_pack(K, True), 1)
     v = enc(C.attention_pack(V, True), 2)
     offsets = list(range(NT))
-    steps = sorted({o for o in offsets if o} | {2 * NT * (1 << i) for i in range(4)})
+    steps = sorted({o for o in offsets if o} | {x for st in C.attention_sum_steps(NT, D) for x in st if x})
     keys = {}
     for st in steps:
         a, e = S.key_draws(seed, P.galois_elt(st), P.mods, P.N, P.dnum)
