@@ -5,8 +5,8 @@
 // 2n.  Q sits at slot f 2n + t for t < n (zeros at t >= n); K and V are
 // token-duplicated (slot f 2n + t holds X[f][t mod n] for every t < 2n), so
 // that a slot rotation by delta < n shifts every feature's tokens cyclically.
-//   scores:  S_delta = HMRR(Q, rot_delta(K)), then S <- S + rot_{2n 2^i}(S),
-//            i < log2 d: every feature block holds
+//   scores:  P = HMRR(Q, rot_delta(K)), then S_delta = sum_{h<d} rot_{2n h}(P)
+//            as two hoisted rotate-and-sums (d = d1 d2): every feature block holds
 //            sum_f Q[f][t] K[f][(t + delta) mod n] at t < n (0 at t >= n);
 //   Softmax: the caller shifts S_delta by a known bound and evaluates its
 //            exponential with he_poly_eval_ps15 (no division by row sums);
@@ -91,8 +91,17 @@ extern "C" int he_attention_scores(he_ctx* c, const he_ct* q, const he_ct* k, in
     std::vector<int32_t> nz;
     std::vector<int> pos;
     if ((rc = split_offsets(c, offsets, n_off, n_tok, nz, pos, what))) return rc;
-    for (int h = 1; h < d; h <<= 1)
-        if ((rc = need_key(c, 2 * n_tok * h, what))) return rc;
+    // feature-sum steps: 2n b (b < d1), then 2n d1 a (a < d2), d = d1 d2
+    int lg = 0;
+    while ((1 << lg) < d) lg++;
+    const int d1 = 1 << ((lg + 1) / 2), d2 = d / d1;
+    std::vector<int32_t> inner, outer;
+    for (int b = 0; b < d1; b++) inner.push_back(2 * n_tok * b);
+    for (int a2 = 0; a2 < d2; a2++) outer.push_back(2 * n_tok * d1 * a2);
+    for (int32_t st : inner)
+        if (st && (rc = need_key(c, st, what))) return rc;
+    for (int32_t st : outer)
+        if (st && (rc = need_key(c, st, what))) return rc;
     const size_t N = c->N, ctw = (size_t)2 * l * N, ctw1 = (size_t)2 * (l - 1) * N;
     for (int i = 0; i < n_off; i++)
         if (!s[i].data || ((uintptr_t)s[i].data & 31)) return set_err(c, HE_EINVAL, "%s: null or unaligned output", what);
@@ -113,21 +122,23 @@ extern "C" int he_attention_scores(he_ctx* c, const he_ct* q, const he_ct* k, in
         Tm.push_back(pool + ctw * nz.size() + ctw1 * i);
     }
     if ((rc = hmrr_many(c, A, B, So, l))) return rc;
-    // the feature sum: S <- S + rot_{2n h}(S), h = 1, 2, .., d/2
+    // the feature sum S = sum_{h<d} rot_{2n h}(P) as two hoisted
+    // rotate-and-sums (one ModUp and one ModDown each; step 0 adds the term
+    // itself): T = sum_b rot_{2n b}(P), S = sum_a rot_{2n d1 a}(T); the
+    // rounds alternate between the outputs and the scratch
     const double scale = q->scale * k->scale / (double)c->primes[l - 1];
     std::vector<he_ct> sc(n_off), tc(n_off);
     for (int i = 0; i < n_off; i++) {
         sc[i] = he_ct{s[i].data, l - 1, scale, 1};
         tc[i] = he_ct{Tm[i], l - 1, scale, 1};
     }
-    // each round: dst = rot(src) + src, the sum taken in the rotation's
-    // ModDown; src and dst alternate between the outputs and the scratch
     int rounds = 0;
-    for (int h = 1; h < d; h <<= 1, rounds++) {
-        std::vector<int32_t> st(n_off, 2 * n_tok * h);
+    for (const std::vector<int32_t>* st : {&inner, &outer}) {
+        if (st->size() < 2) continue;
         const std::vector<he_ct>& src = rounds % 2 ? tc : sc;
         std::vector<he_ct>& dst = rounds % 2 ? sc : tc;
-        if ((rc = rotate_many(c, src.data(), st.data(), dst.data(), n_off, src.data()))) return rc;
+        if ((rc = rotate_sum_hoisted_many(c, src.data(), n_off, st->data(), (int)st->size(), dst.data()))) return rc;
+        rounds++;
     }
     if (rounds % 2)  // an odd number of rounds ends in the scratch
         for (int i = 0; i < n_off; i++)

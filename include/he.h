@@ -389,13 +389,15 @@ int he_pmult_accum_bsgs(he_ctx* ctx, const he_ct* x, int n_in, const uint64_t* d
  * t < n (zeros at t >= n); k and v are token-duplicated (slot f*2n + t holds
  * X[f][t mod n] for every t < 2n).
  * he_attention_scores: for each offset delta = offsets[i] in [0, n_tok),
- *   s[i] = HMRR(q, rot_delta(k)), then s[i] += rot_{2n*h}(s[i]) for
- *   h = 1, 2, .., d/2, so that every feature block of s[i] holds
+ *   P = HMRR(q, rot_delta(k)), then s[i] = sum_{h<d} rot_{2n*h}(P) as two
+ *   hoisted rotate-and-sums (he_rotate_sum_hoisted, step 0 adding the term
+ *   itself): T = sum_{b<d1} rot_{2n*b}(P), s[i] = sum_{a<d2} rot_{2n*d1*a}(T),
+ *   d1 = 2^ceil(log2(d)/2), d2 = d/d1; every feature block of s[i] then holds
  *   sum_f Q[f][t] K[f][(t + delta) mod n] at t < n (0 at t >= n).
  *   The rotations of k are hoisted (he_rotate_hoisted).  q and k at one
  *   level l >= 2; s[i] come back at level l-1, scale q.scale*k.scale/q_{l-1}.
- *   Needs rotation keys for the non-zero offsets and for 2n*h, and the
- *   relinearisation key.
+ *   Needs rotation keys for the non-zero offsets, for 2n*b (0 < b < d1) and
+ *   for 2n*d1*a (0 < a < d2), and the relinearisation key.
  * Softmax between the two calls is the caller's: shift each s[i] by a known
  * bound (he_add_const) and evaluate the exponential by he_poly_eval_ps15.
  * he_attention_output: out = rescale(relinearise(sum_i a[i] (x)

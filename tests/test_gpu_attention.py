@@ -99,8 +99,8 @@ def test_attention_errors():
     assert ei.value.code == he.HE_EINVAL
     # outputs that share storage only in part: views into one buffer (keys of
     # the feature sum present, so that only the overlap is wrong)
-    for h in (1, 2, 4, 8):
-        st.upload_rot(2 * 32 * h)
+    for s_ in sorted({x for st_ in C.attention_sum_steps(32, 16) for x in st_ if x}):
+        st.upload_rot(s_)
     big = st.empty_gpu(2 * P.L)
     half = (P.L - 1) * P.N  # less than one output's [2][L-1][N] words
     s0 = he.Ciphertext(big.data[:2 * P.L * P.N], P.L, 1.0)
