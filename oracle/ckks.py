@@ -952,9 +952,14 @@ def ps_eval_deg15(x, coeffs, rlk, params, top_scale=PS_TOP_SCALE):
         scale is T.  (One rounding per block instead of one per term: the
         pages fix no order, and rescaling is linear up to that rounding.)
       Horner: acc = q_3 at (l0-3, top_scale);
-        acc = HMRR(acc, drop(x4)) + q_2;  acc = HMRR(acc, drop(x4)) + q_1;
-        acc = HMRR(acc, drop(x4)) + q_0, each q_i built at the accumulator's
-        exact level and fp64 scale.  Result level l0-6.
+        acc = HMRR(acc, drop(x4)) + q_i for i = 2, 1, 0, with q_i's products
+        added before the product's rescale: at the product's level l (its
+        scale T q_lambda, lambda = l-1, T = acc.scale x4.scale / q_lambda),
+        acc = rescale(relin(acc (x) drop(x4)) + sum_{j>=1} K_j drop(x^j, l))
+              + round_half_away(c_{4i} T),
+        K_j as above at (lambda, T); one rescale per Horner step.  (Both
+        rescales divide by the same q_lambda and the terms share the nominal
+        scale T q_lambda, so one rounding replaces two.)  Result level l0-6.
     Reading: top_scale = 2^62.  The innermost block q_3 is later multiplied
     by x4^3 = x^12, up to 4^12 ~ 1.7e7 on [-4, 0].  Its absolute error is the
     rescale rounding noise (~7e4 in message units at N = 2^16) divided by its
@@ -984,9 +989,20 @@ def ps_eval_deg15(x, coeffs, rlk, params, top_scale=PS_TOP_SCALE):
 
     acc = build_q(3, l0 - 3, top_scale)
     for i in (2, 1, 0):
-        acc = hm(acc, drop_level(x4, acc["level"]))
-        qi = build_q(i, acc["level"], acc["scale"])
-        acc = make_ct(add(acc, qi, params)["c"], acc["level"], acc["scale"])
+        lev = acc["level"]
+        lam = lev - 1
+        prod_scale = acc["scale"] * x4["scale"]
+        T = prod_scale / params.q[lam]
+        qm = params.q[:lev]
+        c = relinearize(tensor(acc, drop_level(x4, lev), params), lev, rlk, params)
+        for j in (1, 2, 3):
+            xj = drop_level(pw[j], lev)
+            K = ps_const(float(coeffs[4 * i + j]), T, params.q[lam], xj["scale"])
+            t = mul_const(xj, K, params)
+            c = np.stack([add_rows(c[k], t["c"][k], qm) for k in range(2)])
+        acc = rescale(make_ct(c, lev, prod_scale), params)
+        acc = add_const(acc, int(round_half_away(np.float64(float(coeffs[4 * i]) * T))), params)
+        acc = make_ct(acc["c"], lam, T)
     return acc
 
 
