@@ -211,9 +211,20 @@ int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::v
 // b_i of the same i; plus addend_i at level - 1 when addend is not empty); out_i = a_i +
 // b_i at lv limbs (out may equal a); out_i = in_i keeping limbs < lv (out !=
 // in).
+// Terms added to the relinearised products before their rescale (at most
+// three): term j of product i is in[j][i], at level lin[j] >= the product's
+// level and read at that level, times the integer K[j]; with add_k0, K0 is
+// added to c0 after the rescale.
+struct PreRescaleTerms {
+    std::vector<std::vector<const uint64_t*>> in;
+    std::vector<int> lin;
+    std::vector<int64_t> K;
+    bool add_k0 = false;
+    int64_t K0 = 0;
+};
 int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector<const uint64_t*>& b,
               const std::vector<uint64_t*>& out, int level, int room_a = 0, int room_b = 0,
-              const std::vector<const uint64_t*>& addend = {});
+              const std::vector<const uint64_t*>& addend = {}, const PreRescaleTerms* pre = nullptr);
 // out = rescale(relinearise(sum_i tensor(a_i, b_i))) of the pairs at `level`
 // (a_i, b_i as in hmrr_many; out apart from every input).
 int hmrr_sum(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector<const uint64_t*>& b, uint64_t* out,

@@ -135,7 +135,7 @@ __global__ void k_key_canonical_seeded(const uint64_t* __restrict__ in, uint64_t
 // crosses HBM and the rescale takes two transform launches where the
 // unfused form took a lift, two passes and a combine.  Residue for residue
 // the same values.
-constexpr int kRsTerms = 3;
+constexpr int kRsTerms = 4;
 
 struct RescaleIo {
     PtrList in[kRsTerms];  // term j: x_{j,i} at level lin[j]
@@ -599,11 +599,20 @@ int rescale_many(he_ctx* c, const std::vector<const uint64_t*>& in, const std::v
     return rescale_fused(c, &t, 1, level, out, addend, false, 0);
 }
 
+static RowConst row_const_shoup(const he_ctx* c, int level, int64_t K);
+
 // HMult + relinearisation + rescale of n pairs at one level.
 int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vector<const uint64_t*>& b,
               const std::vector<uint64_t*>& out, int level, int room_a, int room_b,
-              const std::vector<const uint64_t*>& addend) {
+              const std::vector<const uint64_t*>& addend, const PreRescaleTerms* pre) {
     const int N = c->N, n = (int)a.size();
+    const int n_pre = pre ? (int)pre->in.size() : 0;
+    if (n_pre > kRsTerms - 1 || (pre && ((int)pre->lin.size() != n_pre || (int)pre->K.size() != n_pre)))
+        return set_err(c, HE_EINVAL, "hmult: %d terms before the rescale", n_pre);
+    for (int j = 0; j < n_pre; j++)
+        if ((int)pre->in[j].size() != n || pre->lin[j] < level)
+            return set_err(c, HE_EINVAL, "hmult: term %d before the rescale", j);
+    if (pre && !addend.empty()) return set_err(c, HE_EINVAL, "hmult: an addend and terms before the rescale");
     if (!c->relin.d) return set_err(c, HE_ENOKEY, "hmult: no relinearisation key");
     if (level < 2) return set_err(c, HE_ELEVEL, "hmult: level %d cannot be rescaled", level);
     if (room_a == 0) room_a = level;
@@ -646,6 +655,22 @@ int hmrr_many(he_ctx* c, const std::vector<const uint64_t*>& a, const std::vecto
         if ((rc = key_switch_split(c, level, io))) return rc;
         std::vector<const uint64_t*> rin(io.out.begin(), io.out.end());
         std::vector<uint64_t*> rout(out.begin() + i0, out.begin() + i0 + m);
+        if (pre) {
+            // rescale(relinearised + sum_j K_j term_j) in one fused rescale,
+            // the product taken with the constant 1
+            std::vector<std::vector<const uint64_t*>> tin(n_pre);
+            RowConst kc[kRsTerms];
+            RsTerm t[kRsTerms];
+            kc[0] = row_const_shoup(c, level, 1);
+            t[0] = RsTerm{&rin, level, &kc[0]};
+            for (int j = 0; j < n_pre; j++) {
+                tin[j].assign(pre->in[j].begin() + i0, pre->in[j].begin() + i0 + m);
+                kc[1 + j] = row_const_shoup(c, level, pre->K[j]);
+                t[1 + j] = RsTerm{&tin[j], pre->lin[j], &kc[1 + j]};
+            }
+            if ((rc = rescale_fused(c, t, 1 + n_pre, level, rout, {}, pre->add_k0, pre->K0))) return rc;
+            continue;
+        }
         std::vector<const uint64_t*> radd;
         if (!addend.empty()) radd.assign(addend.begin() + i0, addend.begin() + i0 + m);
         if ((rc = rescale_many(c, rin, rout, level, radd))) return rc;
@@ -1124,8 +1149,8 @@ extern "C" int he_poly_eval_ps15(he_ctx* c, const he_ct* x, int n, const double*
     if (l0 < 7) return set_err(c, HE_ELEVEL, "ps15: needs level >= 7, got %d", l0);
     if (!c->relin.d) return set_err(c, HE_ENOKEY, "ps15: no relinearisation key");
     const size_t ctw = (size_t)2 * l0 * N;  // room of one ciphertext at the top level
-    // per ciphertext: x2 x3 x4 acc qsum
-    const int nbuf = 5;
+    // per ciphertext: x2 x3 x4 acc
+    const int nbuf = 4;
     uint64_t* pool = nullptr;
     int rc = scratch_slot(c, 3, ctw * nbuf * n, &pool);
     if (rc) return rc;
@@ -1140,7 +1165,7 @@ extern "C" int he_poly_eval_ps15(he_ctx* c, const he_ct* x, int n, const double*
         for (int i = 0; i < n; i++) v[i] = buf(k, i);
         return v;
     };
-    enum { X2, X3, X4, ACC, QSUM };
+    enum { X2, X3, X4, ACC };
     std::vector<const uint64_t*> xd(n);
     for (int i = 0; i < n; i++) xd[i] = x[i].data;
     double sx = x[0].scale;
@@ -1157,39 +1182,40 @@ extern "C" int he_poly_eval_ps15(he_ctx* c, const he_ct* x, int n, const double*
         int pw_level[4] = {0, l0, l0 - 1, l0 - 2};
         double pw_scale[4] = {0, sx, s2, s3};
 
-        // q_blk(x) at (lam, T) into dst buffers (level lam): each x^j dropped
-        // to lam+1 and multiplied by its integer constant, the three summed
-        // and rescaled once, the constant term added last (all in the
-        // launches of one rescale: mul_const_sum_rescale_many)
-        auto build_q = [&](int blk, int lam, double T, int dst) -> int {
-            const int64_t K0 = (int64_t)round_half_away(coeffs[4 * blk] * T);
-            std::vector<std::vector<const uint64_t*>> src;
-            std::vector<int> lin;
-            std::vector<int64_t> K;
+        // the terms of q_blk(x) at (lam, T): each x^j read at lam+1 limbs and
+        // multiplied by its integer constant; the constant term K0
+        auto q_terms = [&](int blk, int lam, double T) {
+            PreRescaleTerms p;
             for (int j = 1; j <= 3; j++) {
                 double cj = coeffs[4 * blk + j];
                 double v = cj * T * (double)c->primes[lam] / pw_scale[j];
-                K.push_back((int64_t)round_half_away(v));
-                src.push_back(j == 1 ? xd : cbufs(j == 2 ? X2 : X3));
-                lin.push_back(pw_level[j]);
+                p.K.push_back((int64_t)round_half_away(v));
+                p.in.push_back(j == 1 ? xd : cbufs(j == 2 ? X2 : X3));
+                p.lin.push_back(pw_level[j]);
             }
-            return mul_const_sum_rescale_many(c, src, lin, lam + 1, K, bufs(dst), true, K0);
+            p.add_k0 = true;
+            p.K0 = (int64_t)round_half_away(coeffs[4 * blk] * T);
+            return p;
         };
         int lev = l0 - 3;
         double T = top_scale;
-        if ((rc = build_q(3, lev, T, ACC))) goto done;
+        {
+            // acc = q_3: the three terms summed and rescaled once, the
+            // constant added (all in the launches of one rescale)
+            const PreRescaleTerms p = q_terms(3, lev, T);
+            if ((rc = mul_const_sum_rescale_many(c, p.in, p.lin, lev + 1, p.K, bufs(ACC), true, p.K0))) goto done;
+        }
         std::vector<uint64_t*> od(n);
         for (int i = 0; i < n; i++) od[i] = out[i].data;
-        // acc <- HMRR(acc, drop(x4)) + q_blk: q_blk built first, x4 read at
-        // the accumulator's level in place, the sum taken in the rescale of
-        // the product, the last one written to the outputs
+        // acc <- rescale(relin(acc (x) drop(x4)) + terms of q_blk) + K0: x4
+        // read at the accumulator's level in place, the block's terms added
+        // in the product's rescale, the last one written to the outputs
         for (int blk = 2; blk >= 0; blk--) {
             const int lev_in = lev;
             T = (T * s4) / (double)c->primes[lev - 1];
             lev -= 1;
-            if ((rc = build_q(blk, lev, T, QSUM))) goto done;
-            if ((rc = hmrr_many(c, cbufs(ACC), cbufs(X4), blk == 0 ? od : bufs(ACC), lev_in, lev_in, l0 - 2,
-                                cbufs(QSUM))))
+            const PreRescaleTerms p = q_terms(blk, lev, T);
+            if ((rc = hmrr_many(c, cbufs(ACC), cbufs(X4), blk == 0 ? od : bufs(ACC), lev_in, lev_in, l0 - 2, {}, &p)))
                 goto done;
         }
         for (int i = 0; i < n; i++) {

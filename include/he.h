@@ -427,8 +427,11 @@ int he_attention_output(he_ctx* ctx, const he_ct* a, const he_ct* v, int n_tok, 
  *         level+1 and multiplied by K = round_half_away(c*T*q_level/S_j)
  *         (fp64, left to right); the three products are summed and the sum
  *         rescaled once; the constant adds round_half_away(c*T);
- *   acc = q_3 at (l0-3, top_scale); acc = HMRR(acc, drop(x4)) + q_i, i = 2, 1, 0,
- *         each q_i at the accumulator's exact level and scale.
+ *   acc = q_3 at (l0-3, top_scale); then for i = 2, 1, 0, at the product's
+ *         level l (lambda = l-1, T = acc.scale*x4.scale/q_lambda):
+ *         acc = rescale(relin(acc (x) drop(x4)) + sum_{j>=1} K_j drop(x^j))
+ *               + round_half_away(c_{4i}*T), K_j as above at (lambda, T):
+ *         q_i's products join the product before its rescale.
  * HMRR = he_hmult_relin_rescale.  x: n ciphertexts at level l0 >= 7;
  * out: n ciphertexts with room for level l0; they come back at level l0-6.
  */
