@@ -158,9 +158,6 @@ struct KsIoList {
     std::vector<uint64_t*> out;
     std::vector<const uint64_t*> add0;
     std::vector<const uint64_t*> add1;
-    // Optional plain addends of c0 (empty, or one per output; entries may be
-    // null): out_0 gains plus0 after add0, read without any automorphism.
-    std::vector<const uint64_t*> plus0;
     // Hoisted mode (non-empty hoist_d): ModUp runs once on each hoist_d[m]
     // (evaluation rows, no automorphism) and output i takes the raised digits
     // of hoist_d[hoist_src[i]] through sigma_{galois[i]}; d[i] must then be
@@ -179,8 +176,8 @@ int key_switch(he_ctx* c, int level, const KsIoList& io);
 int key_switch_split(he_ctx* c, int level, const KsIoList& io);
 int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io);
 size_t key_switch_scratch_words(const he_ctx* c, int n_raised, int n, int level);
-// out_i = rot_{steps_i}(in_i), plus plus_i (same level) when plus is given
-int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, int n, const he_ct* plus = nullptr);
+// out_i = rot_{steps_i}(in_i)
+int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, int n);
 int rotate_hoisted_many(he_ctx* c, const he_ct* in, int n_in, const int32_t* steps, int n_steps, he_ct* out);
 int rotate_sum_many(he_ctx* c, const he_ct* z, int n_out, int n_terms, const int32_t* steps, const he_ct* base,
                     he_ct* out);

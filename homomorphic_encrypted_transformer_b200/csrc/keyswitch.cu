@@ -813,11 +813,10 @@ __global__ void __launch_bounds__(256)
 }
 
 // Outputs of ModDown: out_i = [2][level][N]; add0/add1 (or null) are added
-// to the two polynomials, add0 read through sigma_{g_i} when sig_add0 is set,
-// and plus0 (or null) added to c0 after add0, as it is.
+// to the two polynomials, add0 read through sigma_{g_i} when sig_add0 is set.
 struct MdOut {
     MutPtrList out;
-    PtrList add0, add1, plus0;
+    PtrList add0, add1;
     GalList gal;
     int sig_add0;
 };
@@ -861,8 +860,6 @@ __global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
     const uint64_t g = (poly == 0 && mo.sig_add0) ? mo.gal.g[i] : 0;
     const ulonglong2 w = pinv[t];
     const uint64_t* adt = ad ? ad + (size_t)t * Cf::N : nullptr;
-    const uint64_t* pl = poly == 0 ? mo.plus0.p[i] : nullptr;
-    const uint64_t* plt = pl ? pl + (size_t)t * Cf::N + j0 : nullptr;
 #pragma unroll
     for (int k = 0; k < 4; k++) {
         uint64_t z[4];
@@ -878,14 +875,6 @@ __global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
                 z[2 * h] = add_mod(z[2 * h], sw ? av.y : av.x, q);
                 z[2 * h + 1] = add_mod(z[2 * h + 1], sw ? av.x : av.y, q);
             }
-        }
-        if (plt) {  // may be the output itself: a coherent load
-            uint64_t s0, s1, s2, s3;
-            ldg256(plt + 4 * k, s0, s1, s2, s3);
-            z[0] = add_mod(z[0], s0, q);
-            z[1] = add_mod(z[1], s1, q);
-            z[2] = add_mod(z[2], s2, q);
-            z[3] = add_mod(z[3], s3, q);
         }
         stg256(op + 4 * k, z[0], z[1], z[2], z[3]);
     }
@@ -988,7 +977,6 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
         mo.out.p[i] = i < n_md ? io.out[i] : nullptr;
         mo.add0.p[i] = i < n_md ? io.add0[i] : nullptr;
         mo.add1.p[i] = i < n_md ? io.add1[i] : nullptr;
-        mo.plus0.p[i] = i < n_md && !io.plus0.empty() ? io.plus0[i] : nullptr;
         mdin.p[i] = hoist ? (i < nm ? io.hoist_d[i] : nullptr) : din.p[i];
         mgal.g[i] = hoist ? 0 : gal.g[i];
         xsrc.i[i] = hoist && i < n ? io.hoist_src[i] : i;
@@ -1210,7 +1198,7 @@ int key_switch_chunk(he_ctx* c, int n, int level, const KsIoList& io) {
     {
         int n_add = 0;
         for (int i = 0; i < n_md; i++)
-            n_add += (io.add0[i] != nullptr) + (io.add1[i] != nullptr) + (!io.plus0.empty() && io.plus0[i] != nullptr);
+            n_add += (io.add0[i] != nullptr) + (io.add1[i] != nullptr);
         prof_end(c, HE_PROF_MODDOWN_COMBINE, (6.0 * n_md + n_add) * level * limbB,
                  2.0 * n_md * level * N * (1.0 + 0.5 * sh.s2), 2.0 * n_md * fp_q * N * 0.5 * sh.s2);
     }
@@ -1229,7 +1217,6 @@ int key_switch(he_ctx* c, int level, const KsIoList& io) {
         sub.out.assign(io.out.begin() + i0, io.out.begin() + i0 + m);
         sub.add0.assign(io.add0.begin() + i0, io.add0.begin() + i0 + m);
         sub.add1.assign(io.add1.begin() + i0, io.add1.begin() + i0 + m);
-        if (!io.plus0.empty()) sub.plus0.assign(io.plus0.begin() + i0, io.plus0.begin() + i0 + m);
         int rc = key_switch_chunk(c, m, level, sub);
         if (rc) return rc;
     }
@@ -1273,7 +1260,6 @@ int key_switch_split(he_ctx* c, int level, const KsIoList& io) {
         h.out.assign(io.out.begin() + a, io.out.begin() + b);
         h.add0.assign(io.add0.begin() + a, io.add0.begin() + b);
         h.add1.assign(io.add1.begin() + a, io.add1.begin() + b);
-        if (!io.plus0.empty()) h.plus0.assign(io.plus0.begin() + a, io.plus0.begin() + b);
         return h;
     };
     if ((rc = check_cuda(c, cudaEventRecord(c->ev_fork, c->stream), "fork")) ||
@@ -1302,7 +1288,7 @@ static int ct_ok(he_ctx* c, const he_ct* x, const char* what) {
     return HE_OK;
 }
 
-int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, int n, const he_ct* plus) {
+int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, int n) {
     if (n < 0) return set_err(c, HE_EINVAL, "rotate: negative count");
     if (n == 0) return HE_OK;
     if (!in || !out || !steps) return set_err(c, HE_EINVAL, "rotate: null argument");
@@ -1310,8 +1296,6 @@ int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, in
     for (int i = 0; i < n; i++) {
         int rc = ct_ok(c, &in[i], "rotate");
         if (rc) return rc;
-        if (plus && ((rc = ct_ok(c, &plus[i], "rotate")) || plus[i].level != in[i].level))
-            return rc ? rc : set_err(c, HE_ELEVEL, "rotate: addend level");
         if (in[i].level != level) return set_err(c, HE_ELEVEL, "rotate: mixed levels in a batch");
         if (!out[i].data || ((uintptr_t)out[i].data & 31)) return set_err(c, HE_EINVAL, "rotate: null or unaligned output");
         if (out[i].data == in[i].data) return set_err(c, HE_EINVAL, "rotate: output aliases input");
@@ -1331,10 +1315,9 @@ int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, in
     for (auto& kv : groups) {
         if (kv.first == 1) {  // rotation by a multiple of N/2: identity
             for (int i : kv.second) {
-                int rc = plus ? add_many(c, {in[i].data}, {plus[i].data}, {out[i].data}, level)
-                              : check_cuda(c, cudaMemcpyAsync(out[i].data, in[i].data, ct_words * 8,
-                                                              cudaMemcpyDeviceToDevice, c->stream),
-                                           "rotate copy");
+                int rc = check_cuda(c, cudaMemcpyAsync(out[i].data, in[i].data, ct_words * 8,
+                                                       cudaMemcpyDeviceToDevice, c->stream),
+                                    "rotate copy");
                 if (rc) return rc;
             }
             continue;
@@ -1346,8 +1329,7 @@ int rotate_many(he_ctx* c, const he_ct* in, const int32_t* steps, he_ct* out, in
             io.d.push_back(in[i].data + (size_t)level * c->N);
             io.out.push_back(out[i].data);
             io.add0.push_back(in[i].data);
-            io.add1.push_back(plus ? plus[i].data + (size_t)level * c->N : nullptr);
-            if (plus) io.plus0.push_back(plus[i].data);
+            io.add1.push_back(nullptr);
         }
     }
     if (!io.d.empty()) {
