@@ -94,3 +94,43 @@ def test_mutation_unduplicated_keys_are_caught(head):
     sc = C.attention_scores(head["q"], k_bad, NT, D, [delta], head["keys"], head["rlk"], P)[0]
     got = C.decrypt_decode(sc, s, P).real.reshape(D, 2 * NT)[:, :NT]
     assert np.max(np.abs(got - _scores_plain(head["Q"], head["K"], delta)[None, :])) > 1e-2
+
+
+def test_feature_sum_schedule_matches_doubling_rotations(head):
+    """The feature sum as two hoisted rotate-and-sums (d = 4 x 4 here) and
+    as log2(d) doubling rotations S <- S + rot_{2n 2^i}(S) decrypt to the
+    same slots: the two schedules differ only in key-switching noise."""
+    P, s, keys, rlk = head["P"], head["s"], head["keys"], head["rlk"]
+    inner, outer = C.attention_sum_steps(NT, D)
+    assert inner == [0, 64, 128, 192] and outer == [0, 256, 512, 768]
+    delta = 3
+    hoisted = C.attention_scores(head["q"], head["k"], NT, D, [delta], keys, rlk, P)[0]
+    acc = C.hmult_relin_rescale(head["q"], C.rotate(head["k"], delta, keys[delta], P), rlk, P)
+    for i in range(D.bit_length() - 1):
+        st = 2 * NT * (1 << i)
+        acc = C.add(acc, C.rotate(acc, st, keys[st], P), P)
+    a = C.decrypt_decode(hoisted, s, P)
+    b = C.decrypt_decode(acc, s, P)
+    assert np.max(np.abs(a - b)) < 1e-6
+    assert not np.array_equal(hoisted["c"], acc["c"])  # the residues do differ
+
+
+def test_output_schedule_matches_per_offset_products(head):
+    """A x V with the products' tensors summed and relinearised and rescaled
+    once decrypts to the same slots as the sum of per-offset
+    HMult-relinearise-rescale products: the two differ only in noise and
+    rounding."""
+    P, s, A, v, keys, rlk = head["P"], head["s"], head["A"], head["v"], head["keys"], head["rlk"]
+    offsets = head["offsets"]
+    nz = [o for o in offsets if o]
+    rot = dict(zip(nz, C.rotate_hoisted(v, nz, keys, P)))
+    plain = None
+    for ad, o in zip(A, offsets):
+        vv = C.drop_level(rot[o] if o in rot else v, ad["level"])
+        t = C.hmult_relin_rescale(ad, vv, rlk, P)
+        plain = t if plain is None else C.add(plain, t, P)
+    O = head["O"]
+    assert plain["level"] == O["level"] and plain["scale"] == O["scale"]
+    got, want = C.decrypt_decode(O, s, P), C.decrypt_decode(plain, s, P)
+    assert np.max(np.abs(got - want)) < 1e-6
+    assert not np.array_equal(O["c"], plain["c"])

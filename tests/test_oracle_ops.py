@@ -164,3 +164,45 @@ def test_ps_plain_horner_matches_power_sum():
     x = np.linspace(-4, 0, 101)
     want = sum(c * x ** k for k, c in enumerate(coeffs))
     assert np.allclose(C.ps_eval_plain(x, coeffs).real, want, rtol=0, atol=1e-12)
+
+
+def test_ps_schedule_matches_term_by_term_rescales():
+    """The degree-15 schedule (one rescale per Horner block and per step, the
+    block's products added before the step's rescale) decrypts to the same
+    slots as the plain schedule that rescales every constant-multiplied
+    power on its own and adds the blocks after each HMult-relin-rescale:
+    the two differ only in rounding."""
+    P = C.Params(12, 8, 3, 3)
+    seed = 31
+    z = S.real_slots(seed, P.n_slots, -4.0, 0.0)
+    coeffs = S.poly_coeffs(seed, 15)
+    s, pk, ct = _setup(P, seed, z, 8)
+    a, e = S.key_draws(seed, 2, P.mods, P.N, P.dnum)
+    rlk = C.relin_key(s, a, e, P)
+    fast = C.ps_eval_deg15(ct, coeffs, rlk, P)
+
+    hm = lambda u, v: C.hmult_relin_rescale(u, v, rlk, P)
+    l0 = ct["level"]
+    x2 = hm(ct, ct)
+    x3 = hm(x2, C.drop_level(ct, l0 - 1))
+    x4 = hm(x2, x2)
+    pw = {1: ct, 2: x2, 3: x3}
+
+    def block(i, lam, T):
+        acc = None
+        for j in (1, 2, 3):
+            xj = C.drop_level(pw[j], lam + 1)
+            K = C.ps_const(float(coeffs[4 * i + j]), T, P.q[lam], xj["scale"])
+            t = C.rescale(C.mul_const(xj, K, P), P)
+            acc = t if acc is None else C.make_ct(C.add(acc, t, P)["c"], lam, T)
+        acc = C.add_const(acc, int(C.round_half_away(np.float64(float(coeffs[4 * i]) * T))), P)
+        return C.make_ct(acc["c"], lam, T)
+
+    acc = block(3, l0 - 3, C.PS_TOP_SCALE)
+    for i in (2, 1, 0):
+        acc = hm(acc, C.drop_level(x4, acc["level"]))
+        acc = C.make_ct(C.add(acc, block(i, acc["level"], acc["scale"]), P)["c"], acc["level"], acc["scale"])
+    assert acc["level"] == fast["level"] and acc["scale"] == fast["scale"]
+    got, want = C.decrypt_decode(fast, s, P), C.decrypt_decode(acc, s, P)
+    assert np.max(np.abs(got - want)) < 1e-7
+    assert not np.array_equal(fast["c"], acc["c"])  # the residues do differ
