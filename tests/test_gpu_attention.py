@@ -73,6 +73,34 @@ def test_attention_head_small():
     assert np.max(np.abs(got - want)) < 1e-4
 
 
+def test_attention_output_many_offsets():
+    """A x V over 70 offsets (d = 4 features x 128 tokens at N = 2^11): the
+    tensor sum runs in two launches, the second accumulating onto the first;
+    every output residue equals the oracle's.  The weights are encryptions
+    of seeded slots at level 3, v sits at level 4 (its rotations are read at
+    the weights' level)."""
+    he = lib()
+    d, n_tok = 4, 128
+    st = Setup(11, 6, 2, 3, seed=S.master_seed(5) + 1)
+    P = st.P
+    assert d * 2 * n_tok == P.n_slots
+    offsets = list(range(70))
+    for s_ in offsets[1:]:
+        st.upload_rot(s_)
+    st.upload_relin()
+    keys = {s_: st.oracle_rot_key(s_) for s_ in offsets[1:]}
+    rlk = st.oracle_relin_key()
+    V = S.weights(st.seed, (d, n_tok), -0.5, 0.5, 3)
+    v = st.encrypt(C.attention_pack(V, True), 4, ct_id=0)
+    a = [st.encrypt(S.complex_slots(st.seed, P.n_slots, -1, 1, 10 + i), 3, ct_id=10 + i) for i in offsets]
+    out = st.empty_gpu(3)
+    he.he_attention_output(st.ctx, [st.to_gpu(x) for x in a], st.to_gpu(v), n_tok, offsets, out)
+    he.he_sync(st.ctx)
+    want = C.attention_av(a, v, offsets, keys, rlk, P)
+    assert out.level == want["level"] == 2 and out.scale == want["scale"]
+    assert np.array_equal(st.from_gpu(out), want["c"])
+
+
 def test_attention_errors():
     he = lib()
     st = Setup(11, 10, 4, 3, seed=68)
