@@ -101,6 +101,36 @@ def test_attention_output_many_offsets():
     assert np.array_equal(st.from_gpu(out), want["c"])
 
 
+def test_attention_scores_two_features():
+    """Scores with d = 2 features x 256 tokens at N = 2^11: the feature sum is
+    one hoisted rotate-and-sum (d = 2 x 1), which ends in the scratch set
+    and is copied to the outputs; residues equal the oracle's."""
+    he = lib()
+    d, n_tok = 2, 256
+    st = Setup(11, 4, 2, 3, seed=S.master_seed(5) + 2)
+    P = st.P
+    assert d * 2 * n_tok == P.n_slots
+    inner, outer = C.attention_sum_steps(n_tok, d)
+    assert inner == [0, 2 * n_tok] and outer == [0]
+    offsets = [0, 7, 255]
+    steps = sorted({o for o in offsets if o} | {2 * n_tok})
+    for s_ in steps:
+        st.upload_rot(s_)
+    st.upload_relin()
+    keys = {s_: st.oracle_rot_key(s_) for s_ in steps}
+    Q = S.weights(st.seed, (d, n_tok), -0.25, 0.25, 1)
+    K = S.weights(st.seed, (d, n_tok), -0.25, 0.25, 2)
+    q = st.encrypt(C.attention_pack(Q, False), P.L, ct_id=0)
+    k = st.encrypt(C.attention_pack(K, True), P.L, ct_id=1)
+    sc = [st.empty_gpu(P.L) for _ in offsets]
+    he.he_attention_scores(st.ctx, st.to_gpu(q), st.to_gpu(k), n_tok, d, offsets, sc)
+    he.he_sync(st.ctx)
+    want = C.attention_scores(q, k, n_tok, d, offsets, keys, st.oracle_relin_key(), P)
+    for g, w in zip(sc, want):
+        assert g.level == w["level"] == P.L - 1 and g.scale == w["scale"]
+        assert np.array_equal(st.from_gpu(g), w["c"])
+
+
 def test_attention_errors():
     he = lib()
     st = Setup(11, 10, 4, 3, seed=68)
