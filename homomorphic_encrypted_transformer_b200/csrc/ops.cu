@@ -235,8 +235,8 @@ __global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
     const int r = blockIdx.x * Cf::TR + threadIdx.x / (Cf::C / 16);
     const int j0 = r * Cf::C + 16 * row_lane<LOGN>();
     const uint64_t* a = tmp + (size_t)y * Cf::N + (size_t)r * Cf::C;
-    for (int j = 0; j < io.nterm; j++)  // read after the stages
-        prefetch_l2(io.in[j].p[i] + ((size_t)poly * io.lin[j] + t) * Cf::N + j0);
+    if (io.nterm == 1)  // read after the stages (several terms' lines would crowd L2)
+        prefetch_l2(io.in[0].p[i] + ((size_t)poly * io.lin[0] + t) * Cf::N + j0);
     uint64_t v[16];
     if (q < kFpPrimeLimit) {
         const FpMod m = fpm[t];
