@@ -257,24 +257,34 @@ __global__ void __launch_bounds__(NttCfg<LOGN>::ROW_THREADS, NTT_MIN_BLOCKS)
     const ulonglong2 w = qinv[t];
     const bool k0_here = add_k0 && poly == 0;
     const uint64_t kv = k0.v[t].x;
+    if (io.with_k) {
+        // v <- sum_j K_j x_j - v (mod q), term by term, each term's 16
+        // words read in consecutive loads
+#pragma unroll
+        for (int e = 0; e < 16; e++) v[e] = v[e] ? q - v[e] : 0;
+        for (int j = 0; j < io.nterm; j++) {
+            const uint64_t* xj = io.in[j].p[i] + ((size_t)poly * io.lin[j] + t) * Cf::N + j0;
+            const ulonglong2 kj = kk.k[j].v[t];
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+                uint64_t e4[4];
+                ldg256_ro(xj + 4 * k, e4[0], e4[1], e4[2], e4[3]);
+#pragma unroll
+                for (int e = 0; e < 4; e++) v[4 * k + e] = add_mod(v[4 * k + e], mul_shoup(e4[e], kj.x, kj.y, q), q);
+            }
+        }
+    }
 #pragma unroll
     for (int k = 0; k < 4; k++) {
         uint64_t z[4];
         if (io.with_k) {
-            z[0] = z[1] = z[2] = z[3] = 0;
-            for (int j = 0; j < io.nterm; j++) {
-                uint64_t e4[4];
-                ldg256_ro(io.in[j].p[i] + ((size_t)poly * io.lin[j] + t) * Cf::N + j0 + 4 * k, e4[0], e4[1], e4[2],
-                          e4[3]);
-                const ulonglong2 kj = kk.k[j].v[t];
 #pragma unroll
-                for (int e = 0; e < 4; e++) z[e] = add_mod(z[e], mul_shoup(e4[e], kj.x, kj.y, q), q);
-            }
+            for (int e = 0; e < 4; e++) z[e] = mul_shoup(v[4 * k + e], w.x, w.y, q);
         } else {
             ldg256_ro(io.in[0].p[i] + ((size_t)poly * io.lin[0] + t) * Cf::N + j0 + 4 * k, z[0], z[1], z[2], z[3]);
-        }
 #pragma unroll
-        for (int e = 0; e < 4; e++) z[e] = mul_shoup(z[e] + q - v[4 * k + e], w.x, w.y, q);
+            for (int e = 0; e < 4; e++) z[e] = mul_shoup(z[e] + q - v[4 * k + e], w.x, w.y, q);
+        }
         if (ap) {  // the addend may be the output itself: a coherent load
             uint64_t s0, s1, s2, s3;
             ldg256(ap + 4 * k, s0, s1, s2, s3);
