@@ -121,7 +121,7 @@ int wire_unpack_many(he_ctx* c, const uint8_t* wire, int level, const std::vecto
     const int n = (int)ct.size(), gx = (c->N / 8 + 255) / 256;
     for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
         const int m = std::min(kMaxBatch, n - i0);
-        PtrList none;
+        PtrList none{};
         MutPtrList out;
         for (int i = 0; i < m; i++) out.p[i] = ct[i0 + i];
         k_wire<false><<<dim3(gx, 2 * level, m), 256, 0, c->stream>>>(wire + (size_t)i0 * lay.off[2 * level], nullptr,
@@ -140,7 +140,7 @@ int wire_pack_many(he_ctx* c, const std::vector<const uint64_t*>& ct, int level,
     for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
         const int m = std::min(kMaxBatch, n - i0);
         PtrList in;
-        MutPtrList none;
+        MutPtrList none{};
         for (int i = 0; i < m; i++) in.p[i] = ct[i0 + i];
         k_wire<true><<<dim3(gx, 2 * level, m), 256, 0, c->stream>>>(nullptr, wire + (size_t)i0 * lay.off[2 * level],
                                                                   (size_t)lay.off[2 * level], in, none, level, lay,
